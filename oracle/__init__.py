@@ -1,0 +1,271 @@
+"""fp64 CPU oracle of the GLM-5.3-Flash kpool DSA decode path (numpy front end of oracle.c).
+
+TEST INFRASTRUCTURE. Only the test suite, ``__graft_entry__.smoke()`` and the benchmark's CPU
+baseline leg may import this package. It shares no code with the CUDA path
+(``kpool_indexer_int8_b200``) and does not import it; inputs come from ``synth``.
+
+The arithmetic lives in ``oracle.c`` (plain single-threaded C, fp64); this module only marshals
+numpy arrays and composes the steps in the order the pages give them ("Module glm5next_dsa_ref":
+pool_states -> index_scores -> topk_pools -> expand_selection -> mla_masked_attention;
+"GLM-5.3 Kernels": store_int8 -> sparse MLA over the gathered rows).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+from . import build as _build
+
+ROW_BYTES = 528
+LATENT = 512
+KPOOL = 4
+INVALID = -1
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        _lib = C.CDLL(path)
+        _declare(_lib)
+    return _lib
+
+
+_p = C.c_void_p
+_i64 = C.c_int64
+_i32 = C.c_int
+_f64 = C.c_double
+
+
+def _declare(L):
+    L.oracle_check_dims.argtypes = [_i32] * 6
+    L.oracle_check_dims.restype = _i32
+    L.oracle_store_int8.argtypes = [_p, _p, _i64, _p, _i64]
+    L.oracle_store_int8.restype = _i32
+    L.oracle_dequant_row.argtypes = [_p, _i64, _p]
+    L.oracle_dequant_row.restype = None
+    L.oracle_layer_norm.argtypes = [_p, _i32, _p, _p, _f64, _p]
+    L.oracle_layer_norm.restype = None
+    L.oracle_visible.argtypes = [_i64, _i64, _i64, _i64]
+    L.oracle_visible.restype = _i32
+    L.oracle_n_pools.argtypes = [_i64, _i32]
+    L.oracle_n_pools.restype = _i64
+    L.oracle_n_visible_pools.argtypes = [_i64, _i64, _i64, _i32]
+    L.oracle_n_visible_pools.restype = _i64
+    L.oracle_pool_states.argtypes = [_p, _p, _i32, _i64, _i64, _i32, _p, _p, _f64, _p]
+    L.oracle_pool_states.restype = _i64
+    L.oracle_index_scores.argtypes = [_p, _p, _p, _i32, _i32, _i64, _p]
+    L.oracle_index_scores.restype = None
+    L.oracle_topk_pools.argtypes = [_p, _i64, _i64, _p]
+    L.oracle_topk_pools.restype = _i64
+    L.oracle_expand_selection.argtypes = [_p, _i64, _i64, _i64, _i64, _i32, _i64, _p]
+    L.oracle_expand_selection.restype = _i64
+    L.oracle_rows_from_tokens.argtypes = [_p, _i64, _p, _p]
+    L.oracle_rows_from_tokens.restype = None
+    L.oracle_sparse_mla.argtypes = [_p, _i32, _p, _i64, _p, _i64, _f64, _p, _p]
+    L.oracle_sparse_mla.restype = _i32
+    L.oracle_topk_to_mask.argtypes = [_p, _i64, _i64, _p]
+    L.oracle_topk_to_mask.restype = None
+    L.oracle_masked_attention.argtypes = [_p, _i32, _p, _i64, _p, _i64, _p, _f64, _p, _p]
+    L.oracle_masked_attention.restype = _i32
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data_as(C.c_void_p)
+
+
+# ------------------------------------------------------------------------------------------------
+# one function per oracle step
+# ------------------------------------------------------------------------------------------------
+
+def check_dims(kv_lora_rank=512, qk_rope_head_dim=0, n_heads=64, index_n_heads=32,
+               index_head_dim=128, index_kpool=4) -> bool:
+    return lib().oracle_check_dims(kv_lora_rank, qk_rope_head_dim, n_heads, index_n_heads,
+                                   index_head_dim, index_kpool) == 0
+
+
+def store_int8(latent, slots, cache) -> None:
+    """Quantise ``latent`` (uint16 bf16 bits [n, 512]) into ``cache`` (int8 [n_rows, 528]) in place."""
+    assert cache.dtype == np.int8 and cache.flags.c_contiguous and cache.shape[-1] == ROW_BYTES
+    lat, lp = _c(latent, np.uint16)
+    sl, sp = _c(slots, np.int64)
+    assert lat.shape == (sl.shape[0], LATENT)
+    rc = lib().oracle_store_int8(lp, sp, sl.shape[0], cache.ctypes.data_as(C.c_void_p),
+                                 cache.reshape(-1, ROW_BYTES).shape[0])
+    if rc != 0:
+        raise ValueError("slot past the end of the cache")
+
+
+def dequant_rows(cache, rows) -> np.ndarray:
+    cache = np.ascontiguousarray(cache, dtype=np.int8).reshape(-1, ROW_BYTES)
+    out = np.empty((len(rows), LATENT), dtype=np.float64)
+    for i, r in enumerate(rows):
+        lib().oracle_dequant_row(cache.ctypes.data_as(C.c_void_p), int(r),
+                                 out[i].ctypes.data_as(C.c_void_p))
+    return out
+
+
+def layer_norm(x, w, b, eps) -> np.ndarray:
+    x, xp = _c(x, np.float64)
+    w, wp = _c(w, np.float64)
+    b, bp = _c(b, np.float64)
+    y = np.empty_like(x)
+    lib().oracle_layer_norm(xp, x.shape[0], wp, bp, float(eps), y.ctypes.data_as(C.c_void_p))
+    return y
+
+
+def visible(pad, length, q_pos, t) -> bool:
+    return bool(lib().oracle_visible(int(pad), int(length), int(q_pos), int(t)))
+
+
+def n_pools(length, kpool=KPOOL) -> int:
+    return int(lib().oracle_n_pools(int(length), kpool))
+
+
+def n_visible_pools(pad, length, q_pos, kpool=KPOOL) -> int:
+    return int(lib().oracle_n_visible_pools(int(pad), int(length), int(q_pos), kpool))
+
+
+def pool_states(k_seq, gate_seq, pad, length, ln_w, ln_b, eps, kpool=KPOOL) -> np.ndarray:
+    """Pools of one sequence. ``k_seq``/``gate_seq``: uint16 bf16 bits [>= pad+len, d] in padded
+    coordinates. Returns float64 [len // kpool, d]."""
+    k, kp = _c(k_seq, np.uint16)
+    g, gp = _c(gate_seq, np.uint16)
+    d = k.shape[1]
+    assert k.shape[0] >= pad + length and g.shape == k.shape
+    w, wp = _c(ln_w, np.float32)
+    b, bp = _c(ln_b, np.float32)
+    out = np.empty((max(n_pools(length, kpool), 0), d), dtype=np.float64)
+    n = lib().oracle_pool_states(kp, gp, d, int(pad), int(length), kpool, wp, bp, float(eps),
+                                 out.ctypes.data_as(C.c_void_p))
+    assert n == out.shape[0]
+    return out
+
+
+def index_scores(q_idx, w, pooled, n_vis) -> np.ndarray:
+    """``q_idx`` uint16 bf16 bits [H, D]; ``w`` float32 [H]; ``pooled`` [P, D] (any float dtype,
+    widened exactly to fp64). Returns float64 [n_vis]."""
+    q, qp = _c(q_idx, np.uint16)
+    w, wp = _c(w, np.float32)
+    pl, pp = _c(pooled, np.float64)
+    H, D = q.shape
+    assert pl.shape[1] == D and pl.shape[0] >= n_vis and w.shape == (H,)
+    out = np.empty(int(n_vis), dtype=np.float64)
+    lib().oracle_index_scores(qp, wp, pp, H, D, int(n_vis), out.ctypes.data_as(C.c_void_p))
+    return out
+
+
+def topk_pools(scores, select_k):
+    s, sp = _c(scores, np.float64)
+    out = np.empty(int(select_k), dtype=np.int32)
+    n_sel = lib().oracle_topk_pools(sp, s.shape[0], int(select_k), out.ctypes.data_as(C.c_void_p))
+    return out, int(n_sel)
+
+
+def expand_selection(topk, n_sel, pad, length, q_pos, out_width, kpool=KPOOL):
+    t, tp = _c(topk, np.int32)
+    out = np.empty(int(out_width), dtype=np.int32)
+    n = lib().oracle_expand_selection(tp, int(n_sel), int(pad), int(length), int(q_pos), kpool,
+                                      int(out_width), out.ctypes.data_as(C.c_void_p))
+    if n < 0:
+        raise ValueError("selection does not fit in out_width")
+    return out, int(n)
+
+
+def rows_from_tokens(tok, slot_map_row) -> np.ndarray:
+    t, tp = _c(tok, np.int32)
+    m, mp = _c(slot_map_row, np.int64)
+    out = np.empty_like(t)
+    lib().oracle_rows_from_tokens(tp, t.shape[0], mp, out.ctypes.data_as(C.c_void_p))
+    return out
+
+
+def sparse_mla(q, cache, rows, sm_scale):
+    """``q`` uint16 bf16 bits [Hm, 512]; ``cache`` int8 [n_rows, 528]; ``rows`` int32 [W].
+    Returns (out float64 [Hm, 512], lse float64 [Hm])."""
+    qq, qp = _c(q, np.uint16)
+    cache = np.ascontiguousarray(cache, dtype=np.int8).reshape(-1, ROW_BYTES)
+    r, rp = _c(rows, np.int32)
+    Hm = qq.shape[0]
+    out = np.empty((Hm, LATENT), dtype=np.float64)
+    lse = np.empty(Hm, dtype=np.float64)
+    rc = lib().oracle_sparse_mla(qp, Hm, cache.ctypes.data_as(C.c_void_p), cache.shape[0], rp,
+                                 r.shape[0], float(sm_scale), out.ctypes.data_as(C.c_void_p),
+                                 lse.ctypes.data_as(C.c_void_p))
+    if rc != 0:
+        raise ValueError("index past the end of the cache")
+    return out, lse
+
+
+def topk_to_mask(tok, n_tok) -> np.ndarray:
+    t, tp = _c(tok, np.int32)
+    mask = np.empty(int(n_tok), dtype=np.uint8)
+    lib().oracle_topk_to_mask(tp, t.shape[0], int(n_tok), mask.ctypes.data_as(C.c_void_p))
+    return mask.astype(bool)
+
+
+def masked_attention(q, cache, slot_map_row, mask, sm_scale):
+    qq, qp = _c(q, np.uint16)
+    cache = np.ascontiguousarray(cache, dtype=np.int8).reshape(-1, ROW_BYTES)
+    sm, smp = _c(slot_map_row, np.int64)
+    mk, mkp = _c(mask, np.uint8)
+    Hm = qq.shape[0]
+    out = np.empty((Hm, LATENT), dtype=np.float64)
+    lse = np.empty(Hm, dtype=np.float64)
+    rc = lib().oracle_masked_attention(qp, Hm, cache.ctypes.data_as(C.c_void_p), cache.shape[0],
+                                       smp, mk.shape[0], mkp, float(sm_scale),
+                                       out.ctypes.data_as(C.c_void_p),
+                                       lse.ctypes.data_as(C.c_void_p))
+    if rc != 0:
+        raise ValueError("index past the end of the cache")
+    return out, lse
+
+
+# ------------------------------------------------------------------------------------------------
+# composition of the steps for one workload state (the order of the pages)
+# ------------------------------------------------------------------------------------------------
+
+def build_cache(inp, token_mask=None) -> np.ndarray:
+    """store_int8 of every token (or of the tokens selected by ``token_mask``) into a fresh cache."""
+    cache = np.zeros((inp.n_rows, ROW_BYTES), dtype=np.int8)
+    if token_mask is None:
+        store_int8(inp.latent, inp.slots, cache)
+    else:
+        store_int8(inp.latent[token_mask], inp.slots[token_mask], cache)
+    return cache
+
+
+def build_pools(inp) -> list:
+    """pool_states of every sequence -> list of float64 [n_pools_b, 128]."""
+    return [pool_states(inp.k[b], inp.gate[b], inp.pad[b], inp.len[b], inp.ln_w, inp.ln_b,
+                        inp.wl.ln_eps) for b in range(inp.wl.batch)]
+
+
+def decode_query(inp, n, cache, pools, select_k=None, out_width=None, pooled_override=None,
+                 scores_override=None, attend=True) -> dict:
+    """The whole hot path for query ``n``: index_scores -> topk_pools -> expand_selection ->
+    rows through the slot map -> sparse MLA. ``pooled_override`` replaces the pooled keys of the
+    query's sequence (e.g. the fp32 values a GPU consumed); ``scores_override`` replaces the
+    scores fed to the selection."""
+    wl = inp.wl
+    S = wl.select_k if select_k is None else select_k
+    W = wl.out_width if out_width is None else out_width
+    b = int(inp.q_seq[n])
+    pad, ln, qp = int(inp.pad[b]), int(inp.len[b]), int(inp.q_pos[n])
+    pooled = pools[b] if pooled_override is None else pooled_override
+    n_vis = n_visible_pools(pad, ln, qp)
+    scores = index_scores(inp.q_idx[n], inp.w[n], pooled, n_vis)
+    sel_scores = scores if scores_override is None else scores_override
+    topk, n_sel = topk_pools(sel_scores, S)
+    tok, n_valid = expand_selection(topk, n_sel, pad, ln, qp, W)
+    rows = rows_from_tokens(tok, inp.slot_map[b])
+    res = dict(n_vis=n_vis, scores=scores, topk=topk, n_sel=n_sel, tok=tok, n_valid=n_valid,
+               rows=rows)
+    if attend:
+        res["out"], res["lse"] = sparse_mla(inp.q[n], cache, rows, inp.sm_scale)
+    return res
