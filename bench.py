@@ -1,0 +1,442 @@
+#!/usr/bin/env python
+"""Benchmark of the GLM-5.3-Flash kpool DSA decode hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kernels|reference]
+                    [--workload long_decode] [--states R]
+
+One step = one pass of the whole path over one batch of the workload: store_int8 of the step's
+new token(s) -> kpool_build of the pool(s) they complete -> index scores + top-k -> expand ->
+sparse NoPE MLA (split + combine), all through the C ABI, replayed as one CUDA graph per
+workload state. Inputs are synthetic (``synth``), resident in HBM before timing; R independent
+states (each with its own cache, pooled keys and queries) are rotated so that no step finds the
+previous step's bytes in L2 (8 x ~300 MB >> 126 MB of L2).
+
+Multi-GPU (torchrun): replicas only -- each rank runs its own independent states (no data-path
+collective); value = queries of all ranks / max-over-ranks time (weak scaling).
+
+``--impl reference`` times the fp64 CPU oracle (the reference arm of this build) on a bounded
+sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+KERNEL_LAUNCHES_PER_STEP = 7   # store, kpool, scores, top-k, expand, MLA split, MLA combine
+L2_BYTES = 126 * 1024 * 1024
+
+
+def algorithmic_bytes(inp) -> dict:
+    """Bytes the method must move per step (no partials, no score spills): per query the visible
+    pooled keys (512 B each), q_idx + w, the gathered int8 rows (528 B each), q + out, indices;
+    per step the store of the new rows and the pools they complete."""
+    wl = inp.wl
+    per_q_idx = 0
+    per_q_mla = 0
+    gathered = 0
+    for n in range(len(inp.q_pos)):
+        s = int(inp.q_seq[n])
+        upto = max(0, int(inp.q_pos[n]) - int(inp.pad[s]) + 1)
+        n_vis = min(int(inp.len[s]), upto) // 4
+        n_sel = min(n_vis, wl.select_k)
+        tail = min(upto, int(inp.len[s])) - 4 * n_vis
+        per_q_idx += n_vis * 128 * 4 + 32 * 128 * 2 + 32 * 4 + wl.select_k * 4
+        per_q_mla += (4 * n_sel + tail) * 528 + 2 * wl.n_heads * 512 * 2 + wl.out_width * 4
+        gathered += 4 * n_sel + tail
+    n_new = int(inp.new_token_mask().sum())
+    store = n_new * (1024 + 528 + 8)
+    new_pools = sum(1 for qs, qp in zip(inp.q_seq, inp.q_pos) if (qp - inp.pad[qs] + 1) % 4 == 0)
+    kpool = new_pools * (4 * (256 + 256) + 512)
+    return dict(index=per_q_idx, mla=per_q_mla, store=store, kpool=kpool, gathered=gathered,
+                total=per_q_idx + per_q_mla + store + kpool)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def kernel_source_sha(name: str) -> str:
+    path = os.path.join(ROOT, "kpool_indexer_int8_b200", "csrc", name)
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_file: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu summary, if the kernel's
+    source has not changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(f"{kernel_file}:{workload}")
+    if not d or d.get("source_sha") != kernel_source_sha(kernel_file):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only)
+# ------------------------------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown", 0x1: "gpu_idle",
+               0x2: "applications_clocks_setting", 0x10: "sync_boost"}
+
+    def __init__(self, device_index: int):
+        self.samples = []
+        self.reasons = set()
+        self.ok = False
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = self._handle(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # noqa: BLE001
+            self.err = str(e)
+
+    def _handle(self, device_index):
+        import torch
+        pynvml = self.nv
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        for i in range(pynvml.nvmlDeviceGetCount()):
+            h = pynvml.nvmlDeviceGetHandleByIndex(i)
+            u = pynvml.nvmlDeviceGetUUID(h)
+            u = u.decode() if isinstance(u, bytes) else u
+            if u.replace("GPU-", "") == uuid.replace("GPU-", ""):
+                return h
+        return pynvml.nvmlDeviceGetHandleByIndex(device_index)
+
+    def _sample(self):
+        nv = self.nv
+        self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+        try:
+            r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except AttributeError:
+            r = nv.nvmlDeviceGetCurrentClocksThrottleReasons(self.h)
+        for bit, name in self.REASONS.items():
+            if r & bit and name != "gpu_idle":
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.002)
+
+    def start(self):
+        if self.ok:
+            self._sample()
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+
+    def stop(self):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+            self._sample()
+
+    def summary(self):
+        if not self.ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "error": getattr(self, "err", "no samples")}
+        return {"sm_mhz": float(np.median(self.samples)), "sm_max_mhz": float(self.max_mhz),
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------------------------------------
+# the CPU oracle leg (cpu_baseline and --impl reference)
+# ------------------------------------------------------------------------------------------------
+
+def oracle_decode_throughput(wl, budget_s: float = 12.0, max_queries: int = 64):
+    """Time the fp64 oracle on decode queries of state 0 of the workload: per query the store of
+    its new row, the pool that row completes, scores over all visible pools, top-k, expand and the
+    sparse MLA. The oracle's state (cache, pools) is built beforehand, untimed."""
+    import oracle
+    inp = synth.generate(wl, state=0)
+    cache = oracle.build_cache(inp)
+    pools = oracle.build_pools(inp)
+    new = np.nonzero(inp.new_token_mask())[0]
+    done, t0 = 0, time.perf_counter()
+    elapsed = 0.0
+    while done < max_queries and (elapsed < budget_s or done == 0):
+        n = done % len(inp.q_pos)
+        s = int(inp.q_seq[n])
+        t_new = new[n] if len(new) == len(inp.q_pos) else new[0]
+        oracle.store_int8(inp.latent[t_new:t_new + 1], inp.slots[t_new:t_new + 1], cache)
+        qp, pad = int(inp.q_pos[n]), int(inp.pad[s])
+        if (qp - pad + 1) % 4 == 0:
+            p = (qp - pad + 1) // 4 - 1
+            t = pad + 4 * p
+            pools[s][p] = oracle.pool_states(inp.k[s][t:t + 4], inp.gate[s][t:t + 4], 0, 4,
+                                             inp.ln_w, inp.ln_b, wl.ln_eps)[0]
+        oracle.decode_query(inp, n, cache, pools)
+        done += 1
+        elapsed = time.perf_counter() - t0
+    return done / elapsed, done, elapsed
+
+
+def run_reference(args, wl):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    # one reference step = one whole decode query of the oracle; K steps, cut at ~4 minutes
+    qps, done, el = oracle_decode_throughput(wl, budget_s=240.0, max_queries=max(1, args.steps))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s",
+        "n_gpus": args.gpus, "steps": done, "warmup": 0,
+        "ms_per_step": 1e3 / qps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, args),
+        "cpu_baseline": {"value": qps, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                         "sample": f"{done} decode queries of {wl.name} state 0 in {el:.1f} s"},
+        "e2e": {"value": qps, "unit": "queries/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+METRIC = "decode queries/s and achieved HBM GB/s (% of B200 peak), indexer+sparse MLA"
+
+
+def config_of(wl, args):
+    return {"workload": wl.name, "batch": wl.batch, "context": list(wl.lens) if wl.batch > 1 else wl.lens[0],
+            "queries_per_step": wl.n_queries, "n_heads": wl.n_heads, "select_k": wl.select_k,
+            "out_width": wl.out_width, "kpool": 4, "index_heads": 32, "index_dim": 128,
+            "latent": 512, "states": args.states,
+            "l2": f"rotates {args.states} independent states per rank (inputs >> 126 MB L2)",
+            "launch": "cuda-graph per state", "parallelism": f"replicas x{args.gpus}"}
+
+
+# ------------------------------------------------------------------------------------------------
+# the CUDA path
+# ------------------------------------------------------------------------------------------------
+
+def run_kernels(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=120))
+
+    import kpool_indexer_int8_b200 as kp
+    from kpool_indexer_int8_b200 import pipeline as P
+    from synth import device as sdev
+
+    R = args.states
+    inps, bufs = [], []
+    for r in range(R):
+        inp = synth.generate(wl, state=rank * R + r)
+        b = sdev.allocate_for(inp, dev)
+        sdev.load(inp, b)
+        bufs.append(b)
+        inps.append(inp if r == 0 else None)
+        del inp
+    ab = algorithmic_bytes(inps[0])
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+
+    # one CUDA graph per state
+    graphs = []
+    with torch.cuda.stream(stream):
+        for b in bufs:
+            P.run_step(b)                       # eager once (idempotent step)
+        stream.synchronize()
+        for b in bufs:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                P.run_step(b)
+            graphs.append(g)
+    torch.cuda.synchronize()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # warm-up
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % R].replay()
+    stream.synchronize()
+
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            graphs[i % R].replay()
+        e1.record(stream)
+    stream.synchronize()
+    torch.cuda.synchronize()
+    sampler.stop()
+    barrier()
+    ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    queries = wl.n_queries * args.steps * world
+    value = queries / (ms / 1e3)
+
+    # per-stage device time (same kernels, same buffers, direct launches queued behind a sleep so
+    # the host never starves the GPU; events on the launching stream). "index_scores" is the
+    # scores-only kernel, timed on its own for the roofline of the dominant kernel.
+    stage_names = [nm for nm, _ in P.STAGES] + ["index_scores"]
+
+    def stage_calls(b):
+        nq, ld = b.q_idx.shape[0], b.pooled.shape[1]
+        scratch = b.ws_index.view(torch.float32)[:nq * ld].view(nq, ld)
+        return [lambda fn=fn: fn(b) for _, fn in P.STAGES] + [
+            lambda: kp.glm_index_scores(b.dims, b.q_idx, b.w, b.pooled, b.q_seq, b.q_pos, b.pad,
+                                        b.len, scratch)]
+
+    n_stage_steps = max(1, min(args.steps, 200))
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in stage_names] for _ in range(n_stage_steps)]
+    with torch.cuda.stream(stream):
+        calls = [stage_calls(b) for b in bufs]
+        torch.cuda._sleep(int(1.5e6 * n_stage_steps))      # ~0.75 ms of GPU time per step queued
+        for i in range(n_stage_steps):
+            for j, c in enumerate(calls[i % R]):
+                ev[i][j][0].record(stream)
+                c()
+                ev[i][j][1].record(stream)
+    stream.synchronize()
+    stage_ms = {nm: float(np.mean([ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(n_stage_steps)]))
+                for j, nm in enumerate(stage_names)}
+
+    # end to end through the public API with host buffers: per step the new token's latent, its
+    # k/gate rows, q_idx, w, q (and positions) go host->device from pinned memory, the step runs
+    # through the C-ABI calls, and the output comes back device->host
+    b = bufs[0]
+    inp0 = inps[0]
+    pin = lambda a: a.pin_memory()  # noqa: E731
+    h_lat = pin(b.new_latent.cpu())
+    h_slots = pin(b.new_slots.cpu())
+    h_qidx, h_w, h_q = pin(b.q_idx.cpu()), pin(b.w.cpu()), pin(b.q.cpu())
+    h_qpos, h_qseq, h_pb = pin(b.q_pos.cpu()), pin(b.q_seq.cpu()), pin(b.pool_begin.cpu())
+    kg_ranges = []
+    for sq in sorted(set(int(v) for v in inp0.q_seq)):
+        pos = inp0.q_pos[inp0.q_seq == sq]
+        kg_ranges.append((sq, int(pos.min()), int(pos.max()) + 1))
+    h_k = [pin(b.k[sq, lo:hi].cpu()) for sq, lo, hi in kg_ranges]
+    h_g = [pin(b.gate[sq, lo:hi].cpu()) for sq, lo, hi in kg_ranges]
+    h_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_lat, h_slots, h_qidx, h_w, h_q, h_qpos, h_qseq, h_pb, *h_k, *h_g))
+    d2h = h_out.numel() * h_out.element_size()
+    n_e2e = max(1, min(args.steps, 200))
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            P.run_step(b)
+        stream.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(n_e2e):
+            b.new_latent.copy_(h_lat, non_blocking=True)
+            b.new_slots.copy_(h_slots, non_blocking=True)
+            b.q_idx.copy_(h_qidx, non_blocking=True)
+            b.w.copy_(h_w, non_blocking=True)
+            b.q.copy_(h_q, non_blocking=True)
+            b.q_pos.copy_(h_qpos, non_blocking=True)
+            b.q_seq.copy_(h_qseq, non_blocking=True)
+            b.pool_begin.copy_(h_pb, non_blocking=True)
+            for i, (sq, lo, hi) in enumerate(kg_ranges):
+                b.k[sq, lo:hi].copy_(h_k[i], non_blocking=True)
+                b.gate[sq, lo:hi].copy_(h_g[i], non_blocking=True)
+            P.run_step(b)
+            h_out.copy_(b.out, non_blocking=True)
+            stream.synchronize()
+        e2e_s = time.perf_counter() - t0
+    e2e_qps = wl.n_queries * n_e2e / e2e_s
+    if world > 1:
+        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_qps = wl.n_queries * n_e2e * world / float(t.item())
+
+    peak, peak_kind = measured_peaks()
+    idx_ms = stage_ms["index_scores"]
+    achieved = ab["index"] / (idx_ms / 1e3) / 1e9
+    traffic = recorded_traffic("index_scores.cu", wl.name)
+    line = {
+        "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8/bf16 in, f32 math", "data": "synthetic", "config": config_of(wl, args),
+        "achieved_hbm_gbs_per_gpu": ab["total"] / (ms_per_step / 1e3) / 1e9,
+        "algorithmic_bytes_per_step": ab["total"],
+        "tokens_gathered_per_s": ab["gathered"] * args.steps * world / (ms / 1e3),
+        "stage_us": {k: v * 1e3 for k, v in stage_ms.items()},
+        "roofline": {"kernel": "index_scores", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": ab["index"]},
+        "e2e": {"value": e2e_qps, "unit": "queries/s", "h2d_bytes_per_step": int(h2d),
+                "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
+                "api": "C ABI via kpool_indexer_int8_b200 binding, host pinned buffers, sync per step"},
+        "gpu_launches": KERNEL_LAUNCHES_PER_STEP * args.steps,
+        "clocks": sampler.summary(),
+    }
+    line["achieved_hbm_frac_per_gpu"] = line["achieved_hbm_gbs_per_gpu"] / peak
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        qps, done, el = oracle_decode_throughput(wl, budget_s=12.0)
+        line["cpu_baseline"] = {"value": qps, "unit": "queries/s", "cores": 1, "kind": "oracle",
+                                "sample": f"{done} decode queries of {wl.name} state 0 ({el:.1f} s); oracle state built untimed"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graphs
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["kernels", "reference"], default="kernels")
+    ap.add_argument("--workload", default="long_decode", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--states", type=int, default=8)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    wl = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_kernels(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,236 @@
+/*
+ * glm_dsa.h -- C ABI of the GLM-5.3-Flash kpool DSA decode hot path on B200 (sm_100a).
+ *
+ * The path, in the order the pages give it:
+ *   glm_kv_store_int8      -> 528-byte int8 latent cache rows
+ *   glm_kpool_build        -> k_norm LayerNorm + slot-axis softmax pooling into fp32 pooled keys
+ *   glm_index_scores_topk  -> relu head-weighted index scores and the top select_k pools
+ *   glm_expand_selection   -> token indices (+ cache rows), visible tail, -1 padding
+ *   glm_sparse_mla_decode  -> sparse NoPE MLA over the gathered int8 rows (split-KV + combine)
+ *
+ * Conventions for every entry point
+ *   - Pointers named *_dev are device pointers on the current CUDA device; everything else is
+ *     host memory. The caller owns every buffer; the library allocates nothing, keeps no state
+ *     between calls and only enqueues work on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream). Outputs are valid once the stream has reached the call.
+ *   - Device pointers must be 16-byte aligned; leading dimensions are in elements.
+ *   - Arguments are checked on the host before anything is enqueued. A failed check returns a
+ *     negative status and enqueues nothing. GLM_ERR_CUDA means a launch failed (the status of
+ *     cudaGetLastError is reported through glm_last_cuda_error()).
+ *   - Every output element an entry point documents is written (no uninitialised tails).
+ *   - Kernels never trap and never read outside the buffers described here: an index outside
+ *     the documented range is treated as padding (-1) instead of being dereferenced.
+ */
+#ifndef GLM_DSA_H
+#define GLM_DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ------------------------------------------------------------------------------------------ */
+/* Status codes                                                                                */
+/* ------------------------------------------------------------------------------------------ */
+#define GLM_OK 0
+#define GLM_ERR_INVALID_ARG (-1) /* null / misaligned pointer, bad size or leading dimension   */
+#define GLM_ERR_UNSUPPORTED (-2) /* geometry other than the one the kernels are built for      */
+#define GLM_ERR_WORKSPACE (-3)   /* workspace null or smaller than glm_dsa_workspace_size()    */
+#define GLM_ERR_CUDA (-4)        /* a kernel launch failed                                     */
+
+/* Sentinel of an unused index entry ("Module glm5next_dsa_ref": INVALID). */
+#define GLM_INVALID (-1)
+
+/* Bytes of one cache row: 512 int8 codes, one little-endian fp32 scale, 12 zero bytes
+ * ("GLM-5.3 Kernels" README, 'Included': titan_kv.store_int8). */
+#define GLM_ROW_BYTES 528
+
+/*
+ * Geometry of one sparse-attention layer ("Module glm5next_dsa_ref": DsaDims, read from the
+ * config and never defaulted; "GLM-5.3-Flash" pypto-lib page, 'Checkpoint shape').
+ * The kernels are built for kv_lora_rank 512, qk_rope_head_dim 0 (NoPE: the rope slice is
+ * zero-width), index_n_heads 32, index_head_dim 128, index_kpool 4, 1 <= n_heads <= 128.
+ * Any other value gives GLM_ERR_UNSUPPORTED; index_topk is informational (select_k is passed
+ * per call) but must be a positive multiple of index_kpool.
+ */
+typedef struct glm_dsa_dims {
+    int32_t kv_lora_rank;
+    int32_t qk_rope_head_dim;
+    int32_t n_heads;
+    int32_t index_n_heads;
+    int32_t index_head_dim;
+    int32_t index_kpool;
+    int32_t index_topk;
+} glm_dsa_dims;
+
+/* Returns GLM_OK if `dims` is the geometry the kernels implement. */
+int glm_check_dims(const glm_dsa_dims *dims);
+
+/* Human-readable name of a status code (static storage). */
+const char *glm_status_string(int status);
+
+/* cudaError_t value of the last launch that returned GLM_ERR_CUDA on this host thread. */
+int glm_last_cuda_error(void);
+
+/* ------------------------------------------------------------------------------------------ */
+/* store_int8                                                                                  */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * "GLM-5.3 Kernels" README, 'Included' (titan_kv.store_int8): quantise each 512-value BF16 MLA
+ * latent into one 528-byte cache row -- bytes [0,512) int8 codes, [512,516) fp32 scale
+ * (little endian), [516,528) zero -- and scatter it to row slots[i]; slots[i] < 0 is padding
+ * and writes nothing. scale = max(amax, 1e-4f) / 127 (fp32), code = clamp(rint(x / scale), +-127)
+ * with an IEEE fp32 quotient and ties to even.
+ *   latent_dev  bf16 [n, 512], rows contiguous (row stride 1024 bytes)
+ *   slots_dev   int64 [n]
+ *   cache_dev   int8 [n_rows, 528] (rows contiguous; blocks of 256 rows are just consecutive rows)
+ * A slot >= n_rows is outside the contract and is skipped. Duplicate slots race (last writer
+ * undefined). n == 0 is a no-op.
+ */
+int glm_kv_store_int8(const glm_dsa_dims *dims, const void *latent_dev, const int64_t *slots_dev,
+                      int64_t n, int8_t *cache_dev, int64_t n_rows, void *stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* kpool_build                                                                                 */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * "Module glm5next_dsa_ref", pool_states and its traps: k is normalised by k_norm (a LayerNorm
+ * with bias over the 128 channels, eps = ln_eps); pool p of sequence b covers the kpool = 4
+ * tokens t_s = pad[b] + 4p + s (pooling starts at the first valid token); a pool exists only if
+ * all 4 slots are valid tokens (p < len[b] / 4); the 4 slots are mixed per channel by a softmax
+ * of the gates over the slot axis:
+ *     pooled[b][p][d] = sum_s softmax_s(gate[b][t_s][d]) * LN(k[b][t_s])[d]      (fp32)
+ *   k_dev, gate_dev  bf16 [batch, ld_tokens, 128]: token t of sequence b at row b*ld_tokens + t
+ *                    (padded coordinates; positions < pad[b] are padding and never read)
+ *   ln_w_dev, ln_b_dev  fp32 [128]
+ *   pad_dev, len_dev    int32 [batch]: first valid position and valid length of each sequence
+ *   pool_begin_dev      int32 [batch] or NULL (= 0): first pool to (re)build per sequence
+ *   max_new_pools       pools built per sequence: p in [pool_begin, min(pool_begin +
+ *                       max_new_pools, len/4, ld_pools)); e.g. 1 for a decode step
+ *   pooled_dev          fp32 [batch, ld_pools, 128]; pools outside that range are not touched
+ *   n_pools_dev         int32 [batch] or NULL: receives len[b] / 4 (capped at ld_pools)
+ * Requires pad[b] + len[b] <= ld_tokens (not checked on the device: rows past it are not read).
+ */
+int glm_kpool_build(const glm_dsa_dims *dims, const void *k_dev, const void *gate_dev,
+                    int64_t ld_tokens, const float *ln_w_dev, const float *ln_b_dev, float ln_eps,
+                    const int32_t *pad_dev, const int32_t *len_dev, const int32_t *pool_begin_dev,
+                    int32_t batch, int32_t max_new_pools, float *pooled_dev, int64_t ld_pools,
+                    int32_t *n_pools_dev, void *stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* index_scores + topk_pools                                                                   */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * "Module glm5next_dsa_ref", index_scores (matmul -> relu -> head-weighted sum) and topk_pools.
+ * For query n of sequence b = q_seq[n] at padded position q_pos[n], the visible pools are the
+ * existing pools whose 4 slots are all visible (causal, not padding):
+ *     n_vis = min(len[b] / 4, max(0, q_pos - pad[b] + 1) / 4, ld_pools)
+ *     score[n][p] = sum_h w[n][h] * max(0, sum_d q_idx[n][h][d] * pooled[b][p][d]),  p < n_vis
+ * and the selection is the min(select_k, n_vis) highest scores, ordered by score descending
+ * with ties to the lower pool id (-0.0 == +0.0), followed by -1 up to select_k.
+ *   q_idx_dev   bf16 [n_q, 32, 128]        w_dev  fp32 [n_q, 32]
+ *   pooled_dev  fp32 [batch, ld_pools, 128] (from glm_kpool_build)
+ *   q_seq_dev, q_pos_dev  int32 [n_q];     pad_dev, len_dev  int32 [batch]
+ *   scores_dev  fp32 [n_q, ld_pools] or NULL: receives the scores (entries p >= n_vis are -inf)
+ *   topk_dev    int32 [n_q, select_k]      n_sel_dev  int32 [n_q] or NULL
+ *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, ...)
+ * 1 <= select_k <= 2048. The fp32 scores are computed on tensor cores from an exact three-term
+ * bf16 split of the pooled keys (max relative error well below 1e-4).
+ */
+int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx_dev, const float *w_dev,
+                          const float *pooled_dev, int64_t ld_pools, const int32_t *q_seq_dev,
+                          const int32_t *q_pos_dev, const int32_t *pad_dev, const int32_t *len_dev,
+                          int32_t batch, int32_t n_q, int32_t select_k, float *scores_dev,
+                          int32_t *topk_dev, int32_t *n_sel_dev, void *workspace_dev,
+                          size_t ws_bytes, void *stream);
+
+/*
+ * The scores alone ("Module glm5next_dsa_ref", index_scores): the same scores as
+ * glm_index_scores_topk, written to scores_dev fp32 [n_q, ld_pools] (entries p >= n_vis are
+ * -inf), without the selection. No workspace.
+ */
+int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx_dev, const float *w_dev,
+                     const float *pooled_dev, int64_t ld_pools, const int32_t *q_seq_dev,
+                     const int32_t *q_pos_dev, const int32_t *pad_dev, const int32_t *len_dev,
+                     int32_t batch, int32_t n_q, float *scores_dev, void *stream);
+
+/*
+ * The selection alone, on given scores ("Module glm5next_dsa_ref", topk_pools): for each query
+ * n, the min(select_k, n_visible[n]) highest of scores[n][0 .. n_visible[n]) in the order above,
+ * then -1. Used to check the selection bit-exactly on externally supplied scores.
+ *   scores_dev  fp32 [n_q, ld_scores];  n_visible_dev int32 [n_q] (clamped to [0, ld_scores])
+ *   topk_dev    int32 [n_q, select_k];  n_sel_dev int32 [n_q] or NULL
+ * NaN scores are outside the contract.
+ */
+int glm_topk_pools(const float *scores_dev, int64_t ld_scores, const int32_t *n_visible_dev,
+                   int32_t n_q, int32_t select_k, int32_t *topk_dev, int32_t *n_sel_dev,
+                   void *workspace_dev, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* expand_selection                                                                            */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * "Module glm5next_dsa_ref", expand_selection and the -1 trap: each selected pool p (in top-k
+ * order) becomes its 4 tokens pad + 4p + 0..3; then the visible tail (tokens pad + 4*n_vis ..
+ * q_pos, at most 3); then -1 up to out_width. Every one of the out_width entries is written.
+ *   topk_dev     int32 [n_q, select_k] (-1 ends the list; entries >= n_vis are treated as -1)
+ *   n_sel_dev    int32 [n_q] or NULL (NULL: the list ends at the first -1)
+ *   slot_map_dev int64 [batch, ld_slot] or NULL: cache row of token t of sequence b, -1 if none
+ *   tok_dev      int32 [n_q, out_width] or NULL: token positions
+ *   rows_dev     int32 [n_q, out_width] or NULL: cache rows (slot_map[b][tok]; tok itself when
+ *                slot_map is NULL); -1 where the token is -1 or has no row
+ * Requires out_width >= 4 * select_k + 3 (the largest possible selection plus a full tail).
+ */
+int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk_dev,
+                         const int32_t *n_sel_dev, const int32_t *q_seq_dev,
+                         const int32_t *q_pos_dev, const int32_t *pad_dev, const int32_t *len_dev,
+                         int32_t batch, int32_t n_q, int32_t select_k,
+                         const int64_t *slot_map_dev, int64_t ld_slot, int32_t out_width,
+                         int32_t *tok_dev, int32_t *rows_dev, void *stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* sparse NoPE MLA decode                                                                      */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * "GLM-5.3 Kernels" README, 'Included' (titan_mla.triton_mla_sparse_attention) and 'The tested
+ * MLA contract': int8 rows are dequantised in-kernel (c = code * scale) and the shared 512-d
+ * latent is both K and V (one KV head, NoPE); softmax and accumulation in fp32:
+ *     s[h][j] = sm_scale * q[n][h] . c_j,  out[n][h] = sum_j softmax_j(s[h])_j c_j,
+ *     lse[n][h] = log sum_j exp(s[h][j])
+ * over the entries j of rows[n] with 0 <= rows[n][j] < n_rows (each entry is one key; -1 is
+ * padding). A query with no valid entry gets out = 0 and lse = -inf. Split-KV: chunks of the
+ * index row run in parallel and a combine kernel merges their partial softmax states.
+ *   q_dev      bf16 [n_q, n_heads, 512]       cache_dev int8 [n_rows, 528]
+ *   rows_dev   int32 [n_q, width]             out_dev   bf16 [n_q, n_heads, 512]
+ *   lse_dev    fp32 [n_q, n_heads] or NULL    out_f32_dev fp32 [n_q, n_heads, 512] or NULL
+ *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width)
+ * 1 <= width <= 65536.
+ */
+int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q_dev, const int8_t *cache_dev,
+                          int64_t n_rows, const int32_t *rows_dev, int32_t n_q, int32_t width,
+                          float sm_scale, void *out_dev, float *lse_dev, float *out_f32_dev,
+                          void *workspace_dev, size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* workspace sizes                                                                             */
+/* ------------------------------------------------------------------------------------------ */
+#define GLM_OP_INDEX_SCORES_TOPK 1
+#define GLM_OP_TOPK_POOLS 2
+#define GLM_OP_SPARSE_MLA 3
+
+/*
+ * Bytes of device workspace an entry point needs (0 if none; (size_t)-1 for bad arguments).
+ *   GLM_OP_INDEX_SCORES_TOPK: n_q, max_pools = ld_pools, select_k
+ *   GLM_OP_TOPK_POOLS:        n_q, max_pools = ld_scores, select_k
+ *   GLM_OP_SPARSE_MLA:        n_q, width (max_pools and select_k unused)
+ */
+size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
+                              int64_t max_pools, int32_t select_k, int32_t width);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GLM_DSA_H */

@@ -1,0 +1,234 @@
+"""Python binding of libglm_dsa.so, the C ABI of the GLM-5.3-Flash kpool DSA decode path (sm_100a).
+
+Argument marshalling only: each function takes torch CUDA tensors, checks dtypes and shapes,
+and calls the C entry point of the same name (include/glm_dsa.h) on the current torch stream.
+Every step of the path runs in the library's CUDA kernels; there is no CPU fallback. Importing
+this package without the built library raises ImportError (build it with
+``python kpool_indexer_int8_b200/build.py``).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libglm_dsa.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python kpool_indexer_int8_b200/build.py`")
+
+lib = C.CDLL(LIB_PATH)
+
+GLM_OK = 0
+GLM_ERR_INVALID_ARG = -1
+GLM_ERR_UNSUPPORTED = -2
+GLM_ERR_WORKSPACE = -3
+GLM_ERR_CUDA = -4
+GLM_INVALID = -1
+GLM_ROW_BYTES = 528
+GLM_OP_INDEX_SCORES_TOPK = 1
+GLM_OP_TOPK_POOLS = 2
+GLM_OP_SPARSE_MLA = 3
+
+EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv_store_int8",
+           "glm_kpool_build", "glm_index_scores", "glm_index_scores_topk", "glm_topk_pools", "glm_expand_selection",
+           "glm_sparse_mla_decode", "glm_dsa_workspace_size")
+
+
+class glm_dsa_dims(C.Structure):
+    """DsaDims of the pages ("Module glm5next_dsa_ref"): passed explicitly, never defaulted."""
+    _fields_ = [("kv_lora_rank", C.c_int32), ("qk_rope_head_dim", C.c_int32),
+                ("n_heads", C.c_int32), ("index_n_heads", C.c_int32),
+                ("index_head_dim", C.c_int32), ("index_kpool", C.c_int32),
+                ("index_topk", C.c_int32)]
+
+
+def make_dims(n_heads: int, kv_lora_rank: int = 512, qk_rope_head_dim: int = 0,
+              index_n_heads: int = 32, index_head_dim: int = 128, index_kpool: int = 4,
+              index_topk: int = 2048) -> glm_dsa_dims:
+    return glm_dsa_dims(kv_lora_rank, qk_rope_head_dim, n_heads, index_n_heads, index_head_dim,
+                        index_kpool, index_topk)
+
+
+_P, _I64, _I32, _F32, _SZ = C.c_void_p, C.c_int64, C.c_int32, C.c_float, C.c_size_t
+_D = C.POINTER(glm_dsa_dims)
+lib.glm_check_dims.argtypes = [_D]
+lib.glm_check_dims.restype = C.c_int
+lib.glm_status_string.argtypes = [C.c_int]
+lib.glm_status_string.restype = C.c_char_p
+lib.glm_last_cuda_error.argtypes = []
+lib.glm_last_cuda_error.restype = C.c_int
+lib.glm_kv_store_int8.argtypes = [_D, _P, _P, _I64, _P, _I64, _P]
+lib.glm_kv_store_int8.restype = C.c_int
+lib.glm_kpool_build.argtypes = [_D, _P, _P, _I64, _P, _P, _F32, _P, _P, _P, _I32, _I32, _P, _I64, _P, _P]
+lib.glm_kpool_build.restype = C.c_int
+lib.glm_index_scores_topk.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32, _P, _P,
+                                      _P, _P, _SZ, _P]
+lib.glm_index_scores_topk.restype = C.c_int
+lib.glm_index_scores.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P]
+lib.glm_index_scores.restype = C.c_int
+lib.glm_topk_pools.argtypes = [_P, _I64, _P, _I32, _I32, _P, _P, _P, _SZ, _P]
+lib.glm_topk_pools.restype = C.c_int
+lib.glm_expand_selection.argtypes = [_D, _P, _P, _P, _P, _P, _P, _I32, _I32, _I32, _P, _I64, _I32, _P,
+                                     _P, _P]
+lib.glm_expand_selection.restype = C.c_int
+lib.glm_sparse_mla_decode.argtypes = [_D, _P, _P, _I64, _P, _I32, _I32, _F32, _P, _P, _P, _P, _SZ, _P]
+lib.glm_sparse_mla_decode.restype = C.c_int
+lib.glm_dsa_workspace_size.argtypes = [_D, _I32, _I32, _I64, _I32, _I32]
+lib.glm_dsa_workspace_size.restype = C.c_size_t
+
+
+class GlmError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        msg = lib.glm_status_string(status).decode()
+        if status == GLM_ERR_CUDA:
+            msg += f" (cudaError {lib.glm_last_cuda_error()})"
+        super().__init__(f"{what}: {msg} [{status}]")
+        self.status = status
+
+
+def _check(status: int, what: str) -> None:
+    if status != GLM_OK:
+        raise GlmError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return C.c_void_p(s.cuda_stream)
+
+
+def _dev(t, dtype, name, ndim=None):
+    if t is None:
+        return
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got {t.dim()}")
+
+
+def check_dims(dims: glm_dsa_dims) -> int:
+    return lib.glm_check_dims(C.byref(dims))
+
+
+def glm_dsa_workspace_size(dims, op, n_q, max_pools=0, select_k=1, width=1) -> int:
+    v = lib.glm_dsa_workspace_size(C.byref(dims), op, n_q, max_pools, select_k, width)
+    if v == C.c_size_t(-1).value:
+        raise GlmError(GLM_ERR_INVALID_ARG, "glm_dsa_workspace_size")
+    return int(v)
+
+
+def glm_kv_store_int8(dims, latent, slots, cache, stream=None) -> None:
+    """latent bf16 [n, 512], slots int64 [n], cache int8 [n_rows, 528] (or [blocks, 256, 528])."""
+    _dev(latent, torch.bfloat16, "latent", 2)
+    _dev(slots, torch.int64, "slots", 1)
+    _dev(cache, torch.int8, "cache")
+    n_rows = cache.numel() // GLM_ROW_BYTES
+    _check(lib.glm_kv_store_int8(C.byref(dims), _ptr(latent), _ptr(slots), latent.shape[0],
+                                 _ptr(cache), n_rows, _stream(stream)), "glm_kv_store_int8")
+
+
+def glm_kpool_build(dims, k, gate, ln_w, ln_b, ln_eps, pad, length, pooled, pool_begin=None,
+                    max_new_pools=None, n_pools=None, stream=None) -> None:
+    """k, gate bf16 [B, ld_tokens, 128]; ln_w, ln_b fp32 [128]; pad, length int32 [B];
+    pooled fp32 [B, ld_pools, 128]; pool_begin int32 [B] or None; n_pools int32 [B] or None."""
+    for t, dt, nm in ((k, torch.bfloat16, "k"), (gate, torch.bfloat16, "gate"),
+                      (ln_w, torch.float32, "ln_w"), (ln_b, torch.float32, "ln_b"),
+                      (pad, torch.int32, "pad"), (length, torch.int32, "len"),
+                      (pooled, torch.float32, "pooled"), (pool_begin, torch.int32, "pool_begin"),
+                      (n_pools, torch.int32, "n_pools")):
+        _dev(t, dt, nm)
+    B, ld_tokens = k.shape[0], k.shape[1]
+    ld_pools = pooled.shape[1]
+    if max_new_pools is None:
+        max_new_pools = ld_pools
+    _check(lib.glm_kpool_build(C.byref(dims), _ptr(k), _ptr(gate), ld_tokens, _ptr(ln_w), _ptr(ln_b),
+                               float(ln_eps), _ptr(pad), _ptr(length), _ptr(pool_begin), B,
+                               int(max_new_pools), _ptr(pooled), ld_pools, _ptr(n_pools),
+                               _stream(stream)), "glm_kpool_build")
+
+
+def glm_index_scores_topk(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, select_k, topk,
+                          n_sel=None, scores=None, workspace=None, stream=None) -> None:
+    """q_idx bf16 [n_q, 32, 128], w fp32 [n_q, 32], pooled fp32 [B, ld_pools, 128];
+    topk int32 [n_q, select_k]; scores fp32 [n_q, ld_pools] or None; workspace uint8 tensor."""
+    for t, dt, nm in ((q_idx, torch.bfloat16, "q_idx"), (w, torch.float32, "w"),
+                      (pooled, torch.float32, "pooled"), (q_seq, torch.int32, "q_seq"),
+                      (q_pos, torch.int32, "q_pos"), (pad, torch.int32, "pad"),
+                      (length, torch.int32, "len"), (topk, torch.int32, "topk"),
+                      (n_sel, torch.int32, "n_sel"), (scores, torch.float32, "scores"),
+                      (workspace, torch.uint8, "workspace")):
+        _dev(t, dt, nm)
+    n_q = q_idx.shape[0]
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    _check(lib.glm_index_scores_topk(C.byref(dims), _ptr(q_idx), _ptr(w), _ptr(pooled), pooled.shape[1],
+                                     _ptr(q_seq), _ptr(q_pos), _ptr(pad), _ptr(length), pad.shape[0],
+                                     n_q, int(select_k), _ptr(scores), _ptr(topk), _ptr(n_sel),
+                                     _ptr(workspace), ws_bytes, _stream(stream)),
+           "glm_index_scores_topk")
+
+
+def glm_index_scores(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, scores, stream=None) -> None:
+    """Scores only: scores fp32 [n_q, ld_pools] (entries past the visible pools are -inf)."""
+    for t, dt, nm in ((q_idx, torch.bfloat16, "q_idx"), (w, torch.float32, "w"),
+                      (pooled, torch.float32, "pooled"), (q_seq, torch.int32, "q_seq"),
+                      (q_pos, torch.int32, "q_pos"), (pad, torch.int32, "pad"),
+                      (length, torch.int32, "len"), (scores, torch.float32, "scores")):
+        _dev(t, dt, nm)
+    _check(lib.glm_index_scores(C.byref(dims), _ptr(q_idx), _ptr(w), _ptr(pooled), pooled.shape[1],
+                                _ptr(q_seq), _ptr(q_pos), _ptr(pad), _ptr(length), pad.shape[0],
+                                q_idx.shape[0], _ptr(scores), _stream(stream)), "glm_index_scores")
+
+
+def glm_topk_pools(scores, n_visible, select_k, topk, n_sel=None, workspace=None, stream=None) -> None:
+    """scores fp32 [n_q, ld_scores], n_visible int32 [n_q]; topk int32 [n_q, select_k]."""
+    for t, dt, nm in ((scores, torch.float32, "scores"), (n_visible, torch.int32, "n_visible"),
+                      (topk, torch.int32, "topk"), (n_sel, torch.int32, "n_sel"),
+                      (workspace, torch.uint8, "workspace")):
+        _dev(t, dt, nm)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    _check(lib.glm_topk_pools(_ptr(scores), scores.shape[1], _ptr(n_visible), scores.shape[0],
+                              int(select_k), _ptr(topk), _ptr(n_sel), _ptr(workspace), ws_bytes,
+                              _stream(stream)), "glm_topk_pools")
+
+
+def glm_expand_selection(dims, topk, q_seq, q_pos, pad, length, out_width, n_sel=None,
+                         slot_map=None, tok=None, rows=None, stream=None) -> None:
+    """topk int32 [n_q, select_k]; slot_map int64 [B, ld_slot] or None;
+    tok / rows int32 [n_q, out_width] (at least one)."""
+    for t, dt, nm in ((topk, torch.int32, "topk"), (q_seq, torch.int32, "q_seq"),
+                      (q_pos, torch.int32, "q_pos"), (pad, torch.int32, "pad"),
+                      (length, torch.int32, "len"), (n_sel, torch.int32, "n_sel"),
+                      (slot_map, torch.int64, "slot_map"), (tok, torch.int32, "tok"),
+                      (rows, torch.int32, "rows")):
+        _dev(t, dt, nm)
+    ld_slot = 0 if slot_map is None else slot_map.shape[1]
+    _check(lib.glm_expand_selection(C.byref(dims), _ptr(topk), _ptr(n_sel), _ptr(q_seq), _ptr(q_pos),
+                                    _ptr(pad), _ptr(length), pad.shape[0], topk.shape[0],
+                                    topk.shape[1], _ptr(slot_map), ld_slot, int(out_width),
+                                    _ptr(tok), _ptr(rows), _stream(stream)), "glm_expand_selection")
+
+
+def glm_sparse_mla_decode(dims, q, cache, rows, sm_scale, out, workspace, lse=None, out_f32=None,
+                          stream=None) -> None:
+    """q bf16 [n_q, n_heads, 512]; cache int8 [n_rows, 528]; rows int32 [n_q, width];
+    out bf16 [n_q, n_heads, 512]; lse fp32 [n_q, n_heads] or None; out_f32 fp32 like out or None."""
+    for t, dt, nm in ((q, torch.bfloat16, "q"), (cache, torch.int8, "cache"),
+                      (rows, torch.int32, "rows"), (out, torch.bfloat16, "out"),
+                      (workspace, torch.uint8, "workspace"), (lse, torch.float32, "lse"),
+                      (out_f32, torch.float32, "out_f32")):
+        _dev(t, dt, nm)
+    n_rows = cache.numel() // GLM_ROW_BYTES
+    _check(lib.glm_sparse_mla_decode(C.byref(dims), _ptr(q), _ptr(cache), n_rows, _ptr(rows),
+                                     rows.shape[0], rows.shape[1], float(sm_scale), _ptr(out),
+                                     _ptr(lse), _ptr(out_f32), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)), "glm_sparse_mla_decode")

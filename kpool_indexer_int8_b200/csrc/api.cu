@@ -1,0 +1,236 @@
+// api.cu -- the C ABI (include/glm_dsa.h): host-side argument checks, workspace sizing and the
+// kernel launches of each entry point. Nothing is enqueued unless every check passes.
+#include <cstdint>
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return GLM_OK;
+    g_last_cuda_error = static_cast<int>(e);
+    return GLM_ERR_CUDA;
+}
+
+int num_sms() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Workspace of the sparse MLA: partial accumulators and (m, l) pairs per (query, chunk, head),
+// sized for the smallest chunk any implementation uses.
+size_t mla_workspace(int n_q, int n_heads, int width, int chunk) {
+    const size_t n_chunks = static_cast<size_t>((width + chunk - 1) / chunk);
+    const size_t parts = static_cast<size_t>(n_q) * n_chunks * n_heads;
+    return align_up(parts * glm::kLatent * sizeof(float), 256) + align_up(parts * 2 * sizeof(float), 256);
+}
+
+}  // namespace
+
+extern "C" {
+
+int glm_check_dims(const glm_dsa_dims *d) {
+    if (d == nullptr) return GLM_ERR_INVALID_ARG;
+    if (d->qk_rope_head_dim != 0) return GLM_ERR_UNSUPPORTED;  // NoPE only: zero-width rope slice
+    if (d->kv_lora_rank != glm::kLatent || d->index_n_heads != glm::kIdxHeads ||
+        d->index_head_dim != glm::kIdxDim || d->index_kpool != glm::kKpool)
+        return GLM_ERR_UNSUPPORTED;
+    if (d->n_heads < 1 || d->n_heads > glm::kMaxHeads) return GLM_ERR_UNSUPPORTED;
+    if (d->index_topk <= 0 || d->index_topk % d->index_kpool != 0) return GLM_ERR_INVALID_ARG;
+    return GLM_OK;
+}
+
+const char *glm_status_string(int s) {
+    switch (s) {
+        case GLM_OK: return "ok";
+        case GLM_ERR_INVALID_ARG: return "invalid argument";
+        case GLM_ERR_UNSUPPORTED: return "unsupported geometry";
+        case GLM_ERR_WORKSPACE: return "workspace missing or too small";
+        case GLM_ERR_CUDA: return "CUDA launch failed";
+        default: return "unknown status";
+    }
+}
+
+int glm_last_cuda_error(void) { return g_last_cuda_error; }
+
+int glm_kv_store_int8(const glm_dsa_dims *dims, const void *latent, const int64_t *slots,
+                      int64_t n, int8_t *cache, int64_t n_rows, void *stream) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n < 0 || n_rows < 0) return GLM_ERR_INVALID_ARG;
+    if (n == 0) return GLM_OK;
+    if (!latent || !slots || !cache) return GLM_ERR_INVALID_ARG;
+    if (!aligned(latent, 16) || !aligned(cache, 16) || !aligned(slots, 8)) return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_store_int8(latent, slots, n, cache, n_rows,
+                                              static_cast<cudaStream_t>(stream), num_sms()));
+}
+
+int glm_kpool_build(const glm_dsa_dims *dims, const void *k, const void *gate, int64_t ld_tokens,
+                    const float *ln_w, const float *ln_b, float ln_eps, const int32_t *pad,
+                    const int32_t *len, const int32_t *pool_begin, int32_t batch,
+                    int32_t max_new_pools, float *pooled, int64_t ld_pools, int32_t *n_pools,
+                    void *stream) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (batch < 0 || max_new_pools < 0 || ld_tokens < 0 || ld_pools < 0) return GLM_ERR_INVALID_ARG;
+    if (!(ln_eps >= 0.0f)) return GLM_ERR_INVALID_ARG;
+    if (batch == 0) return GLM_OK;
+    if (!k || !gate || !ln_w || !ln_b || !pad || !len || !pooled) return GLM_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(gate, 16) || !aligned(ln_w, 16) || !aligned(ln_b, 16) ||
+        !aligned(pooled, 16) || !aligned(pad, 4) || !aligned(len, 4) ||
+        (pool_begin && !aligned(pool_begin, 4)) || (n_pools && !aligned(n_pools, 4)))
+        return GLM_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(batch) * max_new_pools > (int64_t(1) << 40)) return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_kpool_build(k, gate, ld_tokens, ln_w, ln_b, ln_eps, pad, len,
+                                               pool_begin, batch, max_new_pools, pooled, ld_pools,
+                                               n_pools, static_cast<cudaStream_t>(stream), num_sms()));
+}
+
+size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
+                              int64_t max_pools, int32_t select_k, int32_t width) {
+    if (glm_check_dims(dims) != GLM_OK || n_q < 0) return static_cast<size_t>(-1);
+    switch (op) {
+        case GLM_OP_INDEX_SCORES_TOPK:
+            if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
+            return align_up(static_cast<size_t>(n_q) * static_cast<size_t>(max_pools) * sizeof(float), 256);
+        case GLM_OP_TOPK_POOLS:
+            if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
+            return 0;
+        case GLM_OP_SPARSE_MLA:
+            if (width < 1 || width > 65536) return static_cast<size_t>(-1);
+            return mla_workspace(n_q, dims->n_heads, width, glm::mla_simt_chunk());
+        default:
+            return static_cast<size_t>(-1);
+    }
+}
+
+int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const float *w,
+                          const float *pooled, int64_t ld_pools, const int32_t *q_seq,
+                          const int32_t *q_pos, const int32_t *pad, const int32_t *len,
+                          int32_t batch, int32_t n_q, int32_t select_k, float *scores,
+                          int32_t *topk, int32_t *n_sel, void *workspace, size_t ws_bytes,
+                          void *stream) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_q < 0 || batch < 0 || ld_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect ||
+        n_q > 65535 || ld_pools > (int64_t(1) << 31) / 128)
+        return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (batch == 0 || !q_idx || !w || !q_seq || !q_pos || !pad || !len || !topk) return GLM_ERR_INVALID_ARG;
+    if (ld_pools > 0 && !pooled) return GLM_ERR_INVALID_ARG;
+    if (!aligned(q_idx, 16) || !aligned(w, 4) || (pooled && !aligned(pooled, 16)) ||
+        !aligned(q_seq, 4) || !aligned(q_pos, 4) || !aligned(pad, 4) || !aligned(len, 4) ||
+        !aligned(topk, 4) || (n_sel && !aligned(n_sel, 4)) || (scores && !aligned(scores, 4)))
+        return GLM_ERR_INVALID_ARG;
+    const size_t need = glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, n_q, ld_pools, select_k, 0);
+    float *sbuf = scores;
+    if (sbuf == nullptr) {
+        if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned(workspace, 16))) return GLM_ERR_WORKSPACE;
+        sbuf = static_cast<float *>(workspace);
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (ld_pools > 0) {
+        rc = cuda_status(glm::launch_index_scores_simt(q_idx, w, pooled, ld_pools, q_seq, q_pos,
+                                                       pad, len, batch, n_q, sbuf, st));
+        if (rc != GLM_OK) return rc;
+    }
+    return cuda_status(glm::launch_topk_fused(sbuf, ld_pools, q_seq, q_pos, pad, len, batch, n_q,
+                                              select_k, topk, n_sel, st));
+}
+
+int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w,
+                     const float *pooled, int64_t ld_pools, const int32_t *q_seq,
+                     const int32_t *q_pos, const int32_t *pad, const int32_t *len, int32_t batch,
+                     int32_t n_q, float *scores, void *stream) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_q < 0 || batch < 0 || ld_pools < 0 || n_q > 65535 || ld_pools > (int64_t(1) << 31) / 128)
+        return GLM_ERR_INVALID_ARG;
+    if (n_q == 0 || ld_pools == 0) return GLM_OK;
+    if (batch == 0 || !q_idx || !w || !pooled || !q_seq || !q_pos || !pad || !len || !scores)
+        return GLM_ERR_INVALID_ARG;
+    if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(pooled, 16) || !aligned(q_seq, 4) ||
+        !aligned(q_pos, 4) || !aligned(pad, 4) || !aligned(len, 4) || !aligned(scores, 4))
+        return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_index_scores_simt(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad,
+                                                     len, batch, n_q, scores,
+                                                     static_cast<cudaStream_t>(stream)));
+}
+
+int glm_topk_pools(const float *scores, int64_t ld_scores, const int32_t *n_visible, int32_t n_q,
+                   int32_t select_k, int32_t *topk, int32_t *n_sel, void *workspace,
+                   size_t ws_bytes, void *stream) {
+    (void)workspace;
+    (void)ws_bytes;
+    if (n_q < 0 || ld_scores < 0 || select_k < 1 || select_k > glm::kMaxSelect || n_q > (1 << 30))
+        return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (!n_visible || !topk || (ld_scores > 0 && !scores)) return GLM_ERR_INVALID_ARG;
+    if ((scores && !aligned(scores, 4)) || !aligned(n_visible, 4) || !aligned(topk, 4) ||
+        (n_sel && !aligned(n_sel, 4)))
+        return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_topk_given(scores, ld_scores, n_visible, n_q, select_k, topk,
+                                              n_sel, static_cast<cudaStream_t>(stream)));
+}
+
+int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk, const int32_t *n_sel,
+                         const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad,
+                         const int32_t *len, int32_t batch, int32_t n_q, int32_t select_k,
+                         const int64_t *slot_map, int64_t ld_slot, int32_t out_width,
+                         int32_t *tok, int32_t *rows, void *stream) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_q < 0 || batch < 0 || select_k < 1 || select_k > (1 << 24) || out_width < 1 || ld_slot < 0 ||
+        n_q > (1 << 30))
+        return GLM_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(out_width) < static_cast<int64_t>(glm::kKpool) * select_k + glm::kKpool - 1)
+        return GLM_ERR_INVALID_ARG;  // the largest selection plus a full tail must fit
+    if (n_q == 0) return GLM_OK;
+    if (batch == 0 || !topk || !q_seq || !q_pos || !pad || !len || (!tok && !rows)) return GLM_ERR_INVALID_ARG;
+    if (!aligned(topk, 4) || (n_sel && !aligned(n_sel, 4)) || !aligned(q_seq, 4) ||
+        !aligned(q_pos, 4) || !aligned(pad, 4) || !aligned(len, 4) ||
+        (slot_map && !aligned(slot_map, 8)) || (tok && !aligned(tok, 4)) || (rows && !aligned(rows, 4)))
+        return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_expand(topk, n_sel, q_seq, q_pos, pad, len, batch, n_q, select_k,
+                                          slot_map, ld_slot, out_width, tok, rows,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t *cache,
+                          int64_t n_rows, const int32_t *rows, int32_t n_q, int32_t width,
+                          float sm_scale, void *out, float *lse, float *out_f32, void *workspace,
+                          size_t ws_bytes, void *stream) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_q < 0 || n_rows < 0 || width < 1 || width > 65536 || n_q > 65535) return GLM_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale)) return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (!q || !rows || !out || (n_rows > 0 && !cache)) return GLM_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || (cache && !aligned(cache, 16)) || !aligned(rows, 4) || !aligned(out, 16) ||
+        (lse && !aligned(lse, 4)) || (out_f32 && !aligned(out_f32, 16)))
+        return GLM_ERR_INVALID_ARG;
+    const int H = dims->n_heads;
+    const size_t need = glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width);
+    if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
+    const int chunk = glm::mla_simt_chunk();
+    const int n_chunks = (width + chunk - 1) / chunk;
+    const size_t parts = static_cast<size_t>(n_q) * n_chunks * H;
+    float *part_acc = static_cast<float *>(workspace);
+    float *part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
+                                               align_up(parts * glm::kLatent * sizeof(float), 256));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = cuda_status(glm::launch_mla_split_simt(q, H, cache, n_rows, rows, n_q, width, sm_scale,
+                                                part_acc, part_ml, st));
+    if (rc != GLM_OK) return rc;
+    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32, lse, st));
+}
+
+}  // extern "C"

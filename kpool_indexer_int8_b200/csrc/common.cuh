@@ -1,0 +1,53 @@
+// common.cuh -- small device helpers shared by the kernels of the kpool DSA decode path.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "glm_dsa.h"
+
+namespace glm {
+
+constexpr int kLatent = 512;        // kv_lora_rank
+constexpr int kRowBytes = 528;      // 512 codes + fp32 scale + 12 zero bytes
+constexpr int kIdxHeads = 32;       // indexer heads
+constexpr int kIdxDim = 128;        // indexer head dim
+constexpr int kKpool = 4;           // tokens per pool
+constexpr int kMaxSelect = 2048;    // largest select_k the top-k kernel sorts on chip
+constexpr int kMaxHeads = 128;      // largest n_heads of the MLA kernels
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+    return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+// Order-preserving map of an fp32 score to an unsigned key (larger score -> larger key);
+// -0.0 is folded onto +0.0 first so that the two compare equal.
+__device__ __forceinline__ uint32_t score_key(float s) {
+    uint32_t u = __float_as_uint(s == 0.0f ? 0.0f : s);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// Number of pools visible to a query at q_pos of a sequence (pad, len): complete pools whose
+// four slots are all at or before q_pos, capped at the pooled-key buffer's capacity.
+__device__ __forceinline__ int visible_pools(int pad, int len, int q_pos, long long ld_pools) {
+    int upto = q_pos - pad + 1;
+    if (upto < 0) upto = 0;
+    int n = min(len, upto) / kKpool;
+    if (len < 0) n = 0;
+    return static_cast<int>(min(static_cast<long long>(n), ld_pools));
+}
+
+}  // namespace glm

@@ -1,0 +1,34 @@
+// kernels.cuh -- launchers behind the C ABI (one per kernel family).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sparse_mla.cuh"
+
+namespace glm {
+
+cudaError_t launch_store_int8(const void *latent, const int64_t *slots, int64_t n, int8_t *cache,
+                              int64_t n_rows, cudaStream_t stream, int num_sms);
+cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_tokens,
+                               const float *ln_w, const float *ln_b, float eps,
+                               const int32_t *pad, const int32_t *len, const int32_t *pool_begin,
+                               int batch, int max_new_pools, float *pooled, int64_t ld_pools,
+                               int32_t *n_pools, cudaStream_t stream, int num_sms);
+cudaError_t launch_index_scores_simt(const void *q_idx, const float *w, const float *pooled,
+                                     int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
+                                     const int32_t *pad, const int32_t *len, int batch, int n_q,
+                                     float *scores, cudaStream_t stream);
+cudaError_t launch_topk_fused(const float *scores, int64_t ld_scores, const int32_t *q_seq,
+                              const int32_t *q_pos, const int32_t *pad, const int32_t *len,
+                              int batch, int n_q, int select_k, int32_t *topk, int32_t *n_sel,
+                              cudaStream_t stream);
+cudaError_t launch_topk_given(const float *scores, int64_t ld_scores, const int32_t *n_visible,
+                              int n_q, int select_k, int32_t *topk, int32_t *n_sel,
+                              cudaStream_t stream);
+cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32_t *q_seq,
+                          const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
+                          int n_q, int select_k, const int64_t *slot_map, int64_t ld_slot, int out_width,
+                          int32_t *tok, int32_t *rows, cudaStream_t stream);
+
+}  // namespace glm

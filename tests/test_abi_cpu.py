@@ -1,0 +1,101 @@
+"""The C-ABI library loads, exports every function include/glm_dsa.h declares, and rejects bad
+arguments on the host before any CUDA call (so these run without a GPU)."""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+kp = pytest.importorskip("kpool_indexer_int8_b200")
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "glm_dsa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(glm_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = _declared()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(kp.lib, n), n
+    assert set(kp.EXPORTS) <= set(names)
+
+
+def test_dims_check_nope_and_geometry():
+    ok = kp.make_dims(64)
+    assert kp.check_dims(ok) == kp.GLM_OK
+    assert kp.check_dims(kp.make_dims(64, qk_rope_head_dim=64)) == kp.GLM_ERR_UNSUPPORTED
+    assert kp.check_dims(kp.make_dims(64, kv_lora_rank=576)) == kp.GLM_ERR_UNSUPPORTED
+    assert kp.check_dims(kp.make_dims(64, index_kpool=8)) == kp.GLM_ERR_UNSUPPORTED
+    assert kp.check_dims(kp.make_dims(0)) == kp.GLM_ERR_UNSUPPORTED
+    assert kp.check_dims(kp.make_dims(129)) == kp.GLM_ERR_UNSUPPORTED
+    assert kp.check_dims(kp.make_dims(16, index_topk=2047)) == kp.GLM_ERR_INVALID_ARG
+    assert kp.lib.glm_check_dims(None) == kp.GLM_ERR_INVALID_ARG
+    assert kp.lib.glm_status_string(kp.GLM_ERR_WORKSPACE) == b"workspace missing or too small"
+
+
+def test_workspace_sizes():
+    d = kp.make_dims(64)
+    assert kp.glm_dsa_workspace_size(d, kp.GLM_OP_INDEX_SCORES_TOPK, 1, 65536, 512) >= 65536 * 4
+    mla = kp.glm_dsa_workspace_size(d, kp.GLM_OP_SPARSE_MLA, 1, width=2176)
+    assert mla >= 2176 // 64 * 64 * 512 * 4
+    assert kp.glm_dsa_workspace_size(d, kp.GLM_OP_SPARSE_MLA, 2, width=2176) >= 2 * mla - 512
+    with pytest.raises(kp.GlmError):
+        kp.glm_dsa_workspace_size(d, kp.GLM_OP_INDEX_SCORES_TOPK, 1, 100, 4096)
+    with pytest.raises(kp.GlmError):
+        kp.glm_dsa_workspace_size(d, 99, 1)
+    with pytest.raises(kp.GlmError):
+        kp.glm_dsa_workspace_size(kp.make_dims(64, qk_rope_head_dim=64), kp.GLM_OP_SPARSE_MLA, 1, width=8)
+
+
+FAKE = C.c_void_p(0x10000)        # 16-byte aligned, never dereferenced: every call below fails first
+MIS = C.c_void_p(0x10004)         # misaligned for 16-byte operands
+
+
+def test_store_rejects_before_launch():
+    L = kp.lib
+    d = C.byref(kp.make_dims(64))
+    bad = C.byref(kp.make_dims(64, qk_rope_head_dim=64))
+    assert L.glm_kv_store_int8(bad, FAKE, FAKE, 1, FAKE, 1, None) == kp.GLM_ERR_UNSUPPORTED
+    assert L.glm_kv_store_int8(d, FAKE, FAKE, -1, FAKE, 1, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kv_store_int8(d, None, FAKE, 1, FAKE, 1, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kv_store_int8(d, MIS, FAKE, 1, FAKE, 1, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kv_store_int8(d, FAKE, FAKE, 1, MIS, 1, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kv_store_int8(d, None, None, 0, None, 0, None) == kp.GLM_OK   # n == 0: no-op
+
+
+def test_expand_requires_room_for_selection_and_tail():
+    L = kp.lib
+    d = C.byref(kp.make_dims(64))
+    # out_width must be >= 4 * select_k + 3
+    assert L.glm_expand_selection(d, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 512, None, 0, 2050,
+                                  FAKE, None, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_expand_selection(d, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1, 0, 512, None, 0, 2051,
+                                  FAKE, None, None) == kp.GLM_OK          # n_q == 0: no-op
+    assert L.glm_expand_selection(d, FAKE, None, FAKE, FAKE, FAKE, FAKE, 1, 1, 512, None, 0, 2051,
+                                  None, None, None) == kp.GLM_ERR_INVALID_ARG  # no output
+
+
+def test_index_and_mla_argument_checks():
+    L = kp.lib
+    d = C.byref(kp.make_dims(64))
+    # select_k out of range
+    assert L.glm_index_scores_topk(d, FAKE, FAKE, FAKE, 16, FAKE, FAKE, FAKE, FAKE, 1, 1, 4096, None,
+                                   FAKE, None, FAKE, 1 << 20, None) == kp.GLM_ERR_INVALID_ARG
+    # missing workspace when scores are not given
+    assert L.glm_index_scores_topk(d, FAKE, FAKE, FAKE, 16, FAKE, FAKE, FAKE, FAKE, 1, 1, 8, None,
+                                   FAKE, None, None, 0, None) == kp.GLM_ERR_WORKSPACE
+    # MLA: workspace too small, width out of range, misaligned q
+    assert L.glm_sparse_mla_decode(d, FAKE, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None, FAKE, 16,
+                                   None) == kp.GLM_ERR_WORKSPACE
+    assert L.glm_sparse_mla_decode(d, FAKE, FAKE, 10, FAKE, 1, 0, 0.04, FAKE, None, None, FAKE, 1 << 30,
+                                   None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_sparse_mla_decode(d, MIS, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None, FAKE, 1 << 30,
+                                   None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_topk_pools(FAKE, 16, FAKE, 1, 0, FAKE, None, None, 0, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kpool_build(d, FAKE, FAKE, 16, FAKE, FAKE, C.c_float(-1.0), FAKE, FAKE, None, 1, 1,
+                             FAKE, 4, None, None) == kp.GLM_ERR_INVALID_ARG

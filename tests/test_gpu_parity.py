@@ -1,0 +1,433 @@
+"""Parity of the CUDA path (through the C ABI) with the fp64 oracle, on the same seeded inputs.
+
+Agreement rules
+  * int8 cache rows, index lists (top-k ids, tokens, cache rows): bit-exact.
+  * top-k: bit-exact when fed the oracle's scores rounded to fp32 (both sides select on the same
+    fp32 values); in the chained path the GPU selection may differ from the oracle's only among
+    pools whose oracle score lies within 1e-4 (relative) of the select_k-th score.
+  * index scores: max over (n, p) of |g - o| / max(|o|, 1e-3 * max_p |o[n, p]|) <= 1e-4.
+  * attention output: max abs err <= 1e-2 and relative L2 error <= 5e-3 against the oracle on the
+    same int8 rows; lse within 1e-3 absolute.
+  * pooled keys (fp32 kernel, fp64 oracle): |g - o| <= 2e-5 * (1 + |o|). Derivation: the LayerNorm
+    sums 128 fp32 terms (relative error <= ~128 * 2**-24 = 7.6e-6 of the largest term, typically
+    ~1e-6), the slot softmax adds a few ulps, so 2e-5 leaves a margin of ~3x over the worst case.
+"""
+import numpy as np
+import pytest
+import torch
+
+import kpool_indexer_int8_b200 as kp
+import oracle
+import synth
+from kpool_indexer_int8_b200 import pipeline as P
+from synth import device as sdev
+
+pytestmark = pytest.mark.gpu
+
+POISON = 0x5A
+
+
+def np_(t):
+    return t.detach().cpu().numpy()
+
+
+def to_dev(a, dtype, dev):
+    return sdev._t(a, dtype, dev)
+
+
+def score_rel_err(g, o):
+    o = np.asarray(o, np.float64)
+    g = np.asarray(g, np.float64)
+    if o.size == 0:
+        return 0.0
+    den = np.maximum(np.abs(o), 1e-3 * np.abs(o).max())
+    den[den == 0] = 1.0
+    return float((np.abs(g - o) / den).max())
+
+
+def attn_errors(g, o):
+    g = np.asarray(g, np.float64)
+    o = np.asarray(o, np.float64)
+    max_abs = float(np.abs(g - o).max()) if o.size else 0.0
+    nrm = np.linalg.norm(o)
+    rel_l2 = float(np.linalg.norm(g - o) / nrm) if nrm > 0 else float(np.linalg.norm(g))
+    return max_abs, rel_l2
+
+
+def assert_attention_close(g, o, what=""):
+    max_abs, rel_l2 = attn_errors(g, o)
+    assert max_abs <= 1e-2 and rel_l2 <= 5e-3, (what, max_abs, rel_l2)
+
+
+# ------------------------------------------------------------------------------------------------
+# store_int8
+# ------------------------------------------------------------------------------------------------
+
+def _store_both(cuda, latent, slots, n_rows):
+    dims = kp.make_dims(16)
+    co = np.full((n_rows, 528), POISON, dtype=np.int8)
+    ok = (slots >= 0) & (slots < n_rows)
+    oracle.store_int8(latent[ok], slots[ok], co)
+    cg = torch.full((n_rows, 528), POISON, dtype=torch.int8, device=cuda)
+    kp.glm_kv_store_int8(dims, to_dev(latent, torch.bfloat16, cuda), to_dev(slots, torch.int64, cuda), cg)
+    torch.cuda.synchronize()
+    return np_(cg), co
+
+
+@pytest.mark.parametrize("wl", [synth.TINY_DECODE, synth.PADDING_DECODE,
+                                synth.custom("permuted", (0, 3), (1000, 517), permute_slots=True,
+                                             outlier_frac=0.05)])
+def test_store_int8_bit_exact(cuda, wl):
+    inp = synth.generate(wl)
+    g, o = _store_both(cuda, inp.latent, inp.slots, inp.n_rows)
+    assert np.array_equal(g, o)
+
+
+def test_store_int8_edge_rows(cuda):
+    # zero rows (amax floor), exact halves (ties to even), the largest bf16 magnitudes, tiny values,
+    # negative slots (no write) and slots past the cache (skipped, never written)
+    rng = np.random.default_rng(0)
+    x = np.zeros((8, 512), np.float32)
+    x[1, :11] = [127, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -0.5, 126.5, -127, -1.5]
+    x[2] = rng.standard_normal(512) * 1e-7
+    x[3] = rng.standard_normal(512) * 3e38 / 5
+    x[4] = -np.abs(rng.standard_normal(512))
+    x[5, 0] = 1.0
+    x[6] = rng.standard_normal(512)
+    x[7] = rng.standard_normal(512)
+    lat = synth.f32_to_bf16_bits(x)
+    slots = np.array([0, 1, 2, 3, 4, -1, 6, 9], dtype=np.int64)   # 9 >= n_rows: skipped
+    g, o = _store_both(cuda, lat, slots, 8)
+    assert np.array_equal(g, o)
+    assert (g[5] == POISON).all() and (g[7] == POISON).all()
+    assert list(g[1, :11]) == [127, 2, 4, -2, -4, 0, 2, 0, 126, -127, -2]
+
+
+def test_store_int8_full_size(cuda):
+    # the long-decode cache: 262,144 rows with 1% outliers, compared in full
+    inp = synth.generate(synth.LONG_DECODE)
+    g, o = _store_both(cuda, inp.latent, inp.slots, inp.n_rows)
+    assert np.array_equal(g, o)
+
+
+# ------------------------------------------------------------------------------------------------
+# kpool_build
+# ------------------------------------------------------------------------------------------------
+
+def _pooled_close(g, o):
+    assert g.shape == o.shape
+    err = np.abs(g.astype(np.float64) - o)
+    assert (err <= 2e-5 * (1 + np.abs(o))).all(), float((err / (1 + np.abs(o))).max())
+
+
+@pytest.mark.parametrize("wl", [synth.TINY_DECODE, synth.PADDING_DECODE])
+def test_kpool_build_full_and_incremental(cuda, wl):
+    inp = synth.generate(wl)
+    pools_o = oracle.build_pools(inp)
+    b = sdev.allocate_for(inp, cuda)
+    sdev.load(inp, b, build_prefix=False)
+    b.pooled.fill_(float("nan"))
+    n_pools = torch.full((wl.batch,), -7, dtype=torch.int32, device=cuda)
+    kp.glm_kpool_build(b.dims, b.k, b.gate, b.ln_w, b.ln_b, wl.ln_eps, b.pad, b.len, b.pooled,
+                       pool_begin=None, max_new_pools=b.pooled.shape[1], n_pools=n_pools)
+    pg = np_(b.pooled)
+    assert list(np_(n_pools)) == [p.shape[0] for p in pools_o]
+    for s, po in enumerate(pools_o):
+        _pooled_close(pg[s, :po.shape[0]], po)
+        assert np.isnan(pg[s, po.shape[0]:]).all()        # no pool past the last complete one
+    # incremental: rebuild only pools [n-3, n-1) of each sequence into a fresh buffer
+    b.pooled.fill_(float("nan"))
+    nps = np.array([p.shape[0] for p in pools_o])
+    begin = np.maximum(nps - 3, 0).astype(np.int32)
+    kp.glm_kpool_build(b.dims, b.k, b.gate, b.ln_w, b.ln_b, wl.ln_eps, b.pad, b.len, b.pooled,
+                       pool_begin=to_dev(begin, torch.int32, cuda), max_new_pools=2)
+    pg = np_(b.pooled)
+    for s, po in enumerate(pools_o):
+        lo, hi = begin[s], min(begin[s] + 2, po.shape[0])
+        _pooled_close(pg[s, lo:hi], po[lo:hi])
+        assert np.isnan(pg[s, :lo]).all() and np.isnan(pg[s, hi:]).all()
+
+
+# ------------------------------------------------------------------------------------------------
+# index scores and top-k
+# ------------------------------------------------------------------------------------------------
+
+def _oracle_scores_on(inp, pooled32):
+    res = []
+    for n in range(len(inp.q_pos)):
+        s = int(inp.q_seq[n])
+        nv = oracle.n_visible_pools(inp.pad[s], inp.len[s], inp.q_pos[n])
+        res.append(oracle.index_scores(inp.q_idx[n], inp.w[n], pooled32[s], nv))
+    return res
+
+
+@pytest.mark.parametrize("wl", [synth.TINY_DECODE, synth.PADDING_DECODE,
+                                synth.custom("causal", (0,), (3000,), select_k=64, chunk=37)])
+def test_index_scores_match_oracle(cuda, wl):
+    inp = synth.generate(wl)
+    pools_o = oracle.build_pools(inp)
+    b = sdev.allocate_for(inp, cuda, keep_scores=True)
+    sdev.load(inp, b, build_prefix=False)
+    ld = b.pooled.shape[1]
+    p32 = np.zeros((wl.batch, ld, 128), np.float32)          # the oracle's pools rounded to fp32
+    for s, po in enumerate(pools_o):
+        p32[s, :po.shape[0]] = po
+    b.pooled.copy_(torch.from_numpy(p32))
+    b.scores.fill_(12345.0)
+    P.index_topk(b)
+    sg = np_(b.scores)
+    for n, so in enumerate(_oracle_scores_on(inp, p32)):
+        assert score_rel_err(sg[n, :len(so)], so) <= 1e-4
+        assert np.isneginf(sg[n, len(so):]).all()
+
+
+def _topk_given(cuda, scores32, n_vis, S):
+    nq, ld = scores32.shape
+    topk = torch.full((nq, S), 777, dtype=torch.int32, device=cuda)
+    n_sel = torch.full((nq,), 777, dtype=torch.int32, device=cuda)
+    kp.glm_topk_pools(torch.from_numpy(scores32).to(cuda), to_dev(n_vis, torch.int32, cuda), S, topk,
+                      n_sel=n_sel)
+    return np_(topk), np_(n_sel)
+
+
+@pytest.mark.parametrize("n,S,ties", [(0, 8, False), (5, 8, False), (8, 8, False), (300, 16, False),
+                                      (300, 16, True), (5000, 512, True), (5000, 1, True),
+                                      (4100, 2048, False), (65536, 512, False), (65536, 512, True),
+                                      (100000, 2048, True)])
+def test_topk_bit_exact_on_oracle_scores(cuda, n, S, ties):
+    rng = np.random.default_rng(n + S)
+    s = rng.standard_normal(max(n, 1)) * 20 + 60
+    if ties:
+        s = np.round(s * 4) / 4                        # heavy ties
+        s[rng.random(s.shape) < 0.05] = 0.0
+        s[rng.random(s.shape) < 0.05] = -0.0
+    s32 = s.astype(np.float32)
+    scores = np.full((2, max(n, 1) + 3), np.nan, np.float32)   # entries past n_vis are never read
+    scores[0, :max(n, 1)] = s32
+    scores[1, :max(n, 1)] = -s32                        # negative scores too
+    n_vis = np.array([n, max(0, n - 1)], dtype=np.int32)
+    tg, ng = _topk_given(cuda, scores, n_vis, S)
+    for q in range(2):
+        want, n_sel = oracle.topk_pools(scores[q, :n_vis[q]].astype(np.float64), S)
+        assert np.array_equal(tg[q], want), q
+        assert ng[q] == n_sel
+
+
+def test_index_topk_fused_selection(cuda):
+    inp = synth.generate(synth.PADDING_DECODE)
+    pools_o = oracle.build_pools(inp)
+    b = sdev.allocate_for(inp, cuda)
+    sdev.load(inp, b, build_prefix=False)
+    p32 = np.zeros(tuple(b.pooled.shape), np.float32)
+    for s, po in enumerate(pools_o):
+        p32[s, :po.shape[0]] = po
+    b.pooled.copy_(torch.from_numpy(p32))
+    b.topk.fill_(555)
+    P.index_topk(b)
+    tg, ng = np_(b.topk), np_(b.n_sel)
+    for n, so in enumerate(_oracle_scores_on(inp, p32)):
+        want, n_sel = oracle.topk_pools(so, inp.wl.select_k)
+        assert ng[n] == n_sel
+        _selection_agrees(tg[n], want, so, n_sel)
+
+
+def _selection_agrees(got, want, scores, n_sel):
+    """Equal, except that pools whose score is within 1e-4 (relative) of the select_k-th score
+    may be exchanged among themselves."""
+    assert (got[n_sel:] == -1).all()
+    if np.array_equal(got, want) or n_sel == 0:
+        return 0
+    thr = scores[want[n_sel - 1]]
+    tol = 1e-4 * max(abs(thr), 1e-30)
+    gs, ws = set(got[:n_sel].tolist()), set(want[:n_sel].tolist())
+    for p in gs ^ ws:
+        assert abs(scores[p] - thr) <= tol, (p, scores[p], thr)
+    assert len(gs) == n_sel
+    return len(gs ^ ws) // 2
+
+
+# ------------------------------------------------------------------------------------------------
+# expand_selection
+# ------------------------------------------------------------------------------------------------
+
+@pytest.mark.parametrize("wl", [synth.TINY_DECODE, synth.PADDING_DECODE,
+                                synth.custom("edge", (5, 0, 2), (3, 7, 4), select_k=4, out_width=19),
+                                synth.custom("causal_e", (1,), (800,), select_k=8, chunk=23,
+                                             permute_slots=True)])
+@pytest.mark.parametrize("with_nsel", [True, False])
+def test_expand_bit_exact(cuda, wl, with_nsel):
+    inp = synth.generate(wl)
+    rng = np.random.default_rng(1)
+    nq, S, W = len(inp.q_pos), wl.select_k, wl.out_width
+    topk = np.full((nq, S), -1, np.int32)
+    nsel = np.zeros(nq, np.int32)
+    want_tok = np.zeros((nq, W), np.int32)
+    want_rows = np.zeros((nq, W), np.int32)
+    for n in range(nq):
+        s = int(inp.q_seq[n])
+        nv = oracle.n_visible_pools(inp.pad[s], inp.len[s], inp.q_pos[n])
+        topk[n], nsel[n] = oracle.topk_pools(rng.standard_normal(nv), S)
+        want_tok[n], _ = oracle.expand_selection(topk[n], nsel[n], inp.pad[s], inp.len[s], inp.q_pos[n], W)
+        want_rows[n] = oracle.rows_from_tokens(want_tok[n], inp.slot_map[s])
+    dims = kp.make_dims(wl.n_heads)
+    tok = torch.full((nq, W), 999, dtype=torch.int32, device=cuda)
+    rows = torch.full((nq, W), 999, dtype=torch.int32, device=cuda)
+    kp.glm_expand_selection(dims, to_dev(topk, torch.int32, cuda), to_dev(inp.q_seq, torch.int32, cuda),
+                            to_dev(inp.q_pos, torch.int32, cuda), to_dev(inp.pad, torch.int32, cuda),
+                            to_dev(inp.len, torch.int32, cuda), W,
+                            n_sel=to_dev(nsel, torch.int32, cuda) if with_nsel else None,
+                            slot_map=to_dev(inp.slot_map, torch.int64, cuda), tok=tok, rows=rows)
+    assert np.array_equal(np_(tok), want_tok)
+    assert np.array_equal(np_(rows), want_rows)
+    # without a slot map the rows are the tokens themselves
+    rows2 = torch.full((nq, W), 999, dtype=torch.int32, device=cuda)
+    kp.glm_expand_selection(dims, to_dev(topk, torch.int32, cuda), to_dev(inp.q_seq, torch.int32, cuda),
+                            to_dev(inp.q_pos, torch.int32, cuda), to_dev(inp.pad, torch.int32, cuda),
+                            to_dev(inp.len, torch.int32, cuda), W, rows=rows2)
+    assert np.array_equal(np_(rows2), want_tok)
+
+
+# ------------------------------------------------------------------------------------------------
+# sparse MLA
+# ------------------------------------------------------------------------------------------------
+
+def _mla_case(cuda, n_heads, rows, cache, q, sm):
+    nq, W = rows.shape
+    dims = kp.make_dims(n_heads)
+    ws = torch.empty(kp.glm_dsa_workspace_size(dims, kp.GLM_OP_SPARSE_MLA, nq, width=W), dtype=torch.uint8,
+                     device=cuda)
+    ws.fill_(0xFF)                                       # NaN-filled scratch must not leak through
+    out = torch.full((nq, n_heads, 512), 7.0, dtype=torch.bfloat16, device=cuda)
+    o32 = torch.full((nq, n_heads, 512), 7.0, dtype=torch.float32, device=cuda)
+    lse = torch.full((nq, n_heads), 7.0, dtype=torch.float32, device=cuda)
+    kp.glm_sparse_mla_decode(dims, to_dev(q, torch.bfloat16, cuda), torch.from_numpy(cache).to(cuda),
+                             to_dev(rows, torch.int32, cuda), sm, out, ws, lse=lse, out_f32=o32)
+    return np_(out.float()), np_(o32), np_(lse)
+
+
+@pytest.mark.parametrize("n_heads,W,n_valid,n_rows", [(16, 80, 64, 512), (64, 2176, 2048, 5000),
+                                                      (64, 2176, 2051, 3000), (128, 67, 67, 100),
+                                                      (64, 1, 1, 10), (16, 300, 0, 10),
+                                                      (64, 200, 3, 50), (16, 1000, 999, 5000)])
+def test_sparse_mla_matches_oracle(cuda, n_heads, W, n_valid, n_rows):
+    rng = np.random.default_rng(W + n_heads)
+    lat = synth.f32_to_bf16_bits(rng.standard_normal((n_rows, 512)).astype(np.float32))
+    lat[rng.random(n_rows) < 0.01] = synth.f32_to_bf16_bits(rng.standard_normal((1, 512)).astype(np.float32) * 8)
+    cache = np.zeros((n_rows, 528), np.int8)
+    oracle.store_int8(lat, np.arange(n_rows, dtype=np.int64), cache)
+    nq = 3
+    rows = np.full((nq, W), -1, np.int32)
+    for n in range(nq):
+        r = rng.choice(n_rows, size=min(n_valid, n_rows), replace=False).astype(np.int32)
+        pos = rng.choice(W, size=len(r), replace=False) if n == 1 else np.arange(len(r))
+        rows[n, pos] = r                                # query 1 has the -1 entries interleaved
+    q = synth.f32_to_bf16_bits(rng.standard_normal((nq, n_heads, 512)).astype(np.float32))
+    sm = float(np.float32(512 ** -0.5))
+    og, o32, lg = _mla_case(cuda, n_heads, rows, cache, q, sm)
+    for n in range(nq):
+        oo, lo = oracle.sparse_mla(q[n], cache, rows[n], sm)
+        assert_attention_close(o32[n], oo, "f32")
+        assert_attention_close(og[n], oo, "bf16")
+        if n_valid == 0:
+            assert np.isneginf(lg[n]).all() and not o32[n].any() and not og[n].any()
+        else:
+            np.testing.assert_allclose(lg[n], lo, atol=1e-3, rtol=0)
+
+
+def test_sparse_mla_skips_out_of_range_rows(cuda):
+    rng = np.random.default_rng(5)
+    n_rows = 64
+    lat = synth.f32_to_bf16_bits(rng.standard_normal((n_rows, 512)).astype(np.float32))
+    cache = np.zeros((n_rows, 528), np.int8)
+    oracle.store_int8(lat, np.arange(n_rows, dtype=np.int64), cache)
+    rows = np.array([[3, 64, 9, 1 << 30, -5, 17, 63]], np.int32)   # 64 and 1<<30 are past the cache
+    q = synth.f32_to_bf16_bits(rng.standard_normal((1, 16, 512)).astype(np.float32))
+    sm = float(np.float32(512 ** -0.5))
+    _, o32, lg = _mla_case(cuda, 16, rows, cache, q, sm)
+    clean = np.where((rows >= 0) & (rows < n_rows), rows, -1)
+    oo, lo = oracle.sparse_mla(q[0], cache, clean[0], sm)
+    assert_attention_close(o32[0], oo)
+
+
+# ------------------------------------------------------------------------------------------------
+# the whole chain
+# ------------------------------------------------------------------------------------------------
+
+def _run_chain(cuda, inp):
+    b = sdev.allocate_for(inp, cuda, keep_scores=True, keep_f32=True)
+    sdev.load(inp, b, build_prefix=True)
+    for t in (b.topk, b.tok, b.rows):
+        t.fill_(4242)
+    b.out.fill_(3.0)
+    P.run_step(b)
+    torch.cuda.synchronize()
+    return b
+
+
+def _check_chain(inp, b, queries=None, check_cache_rows=None):
+    """Compare a GPU step with the oracle's step on the same inputs (oracle state built by the
+    oracle itself). Returns the number of queries whose selection differed inside the tie band."""
+    cache_o = oracle.build_cache(inp)
+    pools_o = oracle.build_pools(inp)
+    cg = np_(b.cache)
+    if check_cache_rows is None:
+        assert np.array_equal(cg, cache_o)
+    else:
+        assert np.array_equal(cg[check_cache_rows], cache_o[check_cache_rows])
+    pg = np_(b.pooled)
+    for s, po in enumerate(pools_o):
+        _pooled_close(pg[s, :po.shape[0]], po)
+    sg, tg, ng, tokg, rowg = np_(b.scores), np_(b.topk), np_(b.n_sel), np_(b.tok), np_(b.rows)
+    o32 = np_(b.out_f32)
+    diffs = 0
+    for n in (range(len(inp.q_pos)) if queries is None else queries):
+        r = oracle.decode_query(inp, n, cache_o, pools_o)
+        nv = r["n_vis"]
+        assert score_rel_err(sg[n, :nv], r["scores"]) <= 1e-4
+        assert ng[n] == r["n_sel"]
+        d = _selection_agrees(tg[n], r["topk"], r["scores"], r["n_sel"])
+        if d == 0:
+            assert np.array_equal(tokg[n], r["tok"]) and np.array_equal(rowg[n], r["rows"])
+            assert_attention_close(o32[n], r["out"], f"query {n}")
+            assert_attention_close(np_(b.out[n].float()), r["out"], f"query {n} bf16")
+        else:
+            diffs += 1
+            # same selection as a set of pools up to the tie band: the tokens are still all valid
+            s = int(inp.q_seq[n])
+            valid = tokg[n][tokg[n] >= 0]
+            assert all(oracle.visible(inp.pad[s], inp.len[s], inp.q_pos[n], t) for t in valid)
+    return diffs
+
+
+@pytest.mark.parametrize("wl", [synth.TINY_DECODE, synth.PADDING_DECODE,
+                                synth.custom("batched_small", (0, 0, 0, 0), (9000, 4099, 20000, 33),
+                                             n_heads=64, select_k=512, out_width=2176,
+                                             permute_slots=True, seed=33),
+                                synth.custom("prefill_small", (0,), (6000,), n_heads=64, select_k=128,
+                                             out_width=515, chunk=300, seed=44)])
+def test_decode_step_matches_oracle(cuda, wl):
+    inp = synth.generate(wl)
+    b = _run_chain(cuda, inp)
+    assert _check_chain(inp, b) <= max(1, len(inp.q_pos) // 10)
+
+
+def test_long_decode_full_size(cuda):
+    # the benchmark's workload and launch configuration: 262,144-token context, 65,536 pools
+    inp = synth.generate(synth.LONG_DECODE)
+    b = _run_chain(cuda, inp)
+    assert _check_chain(inp, b) == 0
+
+
+def test_batched_decode_full_size(cuda):
+    inp = synth.generate(synth.BATCHED_DECODE)
+    b = _run_chain(cuda, inp)
+    rng = np.random.default_rng(0)
+    rows = rng.choice(inp.n_rows, size=20000, replace=False)
+    assert _check_chain(inp, b, check_cache_rows=rows) <= 1
+
+
+def test_chunked_prefill_sampled(cuda):
+    inp = synth.generate(synth.CHUNKED_PREFILL)
+    b = _run_chain(cuda, inp)
+    rows = np.concatenate([np.arange(131072 - 8, 135168), np.arange(0, 4096, 37)])
+    assert _check_chain(inp, b, queries=[0, 1, 2, 3, 1000, 2047, 4095], check_cache_rows=rows) <= 1
