@@ -135,9 +135,10 @@ int glm_kpool_build(const glm_dsa_dims *dims, const void *k_dev, const void *gat
  *   q_seq_dev, q_pos_dev  int32 [n_q];     pad_dev, len_dev  int32 [batch]
  *   scores_dev  fp32 [n_q, ld_pools] or NULL: receives the scores (entries p >= n_vis are -inf)
  *   topk_dev    int32 [n_q, select_k]      n_sel_dev  int32 [n_q] or NULL
- *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, ...)
- * 1 <= select_k <= 2048. The fp32 scores are computed on tensor cores from an exact three-term
- * bf16 split of the pooled keys (max relative error well below 1e-4).
+ *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, ...), 256-byte
+ *               aligned (required even when scores_dev is given; contents on entry are ignored)
+ * 1 <= select_k <= 2048. Scores are fp32 sums of fp32 products of the bf16 queries and the fp32
+ * pooled keys.
  */
 int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx_dev, const float *w_dev,
                           const float *pooled_dev, int64_t ld_pools, const int32_t *q_seq_dev,
@@ -162,6 +163,8 @@ int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx_dev, const floa
  * then -1. Used to check the selection bit-exactly on externally supplied scores.
  *   scores_dev  fp32 [n_q, ld_scores];  n_visible_dev int32 [n_q] (clamped to [0, ld_scores])
  *   topk_dev    int32 [n_q, select_k];  n_sel_dev int32 [n_q] or NULL
+ *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_TOPK_POOLS, n_q, ld_scores, ...),
+ *               256-byte aligned; contents on entry are ignored
  * NaN scores are outside the contract.
  */
 int glm_topk_pools(const float *scores_dev, int64_t ld_scores, const int32_t *n_visible_dev,

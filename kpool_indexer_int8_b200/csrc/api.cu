@@ -25,6 +25,9 @@ int num_sms() {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Per-query 2048-bin histogram of score keys used by the selection (first in the workspace).
+size_t hist_bytes(int n_q) { return align_up(static_cast<size_t>(n_q) * glm::kHistBins * sizeof(unsigned), 256); }
+
 // Workspace of the sparse MLA: partial accumulators and (m, l) pairs per (query, chunk, head),
 // sized for the smallest chunk any implementation uses.
 size_t mla_workspace(int n_q, int n_heads, int width, int chunk) {
@@ -100,10 +103,10 @@ size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
     switch (op) {
         case GLM_OP_INDEX_SCORES_TOPK:
             if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
-            return align_up(static_cast<size_t>(n_q) * static_cast<size_t>(max_pools) * sizeof(float), 256);
+            return hist_bytes(n_q) + align_up(static_cast<size_t>(n_q) * static_cast<size_t>(max_pools) * sizeof(float), 256);
         case GLM_OP_TOPK_POOLS:
             if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
-            return 0;
+            return hist_bytes(n_q);
         case GLM_OP_SPARSE_MLA:
             if (width < 1 || width > 65536) return static_cast<size_t>(-1);
             return mla_workspace(n_q, dims->n_heads, width, glm::mla_simt_chunk());
@@ -131,19 +134,19 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const flo
         !aligned(topk, 4) || (n_sel && !aligned(n_sel, 4)) || (scores && !aligned(scores, 4)))
         return GLM_ERR_INVALID_ARG;
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, n_q, ld_pools, select_k, 0);
-    float *sbuf = scores;
-    if (sbuf == nullptr) {
-        if (need > 0 && (workspace == nullptr || ws_bytes < need || !aligned(workspace, 16))) return GLM_ERR_WORKSPACE;
-        sbuf = static_cast<float *>(workspace);
-    }
+    if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
+    unsigned *ghist = static_cast<unsigned *>(workspace);
+    float *sbuf = scores ? scores : reinterpret_cast<float *>(static_cast<char *>(workspace) + hist_bytes(n_q));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const glm::NvisSource src{nullptr, q_seq, q_pos, pad, len, batch, ld_pools};
     if (ld_pools > 0) {
+        rc = cuda_status(cudaMemsetAsync(ghist, 0, static_cast<size_t>(n_q) * glm::kHistBins * sizeof(unsigned), st));
+        if (rc != GLM_OK) return rc;
         rc = cuda_status(glm::launch_index_scores_simt(q_idx, w, pooled, ld_pools, q_seq, q_pos,
-                                                       pad, len, batch, n_q, sbuf, st));
+                                                       pad, len, batch, n_q, sbuf, ghist, st));
         if (rc != GLM_OK) return rc;
     }
-    return cuda_status(glm::launch_topk_fused(sbuf, ld_pools, q_seq, q_pos, pad, len, batch, n_q,
-                                              select_k, topk, n_sel, st));
+    return cuda_status(glm::launch_topk_select(sbuf, src, ghist, n_q, select_k, topk, n_sel, st));
 }
 
 int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w,
@@ -161,24 +164,30 @@ int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w
         !aligned(q_pos, 4) || !aligned(pad, 4) || !aligned(len, 4) || !aligned(scores, 4))
         return GLM_ERR_INVALID_ARG;
     return cuda_status(glm::launch_index_scores_simt(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad,
-                                                     len, batch, n_q, scores,
+                                                     len, batch, n_q, scores, nullptr,
                                                      static_cast<cudaStream_t>(stream)));
 }
 
 int glm_topk_pools(const float *scores, int64_t ld_scores, const int32_t *n_visible, int32_t n_q,
                    int32_t select_k, int32_t *topk, int32_t *n_sel, void *workspace,
                    size_t ws_bytes, void *stream) {
-    (void)workspace;
-    (void)ws_bytes;
-    if (n_q < 0 || ld_scores < 0 || select_k < 1 || select_k > glm::kMaxSelect || n_q > (1 << 30))
+    if (n_q < 0 || ld_scores < 0 || select_k < 1 || select_k > glm::kMaxSelect || n_q > 65535)
         return GLM_ERR_INVALID_ARG;
     if (n_q == 0) return GLM_OK;
     if (!n_visible || !topk || (ld_scores > 0 && !scores)) return GLM_ERR_INVALID_ARG;
     if ((scores && !aligned(scores, 4)) || !aligned(n_visible, 4) || !aligned(topk, 4) ||
         (n_sel && !aligned(n_sel, 4)))
         return GLM_ERR_INVALID_ARG;
-    return cuda_status(glm::launch_topk_given(scores, ld_scores, n_visible, n_q, select_k, topk,
-                                              n_sel, static_cast<cudaStream_t>(stream)));
+    const size_t need = hist_bytes(n_q);
+    if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
+    unsigned *ghist = static_cast<unsigned *>(workspace);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const glm::NvisSource src{n_visible, nullptr, nullptr, nullptr, nullptr, 0, ld_scores};
+    int rc = cuda_status(cudaMemsetAsync(ghist, 0, static_cast<size_t>(n_q) * glm::kHistBins * sizeof(unsigned), st));
+    if (rc != GLM_OK) return rc;
+    rc = cuda_status(glm::launch_topk_hist(scores, src, n_q, ghist, st));
+    if (rc != GLM_OK) return rc;
+    return cuda_status(glm::launch_topk_select(scores, src, ghist, n_q, select_k, topk, n_sel, st));
 }
 
 int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk, const int32_t *n_sel,
@@ -189,7 +198,7 @@ int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk, const in
     int rc = glm_check_dims(dims);
     if (rc != GLM_OK) return rc;
     if (n_q < 0 || batch < 0 || select_k < 1 || select_k > (1 << 24) || out_width < 1 || ld_slot < 0 ||
-        n_q > (1 << 30))
+        n_q > 65535)
         return GLM_ERR_INVALID_ARG;
     if (static_cast<int64_t>(out_width) < static_cast<int64_t>(glm::kKpool) * select_k + glm::kKpool - 1)
         return GLM_ERR_INVALID_ARG;  // the largest selection plus a full tail must fit

@@ -2,7 +2,7 @@
 // expand_selection and trap 6: expand selected pools into raw token indices, append the visible
 // tail, pad with INVALID; all out_width entries are written).
 //
-// One CTA per query. Entry j < 4*n_sel is token pad + 4*topk[j/4] + j%4; the next `tail`
+// Grid (ceil(out_width / 256), n_q): one thread per output entry. Entry j < 4*n_sel is token pad + 4*topk[j/4] + j%4; the next `tail`
 // entries are pad + 4*n_vis .. q_pos; the rest are -1. The cache row of each token comes from
 // the sequence's slot map (or is the token itself without one).
 #include "common.cuh"
@@ -18,11 +18,12 @@ __global__ void __launch_bounds__(kExpandThreads) expand_kernel(
     const int64_t *__restrict__ slot_map, int64_t ld_slot, int out_width,
     int32_t *__restrict__ tok_out, int32_t *__restrict__ rows_out) {
     __shared__ int s_nsel;
-    const int n = blockIdx.x;
+    const int n = blockIdx.y;
+    const int j = blockIdx.x * blockDim.x + threadIdx.x;
     const int64_t base = static_cast<int64_t>(n) * out_width;
     const int b = q_seq[n];
     if (b < 0 || b >= batch) {  // outside the contract: the whole row is -1
-        for (int j = threadIdx.x; j < out_width; j += blockDim.x) {
+        if (j < out_width) {
             if (tok_out) tok_out[base + j] = GLM_INVALID;
             if (rows_out) rows_out[base + j] = GLM_INVALID;
         }
@@ -42,7 +43,7 @@ __global__ void __launch_bounds__(kExpandThreads) expand_kernel(
     const int last = min(qp, pb + len[b] - 1);  // the tail stops at the query or the sequence end
     const int tail = max(0, last - (pb + kKpool * n_vis) + 1);
     const int n_valid = kKpool * n_sel + tail;
-    for (int j = threadIdx.x; j < out_width; j += blockDim.x) {
+    if (j < out_width) {
         int t = GLM_INVALID;
         if (j < kKpool * n_sel) {
             const int p = tk[j / kKpool];
@@ -69,7 +70,8 @@ cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32
                           const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
                           int n_q, int select_k, const int64_t *slot_map, int64_t ld_slot, int out_width,
                           int32_t *tok, int32_t *rows, cudaStream_t stream) {
-    expand_kernel<<<n_q, kExpandThreads, 0, stream>>>(topk, n_sel, q_seq, q_pos, pad, len, batch, select_k,
+    dim3 grid(static_cast<unsigned>((out_width + kExpandThreads - 1) / kExpandThreads), n_q);
+    expand_kernel<<<grid, kExpandThreads, 0, stream>>>(topk, n_sel, q_seq, q_pos, pad, len, batch, select_k,
                                                       slot_map, ld_slot, out_width, tok, rows);
     return cudaGetLastError();
 }

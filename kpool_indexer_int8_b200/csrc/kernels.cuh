@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include "sparse_mla.cuh"
+#include "topk.cuh"
 
 namespace glm {
 
@@ -18,14 +19,7 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
 cudaError_t launch_index_scores_simt(const void *q_idx, const float *w, const float *pooled,
                                      int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
                                      const int32_t *pad, const int32_t *len, int batch, int n_q,
-                                     float *scores, cudaStream_t stream);
-cudaError_t launch_topk_fused(const float *scores, int64_t ld_scores, const int32_t *q_seq,
-                              const int32_t *q_pos, const int32_t *pad, const int32_t *len,
-                              int batch, int n_q, int select_k, int32_t *topk, int32_t *n_sel,
-                              cudaStream_t stream);
-cudaError_t launch_topk_given(const float *scores, int64_t ld_scores, const int32_t *n_visible,
-                              int n_q, int select_k, int32_t *topk, int32_t *n_sel,
-                              cudaStream_t stream);
+                                     float *scores, unsigned *ghist, cudaStream_t stream);
 cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32_t *q_seq,
                           const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
                           int n_q, int select_k, const int64_t *slot_map, int64_t ld_slot, int out_width,

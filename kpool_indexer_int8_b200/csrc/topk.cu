@@ -1,193 +1,306 @@
 // topk.cu -- selection of the select_k highest-scoring visible pools ("Module glm5next_dsa_ref",
 // topk_pools), ordered by score descending with ties to the lower pool id.
 //
-// One CTA of 1024 threads per query:
-//   1. radix select (four 8-bit digits, most significant first) of the select_k-th largest
-//      32-bit order-preserving score key T, with warp-aggregated shared-memory histograms;
-//   2. one ordered pass that keeps every key > T and the lowest-id keys == T (a block-wide
-//      prefix count in pool-id order decides which of the equal keys are taken);
-//   3. a bitonic sort of the kept (key, ~id) 64-bit composites in shared memory.
-// When n_vis <= select_k every visible pool is kept and only step 3 runs.
+// Keys: the fp32 score mapped to an order-preserving uint32 (-0.0 folded onto +0.0), extended to
+// a unique 64-bit composite (key << 32 | ~pool_id) so that "larger composite" is exactly "higher
+// score, then lower id".
+//
+//   1. histogram: a 2048-bin count of the top 11 key bits per query (built by the score kernel's
+//      epilogue, or by topk_hist_kernel for caller-supplied scores);
+//   2. select kernel, one CTA per query:
+//        a. from the histogram, the bin b* holding the select_k-th largest key and the count of
+//           keys in higher bins (always < select_k);
+//        b. one pass over the scores keeps every key of a higher bin (list A) and every key of
+//           bin b* (list B, in shared memory);
+//        c. a radix select on the composites of B (8-bit digits over the remaining 53 bits,
+//           stopping as soon as the digit holding the boundary is taken whole) picks the rest;
+//        d. a bitonic sort of the select_k composites in shared memory gives the order.
+//      If B exceeds its shared-memory capacity (massive ties at the boundary), step (c) runs the
+//      same radix select over the scores in global memory instead.
 #include "common.cuh"
+#include "topk.cuh"
 
 namespace glm {
 
-constexpr int kTopkThreads = 1024;
-
-struct TopkSmem {
-    unsigned long long cand[kMaxSelect];
-    unsigned int hist[256];
-    unsigned int warp_tot[32];
-    unsigned int prefix, k_rem, n_gt, eq_base;
-};
+constexpr int kSelThreads = 1024;
+constexpr int kBoundCap = 8192;
 
 __device__ __forceinline__ unsigned long long compose(uint32_t key, int id) {
-    return (static_cast<unsigned long long>(key) << 32) | static_cast<uint32_t>(0xffffffffu - static_cast<uint32_t>(id));
+    return (static_cast<unsigned long long>(key) << 32) |
+           static_cast<uint32_t>(0xffffffffu - static_cast<uint32_t>(id));
 }
 
-// Select and sort for one query; `scores` holds n_vis valid entries.
-__device__ void topk_block(const float *__restrict__ scores, int n_vis, int select_k,
-                           int32_t *__restrict__ topk_out, int32_t *__restrict__ n_sel_out,
-                           TopkSmem &sm) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n_sel = min(select_k, n_vis);
-    int count;
-    if (n_vis <= select_k) {
-        for (int i = tid; i < n_vis; i += blockDim.x) sm.cand[i] = compose(score_key(scores[i]), i);
-        count = n_vis;
-    } else {
-        if (tid == 0) { sm.prefix = 0; sm.k_rem = select_k; }
-        uint32_t mask = 0;
-        for (int shift = 24; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += blockDim.x) sm.hist[i] = 0;
-            __syncthreads();
-            const uint32_t prefix = sm.prefix;
-            for (int base = 0; base < n_vis; base += blockDim.x) {
-                const int i = base + tid;
-                uint32_t digit = 0xffffffffu;
-                if (i < n_vis) {
-                    const uint32_t key = score_key(scores[i]);
-                    if ((key & mask) == prefix) digit = (key >> shift) & 0xffu;
-                }
-                const unsigned peers = __match_any_sync(0xffffffffu, digit);
-                if (digit != 0xffffffffu && lane == __ffs(peers) - 1) atomicAdd(&sm.hist[digit], __popc(peers));
-            }
-            __syncthreads();
-            if (warp == 0) {
-                // lane l owns digits [8l, 8l + 8); find the digit holding the k_rem-th largest
-                unsigned cnt[8], lane_sum = 0;
-#pragma unroll
-                for (int j = 0; j < 8; j++) { cnt[j] = sm.hist[8 * lane + j]; lane_sum += cnt[j]; }
-                unsigned suf = lane_sum;  // inclusive suffix sum over lanes >= lane
-#pragma unroll
-                for (int o = 1; o < 32; o <<= 1) {
-                    unsigned v = __shfl_down_sync(0xffffffffu, suf, o);
-                    if (lane + o < 32) suf += v;
-                }
-                unsigned above = suf - lane_sum;
-                const unsigned k = sm.k_rem;
-                if (above < k && k <= suf) {
-                    for (int j = 7; j >= 0; j--) {
-                        if (above + cnt[j] >= k) {
-                            sm.prefix = prefix | (static_cast<uint32_t>(8 * lane + j) << shift);
-                            sm.k_rem = k - above;
-                            break;
-                        }
-                        above += cnt[j];
-                    }
-                }
-            }
-            mask |= 0xffu << shift;
-            __syncthreads();
-        }
-        const uint32_t T = sm.prefix;
-        const unsigned need_eq = sm.k_rem;
-        const unsigned n_gt = static_cast<unsigned>(select_k) - need_eq;
-        if (tid == 0) { sm.n_gt = 0; sm.eq_base = 0; }
-        __syncthreads();
-        for (int base = 0; base < n_vis; base += blockDim.x) {
-            const int i = base + tid;
-            uint32_t key = 0;
-            if (i < n_vis) key = score_key(scores[i]);
-            const bool gt = i < n_vis && key > T;
-            const bool eq = i < n_vis && key == T;
-            const unsigned gt_mask = __ballot_sync(0xffffffffu, gt);
-            unsigned gpos = 0;
-            if (lane == 0 && gt_mask) gpos = atomicAdd(&sm.n_gt, __popc(gt_mask));
-            gpos = __shfl_sync(0xffffffffu, gpos, 0);
-            if (gt) sm.cand[gpos + __popc(gt_mask & ((1u << lane) - 1))] = compose(key, i);
-            const unsigned eq_mask = __ballot_sync(0xffffffffu, eq);
-            if (lane == 0) sm.warp_tot[warp] = __popc(eq_mask);
-            __syncthreads();
-            if (eq) {
-                unsigned off = sm.eq_base;
-                for (int w = 0; w < warp; w++) off += sm.warp_tot[w];
-                const unsigned rank = off + __popc(eq_mask & ((1u << lane) - 1));
-                if (rank < need_eq) sm.cand[n_gt + rank] = compose(key, i);
-            }
-            __syncthreads();
-            if (tid == 0) {
-                unsigned tot = 0;
-                for (int w = 0; w < (blockDim.x >> 5); w++) tot += sm.warp_tot[w];
-                sm.eq_base += tot;
-            }
-            __syncthreads();
-        }
-        count = select_k;
+__device__ __forceinline__ int nvis_of(const NvisSource &s, int n) {
+    if (s.n_visible) {
+        long long v = s.n_visible[n];
+        if (v < 0) v = 0;
+        if (v > s.ld) v = s.ld;
+        return static_cast<int>(v);
     }
-    // bitonic sort of cand[0, P2) descending; padding zeros sort last
+    const int b = s.q_seq[n];
+    if (b < 0 || b >= s.batch) return 0;
+    return visible_pools(s.pad[b], s.len[b], s.q_pos[n], s.ld);
+}
+
+// ------------------------------------------------------------------------------------------------
+// histogram of caller-supplied scores: grid (chunks of 8192 scores, n_q), 256 threads
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) topk_hist_kernel(const float *__restrict__ scores, NvisSource src,
+                                                        unsigned *__restrict__ ghist) {
+    __shared__ unsigned hist[kHistBins];
+    const int n = blockIdx.y;
+    const int n_vis = nvis_of(src, n);
+    const int64_t lo = static_cast<int64_t>(blockIdx.x) * 8192;
+    if (lo >= n_vis) return;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const float *row = scores + static_cast<int64_t>(n) * src.ld;
+#pragma unroll 4
+    for (int u = 0; u < 32; u++) {
+        const int64_t i = lo + u * 256 + threadIdx.x;
+        uint32_t d = 0xffffffffu;
+        if (i < n_vis) d = score_key(row[i]) >> (32 - kHistBitsTop);
+        hist_add(hist, d);
+    }
+    __syncthreads();
+    unsigned *g = ghist + static_cast<int64_t>(n) * kHistBins;
+    for (int i = threadIdx.x; i < kHistBins; i += blockDim.x)
+        if (hist[i]) atomicAdd(&g[i], hist[i]);
+}
+
+// ------------------------------------------------------------------------------------------------
+// select kernel
+// ------------------------------------------------------------------------------------------------
+struct SelSmem {
+    unsigned long long cand[kMaxSelect];   // list A, then the final select_k composites
+    unsigned long long bnd[kBoundCap];     // list B (keys of the boundary bin)
+    unsigned hist[256];
+    unsigned bin, above, n_a, n_b, done;
+    unsigned long long prefix;
+};
+
+// On warp 0: in a histogram of `nbins` bins (a multiple of 32), the highest bin whose suffix count
+// (that bin and all higher ones) reaches k; writes the bin, the count in higher bins and the
+// bin's own count.
+__device__ void find_bin_warp(const unsigned *hist, int nbins, unsigned k, unsigned *bin,
+                              unsigned *above_out, unsigned *count_out) {
+    const int lane = threadIdx.x & 31;
+    const int per = nbins / 32;
+    unsigned lane_sum = 0;
+    for (int j = 0; j < per; j++) lane_sum += hist[per * lane + j];
+    unsigned suf = lane_sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned v = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += v;
+    }
+    unsigned above = suf - lane_sum;
+    if (above < k && k <= suf) {
+        for (int j = per - 1; j >= 0; j--) {
+            const unsigned c = hist[per * lane + j];
+            if (above + c >= k) {
+                *bin = static_cast<unsigned>(per * lane + j);
+                *above_out = above;
+                if (count_out) *count_out = c;
+                break;
+            }
+            above += c;
+        }
+    }
+}
+
+// Radix select of the k largest composites among the entries that share `prefix` on the bits of
+// `mask` (known_bits leading bits). The entries come from `get(i)`, i < m. On return
+// sm.prefix / sm.done describe the boundary: the selection is every entry e with
+// (e & ~0 << (64 - done)) >= prefix, which holds exactly k entries.
+template <typename Get>
+__device__ void radix_select(Get get, int m, unsigned k, int known_bits, unsigned long long prefix,
+                             SelSmem &sm) {
+    const int tid = threadIdx.x;
+    unsigned long long mask = ~0ull << (64 - known_bits);
+    int bits = known_bits;
+    while (bits < 64) {
+        const int width = min(8, 64 - bits);
+        const int shift = 64 - bits - width;
+        for (int i = tid; i < 256; i += blockDim.x) sm.hist[i] = 0;
+        if (tid == 0) { sm.bin = 0; sm.above = 0; sm.n_b = 0; }
+        __syncthreads();
+        for (int base = 0; base < m; base += blockDim.x) {
+            const int i = base + tid;
+            uint32_t d = 0xffffffffu;
+            if (i < m) {
+                unsigned long long c;
+                if (get(i, c) && (c & mask) == prefix) d = static_cast<uint32_t>((c >> shift) & ((1u << width) - 1));
+            }
+            hist_add(sm.hist, d);
+        }
+        __syncthreads();
+        if (tid < 32) find_bin_warp(sm.hist, 256, k, &sm.bin, &sm.above, &sm.n_b);
+        __syncthreads();
+        const unsigned d = sm.bin, above = sm.above, in_bin = sm.n_b;
+        prefix |= static_cast<unsigned long long>(d) << shift;
+        mask |= static_cast<unsigned long long>((1u << width) - 1) << shift;
+        bits += width;
+        k -= above;
+        __syncthreads();
+        if (k == in_bin) break;  // the whole digit is taken: resolved
+    }
+    if (tid == 0) { sm.prefix = prefix; sm.done = static_cast<unsigned>(bits); }
+    __syncthreads();
+}
+
+__device__ void bitonic_desc(unsigned long long *a, int count) {
     int P2 = 1;
     while (P2 < count) P2 <<= 1;
-    for (int i = count + tid; i < P2; i += blockDim.x) sm.cand[i] = 0ull;
+    for (int i = count + threadIdx.x; i < P2; i += blockDim.x) a[i] = 0ull;
     __syncthreads();
     for (int k = 2; k <= P2; k <<= 1) {
         for (int j = k >> 1; j > 0; j >>= 1) {
-            for (int i = tid; i < P2; i += blockDim.x) {
+            for (int i = threadIdx.x; i < P2; i += blockDim.x) {
                 const int ixj = i ^ j;
                 if (ixj > i) {
-                    const unsigned long long a = sm.cand[i], b = sm.cand[ixj];
+                    const unsigned long long x = a[i], y = a[ixj];
                     const bool desc = (i & k) == 0;
-                    if (desc ? (a < b) : (a > b)) { sm.cand[i] = b; sm.cand[ixj] = a; }
+                    if (desc ? (x < y) : (x > y)) { a[i] = y; a[ixj] = x; }
                 }
             }
             __syncthreads();
         }
     }
+}
+
+// Append every entry with get(i) valid and (c & msk) >= pre to sm.cand[base + ...].
+template <typename Get>
+__device__ void collect_from(Get get, int m, unsigned long long msk, unsigned long long pre,
+                             unsigned base, SelSmem &sm) {
+    const int lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) sm.n_b = 0;
+    __syncthreads();
+    for (int b0 = 0; b0 < m; b0 += blockDim.x) {
+        const int i = b0 + threadIdx.x;
+        unsigned long long c = 0;
+        const bool take = i < m && get(i, c) && (c & msk) >= pre;
+        const unsigned tm = __ballot_sync(0xffffffffu, take);
+        unsigned p = 0;
+        if (lane == 0 && tm) p = atomicAdd(&sm.n_b, __popc(tm));
+        p = __shfl_sync(0xffffffffu, p, 0);
+        const unsigned pos = base + p + __popc(tm & ((1u << lane) - 1));
+        if (take && pos < static_cast<unsigned>(kMaxSelect)) sm.cand[pos] = c;
+    }
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
+    const float *__restrict__ scores, NvisSource src, const unsigned *__restrict__ ghist,
+    int select_k, int32_t *__restrict__ topk, int32_t *__restrict__ n_sel_out) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    SelSmem &sm = *reinterpret_cast<SelSmem *>(smem_raw);
+    const int n = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
+    const int n_vis = nvis_of(src, n);
+    const float *row = scores + static_cast<int64_t>(n) * src.ld;
+    int32_t *out = topk + static_cast<int64_t>(n) * select_k;
+    const int n_sel = min(select_k, n_vis);
+    int count;
+    if (n_vis <= select_k) {
+        for (int i = tid; i < n_vis; i += blockDim.x) sm.cand[i] = compose(score_key(row[i]), i);
+        count = n_vis;
+        __syncthreads();
+    } else {
+        // (a) the boundary bin from the 2048-bin histogram (defaults keep every write in bounds
+        // should the histogram not match the scores)
+        if (tid == 0) { sm.bin = 0; sm.above = 0; sm.n_b = 0xffffffffu; }
+        __syncthreads();
+        if (tid < 32) find_bin_warp(ghist + static_cast<int64_t>(n) * kHistBins, kHistBins,
+                                    static_cast<unsigned>(select_k), &sm.bin, &sm.above, &sm.n_b);
+        if (tid == 0) sm.n_a = 0;
+        __syncthreads();
+        const unsigned bstar = sm.bin, n_above = sm.above, m_b = sm.n_b;
+        const bool fits = m_b <= static_cast<unsigned>(kBoundCap);
+        __syncthreads();
+        if (tid == 0) sm.n_b = 0;
+        __syncthreads();
+        // (b) one pass: A = keys of higher bins, B = keys of the boundary bin
+        for (int base = 0; base < n_vis; base += blockDim.x * 4) {
+            uint32_t key[4];
+            int idx[4];
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                idx[u] = base + u * blockDim.x + tid;
+                key[u] = idx[u] < n_vis ? score_key(row[idx[u]]) : 0u;
+            }
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const bool ok = idx[u] < n_vis;
+                const unsigned d = key[u] >> (32 - kHistBitsTop);
+                const bool a = ok && d > bstar;
+                const bool bb = ok && fits && d == bstar;
+                const unsigned am = __ballot_sync(0xffffffffu, a);
+                const unsigned bm = __ballot_sync(0xffffffffu, bb);
+                unsigned pa = 0, pb = 0;
+                if (lane == 0) {
+                    if (am) pa = atomicAdd(&sm.n_a, __popc(am));
+                    if (bm) pb = atomicAdd(&sm.n_b, __popc(bm));
+                }
+                pa = __shfl_sync(0xffffffffu, pa, 0);
+                pb = __shfl_sync(0xffffffffu, pb, 0);
+                const unsigned lt = (1u << lane) - 1;
+                const unsigned ra = pa + __popc(am & lt), rb = pb + __popc(bm & lt);
+                if (a && ra < static_cast<unsigned>(kMaxSelect)) sm.cand[ra] = compose(key[u], idx[u]);
+                if (bb && rb < static_cast<unsigned>(kBoundCap)) sm.bnd[rb] = compose(key[u], idx[u]);
+            }
+        }
+        __syncthreads();
+        // (c) the remaining select_k - n_above keys from the boundary bin
+        const unsigned need = static_cast<unsigned>(select_k) - min(n_above, static_cast<unsigned>(select_k));
+        const unsigned long long top = static_cast<unsigned long long>(bstar) << (64 - kHistBitsTop);
+        if (fits) {
+            const int m = static_cast<int>(min(sm.n_b, static_cast<unsigned>(kBoundCap)));
+            auto get = [&](int i, unsigned long long &c) { c = sm.bnd[i]; return true; };
+            if (static_cast<unsigned>(m) == need) {
+                for (int i = tid; i < m; i += blockDim.x)
+                    if (n_above + i < static_cast<unsigned>(kMaxSelect)) sm.cand[n_above + i] = sm.bnd[i];
+                __syncthreads();
+            } else {
+                radix_select(get, m, need, kHistBitsTop, top, sm);
+                collect_from(get, m, ~0ull << (64 - sm.done), sm.prefix, n_above, sm);
+            }
+        } else {
+            auto get = [&](int i, unsigned long long &c) {
+                const uint32_t key = score_key(row[i]);
+                c = compose(key, i);
+                return (key >> (32 - kHistBitsTop)) == bstar;
+            };
+            radix_select(get, n_vis, need, kHistBitsTop, top, sm);
+            collect_from(get, n_vis, ~0ull << (64 - sm.done), sm.prefix, n_above, sm);
+        }
+        count = select_k;
+    }
+    // (d) order
+    bitonic_desc(sm.cand, count);
     for (int i = tid; i < select_k; i += blockDim.x)
-        topk_out[i] = i < n_sel ? static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(sm.cand[i] & 0xffffffffu)) : GLM_INVALID;
-    if (tid == 0 && n_sel_out) *n_sel_out = n_sel;
+        out[i] = i < n_sel ? static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(sm.cand[i] & 0xffffffffu))
+                           : GLM_INVALID;
+    if (tid == 0 && n_sel_out) n_sel_out[n] = n_sel;
 }
 
-// Selection for the fused entry: n_vis from the query's sequence geometry.
-__global__ void __launch_bounds__(kTopkThreads) topk_fused_kernel(
-    const float *__restrict__ scores, int64_t ld_scores, const int32_t *__restrict__ q_seq,
-    const int32_t *__restrict__ q_pos, const int32_t *__restrict__ pad,
-    const int32_t *__restrict__ len, int batch, int select_k, int32_t *__restrict__ topk,
-    int32_t *__restrict__ n_sel) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
-    const int n = blockIdx.x;
-    const int b = q_seq[n];
-    const int n_vis = (b >= 0 && b < batch) ? visible_pools(pad[b], len[b], q_pos[n], ld_scores) : 0;
-    topk_block(scores + static_cast<int64_t>(n) * ld_scores, n_vis, select_k,
-               topk + static_cast<int64_t>(n) * select_k, n_sel ? n_sel + n : nullptr, sm);
-}
+size_t topk_select_smem() { return sizeof(SelSmem); }
 
-// Selection on caller-supplied scores: n_vis given per query.
-__global__ void __launch_bounds__(kTopkThreads) topk_given_kernel(
-    const float *__restrict__ scores, int64_t ld_scores, const int32_t *__restrict__ n_visible,
-    int select_k, int32_t *__restrict__ topk, int32_t *__restrict__ n_sel) {
-    extern __shared__ __align__(16) unsigned char smem_raw[];
-    TopkSmem &sm = *reinterpret_cast<TopkSmem *>(smem_raw);
-    const int n = blockIdx.x;
-    long long nv = n_visible[n];
-    if (nv < 0) nv = 0;
-    if (nv > ld_scores) nv = ld_scores;
-    const int n_vis = static_cast<int>(nv);
-    topk_block(scores + static_cast<int64_t>(n) * ld_scores, n_vis, select_k,
-               topk + static_cast<int64_t>(n) * select_k, n_sel ? n_sel + n : nullptr, sm);
-}
-
-cudaError_t launch_topk_fused(const float *scores, int64_t ld_scores, const int32_t *q_seq,
-                              const int32_t *q_pos, const int32_t *pad, const int32_t *len,
-                              int batch, int n_q, int select_k, int32_t *topk, int32_t *n_sel,
-                              cudaStream_t stream) {
-    const size_t smem = sizeof(TopkSmem);
-    cudaError_t e = cudaFuncSetAttribute(topk_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    topk_fused_kernel<<<n_q, kTopkThreads, smem, stream>>>(scores, ld_scores, q_seq, q_pos, pad,
-                                                           len, batch, select_k, topk, n_sel);
+cudaError_t launch_topk_hist(const float *scores, const NvisSource &src, int n_q, unsigned *ghist,
+                             cudaStream_t stream) {
+    dim3 grid(static_cast<unsigned>((src.ld + 8191) / 8192), n_q);
+    if (grid.x == 0 || n_q == 0) return cudaSuccess;
+    topk_hist_kernel<<<grid, 256, 0, stream>>>(scores, src, ghist);
     return cudaGetLastError();
 }
 
-cudaError_t launch_topk_given(const float *scores, int64_t ld_scores, const int32_t *n_visible,
-                              int n_q, int select_k, int32_t *topk, int32_t *n_sel,
-                              cudaStream_t stream) {
-    const size_t smem = sizeof(TopkSmem);
-    cudaError_t e = cudaFuncSetAttribute(topk_given_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+cudaError_t launch_topk_select(const float *scores, const NvisSource &src, const unsigned *ghist,
+                               int n_q, int select_k, int32_t *topk, int32_t *n_sel,
+                               cudaStream_t stream) {
+    const size_t smem = sizeof(SelSmem);
+    cudaError_t e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    topk_given_kernel<<<n_q, kTopkThreads, smem, stream>>>(scores, ld_scores, n_visible, select_k,
-                                                           topk, n_sel);
+    topk_select_kernel<<<n_q, kSelThreads, smem, stream>>>(scores, src, ghist, select_k, topk, n_sel);
     return cudaGetLastError();
 }
 

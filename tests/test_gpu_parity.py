@@ -6,8 +6,10 @@ Agreement rules
     fp32 values); in the chained path the GPU selection may differ from the oracle's only among
     pools whose oracle score lies within 1e-4 (relative) of the select_k-th score.
   * index scores: max over (n, p) of |g - o| / max(|o|, 1e-3 * max_p |o[n, p]|) <= 1e-4.
-  * attention output: max abs err <= 1e-2 and relative L2 error <= 5e-3 against the oracle on the
-    same int8 rows; lse within 1e-3 absolute.
+  * attention output: the fp32 output within max abs err <= 1e-2 and relative L2 error <= 5e-3
+    of the oracle on the same int8 rows; the bf16 output equal to the fp32 output rounded to
+    nearest-even bf16 (bit-exact: a bf16 value near 16 alone carries a 0.0625 rounding step, so
+    the absolute bound is stated on the fp32 result); lse within 1e-3 absolute.
   * pooled keys (fp32 kernel, fp64 oracle): |g - o| <= 2e-5 * (1 + |o|). Derivation: the LayerNorm
     sums 128 fp32 terms (relative error <= ~128 * 2**-24 = 7.6e-6 of the largest term, typically
     ~1e-6), the slot softmax adds a few ulps, so 2e-5 leaves a margin of ~3x over the worst case.
@@ -57,6 +59,11 @@ def attn_errors(g, o):
 def assert_attention_close(g, o, what=""):
     max_abs, rel_l2 = attn_errors(g, o)
     assert max_abs <= 1e-2 and rel_l2 <= 5e-3, (what, max_abs, rel_l2)
+
+
+def assert_bf16_is_rounded_f32(out_bf16_bits, out_f32):
+    assert np.array_equal(np.asarray(out_bf16_bits, np.uint16),
+                          synth.f32_to_bf16_bits(np.asarray(out_f32, np.float32)))
 
 
 # ------------------------------------------------------------------------------------------------
@@ -228,22 +235,44 @@ def test_index_topk_fused_selection(cuda):
     for n, so in enumerate(_oracle_scores_on(inp, p32)):
         want, n_sel = oracle.topk_pools(so, inp.wl.select_k)
         assert ng[n] == n_sel
-        _selection_agrees(tg[n], want, so, n_sel)
+        assert _selection_agrees(tg[n], want, so, n_sel) == 0
 
 
 def _selection_agrees(got, want, scores, n_sel):
-    """Equal, except that pools whose score is within 1e-4 (relative) of the select_k-th score
-    may be exchanged among themselves."""
+    """The GPU selection against the oracle's (scores = the oracle's fp64 scores). Equal as sets,
+    except that pools whose score is within 1e-4 (relative) of the select_k-th score may be
+    exchanged; and in an order that is non-increasing in oracle score up to that tolerance (pools
+    closer than the fp32 rounding of their scores may come in either order). Returns the number
+    of exchanged pools."""
     assert (got[n_sel:] == -1).all()
-    if np.array_equal(got, want) or n_sel == 0:
+    if n_sel == 0:
         return 0
     thr = scores[want[n_sel - 1]]
     tol = 1e-4 * max(abs(thr), 1e-30)
-    gs, ws = set(got[:n_sel].tolist()), set(want[:n_sel].tolist())
+    g = got[:n_sel]
+    assert (g >= 0).all() and (g < len(scores)).all() and len(set(g.tolist())) == n_sel
+    gs, ws = set(g.tolist()), set(want[:n_sel].tolist())
     for p in gs ^ ws:
         assert abs(scores[p] - thr) <= tol, (p, scores[p], thr)
-    assert len(gs) == n_sel
+    sg = scores[g]
+    suffix_max = np.maximum.accumulate(sg[::-1])[::-1]
+    band = 1e-4 * np.maximum(np.abs(sg), 1e-30)
+    assert (sg[:-1] >= suffix_max[1:] - band[:-1]).all(), "order not descending within tolerance"
     return len(gs ^ ws) // 2
+
+
+def _expanded_is_valid(tok, rows, topk, n_sel, want_tok, inp, n):
+    """Expanded tokens of a selection that matches the oracle's as a set: every 4-token block is
+    the pool of the same position of the GPU's own top-k list, ascending; the tail and the -1
+    padding equal the oracle's exactly; rows are the slot map of the tokens."""
+    s = int(inp.q_seq[n])
+    pad = int(inp.pad[s])
+    for i in range(n_sel):
+        assert list(tok[4 * i:4 * i + 4]) == [pad + 4 * int(topk[i]) + j for j in range(4)]
+    assert np.array_equal(tok[4 * n_sel:], want_tok[4 * n_sel:])
+    assert sorted(tok[:4 * n_sel].tolist()) == sorted(want_tok[:4 * n_sel].tolist())
+    sm = inp.slot_map[s]
+    assert np.array_equal(rows, np.where(tok >= 0, sm[np.maximum(tok, 0)], -1))
 
 
 # ------------------------------------------------------------------------------------------------
@@ -302,7 +331,7 @@ def _mla_case(cuda, n_heads, rows, cache, q, sm):
     lse = torch.full((nq, n_heads), 7.0, dtype=torch.float32, device=cuda)
     kp.glm_sparse_mla_decode(dims, to_dev(q, torch.bfloat16, cuda), torch.from_numpy(cache).to(cuda),
                              to_dev(rows, torch.int32, cuda), sm, out, ws, lse=lse, out_f32=o32)
-    return np_(out.float()), np_(o32), np_(lse)
+    return np_(out.view(torch.int16)).view(np.uint16), np_(o32), np_(lse)
 
 
 @pytest.mark.parametrize("n_heads,W,n_valid,n_rows", [(16, 80, 64, 512), (64, 2176, 2048, 5000),
@@ -327,9 +356,9 @@ def test_sparse_mla_matches_oracle(cuda, n_heads, W, n_valid, n_rows):
     for n in range(nq):
         oo, lo = oracle.sparse_mla(q[n], cache, rows[n], sm)
         assert_attention_close(o32[n], oo, "f32")
-        assert_attention_close(og[n], oo, "bf16")
+        assert_bf16_is_rounded_f32(og[n], o32[n])
         if n_valid == 0:
-            assert np.isneginf(lg[n]).all() and not o32[n].any() and not og[n].any()
+            assert np.isneginf(lg[n]).all() and not o32[n].any() and not (og[n] & 0x7fff).any()
         else:
             np.testing.assert_allclose(lg[n], lo, atol=1e-3, rtol=0)
 
@@ -387,9 +416,12 @@ def _check_chain(inp, b, queries=None, check_cache_rows=None):
         assert ng[n] == r["n_sel"]
         d = _selection_agrees(tg[n], r["topk"], r["scores"], r["n_sel"])
         if d == 0:
-            assert np.array_equal(tokg[n], r["tok"]) and np.array_equal(rowg[n], r["rows"])
+            if np.array_equal(tg[n], r["topk"]):
+                assert np.array_equal(tokg[n], r["tok"]) and np.array_equal(rowg[n], r["rows"])
+            else:
+                _expanded_is_valid(tokg[n], rowg[n], tg[n], r["n_sel"], r["tok"], inp, n)
             assert_attention_close(o32[n], r["out"], f"query {n}")
-            assert_attention_close(np_(b.out[n].float()), r["out"], f"query {n} bf16")
+            assert_bf16_is_rounded_f32(np_(b.out[n].view(torch.int16)).view(np.uint16), o32[n])
         else:
             diffs += 1
             # same selection as a set of pools up to the tie band: the tokens are still all valid
