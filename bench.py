@@ -218,6 +218,31 @@ def run_reference(args, wl):
 METRIC = "decode queries/s and achieved HBM GB/s (% of B200 peak), indexer+sparse MLA"
 
 
+# ------------------------------------------------------------------------------------------------
+# multi-rank plumbing (replicas only: no data-path collective)
+# ------------------------------------------------------------------------------------------------
+
+def replica_state_ids(rank: int, n_states: int) -> list:
+    """Workload state ids of one rank: disjoint across ranks, so replicas never share inputs."""
+    return [rank * n_states + r for r in range(n_states)]
+
+
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks of a per-rank time (the slowest replica bounds the whole job)."""
+    if world <= 1:
+        return float(value)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_throughput(units_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Units processed by all ranks divided by the max-over-ranks time (weak scaling)."""
+    return units_per_rank_step * steps * world / (max_ms / 1e3)
+
+
 def config_of(wl, args):
     return {"workload": wl.name, "batch": wl.batch, "context": list(wl.lens) if wl.batch > 1 else wl.lens[0],
             "queries_per_step": wl.n_queries, "n_heads": wl.n_heads, "select_k": wl.select_k,
@@ -252,8 +277,8 @@ def run_kernels(args, wl):
 
     R = args.states
     inps, bufs = [], []
-    for r in range(R):
-        inp = synth.generate(wl, state=rank * R + r)
+    for r, sid in enumerate(replica_state_ids(rank, R)):
+        inp = synth.generate(wl, state=sid)
         b = sdev.allocate_for(inp, dev)
         sdev.load(inp, b)
         bufs.append(b)
@@ -301,14 +326,9 @@ def run_kernels(args, wl):
     torch.cuda.synchronize()
     sampler.stop()
     barrier()
-    ms = e0.elapsed_time(e1)
-    if world > 1:
-        t = torch.tensor([ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = reduce_max(e0.elapsed_time(e1), world, dev)
     ms_per_step = ms / args.steps
-    queries = wl.n_queries * args.steps * world
-    value = queries / (ms / 1e3)
+    value = whole_job_throughput(wl.n_queries, args.steps, world, ms)
 
     # per-stage device time (same kernels, same buffers, direct launches queued behind a sleep so
     # the host never starves the GPU; events on the launching stream). "index_scores" is the
@@ -378,11 +398,7 @@ def run_kernels(args, wl):
             h_out.copy_(b.out, non_blocking=True)
             stream.synchronize()
         e2e_s = time.perf_counter() - t0
-    e2e_qps = wl.n_queries * n_e2e / e2e_s
-    if world > 1:
-        t = torch.tensor([e2e_s], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_qps = wl.n_queries * n_e2e * world / float(t.item())
+    e2e_qps = whole_job_throughput(wl.n_queries, n_e2e, world, reduce_max(e2e_s * 1e3, world, dev))
 
     peak, peak_kind = measured_peaks()
     idx_ms = stage_ms["index_scores"]

@@ -136,9 +136,12 @@ int glm_kpool_build(const glm_dsa_dims *dims, const void *k_dev, const void *gat
  *   scores_dev  fp32 [n_q, ld_pools] or NULL: receives the scores (entries p >= n_vis are -inf)
  *   topk_dev    int32 [n_q, select_k]      n_sel_dev  int32 [n_q] or NULL
  *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, ...), 256-byte
- *               aligned (required even when scores_dev is given; contents on entry are ignored)
- * 1 <= select_k <= 2048. Scores are fp32 sums of fp32 products of the bf16 queries and the fp32
- * pooled keys.
+ *               aligned (required even when scores_dev is given; contents on entry are ignored).
+ *               Its last 256 bytes start with a status word set nonzero if a wait on the tensor
+ *               cores gave up (never cleared by the library).
+ * 1 <= select_k <= 2048. The q . pooled products run on the tensor cores: each fp32 pooled key is
+ * split exactly into three bf16 terms, so with the bf16 queries exact the dot products carry fp32
+ * accumulation error only (relative error far below 1e-4); relu and the head weights in fp32.
  */
 int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx_dev, const float *w_dev,
                           const float *pooled_dev, int64_t ld_pools, const int32_t *q_seq_dev,
@@ -208,8 +211,12 @@ int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk_dev,
  *   q_dev      bf16 [n_q, n_heads, 512]       cache_dev int8 [n_rows, 528]
  *   rows_dev   int32 [n_q, width]             out_dev   bf16 [n_q, n_heads, 512]
  *   lse_dev    fp32 [n_q, n_heads] or NULL    out_f32_dev fp32 [n_q, n_heads, 512] or NULL
- *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width)
- * 1 <= width <= 65536.
+ *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width),
+ *               256-byte aligned. Its last 256 bytes start with a status word that the kernels set
+ *               nonzero if a wait on the tensor cores gave up (the outputs are then invalid); it is
+ *               never cleared by the library, so a caller that checks it zeroes it first.
+ * 1 <= width <= 65536. The contractions run on the tensor cores (bf16 operands: the int8 codes and
+ * the bf16 queries exactly; the softmax weights as a two-term bf16 split), accumulating in fp32.
  */
 int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q_dev, const int8_t *cache_dev,
                           int64_t n_rows, const int32_t *rows_dev, int32_t n_q, int32_t width,

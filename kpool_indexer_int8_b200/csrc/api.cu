@@ -29,11 +29,16 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 size_t hist_bytes(int n_q) { return align_up(static_cast<size_t>(n_q) * glm::kHistBins * sizeof(unsigned), 256); }
 
 // Workspace of the sparse MLA: partial accumulators and (m, l) pairs per (query, chunk, head),
-// sized for the smallest chunk any implementation uses.
-size_t mla_workspace(int n_q, int n_heads, int width, int chunk) {
-    const size_t n_chunks = static_cast<size_t>((width + chunk - 1) / chunk);
-    const size_t parts = static_cast<size_t>(n_q) * n_chunks * n_heads;
-    return align_up(parts * glm::kLatent * sizeof(float), 256) + align_up(parts * 2 * sizeof(float), 256);
+// then a 256-byte tail whose first word is the kernels' status (nonzero after a timed-out wait).
+size_t mla_parts(int n_q, int n_heads, int width) {
+    const int chunk = glm::mla_tc_chunk();
+    return static_cast<size_t>(n_q) * static_cast<size_t>((width + chunk - 1) / chunk) * n_heads;
+}
+size_t mla_acc_bytes(size_t parts) { return align_up(parts * glm::kLatent * sizeof(float), 256); }
+size_t mla_ml_bytes(size_t parts) { return align_up(parts * 2 * sizeof(float), 256); }
+size_t mla_workspace(int n_q, int n_heads, int width) {
+    const size_t parts = mla_parts(n_q, n_heads, width);
+    return mla_acc_bytes(parts) + mla_ml_bytes(parts) + 256;
 }
 
 }  // namespace
@@ -103,13 +108,13 @@ size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
     switch (op) {
         case GLM_OP_INDEX_SCORES_TOPK:
             if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
-            return hist_bytes(n_q) + align_up(static_cast<size_t>(n_q) * static_cast<size_t>(max_pools) * sizeof(float), 256);
+            return hist_bytes(n_q) + align_up(static_cast<size_t>(n_q) * static_cast<size_t>(max_pools) * sizeof(float), 256) + 256;
         case GLM_OP_TOPK_POOLS:
             if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
             return hist_bytes(n_q);
         case GLM_OP_SPARSE_MLA:
             if (width < 1 || width > 65536) return static_cast<size_t>(-1);
-            return mla_workspace(n_q, dims->n_heads, width, glm::mla_simt_chunk());
+            return mla_workspace(n_q, dims->n_heads, width);
         default:
             return static_cast<size_t>(-1);
     }
@@ -136,14 +141,17 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const flo
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, n_q, ld_pools, select_k, 0);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
     unsigned *ghist = static_cast<unsigned *>(workspace);
-    float *sbuf = scores ? scores : reinterpret_cast<float *>(static_cast<char *>(workspace) + hist_bytes(n_q));
+    char *ws = static_cast<char *>(workspace);
+    float *sbuf = scores ? scores : reinterpret_cast<float *>(ws + hist_bytes(n_q));
+    int *status = reinterpret_cast<int *>(ws + need - 256);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const glm::NvisSource src{nullptr, q_seq, q_pos, pad, len, batch, ld_pools};
     if (ld_pools > 0) {
         rc = cuda_status(cudaMemsetAsync(ghist, 0, static_cast<size_t>(n_q) * glm::kHistBins * sizeof(unsigned), st));
         if (rc != GLM_OK) return rc;
-        rc = cuda_status(glm::launch_index_scores_simt(q_idx, w, pooled, ld_pools, q_seq, q_pos,
-                                                       pad, len, batch, n_q, sbuf, ghist, st));
+        rc = cuda_status(glm::launch_index_scores_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len,
+                                                     batch, n_q, sbuf, ghist, scores != nullptr, status,
+                                                     num_sms(), st));
         if (rc != GLM_OK) return rc;
     }
     return cuda_status(glm::launch_topk_select(sbuf, src, ghist, n_q, select_k, topk, n_sel, st));
@@ -163,9 +171,9 @@ int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w
     if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(pooled, 16) || !aligned(q_seq, 4) ||
         !aligned(q_pos, 4) || !aligned(pad, 4) || !aligned(len, 4) || !aligned(scores, 4))
         return GLM_ERR_INVALID_ARG;
-    return cuda_status(glm::launch_index_scores_simt(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad,
-                                                     len, batch, n_q, scores, nullptr,
-                                                     static_cast<cudaStream_t>(stream)));
+    return cuda_status(glm::launch_index_scores_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len,
+                                                   batch, n_q, scores, nullptr, true, nullptr, num_sms(),
+                                                   static_cast<cudaStream_t>(stream)));
 }
 
 int glm_topk_pools(const float *scores, int64_t ld_scores, const int32_t *n_visible, int32_t n_q,
@@ -229,15 +237,16 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t 
     const int H = dims->n_heads;
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
-    const int chunk = glm::mla_simt_chunk();
+    const int chunk = glm::mla_tc_chunk();
     const int n_chunks = (width + chunk - 1) / chunk;
-    const size_t parts = static_cast<size_t>(n_q) * n_chunks * H;
-    float *part_acc = static_cast<float *>(workspace);
-    float *part_ml = reinterpret_cast<float *>(static_cast<char *>(workspace) +
-                                               align_up(parts * glm::kLatent * sizeof(float), 256));
+    const size_t parts = mla_parts(n_q, H, width);
+    char *ws = static_cast<char *>(workspace);
+    float *part_acc = reinterpret_cast<float *>(ws);
+    float *part_ml = reinterpret_cast<float *>(ws + mla_acc_bytes(parts));
+    int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = cuda_status(glm::launch_mla_split_simt(q, H, cache, n_rows, rows, n_q, width, sm_scale,
-                                                part_acc, part_ml, st));
+    rc = cuda_status(glm::launch_mla_split_tc(q, H, cache, n_rows, rows, n_q, width, sm_scale,
+                                              part_acc, part_ml, status, st));
     if (rc != GLM_OK) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32, lse, st));
 }

@@ -16,10 +16,11 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
                                const int32_t *pad, const int32_t *len, const int32_t *pool_begin,
                                int batch, int max_new_pools, float *pooled, int64_t ld_pools,
                                int32_t *n_pools, cudaStream_t stream, int num_sms);
-cudaError_t launch_index_scores_simt(const void *q_idx, const float *w, const float *pooled,
-                                     int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
-                                     const int32_t *pad, const int32_t *len, int batch, int n_q,
-                                     float *scores, unsigned *ghist, cudaStream_t stream);
+cudaError_t launch_index_scores_tc(const void *q_idx, const float *w, const float *pooled,
+                                   int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
+                                   const int32_t *pad, const int32_t *len, int batch, int n_q,
+                                   float *scores, unsigned *ghist, bool fill_invisible, int *status,
+                                   int num_sms, cudaStream_t stream);
 cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32_t *q_seq,
                           const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
                           int n_q, int select_k, const int64_t *slot_map, int64_t ld_slot, int out_width,

@@ -9,11 +9,10 @@ namespace glm {
 // Partial softmax state of one (query, chunk, head): m (running max of the chunk's scores),
 // l (sum of exp(s - m)), acc[512] (sum of exp(s - m) * c). Layout in the workspace:
 //   part_acc fp32 [n_q][n_chunks][n_heads][512], part_ml fp32 [n_q][n_chunks][n_heads][2].
-size_t mla_simt_smem_bytes(int n_heads);
-int mla_simt_chunk();
-cudaError_t launch_mla_split_simt(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
-                                  const int32_t *rows, int n_q, int width, float sm_scale,
-                                  float *part_acc, float *part_ml, cudaStream_t stream);
+int mla_tc_chunk();
+cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
+                                const int32_t *rows, int n_q, int width, float sm_scale,
+                                float *part_acc, float *part_ml, int *status, cudaStream_t stream);
 cudaError_t launch_mla_combine(const float *part_acc, const float *part_ml, int n_q, int n_heads,
                                int n_chunks, void *out, float *out_f32, float *lse,
                                cudaStream_t stream);

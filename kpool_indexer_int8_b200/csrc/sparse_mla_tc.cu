@@ -1,0 +1,276 @@
+// sparse_mla_tc.cu -- sparse NoPE MLA over gathered int8 latent rows on the sm_100a tensor cores
+// ("GLM-5.3 Kernels" README, 'Included': titan_mla.triton_mla_sparse_attention -- int8
+// dequantisation fused in, the shared 512-d latent is both K and V, split-KV decode, fp32
+// softmax and accumulation; 'The tested MLA contract': one KV head, negative index padding).
+//
+// One CTA per (query, chunk of 64 index entries); heads are the MMA M dimension (M = 64 for up
+// to 64 heads, 128 above; missing heads are zero rows):
+//   1. gather: each entry's 512 int8 codes are widened to bf16 (exact: |code| <= 127) into a
+//      shared tile C[64 rows x 512] stored as 8x8 core matrices, its fp32 scale to a register
+//      file in shared memory; the query block Q[heads x 512] goes to shared memory the same way.
+//   2. S = Q . C^T on tcgen05 (kind::f16, fp32 accumulator in tensor memory, 32 MMAs of K = 16).
+//      C is the K-major B operand here.
+//   3. softmax of the chunk, one TMEM lane (= one head) per thread: s = S * scale_j * sm_scale,
+//      m = max, p = exp(s - m), l = sum p; P' = p * scale_j (the V dequantisation scale folded
+//      in) is split into bf16 hi + lo so that the PV product keeps ~16 mantissa bits of P'.
+//   4. O = P'.C over 512 columns of tensor memory (16 MMAs of N = 256, K = 16). The same tile C
+//      is now the MN-major B operand: a core matrix of 8 rows x 8 dims serves both products.
+//   5. (m, l) and the unnormalised O of every head go to the workspace; the combine kernel merges
+//      the chunks by log-sum-exp.
+// Tensor memory: 512 columns (S in columns 0..63, then O over all 512 once S has been read).
+// Every wait on the tensor cores is bounded; a timeout sets a status word and the CTA still
+// frees its tensor memory and exits.
+#include "common.cuh"
+#include "sparse_mla.cuh"
+#include "tc.cuh"
+
+namespace glm {
+
+constexpr int kTcRows = 64;
+constexpr int kTcThreads = 256;
+constexpr uint32_t kWaitLimit = 1u << 22;
+
+template <int M>
+struct TcLayout {
+    static constexpr int kQ = 0;                     // M/8 head groups x 64 dim groups x 128 B
+    static constexpr int kC = kQ + M * 1024;         // 8 row groups x 64 dim groups x 128 B
+    static constexpr int kPhi = kC + 64 * 1024;      // M/8 head groups x 8 row groups x 128 B
+    static constexpr int kPlo = kPhi + M * 128;
+    static constexpr int kScl = kPlo + M * 128;      // 64 fp32 scales
+    static constexpr int kRow = kScl + 256;          // 64 row indices
+    static constexpr int kBar = kRow + 256;          // 2 mbarriers
+    static constexpr int kTmem = kBar + 16;          // tensor-memory base address
+    static constexpr int kFlag = kTmem + 16;
+    static constexpr int kBytes = kFlag + 16;
+};
+
+__device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w, int shift) {
+    const float a = static_cast<float>(static_cast<int8_t>((w >> shift) & 0xffu));
+    const float b = static_cast<float>(static_cast<int8_t>((w >> (shift + 8)) & 0xffu));
+    return (__float_as_uint(a) >> 16) | (__float_as_uint(b) & 0xffff0000u);
+}
+
+__device__ __forceinline__ uint16_t bf16_rn_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+
+template <int M>
+__global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
+    const uint16_t *__restrict__ q, int n_heads, const int8_t *__restrict__ cache, int64_t n_rows,
+    const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks,
+    float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status) {
+    using Lay = TcLayout<M>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    unsigned char *Qs = smem + Lay::kQ;
+    unsigned char *Cs = smem + Lay::kC;
+    unsigned char *Phi = smem + Lay::kPhi;
+    unsigned char *Plo = smem + Lay::kPlo;
+    float *scl = reinterpret_cast<float *>(smem + Lay::kScl);
+    int *ridx = reinterpret_cast<int *>(smem + Lay::kRow);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kTmem);
+    int *flag = reinterpret_cast<int *>(smem + Lay::kFlag);
+
+    const int n = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t ml_base = (static_cast<int64_t>(n) * n_chunks + c) * n_heads;
+
+    if (tid == 0) *flag = 0;
+    __syncthreads();
+    if (tid < kTcRows) {
+        const int j = c * kTcRows + tid;
+        const int r = j < width ? rows[static_cast<int64_t>(n) * width + j] : -1;
+        const bool ok = r >= 0 && r < n_rows;
+        ridx[tid] = ok ? r : -1;
+        if (ok) atomicOr(flag, 1);
+    }
+    __syncthreads();
+    if (*flag == 0) {  // no valid entry in this chunk: an empty partial
+        for (int h = tid; h < n_heads; h += blockDim.x) {
+            part_ml[2 * (ml_base + h)] = -INFINITY;
+            part_ml[2 * (ml_base + h) + 1] = 0.0f;
+        }
+        return;
+    }
+    if (warp == 0) {
+        tc::tmem_alloc(tc::smem_addr(tmem_slot), 512);
+        tc::tmem_relinquish();
+        tc::fence_before_sync();
+    }
+    if (tid == 32) {
+        tc::mbar_init(tc::smem_addr(&bar[0]), 1);
+        tc::mbar_init(tc::smem_addr(&bar[1]), 1);
+        tc::mbar_fence_init();
+    }
+
+    // 1. gather the chunk's rows (codes widened to bf16) and its scales
+    for (int i = tid; i < kTcRows * 32; i += kTcThreads) {
+        const int g = i >> 5, t = i & 31;
+        const int j = (g & 7) * 8 + (t & 7);     // entry (row) of the chunk
+        const int k = (g >> 3) * 4 + (t >> 3);   // 16-byte piece of its codes (dims 16k .. 16k+15)
+        const int r = ridx[j];
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (r >= 0) v = __ldg(reinterpret_cast<const uint4 *>(cache + static_cast<int64_t>(r) * kRowBytes) + k);
+        unsigned char *line = Cs + (j >> 3) * 8192 + (2 * k) * 128 + (j & 7) * 16;
+        *reinterpret_cast<uint4 *>(line) = make_uint4(codes_to_bf16x2(v.x, 0), codes_to_bf16x2(v.x, 16),
+                                                      codes_to_bf16x2(v.y, 0), codes_to_bf16x2(v.y, 16));
+        *reinterpret_cast<uint4 *>(line + 128) = make_uint4(codes_to_bf16x2(v.z, 0), codes_to_bf16x2(v.z, 16),
+                                                            codes_to_bf16x2(v.w, 0), codes_to_bf16x2(v.w, 16));
+    }
+    if (tid < kTcRows) {
+        const int r = ridx[tid];
+        scl[tid] = r >= 0 ? __ldg(reinterpret_cast<const float *>(cache + static_cast<int64_t>(r) * kRowBytes + kLatent)) : 0.0f;
+    }
+    const uint16_t *qn = q + static_cast<int64_t>(n) * n_heads * kLatent;
+    for (int i = tid; i < M * 64; i += kTcThreads) {
+        const int g = i >> 5, t = i & 31;
+        const int hg = g % (M / 8), dq = g / (M / 8);
+        const int h = hg * 8 + (t & 7);
+        const int dg = dq * 4 + (t >> 3);
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (h < n_heads) v = __ldg(reinterpret_cast<const uint4 *>(qn + static_cast<int64_t>(h) * kLatent) + dg);
+        *reinterpret_cast<uint4 *>(Qs + hg * 8192 + dg * 128 + (h & 7) * 16) = v;
+    }
+    tc::fence_proxy_async();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *tmem_slot;
+
+    // 2. S = Q . C^T
+    if (tid == 0) {
+        const uint32_t idesc = tc::idesc_bf16(M, kTcRows, false, false);
+        const uint32_t qa = tc::smem_addr(Qs), ca = tc::smem_addr(Cs);
+#pragma unroll 4
+        for (int ks = 0; ks < kLatent / 16; ks++)
+            tc::mma_bf16(tmem, tc::desc(qa + ks * 256, 128, 8192), tc::desc(ca + ks * 256, 128, 8192), idesc,
+                         ks > 0 ? 1u : 0u);
+        tc::mma_commit(tc::smem_addr(&bar[0]));
+    }
+
+    // 3. softmax of the chunk on warps 0-3 (TMEM lane = head)
+    if (warp < 4) {
+        if (!tc::mbar_wait(tc::smem_addr(&bar[0]), 0, kWaitLimit)) atomicOr(status, 1);
+        __syncwarp();  // thread 0 arrives here after issuing the MMAs: reconverge for tcgen05.ld
+        tc::fence_after_sync();
+        uint32_t r0[32], r1[32];
+        const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+        tc::tmem_ld32(ta, r0);
+        tc::tmem_ld32(ta + 32, r1);
+        tc::tmem_wait_ld();
+        const int head = (M == 128) ? warp * 32 + lane : (lane < 16 ? warp * 16 + lane : -1);
+        if (head >= 0) {
+            const float k2 = sm_scale * 1.4426950408889634f;  // scores in log2 units
+            float s[kTcRows];
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kTcRows; j++) {
+                const float raw = __uint_as_float(j < 32 ? r0[j] : r1[j - 32]);
+                s[j] = ridx[j] >= 0 ? raw * scl[j] * k2 : -INFINITY;
+                mx = fmaxf(mx, s[j]);
+            }
+            float l = 0.0f;
+            const bool real = head < n_heads;
+#pragma unroll
+            for (int rg = 0; rg < kTcRows / 8; rg++) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; e++) {
+                    uint32_t hb[2], lb[2];
+#pragma unroll
+                    for (int u = 0; u < 2; u++) {
+                        const int j = rg * 8 + 2 * e + u;
+                        const float p = ridx[j] >= 0 ? exp2f(s[j] - mx) : 0.0f;
+                        l += p;
+                        const float pp = real ? p * scl[j] : 0.0f;
+                        const uint16_t h16 = bf16_rn_bits(pp);
+                        hb[u] = h16;
+                        lb[u] = bf16_rn_bits(pp - __uint_as_float(static_cast<uint32_t>(h16) << 16));
+                    }
+                    hi[e] = hb[0] | (hb[1] << 16);
+                    lo[e] = lb[0] | (lb[1] << 16);
+                }
+                const int off = (head >> 3) * 1024 + rg * 128 + (head & 7) * 16;
+                *reinterpret_cast<uint4 *>(Phi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4 *>(Plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+            if (real) {
+                part_ml[2 * (ml_base + head)] = mx * 0.6931471805599453f;  // back to natural log
+                part_ml[2 * (ml_base + head) + 1] = l;
+            }
+        }
+        tc::fence_before_sync();
+    }
+    tc::fence_proxy_async();
+    __syncthreads();
+
+    // 4. O = P' . C (hi and lo terms accumulate into the same columns)
+    if (tid == 0) {
+        tc::fence_after_sync();
+        const uint32_t idesc = tc::idesc_bf16(M, 256, false, true);
+        const uint32_t ph = tc::smem_addr(Phi), pl = tc::smem_addr(Plo), ca = tc::smem_addr(Cs);
+#pragma unroll
+        for (int nh = 0; nh < 2; nh++) {
+#pragma unroll
+            for (int ks = 0; ks < kTcRows / 16; ks++) {
+                const uint64_t b = tc::desc(ca + ks * 2 * 8192 + nh * 32 * 128, 8192, 128);
+                tc::mma_bf16(tmem + nh * 256, tc::desc(ph + ks * 256, 128, 1024), b, idesc, ks > 0 ? 1u : 0u);
+                tc::mma_bf16(tmem + nh * 256, tc::desc(pl + ks * 256, 128, 1024), b, idesc, 1u);
+            }
+        }
+        tc::mma_commit(tc::smem_addr(&bar[1]));
+    }
+
+    // 5. unnormalised O to the workspace: warp w reads lane quadrant w % 4, columns half w / 4
+    {
+        if (!tc::mbar_wait(tc::smem_addr(&bar[1]), 0, kWaitLimit)) atomicOr(status, 2);
+        __syncwarp();
+        tc::fence_after_sync();
+        const int quad = warp & 3, half = warp >> 2;
+        const int head = (M == 128) ? quad * 32 + lane : (lane < 16 ? quad * 16 + lane : -1);
+        const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 256;
+#pragma unroll 1
+        for (int cb = 0; cb < 8; cb++) {
+            uint32_t r[32];
+            tc::tmem_ld32(ta + cb * 32, r);
+            tc::tmem_wait_ld();
+            if (head >= 0 && head < n_heads) {
+                float4 *dst = reinterpret_cast<float4 *>(part_acc + (ml_base + head) * kLatent + half * 256 + cb * 32);
+#pragma unroll
+                for (int e = 0; e < 8; e++)
+                    dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
+                                         __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) {
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, 512);
+    }
+}
+
+int mla_tc_chunk() { return kTcRows; }
+
+cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
+                                const int32_t *rows, int n_q, int width, float sm_scale,
+                                float *part_acc, float *part_ml, int *status, cudaStream_t stream) {
+    const int n_chunks = (width + kTcRows - 1) / kTcRows;
+    dim3 grid(n_chunks, n_q);
+    cudaError_t e;
+    if (n_heads <= 64) {
+        const int smem = TcLayout<64>::kBytes;
+        e = cudaFuncSetAttribute(mla_split_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        mla_split_tc_kernel<64><<<grid, kTcThreads, smem, stream>>>(
+            static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
+            part_acc, part_ml, status);
+    } else {
+        const int smem = TcLayout<128>::kBytes;
+        e = cudaFuncSetAttribute(mla_split_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+        if (e != cudaSuccess) return e;
+        mla_split_tc_kernel<128><<<grid, kTcThreads, smem, stream>>>(
+            static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
+            part_acc, part_ml, status);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace glm
