@@ -209,9 +209,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
         // (a) the boundary bin from the 2048-bin histogram (defaults keep every write in bounds
         // should the histogram not match the scores)
         if (tid == 0) { sm.bin = 0; sm.above = 0; sm.n_b = 0xffffffffu; }
+        unsigned *h_stage = reinterpret_cast<unsigned *>(sm.bnd);  // free until step (b)
+        for (int i = tid; i < kHistBins; i += blockDim.x) h_stage[i] = ghist[static_cast<int64_t>(n) * kHistBins + i];
         __syncthreads();
-        if (tid < 32) find_bin_warp(ghist + static_cast<int64_t>(n) * kHistBins, kHistBins,
-                                    static_cast<unsigned>(select_k), &sm.bin, &sm.above, &sm.n_b);
+        if (tid < 32) find_bin_warp(h_stage, kHistBins, static_cast<unsigned>(select_k), &sm.bin, &sm.above, &sm.n_b);
         if (tid == 0) sm.n_a = 0;
         __syncthreads();
         const unsigned bstar = sm.bin, n_above = sm.above, m_b = sm.n_b;
@@ -219,34 +220,61 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(
         __syncthreads();
         if (tid == 0) sm.n_b = 0;
         __syncthreads();
-        // (b) one pass: A = keys of higher bins, B = keys of the boundary bin
-        for (int base = 0; base < n_vis; base += blockDim.x * 4) {
-            uint32_t key[4];
-            int idx[4];
-#pragma unroll
-            for (int u = 0; u < 4; u++) {
-                idx[u] = base + u * blockDim.x + tid;
-                key[u] = idx[u] < n_vis ? score_key(row[idx[u]]) : 0u;
+        // (b) one pass: A = keys of higher bins, B = keys of the boundary bin. 16 scores per thread
+        // per round (four 16-byte loads when the row is 16-byte aligned) keep ~64 KB in flight.
+        auto classify = [&](int idx, uint32_t key, bool ok) {
+            const unsigned d = key >> (32 - kHistBitsTop);
+            const bool a = ok && d > bstar;
+            const bool bb = ok && fits && d == bstar;
+            const unsigned am = __ballot_sync(0xffffffffu, a);
+            const unsigned bm = __ballot_sync(0xffffffffu, bb);
+            unsigned pa = 0, pb = 0;
+            if (lane == 0) {
+                if (am) pa = atomicAdd(&sm.n_a, __popc(am));
+                if (bm) pb = atomicAdd(&sm.n_b, __popc(bm));
             }
+            pa = __shfl_sync(0xffffffffu, pa, 0);
+            pb = __shfl_sync(0xffffffffu, pb, 0);
+            const unsigned lt = (1u << lane) - 1;
+            const unsigned ra = pa + __popc(am & lt), rb = pb + __popc(bm & lt);
+            if (a && ra < static_cast<unsigned>(kMaxSelect)) sm.cand[ra] = compose(key, idx);
+            if (bb && rb < static_cast<unsigned>(kBoundCap)) sm.bnd[rb] = compose(key, idx);
+        };
+        if ((reinterpret_cast<uintptr_t>(row) & 15) == 0) {
+            const int n4 = n_vis >> 2;
+            const float4 *row4 = reinterpret_cast<const float4 *>(row);
+            for (int base = 0; base < n4; base += blockDim.x * 4) {
+                float4 v[4];
 #pragma unroll
-            for (int u = 0; u < 4; u++) {
-                const bool ok = idx[u] < n_vis;
-                const unsigned d = key[u] >> (32 - kHistBitsTop);
-                const bool a = ok && d > bstar;
-                const bool bb = ok && fits && d == bstar;
-                const unsigned am = __ballot_sync(0xffffffffu, a);
-                const unsigned bm = __ballot_sync(0xffffffffu, bb);
-                unsigned pa = 0, pb = 0;
-                if (lane == 0) {
-                    if (am) pa = atomicAdd(&sm.n_a, __popc(am));
-                    if (bm) pb = atomicAdd(&sm.n_b, __popc(bm));
+                for (int u = 0; u < 4; u++) {
+                    const int i4 = base + u * blockDim.x + tid;
+                    v[u] = i4 < n4 ? row4[i4] : make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                pa = __shfl_sync(0xffffffffu, pa, 0);
-                pb = __shfl_sync(0xffffffffu, pb, 0);
-                const unsigned lt = (1u << lane) - 1;
-                const unsigned ra = pa + __popc(am & lt), rb = pb + __popc(bm & lt);
-                if (a && ra < static_cast<unsigned>(kMaxSelect)) sm.cand[ra] = compose(key[u], idx[u]);
-                if (bb && rb < static_cast<unsigned>(kBoundCap)) sm.bnd[rb] = compose(key[u], idx[u]);
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const int i4 = base + u * blockDim.x + tid;
+                    const bool ok = i4 < n4;
+                    classify(4 * i4 + 0, score_key(v[u].x), ok);
+                    classify(4 * i4 + 1, score_key(v[u].y), ok);
+                    classify(4 * i4 + 2, score_key(v[u].z), ok);
+                    classify(4 * i4 + 3, score_key(v[u].w), ok);
+                }
+            }
+            for (int i = 4 * n4 + tid; i < 4 * n4 + 32 * ((n_vis - 4 * n4 + 31) / 32); i += blockDim.x)
+                classify(i, i < n_vis ? score_key(row[i]) : 0u, i < n_vis);
+        } else {
+            for (int base = 0; base < n_vis; base += blockDim.x * 4) {
+                uint32_t key[4];
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const int i = base + u * blockDim.x + tid;
+                    key[u] = i < n_vis ? score_key(row[i]) : 0u;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const int i = base + u * blockDim.x + tid;
+                    classify(i, key[u], i < n_vis);
+                }
             }
         }
         __syncthreads();

@@ -192,8 +192,12 @@ def _topk_given(cuda, scores32, n_vis, S):
     nq, ld = scores32.shape
     topk = torch.full((nq, S), 777, dtype=torch.int32, device=cuda)
     n_sel = torch.full((nq,), 777, dtype=torch.int32, device=cuda)
+    dims = kp.make_dims(16)
+    ws = torch.empty(kp.glm_dsa_workspace_size(dims, kp.GLM_OP_TOPK_POOLS, nq, ld, S), dtype=torch.uint8,
+                     device=cuda)
+    ws.fill_(0xA5)                                   # contents on entry must not matter
     kp.glm_topk_pools(torch.from_numpy(scores32).to(cuda), to_dev(n_vis, torch.int32, cuda), S, topk,
-                      n_sel=n_sel)
+                      n_sel=n_sel, workspace=ws)
     return np_(topk), np_(n_sel)
 
 
