@@ -223,6 +223,31 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q_dev, const int
                           float sm_scale, void *out_dev, float *lse_dev, float *out_f32_dev,
                           void *workspace_dev, size_t ws_bytes, void *stream);
 
+/*
+ * The same sparse NoPE MLA decode without a workspace argument. The pages have no counterpart:
+ * this entry point exists for callers that cannot allocate device memory where they run the
+ * attention -- plugin interfaces that pass a kernel only its inputs and outputs, and serving
+ * loops that allow no allocation after start-up. Arguments, results and checks are those of
+ * glm_sparse_mla_decode minus the workspace; the split partials live instead in one fixed
+ * scratch array of GLM_NOALLOC_SCRATCH_BYTES compiled into the library (held on every GPU that
+ * loads the library until the process exits). This call itself allocates nothing.
+ *   - A request needing more than the scratch holds -- n_q * ceil(width / 64) * n_heads partials of
+ *     2,056 bytes each, each region rounded up to 256 bytes, plus 256 bytes -- returns
+ *     GLM_ERR_WORKSPACE before anything is enqueued (one 64-head query of width 2,176 needs about
+ *     4.5 MiB, one 128-head query about 9 MiB).
+ *   - The first call on a device looks up the scratch's device address for that device (the
+ *     device current at the call); make that first call before any stream capture.
+ *   - Every call shares the one array, and the status word is cleared at the start of each call:
+ *     calls that overlap on the GPU (other streams, other host threads) race on it and must be
+ *     serialised by the caller.
+ *   - GLM_ERR_CUDA does not update glm_last_cuda_error().
+ */
+#define GLM_NOALLOC_SCRATCH_BYTES (16u << 20)
+int glm_sparse_mla_decode_noalloc(const glm_dsa_dims *dims, const void *q_dev,
+                                  const int8_t *cache_dev, int64_t n_rows, const int32_t *rows_dev,
+                                  int32_t n_q, int32_t width, float sm_scale, void *out_dev,
+                                  float *lse_dev, float *out_f32_dev, void *stream);
+
 /* ------------------------------------------------------------------------------------------ */
 /* workspace sizes                                                                             */
 /* ------------------------------------------------------------------------------------------ */

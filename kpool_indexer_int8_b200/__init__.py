@@ -232,3 +232,26 @@ def glm_sparse_mla_decode(dims, q, cache, rows, sm_scale, out, workspace, lse=No
                                      rows.shape[0], rows.shape[1], float(sm_scale), _ptr(out),
                                      _ptr(lse), _ptr(out_f32), _ptr(workspace), workspace.numel(),
                                      _stream(stream)), "glm_sparse_mla_decode")
+
+
+# ------------------------------------------------------------------------------------------------
+# allocation-free variant of the sparse MLA decode (for callers that cannot allocate a workspace)
+# ------------------------------------------------------------------------------------------------
+GLM_NOALLOC_SCRATCH_BYTES = 16 << 20
+lib.glm_sparse_mla_decode_noalloc.argtypes = [_D, _P, _P, _I64, _P, _I32, _I32, _F32, _P, _P, _P, _P]
+lib.glm_sparse_mla_decode_noalloc.restype = C.c_int
+
+
+def glm_sparse_mla_decode_noalloc(dims, q, cache, rows, sm_scale, out, lse=None, out_f32=None,
+                                  stream=None) -> None:
+    """glm_sparse_mla_decode without a workspace: the split partials live in a fixed scratch inside
+    the library (for callers that cannot allocate). Same tensors as glm_sparse_mla_decode."""
+    for t, dt, nm in ((q, torch.bfloat16, "q"), (cache, torch.int8, "cache"),
+                      (rows, torch.int32, "rows"), (out, torch.bfloat16, "out"),
+                      (lse, torch.float32, "lse"), (out_f32, torch.float32, "out_f32")):
+        _dev(t, dt, nm)
+    n_rows = cache.numel() // GLM_ROW_BYTES
+    _check(lib.glm_sparse_mla_decode_noalloc(C.byref(dims), _ptr(q), _ptr(cache), n_rows, _ptr(rows),
+                                             rows.shape[0], rows.shape[1], float(sm_scale), _ptr(out),
+                                             _ptr(lse), _ptr(out_f32), _stream(stream)),
+           "glm_sparse_mla_decode_noalloc")
