@@ -25,8 +25,35 @@ int num_sms() {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Per-query 2048-bin histogram of score keys used by the selection (first in the workspace).
-size_t hist_bytes(int n_q) { return align_up(static_cast<size_t>(n_q) * glm::kHistBins * sizeof(unsigned), 256); }
+// Workspace of a selection (first in the workspace of both selection entry points): per query a
+// 2048-bin histogram of score keys and 4 counters (zeroed by one memset before each selection),
+// then list A (select_k-bound candidates above the boundary bin) and list B (the boundary bin).
+struct SelWs {
+    unsigned *hist;
+    unsigned *counters;
+    unsigned long long *alist;
+    unsigned long long *blist;
+    size_t zero_bytes;
+};
+size_t sel_zero_bytes(int n_q) { return static_cast<size_t>(n_q) * (glm::kHistBins + 4) * sizeof(unsigned); }
+size_t sel_bytes(int n_q, int64_t ld) {
+    const size_t ldb = static_cast<size_t>(ld > 0 ? ld : 1);
+    return align_up(sel_zero_bytes(n_q), 256) +
+           align_up(static_cast<size_t>(n_q) * glm::kMaxSelect * sizeof(unsigned long long), 256) +
+           align_up(static_cast<size_t>(n_q) * ldb * sizeof(unsigned long long), 256);
+}
+SelWs sel_layout(void *base, int n_q, int64_t ld) {
+    char *p = static_cast<char *>(base);
+    SelWs w;
+    w.hist = reinterpret_cast<unsigned *>(p);
+    w.counters = w.hist + static_cast<size_t>(n_q) * glm::kHistBins;
+    w.zero_bytes = sel_zero_bytes(n_q);
+    p += align_up(w.zero_bytes, 256);
+    w.alist = reinterpret_cast<unsigned long long *>(p);
+    p += align_up(static_cast<size_t>(n_q) * glm::kMaxSelect * sizeof(unsigned long long), 256);
+    w.blist = reinterpret_cast<unsigned long long *>(p);
+    return w;
+}
 
 // Workspace of the sparse MLA: partial accumulators and (m, l) pairs per (query, chunk, head),
 // then a 256-byte tail whose first word is the kernels' status (nonzero after a timed-out wait).
@@ -108,10 +135,11 @@ size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
     switch (op) {
         case GLM_OP_INDEX_SCORES_TOPK:
             if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
-            return hist_bytes(n_q) + align_up(static_cast<size_t>(n_q) * static_cast<size_t>(max_pools) * sizeof(float), 256) + 256;
+            return sel_bytes(n_q, max_pools) +
+                   align_up(static_cast<size_t>(n_q) * static_cast<size_t>(max_pools) * sizeof(float), 256) + 256;
         case GLM_OP_TOPK_POOLS:
             if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
-            return hist_bytes(n_q);
+            return sel_bytes(n_q, max_pools);
         case GLM_OP_SPARSE_MLA:
             if (width < 1 || width > 65536) return static_cast<size_t>(-1);
             return mla_workspace(n_q, dims->n_heads, width);
@@ -140,21 +168,22 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const flo
         return GLM_ERR_INVALID_ARG;
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, n_q, ld_pools, select_k, 0);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
-    unsigned *ghist = static_cast<unsigned *>(workspace);
+    const SelWs sw = sel_layout(workspace, n_q, ld_pools);
     char *ws = static_cast<char *>(workspace);
-    float *sbuf = scores ? scores : reinterpret_cast<float *>(ws + hist_bytes(n_q));
+    float *sbuf = scores ? scores : reinterpret_cast<float *>(ws + sel_bytes(n_q, ld_pools));
     int *status = reinterpret_cast<int *>(ws + need - 256);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const glm::NvisSource src{nullptr, q_seq, q_pos, pad, len, batch, ld_pools};
+    rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
+    if (rc != GLM_OK) return rc;
     if (ld_pools > 0) {
-        rc = cuda_status(cudaMemsetAsync(ghist, 0, static_cast<size_t>(n_q) * glm::kHistBins * sizeof(unsigned), st));
-        if (rc != GLM_OK) return rc;
         rc = cuda_status(glm::launch_index_scores_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len,
-                                                     batch, n_q, sbuf, ghist, scores != nullptr, status,
+                                                     batch, n_q, sbuf, sw.hist, scores != nullptr, status,
                                                      num_sms(), st));
         if (rc != GLM_OK) return rc;
     }
-    return cuda_status(glm::launch_topk_select(sbuf, src, ghist, n_q, select_k, topk, n_sel, st));
+    return cuda_status(glm::launch_topk_collect(sbuf, src, sw.hist, sw.counters, sw.alist, sw.blist, n_q,
+                                                select_k, topk, n_sel, st));
 }
 
 int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w,
@@ -186,16 +215,17 @@ int glm_topk_pools(const float *scores, int64_t ld_scores, const int32_t *n_visi
     if ((scores && !aligned(scores, 4)) || !aligned(n_visible, 4) || !aligned(topk, 4) ||
         (n_sel && !aligned(n_sel, 4)))
         return GLM_ERR_INVALID_ARG;
-    const size_t need = hist_bytes(n_q);
+    const size_t need = sel_bytes(n_q, ld_scores);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
-    unsigned *ghist = static_cast<unsigned *>(workspace);
+    const SelWs sw = sel_layout(workspace, n_q, ld_scores);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const glm::NvisSource src{n_visible, nullptr, nullptr, nullptr, nullptr, 0, ld_scores};
-    int rc = cuda_status(cudaMemsetAsync(ghist, 0, static_cast<size_t>(n_q) * glm::kHistBins * sizeof(unsigned), st));
+    int rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
     if (rc != GLM_OK) return rc;
-    rc = cuda_status(glm::launch_topk_hist(scores, src, n_q, ghist, st));
+    rc = cuda_status(glm::launch_topk_hist(scores, src, n_q, sw.hist, st));
     if (rc != GLM_OK) return rc;
-    return cuda_status(glm::launch_topk_select(scores, src, ghist, n_q, select_k, topk, n_sel, st));
+    return cuda_status(glm::launch_topk_collect(scores, src, sw.hist, sw.counters, sw.alist, sw.blist, n_q,
+                                                select_k, topk, n_sel, st));
 }
 
 int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk, const int32_t *n_sel,

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "glm_dsa.h"
 
 namespace glm {
@@ -48,6 +50,31 @@ __device__ __forceinline__ int visible_pools(int pad, int len, int q_pos, long l
     int n = min(len, upto) / kKpool;
     if (len < 0) n = 0;
     return static_cast<int>(min(static_cast<long long>(n), ld_pools));
+}
+
+// Programmatic dependent launch: a kernel launched with launch_pdl may start while the previous
+// kernel of the stream is still running; pdl_begin() makes it wait (before any global memory
+// access) until that kernel has finished and its writes are visible, then lets the next kernel
+// of the stream be scheduled. Without the launch attribute both instructions are no-ops.
+__device__ __forceinline__ void pdl_begin() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(std::forward<Args>(args))...);
 }
 
 }  // namespace glm

@@ -17,6 +17,7 @@ __global__ void __launch_bounds__(kExpandThreads) expand_kernel(
     const int32_t *__restrict__ pad, const int32_t *__restrict__ len, int batch, int select_k,
     const int64_t *__restrict__ slot_map, int64_t ld_slot, int out_width,
     int32_t *__restrict__ tok_out, int32_t *__restrict__ rows_out) {
+    pdl_begin();
     __shared__ int s_nsel;
     const int n = blockIdx.y;
     const int j = blockIdx.x * blockDim.x + threadIdx.x;
@@ -71,7 +72,7 @@ cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32
                           int n_q, int select_k, const int64_t *slot_map, int64_t ld_slot, int out_width,
                           int32_t *tok, int32_t *rows, cudaStream_t stream) {
     dim3 grid(static_cast<unsigned>((out_width + kExpandThreads - 1) / kExpandThreads), n_q);
-    expand_kernel<<<grid, kExpandThreads, 0, stream>>>(topk, n_sel, q_seq, q_pos, pad, len, batch, select_k,
+    launch_pdl(expand_kernel, dim3(grid), dim3(kExpandThreads), 0, stream, topk, n_sel, q_seq, q_pos, pad, len, batch, select_k,
                                                       slot_map, ld_slot, out_width, tok, rows);
     return cudaGetLastError();
 }

@@ -4,16 +4,17 @@
 //     score[n][p] = sum_h w[n][h] * max(0, sum_d q_idx[n][h][d] * pooled[b][p][d])
 //
 // Decode form: grid (G, n_q), G ~ SMs / n_q; CTA g of query n owns a contiguous range of the
-// query's visible pools and walks it in tiles of 128 pools:
-//   * the fp32 pooled keys of a tile (64 KB) are read straight into registers, one tile ahead of
-//     the tensor cores (each warp load covers 8 pools x 128 contiguous bytes);
-//   * each fp32 value x is split exactly into three bf16 terms (hi = rn(x), mid = rn(x - hi),
-//     lo = rn(x - hi - mid)) written as 8x8 core matrices into a double-buffered shared tile;
-//   * per term, 8 UMMAs (M = 128 pools, N = 32 heads, K = 16) accumulate q . term into an fp32
-//     tile of tensor memory (double-buffered, 2 x 32 columns): with bf16 q exact, the three terms
-//     reproduce q . x to fp32 accumulation accuracy;
-//   * the epilogue (one TMEM lane = one pool per thread) applies relu and the head weights,
-//     writes the score and adds its top-11-bit key digit to the selection histogram.
+// query's visible pools. Warp-specialised pipeline, every hand-off an mbarrier:
+//   * producer (warp 0): 1-D bulk copies of 32 pools (16 KB, contiguous) into 4 staging slots;
+//   * converters (warps 8-15): split each fp32 value x exactly into three bf16 terms
+//     (hi = rn(x), mid = rn(x - hi), lo = rn(x - hi - mid)) written as K-major tiles of 64 pools in
+//     the 128-byte swizzle layout (lane reads 16 consecutive bytes of a pool row, writes 8 bytes of
+//     a swizzled 128-byte row: no bank conflicts); two tile buffers;
+//   * MMA issuer (warp 1): per term 8 UMMAs (M = 64 pools, N = 32 heads, K = 16) into one of two
+//     fp32 tensor-memory accumulators; with the bf16 query exact, the three terms reproduce q . x
+//     to fp32 accumulation accuracy;
+//   * epilogue (warps 4-7, one TMEM lane quadrant each): relu and head weights, the score, and its
+//     top-11-bit key digit added to the selection histogram.
 // HBM-bound: 512 bytes of pooled key per pool; the tensor cores run at a few percent.
 #include "common.cuh"
 #include "tc.cuh"
@@ -21,35 +22,42 @@
 
 namespace glm {
 
-constexpr int kIxThreads = 256;
-constexpr int kIxTile = 128;                       // pools per tile (UMMA M)
-constexpr int kIxTermBytes = kIxTile * kIdxDim * 2; // one bf16 term of a tile: 32 KB
+constexpr int kIxThreads = 512;                        // 16 warps, see the roles above
+constexpr int kIxTile = 64;                            // pools per tile (UMMA M)
+constexpr int kIxChunk = 32;                           // pools per bulk copy (2 per tile)
+constexpr int kIxStages = 4;                           // bulk copies in flight
+constexpr int kIxConv = 8;                             // converter warps
+constexpr int kIxAtomBytes = kIxTile * 128;            // 64 rows x 128 bytes (64 dims): 8 KB
+constexpr int kIxTermBytes = 2 * kIxAtomBytes;         // one bf16 term of a tile: 16 KB
+constexpr int kIxBufBytes = 3 * kIxTermBytes;          // three terms: 48 KB
+constexpr int kIxStageBytes = kIxChunk * kIdxDim * 4;  // 16 KB of fp32 pooled keys
 constexpr uint32_t kIxWaitLimit = 1u << 22;
 
-struct IxLayout {
-    static constexpr int kA = 0;                                  // [2 buffers][3 terms][32 KB]
-    static constexpr int kQ = kA + 2 * 3 * kIxTermBytes;          // 32 heads x 128 dims bf16 (8 KB)
-    static constexpr int kHist = kQ + kIdxHeads * kIdxDim * 2;    // 2048 uint32
-    static constexpr int kW = kHist + kHistBins * 4;              // 32 fp32 head weights
-    static constexpr int kBar = kW + kIdxHeads * 4;               // 2 mbarriers
-    static constexpr int kTmem = kBar + 16;
+struct IxLayout {                                      // offsets from a 1024-byte aligned base
+    static constexpr int kTerms = 0;                                  // [2 buffers][3 terms][16 KB]
+    static constexpr int kStage = kTerms + 2 * kIxBufBytes;           // [4 stages][16 KB]
+    static constexpr int kQ = kStage + kIxStages * kIxStageBytes;     // 32 heads x 128 dims bf16
+    static constexpr int kHist = kQ + kIdxHeads * kIdxDim * 2;        // 2048 uint32
+    static constexpr int kW = kHist + kHistBins * 4;                  // 32 fp32 head weights
+    static constexpr int kBar = kW + kIdxHeads * 4;                   // 16 mbarriers
+    static constexpr int kTmem = kBar + 16 * 8;
     static constexpr int kBytes = kTmem + 16;
+    static constexpr int kAlloc = kBytes + 1024;                      // room to align the base
 };
+// mbarrier indices
+constexpr int kBarStFull = 0;     // [4] staging slot filled (producer, tx bytes)
+constexpr int kBarStEmpty = 4;    // [4] staging slot read (8 converter warps)
+constexpr int kBarTmFull = 8;     // [2] tile buffer written (8 warps x 2 chunk slots)
+constexpr int kBarTmEmpty = 10;   // [2] tile buffer read by the MMAs (commit)
+constexpr int kBarAccFull = 12;   // [2] accumulator ready (commit)
+constexpr int kBarAccEmpty = 14;  // [2] accumulator read (4 epilogue warps)
 
 __device__ __forceinline__ uint32_t bf16_pair(float a, float b) {
-    return static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(a))) |
-           (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(b))) << 16);
+    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low half), .y = b
+    return *reinterpret_cast<const uint32_t *>(&v);
 }
 __device__ __forceinline__ float bf16_lo_f(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
-
-__device__ __forceinline__ float4 ld_stream(const float *p) {
-    float4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "l"(p));
-    return v;
-}
 
 __global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
     const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
@@ -57,12 +65,14 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ pad,
     const int32_t *__restrict__ len, int batch, float *__restrict__ scores,
     unsigned *__restrict__ ghist, int fill_invisible, int *__restrict__ status) {
-    extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char *A = smem + IxLayout::kA;
+    pdl_begin();
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
+    unsigned char *terms = smem + IxLayout::kTerms;
+    unsigned char *stage = smem + IxLayout::kStage;
     unsigned char *Qs = smem + IxLayout::kQ;
     unsigned *hist = reinterpret_cast<unsigned *>(smem + IxLayout::kHist);
     float *ws = reinterpret_cast<float *>(smem + IxLayout::kW);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + IxLayout::kBar);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + IxLayout::kTmem);
 
     const int n = blockIdx.y, g = blockIdx.x, G = gridDim.x;
@@ -83,122 +93,145 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
     const int lo = g * per;
     const int hi = min(n_vis, lo + per);
     if (lo >= hi) return;
+    const int n_chunks = (hi - lo + kIxChunk - 1) / kIxChunk;
     const int n_tiles = (hi - lo + kIxTile - 1) / kIxTile;
+    const float *src = pooled + (static_cast<int64_t>(b) * ld_pools + lo) * kIdxDim;
 
+    const uint32_t bar0 = tc::smem_addr(smem + IxLayout::kBar);
+    auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
     if (warp == 0) {
         tc::tmem_alloc(tc::smem_addr(tmem_slot), 64);
         tc::tmem_relinquish();
         tc::fence_before_sync();
     }
     if (tid == 32) {
-        tc::mbar_init(tc::smem_addr(&bar[0]), 1);
-        tc::mbar_init(tc::smem_addr(&bar[1]), 1);
+        for (int i = 0; i < 4; i++) tc::mbar_init(bar(kBarStFull + i), 1);
+        for (int i = 0; i < 4; i++) tc::mbar_init(bar(kBarStEmpty + i), kIxConv);
+        for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarTmFull + i), 2 * kIxConv);
+        for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarTmEmpty + i), 1);
+        for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccFull + i), 1);
+        for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccEmpty + i), 4);
         tc::mbar_fence_init();
     }
     // query block (bf16 [32 x 128], core matrices: head group stride 2048 B, dim group 128 B)
-    const uint16_t *qn = q_idx + static_cast<int64_t>(n) * kIdxHeads * kIdxDim;
-    for (int i = tid; i < kIdxHeads * kIdxDim / 8; i += kIxThreads) {
-        const int h = i >> 4, dg = i & 15;
+    {
+        const uint16_t *qn = q_idx + static_cast<int64_t>(n) * kIdxHeads * kIdxDim;
+        const int i = tid, h = i >> 4, dg = i & 15;   // 512 pieces of 16 bytes, one per thread
         *reinterpret_cast<uint4 *>(Qs + (h >> 3) * 2048 + dg * 128 + (h & 7) * 16) =
-            __ldg(reinterpret_cast<const uint4 *>(qn + h * kIdxDim) + dg);
+            __ldg(reinterpret_cast<const uint4 *>(qn) + i);
     }
     if (tid < kIdxHeads) ws[tid] = w[static_cast<int64_t>(n) * kIdxHeads + tid];
     if (ghist)
         for (int i = tid; i < kHistBins; i += kIxThreads) hist[i] = 0;
-
-    const float *prow = pooled + static_cast<int64_t>(b) * ld_pools * kIdxDim;
-    // unit u = it * 8 + warp covers pool group u % 16 (8 pools) and dim quad u / 16 (32 dims)
-    float4 v[8][2];
-    auto load_tile = [&](int t) {
-#pragma unroll
-        for (int it = 0; it < 8; it++) {
-            const int u = it * 8 + warp;
-            const int p = lo + t * kIxTile + (u & 15) * 8 + (lane & 7);
-            const int d0 = (u >> 4) * 32 + (lane >> 3) * 8;
-            if (p < hi) {
-                v[it][0] = ld_stream(prow + static_cast<int64_t>(p) * kIdxDim + d0);
-                v[it][1] = ld_stream(prow + static_cast<int64_t>(p) * kIdxDim + d0 + 4);
-            } else {
-                v[it][0] = make_float4(0.f, 0.f, 0.f, 0.f);
-                v[it][1] = make_float4(0.f, 0.f, 0.f, 0.f);
-            }
-        }
-    };
-    auto store_tile = [&](int buf) {
-        unsigned char *base = A + buf * 3 * kIxTermBytes;
-#pragma unroll
-        for (int it = 0; it < 8; it++) {
-            const int u = it * 8 + warp;
-            const int off = (u & 15) * 2048 + ((u >> 4) * 4 + (lane >> 3)) * 128 + (lane & 7) * 16;
-            const float x[8] = {v[it][0].x, v[it][0].y, v[it][0].z, v[it][0].w,
-                                v[it][1].x, v[it][1].y, v[it][1].z, v[it][1].w};
-            uint32_t h[4], m[4], l[4];
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                h[e] = bf16_pair(x[2 * e], x[2 * e + 1]);
-                const float r0 = x[2 * e] - bf16_lo_f(h[e]), r1 = x[2 * e + 1] - bf16_hi_f(h[e]);
-                m[e] = bf16_pair(r0, r1);
-                l[e] = bf16_pair(r0 - bf16_lo_f(m[e]), r1 - bf16_hi_f(m[e]));
-            }
-            *reinterpret_cast<uint4 *>(base + off) = make_uint4(h[0], h[1], h[2], h[3]);
-            *reinterpret_cast<uint4 *>(base + kIxTermBytes + off) = make_uint4(m[0], m[1], m[2], m[3]);
-            *reinterpret_cast<uint4 *>(base + 2 * kIxTermBytes + off) = make_uint4(l[0], l[1], l[2], l[3]);
-        }
-    };
-
-    load_tile(0);
+    tc::fence_proxy_async();
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t idesc = tc::idesc_bf16(kIxTile, kIdxHeads, false, false);
-    const uint32_t a_addr = tc::smem_addr(A), q_addr = tc::smem_addr(Qs);
     bool ok = true;
 
-    auto epilogue = [&](int t) {
-        const int buf = t & 1;
-        if (!tc::mbar_wait(tc::smem_addr(&bar[buf]), (t >> 1) & 1, kIxWaitLimit)) ok = false;
-        __syncwarp();
-        tc::fence_after_sync();
-        uint32_t r[32];
-        tc::tmem_ld32(tmem + (static_cast<uint32_t>(warp * 32) << 16) + buf * 32, r);
-        tc::tmem_wait_ld();
-        const int p = lo + t * kIxTile + warp * 32 + lane;
-        uint32_t digit = 0xffffffffu;
-        if (p < hi) {
-            float s = 0.0f;
-#pragma unroll
-            for (int h2 = 0; h2 < kIdxHeads; h2++) s = fmaf(ws[h2], fmaxf(__uint_as_float(r[h2]), 0.0f), s);
-            srow[p] = s;
-            digit = score_key(s) >> (32 - kHistBitsTop);
-        }
-        if (ghist) hist_add(hist, digit);
-    };
-
-    for (int t = 0; t < n_tiles; t++) {
-        const int buf = t & 1;
-        if (t >= 2) {  // the MMAs of tile t-2 have released this buffer
-            if (!tc::mbar_wait(tc::smem_addr(&bar[buf]), ((t - 2) >> 1) & 1, kIxWaitLimit)) ok = false;
-        }
-        store_tile(buf);
-        if (t + 1 < n_tiles) load_tile(t + 1);
-        tc::fence_proxy_async();
-        __syncthreads();
-        if (tid == 0) {
-            tc::fence_after_sync();
-            const uint32_t d = tmem + buf * 32;
-#pragma unroll
-            for (int term = 0; term < 3; term++) {
-                const uint32_t ab = a_addr + (buf * 3 + term) * kIxTermBytes;
-#pragma unroll
-                for (int ks = 0; ks < kIdxDim / 16; ks++)
-                    tc::mma_bf16(d, tc::desc(ab + ks * 256, 128, 2048), tc::desc(q_addr + ks * 256, 128, 2048),
-                                 idesc, (term > 0 || ks > 0) ? 1u : 0u);
+    if (warp == 0) {
+        // ---------------- producer ----------------
+        if (lane == 0) {
+            const uint32_t stage_addr = tc::smem_addr(stage);
+            for (int c = 0; c < n_chunks; c++) {
+                const int slot = c % kIxStages;
+                if (c >= kIxStages && !tc::mbar_wait(bar(kBarStEmpty + slot), ((c / kIxStages) - 1) & 1, kIxWaitLimit))
+                    ok = false;
+                const uint32_t bytes = static_cast<uint32_t>(min(kIxChunk, hi - lo - c * kIxChunk)) * kIdxDim * 4;
+                tc::mbar_arrive_expect_tx(bar(kBarStFull + slot), bytes);
+                tc::bulk_g2s(stage_addr + slot * kIxStageBytes, src + static_cast<int64_t>(c) * kIxChunk * kIdxDim,
+                             bytes, bar(kBarStFull + slot));
             }
-            tc::mma_commit(tc::smem_addr(&bar[buf]));
         }
-        if (t >= 1 && warp < 4) epilogue(t - 1);
+    } else if (warp == 1) {
+        // ---------------- MMA issuer ----------------
+        if (lane == 0) {
+            const uint32_t idesc = tc::idesc_bf16(kIxTile, kIdxHeads, false, false);
+            const uint32_t terms_addr = tc::smem_addr(terms), q_addr = tc::smem_addr(Qs);
+            for (int t = 0; t < n_tiles; t++) {
+                const int tb = t & 1;
+                if (!tc::mbar_wait(bar(kBarTmFull + tb), (t >> 1) & 1, kIxWaitLimit)) ok = false;
+                if (t >= 2 && !tc::mbar_wait(bar(kBarAccEmpty + tb), ((t >> 1) - 1) & 1, kIxWaitLimit)) ok = false;
+                tc::fence_after_sync();
+                const uint32_t d = tmem + tb * 32;
+#pragma unroll
+                for (int term = 0; term < 3; term++) {
+#pragma unroll
+                    for (int ks = 0; ks < kIdxDim / 16; ks++) {
+                        const uint32_t a = terms_addr + tb * kIxBufBytes + term * kIxTermBytes +
+                                           (ks >> 2) * kIxAtomBytes + (ks & 3) * 32;
+                        tc::mma_bf16(d, tc::desc_sw128(a, 1024), tc::desc(q_addr + ks * 256, 128, 2048), idesc,
+                                     (term > 0 || ks > 0) ? 1u : 0u);
+                    }
+                }
+                tc::mma_commit(bar(kBarTmEmpty + tb));
+                tc::mma_commit(bar(kBarAccFull + tb));
+            }
+        }
+    } else if (warp >= 4 && warp < 8) {
+        // ---------------- epilogue: TMEM lane quadrant (warp % 4), rows 16q .. 16q+15 ----------------
+        const int qd = warp & 3;
+        for (int t = 0; t < n_tiles; t++) {
+            const int tb = t & 1;
+            if (!tc::mbar_wait(bar(kBarAccFull + tb), (t >> 1) & 1, kIxWaitLimit)) ok = false;
+            __syncwarp();
+            tc::fence_after_sync();
+            uint32_t r[32];
+            tc::tmem_ld32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + tb * 32, r);
+            tc::tmem_wait_ld();
+            const int p = lo + t * kIxTile + qd * 16 + lane;
+            uint32_t digit = 0xffffffffu;
+            if (lane < 16 && p < hi) {
+                float s = 0.0f;
+#pragma unroll
+                for (int h2 = 0; h2 < kIdxHeads; h2++) s = fmaf(ws[h2], fmaxf(__uint_as_float(r[h2]), 0.0f), s);
+                srow[p] = s;
+                digit = score_key(s) >> (32 - kHistBitsTop);
+            }
+            if (ghist) hist_add(hist, digit);
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(kBarAccEmpty + tb));
+        }
+    } else if (warp >= 16 - kIxConv) {
+        // ---------------- converters ----------------
+        const int cw = warp - (16 - kIxConv);
+        for (int t = 0; t < n_tiles; t++) {
+            const int tb = t & 1;
+            if (t >= 2 && !tc::mbar_wait(bar(kBarTmEmpty + tb), ((t >> 1) - 1) & 1, kIxWaitLimit)) ok = false;
+            unsigned char *buf = terms + tb * kIxBufBytes;
+            for (int half = 0; half < 2; half++) {
+                const int c = 2 * t + half;
+                if (c < n_chunks) {
+                    const int slot = c % kIxStages;
+                    if (!tc::mbar_wait(bar(kBarStFull + slot), (c / kIxStages) & 1, kIxWaitLimit)) ok = false;
+                    const unsigned char *st = stage + slot * kIxStageBytes;
+#pragma unroll
+                    for (int pi = 0; pi < kIxChunk / kIxConv; pi++) {
+                        const int pc = cw * (kIxChunk / kIxConv) + pi;   // pool within the chunk
+                        const int r = half * kIxChunk + pc;              // row within the tile
+                        const float4 x = *reinterpret_cast<const float4 *>(st + pc * (kIdxDim * 4) + lane * 16);
+                        const uint32_t h0 = bf16_pair(x.x, x.y), h1 = bf16_pair(x.z, x.w);
+                        const float r0 = x.x - bf16_lo_f(h0), r1 = x.y - bf16_hi_f(h0);
+                        const float r2 = x.z - bf16_lo_f(h1), r3 = x.w - bf16_hi_f(h1);
+                        const uint32_t m0 = bf16_pair(r0, r1), m1 = bf16_pair(r2, r3);
+                        const uint32_t l0 = bf16_pair(r0 - bf16_lo_f(m0), r1 - bf16_hi_f(m0));
+                        const uint32_t l1 = bf16_pair(r2 - bf16_lo_f(m1), r3 - bf16_hi_f(m1));
+                        const int off = (lane >> 4) * kIxAtomBytes + r * 128 +
+                                        ((((lane & 15) >> 1) ^ (r & 7)) << 4) + (lane & 1) * 8;
+                        *reinterpret_cast<uint2 *>(buf + off) = make_uint2(h0, h1);
+                        *reinterpret_cast<uint2 *>(buf + kIxTermBytes + off) = make_uint2(m0, m1);
+                        *reinterpret_cast<uint2 *>(buf + 2 * kIxTermBytes + off) = make_uint2(l0, l1);
+                    }
+                    __syncwarp();
+                    if (lane == 0) tc::mbar_arrive(bar(kBarStEmpty + slot));
+                }
+                tc::fence_proxy_async();
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(kBarTmFull + tb));
+            }
+        }
     }
-    if (warp < 4) epilogue(n_tiles - 1);
     if (!ok && status) atomicOr(status, 4);
     tc::fence_before_sync();
     __syncthreads();
@@ -222,12 +255,11 @@ cudaError_t launch_index_scores_tc(const void *q_idx, const float *w, const floa
     if (G < 1) G = 1;
     const int64_t max_tiles = (ld_pools + kIxTile - 1) / kIxTile;
     if (G > max_tiles) G = static_cast<int>(max_tiles > 0 ? max_tiles : 1);
-    const int smem = IxLayout::kBytes;
+    const int smem = IxLayout::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(index_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(G, n_q);
-    index_scores_tc_kernel<<<grid, kIxThreads, smem, stream>>>(
-        static_cast<const uint16_t *>(q_idx), w, pooled, ld_pools, q_seq, q_pos, pad, len, batch,
+    launch_pdl(index_scores_tc_kernel, dim3(grid), dim3(kIxThreads), smem, stream, static_cast<const uint16_t *>(q_idx), w, pooled, ld_pools, q_seq, q_pos, pad, len, batch,
         scores, ghist, fill_invisible ? 1 : 0, status);
     return cudaGetLastError();
 }

@@ -17,6 +17,7 @@ __global__ void __launch_bounds__(256) kpool_build_kernel(
     const int32_t *__restrict__ pad, const int32_t *__restrict__ len,
     const int32_t *__restrict__ pool_begin, int batch, int max_new_pools,
     float *__restrict__ pooled, int64_t ld_pools, int32_t *__restrict__ n_pools_out) {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     if (n_pools_out != nullptr && blockIdx.x == 0) {
         for (int b = threadIdx.x; b < batch; b += blockDim.x) {
@@ -86,9 +87,9 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
     if (blocks < 1) blocks = 1;
     int64_t cap = static_cast<int64_t>(num_sms) * 16;
     if (blocks > cap) blocks = cap;
-    kpool_build_kernel<<<static_cast<unsigned>(blocks), 32 * warps_per_block, 0, stream>>>(
-        static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(gate), ld_tokens, ln_w,
-        ln_b, eps, pad, len, pool_begin, batch, max_new_pools, pooled, ld_pools, n_pools);
+    launch_pdl(kpool_build_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * warps_per_block), 0, stream,
+               static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(gate), ld_tokens, ln_w, ln_b, eps,
+               pad, len, pool_begin, batch, max_new_pools, pooled, ld_pools, n_pools);
     return cudaGetLastError();
 }
 

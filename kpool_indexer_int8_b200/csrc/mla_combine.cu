@@ -10,34 +10,68 @@
 
 namespace glm {
 
+constexpr int kMaxCombineChunks = 1024;  // 65536 / 64
+
 __global__ void __launch_bounds__(128) mla_combine_kernel(const float *__restrict__ part_acc,
                                                           const float *__restrict__ part_ml,
                                                           int n_heads, int n_chunks,
                                                           uint16_t *__restrict__ out,
                                                           float *__restrict__ out_f32,
                                                           float *__restrict__ lse) {
+    pdl_begin();
+    __shared__ float wgt[kMaxCombineChunks];
+    __shared__ float red[4];
     const int h = blockIdx.x, n = blockIdx.y, t = threadIdx.x;
     const int64_t base = static_cast<int64_t>(n) * n_chunks * n_heads + h;
-    float M = -INFINITY;
-    for (int c = 0; c < n_chunks; c++) {
-        const float l = part_ml[2 * (base + static_cast<int64_t>(c) * n_heads) + 1];
-        if (l > 0.0f) M = fmaxf(M, part_ml[2 * (base + static_cast<int64_t>(c) * n_heads)]);
+    // every chunk's (m, l) at once: one round trip instead of one per chunk
+    float mx = -INFINITY;
+    for (int c = t; c < n_chunks; c += blockDim.x) {
+        const float2 ml = *reinterpret_cast<const float2 *>(part_ml + 2 * (base + static_cast<int64_t>(c) * n_heads));
+        wgt[c] = ml.y > 0.0f ? ml.x : -INFINITY;   // the chunk's max, or -inf if it had no entry
+        if (ml.y > 0.0f) mx = fmaxf(mx, ml.x);
     }
+    mx = warp_max(mx);
+    if ((t & 31) == 0) red[t >> 5] = mx;
+    __syncthreads();
+    const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    __syncthreads();
+    float Lp = 0.0f;
+    for (int c = t; c < n_chunks; c += blockDim.x) {
+        const float m = wgt[c];
+        const float wc = (m == -INFINITY || M == -INFINITY) ? 0.0f : expf(m - M);
+        wgt[c] = wc;
+        Lp = fmaf(part_ml[2 * (base + static_cast<int64_t>(c) * n_heads) + 1], wc, Lp);
+    }
+    Lp = warp_sum(Lp);
+    if ((t & 31) == 0) red[t >> 5] = Lp;
+    __syncthreads();
+    const float L = (red[0] + red[1]) + (red[2] + red[3]);
+    // weighted sum of the chunk accumulators, four chunks in flight per thread
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    float L = 0.0f;
-    if (M != -INFINITY) {
-        for (int c = 0; c < n_chunks; c++) {
-            const int64_t idx = base + static_cast<int64_t>(c) * n_heads;
-            const float l = part_ml[2 * idx + 1];
-            if (!(l > 0.0f)) continue;
-            const float wgt = expf(part_ml[2 * idx] - M);
-            L = fmaf(l, wgt, L);
-            const float4 v = reinterpret_cast<const float4 *>(part_acc + idx * kLatent)[t];
-            a.x = fmaf(wgt, v.x, a.x);
-            a.y = fmaf(wgt, v.y, a.y);
-            a.z = fmaf(wgt, v.z, a.z);
-            a.w = fmaf(wgt, v.w, a.w);
+    int c = 0;
+    for (; c + 4 <= n_chunks; c += 4) {
+        float4 v[4];
+#pragma unroll
+        for (int u = 0; u < 4; u++)
+            v[u] = wgt[c + u] > 0.0f ? reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(c + u) * n_heads) * kLatent)[t]
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 4; u++) {
+            const float wc = wgt[c + u];
+            a.x = fmaf(wc, v[u].x, a.x);
+            a.y = fmaf(wc, v[u].y, a.y);
+            a.z = fmaf(wc, v[u].z, a.z);
+            a.w = fmaf(wc, v[u].w, a.w);
         }
+    }
+    for (; c < n_chunks; c++) {
+        const float wc = wgt[c];
+        if (!(wc > 0.0f)) continue;
+        const float4 v = reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(c) * n_heads) * kLatent)[t];
+        a.x = fmaf(wc, v.x, a.x);
+        a.y = fmaf(wc, v.y, a.y);
+        a.z = fmaf(wc, v.z, a.z);
+        a.w = fmaf(wc, v.w, a.w);
     }
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
     const float o[4] = {a.x * inv, a.y * inv, a.z * inv, a.w * inv};
@@ -55,7 +89,7 @@ cudaError_t launch_mla_combine(const float *part_acc, const float *part_ml, int 
                                int n_chunks, void *out, float *out_f32, float *lse,
                                cudaStream_t stream) {
     dim3 grid(n_heads, n_q);
-    mla_combine_kernel<<<grid, 128, 0, stream>>>(part_acc, part_ml, n_heads, n_chunks,
+    launch_pdl(mla_combine_kernel, dim3(grid), dim3(128), 0, stream, part_acc, part_ml, n_heads, n_chunks,
                                                  static_cast<uint16_t *>(out), out_f32, lse);
     return cudaGetLastError();
 }

@@ -13,11 +13,15 @@
 //   3. softmax of the chunk, one TMEM lane (= one head) per thread: s = S * scale_j * sm_scale,
 //      m = max, p = exp(s - m), l = sum p; P' = p * scale_j (the V dequantisation scale folded
 //      in) is split into bf16 hi + lo so that the PV product keeps ~16 mantissa bits of P'.
-//   4. O = P'.C over 512 columns of tensor memory (16 MMAs of N = 256, K = 16). The same tile C
-//      is now the MN-major B operand: a core matrix of 8 rows x 8 dims serves both products.
-//   5. (m, l) and the unnormalised O of every head go to the workspace; the combine kernel merges
-//      the chunks by log-sum-exp.
-// Tensor memory: 512 columns (S in columns 0..63, then O over all 512 once S has been read).
+//   4. O^T = C^T . P'^T: the 512 latent dims are the M dimension (4 tiles of M = 128) and the heads
+//      the N dimension, so that in tensor memory one lane holds one latent dim of every head. The
+//      same tile C is now the MN-major A operand (a core matrix of 8 rows x 8 dims serves both
+//      products) and P' the K-major B operand; 2 terms x 4 K-steps x 4 tiles = 32 MMAs.
+//   5. (m, l) and the unnormalised O of every head go to the workspace (one lane per latent dim:
+//      each warp store is 32 consecutive floats of one head); the combine kernel merges the
+//      chunks by log-sum-exp.
+// Tensor memory: 512 columns (S in columns 0..M-1, then the 4 O^T tiles of M columns each over
+// columns 0..4M-1 once S has been read).
 // Every wait on the tensor cores is bounded; a timeout sets a status word and the CTA still
 // frees its tensor memory and exits.
 #include "common.cuh"
@@ -57,6 +61,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
     const uint16_t *__restrict__ q, int n_heads, const int8_t *__restrict__ cache, int64_t n_rows,
     const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks,
     float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status) {
+    pdl_begin();
     using Lay = TcLayout<M>;
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *Qs = smem + Lay::kQ;
@@ -100,33 +105,60 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
         tc::mbar_fence_init();
     }
 
-    // 1. gather the chunk's rows (codes widened to bf16) and its scales
-    for (int i = tid; i < kTcRows * 32; i += kTcThreads) {
-        const int g = i >> 5, t = i & 31;
-        const int j = (g & 7) * 8 + (t & 7);     // entry (row) of the chunk
-        const int k = (g >> 3) * 4 + (t >> 3);   // 16-byte piece of its codes (dims 16k .. 16k+15)
-        const int r = ridx[j];
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (r >= 0) v = __ldg(reinterpret_cast<const uint4 *>(cache + static_cast<int64_t>(r) * kRowBytes) + k);
-        unsigned char *line = Cs + (j >> 3) * 8192 + (2 * k) * 128 + (j & 7) * 16;
-        *reinterpret_cast<uint4 *>(line) = make_uint4(codes_to_bf16x2(v.x, 0), codes_to_bf16x2(v.x, 16),
-                                                      codes_to_bf16x2(v.y, 0), codes_to_bf16x2(v.y, 16));
-        *reinterpret_cast<uint4 *>(line + 128) = make_uint4(codes_to_bf16x2(v.z, 0), codes_to_bf16x2(v.z, 16),
-                                                            codes_to_bf16x2(v.w, 0), codes_to_bf16x2(v.w, 16));
-    }
-    if (tid < kTcRows) {
-        const int r = ridx[tid];
-        scl[tid] = r >= 0 ? __ldg(reinterpret_cast<const float *>(cache + static_cast<int64_t>(r) * kRowBytes + kLatent)) : 0.0f;
-    }
+    // 1. gather the chunk's rows (codes widened to bf16) and its scales; every global load of a
+    //    thread is issued before any of them is used, so the CTA waits for one round trip
+    constexpr int kRowIters = kTcRows * 32 / kTcThreads;   // 16-byte code pieces per thread
+    constexpr int kQIters = M * 64 / kTcThreads;           // 16-byte query pieces per thread
     const uint16_t *qn = q + static_cast<int64_t>(n) * n_heads * kLatent;
-    for (int i = tid; i < M * 64; i += kTcThreads) {
-        const int g = i >> 5, t = i & 31;
-        const int hg = g % (M / 8), dq = g / (M / 8);
-        const int h = hg * 8 + (t & 7);
-        const int dg = dq * 4 + (t >> 3);
-        uint4 v = make_uint4(0u, 0u, 0u, 0u);
-        if (h < n_heads) v = __ldg(reinterpret_cast<const uint4 *>(qn + static_cast<int64_t>(h) * kLatent) + dg);
-        *reinterpret_cast<uint4 *>(Qs + hg * 8192 + dg * 128 + (h & 7) * 16) = v;
+    {
+        uint4 v[kRowIters];
+#pragma unroll
+        for (int it = 0; it < kRowIters; it++) {
+            const int i = it * kTcThreads + tid;
+            const int g = i >> 5, t = i & 31;
+            const int j = (g & 7) * 8 + (t & 7);     // entry (row) of the chunk
+            const int k = (g >> 3) * 4 + (t >> 3);   // 16-byte piece of its codes (dims 16k .. 16k+15)
+            const int r = ridx[j];
+            v[it] = r >= 0 ? __ldg(reinterpret_cast<const uint4 *>(cache + static_cast<int64_t>(r) * kRowBytes) + k)
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
+        float sc = 0.0f;
+        if (tid < kTcRows) {
+            const int r = ridx[tid];
+            if (r >= 0) sc = __ldg(reinterpret_cast<const float *>(cache + static_cast<int64_t>(r) * kRowBytes + kLatent));
+        }
+        uint4 qv[kQIters];
+#pragma unroll
+        for (int it = 0; it < kQIters; it++) {
+            const int i = it * kTcThreads + tid;
+            const int g = i >> 5, t = i & 31;
+            const int h = (g % (M / 8)) * 8 + (t & 7);
+            const int dg = (g / (M / 8)) * 4 + (t >> 3);
+            qv[it] = h < n_heads ? __ldg(reinterpret_cast<const uint4 *>(qn + static_cast<int64_t>(h) * kLatent) + dg)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int it = 0; it < kRowIters; it++) {
+            const int i = it * kTcThreads + tid;
+            const int g = i >> 5, t = i & 31;
+            const int j = (g & 7) * 8 + (t & 7);
+            const int k = (g >> 3) * 4 + (t >> 3);
+            unsigned char *line = Cs + (j >> 3) * 8192 + (2 * k) * 128 + (j & 7) * 16;
+            *reinterpret_cast<uint4 *>(line) = make_uint4(codes_to_bf16x2(v[it].x, 0), codes_to_bf16x2(v[it].x, 16),
+                                                          codes_to_bf16x2(v[it].y, 0), codes_to_bf16x2(v[it].y, 16));
+            *reinterpret_cast<uint4 *>(line + 128) = make_uint4(codes_to_bf16x2(v[it].z, 0), codes_to_bf16x2(v[it].z, 16),
+                                                                codes_to_bf16x2(v[it].w, 0), codes_to_bf16x2(v[it].w, 16));
+        }
+        if (tid < kTcRows) scl[tid] = sc;
+#pragma unroll
+        for (int it = 0; it < kQIters; it++) {
+            const int i = it * kTcThreads + tid;
+            const int g = i >> 5, t = i & 31;
+            const int hg = g % (M / 8);
+            const int h = hg * 8 + (t & 7);
+            const int dg = (g / (M / 8)) * 4 + (t >> 3);
+            *reinterpret_cast<uint4 *>(Qs + hg * 8192 + dg * 128 + (h & 7) * 16) = qv[it];
+        }
     }
     tc::fence_proxy_async();
     __syncthreads();
@@ -200,42 +232,41 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
     tc::fence_proxy_async();
     __syncthreads();
 
-    // 4. O = P' . C (hi and lo terms accumulate into the same columns)
+    // 4. O^T = C^T . P'^T (hi and lo terms accumulate into the same columns)
     if (tid == 0) {
         tc::fence_after_sync();
-        const uint32_t idesc = tc::idesc_bf16(M, 256, false, true);
+        const uint32_t idesc = tc::idesc_bf16(128, M, true, false);
         const uint32_t ph = tc::smem_addr(Phi), pl = tc::smem_addr(Plo), ca = tc::smem_addr(Cs);
 #pragma unroll
-        for (int nh = 0; nh < 2; nh++) {
+        for (int mt = 0; mt < kLatent / 128; mt++) {
 #pragma unroll
             for (int ks = 0; ks < kTcRows / 16; ks++) {
-                const uint64_t b = tc::desc(ca + ks * 2 * 8192 + nh * 32 * 128, 8192, 128);
-                tc::mma_bf16(tmem + nh * 256, tc::desc(ph + ks * 256, 128, 1024), b, idesc, ks > 0 ? 1u : 0u);
-                tc::mma_bf16(tmem + nh * 256, tc::desc(pl + ks * 256, 128, 1024), b, idesc, 1u);
+                const uint64_t a = tc::desc(ca + ks * 2 * 8192 + mt * 16 * 128, 8192, 128);
+                tc::mma_bf16(tmem + mt * M, a, tc::desc(ph + ks * 256, 128, 1024), idesc, ks > 0 ? 1u : 0u);
+                tc::mma_bf16(tmem + mt * M, a, tc::desc(pl + ks * 256, 128, 1024), idesc, 1u);
             }
         }
         tc::mma_commit(tc::smem_addr(&bar[1]));
     }
 
-    // 5. unnormalised O to the workspace: warp w reads lane quadrant w % 4, columns half w / 4
+    // 5. unnormalised O to the workspace: tile mt, lane quadrant q (latent dims 128 mt + 32 q + lane)
     {
         if (!tc::mbar_wait(tc::smem_addr(&bar[1]), 0, kWaitLimit)) atomicOr(status, 2);
         __syncwarp();
         tc::fence_after_sync();
-        const int quad = warp & 3, half = warp >> 2;
-        const int head = (M == 128) ? quad * 32 + lane : (lane < 16 ? quad * 16 + lane : -1);
-        const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + half * 256;
+        const int quad = warp & 3;
 #pragma unroll 1
-        for (int cb = 0; cb < 8; cb++) {
-            uint32_t r[32];
-            tc::tmem_ld32(ta + cb * 32, r);
-            tc::tmem_wait_ld();
-            if (head >= 0 && head < n_heads) {
-                float4 *dst = reinterpret_cast<float4 *>(part_acc + (ml_base + head) * kLatent + half * 256 + cb * 32);
+        for (int mt = warp >> 2; mt < kLatent / 128; mt += 2) {
+            const int dim = mt * 128 + quad * 32 + lane;
+            const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + mt * M;
+#pragma unroll 1
+            for (int hb = 0; hb < M; hb += 32) {
+                uint32_t r[32];
+                tc::tmem_ld32(ta + hb, r);
+                tc::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 8; e++)
-                    dst[e] = make_float4(__uint_as_float(r[4 * e]), __uint_as_float(r[4 * e + 1]),
-                                         __uint_as_float(r[4 * e + 2]), __uint_as_float(r[4 * e + 3]));
+                for (int e = 0; e < 32; e++)
+                    if (hb + e < n_heads) part_acc[(ml_base + hb + e) * kLatent + dim] = __uint_as_float(r[e]);
             }
         }
     }
@@ -259,15 +290,13 @@ cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache,
         const int smem = TcLayout<64>::kBytes;
         e = cudaFuncSetAttribute(mla_split_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        mla_split_tc_kernel<64><<<grid, kTcThreads, smem, stream>>>(
-            static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
+        launch_pdl(mla_split_tc_kernel<64>, dim3(grid), dim3(kTcThreads), smem, stream, static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
             part_acc, part_ml, status);
     } else {
         const int smem = TcLayout<128>::kBytes;
         e = cudaFuncSetAttribute(mla_split_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        mla_split_tc_kernel<128><<<grid, kTcThreads, smem, stream>>>(
-            static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
+        launch_pdl(mla_split_tc_kernel<128>, dim3(grid), dim3(kTcThreads), smem, stream, static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
             part_acc, part_ml, status);
     }
     return cudaGetLastError();

@@ -14,6 +14,7 @@ __global__ void __launch_bounds__(256) store_int8_kernel(const uint16_t *__restr
                                                          const int64_t *__restrict__ slots,
                                                          int64_t n, int8_t *__restrict__ cache,
                                                          int64_t n_rows) {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     for (int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -59,8 +60,8 @@ cudaError_t launch_store_int8(const void *latent, const int64_t *slots, int64_t 
     int64_t blocks = (n + warps_per_block - 1) / warps_per_block;
     int64_t cap = static_cast<int64_t>(num_sms) * 16;
     if (blocks > cap) blocks = cap;
-    store_int8_kernel<<<static_cast<unsigned>(blocks), 32 * warps_per_block, 0, stream>>>(
-        static_cast<const uint16_t *>(latent), slots, n, cache, n_rows);
+    launch_pdl(store_int8_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * warps_per_block), 0, stream,
+               static_cast<const uint16_t *>(latent), slots, n, cache, n_rows);
     return cudaGetLastError();
 }
 

@@ -28,6 +28,29 @@ __device__ __forceinline__ uint64_t desc(uint32_t saddr, uint32_t lbo_bytes, uin
     return d;                              // base offset 0, legacy LBO mode, layout SWIZZLE_NONE
 }
 
+// Descriptor of a K-major operand in the 128-byte swizzle layout: rows of 128 bytes (64 bf16
+// elements of K), 16-byte chunks of row r stored at chunk position (chunk ^ (r % 8)), 8-row groups
+// sbo_bytes apart; the atom base must be 1024-byte aligned (advancing the start inside a row by
+// k * 32 bytes selects the K = 16 slice k).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr, uint32_t sbo_bytes) {
+    uint64_t d = static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1) << 16;  // leading byte offset (unused for swizzled K-major)
+    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
+    return d;
+}
+
+// 1-D bulk copy global -> shared completing on an mbarrier (16-byte aligned, size % 16 == 0).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst_smem, const void *src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst_smem),
+                 "l"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t mbar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(mbar), "r"(bytes) : "memory");
+}
+
 // Instruction descriptor of kind::f16 with bf16 A and B and an fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major, bool b_mn_major) {
     return (1u << 4)                                   // D format: f32
@@ -101,6 +124,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t mbar, uint32_t parity) {
         : "r"(mbar), "r"(parity)
         : "memory");
     return ok != 0;
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t mbar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(mbar) : "memory");
 }
 // Bounded wait: gives up after `limit` polls (each poll may itself block for a while in hardware)
 // and returns false, so that a kernel never spins forever.

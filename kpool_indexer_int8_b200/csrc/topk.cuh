@@ -28,11 +28,17 @@ __device__ __forceinline__ void hist_add(unsigned *hist, uint32_t digit) {
     if (digit != 0xffffffffu && (threadIdx.x & 31) == __ffs(peers) - 1) atomicAdd(&hist[digit], __popc(peers));
 }
 
+// Workspace of a selection, per query: the histogram (kHistBins uint32) and four uint32
+// counters (list A size, list B size, finished CTAs) -- both zeroed before each selection --,
+// list A (kMaxSelect uint64 composites) and list B (ld uint64 composites).
 size_t topk_select_smem();
+cudaError_t launch_zero(void *p, size_t bytes, cudaStream_t stream);   // p 16-byte aligned
+int topk_collect_ctas(int64_t ld);
 cudaError_t launch_topk_hist(const float *scores, const NvisSource &src, int n_q, unsigned *ghist,
                              cudaStream_t stream);
-cudaError_t launch_topk_select(const float *scores, const NvisSource &src, const unsigned *ghist,
-                               int n_q, int select_k, int32_t *topk, int32_t *n_sel,
-                               cudaStream_t stream);
+cudaError_t launch_topk_collect(const float *scores, const NvisSource &src, const unsigned *ghist,
+                                unsigned *counters, unsigned long long *alist,
+                                unsigned long long *blist, int n_q, int select_k, int32_t *topk,
+                                int32_t *n_sel, cudaStream_t stream);
 
 }  // namespace glm

@@ -204,11 +204,18 @@ def _topk_given(cuda, scores32, n_vis, S):
 @pytest.mark.parametrize("n,S,ties", [(0, 8, False), (5, 8, False), (8, 8, False), (300, 16, False),
                                       (300, 16, True), (5000, 512, True), (5000, 1, True),
                                       (4100, 2048, False), (65536, 512, False), (65536, 512, True),
-                                      (100000, 2048, True)])
+                                      (100000, 2048, True), (65536, 512, "uniform"),
+                                      (65536, 512, "equal"), (70000, 2048, "uniform")])
 def test_topk_bit_exact_on_oracle_scores(cuda, n, S, ties):
+    # "uniform" puts ~8000 scores in the boundary bin of the 11-bit histogram (the path that selects
+    # from the global list); "equal" leaves only the pool ids to decide
     rng = np.random.default_rng(n + S)
     s = rng.standard_normal(max(n, 1)) * 20 + 60
-    if ties:
+    if ties == "uniform":
+        s = rng.random(max(n, 1))
+    elif ties == "equal":
+        s = np.full(max(n, 1), 3.5)
+    elif ties:
         s = np.round(s * 4) / 4                        # heavy ties
         s[rng.random(s.shape) < 0.05] = 0.0
         s[rng.random(s.shape) < 0.05] = -0.0
