@@ -23,6 +23,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import subprocess
 import sys
 import threading
@@ -35,7 +36,7 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-KERNEL_LAUNCHES_PER_STEP = 7   # store, kpool, scores, top-k, expand, MLA split, MLA combine
+KERNEL_LAUNCHES_PER_STEP = 8   # store, kpool, zero, scores, top-k, expand, MLA split, MLA combine
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -73,8 +74,23 @@ def measured_peaks():
 
 
 def kernel_source_sha(name: str) -> str:
-    path = os.path.join(ROOT, "kpool_indexer_int8_b200", "csrc", name)
-    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    """Hash of a kernel source file and of every local header it includes (recursively), so that
+    a recorded counter goes stale when anything compiled into the kernel changes."""
+    csrc = os.path.join(ROOT, "kpool_indexer_int8_b200", "csrc")
+    h = hashlib.sha256()
+    seen, todo = set(), [name]
+    while todo:
+        f = todo.pop(0)
+        if f in seen:
+            continue
+        seen.add(f)
+        path = os.path.join(csrc, f)
+        if not os.path.exists(path):
+            path = os.path.join(ROOT, "include", f)
+        text = open(path, "rb").read()
+        h.update(f.encode() + b"\0" + text)
+        todo += re.findall(r'#include "([^"]+)"', text.decode())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel_file: str, workload: str):
@@ -403,7 +419,7 @@ def run_kernels(args, wl):
     peak, peak_kind = measured_peaks()
     idx_ms = stage_ms["index_scores"]
     achieved = ab["index"] / (idx_ms / 1e3) / 1e9
-    traffic = recorded_traffic("index_scores.cu", wl.name)
+    traffic = recorded_traffic("index_scores_tc.cu", wl.name)
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
