@@ -6,6 +6,7 @@
  *   glm_kpool_build        -> k_norm LayerNorm + slot-axis softmax pooling into fp32 pooled keys
  *   glm_index_scores_topk  -> relu head-weighted index scores and the top select_k pools
  *   glm_expand_selection   -> token indices (+ cache rows), visible tail, -1 padding
+ *   (glm_index_topk_expand -> the two above in one launch)
  *   glm_sparse_mla_decode  -> sparse NoPE MLA over the gathered int8 rows (split-KV + combine)
  *
  * Conventions for every entry point
@@ -137,8 +138,9 @@ int glm_kpool_build(const glm_dsa_dims *dims, const void *k_dev, const void *gat
  *   topk_dev    int32 [n_q, select_k]      n_sel_dev  int32 [n_q] or NULL
  *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, ...), 256-byte
  *               aligned (required even when scores_dev is given; contents on entry are ignored).
- *               Its last 256 bytes start with a status word set nonzero if a wait on the tensor
- *               cores gave up (never cleared by the library).
+ *               Its last 256 bytes start with a status word set nonzero if a wait gave up (on the
+ *               tensor cores, or of the CTAs of one query for one another); the outputs are then
+ *               invalid. The library never clears it.
  * 1 <= select_k <= 2048. The q . pooled products run on the tensor cores: each fp32 pooled key is
  * split exactly into three bf16 terms, so with the bf16 queries exact the dot products carry fp32
  * accumulation error only (relative error far below 1e-4); relu and the head weights in fp32.
@@ -148,6 +150,24 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx_dev, const
                           const int32_t *q_pos_dev, const int32_t *pad_dev, const int32_t *len_dev,
                           int32_t batch, int32_t n_q, int32_t select_k, float *scores_dev,
                           int32_t *topk_dev, int32_t *n_sel_dev, void *workspace_dev,
+                          size_t ws_bytes, void *stream);
+
+/*
+ * glm_index_scores_topk followed by glm_expand_selection, in one launch: the same scores, top-k
+ * row and n_sel, plus the expansion of the selection into token positions and cache rows
+ * ("Module glm5next_dsa_ref", expand_selection; the rules and arguments of glm_expand_selection:
+ * slot_map_dev int64 [batch, ld_slot] or NULL, tok_dev / rows_dev int32 [n_q, out_width], at
+ * least one of them non-NULL, out_width >= 4 * select_k + 3). Every output equals what the two
+ * separate calls produce. The workspace is that of GLM_OP_INDEX_SCORES_TOPK.
+ * When the selection of a query spans several CTAs they meet at a grid barrier (the launch is
+ * cooperative); a wait that gives up sets the status word nonzero and leaves the outputs invalid.
+ */
+int glm_index_topk_expand(const glm_dsa_dims *dims, const void *q_idx_dev, const float *w_dev,
+                          const float *pooled_dev, int64_t ld_pools, const int32_t *q_seq_dev,
+                          const int32_t *q_pos_dev, const int32_t *pad_dev, const int32_t *len_dev,
+                          int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map_dev,
+                          int64_t ld_slot, int32_t out_width, float *scores_dev, int32_t *topk_dev,
+                          int32_t *n_sel_dev, int32_t *tok_dev, int32_t *rows_dev, void *workspace_dev,
                           size_t ws_bytes, void *stream);
 
 /*

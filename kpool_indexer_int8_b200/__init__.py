@@ -33,7 +33,8 @@ GLM_OP_TOPK_POOLS = 2
 GLM_OP_SPARSE_MLA = 3
 
 EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv_store_int8",
-           "glm_kpool_build", "glm_index_scores", "glm_index_scores_topk", "glm_topk_pools", "glm_expand_selection",
+           "glm_kpool_build", "glm_index_scores", "glm_index_scores_topk", "glm_index_topk_expand",
+           "glm_topk_pools", "glm_expand_selection",
            "glm_sparse_mla_decode", "glm_dsa_workspace_size")
 
 
@@ -67,6 +68,9 @@ lib.glm_kpool_build.restype = C.c_int
 lib.glm_index_scores_topk.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32, _P, _P,
                                       _P, _P, _SZ, _P]
 lib.glm_index_scores_topk.restype = C.c_int
+lib.glm_index_topk_expand.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32, _P, _I64,
+                                      _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]
+lib.glm_index_topk_expand.restype = C.c_int
 lib.glm_index_scores.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P]
 lib.glm_index_scores.restype = C.c_int
 lib.glm_topk_pools.argtypes = [_P, _I64, _P, _I32, _I32, _P, _P, _P, _SZ, _P]
@@ -175,6 +179,29 @@ def glm_index_scores_topk(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, sel
                                      n_q, int(select_k), _ptr(scores), _ptr(topk), _ptr(n_sel),
                                      _ptr(workspace), ws_bytes, _stream(stream)),
            "glm_index_scores_topk")
+
+
+def glm_index_topk_expand(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, select_k, topk,
+                          out_width, n_sel=None, slot_map=None, tok=None, rows=None, scores=None,
+                          workspace=None, stream=None) -> None:
+    """glm_index_scores_topk and glm_expand_selection in one launch: the arguments of both
+    (tok / rows int32 [n_q, out_width], at least one; slot_map int64 [B, ld_slot] or None)."""
+    for t, dt, nm in ((q_idx, torch.bfloat16, "q_idx"), (w, torch.float32, "w"),
+                      (pooled, torch.float32, "pooled"), (q_seq, torch.int32, "q_seq"),
+                      (q_pos, torch.int32, "q_pos"), (pad, torch.int32, "pad"),
+                      (length, torch.int32, "len"), (topk, torch.int32, "topk"),
+                      (n_sel, torch.int32, "n_sel"), (slot_map, torch.int64, "slot_map"),
+                      (tok, torch.int32, "tok"), (rows, torch.int32, "rows"),
+                      (scores, torch.float32, "scores"), (workspace, torch.uint8, "workspace")):
+        _dev(t, dt, nm)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    ld_slot = 0 if slot_map is None else slot_map.shape[1]
+    _check(lib.glm_index_topk_expand(C.byref(dims), _ptr(q_idx), _ptr(w), _ptr(pooled), pooled.shape[1],
+                                     _ptr(q_seq), _ptr(q_pos), _ptr(pad), _ptr(length), pad.shape[0],
+                                     q_idx.shape[0], int(select_k), _ptr(slot_map), ld_slot,
+                                     int(out_width), _ptr(scores), _ptr(topk), _ptr(n_sel), _ptr(tok),
+                                     _ptr(rows), _ptr(workspace), ws_bytes, _stream(stream)),
+           "glm_index_topk_expand")
 
 
 def glm_index_scores(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, scores, stream=None) -> None:

@@ -4,6 +4,7 @@
 
 #include "common.cuh"
 #include "kernels.cuh"
+#include "select.cuh"
 
 namespace {
 
@@ -25,32 +26,42 @@ int num_sms() {
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Workspace of a selection (first in the workspace of both selection entry points): per query a
-// 2048-bin histogram of score keys and 4 counters (zeroed by one memset before each selection),
-// then list A (select_k-bound candidates above the boundary bin) and list B (the boundary bin).
+// Workspace of a selection (first in the workspace of both selection entry points): per query
+// two 2048-bin histograms of score keys and kCntWords counters (zeroed by one kernel before a
+// selection that spans several CTAs), the list sizes of each CTA, and the per-CTA regions of
+// list A (candidates above the boundary bin) and list B (the boundary bin).
 struct SelWs {
     unsigned *hist;
+    unsigned *hist2;
     unsigned *counters;
+    unsigned *words;
     unsigned long long *alist;
     unsigned long long *blist;
     size_t zero_bytes;
 };
-size_t sel_zero_bytes(int n_q) { return static_cast<size_t>(n_q) * (glm::kHistBins + 4) * sizeof(unsigned); }
+size_t sel_zero_bytes(int n_q) {
+    return static_cast<size_t>(n_q) * (2 * glm::kHistBins + glm::kCntWords) * sizeof(unsigned);
+}
+size_t sel_list_bytes(int n_q, int64_t ld) {
+    return align_up(static_cast<size_t>(n_q) * static_cast<size_t>(glm::sel_list_cap(ld)) *
+                    sizeof(unsigned long long), 256);
+}
+size_t sel_words_bytes(int n_q) { return align_up(static_cast<size_t>(n_q) * glm::kMaxSelCtas * sizeof(unsigned), 256); }
 size_t sel_bytes(int n_q, int64_t ld) {
-    const size_t ldb = static_cast<size_t>(ld > 0 ? ld : 1);
-    return align_up(sel_zero_bytes(n_q), 256) +
-           align_up(static_cast<size_t>(n_q) * glm::kMaxSelect * sizeof(unsigned long long), 256) +
-           align_up(static_cast<size_t>(n_q) * ldb * sizeof(unsigned long long), 256);
+    return align_up(sel_zero_bytes(n_q), 256) + sel_words_bytes(n_q) + 2 * sel_list_bytes(n_q, ld);
 }
 SelWs sel_layout(void *base, int n_q, int64_t ld) {
     char *p = static_cast<char *>(base);
     SelWs w;
     w.hist = reinterpret_cast<unsigned *>(p);
-    w.counters = w.hist + static_cast<size_t>(n_q) * glm::kHistBins;
+    w.hist2 = w.hist + static_cast<size_t>(n_q) * glm::kHistBins;
+    w.counters = w.hist2 + static_cast<size_t>(n_q) * glm::kHistBins;
     w.zero_bytes = sel_zero_bytes(n_q);
     p += align_up(w.zero_bytes, 256);
+    w.words = reinterpret_cast<unsigned *>(p);
+    p += sel_words_bytes(n_q);
     w.alist = reinterpret_cast<unsigned long long *>(p);
-    p += align_up(static_cast<size_t>(n_q) * glm::kMaxSelect * sizeof(unsigned long long), 256);
+    p += sel_list_bytes(n_q, ld);
     w.blist = reinterpret_cast<unsigned long long *>(p);
     return w;
 }
@@ -148,12 +159,13 @@ size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
     }
 }
 
-int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const float *w,
-                          const float *pooled, int64_t ld_pools, const int32_t *q_seq,
-                          const int32_t *q_pos, const int32_t *pad, const int32_t *len,
-                          int32_t batch, int32_t n_q, int32_t select_k, float *scores,
-                          int32_t *topk, int32_t *n_sel, void *workspace, size_t ws_bytes,
-                          void *stream) {
+namespace {
+
+// Checks shared by the two scoring + selection entry points; GLM_OK when the call may proceed.
+int check_index_args(const glm_dsa_dims *dims, const void *q_idx, const float *w, const float *pooled,
+                     int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad,
+                     const int32_t *len, int32_t batch, int32_t n_q, int32_t select_k, const float *scores,
+                     const int32_t *topk, const int32_t *n_sel) {
     int rc = glm_check_dims(dims);
     if (rc != GLM_OK) return rc;
     if (n_q < 0 || batch < 0 || ld_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect ||
@@ -166,6 +178,17 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const flo
         !aligned(q_seq, 4) || !aligned(q_pos, 4) || !aligned(pad, 4) || !aligned(len, 4) ||
         !aligned(topk, 4) || (n_sel && !aligned(n_sel, 4)) || (scores && !aligned(scores, 4)))
         return GLM_ERR_INVALID_ARG;
+    return GLM_OK;
+}
+
+// Scores + selection (+ expansion when tok or rows is given) in one fused launch, preceded by
+// the zeroing of the multi-CTA words when the selection spans several CTAs.
+int run_index_select(const glm_dsa_dims *dims, const void *q_idx, const float *w, const float *pooled,
+                     int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad,
+                     const int32_t *len, int32_t batch, int32_t n_q, int32_t select_k,
+                     const int64_t *slot_map, int64_t ld_slot, int32_t out_width, float *scores,
+                     int32_t *topk, int32_t *n_sel, int32_t *tok, int32_t *rows, void *workspace,
+                     size_t ws_bytes, void *stream) {
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, n_q, ld_pools, select_k, 0);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
     const SelWs sw = sel_layout(workspace, n_q, ld_pools);
@@ -173,17 +196,66 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const flo
     float *sbuf = scores ? scores : reinterpret_cast<float *>(ws + sel_bytes(n_q, ld_pools));
     int *status = reinterpret_cast<int *>(ws + need - 256);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const glm::NvisSource src{nullptr, q_seq, q_pos, pad, len, batch, ld_pools};
-    rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
-    if (rc != GLM_OK) return rc;
-    if (ld_pools > 0) {
-        rc = cuda_status(glm::launch_index_scores_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len,
-                                                     batch, n_q, sbuf, sw.hist, scores != nullptr, status,
-                                                     num_sms(), st));
+    const int sms = num_sms();
+    if (glm::index_select_ctas(n_q, ld_pools, sms) > 1) {
+        const int rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
         if (rc != GLM_OK) return rc;
     }
-    return cuda_status(glm::launch_topk_collect(sbuf, src, sw.hist, sw.counters, sw.alist, sw.blist, n_q,
-                                                select_k, topk, n_sel, st));
+    glm::IxSelectArgs sel{};
+    sel.select_k = select_k;
+    sel.topk = topk;
+    sel.n_sel = n_sel;
+    sel.ghist = sw.hist;
+    sel.ghist2 = sw.hist2;
+    sel.counters = sw.counters;
+    sel.words = sw.words;
+    sel.alist = sw.alist;
+    sel.blist = sw.blist;
+    sel.list_cap = glm::sel_list_cap(ld_pools);
+    sel.slot_map = slot_map;
+    sel.ld_slot = ld_slot;
+    sel.out_width = out_width;
+    sel.tok = tok;
+    sel.rows = rows;
+    return cuda_status(glm::launch_index_select_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch,
+                                                   n_q, sbuf, scores != nullptr, sel, status, sms, st));
+}
+
+}  // namespace
+
+int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const float *w,
+                          const float *pooled, int64_t ld_pools, const int32_t *q_seq,
+                          const int32_t *q_pos, const int32_t *pad, const int32_t *len,
+                          int32_t batch, int32_t n_q, int32_t select_k, float *scores,
+                          int32_t *topk, int32_t *n_sel, void *workspace, size_t ws_bytes,
+                          void *stream) {
+    int rc = check_index_args(dims, q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
+                              scores, topk, n_sel);
+    if (rc != GLM_OK || n_q == 0) return rc;
+    return run_index_select(dims, q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
+                            nullptr, 0, 0, scores, topk, n_sel, nullptr, nullptr, workspace, ws_bytes, stream);
+}
+
+int glm_index_topk_expand(const glm_dsa_dims *dims, const void *q_idx, const float *w,
+                          const float *pooled, int64_t ld_pools, const int32_t *q_seq,
+                          const int32_t *q_pos, const int32_t *pad, const int32_t *len,
+                          int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map,
+                          int64_t ld_slot, int32_t out_width, float *scores, int32_t *topk,
+                          int32_t *n_sel, int32_t *tok, int32_t *rows, void *workspace,
+                          size_t ws_bytes, void *stream) {
+    int rc = check_index_args(dims, q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
+                              scores, topk, n_sel);
+    if (rc != GLM_OK) return rc;
+    if (out_width < 1 || ld_slot < 0) return GLM_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(out_width) < static_cast<int64_t>(glm::kKpool) * select_k + glm::kKpool - 1)
+        return GLM_ERR_INVALID_ARG;  // the largest selection plus a full tail must fit
+    if (n_q == 0) return GLM_OK;
+    if (!tok && !rows) return GLM_ERR_INVALID_ARG;
+    if ((slot_map && !aligned(slot_map, 8)) || (tok && !aligned(tok, 4)) || (rows && !aligned(rows, 4)))
+        return GLM_ERR_INVALID_ARG;
+    return run_index_select(dims, q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
+                            slot_map, ld_slot, out_width, scores, topk, n_sel, tok, rows, workspace, ws_bytes,
+                            stream);
 }
 
 int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w,
@@ -200,8 +272,9 @@ int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w
     if (!aligned(q_idx, 16) || !aligned(w, 4) || !aligned(pooled, 16) || !aligned(q_seq, 4) ||
         !aligned(q_pos, 4) || !aligned(pad, 4) || !aligned(len, 4) || !aligned(scores, 4))
         return GLM_ERR_INVALID_ARG;
-    return cuda_status(glm::launch_index_scores_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len,
-                                                   batch, n_q, scores, nullptr, true, nullptr, num_sms(),
+    const glm::IxSelectArgs none{};   // topk == nullptr: scores only
+    return cuda_status(glm::launch_index_select_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len,
+                                                   batch, n_q, scores, true, none, nullptr, num_sms(),
                                                    static_cast<cudaStream_t>(stream)));
 }
 
@@ -224,8 +297,8 @@ int glm_topk_pools(const float *scores, int64_t ld_scores, const int32_t *n_visi
     if (rc != GLM_OK) return rc;
     rc = cuda_status(glm::launch_topk_hist(scores, src, n_q, sw.hist, st));
     if (rc != GLM_OK) return rc;
-    return cuda_status(glm::launch_topk_collect(scores, src, sw.hist, sw.counters, sw.alist, sw.blist, n_q,
-                                                select_k, topk, n_sel, st));
+    return cuda_status(glm::launch_topk_collect(scores, src, sw.hist, sw.hist2, sw.counters, sw.words, sw.alist,
+                                                sw.blist, n_q, select_k, topk, n_sel, st));
 }
 
 int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk, const int32_t *n_sel,

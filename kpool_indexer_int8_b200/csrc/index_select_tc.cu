@@ -1,10 +1,11 @@
-// index_scores_tc.cu -- relu head-weighted index scores on the sm_100a tensor cores
-// ("Module glm5next_dsa_ref", index_scores: the matmul -> relu -> head-weighted sum chain;
-// "GLM-5.3-Flash" pypto-lib page, 'Checkpoint shape': indexer 32 heads x 128):
+// index_select_tc.cu -- relu head-weighted index scores on the sm_100a tensor cores, fused with
+// the top-k pool selection and its expansion into token indices and cache rows
+// ("Module glm5next_dsa_ref": index_scores -- matmul -> relu -> head-weighted sum --, topk_pools
+// and expand_selection; "GLM-5.3-Flash" pypto-lib page, 'Checkpoint shape': indexer 32 heads x 128):
 //     score[n][p] = sum_h w[n][h] * max(0, sum_d q_idx[n][h][d] * pooled[b][p][d])
 //
-// Decode form: grid (G, n_q), G ~ SMs / n_q; CTA g of query n owns a contiguous range of the
-// query's visible pools. Warp-specialised pipeline, every hand-off an mbarrier:
+// Grid (G, n_q): CTA g of query n owns a contiguous range of the query's visible pools.
+// Phase 1, scoring -- a warp-specialised pipeline, every hand-off an mbarrier:
 //   * producer (warp 0): 1-D bulk copies of 32 pools (16 KB, contiguous) into 4 staging slots;
 //   * converters (warps 8-15): split each fp32 value x exactly into three bf16 terms
 //     (hi = rn(x), mid = rn(x - hi), lo = rn(x - hi - mid)) written as K-major tiles of 64 pools in
@@ -13,11 +14,20 @@
 //   * MMA issuer (warp 1): per term 8 UMMAs (M = 64 pools, N = 32 heads, K = 16) into one of two
 //     fp32 tensor-memory accumulators; with the bf16 query exact, the three terms reproduce q . x
 //     to fp32 accumulation accuracy;
-//   * epilogue (warps 4-7, one TMEM lane quadrant each): relu and head weights, the score, and its
-//     top-11-bit key digit added to the selection histogram.
-// HBM-bound: 512 bytes of pooled key per pool; the tensor cores run at a few percent.
+//   * epilogue (warps 4-7, one TMEM lane quadrant each): relu and head weights, the score (to
+//     global memory and, when the range is short enough, to shared memory), and its top-11-bit
+//     key digit counted in the CTA's histogram.
+// Phase 2, selection (select.cuh): with G > 1 the CTA histograms are summed in global memory and
+// the G CTAs of a query meet at a grid barrier (the launch is cooperative, so all CTAs are
+// resident; the wait is bounded); every CTA then classifies its own scores against the boundary
+// bin, appends them to the query's global lists, and the last CTA to finish (ticket) completes
+// the selection, sorts it, and writes the top-k row, n_sel and the expanded token / row indices.
+// With G = 1 the one CTA does all of it on chip.
+// Phase 1 is HBM-bound: 512 bytes of pooled key per pool; the tensor cores run at a few percent.
 #include "common.cuh"
 #include "tc.cuh"
+#include "kernels.cuh"
+#include "select.cuh"
 #include "topk.cuh"
 
 namespace glm {
@@ -33,17 +43,24 @@ constexpr int kIxBufBytes = 3 * kIxTermBytes;          // three terms: 48 KB
 constexpr int kIxStageBytes = kIxChunk * kIdxDim * 4;  // 16 KB of fp32 pooled keys
 constexpr uint32_t kIxWaitLimit = 1u << 22;
 
+constexpr int kIxLocalCap = 4096;                      // scores of a CTA kept in shared memory
+
 struct IxLayout {                                      // offsets from a 1024-byte aligned base
     static constexpr int kTerms = 0;                                  // [2 buffers][3 terms][16 KB]
     static constexpr int kStage = kTerms + 2 * kIxBufBytes;           // [4 stages][16 KB]
     static constexpr int kQ = kStage + kIxStages * kIxStageBytes;     // 32 heads x 128 dims bf16
     static constexpr int kHist = kQ + kIdxHeads * kIdxDim * 2;        // 2048 uint32
-    static constexpr int kW = kHist + kHistBins * 4;                  // 32 fp32 head weights
+    static constexpr int kLocal = kHist + kHistBins * 4;              // kIxLocalCap fp32 scores
+    static constexpr int kW = kLocal + kIxLocalCap * 4;               // 32 fp32 head weights
     static constexpr int kBar = kW + kIdxHeads * 4;                   // 16 mbarriers
     static constexpr int kTmem = kBar + 16 * 8;
-    static constexpr int kBytes = kTmem + 16;
+    static constexpr int kFlag = kTmem + 16;
+    static constexpr int kBytes = kFlag + 16;
     static constexpr int kAlloc = kBytes + 1024;                      // room to align the base
 };
+// The selection's working set overlays the tile buffers and staging slots once scoring is over.
+static_assert(sizeof(SelShared) <= IxLayout::kQ, "selection working set must fit the scoring buffers");
+
 // mbarrier indices
 constexpr int kBarStFull = 0;     // [4] staging slot filled (producer, tx bytes)
 constexpr int kBarStEmpty = 4;    // [4] staging slot read (8 converter warps)
@@ -59,12 +76,47 @@ __device__ __forceinline__ uint32_t bf16_pair(float a, float b) {
 __device__ __forceinline__ float bf16_lo_f(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
 
-__global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
+// Write the outputs of a query whose selection is final (s.cand[0 .. count) sorted): the top-k
+// row, n_sel, and the expansion into tokens / cache rows (the rules of expand_selection).
+__device__ __forceinline__ void write_outputs(const IxSelectArgs &sel, int n, int b, bool valid_b, int pb,
+                                              int seq_len, int qp, unsigned count, const SelShared &s) {
+    write_selection(sel.topk + static_cast<int64_t>(n) * sel.select_k, sel.select_k, count, s);
+    if (threadIdx.x == 0 && sel.n_sel) sel.n_sel[n] = static_cast<int32_t>(count);
+    if (!sel.tok && !sel.rows) return;
+    const int64_t base = static_cast<int64_t>(n) * sel.out_width;
+    int nvx = 0, n_valid = 0, ns = 0;
+    if (valid_b) {
+        nvx = visible_pools(pb, seq_len, qp, 0x7fffffffll);   // uncapped, as the expansion defines it
+        ns = min(static_cast<int>(count), nvx);
+        const int last = min(qp, pb + seq_len - 1);            // the tail stops at the query or the end
+        const int tail = max(0, last - (pb + kKpool * nvx) + 1);
+        n_valid = kKpool * ns + tail;
+    }
+    for (int j = threadIdx.x; j < sel.out_width; j += blockDim.x) {
+        int t = GLM_INVALID;
+        if (j < kKpool * ns) t = pb + kKpool * id_of(s.cand[j / kKpool]) + (j % kKpool);
+        else if (j < n_valid) t = pb + kKpool * nvx + (j - kKpool * ns);
+        if (sel.tok) sel.tok[base + j] = t;
+        if (sel.rows) {
+            int r = t;
+            if (sel.slot_map) {
+                r = GLM_INVALID;
+                if (t >= 0 && t < sel.ld_slot) {
+                    const int64_t v = sel.slot_map[static_cast<int64_t>(b) * sel.ld_slot + t];
+                    r = (v >= 0 && v <= 0x7fffffffll) ? static_cast<int>(v) : GLM_INVALID;
+                }
+            }
+            sel.rows[base + j] = r;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kIxThreads, 1) index_select_tc_kernel(
     const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
     const float *__restrict__ pooled, int64_t ld_pools, const int32_t *__restrict__ q_seq,
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ pad,
-    const int32_t *__restrict__ len, int batch, float *__restrict__ scores,
-    unsigned *__restrict__ ghist, int fill_invisible, int *__restrict__ status) {
+    const int32_t *__restrict__ len, int batch, float *__restrict__ scores, int fill_invisible,
+    IxSelectArgs sel, int *__restrict__ status) {
     pdl_begin();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
@@ -72,14 +124,21 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
     unsigned char *stage = smem + IxLayout::kStage;
     unsigned char *Qs = smem + IxLayout::kQ;
     unsigned *hist = reinterpret_cast<unsigned *>(smem + IxLayout::kHist);
+    float *sloc = reinterpret_cast<float *>(smem + IxLayout::kLocal);
     float *ws = reinterpret_cast<float *>(smem + IxLayout::kW);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + IxLayout::kTmem);
+    unsigned *flag = reinterpret_cast<unsigned *>(smem + IxLayout::kFlag);
 
     const int n = blockIdx.y, g = blockIdx.x, G = gridDim.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int b = q_seq[n];
-    const int n_vis = (b >= 0 && b < batch) ? visible_pools(pad[b], len[b], q_pos[n], ld_pools) : 0;
+    const bool valid_b = b >= 0 && b < batch;
+    const int pb = valid_b ? pad[b] : 0, seq_len = valid_b ? len[b] : 0, qp = q_pos[n];
+    const int n_vis = valid_b ? visible_pools(pb, seq_len, qp, ld_pools) : 0;
     float *srow = scores + static_cast<int64_t>(n) * ld_pools;
+    const bool select = sel.topk != nullptr;
+    const bool multi = select && G > 1;
+    SelShared &s = *reinterpret_cast<SelShared *>(terms);
 
     if (fill_invisible) {  // entries past the visible pools are -inf (split over the CTAs)
         const int64_t rest = ld_pools - n_vis;
@@ -88,11 +147,16 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
         const int64_t f1 = min(f0 + share, ld_pools);
         for (int64_t i = f0 + tid; i < f1; i += kIxThreads) srow[i] = -INFINITY;
     }
+    if (n_vis == 0) {   // nothing to score or select: CTA 0 writes the empty outputs
+        if (select && g == 0) write_outputs(sel, n, b, valid_b, pb, seq_len, qp, 0u, s);
+        return;
+    }
     int per = (n_vis + G - 1) / G;
     if (per < kIxTile) per = kIxTile;
-    const int lo = g * per;
+    const int lo = min(n_vis, g * per);
     const int hi = min(n_vis, lo + per);
-    if (lo >= hi) return;
+    const bool keep_local = select && per <= kIxLocalCap;
+    if (lo < hi) {
     const int n_chunks = (hi - lo + kIxChunk - 1) / kIxChunk;
     const int n_tiles = (hi - lo + kIxTile - 1) / kIxTile;
     const float *src = pooled + (static_cast<int64_t>(b) * ld_pools + lo) * kIdxDim;
@@ -121,7 +185,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
             __ldg(reinterpret_cast<const uint4 *>(qn) + i);
     }
     if (tid < kIdxHeads) ws[tid] = w[static_cast<int64_t>(n) * kIdxHeads + tid];
-    if (ghist)
+    if (select)
         for (int i = tid; i < kHistBins; i += kIxThreads) hist[i] = 0;
     tc::fence_proxy_async();
     __syncthreads();
@@ -182,13 +246,14 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
             const int p = lo + t * kIxTile + qd * 16 + lane;
             uint32_t digit = 0xffffffffu;
             if (lane < 16 && p < hi) {
-                float s = 0.0f;
+                float sc = 0.0f;
 #pragma unroll
-                for (int h2 = 0; h2 < kIdxHeads; h2++) s = fmaf(ws[h2], fmaxf(__uint_as_float(r[h2]), 0.0f), s);
-                srow[p] = s;
-                digit = score_key(s) >> (32 - kHistBitsTop);
+                for (int h2 = 0; h2 < kIdxHeads; h2++) sc = fmaf(ws[h2], fmaxf(__uint_as_float(r[h2]), 0.0f), sc);
+                srow[p] = sc;
+                if (keep_local) sloc[p - lo] = sc;
+                digit = score_key(sc) >> (32 - kHistBitsTop);
             }
-            if (ghist) hist_add(hist, digit);
+            if (select && digit != 0xffffffffu) atomicAdd(&hist[digit], 1u);
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(kBarAccEmpty + tb));
@@ -235,33 +300,104 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_scores_tc_kernel(
     if (!ok && status) atomicOr(status, 4);
     tc::fence_before_sync();
     __syncthreads();
-    if (ghist) {
-        unsigned *gh = ghist + static_cast<int64_t>(n) * kHistBins;
-        for (int i = tid; i < kHistBins; i += kIxThreads)
-            if (hist[i]) atomicAdd(&gh[i], hist[i]);
-    }
     if (warp == 0) {
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 64);
     }
+    if (multi) {   // this CTA's histogram into the query's
+        unsigned *gh = sel.ghist + static_cast<int64_t>(n) * kHistBins;
+        for (int i = tid; i < kHistBins; i += kIxThreads)
+            if (hist[i]) atomicAdd(&gh[i], hist[i]);
+    }
+    }   // lo < hi
+    if (!select) return;
+
+    // ---------------- phase 2: selection (every MMA and bulk copy of this CTA has completed) ----------------
+    unsigned *cnt = sel.counters + static_cast<int64_t>(n) * kCntWords;
+    if (multi) {   // grid barrier of the query's CTAs, then the summed histogram
+        __syncthreads();
+        if (tid == 0) {   // release this CTA's histogram, arrive, wait (acquire) for the others
+            __threadfence();
+            atomicAdd(&cnt[kCntArrive], 1u);
+            uint32_t it = 0;
+            while (ld_acquire(&cnt[kCntArrive]) < static_cast<unsigned>(G) && ++it < kSelWaitLimit) __nanosleep(64);
+            *flag = it >= kSelWaitLimit;
+            if (*flag && status) atomicOr(status, 8);
+        }
+        __syncthreads();
+        if (*flag) return;   // gave up waiting: the status word reports it
+        const uint4 *gh = reinterpret_cast<const uint4 *>(sel.ghist + static_cast<int64_t>(n) * kHistBins);
+        for (int i = tid; i < kHistBins / 4; i += kIxThreads) reinterpret_cast<uint4 *>(hist)[i] = __ldcg(gh + i);
+        __syncthreads();
+    }
+    const unsigned count = static_cast<unsigned>(min(sel.select_k, n_vis));
+    int bstar = -1;   // every visible pool is selected
+    if (n_vis > sel.select_k) {
+        block_find_bin(hist, static_cast<unsigned>(sel.select_k), s);
+        bstar = static_cast<int>(s.bin);
+    }
+    if (tid == 0) { s.n_a = 0; s.n_b = 0; }
+    if (!multi)
+        for (int i = tid; i < kHistBins; i += kIxThreads) s.hist2[i] = 0;
+    __syncthreads();
+    unsigned *h2 = multi ? sel.ghist2 + static_cast<int64_t>(n) * kHistBins : s.hist2;
+    auto score_at = [&](int i) { return keep_local ? sloc[i - lo] : __ldcg(srow + i); };
+    classify_range(score_at, lo, hi, bstar, h2, s);   // lo = 0, hi = n_vis when G = 1
+    __syncthreads();
+    if (sel.rows && sel.slot_map) {   // warm L2 with the slot-map lines the expansion may read
+        const unsigned la = min(s.n_a, static_cast<unsigned>(kMaxSelect));
+        const unsigned lb = min(s.n_b, static_cast<unsigned>(kBoundCap));
+        for (unsigned i = tid; i < la + lb; i += kIxThreads) {
+            const int p = id_of(i < la ? s.cand[i] : s.bnd[i - la]);
+            const long long t0 = pb + static_cast<long long>(kKpool) * p;
+            if (t0 >= 0 && t0 + kKpool <= sel.ld_slot)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(sel.slot_map + static_cast<int64_t>(b) * sel.ld_slot + t0));
+        }
+    }
+    unsigned nA, nB;
+    bool b_complete;
+    if (multi) {
+        if (!merge_lists_multi(cnt, sel.words + static_cast<int64_t>(n) * kMaxSelCtas,
+                               sel.alist + static_cast<int64_t>(n) * sel.list_cap,
+                               sel.blist + static_cast<int64_t>(n) * sel.list_cap, per,
+                               sel.ghist2 + static_cast<int64_t>(n) * kHistBins, G, nA, nB, b_complete, s))
+            return;
+    } else {
+        nA = min(s.n_a, static_cast<unsigned>(kMaxSelect));
+        nB = s.n_b;
+        b_complete = nB <= static_cast<unsigned>(kBoundCap);
+    }
+    const unsigned long long top = static_cast<unsigned long long>(bstar < 0 ? 0 : bstar);
+    auto get_b = [&](int i) -> unsigned long long {   // list B straight from the scores
+        const uint32_t key = score_key(__ldcg(srow + i));
+        return (key >> (32 - kHistBitsTop)) == top ? compose(key, i) : 0ull;
+    };
+    finish_selection(count, nA, nB, b_complete, bstar, s.hist2, get_b, n_vis, s);
+    write_outputs(sel, n, b, valid_b, pb, seq_len, qp, count, s);
 }
 
-cudaError_t launch_index_scores_tc(const void *q_idx, const float *w, const float *pooled,
-                                   int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
-                                   const int32_t *pad, const int32_t *len, int batch, int n_q,
-                                   float *scores, unsigned *ghist, bool fill_invisible, int *status,
-                                   int num_sms, cudaStream_t stream) {
-    int G = (num_sms + n_q - 1) / n_q;
+int index_select_ctas(int n_q, int64_t ld_pools, int num_sms) {
+    int G = num_sms / n_q;   // every CTA resident at once (one per SM): the selection's grid barrier
     if (G < 1) G = 1;
     const int64_t max_tiles = (ld_pools + kIxTile - 1) / kIxTile;
     if (G > max_tiles) G = static_cast<int>(max_tiles > 0 ? max_tiles : 1);
+    return G;
+}
+
+cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const float *pooled,
+                                   int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
+                                   const int32_t *pad, const int32_t *len, int batch, int n_q,
+                                   float *scores, bool fill_invisible, const IxSelectArgs &sel,
+                                   int *status, int num_sms, cudaStream_t stream) {
+    const int G = index_select_ctas(n_q, ld_pools, num_sms);
     const int smem = IxLayout::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(index_scores_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(index_select_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    dim3 grid(G, n_q);
-    launch_pdl(index_scores_tc_kernel, dim3(grid), dim3(kIxThreads), smem, stream, static_cast<const uint16_t *>(q_idx), w, pooled, ld_pools, q_seq, q_pos, pad, len, batch,
-        scores, ghist, fill_invisible ? 1 : 0, status);
-    return cudaGetLastError();
+    const bool coop = sel.topk != nullptr && G > 1;
+    e = launch_pdl_coop(index_select_tc_kernel, dim3(G, n_q), dim3(kIxThreads), smem, stream, coop,
+                        static_cast<const uint16_t *>(q_idx), w, pooled, ld_pools, q_seq, q_pos, pad, len,
+                        batch, scores, fill_invisible ? 1 : 0, sel, status);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 }  // namespace glm

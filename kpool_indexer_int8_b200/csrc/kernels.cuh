@@ -16,11 +16,32 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
                                const int32_t *pad, const int32_t *len, const int32_t *pool_begin,
                                int batch, int max_new_pools, float *pooled, int64_t ld_pools,
                                int32_t *n_pools, cudaStream_t stream, int num_sms);
-cudaError_t launch_index_scores_tc(const void *q_idx, const float *w, const float *pooled,
+// Selection and expansion arguments of the fused index kernel; topk == nullptr: scores only.
+// The multi-CTA words (ghist, ghist2, counters: 2 kHistBins + kCntWords uint32 per query) must
+// be zero at launch when index_select_ctas() > 1.
+struct IxSelectArgs {
+    int select_k;
+    int32_t *topk;                 // [n_q][select_k]
+    int32_t *n_sel;                // [n_q] or null
+    unsigned *ghist;               // [n_q][kHistBins] level-1 histograms
+    unsigned *ghist2;              // [n_q][kHistBins] level-2 histograms
+    unsigned *counters;            // [n_q][kCntWords]
+    unsigned *words;               // [n_q][kMaxSelCtas] list sizes of each CTA
+    unsigned long long *alist;     // [n_q][list_cap] per-CTA regions of list A
+    unsigned long long *blist;     // [n_q][list_cap] per-CTA regions of list B
+    long long list_cap;            // sel_list_cap(ld_pools)
+    const int64_t *slot_map;       // expansion: [batch][ld_slot] or null
+    long long ld_slot;
+    int out_width;
+    int32_t *tok;                  // [n_q][out_width] or null
+    int32_t *rows;                 // [n_q][out_width] or null
+};
+int index_select_ctas(int n_q, int64_t ld_pools, int num_sms);
+cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const float *pooled,
                                    int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
                                    const int32_t *pad, const int32_t *len, int batch, int n_q,
-                                   float *scores, unsigned *ghist, bool fill_invisible, int *status,
-                                   int num_sms, cudaStream_t stream);
+                                   float *scores, bool fill_invisible, const IxSelectArgs &sel,
+                                   int *status, int num_sms, cudaStream_t stream);
 cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32_t *q_seq,
                           const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
                           int n_q, int select_k, const int64_t *slot_map, int64_t ld_slot, int out_width,

@@ -7,7 +7,8 @@ topk_pools -> expand_selection -> masked attention):
     glm_kv_store_int8 -> glm_kpool_build -> glm_index_scores_topk -> glm_expand_selection
       -> glm_sparse_mla_decode
 
-This module only owns device buffers (allocated with torch) and marshals them into the calls;
+A step runs the scoring, selection and expansion as one call (glm_index_topk_expand, one fused
+launch); the separate calls remain for checking each stage on its own. This module only owns device buffers (allocated with torch) and marshals them into the calls;
 all arithmetic runs in the library's kernels.
 """
 from __future__ import annotations
@@ -18,8 +19,8 @@ from typing import Optional
 import torch
 
 from . import (GLM_OP_INDEX_SCORES_TOPK, GLM_OP_SPARSE_MLA, GLM_ROW_BYTES, glm_dsa_workspace_size,
-               glm_expand_selection, glm_index_scores_topk, glm_kpool_build, glm_kv_store_int8,
-               glm_sparse_mla_decode, make_dims)
+               glm_expand_selection, glm_index_scores_topk, glm_index_topk_expand, glm_kpool_build,
+               glm_kv_store_int8, glm_sparse_mla_decode, make_dims)
 
 LATENT = 512
 IDX_HEADS = 32
@@ -132,13 +133,19 @@ def expand(b: DecodeBuffers, stream=None) -> None:
                          n_sel=b.n_sel, slot_map=b.slot_map, tok=b.tok, rows=b.rows, stream=stream)
 
 
+def index_topk_expand(b: DecodeBuffers, stream=None) -> None:
+    glm_index_topk_expand(b.dims, b.q_idx, b.w, b.pooled, b.q_seq, b.q_pos, b.pad, b.len, b.select_k,
+                          b.topk, b.out_width, n_sel=b.n_sel, slot_map=b.slot_map, tok=b.tok, rows=b.rows,
+                          scores=b.scores, workspace=b.ws_index, stream=stream)
+
+
 def attend(b: DecodeBuffers, stream=None) -> None:
     glm_sparse_mla_decode(b.dims, b.q, b.cache, b.rows, b.sm_scale, b.out, b.ws_mla, lse=b.lse,
                           out_f32=b.out_f32, stream=stream)
 
 
-STAGES = (("store_int8", store), ("kpool_build", build_pools), ("index_scores_topk", index_topk),
-          ("expand_selection", expand), ("sparse_mla_decode", attend))
+STAGES = (("store_int8", store), ("kpool_build", build_pools), ("index_topk_expand", index_topk_expand),
+          ("sparse_mla_decode", attend))
 
 
 def run_step(b: DecodeBuffers, stream=None) -> None:

@@ -80,6 +80,22 @@ def test_expand_requires_room_for_selection_and_tail():
                                   None, None, None) == kp.GLM_ERR_INVALID_ARG  # no output
 
 
+def test_fused_index_expand_argument_checks():
+    L = kp.lib
+    d = C.byref(kp.make_dims(64))
+    args = lambda sk, ow, tok, rows, ws_bytes: (d, FAKE, FAKE, FAKE, 16, FAKE, FAKE, FAKE, FAKE, 1, 1, sk,  # noqa: E731
+                                                None, 0, ow, None, FAKE, None, tok, rows, FAKE, ws_bytes, None)
+    # out_width must hold the largest selection plus a full tail
+    assert L.glm_index_topk_expand(*args(512, 2050, FAKE, None, 1 << 30)) == kp.GLM_ERR_INVALID_ARG
+    # no expansion output at all
+    assert L.glm_index_topk_expand(*args(512, 2051, None, None, 1 << 30)) == kp.GLM_ERR_INVALID_ARG
+    # misaligned expansion output
+    assert L.glm_index_topk_expand(*args(512, 2051, C.c_void_p(0x10002), None, 1 << 30)) == kp.GLM_ERR_INVALID_ARG
+    # select_k out of range, then a workspace that is too small
+    assert L.glm_index_topk_expand(*args(4096, 16387, FAKE, None, 1 << 30)) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_index_topk_expand(*args(8, 35, FAKE, FAKE, 16)) == kp.GLM_ERR_WORKSPACE
+
+
 def test_index_and_mla_argument_checks():
     L = kp.lib
     d = C.byref(kp.make_dims(64))

@@ -249,6 +249,64 @@ def test_index_topk_fused_selection(cuda):
         assert _selection_agrees(tg[n], want, so, n_sel) == 0
 
 
+_FUSED_CASES = [synth.TINY_DECODE, synth.PADDING_DECODE,
+                synth.custom("multi_q", (0, 3, 0, 1, 0, 2, 0, 0), (9000, 4099, 20000, 33, 64, 70001, 2048, 5),
+                             n_heads=64, select_k=512, out_width=2176, permute_slots=True, seed=35),
+                synth.custom("one_long", (1,), (131075,), n_heads=64, select_k=2048, out_width=8195, seed=36)]
+
+
+@pytest.mark.parametrize("wl", _FUSED_CASES, ids=lambda w: w.name)
+@pytest.mark.parametrize("pattern", ["synth", "few", "equal"])
+def test_fused_select_expand_bit_exact_on_own_scores(cuda, wl, pattern):
+    # the one-launch scores + selection + expansion: its top-k rows must be exactly the oracle's
+    # selection of the scores it wrote, and its tokens / rows exactly the oracle's expansion of
+    # that selection ("few": 3 distinct pooled keys, "equal": one -- only pool ids decide)
+    inp = synth.generate(wl)
+    b = sdev.allocate_for(inp, cuda, keep_scores=True)
+    sdev.load(inp, b, build_prefix=True)
+    if pattern == "few":
+        b.pooled.copy_(b.pooled[:, torch.arange(b.pooled.shape[1], device=cuda) % 3])
+    elif pattern == "equal":
+        b.pooled.copy_(b.pooled[:, :1].expand_as(b.pooled))
+    for t in (b.topk, b.n_sel, b.tok, b.rows):
+        t.fill_(4242)
+    b.scores.fill_(7.0)
+    for _ in range(2):                      # twice: the multi-CTA words must be reset every call
+        b.ws_index.fill_(0xA5)
+        b.ws_index[-256:].zero_()           # the status word
+        P.index_topk_expand(b)
+    torch.cuda.synchronize()
+    assert int(b.ws_index[-256:-252].view(torch.int32).item()) == 0
+    sg, tg, ng, tokg, rowg = np_(b.scores), np_(b.topk), np_(b.n_sel), np_(b.tok), np_(b.rows)
+    S, W = wl.select_k, wl.out_width
+    for n in range(len(inp.q_pos)):
+        s = int(inp.q_seq[n])
+        nv = oracle.n_visible_pools(inp.pad[s], inp.len[s], inp.q_pos[n])
+        assert np.isneginf(sg[n, nv:]).all()
+        want, n_sel = oracle.topk_pools(sg[n, :nv].astype(np.float64), S)
+        assert ng[n] == n_sel, n
+        assert np.array_equal(tg[n], want), n
+        want_tok, _ = oracle.expand_selection(want, n_sel, inp.pad[s], inp.len[s], inp.q_pos[n], W)
+        assert np.array_equal(tokg[n], want_tok), n
+        sm = inp.slot_map[s]
+        assert np.array_equal(rowg[n], np.where(want_tok >= 0, sm[np.maximum(want_tok, 0)], -1)), n
+
+
+def test_fused_entry_equals_separate_entries(cuda):
+    inp = synth.generate(_FUSED_CASES[2])
+    b = sdev.allocate_for(inp, cuda, keep_scores=True)
+    sdev.load(inp, b, build_prefix=True)
+    P.index_topk_expand(b)
+    fused = [np_(t).copy() for t in (b.scores, b.topk, b.n_sel, b.tok, b.rows)]
+    for t in (b.scores, b.topk, b.n_sel, b.tok, b.rows):
+        t.fill_(99)
+    P.index_topk(b)
+    P.expand(b)
+    sep = [np_(t) for t in (b.scores, b.topk, b.n_sel, b.tok, b.rows)]
+    for f, g in zip(fused, sep):
+        assert np.array_equal(f, g)
+
+
 def _selection_agrees(got, want, scores, n_sel):
     """The GPU selection against the oracle's (scores = the oracle's fp64 scores). Equal as sets,
     except that pools whose score is within 1e-4 (relative) of the select_k-th score may be
