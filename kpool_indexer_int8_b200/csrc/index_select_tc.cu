@@ -92,21 +92,28 @@ __device__ __forceinline__ void write_outputs(const IxSelectArgs &sel, int n, in
         const int tail = max(0, last - (pb + kKpool * nvx) + 1);
         n_valid = kKpool * ns + tail;
     }
-    for (int j = threadIdx.x; j < sel.out_width; j += blockDim.x) {
-        int t = GLM_INVALID;
-        if (j < kKpool * ns) t = pb + kKpool * id_of(s.cand[j / kKpool]) + (j % kKpool);
-        else if (j < n_valid) t = pb + kKpool * nvx + (j - kKpool * ns);
-        if (sel.tok) sel.tok[base + j] = t;
-        if (sel.rows) {
-            int r = t;
-            if (sel.slot_map) {
-                r = GLM_INVALID;
-                if (t >= 0 && t < sel.ld_slot) {
-                    const int64_t v = sel.slot_map[static_cast<int64_t>(b) * sel.ld_slot + t];
-                    r = (v >= 0 && v <= 0x7fffffffll) ? static_cast<int>(v) : GLM_INVALID;
-                }
-            }
-            sel.rows[base + j] = r;
+    constexpr int kU = 5;   // entries per thread in flight (slot-map loads issued together)
+    for (int j0 = 0; j0 < sel.out_width; j0 += kU * static_cast<int>(blockDim.x)) {
+        int tv[kU];
+        long long rv[kU];
+#pragma unroll
+        for (int u = 0; u < kU; u++) {
+            const int j = j0 + u * static_cast<int>(blockDim.x) + static_cast<int>(threadIdx.x);
+            int t = GLM_INVALID;
+            if (j < kKpool * ns) t = pb + kKpool * id_of(s.cand[j / kKpool]) + (j % kKpool);
+            else if (j < n_valid) t = pb + kKpool * nvx + (j - kKpool * ns);
+            tv[u] = t;
+            rv[u] = t;
+            if (sel.rows && sel.slot_map)
+                rv[u] = (t >= 0 && t < sel.ld_slot) ? sel.slot_map[static_cast<int64_t>(b) * sel.ld_slot + t] : -1ll;
+        }
+#pragma unroll
+        for (int u = 0; u < kU; u++) {
+            const int j = j0 + u * static_cast<int>(blockDim.x) + static_cast<int>(threadIdx.x);
+            if (j >= sel.out_width) continue;
+            if (sel.tok) sel.tok[base + j] = tv[u];
+            if (sel.rows)
+                sel.rows[base + j] = (rv[u] >= 0 && rv[u] <= 0x7fffffffll) ? static_cast<int>(rv[u]) : GLM_INVALID;
         }
     }
 }
@@ -317,11 +324,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_select_tc_kernel(
     if (multi) {   // grid barrier of the query's CTAs, then the summed histogram
         __syncthreads();
         if (tid == 0) {   // release this CTA's histogram, arrive, wait (acquire) for the others
-            __threadfence();
-            atomicAdd(&cnt[kCntArrive], 1u);
-            uint32_t it = 0;
-            while (ld_acquire(&cnt[kCntArrive]) < static_cast<unsigned>(G) && ++it < kSelWaitLimit) __nanosleep(64);
-            *flag = it >= kSelWaitLimit;
+            *flag = grid_barrier(&cnt[kCntArrive], G) ? 0u : 1u;
             if (*flag && status) atomicOr(status, 8);
         }
         __syncthreads();

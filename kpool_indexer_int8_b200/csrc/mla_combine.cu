@@ -4,78 +4,99 @@
 //   M = max_c m_c,  L = sum_c l_c e^{m_c - M},  out = (sum_c e^{m_c - M} acc_c) / L,
 //   lse = M + log L.
 // Chunks with l = 0 (no valid entry) are skipped without reading their accumulator.
-// One CTA of 128 threads per (query, head); thread t owns output columns [4t, 4t + 4).
 #include "common.cuh"
 #include "sparse_mla.cuh"
 
 namespace glm {
 
 constexpr int kMaxCombineChunks = 1024;  // 65536 / 64
+constexpr int kCombineThreads = 512;
+constexpr int kChunkGroups = kCombineThreads / (kLatent / 4);   // 4 groups of 128 threads
 
-__global__ void __launch_bounds__(128) mla_combine_kernel(const float *__restrict__ part_acc,
-                                                          const float *__restrict__ part_ml,
-                                                          int n_heads, int n_chunks,
-                                                          uint16_t *__restrict__ out,
-                                                          float *__restrict__ out_f32,
-                                                          float *__restrict__ lse) {
+// One CTA of 512 threads per (head, query): thread t owns output columns [4 (t % 128), +4) of
+// chunk group t / 128 (chunks c = group, group + 4, ...), all of its chunk loads in flight at
+// once; the 4 group sums are added in shared memory.
+__global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const float *__restrict__ part_acc,
+                                                                      const float *__restrict__ part_ml,
+                                                                      int n_heads, int n_chunks,
+                                                                      uint16_t *__restrict__ out,
+                                                                      float *__restrict__ out_f32,
+                                                                      float *__restrict__ lse) {
     pdl_begin();
     __shared__ float wgt[kMaxCombineChunks];
-    __shared__ float red[4];
-    const int h = blockIdx.x, n = blockIdx.y, t = threadIdx.x;
+    __shared__ float red[kCombineThreads / 32];
+    __shared__ float4 part[kChunkGroups - 1][kLatent / 4];
+    const int h = blockIdx.x, n = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int64_t base = static_cast<int64_t>(n) * n_chunks * n_heads + h;
-    // every chunk's (m, l) at once: one round trip instead of one per chunk
+    // every chunk's (m, l) at once; M = the largest m of a chunk with an entry
     float mx = -INFINITY;
-    for (int c = t; c < n_chunks; c += blockDim.x) {
+    for (int c = t; c < n_chunks; c += kCombineThreads) {
         const float2 ml = *reinterpret_cast<const float2 *>(part_ml + 2 * (base + static_cast<int64_t>(c) * n_heads));
-        wgt[c] = ml.y > 0.0f ? ml.x : -INFINITY;   // the chunk's max, or -inf if it had no entry
+        wgt[c] = ml.y > 0.0f ? ml.x : -INFINITY;
         if (ml.y > 0.0f) mx = fmaxf(mx, ml.x);
     }
     mx = warp_max(mx);
-    if ((t & 31) == 0) red[t >> 5] = mx;
+    if (lane == 0) red[warp] = mx;
     __syncthreads();
-    const float M = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    float M = lane < kCombineThreads / 32 ? red[lane] : -INFINITY;
+    M = warp_max(M);
     __syncthreads();
     float Lp = 0.0f;
-    for (int c = t; c < n_chunks; c += blockDim.x) {
+    for (int c = t; c < n_chunks; c += kCombineThreads) {
         const float m = wgt[c];
         const float wc = (m == -INFINITY || M == -INFINITY) ? 0.0f : expf(m - M);
         wgt[c] = wc;
         Lp = fmaf(part_ml[2 * (base + static_cast<int64_t>(c) * n_heads) + 1], wc, Lp);
     }
     Lp = warp_sum(Lp);
-    if ((t & 31) == 0) red[t >> 5] = Lp;
+    if (lane == 0) red[warp] = Lp;
     __syncthreads();
-    const float L = (red[0] + red[1]) + (red[2] + red[3]);
-    // weighted sum of the chunk accumulators, four chunks in flight per thread
+    float L = lane < kCombineThreads / 32 ? red[lane] : 0.0f;
+    L = warp_sum(L);
+    // this thread's columns over its chunk group, eight chunk loads in flight
+    const int col = t % (kLatent / 4), grp = t / (kLatent / 4);
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    int c = 0;
-    for (; c + 4 <= n_chunks; c += 4) {
-        float4 v[4];
+    int c = grp;
+    for (; c + 7 * kChunkGroups < n_chunks; c += 8 * kChunkGroups) {
+        float4 v[8];
 #pragma unroll
-        for (int u = 0; u < 4; u++)
-            v[u] = wgt[c + u] > 0.0f ? reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(c + u) * n_heads) * kLatent)[t]
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int u = 0; u < 8; u++) {
+            const int cu = c + u * kChunkGroups;
+            v[u] = wgt[cu] > 0.0f ? reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(cu) * n_heads) * kLatent)[col]
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-        for (int u = 0; u < 4; u++) {
-            const float wc = wgt[c + u];
+        for (int u = 0; u < 8; u++) {
+            const float wc = wgt[c + u * kChunkGroups];
             a.x = fmaf(wc, v[u].x, a.x);
             a.y = fmaf(wc, v[u].y, a.y);
             a.z = fmaf(wc, v[u].z, a.z);
             a.w = fmaf(wc, v[u].w, a.w);
         }
     }
-    for (; c < n_chunks; c++) {
+    for (; c < n_chunks; c += kChunkGroups) {
         const float wc = wgt[c];
         if (!(wc > 0.0f)) continue;
-        const float4 v = reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(c) * n_heads) * kLatent)[t];
+        const float4 v = reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(c) * n_heads) * kLatent)[col];
         a.x = fmaf(wc, v.x, a.x);
         a.y = fmaf(wc, v.y, a.y);
         a.z = fmaf(wc, v.z, a.z);
         a.w = fmaf(wc, v.w, a.w);
     }
+    if (grp > 0) part[grp - 1][col] = a;
+    __syncthreads();
+    if (grp > 0) return;
+#pragma unroll
+    for (int g2 = 0; g2 < kChunkGroups - 1; g2++) {
+        const float4 b = part[g2][col];
+        a.x += b.x;
+        a.y += b.y;
+        a.z += b.z;
+        a.w += b.w;
+    }
     const float inv = L > 0.0f ? 1.0f / L : 0.0f;
     const float o[4] = {a.x * inv, a.y * inv, a.z * inv, a.w * inv};
-    const int64_t ob = (static_cast<int64_t>(n) * n_heads + h) * kLatent + 4 * t;
+    const int64_t ob = (static_cast<int64_t>(n) * n_heads + h) * kLatent + 4 * col;
     uint32_t lo = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o[0]))) |
                   (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o[1]))) << 16);
     uint32_t hi = static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o[2]))) |
@@ -89,8 +110,8 @@ cudaError_t launch_mla_combine(const float *part_acc, const float *part_ml, int 
                                int n_chunks, void *out, float *out_f32, float *lse,
                                cudaStream_t stream) {
     dim3 grid(n_heads, n_q);
-    launch_pdl(mla_combine_kernel, dim3(grid), dim3(128), 0, stream, part_acc, part_ml, n_heads, n_chunks,
-                                                 static_cast<uint16_t *>(out), out_f32, lse);
+    launch_pdl(mla_combine_kernel, dim3(grid), dim3(kCombineThreads), 0, stream, part_acc, part_ml, n_heads,
+               n_chunks, static_cast<uint16_t *>(out), out_f32, lse);
     return cudaGetLastError();
 }
 

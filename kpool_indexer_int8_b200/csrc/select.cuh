@@ -69,6 +69,26 @@ __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
     return v;
 }
 
+// Ticket of a CTA (one thread, after a bar.sync that orders its CTA's writes): a release-acquire
+// atomic increment; true on the CTA that completes the count, which then sees every CTA's writes.
+__device__ __forceinline__ bool take_ticket(unsigned *ctr, int n_ctas) {
+    unsigned old;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(ctr) : "memory");
+    return old == static_cast<unsigned>(n_ctas - 1);
+}
+
+// Grid barrier of the n_ctas CTAs of one query (one thread per CTA, after a bar.sync; every CTA
+// resident): release-increment, then acquire-poll until all have arrived. Returns false if the
+// wait gave up after kSelWaitLimit polls.
+__device__ __forceinline__ bool grid_barrier(unsigned *ctr, int n_ctas) {
+    asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
+    for (uint32_t it = 0; it < kSelWaitLimit; it++) {
+        if (ld_acquire(ctr) >= static_cast<unsigned>(n_ctas)) return true;
+        __nanosleep(32);
+    }
+    return false;
+}
+
 // On warp 0 only: in a histogram of `nbins` bins (a multiple of 32) the highest bin whose suffix
 // count (it and all higher bins) reaches k; writes s.bin, s.above (count in higher bins) and
 // s.count (the bin's own count). Requires k <= total.
@@ -512,11 +532,8 @@ __device__ __forceinline__ bool merge_lists_multi(unsigned *cnt, unsigned *words
     for (unsigned i = tid; i < lb; i += blockDim.x) my_b[i] = s.bnd[i];
     if (tid == 0) words[g] = la | (lb << 11) | (s.n_b > static_cast<unsigned>(kBoundCap) ? 1u << 24 : 0u);
     __syncthreads();
-    if (tid == 0) {   // release this CTA's lists, take the ticket; the last CTA acquires everyone's
-        __threadfence();
-        s.last = atomicAdd(&cnt[kCntTicket], 1u) == static_cast<unsigned>(n_ctas - 1);
-        if (s.last) __threadfence();
-    }
+    if (tid == 0)   // release this CTA's lists and take the ticket; the last CTA acquires everyone's
+        s.last = take_ticket(&cnt[kCntTicket], n_ctas);
     __syncthreads();
     if (!s.last) return false;
     if (warp == 0) {

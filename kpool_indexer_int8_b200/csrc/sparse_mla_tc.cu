@@ -10,9 +10,10 @@
 //      file in shared memory; the query block Q[heads x 512] goes to shared memory the same way.
 //   2. S = Q . C^T on tcgen05 (kind::f16, fp32 accumulator in tensor memory, 32 MMAs of K = 16).
 //      C is the K-major B operand here.
-//   3. softmax of the chunk, one TMEM lane (= one head) per thread: s = S * scale_j * sm_scale,
-//      m = max, p = exp(s - m), l = sum p; P' = p * scale_j (the V dequantisation scale folded
-//      in) is split into bf16 hi + lo so that the PV product keeps ~16 mantissa bits of P'.
+//   3. softmax of the chunk, two threads per head (one TMEM lane, half of the entries each, the
+//      halves' maxima and sums exchanged in shared memory): s = S * scale_j * sm_scale, m = max,
+//      p = exp(s - m), l = sum p; P' = p * scale_j (the V dequantisation scale folded in) is split
+//      into bf16 hi + lo so that the PV product keeps ~16 mantissa bits of P'.
 //   4. O^T = C^T . P'^T: the 512 latent dims are the M dimension (4 tiles of M = 128) and the heads
 //      the N dimension, so that in tensor memory one lane holds one latent dim of every head. The
 //      same tile C is now the MN-major A operand (a core matrix of 8 rows x 8 dims serves both
@@ -45,7 +46,9 @@ struct TcLayout {
     static constexpr int kBar = kRow + 256;          // 2 mbarriers
     static constexpr int kTmem = kBar + 16;          // tensor-memory base address
     static constexpr int kFlag = kTmem + 16;
-    static constexpr int kBytes = kFlag + 16;
+    static constexpr int kPmax = kFlag + 16;         // [2 column halves][128 heads] partial maxima
+    static constexpr int kPl = kPmax + 2 * 128 * 4;  // [2][128] partial sums
+    static constexpr int kBytes = kPl + 2 * 128 * 4;
 };
 
 __device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w, int shift) {
@@ -176,39 +179,46 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
         tc::mma_commit(tc::smem_addr(&bar[0]));
     }
 
-    // 3. softmax of the chunk on warps 0-3 (TMEM lane = head)
-    if (warp < 4) {
+    // 3. softmax of the chunk on all 8 warps: warp w reads TMEM lane quadrant w % 4 (lane = head)
+    //    and the columns (entries) [32 (w / 4), +32); the two halves of a head exchange their
+    //    maxima and sums through shared memory
+    {
+        float *pmax = reinterpret_cast<float *>(smem + Lay::kPmax);
+        float *pl = reinterpret_cast<float *>(smem + Lay::kPl);
+        const int quad = warp & 3, hf = warp >> 2;
         if (!tc::mbar_wait(tc::smem_addr(&bar[0]), 0, kWaitLimit)) atomicOr(status, 1);
         __syncwarp();  // thread 0 arrives here after issuing the MMAs: reconverge for tcgen05.ld
         tc::fence_after_sync();
-        uint32_t r0[32], r1[32];
-        const uint32_t ta = tmem + (static_cast<uint32_t>(warp * 32) << 16);
-        tc::tmem_ld32(ta, r0);
-        tc::tmem_ld32(ta + 32, r1);
+        uint32_t r[32];
+        tc::tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + hf * 32, r);
         tc::tmem_wait_ld();
-        const int head = (M == 128) ? warp * 32 + lane : (lane < 16 ? warp * 16 + lane : -1);
-        if (head >= 0) {
-            const float k2 = sm_scale * 1.4426950408889634f;  // scores in log2 units
-            float s[kTcRows];
-            float mx = -INFINITY;
+        const int head = (M == 128) ? quad * 32 + lane : (lane < 16 ? quad * 16 + lane : -1);
+        const float k2 = sm_scale * 1.4426950408889634f;  // scores in log2 units
+        float sv[32];
+        float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < kTcRows; j++) {
-                const float raw = __uint_as_float(j < 32 ? r0[j] : r1[j - 32]);
-                s[j] = ridx[j] >= 0 ? raw * scl[j] * k2 : -INFINITY;
-                mx = fmaxf(mx, s[j]);
-            }
+        for (int jj = 0; jj < 32; jj++) {
+            const int j = hf * 32 + jj;
+            sv[jj] = ridx[j] >= 0 ? __uint_as_float(r[jj]) * scl[j] * k2 : -INFINITY;
+            mx = fmaxf(mx, sv[jj]);
+        }
+        if (head >= 0) pmax[hf * 128 + head] = mx;
+        __syncthreads();
+        if (head >= 0) {
+            mx = fmaxf(pmax[head], pmax[128 + head]);
             float l = 0.0f;
             const bool real = head < n_heads;
 #pragma unroll
-            for (int rg = 0; rg < kTcRows / 8; rg++) {
+            for (int rq = 0; rq < 4; rq++) {
+                const int rg = hf * 4 + rq;   // row group of 8 entries
                 uint32_t hi[4], lo[4];
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
                     uint32_t hb[2], lb[2];
 #pragma unroll
                     for (int u = 0; u < 2; u++) {
-                        const int j = rg * 8 + 2 * e + u;
-                        const float p = ridx[j] >= 0 ? exp2f(s[j] - mx) : 0.0f;
+                        const int jj = rq * 8 + 2 * e + u, j = hf * 32 + jj;
+                        const float p = ridx[j] >= 0 ? exp2f(sv[jj] - mx) : 0.0f;
                         l += p;
                         const float pp = real ? p * scl[j] : 0.0f;
                         const uint16_t h16 = bf16_rn_bits(pp);
@@ -222,15 +232,22 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
                 *reinterpret_cast<uint4 *>(Phi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                 *reinterpret_cast<uint4 *>(Plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
-            if (real) {
-                part_ml[2 * (ml_base + head)] = mx * 0.6931471805599453f;  // back to natural log
-                part_ml[2 * (ml_base + head) + 1] = l;
-            }
+            pl[hf * 128 + head] = l;
+            pmax[hf * 128 + head] = mx;   // (same value in both halves)
         }
         tc::fence_before_sync();
     }
     tc::fence_proxy_async();
     __syncthreads();
+    if (warp < 4) {   // (m, l) of each head, natural-log units
+        const float *pmax = reinterpret_cast<const float *>(smem + Lay::kPmax);
+        const float *pl = reinterpret_cast<const float *>(smem + Lay::kPl);
+        const int head = (M == 128) ? warp * 32 + lane : (lane < 16 ? warp * 16 + lane : -1);
+        if (head >= 0 && head < n_heads) {
+            part_ml[2 * (ml_base + head)] = pmax[head] * 0.6931471805599453f;
+            part_ml[2 * (ml_base + head) + 1] = pl[head] + pl[128 + head];
+        }
+    }
 
     // 4. O^T = C^T . P'^T (hi and lo terms accumulate into the same columns)
     if (tid == 0) {
