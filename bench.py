@@ -36,7 +36,11 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-KERNEL_LAUNCHES_PER_STEP = 6   # store, kpool, zero, scores+top-k+expansion, MLA split, MLA combine
+def kernel_launches_per_step(wl, num_sms: int) -> int:
+    """Kernels of one glm_dsa_decode_step: store + pool build + zeroing, scores + top-k + expansion,
+    MLA split (with the combine in-kernel when every split CTA is resident at once), else + combine."""
+    n_chunks = (wl.out_width + 63) // 64
+    return 3 if wl.n_queries * n_chunks <= num_sms else 4
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -437,7 +441,7 @@ def run_kernels(args, wl):
         "e2e": {"value": e2e_qps, "unit": "queries/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
                 "api": "C ABI via kpool_indexer_int8_b200 binding, host pinned buffers, sync per step"},
-        "gpu_launches": KERNEL_LAUNCHES_PER_STEP * args.steps,
+        "gpu_launches": kernel_launches_per_step(wl, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
         "clocks": sampler.summary(),
     }
     line["achieved_hbm_frac_per_gpu"] = line["achieved_hbm_gbs_per_gpu"] / peak

@@ -7,6 +7,7 @@
  *   glm_index_scores_topk  -> relu head-weighted index scores and the top select_k pools
  *   glm_expand_selection   -> token indices (+ cache rows), visible tail, -1 padding
  *   (glm_index_topk_expand -> the two above in one launch)
+ *   (glm_dsa_decode_step   -> the whole step in one call)
  *   glm_sparse_mla_decode  -> sparse NoPE MLA over the gathered int8 rows (split-KV + combine)
  *
  * Conventions for every entry point
@@ -269,17 +270,87 @@ int glm_sparse_mla_decode_noalloc(const glm_dsa_dims *dims, const void *q_dev,
                                   float *lse_dev, float *out_f32_dev, void *stream);
 
 /* ------------------------------------------------------------------------------------------ */
+/* the whole decode step in one call                                                           */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * Arguments of glm_dsa_decode_step: those of glm_kv_store_int8, glm_kpool_build,
+ * glm_index_topk_expand and glm_sparse_mla_decode (same names, meanings, layouts and rules; the
+ * cache rows written by the store are the rows the attention reads, so slot_map_dev must map the
+ * new tokens to the slots in slots_dev). Every pointer is a device pointer.
+ */
+typedef struct glm_dsa_step {
+    /* store_int8: n_new new latent rows */
+    const void *latent_dev;        /* bf16 [n_new, 512]                  */
+    const int64_t *slots_dev;      /* int64 [n_new]                      */
+    int64_t n_new;
+    int8_t *cache_dev;             /* int8 [n_rows, 528]                 */
+    int64_t n_rows;
+    /* kpool_build: up to max_new_pools new pools per sequence from pool_begin_dev */
+    const void *k_dev;             /* bf16 [batch, ld_tokens, 128]       */
+    const void *gate_dev;          /* bf16 [batch, ld_tokens, 128]       */
+    int64_t ld_tokens;
+    const float *ln_w_dev;         /* fp32 [128]                         */
+    const float *ln_b_dev;         /* fp32 [128]                         */
+    float ln_eps;
+    const int32_t *pad_dev;        /* int32 [batch]                      */
+    const int32_t *len_dev;        /* int32 [batch]                      */
+    const int32_t *pool_begin_dev; /* int32 [batch] or NULL              */
+    int32_t batch;
+    int32_t max_new_pools;
+    float *pooled_dev;             /* fp32 [batch, ld_pools, 128]        */
+    int64_t ld_pools;
+    /* index scores, top-k, expansion */
+    const void *q_idx_dev;         /* bf16 [n_q, 32, 128]                */
+    const float *w_dev;            /* fp32 [n_q, 32]                     */
+    const int32_t *q_seq_dev;      /* int32 [n_q]                        */
+    const int32_t *q_pos_dev;      /* int32 [n_q]                        */
+    int32_t n_q;
+    int32_t select_k;
+    const int64_t *slot_map_dev;   /* int64 [batch, ld_slot] or NULL     */
+    int64_t ld_slot;
+    int32_t out_width;             /* >= 4 * select_k + 3                */
+    float *scores_dev;             /* fp32 [n_q, ld_pools] or NULL       */
+    int32_t *topk_dev;             /* int32 [n_q, select_k]              */
+    int32_t *n_sel_dev;            /* int32 [n_q] or NULL                */
+    int32_t *tok_dev;              /* int32 [n_q, out_width] or NULL     */
+    int32_t *rows_dev;             /* int32 [n_q, out_width]             */
+    /* sparse MLA over rows_dev */
+    const void *q_dev;             /* bf16 [n_q, n_heads, 512]           */
+    float sm_scale;
+    void *out_dev;                 /* bf16 [n_q, n_heads, 512]           */
+    float *lse_dev;                /* fp32 [n_q, n_heads] or NULL        */
+    float *out_f32_dev;            /* fp32 [n_q, n_heads, 512] or NULL   */
+} glm_dsa_step;
+
+/*
+ * One decode (or prefill-chunk) step: glm_kv_store_int8, glm_kpool_build, glm_index_topk_expand
+ * and glm_sparse_mla_decode on the same stream, with the same results as those four calls in
+ * that order. It runs as three kernels (four when the attention does not fit one wave of CTAs):
+ * the store, the pool build and the zeroing of the step's counters share the first; the sparse
+ * attention merges its split-KV partials in-kernel when all of its CTAs are resident at once.
+ *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_DECODE_STEP, n_q, ld_pools,
+ *               select_k, out_width), 256-byte aligned, contents on entry ignored. Its last 256
+ *               bytes start with a status word set nonzero when a wait gave up (outputs invalid;
+ *               never cleared by the library).
+ * Checks: those of the four calls; the first failing one is returned and nothing is enqueued.
+ */
+int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *step, void *workspace_dev,
+                        size_t ws_bytes, void *stream);
+
+/* ------------------------------------------------------------------------------------------ */
 /* workspace sizes                                                                             */
 /* ------------------------------------------------------------------------------------------ */
 #define GLM_OP_INDEX_SCORES_TOPK 1
 #define GLM_OP_TOPK_POOLS 2
 #define GLM_OP_SPARSE_MLA 3
+#define GLM_OP_DECODE_STEP 4
 
 /*
  * Bytes of device workspace an entry point needs (0 if none; (size_t)-1 for bad arguments).
  *   GLM_OP_INDEX_SCORES_TOPK: n_q, max_pools = ld_pools, select_k
  *   GLM_OP_TOPK_POOLS:        n_q, max_pools = ld_scores, select_k
  *   GLM_OP_SPARSE_MLA:        n_q, width (max_pools and select_k unused)
+ *   GLM_OP_DECODE_STEP:       n_q, max_pools = ld_pools, select_k, width = out_width
  */
 size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
                               int64_t max_pools, int32_t select_k, int32_t width);

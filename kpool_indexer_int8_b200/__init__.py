@@ -31,9 +31,11 @@ GLM_ROW_BYTES = 528
 GLM_OP_INDEX_SCORES_TOPK = 1
 GLM_OP_TOPK_POOLS = 2
 GLM_OP_SPARSE_MLA = 3
+GLM_OP_DECODE_STEP = 4
 
 EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv_store_int8",
            "glm_kpool_build", "glm_index_scores", "glm_index_scores_topk", "glm_index_topk_expand",
+           "glm_dsa_decode_step",
            "glm_topk_pools", "glm_expand_selection",
            "glm_sparse_mla_decode", "glm_dsa_workspace_size")
 
@@ -44,6 +46,25 @@ class glm_dsa_dims(C.Structure):
                 ("n_heads", C.c_int32), ("index_n_heads", C.c_int32),
                 ("index_head_dim", C.c_int32), ("index_kpool", C.c_int32),
                 ("index_topk", C.c_int32)]
+
+
+class glm_dsa_step(C.Structure):
+    """Arguments of glm_dsa_decode_step (every pointer a device pointer, None allowed where the
+    C header allows NULL)."""
+    _fields_ = [("latent_dev", C.c_void_p), ("slots_dev", C.c_void_p), ("n_new", C.c_int64),
+                ("cache_dev", C.c_void_p), ("n_rows", C.c_int64),
+                ("k_dev", C.c_void_p), ("gate_dev", C.c_void_p), ("ld_tokens", C.c_int64),
+                ("ln_w_dev", C.c_void_p), ("ln_b_dev", C.c_void_p), ("ln_eps", C.c_float),
+                ("pad_dev", C.c_void_p), ("len_dev", C.c_void_p), ("pool_begin_dev", C.c_void_p),
+                ("batch", C.c_int32), ("max_new_pools", C.c_int32), ("pooled_dev", C.c_void_p),
+                ("ld_pools", C.c_int64),
+                ("q_idx_dev", C.c_void_p), ("w_dev", C.c_void_p), ("q_seq_dev", C.c_void_p),
+                ("q_pos_dev", C.c_void_p), ("n_q", C.c_int32), ("select_k", C.c_int32),
+                ("slot_map_dev", C.c_void_p), ("ld_slot", C.c_int64), ("out_width", C.c_int32),
+                ("scores_dev", C.c_void_p), ("topk_dev", C.c_void_p), ("n_sel_dev", C.c_void_p),
+                ("tok_dev", C.c_void_p), ("rows_dev", C.c_void_p),
+                ("q_dev", C.c_void_p), ("sm_scale", C.c_float), ("out_dev", C.c_void_p),
+                ("lse_dev", C.c_void_p), ("out_f32_dev", C.c_void_p)]
 
 
 def make_dims(n_heads: int, kv_lora_rank: int = 512, qk_rope_head_dim: int = 0,
@@ -71,6 +92,8 @@ lib.glm_index_scores_topk.restype = C.c_int
 lib.glm_index_topk_expand.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32, _P, _I64,
                                       _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]
 lib.glm_index_topk_expand.restype = C.c_int
+lib.glm_dsa_decode_step.argtypes = [_D, C.POINTER(glm_dsa_step), _P, _SZ, _P]
+lib.glm_dsa_decode_step.restype = C.c_int
 lib.glm_index_scores.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P]
 lib.glm_index_scores.restype = C.c_int
 lib.glm_topk_pools.argtypes = [_P, _I64, _P, _I32, _I32, _P, _P, _P, _SZ, _P]
@@ -202,6 +225,43 @@ def glm_index_topk_expand(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, sel
                                      int(out_width), _ptr(scores), _ptr(topk), _ptr(n_sel), _ptr(tok),
                                      _ptr(rows), _ptr(workspace), ws_bytes, _stream(stream)),
            "glm_index_topk_expand")
+
+
+def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_eps, pad, length, pool_begin,
+                        max_new_pools, pooled, q_idx, w, q_seq, q_pos, select_k, out_width, slot_map, rows,
+                        topk, q, sm_scale, out, workspace, n_sel=None, tok=None, scores=None, lse=None,
+                        out_f32=None, stream=None) -> None:
+    """The whole step in one call: the arguments of glm_kv_store_int8, glm_kpool_build,
+    glm_index_topk_expand and glm_sparse_mla_decode (same tensors and rules)."""
+    for t, dt, nm in ((latent, torch.bfloat16, "latent"), (slots, torch.int64, "slots"), (cache, torch.int8, "cache"),
+                      (k, torch.bfloat16, "k"), (gate, torch.bfloat16, "gate"), (ln_w, torch.float32, "ln_w"),
+                      (ln_b, torch.float32, "ln_b"), (pad, torch.int32, "pad"), (length, torch.int32, "len"),
+                      (pool_begin, torch.int32, "pool_begin"), (pooled, torch.float32, "pooled"),
+                      (q_idx, torch.bfloat16, "q_idx"), (w, torch.float32, "w"), (q_seq, torch.int32, "q_seq"),
+                      (q_pos, torch.int32, "q_pos"), (slot_map, torch.int64, "slot_map"), (rows, torch.int32, "rows"),
+                      (topk, torch.int32, "topk"), (q, torch.bfloat16, "q"), (out, torch.bfloat16, "out"),
+                      (workspace, torch.uint8, "workspace"), (n_sel, torch.int32, "n_sel"), (tok, torch.int32, "tok"),
+                      (scores, torch.float32, "scores"), (lse, torch.float32, "lse"), (out_f32, torch.float32, "out_f32")):
+        _dev(t, dt, nm)
+    a = glm_dsa_step()
+    v = lambda t: None if t is None else t.data_ptr()  # noqa: E731
+    a.latent_dev, a.slots_dev, a.n_new = v(latent), v(slots), slots.shape[0]
+    a.cache_dev, a.n_rows = v(cache), cache.shape[0]
+    a.k_dev, a.gate_dev, a.ld_tokens = v(k), v(gate), k.shape[1]
+    a.ln_w_dev, a.ln_b_dev, a.ln_eps = v(ln_w), v(ln_b), float(ln_eps)
+    a.pad_dev, a.len_dev, a.pool_begin_dev = v(pad), v(length), v(pool_begin)
+    a.batch, a.max_new_pools = pad.shape[0], int(max_new_pools)
+    a.pooled_dev, a.ld_pools = v(pooled), pooled.shape[1]
+    a.q_idx_dev, a.w_dev, a.q_seq_dev, a.q_pos_dev = v(q_idx), v(w), v(q_seq), v(q_pos)
+    a.n_q, a.select_k = q_idx.shape[0], int(select_k)
+    a.slot_map_dev, a.ld_slot = v(slot_map), (0 if slot_map is None else slot_map.shape[1])
+    a.out_width = int(out_width)
+    a.scores_dev, a.topk_dev, a.n_sel_dev, a.tok_dev, a.rows_dev = v(scores), v(topk), v(n_sel), v(tok), v(rows)
+    a.q_dev, a.sm_scale, a.out_dev = v(q), float(sm_scale), v(out)
+    a.lse_dev, a.out_f32_dev = v(lse), v(out_f32)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    _check(lib.glm_dsa_decode_step(C.byref(dims), C.byref(a), _ptr(workspace), ws_bytes, _stream(stream)),
+           "glm_dsa_decode_step")
 
 
 def glm_index_scores(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, scores, stream=None) -> None:

@@ -74,9 +74,69 @@ size_t mla_parts(int n_q, int n_heads, int width) {
 }
 size_t mla_acc_bytes(size_t parts) { return align_up(parts * glm::kLatent * sizeof(float), 256); }
 size_t mla_ml_bytes(size_t parts) { return align_up(parts * 2 * sizeof(float), 256); }
+// Host checks of each stage's arguments (GLM_OK: may proceed; a count of zero is accepted).
+int check_store(const glm_dsa_dims *dims, const void *latent, const int64_t *slots, int64_t n,
+                const int8_t *cache, int64_t n_rows) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n < 0 || n_rows < 0) return GLM_ERR_INVALID_ARG;
+    if (n == 0) return GLM_OK;
+    if (!latent || !slots || !cache) return GLM_ERR_INVALID_ARG;
+    if (!aligned(latent, 16) || !aligned(cache, 16) || !aligned(slots, 8)) return GLM_ERR_INVALID_ARG;
+    return GLM_OK;
+}
+
+int check_kpool(const glm_dsa_dims *dims, const void *k, const void *gate, int64_t ld_tokens,
+                const float *ln_w, const float *ln_b, float ln_eps, const int32_t *pad, const int32_t *len,
+                const int32_t *pool_begin, int32_t batch, int32_t max_new_pools, const float *pooled,
+                int64_t ld_pools, const int32_t *n_pools) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (batch < 0 || max_new_pools < 0 || ld_tokens < 0 || ld_pools < 0) return GLM_ERR_INVALID_ARG;
+    if (!(ln_eps >= 0.0f)) return GLM_ERR_INVALID_ARG;
+    if (batch == 0) return GLM_OK;
+    if (!k || !gate || !ln_w || !ln_b || !pad || !len || !pooled) return GLM_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(gate, 16) || !aligned(ln_w, 16) || !aligned(ln_b, 16) ||
+        !aligned(pooled, 16) || !aligned(pad, 4) || !aligned(len, 4) ||
+        (pool_begin && !aligned(pool_begin, 4)) || (n_pools && !aligned(n_pools, 4)))
+        return GLM_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(batch) * max_new_pools > (int64_t(1) << 40)) return GLM_ERR_INVALID_ARG;
+    return GLM_OK;
+}
+
+int check_mla(const glm_dsa_dims *dims, const void *q, const int8_t *cache, int64_t n_rows, const int32_t *rows,
+              int32_t n_q, int32_t width, float sm_scale, const void *out, const float *lse, const float *out_f32) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_q < 0 || n_rows < 0 || width < 1 || width > 65536 || n_q > 65535) return GLM_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale)) return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (!q || !rows || !out || (n_rows > 0 && !cache)) return GLM_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || (cache && !aligned(cache, 16)) || !aligned(rows, 4) || !aligned(out, 16) ||
+        (lse && !aligned(lse, 4)) || (out_f32 && !aligned(out_f32, 16)))
+        return GLM_ERR_INVALID_ARG;
+    return GLM_OK;
+}
+
 size_t mla_workspace(int n_q, int n_heads, int width) {
     const size_t parts = mla_parts(n_q, n_heads, width);
     return mla_acc_bytes(parts) + mla_ml_bytes(parts) + 256;
+}
+
+// Workspace of a fused step: the selection's (with its score rows), the attention's, the
+// attention's barrier counters, and a 256-byte status tail shared by every kernel of the step.
+struct StepLayout {
+    size_t idx, mla, ctr, total;
+};
+StepLayout step_layout(const glm_dsa_dims *dims, int n_q, int64_t ld, int width) {
+    StepLayout L;
+    const size_t idx = sel_bytes(n_q, ld) +
+                       align_up(static_cast<size_t>(n_q) * static_cast<size_t>(ld > 0 ? ld : 0) * sizeof(float), 256) + 256;
+    L.idx = 0;
+    L.mla = idx;
+    L.ctr = idx + mla_workspace(n_q, dims->n_heads, width);
+    L.total = L.ctr + align_up(static_cast<size_t>(n_q) * sizeof(unsigned), 256) + 256;
+    return L;
 }
 
 }  // namespace
@@ -109,12 +169,8 @@ int glm_last_cuda_error(void) { return g_last_cuda_error; }
 
 int glm_kv_store_int8(const glm_dsa_dims *dims, const void *latent, const int64_t *slots,
                       int64_t n, int8_t *cache, int64_t n_rows, void *stream) {
-    int rc = glm_check_dims(dims);
-    if (rc != GLM_OK) return rc;
-    if (n < 0 || n_rows < 0) return GLM_ERR_INVALID_ARG;
-    if (n == 0) return GLM_OK;
-    if (!latent || !slots || !cache) return GLM_ERR_INVALID_ARG;
-    if (!aligned(latent, 16) || !aligned(cache, 16) || !aligned(slots, 8)) return GLM_ERR_INVALID_ARG;
+    const int rc = check_store(dims, latent, slots, n, cache, n_rows);
+    if (rc != GLM_OK || n == 0) return rc;
     return cuda_status(glm::launch_store_int8(latent, slots, n, cache, n_rows,
                                               static_cast<cudaStream_t>(stream), num_sms()));
 }
@@ -124,17 +180,9 @@ int glm_kpool_build(const glm_dsa_dims *dims, const void *k, const void *gate, i
                     const int32_t *len, const int32_t *pool_begin, int32_t batch,
                     int32_t max_new_pools, float *pooled, int64_t ld_pools, int32_t *n_pools,
                     void *stream) {
-    int rc = glm_check_dims(dims);
-    if (rc != GLM_OK) return rc;
-    if (batch < 0 || max_new_pools < 0 || ld_tokens < 0 || ld_pools < 0) return GLM_ERR_INVALID_ARG;
-    if (!(ln_eps >= 0.0f)) return GLM_ERR_INVALID_ARG;
-    if (batch == 0) return GLM_OK;
-    if (!k || !gate || !ln_w || !ln_b || !pad || !len || !pooled) return GLM_ERR_INVALID_ARG;
-    if (!aligned(k, 16) || !aligned(gate, 16) || !aligned(ln_w, 16) || !aligned(ln_b, 16) ||
-        !aligned(pooled, 16) || !aligned(pad, 4) || !aligned(len, 4) ||
-        (pool_begin && !aligned(pool_begin, 4)) || (n_pools && !aligned(n_pools, 4)))
-        return GLM_ERR_INVALID_ARG;
-    if (static_cast<int64_t>(batch) * max_new_pools > (int64_t(1) << 40)) return GLM_ERR_INVALID_ARG;
+    const int rc = check_kpool(dims, k, gate, ld_tokens, ln_w, ln_b, ln_eps, pad, len, pool_begin, batch,
+                               max_new_pools, pooled, ld_pools, n_pools);
+    if (rc != GLM_OK || batch == 0) return rc;
     return cuda_status(glm::launch_kpool_build(k, gate, ld_tokens, ln_w, ln_b, ln_eps, pad, len,
                                                pool_begin, batch, max_new_pools, pooled, ld_pools,
                                                n_pools, static_cast<cudaStream_t>(stream), num_sms()));
@@ -154,12 +202,22 @@ size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
         case GLM_OP_SPARSE_MLA:
             if (width < 1 || width > 65536) return static_cast<size_t>(-1);
             return mla_workspace(n_q, dims->n_heads, width);
+        case GLM_OP_DECODE_STEP:
+            if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect || width < 1 || width > 65536)
+                return static_cast<size_t>(-1);
+            return step_layout(dims, n_q, max_pools, width).total;
         default:
             return static_cast<size_t>(-1);
     }
 }
 
 namespace {
+
+int enqueue_index_select(const void *q_idx, const float *w, const float *pooled, int64_t ld_pools,
+                         const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad, const int32_t *len,
+                         int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map, int64_t ld_slot,
+                         int32_t out_width, float *scores, int32_t *topk, int32_t *n_sel, int32_t *tok,
+                         int32_t *rows, void *workspace, int *status, bool zero, int sms, cudaStream_t st);
 
 // Checks shared by the two scoring + selection entry points; GLM_OK when the call may proceed.
 int check_index_args(const glm_dsa_dims *dims, const void *q_idx, const float *w, const float *pooled,
@@ -191,13 +249,27 @@ int run_index_select(const glm_dsa_dims *dims, const void *q_idx, const float *w
                      size_t ws_bytes, void *stream) {
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, n_q, ld_pools, select_k, 0);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
+    int *status = reinterpret_cast<int *>(static_cast<char *>(workspace) + need - 256);
+    return enqueue_index_select(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k, slot_map,
+                                ld_slot, out_width, scores, topk, n_sel, tok, rows, workspace, status, true,
+                                num_sms(), static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+namespace {
+
+// The fused index launch on a workspace laid out by sel_layout (+ the score rows); `zero`: also
+// enqueue the zeroing of the multi-CTA words (false when the caller has zeroed them already).
+int enqueue_index_select(const void *q_idx, const float *w, const float *pooled, int64_t ld_pools,
+                         const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad, const int32_t *len,
+                         int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map, int64_t ld_slot,
+                         int32_t out_width, float *scores, int32_t *topk, int32_t *n_sel, int32_t *tok,
+                         int32_t *rows, void *workspace, int *status, bool zero, int sms, cudaStream_t st) {
     const SelWs sw = sel_layout(workspace, n_q, ld_pools);
     char *ws = static_cast<char *>(workspace);
     float *sbuf = scores ? scores : reinterpret_cast<float *>(ws + sel_bytes(n_q, ld_pools));
-    int *status = reinterpret_cast<int *>(ws + need - 256);
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int sms = num_sms();
-    if (glm::index_select_ctas(n_q, ld_pools, sms) > 1) {
+    if (zero && glm::index_select_ctas(n_q, ld_pools, sms) > 1) {
         const int rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
         if (rc != GLM_OK) return rc;
     }
@@ -328,15 +400,8 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t 
                           int64_t n_rows, const int32_t *rows, int32_t n_q, int32_t width,
                           float sm_scale, void *out, float *lse, float *out_f32, void *workspace,
                           size_t ws_bytes, void *stream) {
-    int rc = glm_check_dims(dims);
-    if (rc != GLM_OK) return rc;
-    if (n_q < 0 || n_rows < 0 || width < 1 || width > 65536 || n_q > 65535) return GLM_ERR_INVALID_ARG;
-    if (!(sm_scale == sm_scale)) return GLM_ERR_INVALID_ARG;
-    if (n_q == 0) return GLM_OK;
-    if (!q || !rows || !out || (n_rows > 0 && !cache)) return GLM_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || (cache && !aligned(cache, 16)) || !aligned(rows, 4) || !aligned(out, 16) ||
-        (lse && !aligned(lse, 4)) || (out_f32 && !aligned(out_f32, 16)))
-        return GLM_ERR_INVALID_ARG;
+    int rc = check_mla(dims, q, cache, n_rows, rows, n_q, width, sm_scale, out, lse, out_f32);
+    if (rc != GLM_OK || n_q == 0) return rc;
     const int H = dims->n_heads;
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
@@ -349,9 +414,90 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t 
     int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = cuda_status(glm::launch_mla_split_tc(q, H, cache, n_rows, rows, n_q, width, sm_scale,
-                                              part_acc, part_ml, status, st));
+                                              part_acc, part_ml, status, st, glm::MlaCombineArgs{}));
     if (rc != GLM_OK) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32, lse, st));
+}
+
+int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *workspace, size_t ws_bytes,
+                        void *stream) {
+    if (a == nullptr) return GLM_ERR_INVALID_ARG;
+    int rc = check_store(dims, a->latent_dev, a->slots_dev, a->n_new, a->cache_dev, a->n_rows);
+    if (rc != GLM_OK) return rc;
+    rc = check_kpool(dims, a->k_dev, a->gate_dev, a->ld_tokens, a->ln_w_dev, a->ln_b_dev, a->ln_eps, a->pad_dev,
+                     a->len_dev, a->pool_begin_dev, a->batch, a->max_new_pools, a->pooled_dev, a->ld_pools, nullptr);
+    if (rc != GLM_OK) return rc;
+    rc = check_index_args(dims, a->q_idx_dev, a->w_dev, a->pooled_dev, a->ld_pools, a->q_seq_dev, a->q_pos_dev,
+                          a->pad_dev, a->len_dev, a->batch, a->n_q, a->select_k, a->scores_dev, a->topk_dev,
+                          a->n_sel_dev);
+    if (rc != GLM_OK) return rc;
+    if (a->out_width < 1 || a->ld_slot < 0 ||
+        static_cast<int64_t>(a->out_width) < static_cast<int64_t>(glm::kKpool) * a->select_k + glm::kKpool - 1)
+        return GLM_ERR_INVALID_ARG;
+    if (a->n_q > 0 && !a->rows_dev) return GLM_ERR_INVALID_ARG;   // the attention reads them
+    if ((a->slot_map_dev && !aligned(a->slot_map_dev, 8)) || (a->tok_dev && !aligned(a->tok_dev, 4)) ||
+        (a->rows_dev && !aligned(a->rows_dev, 4)))
+        return GLM_ERR_INVALID_ARG;
+    rc = check_mla(dims, a->q_dev, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width, a->sm_scale,
+                   a->out_dev, a->lse_dev, a->out_f32_dev);
+    if (rc != GLM_OK) return rc;
+    const StepLayout L = step_layout(dims, a->n_q, a->ld_pools, a->out_width);
+    if (workspace == nullptr || ws_bytes < L.total || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
+    char *ws = static_cast<char *>(workspace);
+    int *status = reinterpret_cast<int *>(ws + L.total - 256);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int sms = num_sms();
+    const bool idx_multi = a->n_q > 0 && glm::index_select_ctas(a->n_q, a->ld_pools, sms) > 1;
+    const bool mla_fused = a->n_q > 0 && glm::mla_combine_fits_in_kernel(a->n_q, a->out_width, sms);
+    const SelWs sw = sel_layout(ws + L.idx, a->n_q, a->ld_pools);
+    glm::StepPrepArgs p{};
+    p.latent = static_cast<const uint16_t *>(a->latent_dev);
+    p.slots = a->slots_dev;
+    p.n_new = a->n_new;
+    p.cache = a->cache_dev;
+    p.n_rows = a->n_rows;
+    p.k = static_cast<const uint16_t *>(a->k_dev);
+    p.gate = static_cast<const uint16_t *>(a->gate_dev);
+    p.ld_tokens = a->ld_tokens;
+    p.ln_w = a->ln_w_dev;
+    p.ln_b = a->ln_b_dev;
+    p.ln_eps = a->ln_eps;
+    p.pad = a->pad_dev;
+    p.len = a->len_dev;
+    p.pool_begin = a->pool_begin_dev;
+    p.batch = a->batch;
+    p.max_new_pools = a->max_new_pools;
+    p.pooled = a->pooled_dev;
+    p.ld_pools = a->ld_pools;
+    p.zero0 = reinterpret_cast<uint4 *>(sw.hist);
+    p.zero0_n16 = idx_multi ? static_cast<int64_t>(align_up(sw.zero_bytes, 16) / 16) : 0;
+    p.zero1 = reinterpret_cast<uint4 *>(ws + L.ctr);
+    p.zero1_n16 = mla_fused ? static_cast<int64_t>(align_up(static_cast<size_t>(a->n_q) * sizeof(unsigned), 16) / 16) : 0;
+    rc = cuda_status(glm::launch_step_prep(p, st));
+    if (rc != GLM_OK || a->n_q == 0) return rc;
+    rc = enqueue_index_select(a->q_idx_dev, a->w_dev, a->pooled_dev, a->ld_pools, a->q_seq_dev, a->q_pos_dev,
+                              a->pad_dev, a->len_dev, a->batch, a->n_q, a->select_k, a->slot_map_dev, a->ld_slot,
+                              a->out_width, a->scores_dev, a->topk_dev, a->n_sel_dev, a->tok_dev, a->rows_dev,
+                              ws + L.idx, status, false, sms, st);
+    if (rc != GLM_OK) return rc;
+    const int H = dims->n_heads;
+    const int chunk = glm::mla_tc_chunk();
+    const int n_chunks = (a->out_width + chunk - 1) / chunk;
+    const size_t parts = mla_parts(a->n_q, H, a->out_width);
+    float *part_acc = reinterpret_cast<float *>(ws + L.mla);
+    float *part_ml = reinterpret_cast<float *>(ws + L.mla + mla_acc_bytes(parts));
+    glm::MlaCombineArgs comb{};
+    if (mla_fused) {
+        comb.counter = reinterpret_cast<unsigned *>(ws + L.ctr);
+        comb.out = static_cast<uint16_t *>(a->out_dev);
+        comb.out_f32 = a->out_f32_dev;
+        comb.lse = a->lse_dev;
+    }
+    rc = cuda_status(glm::launch_mla_split_tc(a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
+                                              a->sm_scale, part_acc, part_ml, status, st, comb));
+    if (rc != GLM_OK || mla_fused) return rc;
+    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, n_chunks, a->out_dev, a->out_f32_dev,
+                                               a->lse_dev, st));
 }
 
 }  // extern "C"

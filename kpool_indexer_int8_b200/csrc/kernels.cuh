@@ -42,6 +42,33 @@ cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const floa
                                    const int32_t *pad, const int32_t *len, int batch, int n_q,
                                    float *scores, bool fill_invisible, const IxSelectArgs &sel,
                                    int *status, int num_sms, cudaStream_t stream);
+// The fused step's first kernel: store rows, build pools, zero two word ranges (16-byte units).
+struct StepPrepArgs {
+    const uint16_t *latent;
+    const int64_t *slots;
+    int64_t n_new;
+    int8_t *cache;
+    int64_t n_rows;
+    const uint16_t *k;
+    const uint16_t *gate;
+    int64_t ld_tokens;
+    const float *ln_w;
+    const float *ln_b;
+    float ln_eps;
+    const int32_t *pad;
+    const int32_t *len;
+    const int32_t *pool_begin;
+    int batch;
+    int max_new_pools;
+    float *pooled;
+    int64_t ld_pools;
+    uint4 *zero0;
+    int64_t zero0_n16;
+    uint4 *zero1;
+    int64_t zero1_n16;
+};
+cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream);
+
 cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32_t *q_seq,
                           const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
                           int n_q, int select_k, const int64_t *slot_map, int64_t ld_slot, int out_width,

@@ -7,7 +7,7 @@
 // normalises each token with two warp reductions (mean, then biased variance), mixes the four
 // slots with a per-channel softmax of the gates and stores 16 bytes of the fp32 pool row.
 // HBM-bound: 4 * (256 + 256) bytes read and 512 written per pool.
-#include "common.cuh"
+#include "append.cuh"
 
 namespace glm {
 
@@ -31,49 +31,8 @@ __global__ void __launch_bounds__(256) kpool_build_kernel(
     const int64_t items = static_cast<int64_t>(batch) * max_new_pools;
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-         it < items; it += warps_total) {
-        const int b = static_cast<int>(it / max_new_pools);
-        const int i = static_cast<int>(it % max_new_pools);
-        const int p = (pool_begin ? pool_begin[b] : 0) + i;
-        const int n_seq_pools = len[b] > 0 ? len[b] / kKpool : 0;
-        if (p < 0 || p >= n_seq_pools || p >= ld_pools) continue;
-        const int64_t t0 = static_cast<int64_t>(b) * ld_tokens + pad[b] + static_cast<int64_t>(p) * kKpool;
-        float y[kKpool][4], g[kKpool][4];
-#pragma unroll
-        for (int s = 0; s < kKpool; s++) {
-            const uint2 kv = reinterpret_cast<const uint2 *>(k + (t0 + s) * kIdxDim)[lane];
-            const uint2 gv = reinterpret_cast<const uint2 *>(gate + (t0 + s) * kIdxDim)[lane];
-            float x[4] = {__uint_as_float(kv.x << 16), __uint_as_float(kv.x & 0xffff0000u),
-                          __uint_as_float(kv.y << 16), __uint_as_float(kv.y & 0xffff0000u)};
-            g[s][0] = __uint_as_float(gv.x << 16);
-            g[s][1] = __uint_as_float(gv.x & 0xffff0000u);
-            g[s][2] = __uint_as_float(gv.y << 16);
-            g[s][3] = __uint_as_float(gv.y & 0xffff0000u);
-            const float mean = warp_sum((x[0] + x[1]) + (x[2] + x[3])) * (1.0f / kIdxDim);
-            float d0 = x[0] - mean, d1 = x[1] - mean, d2 = x[2] - mean, d3 = x[3] - mean;
-            const float var = warp_sum((d0 * d0 + d1 * d1) + (d2 * d2 + d3 * d3)) * (1.0f / kIdxDim);
-            const float inv = 1.0f / sqrtf(var + eps);
-            y[s][0] = d0 * inv * lw[0] + lb[0];
-            y[s][1] = d1 * inv * lw[1] + lb[1];
-            y[s][2] = d2 * inv * lw[2] + lb[2];
-            y[s][3] = d3 * inv * lw[3] + lb[3];
-        }
-        float out[4];
-#pragma unroll
-        for (int c = 0; c < 4; c++) {
-            float m = fmaxf(fmaxf(g[0][c], g[1][c]), fmaxf(g[2][c], g[3][c]));
-            float num = 0.0f, den = 0.0f;
-#pragma unroll
-            for (int s = 0; s < kKpool; s++) {
-                float e = expf(g[s][c] - m);
-                den += e;
-                num += e * y[s][c];
-            }
-            out[c] = num / den;
-        }
-        reinterpret_cast<float4 *>(pooled + (static_cast<int64_t>(b) * ld_pools + p) * kIdxDim)[lane] =
-            make_float4(out[0], out[1], out[2], out[3]);
-    }
+         it < items; it += warps_total)
+        kpool_build_item(k, gate, ld_tokens, lw, lb, eps, pad, len, pool_begin, max_new_pools, pooled, ld_pools, it);
 }
 
 cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_tokens,

@@ -1,0 +1,52 @@
+// step.cu -- the first kernel of a fused decode step: the int8 store of the new latent rows
+// ("GLM-5.3 Kernels" README, 'Included': titan_kv.store_int8), the build of the new pools
+// ("Module glm5next_dsa_ref", pool_states) and the zeroing of the step's cross-CTA counters, as
+// three independent groups of CTAs of one launch (one warp per row, one warp per pool, 16 bytes
+// per thread of zeros), so that the three short jobs overlap instead of following one another.
+#include "append.cuh"
+#include "kernels.cuh"
+
+namespace glm {
+
+constexpr int kPrepThreads = 256;
+constexpr int kPrepWarps = kPrepThreads / 32;
+
+__global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(StepPrepArgs a, int store_ctas, int pool_ctas) {
+    pdl_begin();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int cta = blockIdx.x;
+    if (cta < store_ctas) {
+        const int64_t row = static_cast<int64_t>(cta) * kPrepWarps + warp;
+        if (row < a.n_new) store_int8_row(a.latent, a.slots, row, a.cache, a.n_rows);
+        return;
+    }
+    cta -= store_ctas;
+    if (cta < pool_ctas) {
+        const int64_t it = static_cast<int64_t>(cta) * kPrepWarps + warp;
+        if (it >= static_cast<int64_t>(a.batch) * a.max_new_pools) return;
+        const float4 w4 = reinterpret_cast<const float4 *>(a.ln_w)[lane];
+        const float4 b4 = reinterpret_cast<const float4 *>(a.ln_b)[lane];
+        const float lw[4] = {w4.x, w4.y, w4.z, w4.w}, lb[4] = {b4.x, b4.y, b4.z, b4.w};
+        kpool_build_item(a.k, a.gate, a.ld_tokens, lw, lb, a.ln_eps, a.pad, a.len, a.pool_begin, a.max_new_pools,
+                         a.pooled, a.ld_pools, it);
+        return;
+    }
+    cta -= pool_ctas;
+    const int64_t i = static_cast<int64_t>(cta) * kPrepThreads + threadIdx.x;
+    if (i < a.zero0_n16) a.zero0[i] = make_uint4(0u, 0u, 0u, 0u);
+    else if (i - a.zero0_n16 < a.zero1_n16) a.zero1[i - a.zero0_n16] = make_uint4(0u, 0u, 0u, 0u);
+}
+
+cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream) {
+    const int64_t items = static_cast<int64_t>(a.batch) * a.max_new_pools;
+    const int store_ctas = static_cast<int>((a.n_new + kPrepWarps - 1) / kPrepWarps);
+    const int pool_ctas = static_cast<int>((items + kPrepWarps - 1) / kPrepWarps);
+    const int zero_ctas = static_cast<int>((a.zero0_n16 + a.zero1_n16 + kPrepThreads - 1) / kPrepThreads);
+    const int total = store_ctas + pool_ctas + zero_ctas;
+    if (total == 0) return cudaSuccess;
+    launch_pdl(step_prep_kernel, dim3(static_cast<unsigned>(total)), dim3(kPrepThreads), 0, stream, a, store_ctas,
+               pool_ctas);
+    return cudaGetLastError();
+}
+
+}  // namespace glm

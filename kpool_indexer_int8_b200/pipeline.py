@@ -7,8 +7,9 @@ topk_pools -> expand_selection -> masked attention):
     glm_kv_store_int8 -> glm_kpool_build -> glm_index_scores_topk -> glm_expand_selection
       -> glm_sparse_mla_decode
 
-A step runs the scoring, selection and expansion as one call (glm_index_topk_expand, one fused
-launch); the separate calls remain for checking each stage on its own. This module only owns device buffers (allocated with torch) and marshals them into the calls;
+A step runs as one call (glm_dsa_decode_step: the store, the pool build, the fused scoring +
+selection + expansion and the sparse attention in three or four kernels); run_stages issues the
+separate calls, for checking each stage on its own. This module only owns device buffers (allocated with torch) and marshals them into the calls;
 all arithmetic runs in the library's kernels.
 """
 from __future__ import annotations
@@ -18,9 +19,9 @@ from typing import Optional
 
 import torch
 
-from . import (GLM_OP_INDEX_SCORES_TOPK, GLM_OP_SPARSE_MLA, GLM_ROW_BYTES, glm_dsa_workspace_size,
-               glm_expand_selection, glm_index_scores_topk, glm_index_topk_expand, glm_kpool_build,
-               glm_kv_store_int8, glm_sparse_mla_decode, make_dims)
+from . import (GLM_OP_DECODE_STEP, GLM_OP_INDEX_SCORES_TOPK, GLM_OP_SPARSE_MLA, GLM_ROW_BYTES,
+               glm_dsa_decode_step, glm_dsa_workspace_size, glm_expand_selection, glm_index_scores_topk,
+               glm_index_topk_expand, glm_kpool_build, glm_kv_store_int8, glm_sparse_mla_decode, make_dims)
 
 LATENT = 512
 IDX_HEADS = 32
@@ -65,6 +66,7 @@ class DecodeBuffers:
     lse: torch.Tensor        # fp32 [n_q, Hm]
     ws_index: torch.Tensor   # uint8 workspace
     ws_mla: torch.Tensor     # uint8 workspace
+    ws_step: torch.Tensor    # uint8 workspace of the one-call step
     scores: Optional[torch.Tensor] = None  # fp32 [n_q, ld_pools] when requested
     out_f32: Optional[torch.Tensor] = None
 
@@ -77,6 +79,7 @@ def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_
     f = dict(device=device)
     ws_i = glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, n_q, ld_pools, select_k)
     ws_m = glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, width=out_width)
+    ws_s = glm_dsa_workspace_size(dims, GLM_OP_DECODE_STEP, n_q, ld_pools, select_k, out_width)
     return DecodeBuffers(
         dims=dims, select_k=select_k, out_width=out_width, sm_scale=sm_scale, ln_eps=ln_eps,
         cache=torch.zeros(n_rows, GLM_ROW_BYTES, dtype=torch.int8, **f),
@@ -105,6 +108,7 @@ def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_
         lse=torch.zeros(n_q, n_heads, dtype=torch.float32, **f),
         ws_index=torch.empty(max(ws_i, 1), dtype=torch.uint8, **f),
         ws_mla=torch.empty(max(ws_m, 1), dtype=torch.uint8, **f),
+        ws_step=torch.empty(max(ws_s, 1), dtype=torch.uint8, **f),
         scores=torch.empty(n_q, ld_pools, dtype=torch.float32, **f) if keep_scores else None,
         out_f32=torch.empty(n_q, n_heads, LATENT, dtype=torch.float32, **f) if keep_f32 else None,
     )
@@ -148,7 +152,18 @@ STAGES = (("store_int8", store), ("kpool_build", build_pools), ("index_topk_expa
           ("sparse_mla_decode", attend))
 
 
-def run_step(b: DecodeBuffers, stream=None) -> None:
-    """One whole step: every stage of the path, in order, on one stream."""
+def run_stages(b: DecodeBuffers, stream=None) -> None:
+    """One whole step as the separate calls, in order, on one stream."""
     for _, fn in STAGES:
         fn(b, stream=stream)
+
+
+def run_step(b: DecodeBuffers, stream=None) -> None:
+    """One whole step through the one-call entry point."""
+    glm_dsa_decode_step(b.dims, latent=b.new_latent, slots=b.new_slots, cache=b.cache, k=b.k, gate=b.gate,
+                        ln_w=b.ln_w, ln_b=b.ln_b, ln_eps=b.ln_eps, pad=b.pad, length=b.len,
+                        pool_begin=b.pool_begin, max_new_pools=b.max_new_pools, pooled=b.pooled, q_idx=b.q_idx,
+                        w=b.w, q_seq=b.q_seq, q_pos=b.q_pos, select_k=b.select_k, out_width=b.out_width,
+                        slot_map=b.slot_map, rows=b.rows, topk=b.topk, q=b.q, sm_scale=b.sm_scale, out=b.out,
+                        workspace=b.ws_step, n_sel=b.n_sel, tok=b.tok, scores=b.scores, lse=b.lse,
+                        out_f32=b.out_f32, stream=stream)

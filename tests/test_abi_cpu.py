@@ -3,6 +3,7 @@ arguments on the host before any CUDA call (so these run without a GPU)."""
 import ctypes as C
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -115,3 +116,35 @@ def test_index_and_mla_argument_checks():
     assert L.glm_topk_pools(FAKE, 16, FAKE, 1, 0, FAKE, None, None, 0, None) == kp.GLM_ERR_INVALID_ARG
     assert L.glm_kpool_build(d, FAKE, FAKE, 16, FAKE, FAKE, C.c_float(-1.0), FAKE, FAKE, None, 1, 1,
                              FAKE, 4, None, None) == kp.GLM_ERR_INVALID_ARG
+
+
+def test_step_struct_layout_matches_the_header(tmp_path):
+    # the ctypes mirror of glm_dsa_step must have the C compiler's field offsets and size
+    fields = [f for f, _ in kp.glm_dsa_step._fields_]
+    src = tmp_path / "layout.c"
+    src.write_text('#include <stddef.h>\n#include <stdio.h>\n#include "glm_dsa.h"\nint main(void) {\n' +
+                   "".join(f'    printf("%zu\\n", offsetof(glm_dsa_step, {f}));\n' for f in fields) +
+                   '    printf("%zu\\n", sizeof(glm_dsa_step));\n    return 0;\n}\n')
+    exe = tmp_path / "layout"
+    subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), str(src), "-o", str(exe)], check=True)
+    got = [int(x) for x in subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()]
+    want = [getattr(kp.glm_dsa_step, f).offset for f in fields] + [C.sizeof(kp.glm_dsa_step)]
+    assert got == want
+
+
+def test_step_argument_checks():
+    L = kp.lib
+    d = C.byref(kp.make_dims(64))
+    assert L.glm_dsa_decode_step(d, None, FAKE, 1 << 30, None) == kp.GLM_ERR_INVALID_ARG
+    a = kp.glm_dsa_step()                       # all counts zero, every pointer NULL
+    a.out_width, a.select_k, a.sm_scale = 2051, 512, 0.04
+    a.ld_pools = 16
+    assert L.glm_dsa_decode_step(d, C.byref(a), None, 0, None) == kp.GLM_ERR_WORKSPACE    # nothing else missing
+    a.out_width = 2050                         # below 4 * select_k + 3
+    assert L.glm_dsa_decode_step(d, C.byref(a), FAKE, 1 << 30, None) == kp.GLM_ERR_INVALID_ARG
+    a.out_width = 2051
+    a.n_new, a.latent_dev = 1, None             # a new row without its latent
+    assert L.glm_dsa_decode_step(d, C.byref(a), FAKE, 1 << 30, None) == kp.GLM_ERR_INVALID_ARG
+    a.n_new = 0
+    need = kp.glm_dsa_workspace_size(kp.make_dims(64), kp.GLM_OP_DECODE_STEP, 0, 16, 512, 2051)
+    assert L.glm_dsa_decode_step(d, C.byref(a), FAKE, need - 1, None) == kp.GLM_ERR_WORKSPACE

@@ -512,6 +512,44 @@ def test_decode_step_matches_oracle(cuda, wl):
     assert _check_chain(inp, b) <= max(1, len(inp.q_pos) // 10)
 
 
+@pytest.mark.parametrize("wl", [synth.PADDING_DECODE,
+                                synth.custom("batched_small2", (0, 0, 0, 0), (9000, 4099, 20000, 33),
+                                             n_heads=64, select_k=512, out_width=2176,
+                                             permute_slots=True, seed=37)])
+def test_one_call_step_equals_separate_calls(cuda, wl):
+    # glm_dsa_decode_step (fused kernels, in-kernel attention combine where it fits) against the
+    # separate entry points on the same inputs: identical integers, attention within rounding
+    inp = synth.generate(wl)
+    outs = []
+    for runner in (P.run_stages, P.run_step):
+        b = sdev.allocate_for(inp, cuda, keep_scores=True, keep_f32=True)
+        sdev.load(inp, b, build_prefix=True)
+        b.ws_step.fill_(0xA5)
+        b.ws_step[-256:].zero_()
+        runner(b)
+        torch.cuda.synchronize()
+        outs.append(b)
+    a, c = outs
+    assert int(c.ws_step[-256:-252].view(torch.int32).item()) == 0
+    for name in ("cache", "pooled", "scores", "topk", "n_sel", "tok", "rows"):
+        assert torch.equal(getattr(a, name), getattr(c, name)), name
+    assert np.allclose(np_(c.out_f32), np_(a.out_f32), rtol=1e-5, atol=1e-6)   # merge order only
+    assert_bf16_is_rounded_f32(np_(c.out.view(torch.int16)).view(np.uint16), np_(c.out_f32))
+    la, lc = np_(a.lse), np_(c.lse)
+    assert np.allclose(la, lc, atol=1e-4, rtol=0)
+
+
+def test_separate_calls_match_oracle(cuda):
+    inp = synth.generate(synth.PADDING_DECODE)
+    b = sdev.allocate_for(inp, cuda, keep_scores=True, keep_f32=True)
+    sdev.load(inp, b, build_prefix=True)
+    for t in (b.topk, b.tok, b.rows):
+        t.fill_(4242)
+    P.run_stages(b)
+    torch.cuda.synchronize()
+    assert _check_chain(inp, b) <= 1
+
+
 def test_long_decode_full_size(cuda):
     # the benchmark's workload and launch configuration: 262,144-token context, 65,536 pools
     inp = synth.generate(synth.LONG_DECODE)
