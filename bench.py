@@ -37,11 +37,9 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 def kernel_launches_per_step(wl, num_sms: int) -> int:
-    """Kernels of one glm_dsa_decode_step: store + pool build + zeroing, scores + top-k + expansion,
-    MLA split (with the combine in-kernel when every split CTA is resident at once), else + combine."""
-    n_chunks = (wl.out_width + 63) // 64
-    return 3 if wl.n_queries * n_chunks <= num_sms else 4
-L2_BYTES = 126 * 1024 * 1024
+    """Kernels of one glm_dsa_decode_step: store + pool build + zeroing of the selection words,
+    scores + top-k + expansion, MLA split, MLA combine."""
+    return 4
 
 
 def algorithmic_bytes(inp) -> dict:

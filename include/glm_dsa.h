@@ -325,9 +325,9 @@ typedef struct glm_dsa_step {
 /*
  * One decode (or prefill-chunk) step: glm_kv_store_int8, glm_kpool_build, glm_index_topk_expand
  * and glm_sparse_mla_decode on the same stream, with the same results as those four calls in
- * that order. It runs as three kernels (four when the attention does not fit one wave of CTAs):
- * the store, the pool build and the zeroing of the step's counters share the first; the sparse
- * attention merges its split-KV partials in-kernel when all of its CTAs are resident at once.
+ * that order. It runs as four kernels: the store, the pool build and the zeroing of the step's
+ * counters share the first; then the fused scoring + selection + expansion; then the split and
+ * the combine of the sparse attention.
  *   workspace_dev / ws_bytes: >= glm_dsa_workspace_size(dims, GLM_OP_DECODE_STEP, n_q, ld_pools,
  *               select_k, out_width), 256-byte aligned, contents on entry ignored. Its last 256
  *               bytes start with a status word set nonzero when a wait gave up (outputs invalid;

@@ -123,10 +123,10 @@ size_t mla_workspace(int n_q, int n_heads, int width) {
     return mla_acc_bytes(parts) + mla_ml_bytes(parts) + 256;
 }
 
-// Workspace of a fused step: the selection's (with its score rows), the attention's, the
-// attention's barrier counters, and a 256-byte status tail shared by every kernel of the step.
+// Workspace of a fused step: the selection's (with its score rows), the attention's, and a
+// 256-byte status tail shared by every kernel of the step.
 struct StepLayout {
-    size_t idx, mla, ctr, total;
+    size_t idx, mla, total;
 };
 StepLayout step_layout(const glm_dsa_dims *dims, int n_q, int64_t ld, int width) {
     StepLayout L;
@@ -134,8 +134,7 @@ StepLayout step_layout(const glm_dsa_dims *dims, int n_q, int64_t ld, int width)
                        align_up(static_cast<size_t>(n_q) * static_cast<size_t>(ld > 0 ? ld : 0) * sizeof(float), 256) + 256;
     L.idx = 0;
     L.mla = idx;
-    L.ctr = idx + mla_workspace(n_q, dims->n_heads, width);
-    L.total = L.ctr + align_up(static_cast<size_t>(n_q) * sizeof(unsigned), 256) + 256;
+    L.total = idx + mla_workspace(n_q, dims->n_heads, width) + 256;
     return L;
 }
 
@@ -414,7 +413,7 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t 
     int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = cuda_status(glm::launch_mla_split_tc(q, H, cache, n_rows, rows, n_q, width, sm_scale,
-                                              part_acc, part_ml, status, st, glm::MlaCombineArgs{}));
+                                              part_acc, part_ml, status, st));
     if (rc != GLM_OK) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32, lse, st));
 }
@@ -448,7 +447,6 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int sms = num_sms();
     const bool idx_multi = a->n_q > 0 && glm::index_select_ctas(a->n_q, a->ld_pools, sms) > 1;
-    const bool mla_fused = a->n_q > 0 && glm::mla_combine_fits_in_kernel(a->n_q, a->out_width, sms);
     const SelWs sw = sel_layout(ws + L.idx, a->n_q, a->ld_pools);
     glm::StepPrepArgs p{};
     p.latent = static_cast<const uint16_t *>(a->latent_dev);
@@ -469,10 +467,8 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     p.max_new_pools = a->max_new_pools;
     p.pooled = a->pooled_dev;
     p.ld_pools = a->ld_pools;
-    p.zero0 = reinterpret_cast<uint4 *>(sw.hist);
-    p.zero0_n16 = idx_multi ? static_cast<int64_t>(align_up(sw.zero_bytes, 16) / 16) : 0;
-    p.zero1 = reinterpret_cast<uint4 *>(ws + L.ctr);
-    p.zero1_n16 = mla_fused ? static_cast<int64_t>(align_up(static_cast<size_t>(a->n_q) * sizeof(unsigned), 16) / 16) : 0;
+    p.zero = reinterpret_cast<uint4 *>(sw.hist);
+    p.zero_n16 = idx_multi ? static_cast<int64_t>(align_up(sw.zero_bytes, 16) / 16) : 0;
     rc = cuda_status(glm::launch_step_prep(p, st));
     if (rc != GLM_OK || a->n_q == 0) return rc;
     rc = enqueue_index_select(a->q_idx_dev, a->w_dev, a->pooled_dev, a->ld_pools, a->q_seq_dev, a->q_pos_dev,
@@ -486,16 +482,9 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     const size_t parts = mla_parts(a->n_q, H, a->out_width);
     float *part_acc = reinterpret_cast<float *>(ws + L.mla);
     float *part_ml = reinterpret_cast<float *>(ws + L.mla + mla_acc_bytes(parts));
-    glm::MlaCombineArgs comb{};
-    if (mla_fused) {
-        comb.counter = reinterpret_cast<unsigned *>(ws + L.ctr);
-        comb.out = static_cast<uint16_t *>(a->out_dev);
-        comb.out_f32 = a->out_f32_dev;
-        comb.lse = a->lse_dev;
-    }
     rc = cuda_status(glm::launch_mla_split_tc(a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
-                                              a->sm_scale, part_acc, part_ml, status, st, comb));
-    if (rc != GLM_OK || mla_fused) return rc;
+                                              a->sm_scale, part_acc, part_ml, status, st));
+    if (rc != GLM_OK) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, n_chunks, a->out_dev, a->out_f32_dev,
                                                a->lse_dev, st));
 }

@@ -42,7 +42,7 @@ cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const floa
                                    const int32_t *pad, const int32_t *len, int batch, int n_q,
                                    float *scores, bool fill_invisible, const IxSelectArgs &sel,
                                    int *status, int num_sms, cudaStream_t stream);
-// The fused step's first kernel: store rows, build pools, zero two word ranges (16-byte units).
+// The fused step's first kernel: store rows, build pools, zero a word range (16-byte units).
 struct StepPrepArgs {
     const uint16_t *latent;
     const int64_t *slots;
@@ -62,10 +62,8 @@ struct StepPrepArgs {
     int max_new_pools;
     float *pooled;
     int64_t ld_pools;
-    uint4 *zero0;
-    int64_t zero0_n16;
-    uint4 *zero1;
-    int64_t zero1_n16;
+    uint4 *zero;
+    int64_t zero_n16;
 };
 cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream);
 

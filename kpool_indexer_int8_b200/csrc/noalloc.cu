@@ -84,7 +84,7 @@ extern "C" int glm_sparse_mla_decode_noalloc(const glm_dsa_dims *dims, const voi
     rc = noalloc_cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st));
     if (rc != GLM_OK) return rc;
     rc = noalloc_cuda_status(glm::launch_mla_split_tc(q, H, cache, n_rows, rows, n_q, width, sm_scale,
-                                                      part_acc, part_ml, status, st, glm::MlaCombineArgs{}));
+                                                      part_acc, part_ml, status, st));
     if (rc != GLM_OK) return rc;
     return noalloc_cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32,
                                                        lse, st));

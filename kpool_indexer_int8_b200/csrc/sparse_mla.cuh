@@ -11,20 +11,9 @@ namespace glm {
 //   part_acc fp32 [n_q][n_chunks][n_heads][512], part_ml fp32 [n_q][n_chunks][n_heads][2].
 int mla_tc_chunk();
 
-// In-kernel combine of a single-wave split (all n_q * n_chunks CTAs resident): counter[n] (zero at
-// launch) is the grid barrier of query n; the outputs are written by the split kernel itself.
-// counter == nullptr: the split only writes the partials (the combine kernel merges them).
-struct MlaCombineArgs {
-    unsigned *counter;   // [n_q]
-    uint16_t *out;       // bf16 [n_q][n_heads][512]
-    float *out_f32;      // or null
-    float *lse;          // or null
-};
-bool mla_combine_fits_in_kernel(int n_q, int width, int num_sms);
 cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
                                 const int32_t *rows, int n_q, int width, float sm_scale,
-                                float *part_acc, float *part_ml, int *status, cudaStream_t stream,
-                                const MlaCombineArgs &comb);
+                                float *part_acc, float *part_ml, int *status, cudaStream_t stream);
 cudaError_t launch_mla_combine(const float *part_acc, const float *part_ml, int n_q, int n_heads,
                                int n_chunks, void *out, float *out_f32, float *lse,
                                cudaStream_t stream);

@@ -27,7 +27,6 @@
 // frees its tensor memory and exits.
 #include "common.cuh"
 #include "sparse_mla.cuh"
-#include "select.cuh"
 #include "tc.cuh"
 
 namespace glm {
@@ -60,102 +59,11 @@ __device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w, int shift) {
 
 __device__ __forceinline__ uint16_t bf16_rn_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 
-// In-kernel combine (single-wave grids): after every chunk of query n has written its partial,
-// the chunk CTAs meet at a grid barrier and CTA c merges output columns [per c, per (c + 1)) of the
-// query's flattened [head][512] output (as float4 columns) with the rule of the combine kernel:
-// M = max m, weights e^{m - M}, L = sum l e^{m - M}, out = sum e^{m - M} acc / L, lse = M + log L.
-// Shared memory (the operand buffers, free by now) holds each covered head's weights.
-__device__ __noinline__ void combine_in_kernel(const float *__restrict__ part_acc, const float *__restrict__ part_ml,
-                                               int n_heads, int n_chunks, const MlaCombineArgs comb,
-                                               int *__restrict__ status, unsigned char *smem) {
-    const int n = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    unsigned *go = reinterpret_cast<unsigned *>(smem);
-    __syncthreads();
-    if (tid == 0) {
-        const bool ok = grid_barrier(&comb.counter[n], n_chunks);
-        *go = ok ? 1u : 0u;
-        if (!ok) atomicOr(status, 8);
-    }
-    __syncthreads();
-    if (*go == 0u) return;
-    constexpr int kCols = kLatent / 4;
-    const int total = n_heads * kCols, per = (total + n_chunks - 1) / n_chunks;
-    const int f0 = min(total, c * per), f1 = min(total, f0 + per);
-    if (f0 >= f1) return;
-    const int h0 = f0 / kCols, nh = (f1 - 1) / kCols - h0 + 1;
-    float *wts = reinterpret_cast<float *>(smem + 16);            // [nh][n_chunks] m, then weight
-    float *ls = wts + nh * n_chunks;                              // [nh][n_chunks] l
-    float *stat = ls + nh * n_chunks;                             // [nh][2] M, L
-    const int64_t qb = static_cast<int64_t>(n) * n_chunks;
-    for (int i = tid; i < nh * n_chunks; i += blockDim.x) {
-        const int hh = i / n_chunks, cc = i % n_chunks;
-        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(part_ml) + (qb + cc) * n_heads + h0 + hh);
-        wts[i] = ml.y > 0.0f ? ml.x : -INFINITY;
-        ls[i] = ml.y;
-    }
-    __syncthreads();
-    for (int hh = warp; hh < nh; hh += blockDim.x >> 5) {   // one warp per covered head
-        float mx = -INFINITY;
-        for (int cc = lane; cc < n_chunks; cc += 32) mx = fmaxf(mx, wts[hh * n_chunks + cc]);
-        mx = warp_max(mx);
-        float L = 0.0f;
-        for (int cc = lane; cc < n_chunks; cc += 32) {
-            const float m = wts[hh * n_chunks + cc];
-            const float wc = (m == -INFINITY || mx == -INFINITY) ? 0.0f : expf(m - mx);
-            wts[hh * n_chunks + cc] = wc;
-            L = fmaf(ls[hh * n_chunks + cc], wc, L);
-        }
-        L = warp_sum(L);
-        if (lane == 0) { stat[2 * hh] = mx; stat[2 * hh + 1] = L; }
-    }
-    __syncthreads();
-    for (int f = f0 + tid; f < f1; f += blockDim.x) {
-        const int h = f / kCols, col = f % kCols, hh = h - h0;
-        const float *w = wts + hh * n_chunks;
-        float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-        int cc = 0;
-        for (; cc + 8 <= n_chunks; cc += 8) {
-            float4 v[8];
-#pragma unroll
-            for (int u = 0; u < 8; u++)
-                v[u] = w[cc + u] > 0.0f ? __ldcg(reinterpret_cast<const float4 *>(part_acc + ((qb + cc + u) * n_heads + h) * kLatent) + col)
-                                        : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int u = 0; u < 8; u++) {
-                const float wc = w[cc + u];
-                a.x = fmaf(wc, v[u].x, a.x);
-                a.y = fmaf(wc, v[u].y, a.y);
-                a.z = fmaf(wc, v[u].z, a.z);
-                a.w = fmaf(wc, v[u].w, a.w);
-            }
-        }
-        for (; cc < n_chunks; cc++) {
-            const float wc = w[cc];
-            if (!(wc > 0.0f)) continue;
-            const float4 v = __ldcg(reinterpret_cast<const float4 *>(part_acc + ((qb + cc) * n_heads + h) * kLatent) + col);
-            a.x = fmaf(wc, v.x, a.x);
-            a.y = fmaf(wc, v.y, a.y);
-            a.z = fmaf(wc, v.z, a.z);
-            a.w = fmaf(wc, v.w, a.w);
-        }
-        const float L = stat[2 * hh + 1];
-        const float inv = L > 0.0f ? 1.0f / L : 0.0f;
-        const float o[4] = {a.x * inv, a.y * inv, a.z * inv, a.w * inv};
-        const int64_t ob = (static_cast<int64_t>(n) * n_heads + h) * kLatent + 4 * col;
-        const uint32_t lo = static_cast<uint32_t>(bf16_rn_bits(o[0])) | (static_cast<uint32_t>(bf16_rn_bits(o[1])) << 16);
-        const uint32_t hi = static_cast<uint32_t>(bf16_rn_bits(o[2])) | (static_cast<uint32_t>(bf16_rn_bits(o[3])) << 16);
-        *reinterpret_cast<uint2 *>(comb.out + ob) = make_uint2(lo, hi);
-        if (comb.out_f32) *reinterpret_cast<float4 *>(comb.out_f32 + ob) = make_float4(o[0], o[1], o[2], o[3]);
-        if (comb.lse && col == 0)
-            comb.lse[static_cast<int64_t>(n) * n_heads + h] = L > 0.0f ? stat[2 * hh] + logf(L) : -INFINITY;
-    }
-}
-
 template <int M>
 __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
     const uint16_t *__restrict__ q, int n_heads, const int8_t *__restrict__ cache, int64_t n_rows,
     const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks,
-    float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status, MlaCombineArgs comb) {
+    float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status) {
     pdl_begin();
     using Lay = TcLayout<M>;
     extern __shared__ __align__(128) unsigned char smem[];
@@ -187,7 +95,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
             part_ml[2 * (ml_base + h)] = -INFINITY;
             part_ml[2 * (ml_base + h) + 1] = 0.0f;
         }
-        if (comb.counter) combine_in_kernel(part_acc, part_ml, n_heads, n_chunks, comb, status, smem);
         return;
     }
     if (warp == 0) {
@@ -386,40 +293,32 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 512);
     }
-    if (comb.counter) combine_in_kernel(part_acc, part_ml, n_heads, n_chunks, comb, status, smem);
 }
 
 int mla_tc_chunk() { return kTcRows; }
 
 cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
                                 const int32_t *rows, int n_q, int width, float sm_scale,
-                                float *part_acc, float *part_ml, int *status, cudaStream_t stream,
-                                const MlaCombineArgs &comb) {
+                                float *part_acc, float *part_ml, int *status, cudaStream_t stream) {
     const int n_chunks = (width + kTcRows - 1) / kTcRows;
     dim3 grid(n_chunks, n_q);
-    const bool coop = comb.counter != nullptr;   // the in-kernel combine waits on its grid
     cudaError_t e;
     if (n_heads <= 64) {
         const int smem = TcLayout<64>::kBytes;
         e = cudaFuncSetAttribute(mla_split_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        e = launch_pdl_coop(mla_split_tc_kernel<64>, dim3(grid), dim3(kTcThreads), smem, stream, coop,
-                            static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
-                            part_acc, part_ml, status, comb);
+        e = launch_pdl(mla_split_tc_kernel<64>, dim3(grid), dim3(kTcThreads), smem, stream,
+                       static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
+                       part_acc, part_ml, status);
     } else {
         const int smem = TcLayout<128>::kBytes;
         e = cudaFuncSetAttribute(mla_split_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
-        e = launch_pdl_coop(mla_split_tc_kernel<128>, dim3(grid), dim3(kTcThreads), smem, stream, coop,
-                            static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
-                            part_acc, part_ml, status, comb);
+        e = launch_pdl(mla_split_tc_kernel<128>, dim3(grid), dim3(kTcThreads), smem, stream,
+                       static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
+                       part_acc, part_ml, status);
     }
     return e != cudaSuccess ? e : cudaGetLastError();
-}
-
-bool mla_combine_fits_in_kernel(int n_q, int width, int num_sms) {
-    const long long ctas = static_cast<long long>(n_q) * ((width + kTcRows - 1) / kTcRows);
-    return ctas <= num_sms && (width + kTcRows - 1) / kTcRows <= kMaxSelCtas;
 }
 
 }  // namespace glm

@@ -33,15 +33,14 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(StepPrepArgs a,
     }
     cta -= pool_ctas;
     const int64_t i = static_cast<int64_t>(cta) * kPrepThreads + threadIdx.x;
-    if (i < a.zero0_n16) a.zero0[i] = make_uint4(0u, 0u, 0u, 0u);
-    else if (i - a.zero0_n16 < a.zero1_n16) a.zero1[i - a.zero0_n16] = make_uint4(0u, 0u, 0u, 0u);
+    if (i < a.zero_n16) a.zero[i] = make_uint4(0u, 0u, 0u, 0u);
 }
 
 cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream) {
     const int64_t items = static_cast<int64_t>(a.batch) * a.max_new_pools;
     const int store_ctas = static_cast<int>((a.n_new + kPrepWarps - 1) / kPrepWarps);
     const int pool_ctas = static_cast<int>((items + kPrepWarps - 1) / kPrepWarps);
-    const int zero_ctas = static_cast<int>((a.zero0_n16 + a.zero1_n16 + kPrepThreads - 1) / kPrepThreads);
+    const int zero_ctas = static_cast<int>((a.zero_n16 + kPrepThreads - 1) / kPrepThreads);
     const int total = store_ctas + pool_ctas + zero_ctas;
     if (total == 0) return cudaSuccess;
     launch_pdl(step_prep_kernel, dim3(static_cast<unsigned>(total)), dim3(kPrepThreads), 0, stream, a, store_ctas,

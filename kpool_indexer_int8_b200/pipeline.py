@@ -8,7 +8,7 @@ topk_pools -> expand_selection -> masked attention):
       -> glm_sparse_mla_decode
 
 A step runs as one call (glm_dsa_decode_step: the store, the pool build, the fused scoring +
-selection + expansion and the sparse attention in three or four kernels); run_stages issues the
+selection + expansion and the sparse attention in four kernels); run_stages issues the
 separate calls, for checking each stage on its own. This module only owns device buffers (allocated with torch) and marshals them into the calls;
 all arithmetic runs in the library's kernels.
 """
