@@ -160,8 +160,10 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx_dev, const
  * slot_map_dev int64 [batch, ld_slot] or NULL, tok_dev / rows_dev int32 [n_q, out_width], at
  * least one of them non-NULL, out_width >= 4 * select_k + 3). Every output equals what the two
  * separate calls produce. The workspace is that of GLM_OP_INDEX_SCORES_TOPK.
- * When the selection of a query spans several CTAs they meet at a grid barrier (the launch is
- * cooperative); a wait that gives up sets the status word nonzero and leaves the outputs invalid.
+ * When the selection of a query spans several CTAs they meet at a grid barrier: the launch sizes
+ * its grid to at most one CTA per SM and needs every CTA resident at once (a GPU shared with
+ * other concurrent work that holds SMs indefinitely breaks that); a wait that gives up sets the
+ * status word nonzero and leaves the outputs invalid.
  */
 int glm_index_topk_expand(const glm_dsa_dims *dims, const void *q_idx_dev, const float *w_dev,
                           const float *pooled_dev, int64_t ld_pools, const int32_t *q_seq_dev,

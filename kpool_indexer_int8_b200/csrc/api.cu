@@ -216,7 +216,8 @@ int enqueue_index_select(const void *q_idx, const float *w, const float *pooled,
                          const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad, const int32_t *len,
                          int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map, int64_t ld_slot,
                          int32_t out_width, float *scores, int32_t *topk, int32_t *n_sel, int32_t *tok,
-                         int32_t *rows, void *workspace, int *status, bool zero, int sms, cudaStream_t st);
+                         int32_t *rows, void *workspace, int *status, bool zero, int sms, cudaStream_t st,
+                         const int32_t *new_pool_begin = nullptr, int new_pools = -1);
 
 // Checks shared by the two scoring + selection entry points; GLM_OK when the call may proceed.
 int check_index_args(const glm_dsa_dims *dims, const void *q_idx, const float *w, const float *pooled,
@@ -264,7 +265,8 @@ int enqueue_index_select(const void *q_idx, const float *w, const float *pooled,
                          const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad, const int32_t *len,
                          int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map, int64_t ld_slot,
                          int32_t out_width, float *scores, int32_t *topk, int32_t *n_sel, int32_t *tok,
-                         int32_t *rows, void *workspace, int *status, bool zero, int sms, cudaStream_t st) {
+                         int32_t *rows, void *workspace, int *status, bool zero, int sms, cudaStream_t st,
+                         const int32_t *new_pool_begin, int new_pools) {
     const SelWs sw = sel_layout(workspace, n_q, ld_pools);
     char *ws = static_cast<char *>(workspace);
     float *sbuf = scores ? scores : reinterpret_cast<float *>(ws + sel_bytes(n_q, ld_pools));
@@ -288,6 +290,9 @@ int enqueue_index_select(const void *q_idx, const float *w, const float *pooled,
     sel.out_width = out_width;
     sel.tok = tok;
     sel.rows = rows;
+    sel.early = new_pools >= 0 ? 1 : 0;   // new_pools < 0: wait for the preceding kernel at the start
+    sel.new_pool_begin = new_pool_begin;
+    sel.new_pools = new_pools >= 0 ? new_pools : 0;
     return cuda_status(glm::launch_index_select_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch,
                                                    n_q, sbuf, scores != nullptr, sel, status, sms, st));
 }
@@ -474,7 +479,8 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     rc = enqueue_index_select(a->q_idx_dev, a->w_dev, a->pooled_dev, a->ld_pools, a->q_seq_dev, a->q_pos_dev,
                               a->pad_dev, a->len_dev, a->batch, a->n_q, a->select_k, a->slot_map_dev, a->ld_slot,
                               a->out_width, a->scores_dev, a->topk_dev, a->n_sel_dev, a->tok_dev, a->rows_dev,
-                              ws + L.idx, status, false, sms, st);
+                              ws + L.idx, status, false, sms, st, a->pool_begin_dev,
+                              a->batch > 0 ? a->max_new_pools : 0);
     if (rc != GLM_OK) return rc;
     const int H = dims->n_heads;
     const int chunk = glm::mla_tc_chunk();
@@ -483,7 +489,7 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     float *part_acc = reinterpret_cast<float *>(ws + L.mla);
     float *part_ml = reinterpret_cast<float *>(ws + L.mla + mla_acc_bytes(parts));
     rc = cuda_status(glm::launch_mla_split_tc(a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
-                                              a->sm_scale, part_acc, part_ml, status, st));
+                                              a->sm_scale, part_acc, part_ml, status, st, true));
     if (rc != GLM_OK) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, n_chunks, a->out_dev, a->out_f32_dev,
                                                a->lse_dev, st));

@@ -18,8 +18,8 @@
 //     global memory and, when the range is short enough, to shared memory), and its top-11-bit
 //     key digit counted in the CTA's histogram.
 // Phase 2, selection (select.cuh): with G > 1 the CTA histograms are summed in global memory and
-// the G CTAs of a query meet at a grid barrier (the launch is cooperative, so all CTAs are
-// resident; the wait is bounded); every CTA then classifies its own scores against the boundary
+// the G CTAs of a query meet at a grid barrier (all CTAs are resident: at most one per SM; the wait
+// is bounded); every CTA then classifies its own scores against the boundary
 // bin, appends them to the query's global lists, and the last CTA to finish (ticket) completes
 // the selection, sorts it, and writes the top-k row, n_sel and the expanded token / row indices.
 // With G = 1 the one CTA does all of it on chip.
@@ -124,7 +124,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_select_tc_kernel(
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ pad,
     const int32_t *__restrict__ len, int batch, float *__restrict__ scores, int fill_invisible,
     IxSelectArgs sel, int *__restrict__ status) {
-    pdl_begin();
+    if (sel.early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    else pdl_begin();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
     unsigned char *terms = smem + IxLayout::kTerms;
@@ -142,6 +143,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_select_tc_kernel(
     const bool valid_b = b >= 0 && b < batch;
     const int pb = valid_b ? pad[b] : 0, seq_len = valid_b ? len[b] : 0, qp = q_pos[n];
     const int n_vis = valid_b ? visible_pools(pb, seq_len, qp, ld_pools) : 0;
+    // pools the preceding kernel may still be writing (early mode): [first_new, first_new + new_pools)
+    const int first_new = (sel.early && valid_b) ? (sel.new_pool_begin ? max(0, sel.new_pool_begin[b]) : 0) : 0;
     float *srow = scores + static_cast<int64_t>(n) * ld_pools;
     const bool select = sel.topk != nullptr;
     const bool multi = select && G > 1;
@@ -155,6 +158,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_select_tc_kernel(
         for (int64_t i = f0 + tid; i < f1; i += kIxThreads) srow[i] = -INFINITY;
     }
     if (n_vis == 0) {   // nothing to score or select: CTA 0 writes the empty outputs
+        if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");
         if (select && g == 0) write_outputs(sel, n, b, valid_b, pb, seq_len, qp, 0u, s);
         return;
     }
@@ -204,8 +208,16 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_select_tc_kernel(
         // ---------------- producer ----------------
         if (lane == 0) {
             const uint32_t stage_addr = tc::smem_addr(stage);
+            bool waited = !sel.early;
             for (int c = 0; c < n_chunks; c++) {
                 const int slot = c % kIxStages;
+                const int c0 = lo + c * kIxChunk;
+                if (!waited && c0 + kIxChunk > first_new && c0 < first_new + sel.new_pools) {
+                    // this chunk holds a pool the preceding kernel writes: wait for it first
+                    asm volatile("griddepcontrol.wait;" ::: "memory");
+                    asm volatile("fence.proxy.async.global;" ::: "memory");
+                    waited = true;
+                }
                 if (c >= kIxStages && !tc::mbar_wait(bar(kBarStEmpty + slot), ((c / kIxStages) - 1) & 1, kIxWaitLimit))
                     ok = false;
                 const uint32_t bytes = static_cast<uint32_t>(min(kIxChunk, hi - lo - c * kIxChunk)) * kIdxDim * 4;
@@ -311,12 +323,14 @@ __global__ void __launch_bounds__(kIxThreads, 1) index_select_tc_kernel(
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 64);
     }
+    if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // before touching the zeroed words
     if (multi) {   // this CTA's histogram into the query's
         unsigned *gh = sel.ghist + static_cast<int64_t>(n) * kHistBins;
         for (int i = tid; i < kHistBins; i += kIxThreads)
             if (hist[i]) atomicAdd(&gh[i], hist[i]);
     }
     }   // lo < hi
+    if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // (CTAs without a score range)
     if (!select) return;
 
     // ---------------- phase 2: selection (every MMA and bulk copy of this CTA has completed) ----------------
@@ -396,10 +410,14 @@ cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const floa
     const int smem = IxLayout::kAlloc;
     cudaError_t e = cudaFuncSetAttribute(index_select_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    const bool coop = sel.topk != nullptr && G > 1;
-    e = launch_pdl_coop(index_select_tc_kernel, dim3(G, n_q), dim3(kIxThreads), smem, stream, coop,
-                        static_cast<const uint16_t *>(q_idx), w, pooled, ld_pools, q_seq, q_pos, pad, len,
-                        batch, scores, fill_invisible ? 1 : 0, sel, status);
+    // No cooperative attribute: a cooperative grid cannot start under programmatic dependent launch
+    // before its predecessor ends, which would forfeit the early streaming. Co-residency of the
+    // grid barrier's CTAs holds by construction: G * n_q <= the SM count at one CTA per SM (the
+    // shared memory allows no second), and a later kernel of the stream can only launch once every
+    // CTA of this one has started. The wait is bounded and reports through the status word.
+    e = launch_pdl(index_select_tc_kernel, dim3(G, n_q), dim3(kIxThreads), smem, stream,
+                   static_cast<const uint16_t *>(q_idx), w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, scores,
+                   fill_invisible ? 1 : 0, sel, status);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -35,6 +35,12 @@ struct IxSelectArgs {
     int out_width;
     int32_t *tok;                  // [n_q][out_width] or null
     int32_t *rows;                 // [n_q][out_width] or null
+    // early != 0 (one-call step): the preceding kernel writes only pooled rows [new_pool_begin[b],
+    // + new_pools) of each sequence b (plus buffers this kernel does not read before it waits), so
+    // the kernel streams every other pooled key before waiting for it
+    int early;
+    const int32_t *new_pool_begin; // [batch] or null (= 0)
+    int new_pools;
 };
 int index_select_ctas(int n_q, int64_t ld_pools, int num_sms);
 cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const float *pooled,

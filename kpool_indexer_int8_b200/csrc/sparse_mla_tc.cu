@@ -63,8 +63,11 @@ template <int M>
 __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
     const uint16_t *__restrict__ q, int n_heads, const int8_t *__restrict__ cache, int64_t n_rows,
     const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks,
-    float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status) {
-    pdl_begin();
+    float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status, int early_q) {
+    // early_q: the query block is an input no preceding kernel writes (the one-call step), so it is
+    // staged before waiting for the preceding kernel; only the row indices wait for it
+    if (early_q) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    else pdl_begin();
     using Lay = TcLayout<M>;
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *Qs = smem + Lay::kQ;
@@ -79,6 +82,35 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
 
     const int n = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t ml_base = (static_cast<int64_t>(n) * n_chunks + c) * n_heads;
+
+    // the query block (bf16 [heads x 512] as core matrices: head group stride 8192 B, dim group 128 B)
+    constexpr int kQIters = M * 64 / kTcThreads;           // 16-byte query pieces per thread
+    const uint16_t *qn = q + static_cast<int64_t>(n) * n_heads * kLatent;
+    uint4 qv[kQIters];
+#pragma unroll
+    for (int it = 0; it < kQIters; it++) {
+        const int i = it * kTcThreads + tid;
+        const int g = i >> 5, t = i & 31;
+        const int h = (g % (M / 8)) * 8 + (t & 7);
+        const int dg = (g / (M / 8)) * 4 + (t >> 3);
+        qv[it] = h < n_heads ? __ldg(reinterpret_cast<const uint4 *>(qn + static_cast<int64_t>(h) * kLatent) + dg)
+                             : make_uint4(0u, 0u, 0u, 0u);
+    }
+    auto store_q = [&]() {
+#pragma unroll
+        for (int it = 0; it < kQIters; it++) {
+            const int i = it * kTcThreads + tid;
+            const int g = i >> 5, t = i & 31;
+            const int hg = g % (M / 8);
+            const int h = hg * 8 + (t & 7);
+            const int dg = (g / (M / 8)) * 4 + (t >> 3);
+            *reinterpret_cast<uint4 *>(Qs + hg * 8192 + dg * 128 + (h & 7) * 16) = qv[it];
+        }
+    };
+    if (early_q) {
+        store_q();
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+    }
 
     if (tid == 0) *flag = 0;
     __syncthreads();
@@ -111,8 +143,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
     // 1. gather the chunk's rows (codes widened to bf16) and its scales; every global load of a
     //    thread is issued before any of them is used, so the CTA waits for one round trip
     constexpr int kRowIters = kTcRows * 32 / kTcThreads;   // 16-byte code pieces per thread
-    constexpr int kQIters = M * 64 / kTcThreads;           // 16-byte query pieces per thread
-    const uint16_t *qn = q + static_cast<int64_t>(n) * n_heads * kLatent;
     {
         uint4 v[kRowIters];
 #pragma unroll
@@ -130,16 +160,6 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
             const int r = ridx[tid];
             if (r >= 0) sc = __ldg(reinterpret_cast<const float *>(cache + static_cast<int64_t>(r) * kRowBytes + kLatent));
         }
-        uint4 qv[kQIters];
-#pragma unroll
-        for (int it = 0; it < kQIters; it++) {
-            const int i = it * kTcThreads + tid;
-            const int g = i >> 5, t = i & 31;
-            const int h = (g % (M / 8)) * 8 + (t & 7);
-            const int dg = (g / (M / 8)) * 4 + (t >> 3);
-            qv[it] = h < n_heads ? __ldg(reinterpret_cast<const uint4 *>(qn + static_cast<int64_t>(h) * kLatent) + dg)
-                                 : make_uint4(0u, 0u, 0u, 0u);
-        }
 #pragma unroll
         for (int it = 0; it < kRowIters; it++) {
             const int i = it * kTcThreads + tid;
@@ -153,15 +173,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
                                                                 codes_to_bf16x2(v[it].w, 0), codes_to_bf16x2(v[it].w, 16));
         }
         if (tid < kTcRows) scl[tid] = sc;
-#pragma unroll
-        for (int it = 0; it < kQIters; it++) {
-            const int i = it * kTcThreads + tid;
-            const int g = i >> 5, t = i & 31;
-            const int hg = g % (M / 8);
-            const int h = hg * 8 + (t & 7);
-            const int dg = (g / (M / 8)) * 4 + (t >> 3);
-            *reinterpret_cast<uint4 *>(Qs + hg * 8192 + dg * 128 + (h & 7) * 16) = qv[it];
-        }
+        if (!early_q) store_q();
     }
     tc::fence_proxy_async();
     __syncthreads();
@@ -299,7 +311,7 @@ int mla_tc_chunk() { return kTcRows; }
 
 cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
                                 const int32_t *rows, int n_q, int width, float sm_scale,
-                                float *part_acc, float *part_ml, int *status, cudaStream_t stream) {
+                                float *part_acc, float *part_ml, int *status, cudaStream_t stream, bool early_q) {
     const int n_chunks = (width + kTcRows - 1) / kTcRows;
     dim3 grid(n_chunks, n_q);
     cudaError_t e;
@@ -309,14 +321,14 @@ cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache,
         if (e != cudaSuccess) return e;
         e = launch_pdl(mla_split_tc_kernel<64>, dim3(grid), dim3(kTcThreads), smem, stream,
                        static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
-                       part_acc, part_ml, status);
+                       part_acc, part_ml, status, early_q ? 1 : 0);
     } else {
         const int smem = TcLayout<128>::kBytes;
         e = cudaFuncSetAttribute(mla_split_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
         if (e != cudaSuccess) return e;
         e = launch_pdl(mla_split_tc_kernel<128>, dim3(grid), dim3(kTcThreads), smem, stream,
                        static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
-                       part_acc, part_ml, status);
+                       part_acc, part_ml, status, early_q ? 1 : 0);
     }
     return e != cudaSuccess ? e : cudaGetLastError();
 }
