@@ -118,7 +118,9 @@ __device__ __forceinline__ void write_outputs(const IxSelectArgs &sel, int n, in
     }
 }
 
-__global__ void __launch_bounds__(kIxThreads, 1) index_select_tc_kernel(
+// At most 96 registers (83 used, no spill): a CTA then fits on an SM beside a CTA of the step's
+// first kernel, so that the grid can start while that kernel runs. Launched with kIxThreads threads.
+__global__ void __maxnreg__(96) index_select_tc_kernel(
     const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
     const float *__restrict__ pooled, int64_t ld_pools, const int32_t *__restrict__ q_seq,
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ pad,
