@@ -60,6 +60,10 @@ def _declare(L):
     L.oracle_pool_states.restype = _i64
     L.oracle_index_scores.argtypes = [_p, _p, _p, _i32, _i32, _i64, _p]
     L.oracle_index_scores.restype = None
+    L.oracle_pool_q8.argtypes = [_p, _i32, _p, _p]
+    L.oracle_pool_q8.restype = None
+    L.oracle_index_scores_q8.argtypes = [_p, _p, _p, _p, _i32, _i32, _i64, _p]
+    L.oracle_index_scores_q8.restype = None
     L.oracle_topk_pools.argtypes = [_p, _i64, _i64, _p]
     L.oracle_topk_pools.restype = _i64
     L.oracle_expand_selection.argtypes = [_p, _i64, _i64, _i64, _i64, _i32, _i64, _p]
@@ -157,6 +161,32 @@ def index_scores(q_idx, w, pooled, n_vis) -> np.ndarray:
     assert pl.shape[1] == D and pl.shape[0] >= n_vis and w.shape == (H,)
     out = np.empty(int(n_vis), dtype=np.float64)
     lib().oracle_index_scores(qp, wp, pp, H, D, int(n_vis), out.ctypes.data_as(C.c_void_p))
+    return out
+
+
+def pool_q8(pooled32):
+    """INT8 indexer state of fp32 pooled keys ``pooled32`` [P, D] (float32): returns
+    (codes int8 [P, D], scales float32 [P]), one scale per row."""
+    x = np.ascontiguousarray(pooled32, dtype=np.float32)
+    P, D = x.shape
+    codes = np.empty((P, D), dtype=np.int8)
+    scales = np.empty(P, dtype=np.float32)
+    for p in range(P):
+        lib().oracle_pool_q8(x[p].ctypes.data_as(C.c_void_p), D, codes[p].ctypes.data_as(C.c_void_p),
+                             scales[p:].ctypes.data_as(C.c_void_p))
+    return codes, scales
+
+
+def index_scores_q8(q_idx, w, codes, scales, n_vis) -> np.ndarray:
+    """Scores on the INT8 indexer state: ``codes`` int8 [P, D], ``scales`` float32 [P]."""
+    q, qp = _c(q_idx, np.uint16)
+    w, wp = _c(w, np.float32)
+    c, cp = _c(codes, np.int8)
+    sc, sp = _c(scales, np.float32)
+    H, D = q.shape
+    assert c.shape[1] == D and c.shape[0] >= n_vis and sc.shape[0] >= n_vis and w.shape == (H,)
+    out = np.empty(int(n_vis), dtype=np.float64)
+    lib().oracle_index_scores_q8(qp, wp, cp, sp, H, D, int(n_vis), out.ctypes.data_as(C.c_void_p))
     return out
 
 

@@ -12,7 +12,8 @@
  *   [DSA-REF]  "Module glm5next_dsa_ref": "Traps this module encodes" and the function list
  *              (layer_norm, pool_states, index_scores, topk_pools, expand_selection, visible,
  *              topk_to_mask, mla_masked_attention, kept_pools, DsaDims, INVALID).
- *   [PYPTO]    "GLM-5.3-Flash" (pypto-lib): "Checkpoint shape", "What is quantized".
+ *   [PYPTO]    "GLM-5.3-Flash" (pypto-lib): "Checkpoint shape", "What is quantized" (incl. the
+ *              INT8 indexer-state variant).
  * Where a page is silent the reading taken is stated beside the code as READING.
  *
  * Arithmetic is fp64 unless the step is an encoding fixed to fp32 (the int8 row's scale and the
@@ -213,6 +214,52 @@ void oracle_index_scores(const uint16_t *q_idx, const float *w, const double *po
         for (int h = 0; h < H; h++) {
             double dot = 0.0;
             for (int d = 0; d < D; d++) dot += bf16(q_idx[h * D + d]) * pooled[p * D + d];
+            s += (double)w[h] * (dot > 0.0 ? dot : 0.0);
+        }
+        scores[p] = s;
+    }
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * pool_q8 -- the INT8 indexer state: [PYPTO] "What is quantized" gives the indexer state cache as
+ * FP32 and names the sibling port's INT8 form with one FP32 scale per row.
+ * READING: a row is one pool's fp32 key (d values). It is quantized with the recipe of the latent
+ * cache rows ([KERNELS] store_int8 and [PYPTO] "What is quantized"): amax floored at
+ * INT8_AMAX_EPS, scale = fl32(amax / 127), code = clamp(round_half_even(fl32(x / scale)), +-127).
+ * ------------------------------------------------------------------------------------------- */
+void oracle_pool_q8(const float *x, int d, int8_t *codes, float *scale_out)
+{
+    double amax = 0.0;
+    for (int j = 0; j < d; j++) {
+        double a = fabs((double)x[j]);
+        if (a > amax) amax = a;
+    }
+    if (amax < amax_floor()) amax = amax_floor();
+    const float scale = (float)(amax / ORACLE_QMAX);
+    for (int j = 0; j < d; j++) {
+        double r = (double)(float)((double)x[j] / (double)scale); /* fp32 quotient        */
+        double c = nearbyint(r);                                  /* ties to even         */
+        if (c > ORACLE_QMAX) c = ORACLE_QMAX;
+        if (c < -ORACLE_QMAX) c = -ORACLE_QMAX;
+        codes[j] = (int8_t)c;
+    }
+    *scale_out = scale;
+}
+
+/* ---------------------------------------------------------------------------------------------
+ * index_scores on the INT8 indexer state: the index_scores chain with each pooled key replaced by
+ * its dequantised value code * scale:
+ *   score[p] = sum_h w[h] * max(0, sum_d q[h][d] * codes[p][d] * scale[p]),  p < n_vis.
+ * ------------------------------------------------------------------------------------------- */
+void oracle_index_scores_q8(const uint16_t *q_idx, const float *w, const int8_t *codes,
+                            const float *scales, int H, int D, int64_t n_vis, double *scores)
+{
+    for (int64_t p = 0; p < n_vis; p++) {
+        double s = 0.0;
+        for (int h = 0; h < H; h++) {
+            double dot = 0.0;
+            for (int d = 0; d < D; d++)
+                dot += bf16(q_idx[h * D + d]) * ((double)codes[p * D + d] * (double)scales[p]);
             s += (double)w[h] * (dot > 0.0 ? dot : 0.0);
         }
         scores[p] = s;
