@@ -42,7 +42,7 @@ def kernel_launches_per_step(wl, num_sms: int) -> int:
     return 4
 
 
-def algorithmic_bytes(inp) -> dict:
+def algorithmic_bytes(inp, key_bytes: int = 512) -> dict:
     """Bytes the method must move per step (no partials, no score spills): per query the visible
     pooled keys (512 B each), q_idx + w, the gathered int8 rows (528 B each), q + out, indices;
     per step the store of the new rows and the pools they complete."""
@@ -56,7 +56,7 @@ def algorithmic_bytes(inp) -> dict:
         n_vis = min(int(inp.len[s]), upto) // 4
         n_sel = min(n_vis, wl.select_k)
         tail = min(upto, int(inp.len[s])) - 4 * n_vis
-        per_q_idx += n_vis * 128 * 4 + 32 * 128 * 2 + 32 * 4 + wl.select_k * 4
+        per_q_idx += n_vis * key_bytes + 32 * 128 * 2 + 32 * 4 + wl.select_k * 4
         per_q_mla += (4 * n_sel + tail) * 528 + 2 * wl.n_heads * 512 * 2 + wl.out_width * 4
         gathered += 4 * n_sel + tail
     n_new = int(inp.new_token_mask().sum())
@@ -266,6 +266,7 @@ def config_of(wl, args):
             "queries_per_step": wl.n_queries, "n_heads": wl.n_heads, "select_k": wl.select_k,
             "out_width": wl.out_width, "kpool": 4, "index_heads": 32, "index_dim": 128,
             "latent": 512, "states": args.states,
+            "pooled_keys": "int8 codes + fp32 scale per pool" if args.pooled == "int8" else "fp32",
             "l2": f"rotates {args.states} independent states per rank (inputs >> 126 MB L2)",
             "launch": f"one cuda graph of {args.states} steps (one per state) per replay", "parallelism": f"replicas x{args.gpus}"}
 
@@ -297,12 +298,12 @@ def run_kernels(args, wl):
     inps, bufs = [], []
     for r, sid in enumerate(replica_state_ids(rank, R)):
         inp = synth.generate(wl, state=sid)
-        b = sdev.allocate_for(inp, dev)
+        b = sdev.allocate_for(inp, dev, q8=args.pooled == "int8")
         sdev.load(inp, b)
         bufs.append(b)
         inps.append(inp if r == 0 else None)
         del inp
-    ab = algorithmic_bytes(inps[0])
+    ab = algorithmic_bytes(inps[0], key_bytes=132 if args.pooled == "int8" else 512)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
@@ -448,7 +449,7 @@ def run_kernels(args, wl):
     # carries the tiny zeroing launch of the multi-CTA selection words)
     idx_ms = idx_launch_ms
     achieved = ab["index"] / (idx_ms / 1e3) / 1e9
-    traffic = recorded_traffic("index_select_tc.cu", wl.name)
+    traffic = recorded_traffic("index_select_tc.cu", wl.name + ("_q8" if args.pooled == "int8" else ""))
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -490,6 +491,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kernels", "reference"], default="kernels")
     ap.add_argument("--workload", default="long_decode", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--states", type=int, default=8)
+    ap.add_argument("--pooled", choices=["fp32", "int8"], default="fp32",
+                    help="indexer state: fp32 pooled keys (the pages' path) or the INT8 variant")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

@@ -121,6 +121,22 @@ int glm_kpool_build(const glm_dsa_dims *dims, const void *k_dev, const void *gat
                     int32_t batch, int32_t max_new_pools, float *pooled_dev, int64_t ld_pools,
                     int32_t *n_pools_dev, void *stream);
 
+/*
+ * The INT8 indexer state ("GLM-5.3-Flash" pypto-lib page, 'What is quantized': the indexer state
+ * cache is FP32 today; the sibling port keeps it in INT8 with one FP32 scale per row). The same
+ * pools as glm_kpool_build, each stored as 128 int8 codes and one fp32 scale instead of 128 fp32
+ * values: scale = max(amax, 1e-4f) / 127 over the pool's fp32 key, code = clamp(rint(x / scale),
+ * +-127) with an IEEE fp32 quotient and ties to even (the recipe of the latent cache rows).
+ *   pooled_codes_dev   int8 [batch, ld_pools, 128] (16-byte aligned)
+ *   pooled_scales_dev  fp32 [batch, ld_pools]
+ * Everything else as glm_kpool_build.
+ */
+int glm_kpool_build_q8(const glm_dsa_dims *dims, const void *k_dev, const void *gate_dev,
+                       int64_t ld_tokens, const float *ln_w_dev, const float *ln_b_dev, float ln_eps,
+                       const int32_t *pad_dev, const int32_t *len_dev, const int32_t *pool_begin_dev,
+                       int32_t batch, int32_t max_new_pools, int8_t *pooled_codes_dev,
+                       float *pooled_scales_dev, int64_t ld_pools, int32_t *n_pools_dev, void *stream);
+
 /* ------------------------------------------------------------------------------------------ */
 /* index_scores + topk_pools                                                                   */
 /* ------------------------------------------------------------------------------------------ */
@@ -172,6 +188,21 @@ int glm_index_topk_expand(const glm_dsa_dims *dims, const void *q_idx_dev, const
                           int64_t ld_slot, int32_t out_width, float *scores_dev, int32_t *topk_dev,
                           int32_t *n_sel_dev, int32_t *tok_dev, int32_t *rows_dev, void *workspace_dev,
                           size_t ws_bytes, void *stream);
+
+/*
+ * glm_index_topk_expand on the INT8 indexer state (glm_kpool_build_q8): each pooled key is
+ * code * scale, so score[n][p] = scale[p] * sum_h w[n][h] * max(0, sum_d q_idx[n][h][d] * code[p][d])
+ * (relu commutes with the positive scale). The codes are exact in bf16, so the products carry
+ * fp32 accumulation error only. Arguments, outputs and workspace as glm_index_topk_expand.
+ */
+int glm_index_topk_expand_q8(const glm_dsa_dims *dims, const void *q_idx_dev, const float *w_dev,
+                             const int8_t *pooled_codes_dev, const float *pooled_scales_dev,
+                             int64_t ld_pools, const int32_t *q_seq_dev, const int32_t *q_pos_dev,
+                             const int32_t *pad_dev, const int32_t *len_dev, int32_t batch, int32_t n_q,
+                             int32_t select_k, const int64_t *slot_map_dev, int64_t ld_slot,
+                             int32_t out_width, float *scores_dev, int32_t *topk_dev, int32_t *n_sel_dev,
+                             int32_t *tok_dev, int32_t *rows_dev, void *workspace_dev, size_t ws_bytes,
+                             void *stream);
 
 /*
  * The scores alone ("Module glm5next_dsa_ref", index_scores): the same scores as
@@ -322,6 +353,9 @@ typedef struct glm_dsa_step {
     void *out_dev;                 /* bf16 [n_q, n_heads, 512]           */
     float *lse_dev;                /* fp32 [n_q, n_heads] or NULL        */
     float *out_f32_dev;            /* fp32 [n_q, n_heads, 512] or NULL   */
+    /* the INT8 indexer state instead of pooled_dev (glm_kpool_build_q8), or NULL */
+    int8_t *pooled_codes_dev;      /* int8 [batch, ld_pools, 128]        */
+    float *pooled_scales_dev;      /* fp32 [batch, ld_pools]             */
 } glm_dsa_step;
 
 /*

@@ -34,7 +34,8 @@ GLM_OP_SPARSE_MLA = 3
 GLM_OP_DECODE_STEP = 4
 
 EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv_store_int8",
-           "glm_kpool_build", "glm_index_scores", "glm_index_scores_topk", "glm_index_topk_expand",
+           "glm_kpool_build", "glm_kpool_build_q8", "glm_index_scores", "glm_index_scores_topk",
+           "glm_index_topk_expand", "glm_index_topk_expand_q8",
            "glm_dsa_decode_step",
            "glm_topk_pools", "glm_expand_selection",
            "glm_sparse_mla_decode", "glm_dsa_workspace_size")
@@ -64,7 +65,8 @@ class glm_dsa_step(C.Structure):
                 ("scores_dev", C.c_void_p), ("topk_dev", C.c_void_p), ("n_sel_dev", C.c_void_p),
                 ("tok_dev", C.c_void_p), ("rows_dev", C.c_void_p),
                 ("q_dev", C.c_void_p), ("sm_scale", C.c_float), ("out_dev", C.c_void_p),
-                ("lse_dev", C.c_void_p), ("out_f32_dev", C.c_void_p)]
+                ("lse_dev", C.c_void_p), ("out_f32_dev", C.c_void_p),
+                ("pooled_codes_dev", C.c_void_p), ("pooled_scales_dev", C.c_void_p)]
 
 
 def make_dims(n_heads: int, kv_lora_rank: int = 512, qk_rope_head_dim: int = 0,
@@ -94,6 +96,11 @@ lib.glm_index_topk_expand.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32
 lib.glm_index_topk_expand.restype = C.c_int
 lib.glm_dsa_decode_step.argtypes = [_D, C.POINTER(glm_dsa_step), _P, _SZ, _P]
 lib.glm_dsa_decode_step.restype = C.c_int
+lib.glm_kpool_build_q8.argtypes = [_D, _P, _P, _I64, _P, _P, _F32, _P, _P, _P, _I32, _I32, _P, _P, _I64, _P, _P]
+lib.glm_kpool_build_q8.restype = C.c_int
+lib.glm_index_topk_expand_q8.argtypes = [_D, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32, _P, _I64,
+                                         _I32, _P, _P, _P, _P, _P, _P, _SZ, _P]
+lib.glm_index_topk_expand_q8.restype = C.c_int
 lib.glm_index_scores.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _P, _P]
 lib.glm_index_scores.restype = C.c_int
 lib.glm_topk_pools.argtypes = [_P, _I64, _P, _I32, _I32, _P, _P, _P, _SZ, _P]
@@ -184,6 +191,49 @@ def glm_kpool_build(dims, k, gate, ln_w, ln_b, ln_eps, pad, length, pooled, pool
                                _stream(stream)), "glm_kpool_build")
 
 
+def glm_kpool_build_q8(dims, k, gate, ln_w, ln_b, ln_eps, pad, length, codes, scales, pool_begin=None,
+                       max_new_pools=None, n_pools=None, stream=None) -> None:
+    """The INT8 indexer state: codes int8 [B, ld_pools, 128], scales fp32 [B, ld_pools]; the other
+    arguments as glm_kpool_build."""
+    for t, dt, nm in ((k, torch.bfloat16, "k"), (gate, torch.bfloat16, "gate"),
+                      (ln_w, torch.float32, "ln_w"), (ln_b, torch.float32, "ln_b"),
+                      (pad, torch.int32, "pad"), (length, torch.int32, "len"),
+                      (codes, torch.int8, "codes"), (scales, torch.float32, "scales"),
+                      (pool_begin, torch.int32, "pool_begin"), (n_pools, torch.int32, "n_pools")):
+        _dev(t, dt, nm)
+    B, ld_tokens = k.shape[0], k.shape[1]
+    ld_pools = codes.shape[1]
+    if max_new_pools is None:
+        max_new_pools = ld_pools
+    _check(lib.glm_kpool_build_q8(C.byref(dims), _ptr(k), _ptr(gate), ld_tokens, _ptr(ln_w), _ptr(ln_b),
+                                  float(ln_eps), _ptr(pad), _ptr(length), _ptr(pool_begin), B,
+                                  int(max_new_pools), _ptr(codes), _ptr(scales), ld_pools, _ptr(n_pools),
+                                  _stream(stream)), "glm_kpool_build_q8")
+
+
+def glm_index_topk_expand_q8(dims, q_idx, w, codes, scales, q_seq, q_pos, pad, length, select_k, topk,
+                             out_width, n_sel=None, slot_map=None, tok=None, rows=None, scores=None,
+                             workspace=None, stream=None) -> None:
+    """glm_index_topk_expand on the INT8 indexer state (codes int8 [B, ld_pools, 128], scales fp32
+    [B, ld_pools])."""
+    for t, dt, nm in ((q_idx, torch.bfloat16, "q_idx"), (w, torch.float32, "w"),
+                      (codes, torch.int8, "codes"), (scales, torch.float32, "scales"),
+                      (q_seq, torch.int32, "q_seq"), (q_pos, torch.int32, "q_pos"), (pad, torch.int32, "pad"),
+                      (length, torch.int32, "len"), (topk, torch.int32, "topk"),
+                      (n_sel, torch.int32, "n_sel"), (slot_map, torch.int64, "slot_map"),
+                      (tok, torch.int32, "tok"), (rows, torch.int32, "rows"),
+                      (scores, torch.float32, "scores"), (workspace, torch.uint8, "workspace")):
+        _dev(t, dt, nm)
+    ws_bytes = 0 if workspace is None else workspace.numel()
+    ld_slot = 0 if slot_map is None else slot_map.shape[1]
+    _check(lib.glm_index_topk_expand_q8(C.byref(dims), _ptr(q_idx), _ptr(w), _ptr(codes), _ptr(scales),
+                                        codes.shape[1], _ptr(q_seq), _ptr(q_pos), _ptr(pad), _ptr(length),
+                                        pad.shape[0], q_idx.shape[0], int(select_k), _ptr(slot_map), ld_slot,
+                                        int(out_width), _ptr(scores), _ptr(topk), _ptr(n_sel), _ptr(tok),
+                                        _ptr(rows), _ptr(workspace), ws_bytes, _stream(stream)),
+           "glm_index_topk_expand_q8")
+
+
 def glm_index_scores_topk(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, select_k, topk,
                           n_sel=None, scores=None, workspace=None, stream=None) -> None:
     """q_idx bf16 [n_q, 32, 128], w fp32 [n_q, 32], pooled fp32 [B, ld_pools, 128];
@@ -230,7 +280,7 @@ def glm_index_topk_expand(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, sel
 def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_eps, pad, length, pool_begin,
                         max_new_pools, pooled, q_idx, w, q_seq, q_pos, select_k, out_width, slot_map, rows,
                         topk, q, sm_scale, out, workspace, n_sel=None, tok=None, scores=None, lse=None,
-                        out_f32=None, stream=None) -> None:
+                        out_f32=None, pooled_codes=None, pooled_scales=None, stream=None) -> None:
     """The whole step in one call: the arguments of glm_kv_store_int8, glm_kpool_build,
     glm_index_topk_expand and glm_sparse_mla_decode (same tensors and rules)."""
     for t, dt, nm in ((latent, torch.bfloat16, "latent"), (slots, torch.int64, "slots"), (cache, torch.int8, "cache"),
@@ -241,7 +291,8 @@ def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_e
                       (q_pos, torch.int32, "q_pos"), (slot_map, torch.int64, "slot_map"), (rows, torch.int32, "rows"),
                       (topk, torch.int32, "topk"), (q, torch.bfloat16, "q"), (out, torch.bfloat16, "out"),
                       (workspace, torch.uint8, "workspace"), (n_sel, torch.int32, "n_sel"), (tok, torch.int32, "tok"),
-                      (scores, torch.float32, "scores"), (lse, torch.float32, "lse"), (out_f32, torch.float32, "out_f32")):
+                      (scores, torch.float32, "scores"), (lse, torch.float32, "lse"), (out_f32, torch.float32, "out_f32"),
+                      (pooled_codes, torch.int8, "pooled_codes"), (pooled_scales, torch.float32, "pooled_scales")):
         _dev(t, dt, nm)
     a = glm_dsa_step()
     v = lambda t: None if t is None else t.data_ptr()  # noqa: E731
@@ -259,6 +310,7 @@ def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_e
     a.scores_dev, a.topk_dev, a.n_sel_dev, a.tok_dev, a.rows_dev = v(scores), v(topk), v(n_sel), v(tok), v(rows)
     a.q_dev, a.sm_scale, a.out_dev = v(q), float(sm_scale), v(out)
     a.lse_dev, a.out_f32_dev = v(lse), v(out_f32)
+    a.pooled_codes_dev, a.pooled_scales_dev = v(pooled_codes), v(pooled_scales)
     ws_bytes = 0 if workspace is None else workspace.numel()
     _check(lib.glm_dsa_decode_step(C.byref(dims), C.byref(a), _ptr(workspace), ws_bytes, _stream(stream)),
            "glm_dsa_decode_step")

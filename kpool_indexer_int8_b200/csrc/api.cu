@@ -88,7 +88,7 @@ int check_store(const glm_dsa_dims *dims, const void *latent, const int64_t *slo
 
 int check_kpool(const glm_dsa_dims *dims, const void *k, const void *gate, int64_t ld_tokens,
                 const float *ln_w, const float *ln_b, float ln_eps, const int32_t *pad, const int32_t *len,
-                const int32_t *pool_begin, int32_t batch, int32_t max_new_pools, const float *pooled,
+                const int32_t *pool_begin, int32_t batch, int32_t max_new_pools, const void *pooled,
                 int64_t ld_pools, const int32_t *n_pools) {
     int rc = glm_check_dims(dims);
     if (rc != GLM_OK) return rc;
@@ -187,6 +187,21 @@ int glm_kpool_build(const glm_dsa_dims *dims, const void *k, const void *gate, i
                                                n_pools, static_cast<cudaStream_t>(stream), num_sms()));
 }
 
+int glm_kpool_build_q8(const glm_dsa_dims *dims, const void *k, const void *gate, int64_t ld_tokens,
+                       const float *ln_w, const float *ln_b, float ln_eps, const int32_t *pad,
+                       const int32_t *len, const int32_t *pool_begin, int32_t batch,
+                       int32_t max_new_pools, int8_t *pooled_codes, float *pooled_scales, int64_t ld_pools,
+                       int32_t *n_pools, void *stream) {
+    const int rc = check_kpool(dims, k, gate, ld_tokens, ln_w, ln_b, ln_eps, pad, len, pool_begin, batch,
+                               max_new_pools, pooled_codes, ld_pools, n_pools);
+    if (rc != GLM_OK || batch == 0) return rc;
+    if (!pooled_scales || !aligned(pooled_scales, 4)) return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_kpool_build(k, gate, ld_tokens, ln_w, ln_b, ln_eps, pad, len, pool_begin, batch,
+                                               max_new_pools, nullptr, ld_pools, n_pools,
+                                               static_cast<cudaStream_t>(stream), num_sms(), pooled_codes,
+                                               pooled_scales));
+}
+
 size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
                               int64_t max_pools, int32_t select_k, int32_t width) {
     if (glm_check_dims(dims) != GLM_OK || n_q < 0) return static_cast<size_t>(-1);
@@ -212,7 +227,8 @@ size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
 
 namespace {
 
-int enqueue_index_select(const void *q_idx, const float *w, const float *pooled, int64_t ld_pools,
+int enqueue_index_select(const void *q_idx, const float *w, const void *keys, const float *key_scales,
+                         int64_t ld_pools,
                          const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad, const int32_t *len,
                          int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map, int64_t ld_slot,
                          int32_t out_width, float *scores, int32_t *topk, int32_t *n_sel, int32_t *tok,
@@ -220,7 +236,7 @@ int enqueue_index_select(const void *q_idx, const float *w, const float *pooled,
                          const int32_t *new_pool_begin = nullptr, int new_pools = -1);
 
 // Checks shared by the two scoring + selection entry points; GLM_OK when the call may proceed.
-int check_index_args(const glm_dsa_dims *dims, const void *q_idx, const float *w, const float *pooled,
+int check_index_args(const glm_dsa_dims *dims, const void *q_idx, const float *w, const void *pooled,
                      int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad,
                      const int32_t *len, int32_t batch, int32_t n_q, int32_t select_k, const float *scores,
                      const int32_t *topk, const int32_t *n_sel) {
@@ -241,7 +257,8 @@ int check_index_args(const glm_dsa_dims *dims, const void *q_idx, const float *w
 
 // Scores + selection (+ expansion when tok or rows is given) in one fused launch, preceded by
 // the zeroing of the multi-CTA words when the selection spans several CTAs.
-int run_index_select(const glm_dsa_dims *dims, const void *q_idx, const float *w, const float *pooled,
+int run_index_select(const glm_dsa_dims *dims, const void *q_idx, const float *w, const void *pooled,
+                     const float *key_scales,
                      int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad,
                      const int32_t *len, int32_t batch, int32_t n_q, int32_t select_k,
                      const int64_t *slot_map, int64_t ld_slot, int32_t out_width, float *scores,
@@ -250,7 +267,7 @@ int run_index_select(const glm_dsa_dims *dims, const void *q_idx, const float *w
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_INDEX_SCORES_TOPK, n_q, ld_pools, select_k, 0);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
     int *status = reinterpret_cast<int *>(static_cast<char *>(workspace) + need - 256);
-    return enqueue_index_select(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k, slot_map,
+    return enqueue_index_select(q_idx, w, pooled, key_scales, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k, slot_map,
                                 ld_slot, out_width, scores, topk, n_sel, tok, rows, workspace, status, true,
                                 num_sms(), static_cast<cudaStream_t>(stream));
 }
@@ -261,7 +278,8 @@ namespace {
 
 // The fused index launch on a workspace laid out by sel_layout (+ the score rows); `zero`: also
 // enqueue the zeroing of the multi-CTA words (false when the caller has zeroed them already).
-int enqueue_index_select(const void *q_idx, const float *w, const float *pooled, int64_t ld_pools,
+int enqueue_index_select(const void *q_idx, const float *w, const void *keys, const float *key_scales,
+                         int64_t ld_pools,
                          const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad, const int32_t *len,
                          int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map, int64_t ld_slot,
                          int32_t out_width, float *scores, int32_t *topk, int32_t *n_sel, int32_t *tok,
@@ -293,7 +311,7 @@ int enqueue_index_select(const void *q_idx, const float *w, const float *pooled,
     sel.early = new_pools >= 0 ? 1 : 0;   // new_pools < 0: wait for the preceding kernel at the start
     sel.new_pool_begin = new_pool_begin;
     sel.new_pools = new_pools >= 0 ? new_pools : 0;
-    return cuda_status(glm::launch_index_select_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch,
+    return cuda_status(glm::launch_index_select_tc(q_idx, w, keys, key_scales, ld_pools, q_seq, q_pos, pad, len, batch,
                                                    n_q, sbuf, scores != nullptr, sel, status, sms, st));
 }
 
@@ -308,7 +326,7 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx, const flo
     int rc = check_index_args(dims, q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
                               scores, topk, n_sel);
     if (rc != GLM_OK || n_q == 0) return rc;
-    return run_index_select(dims, q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
+    return run_index_select(dims, q_idx, w, pooled, nullptr, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
                             nullptr, 0, 0, scores, topk, n_sel, nullptr, nullptr, workspace, ws_bytes, stream);
 }
 
@@ -329,9 +347,32 @@ int glm_index_topk_expand(const glm_dsa_dims *dims, const void *q_idx, const flo
     if (!tok && !rows) return GLM_ERR_INVALID_ARG;
     if ((slot_map && !aligned(slot_map, 8)) || (tok && !aligned(tok, 4)) || (rows && !aligned(rows, 4)))
         return GLM_ERR_INVALID_ARG;
-    return run_index_select(dims, q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
+    return run_index_select(dims, q_idx, w, pooled, nullptr, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
                             slot_map, ld_slot, out_width, scores, topk, n_sel, tok, rows, workspace, ws_bytes,
                             stream);
+}
+
+int glm_index_topk_expand_q8(const glm_dsa_dims *dims, const void *q_idx, const float *w,
+                             const int8_t *pooled_codes, const float *pooled_scales, int64_t ld_pools,
+                             const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad, const int32_t *len,
+                             int32_t batch, int32_t n_q, int32_t select_k, const int64_t *slot_map,
+                             int64_t ld_slot, int32_t out_width, float *scores, int32_t *topk,
+                             int32_t *n_sel, int32_t *tok, int32_t *rows, void *workspace,
+                             size_t ws_bytes, void *stream) {
+    int rc = check_index_args(dims, q_idx, w, pooled_codes, ld_pools, q_seq, q_pos, pad, len, batch, n_q, select_k,
+                              scores, topk, n_sel);
+    if (rc != GLM_OK) return rc;
+    if (out_width < 1 || ld_slot < 0) return GLM_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(out_width) < static_cast<int64_t>(glm::kKpool) * select_k + glm::kKpool - 1)
+        return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (!tok && !rows) return GLM_ERR_INVALID_ARG;
+    if ((ld_pools > 0 && (!pooled_scales || !aligned(pooled_scales, 4))) || (slot_map && !aligned(slot_map, 8)) ||
+        (tok && !aligned(tok, 4)) || (rows && !aligned(rows, 4)))
+        return GLM_ERR_INVALID_ARG;
+    return run_index_select(dims, q_idx, w, pooled_codes, pooled_scales ? pooled_scales : nullptr, ld_pools, q_seq,
+                            q_pos, pad, len, batch, n_q, select_k, slot_map, ld_slot, out_width, scores, topk, n_sel,
+                            tok, rows, workspace, ws_bytes, stream);
 }
 
 int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w,
@@ -349,7 +390,7 @@ int glm_index_scores(const glm_dsa_dims *dims, const void *q_idx, const float *w
         !aligned(q_pos, 4) || !aligned(pad, 4) || !aligned(len, 4) || !aligned(scores, 4))
         return GLM_ERR_INVALID_ARG;
     const glm::IxSelectArgs none{};   // topk == nullptr: scores only
-    return cuda_status(glm::launch_index_select_tc(q_idx, w, pooled, ld_pools, q_seq, q_pos, pad, len,
+    return cuda_status(glm::launch_index_select_tc(q_idx, w, pooled, nullptr, ld_pools, q_seq, q_pos, pad, len,
                                                    batch, n_q, scores, true, none, nullptr, num_sms(),
                                                    static_cast<cudaStream_t>(stream)));
 }
@@ -426,12 +467,15 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t 
 int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *workspace, size_t ws_bytes,
                         void *stream) {
     if (a == nullptr) return GLM_ERR_INVALID_ARG;
+    const bool q8 = a->pooled_codes_dev != nullptr;   // the INT8 indexer state replaces pooled_dev
+    const void *keys = q8 ? static_cast<const void *>(a->pooled_codes_dev) : static_cast<const void *>(a->pooled_dev);
+    if (q8 && (!a->pooled_scales_dev || !aligned(a->pooled_scales_dev, 4))) return GLM_ERR_INVALID_ARG;
     int rc = check_store(dims, a->latent_dev, a->slots_dev, a->n_new, a->cache_dev, a->n_rows);
     if (rc != GLM_OK) return rc;
     rc = check_kpool(dims, a->k_dev, a->gate_dev, a->ld_tokens, a->ln_w_dev, a->ln_b_dev, a->ln_eps, a->pad_dev,
-                     a->len_dev, a->pool_begin_dev, a->batch, a->max_new_pools, a->pooled_dev, a->ld_pools, nullptr);
+                     a->len_dev, a->pool_begin_dev, a->batch, a->max_new_pools, keys, a->ld_pools, nullptr);
     if (rc != GLM_OK) return rc;
-    rc = check_index_args(dims, a->q_idx_dev, a->w_dev, a->pooled_dev, a->ld_pools, a->q_seq_dev, a->q_pos_dev,
+    rc = check_index_args(dims, a->q_idx_dev, a->w_dev, keys, a->ld_pools, a->q_seq_dev, a->q_pos_dev,
                           a->pad_dev, a->len_dev, a->batch, a->n_q, a->select_k, a->scores_dev, a->topk_dev,
                           a->n_sel_dev);
     if (rc != GLM_OK) return rc;
@@ -470,13 +514,16 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     p.pool_begin = a->pool_begin_dev;
     p.batch = a->batch;
     p.max_new_pools = a->max_new_pools;
-    p.pooled = a->pooled_dev;
+    p.pooled = q8 ? nullptr : a->pooled_dev;
+    p.codes = q8 ? a->pooled_codes_dev : nullptr;
+    p.scales = q8 ? a->pooled_scales_dev : nullptr;
     p.ld_pools = a->ld_pools;
     p.zero = reinterpret_cast<uint4 *>(sw.hist);
     p.zero_n16 = idx_multi ? static_cast<int64_t>(align_up(sw.zero_bytes, 16) / 16) : 0;
     rc = cuda_status(glm::launch_step_prep(p, st));
     if (rc != GLM_OK || a->n_q == 0) return rc;
-    rc = enqueue_index_select(a->q_idx_dev, a->w_dev, a->pooled_dev, a->ld_pools, a->q_seq_dev, a->q_pos_dev,
+    rc = enqueue_index_select(a->q_idx_dev, a->w_dev, keys, q8 ? a->pooled_scales_dev : nullptr, a->ld_pools,
+                              a->q_seq_dev, a->q_pos_dev,
                               a->pad_dev, a->len_dev, a->batch, a->n_q, a->select_k, a->slot_map_dev, a->ld_slot,
                               a->out_width, a->scores_dev, a->topk_dev, a->n_sel_dev, a->tok_dev, a->rows_dev,
                               ws + L.idx, status, false, sms, st, a->pool_begin_dev,

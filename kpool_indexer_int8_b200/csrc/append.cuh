@@ -52,7 +52,9 @@ __device__ __forceinline__ void kpool_build_item(const uint16_t *__restrict__ k,
                                                  float eps, const int32_t *__restrict__ pad,
                                                  const int32_t *__restrict__ len,
                                                  const int32_t *__restrict__ pool_begin, int max_new_pools,
-                                                 float *__restrict__ pooled, int64_t ld_pools, int64_t it) {
+                                                 float *__restrict__ pooled, int64_t ld_pools, int64_t it,
+                                                 int8_t *__restrict__ codes = nullptr,
+                                                 float *__restrict__ scales = nullptr) {
     const int lane = threadIdx.x & 31;
     const int b = static_cast<int>(it / max_new_pools);
     const int i = static_cast<int>(it % max_new_pools);
@@ -93,8 +95,25 @@ __device__ __forceinline__ void kpool_build_item(const uint16_t *__restrict__ k,
         }
         out[c] = num / den;
     }
-    reinterpret_cast<float4 *>(pooled + (static_cast<int64_t>(b) * ld_pools + p) * kIdxDim)[lane] =
-        make_float4(out[0], out[1], out[2], out[3]);
+    const int64_t row = static_cast<int64_t>(b) * ld_pools + p;
+    if (codes == nullptr) {
+        reinterpret_cast<float4 *>(pooled + row * kIdxDim)[lane] = make_float4(out[0], out[1], out[2], out[3]);
+        return;
+    }
+    // INT8 indexer state: the row's amax (floored at 1e-4) over 127 is the scale; codes are the
+    // IEEE fp32 quotients rounded half to even, clamped to +-127 (the latent cache rows' recipe)
+    float amax = fmaxf(fmaxf(fabsf(out[0]), fabsf(out[1])), fmaxf(fabsf(out[2]), fabsf(out[3])));
+    amax = fmaxf(warp_max(amax), 1e-4f);
+    const float scale = __fdiv_rn(amax, 127.0f);
+    uint32_t packed = 0;
+#pragma unroll
+    for (int c = 0; c < 4; c++) {
+        int q = __float2int_rn(__fdiv_rn(out[c], scale));
+        q = max(-127, min(127, q));
+        packed |= (static_cast<uint32_t>(q) & 0xffu) << (8 * c);
+    }
+    reinterpret_cast<uint32_t *>(codes + row * kIdxDim)[lane] = packed;
+    if (lane == 0) scales[row] = scale;
 }
 
 }  // namespace glm

@@ -24,6 +24,9 @@
 // the selection, sorts it, and writes the top-k row, n_sel and the expanded token / row indices.
 // With G = 1 the one CTA does all of it on chip.
 // Phase 1 is HBM-bound: 512 bytes of pooled key per pool; the tensor cores run at a few percent.
+// With the INT8 indexer state ("GLM-5.3-Flash" pypto-lib page, 'What is quantized': the indexer
+// cache in INT8 with one FP32 scale per row) a pool is 128 code bytes plus its scale: 4 KB bulk
+// copies into 8 slots, one exact bf16 term (|code| <= 127), the score multiplied by the pool scale.
 #include "common.cuh"
 #include "tc.cuh"
 #include "kernels.cuh"
@@ -35,25 +38,25 @@ namespace glm {
 constexpr int kIxThreads = 512;                        // 16 warps, see the roles above
 constexpr int kIxTile = 64;                            // pools per tile (UMMA M)
 constexpr int kIxChunk = 32;                           // pools per bulk copy (2 per tile)
-constexpr int kIxStages = 4;                           // bulk copies in flight
+constexpr int kIxMaxStages = 8;                        // staging slots (fp32 keys use 4, int8 keys 8)
 constexpr int kIxConv = 8;                             // converter warps
 constexpr int kIxAtomBytes = kIxTile * 128;            // 64 rows x 128 bytes (64 dims): 8 KB
 constexpr int kIxTermBytes = 2 * kIxAtomBytes;         // one bf16 term of a tile: 16 KB
 constexpr int kIxBufBytes = 3 * kIxTermBytes;          // three terms: 48 KB
-constexpr int kIxStageBytes = kIxChunk * kIdxDim * 4;  // 16 KB of fp32 pooled keys
+constexpr int kIxStageRegion = 4 * kIxChunk * kIdxDim * 4;   // 64 KB: 4 x 16 KB fp32 or 8 x 4 KB int8
 constexpr uint32_t kIxWaitLimit = 1u << 22;
 
 constexpr int kIxLocalCap = 4096;                      // scores of a CTA kept in shared memory
 
 struct IxLayout {                                      // offsets from a 1024-byte aligned base
     static constexpr int kTerms = 0;                                  // [2 buffers][3 terms][16 KB]
-    static constexpr int kStage = kTerms + 2 * kIxBufBytes;           // [4 stages][16 KB]
-    static constexpr int kQ = kStage + kIxStages * kIxStageBytes;     // 32 heads x 128 dims bf16
+    static constexpr int kStage = kTerms + 2 * kIxBufBytes;           // staging slots
+    static constexpr int kQ = kStage + kIxStageRegion;                // 32 heads x 128 dims bf16
     static constexpr int kHist = kQ + kIdxHeads * kIdxDim * 2;        // 2048 uint32
     static constexpr int kLocal = kHist + kHistBins * 4;              // kIxLocalCap fp32 scores
     static constexpr int kW = kLocal + kIxLocalCap * 4;               // 32 fp32 head weights
-    static constexpr int kBar = kW + kIdxHeads * 4;                   // 16 mbarriers
-    static constexpr int kTmem = kBar + 16 * 8;
+    static constexpr int kBar = kW + kIdxHeads * 4;                   // 24 mbarriers
+    static constexpr int kTmem = kBar + 24 * 8;
     static constexpr int kFlag = kTmem + 16;
     static constexpr int kBytes = kFlag + 16;
     static constexpr int kAlloc = kBytes + 1024;                      // room to align the base
@@ -62,12 +65,12 @@ struct IxLayout {                                      // offsets from a 1024-by
 static_assert(sizeof(SelShared) <= IxLayout::kQ, "selection working set must fit the scoring buffers");
 
 // mbarrier indices
-constexpr int kBarStFull = 0;     // [4] staging slot filled (producer, tx bytes)
-constexpr int kBarStEmpty = 4;    // [4] staging slot read (8 converter warps)
-constexpr int kBarTmFull = 8;     // [2] tile buffer written (8 warps x 2 chunk slots)
-constexpr int kBarTmEmpty = 10;   // [2] tile buffer read by the MMAs (commit)
-constexpr int kBarAccFull = 12;   // [2] accumulator ready (commit)
-constexpr int kBarAccEmpty = 14;  // [2] accumulator read (4 epilogue warps)
+constexpr int kBarStFull = 0;     // [8] staging slot filled (producer, tx bytes)
+constexpr int kBarStEmpty = 8;    // [8] staging slot read (8 converter warps)
+constexpr int kBarTmFull = 16;    // [2] tile buffer written (8 warps x 2 chunk slots)
+constexpr int kBarTmEmpty = 18;   // [2] tile buffer read by the MMAs (commit)
+constexpr int kBarAccFull = 20;   // [2] accumulator ready (commit)
+constexpr int kBarAccEmpty = 22;  // [2] accumulator read (4 epilogue warps)
 
 __device__ __forceinline__ uint32_t bf16_pair(float a, float b) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low half), .y = b
@@ -120,12 +123,21 @@ __device__ __forceinline__ void write_outputs(const IxSelectArgs &sel, int n, in
 
 // At most 96 registers (83 used, no spill): a CTA then fits on an SM beside a CTA of the step's
 // first kernel, so that the grid can start while that kernel runs. Launched with kIxThreads threads.
+// kQ8: the pooled keys are the INT8 indexer state (int8 codes [B][ld][128], one fp32 scale per
+// pool): one exact bf16 term per key instead of three, and the score is scaled by the pool's scale.
+template <bool kQ8>
 __global__ void __maxnreg__(96) index_select_tc_kernel(
     const uint16_t *__restrict__ q_idx, const float *__restrict__ w,
-    const float *__restrict__ pooled, int64_t ld_pools, const int32_t *__restrict__ q_seq,
+    const void *__restrict__ keys, const float *__restrict__ key_scales, int64_t ld_pools,
+    const int32_t *__restrict__ q_seq,
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ pad,
     const int32_t *__restrict__ len, int batch, float *__restrict__ scores, int fill_invisible,
     IxSelectArgs sel, int *__restrict__ status) {
+    constexpr int kStages = kQ8 ? 8 : 4;                          // staging slots
+    constexpr int kElem = kQ8 ? 1 : 4;                            // bytes per key element
+    constexpr int kStageBytes = kIxChunk * kIdxDim * kElem;       // one chunk of keys
+    constexpr int kNumTerms = kQ8 ? 1 : 3;                        // bf16 terms per key
+    static_assert(kStages * kStageBytes <= kIxStageRegion && kStages <= kIxMaxStages, "staging");
     if (sel.early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     else pdl_begin();
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -172,7 +184,8 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     if (lo < hi) {
     const int n_chunks = (hi - lo + kIxChunk - 1) / kIxChunk;
     const int n_tiles = (hi - lo + kIxTile - 1) / kIxTile;
-    const float *src = pooled + (static_cast<int64_t>(b) * ld_pools + lo) * kIdxDim;
+    const unsigned char *src = static_cast<const unsigned char *>(keys) +
+                               (static_cast<int64_t>(b) * ld_pools + lo) * kIdxDim * kElem;
 
     const uint32_t bar0 = tc::smem_addr(smem + IxLayout::kBar);
     auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
@@ -182,8 +195,8 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
         tc::fence_before_sync();
     }
     if (tid == 32) {
-        for (int i = 0; i < 4; i++) tc::mbar_init(bar(kBarStFull + i), 1);
-        for (int i = 0; i < 4; i++) tc::mbar_init(bar(kBarStEmpty + i), kIxConv);
+        for (int i = 0; i < kStages; i++) tc::mbar_init(bar(kBarStFull + i), 1);
+        for (int i = 0; i < kStages; i++) tc::mbar_init(bar(kBarStEmpty + i), kIxConv);
         for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarTmFull + i), 2 * kIxConv);
         for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarTmEmpty + i), 1);
         for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccFull + i), 1);
@@ -212,7 +225,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             const uint32_t stage_addr = tc::smem_addr(stage);
             bool waited = !sel.early;
             for (int c = 0; c < n_chunks; c++) {
-                const int slot = c % kIxStages;
+                const int slot = c % kStages;
                 const int c0 = lo + c * kIxChunk;
                 if (!waited && c0 + kIxChunk > first_new && c0 < first_new + sel.new_pools) {
                     // this chunk holds a pool the preceding kernel writes: wait for it first
@@ -220,12 +233,12 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                     waited = true;
                 }
-                if (c >= kIxStages && !tc::mbar_wait(bar(kBarStEmpty + slot), ((c / kIxStages) - 1) & 1, kIxWaitLimit))
+                if (c >= kStages && !tc::mbar_wait(bar(kBarStEmpty + slot), ((c / kStages) - 1) & 1, kIxWaitLimit))
                     ok = false;
-                const uint32_t bytes = static_cast<uint32_t>(min(kIxChunk, hi - lo - c * kIxChunk)) * kIdxDim * 4;
+                const uint32_t bytes = static_cast<uint32_t>(min(kIxChunk, hi - lo - c * kIxChunk)) * kIdxDim * kElem;
                 tc::mbar_arrive_expect_tx(bar(kBarStFull + slot), bytes);
-                tc::bulk_g2s(stage_addr + slot * kIxStageBytes, src + static_cast<int64_t>(c) * kIxChunk * kIdxDim,
-                             bytes, bar(kBarStFull + slot));
+                tc::bulk_g2s(stage_addr + slot * kStageBytes, src + static_cast<int64_t>(c) * kStageBytes, bytes,
+                             bar(kBarStFull + slot));
             }
         }
     } else if (warp == 1) {
@@ -240,7 +253,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                 tc::fence_after_sync();
                 const uint32_t d = tmem + tb * 32;
 #pragma unroll
-                for (int term = 0; term < 3; term++) {
+                for (int term = 0; term < kNumTerms; term++) {
 #pragma unroll
                     for (int ks = 0; ks < kIdxDim / 16; ks++) {
                         const uint32_t a = terms_addr + tb * kIxBufBytes + term * kIxTermBytes +
@@ -258,18 +271,21 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
         const int qd = warp & 3;
         for (int t = 0; t < n_tiles; t++) {
             const int tb = t & 1;
+            const int p = lo + t * kIxTile + qd * 16 + lane;
+            float ksc = 1.0f;   // the pool's int8 scale (loaded before the wait)
+            if (kQ8 && lane < 16 && p < hi) ksc = __ldg(key_scales + static_cast<int64_t>(b) * ld_pools + p);
             if (!tc::mbar_wait(bar(kBarAccFull + tb), (t >> 1) & 1, kIxWaitLimit)) ok = false;
             __syncwarp();
             tc::fence_after_sync();
             uint32_t r[32];
             tc::tmem_ld32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + tb * 32, r);
             tc::tmem_wait_ld();
-            const int p = lo + t * kIxTile + qd * 16 + lane;
             uint32_t digit = 0xffffffffu;
             if (lane < 16 && p < hi) {
                 float sc = 0.0f;
 #pragma unroll
                 for (int h2 = 0; h2 < kIdxHeads; h2++) sc = fmaf(ws[h2], fmaxf(__uint_as_float(r[h2]), 0.0f), sc);
+                if (kQ8) sc *= ksc;   // relu(s q.c) = s relu(q.c) for the scale s > 0
                 srow[p] = sc;
                 if (keep_local) sloc[p - lo] = sc;
                 digit = score_key(sc) >> (32 - kHistBitsTop);
@@ -289,13 +305,24 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             for (int half = 0; half < 2; half++) {
                 const int c = 2 * t + half;
                 if (c < n_chunks) {
-                    const int slot = c % kIxStages;
-                    if (!tc::mbar_wait(bar(kBarStFull + slot), (c / kIxStages) & 1, kIxWaitLimit)) ok = false;
-                    const unsigned char *st = stage + slot * kIxStageBytes;
+                    const int slot = c % kStages;
+                    if (!tc::mbar_wait(bar(kBarStFull + slot), (c / kStages) & 1, kIxWaitLimit)) ok = false;
+                    const unsigned char *st = stage + slot * kStageBytes;
 #pragma unroll
                     for (int pi = 0; pi < kIxChunk / kIxConv; pi++) {
                         const int pc = cw * (kIxChunk / kIxConv) + pi;   // pool within the chunk
                         const int r = half * kIxChunk + pc;              // row within the tile
+                        const int off = (lane >> 4) * kIxAtomBytes + r * 128 +
+                                        ((((lane & 15) >> 1) ^ (r & 7)) << 4) + (lane & 1) * 8;
+                        if (kQ8) {   // four int8 codes -> four bf16 (exact: |code| <= 127)
+                            const uint32_t v = *reinterpret_cast<const uint32_t *>(st + pc * kIdxDim + lane * 4);
+                            const float c0 = static_cast<float>(static_cast<int8_t>(v & 0xffu));
+                            const float c1 = static_cast<float>(static_cast<int8_t>((v >> 8) & 0xffu));
+                            const float c2 = static_cast<float>(static_cast<int8_t>((v >> 16) & 0xffu));
+                            const float c3 = static_cast<float>(static_cast<int8_t>(v >> 24));
+                            *reinterpret_cast<uint2 *>(buf + off) = make_uint2(bf16_pair(c0, c1), bf16_pair(c2, c3));
+                            continue;
+                        }
                         const float4 x = *reinterpret_cast<const float4 *>(st + pc * (kIdxDim * 4) + lane * 16);
                         const uint32_t h0 = bf16_pair(x.x, x.y), h1 = bf16_pair(x.z, x.w);
                         const float r0 = x.x - bf16_lo_f(h0), r1 = x.y - bf16_hi_f(h0);
@@ -303,8 +330,6 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                         const uint32_t m0 = bf16_pair(r0, r1), m1 = bf16_pair(r2, r3);
                         const uint32_t l0 = bf16_pair(r0 - bf16_lo_f(m0), r1 - bf16_hi_f(m0));
                         const uint32_t l1 = bf16_pair(r2 - bf16_lo_f(m1), r3 - bf16_hi_f(m1));
-                        const int off = (lane >> 4) * kIxAtomBytes + r * 128 +
-                                        ((((lane & 15) >> 1) ^ (r & 7)) << 4) + (lane & 1) * 8;
                         *reinterpret_cast<uint2 *>(buf + off) = make_uint2(h0, h1);
                         *reinterpret_cast<uint2 *>(buf + kIxTermBytes + off) = make_uint2(m0, m1);
                         *reinterpret_cast<uint2 *>(buf + 2 * kIxTermBytes + off) = make_uint2(l0, l1);
@@ -403,23 +428,24 @@ int index_select_ctas(int n_q, int64_t ld_pools, int num_sms) {
     return G;
 }
 
-cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const float *pooled,
-                                   int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
-                                   const int32_t *pad, const int32_t *len, int batch, int n_q,
-                                   float *scores, bool fill_invisible, const IxSelectArgs &sel,
+cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const void *keys,
+                                   const float *key_scales, int64_t ld_pools, const int32_t *q_seq,
+                                   const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
+                                   int n_q, float *scores, bool fill_invisible, const IxSelectArgs &sel,
                                    int *status, int num_sms, cudaStream_t stream) {
     const int G = index_select_ctas(n_q, ld_pools, num_sms);
     const int smem = IxLayout::kAlloc;
-    cudaError_t e = cudaFuncSetAttribute(index_select_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    auto kernel = key_scales ? index_select_tc_kernel<true> : index_select_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     // No cooperative attribute: a cooperative grid cannot start under programmatic dependent launch
     // before its predecessor ends, which would forfeit the early streaming. Co-residency of the
     // grid barrier's CTAs holds by construction: G * n_q <= the SM count at one CTA per SM (the
     // shared memory allows no second), and a later kernel of the stream can only launch once every
     // CTA of this one has started. The wait is bounded and reports through the status word.
-    e = launch_pdl(index_select_tc_kernel, dim3(G, n_q), dim3(kIxThreads), smem, stream,
-                   static_cast<const uint16_t *>(q_idx), w, pooled, ld_pools, q_seq, q_pos, pad, len, batch, scores,
-                   fill_invisible ? 1 : 0, sel, status);
+    e = launch_pdl(kernel, dim3(G, n_q), dim3(kIxThreads), smem, stream, static_cast<const uint16_t *>(q_idx), w,
+                   keys, key_scales, ld_pools, q_seq, q_pos, pad, len, batch, scores, fill_invisible ? 1 : 0, sel,
+                   status);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 

@@ -15,7 +15,8 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
                                const float *ln_w, const float *ln_b, float eps,
                                const int32_t *pad, const int32_t *len, const int32_t *pool_begin,
                                int batch, int max_new_pools, float *pooled, int64_t ld_pools,
-                               int32_t *n_pools, cudaStream_t stream, int num_sms);
+                               int32_t *n_pools, cudaStream_t stream, int num_sms,
+                               int8_t *codes = nullptr, float *scales = nullptr);   // codes: INT8 state
 // Selection and expansion arguments of the fused index kernel; topk == nullptr: scores only.
 // The multi-CTA words (ghist, ghist2, counters: 2 kHistBins + kCntWords uint32 per query) must
 // be zero at launch when index_select_ctas() > 1.
@@ -43,11 +44,11 @@ struct IxSelectArgs {
     int new_pools;
 };
 int index_select_ctas(int n_q, int64_t ld_pools, int num_sms);
-cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const float *pooled,
-                                   int64_t ld_pools, const int32_t *q_seq, const int32_t *q_pos,
-                                   const int32_t *pad, const int32_t *len, int batch, int n_q,
-                                   float *scores, bool fill_invisible, const IxSelectArgs &sel,
-                                   int *status, int num_sms, cudaStream_t stream);
+cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const void *keys,
+                                   const float *key_scales, int64_t ld_pools, const int32_t *q_seq,
+                                   const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
+                                   int n_q, float *scores, bool fill_invisible, const IxSelectArgs &sel,
+                                   int *status, int num_sms, cudaStream_t stream);   // key_scales: INT8 keys
 // The fused step's first kernel: store rows, build pools, zero a word range (16-byte units).
 struct StepPrepArgs {
     const uint16_t *latent;
@@ -67,6 +68,8 @@ struct StepPrepArgs {
     int batch;
     int max_new_pools;
     float *pooled;
+    int8_t *codes;                 // INT8 indexer state (pooled unused) or null
+    float *scales;
     int64_t ld_pools;
     uint4 *zero;
     int64_t zero_n16;

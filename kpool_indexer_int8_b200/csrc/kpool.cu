@@ -16,7 +16,8 @@ __global__ void __launch_bounds__(256) kpool_build_kernel(
     const float *__restrict__ ln_w, const float *__restrict__ ln_b, float eps,
     const int32_t *__restrict__ pad, const int32_t *__restrict__ len,
     const int32_t *__restrict__ pool_begin, int batch, int max_new_pools,
-    float *__restrict__ pooled, int64_t ld_pools, int32_t *__restrict__ n_pools_out) {
+    float *__restrict__ pooled, int64_t ld_pools, int32_t *__restrict__ n_pools_out,
+    int8_t *__restrict__ codes, float *__restrict__ scales) {
     pdl_begin();
     const int lane = threadIdx.x & 31;
     if (n_pools_out != nullptr && blockIdx.x == 0) {
@@ -32,14 +33,16 @@ __global__ void __launch_bounds__(256) kpool_build_kernel(
     const int64_t warps_total = static_cast<int64_t>(gridDim.x) * (blockDim.x >> 5);
     for (int64_t it = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
          it < items; it += warps_total)
-        kpool_build_item(k, gate, ld_tokens, lw, lb, eps, pad, len, pool_begin, max_new_pools, pooled, ld_pools, it);
+        kpool_build_item(k, gate, ld_tokens, lw, lb, eps, pad, len, pool_begin, max_new_pools, pooled, ld_pools, it,
+                         codes, scales);
 }
 
 cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_tokens,
                                const float *ln_w, const float *ln_b, float eps,
                                const int32_t *pad, const int32_t *len, const int32_t *pool_begin,
                                int batch, int max_new_pools, float *pooled, int64_t ld_pools,
-                               int32_t *n_pools, cudaStream_t stream, int num_sms) {
+                               int32_t *n_pools, cudaStream_t stream, int num_sms, int8_t *codes,
+                               float *scales) {
     const int warps_per_block = 8;
     int64_t items = static_cast<int64_t>(batch) * max_new_pools;
     int64_t blocks = (items + warps_per_block - 1) / warps_per_block;
@@ -48,7 +51,7 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
     if (blocks > cap) blocks = cap;
     launch_pdl(kpool_build_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32 * warps_per_block), 0, stream,
                static_cast<const uint16_t *>(k), static_cast<const uint16_t *>(gate), ld_tokens, ln_w, ln_b, eps,
-               pad, len, pool_begin, batch, max_new_pools, pooled, ld_pools, n_pools);
+               pad, len, pool_begin, batch, max_new_pools, pooled, ld_pools, n_pools, codes, scales);
     return cudaGetLastError();
 }
 

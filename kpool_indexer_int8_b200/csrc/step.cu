@@ -28,7 +28,7 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(StepPrepArgs a,
         const float4 b4 = reinterpret_cast<const float4 *>(a.ln_b)[lane];
         const float lw[4] = {w4.x, w4.y, w4.z, w4.w}, lb[4] = {b4.x, b4.y, b4.z, b4.w};
         kpool_build_item(a.k, a.gate, a.ld_tokens, lw, lb, a.ln_eps, a.pad, a.len, a.pool_begin, a.max_new_pools,
-                         a.pooled, a.ld_pools, it);
+                         a.pooled, a.ld_pools, it, a.codes, a.scales);
         return;
     }
     cta -= pool_ctas;

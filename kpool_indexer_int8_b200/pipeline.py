@@ -21,7 +21,8 @@ import torch
 
 from . import (GLM_OP_DECODE_STEP, GLM_OP_INDEX_SCORES_TOPK, GLM_OP_SPARSE_MLA, GLM_ROW_BYTES,
                glm_dsa_decode_step, glm_dsa_workspace_size, glm_expand_selection, glm_index_scores_topk,
-               glm_index_topk_expand, glm_kpool_build, glm_kv_store_int8, glm_sparse_mla_decode, make_dims)
+               glm_index_topk_expand, glm_index_topk_expand_q8, glm_kpool_build, glm_kpool_build_q8, glm_kv_store_int8,
+               glm_sparse_mla_decode, make_dims)
 
 LATENT = 512
 IDX_HEADS = 32
@@ -69,11 +70,13 @@ class DecodeBuffers:
     ws_step: torch.Tensor    # uint8 workspace of the one-call step
     scores: Optional[torch.Tensor] = None  # fp32 [n_q, ld_pools] when requested
     out_f32: Optional[torch.Tensor] = None
+    pooled_codes: Optional[torch.Tensor] = None   # INT8 indexer state: int8 [B, ld_pools, 128]
+    pooled_scales: Optional[torch.Tensor] = None  #                       fp32 [B, ld_pools]
 
 
 def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_new: int,
              select_k: int, out_width: int, sm_scale: float, ln_eps: float, max_new_pools: int,
-             device, keep_scores: bool = False, keep_f32: bool = False) -> DecodeBuffers:
+             device, keep_scores: bool = False, keep_f32: bool = False, q8: bool = False) -> DecodeBuffers:
     dims = make_dims(n_heads)
     ld_pools = max(1, ld_tokens // KPOOL)
     f = dict(device=device)
@@ -111,6 +114,8 @@ def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_
         ws_step=torch.empty(max(ws_s, 1), dtype=torch.uint8, **f),
         scores=torch.empty(n_q, ld_pools, dtype=torch.float32, **f) if keep_scores else None,
         out_f32=torch.empty(n_q, n_heads, LATENT, dtype=torch.float32, **f) if keep_f32 else None,
+        pooled_codes=torch.zeros(batch, ld_pools, IDX_DIM, dtype=torch.int8, **f) if q8 else None,
+        pooled_scales=torch.zeros(batch, ld_pools, dtype=torch.float32, **f) if q8 else None,
     )
 
 
@@ -119,6 +124,13 @@ def store(b: DecodeBuffers, stream=None) -> None:
 
 
 def build_pools(b: DecodeBuffers, length=None, pool_begin=None, max_new_pools=None, stream=None) -> None:
+    if b.pooled_codes is not None:
+        glm_kpool_build_q8(b.dims, b.k, b.gate, b.ln_w, b.ln_b, b.ln_eps, b.pad,
+                           b.len if length is None else length, b.pooled_codes, b.pooled_scales,
+                           pool_begin=b.pool_begin if pool_begin is None else pool_begin,
+                           max_new_pools=b.max_new_pools if max_new_pools is None else max_new_pools,
+                           stream=stream)
+        return
     glm_kpool_build(b.dims, b.k, b.gate, b.ln_w, b.ln_b, b.ln_eps, b.pad,
                     b.len if length is None else length, b.pooled,
                     pool_begin=b.pool_begin if pool_begin is None else pool_begin,
@@ -138,6 +150,11 @@ def expand(b: DecodeBuffers, stream=None) -> None:
 
 
 def index_topk_expand(b: DecodeBuffers, stream=None) -> None:
+    if b.pooled_codes is not None:
+        glm_index_topk_expand_q8(b.dims, b.q_idx, b.w, b.pooled_codes, b.pooled_scales, b.q_seq, b.q_pos, b.pad,
+                                 b.len, b.select_k, b.topk, b.out_width, n_sel=b.n_sel, slot_map=b.slot_map,
+                                 tok=b.tok, rows=b.rows, scores=b.scores, workspace=b.ws_index, stream=stream)
+        return
     glm_index_topk_expand(b.dims, b.q_idx, b.w, b.pooled, b.q_seq, b.q_pos, b.pad, b.len, b.select_k,
                           b.topk, b.out_width, n_sel=b.n_sel, slot_map=b.slot_map, tok=b.tok, rows=b.rows,
                           scores=b.scores, workspace=b.ws_index, stream=stream)
@@ -166,4 +183,5 @@ def run_step(b: DecodeBuffers, stream=None) -> None:
                         w=b.w, q_seq=b.q_seq, q_pos=b.q_pos, select_k=b.select_k, out_width=b.out_width,
                         slot_map=b.slot_map, rows=b.rows, topk=b.topk, q=b.q, sm_scale=b.sm_scale, out=b.out,
                         workspace=b.ws_step, n_sel=b.n_sel, tok=b.tok, scores=b.scores, lse=b.lse,
-                        out_f32=b.out_f32, stream=stream)
+                        out_f32=b.out_f32, pooled_codes=b.pooled_codes, pooled_scales=b.pooled_scales,
+                        stream=stream)

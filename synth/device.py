@@ -30,14 +30,14 @@ def step_split(inp: Inputs):
     return (inp.len - n_new_seq).astype(np.int32), np.nonzero(new)[0]
 
 
-def allocate_for(inp: Inputs, device, keep_scores=False, keep_f32=False) -> P.DecodeBuffers:
+def allocate_for(inp: Inputs, device, keep_scores=False, keep_f32=False, q8=False) -> P.DecodeBuffers:
     prefix, new_idx = step_split(inp)
     per_seq_new = int(max(1, (inp.len - prefix).max()))
     max_new_pools = per_seq_new // P.KPOOL + 1
     return P.allocate(inp.wl.n_heads, inp.wl.batch, inp.ld_tokens, inp.n_rows, len(inp.q_pos),
                       len(new_idx), inp.wl.select_k, inp.wl.out_width, inp.sm_scale,
                       inp.wl.ln_eps, max_new_pools, device, keep_scores=keep_scores,
-                      keep_f32=keep_f32)
+                      keep_f32=keep_f32, q8=q8)
 
 
 def load(inp: Inputs, b: P.DecodeBuffers, build_prefix: bool = True) -> None:
