@@ -61,8 +61,9 @@ struct IxLayout {                                      // offsets from a 1024-by
     static constexpr int kBytes = kFlag + 16;
     static constexpr int kAlloc = kBytes + 1024;                      // room to align the base
 };
-// The selection's working set overlays the tile buffers and staging slots once scoring is over.
-static_assert(sizeof(SelShared) <= IxLayout::kQ, "selection working set must fit the scoring buffers");
+// The selection's working set overlays the tile buffers once scoring is over.
+// It stays clear of the staging slots, which hold the on-chip 16-bit histogram window.
+static_assert(sizeof(SelShared) <= IxLayout::kStage, "selection working set must fit the tile buffers");
 
 // mbarrier indices
 constexpr int kBarStFull = 0;     // [8] staging slot filled (producer, tx bytes)
@@ -351,10 +352,65 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
         tc::tmem_dealloc(tmem, 64);
     }
     if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // before touching the zeroed words
-    if (multi) {   // this CTA's histogram into the query's
+    if (multi) {   // this CTA's histograms into the query's: the 11-bit one and the 16-bit one
         unsigned *gh = sel.ghist + static_cast<int64_t>(n) * kHistBins;
         for (int i = tid; i < kHistBins; i += kIxThreads)
             if (hist[i]) atomicAdd(&gh[i], hist[i]);
+        // the 16-bit histogram, counted on chip (in the free staging slots), then one atomic per
+        // nonzero 16-bit bin: the query's CTAs meet on a few hundred words, not on every score.
+        // The counters cover the 16-bit bins under the CTA's range of nonzero 11-bit bins, one range
+        // per sign of the score (keys below / above the middle bin); one atomic per score when the
+        // two ranges are too wide for the 64 KB.
+        constexpr unsigned kMid = kHistBins / 2;
+        unsigned n_lo = kMid, n_hi = 0, p_lo = kHistBins, p_hi = kMid;   // [lo, hi] per half, empty
+        for (int i = tid; i < kHistBins; i += kIxThreads)
+            if (hist[i]) {
+                const unsigned u = static_cast<unsigned>(i);
+                if (u < kMid) { n_lo = min(n_lo, u); n_hi = max(n_hi, u + 1); }
+                else { p_lo = min(p_lo, u); p_hi = max(p_hi, u + 1); }
+            }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            n_lo = min(n_lo, __shfl_xor_sync(0xffffffffu, n_lo, o));
+            n_hi = max(n_hi, __shfl_xor_sync(0xffffffffu, n_hi, o));
+            p_lo = min(p_lo, __shfl_xor_sync(0xffffffffu, p_lo, o));
+            p_hi = max(p_hi, __shfl_xor_sync(0xffffffffu, p_hi, o));
+        }
+        if (lane == 0) { s.wsum[warp] = n_lo | (n_hi << 16); s.wcnt[warp] = p_lo | (p_hi << 16); }
+        __syncthreads();
+#pragma unroll 1
+        for (int w2 = 0; w2 < kIxThreads / 32; w2++) {
+            const unsigned a = s.wsum[w2], c = s.wcnt[w2];
+            n_lo = min(n_lo, a & 0xffffu);
+            n_hi = max(n_hi, a >> 16);
+            p_lo = min(p_lo, c & 0xffffu);
+            p_hi = max(p_hi, c >> 16);
+        }
+        unsigned *gf = sel.gfine + static_cast<int64_t>(n) * kFineBins;
+        // window words: [0, wn) the negative half's range from bin fn, [wn, wn + wp) the positive one's from fp
+        const unsigned fn = n_lo * kFineSub, fp = p_lo * kFineSub;
+        const unsigned wn = n_hi > n_lo ? (n_hi - n_lo) * kFineSub : 0u;
+        const unsigned wp = p_hi > p_lo ? (p_hi - p_lo) * kFineSub : 0u;
+        auto fine_of = [&](int i) { return score_key(keep_local ? sloc[i - lo] : __ldcg(srow + i)) >> (32 - kFineBits); };
+        if (wn + wp <= static_cast<unsigned>(kIxStageRegion / 4)) {
+            unsigned *fw = reinterpret_cast<unsigned *>(stage);
+            const int nwin = static_cast<int>(wn + wp);
+            for (int i = tid; i < nwin; i += kIxThreads) fw[i] = 0;
+            __syncthreads();
+            for (int i = lo + tid; i < hi; i += kIxThreads) {
+                const unsigned d = fine_of(i);
+                const unsigned x = d < kMid * kFineSub ? d - fn : wn + (d - fp);
+                if (x < static_cast<unsigned>(nwin)) atomicAdd(&fw[x], 1u);   // always: its 11-bit bin is counted
+            }
+            __syncthreads();
+            for (int i = tid; i < nwin; i += kIxThreads)
+                if (fw[i]) {
+                    const unsigned u = static_cast<unsigned>(i);
+                    atomicAdd(&gf[fine_slot(u < wn ? fn + u : fp + (u - wn))], fw[i]);
+                }
+        } else {   // scores over too wide a range for the counters
+            for (int i = lo + tid; i < hi; i += kIxThreads) atomicAdd(&gf[fine_slot(fine_of(i))], 1u);
+        }
     }
     }   // lo < hi
     if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // (CTAs without a score range)
@@ -379,14 +435,25 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     if (n_vis > sel.select_k) {
         block_find_bin(hist, static_cast<unsigned>(sel.select_k), s);
         bstar = static_cast<int>(s.bin);
+        if (multi) {   // narrow the boundary to one of the 32 16-bit bins inside the 11-bit one
+            if (tid == 0) { s.fbin = static_cast<unsigned>(bstar) * kFineSub; s.fabove = 0; s.fcount = 0; }
+            __syncthreads();
+            if (warp == 0)
+                find_fine_bin_warp(sel.gfine + static_cast<int64_t>(n) * kFineBins, bstar,
+                                   static_cast<unsigned>(sel.select_k) - s.above, s);
+            __syncthreads();
+            bstar = static_cast<int>(s.fbin);
+        }
     }
     if (tid == 0) { s.n_a = 0; s.n_b = 0; }
     if (!multi)
         for (int i = tid; i < kHistBins; i += kIxThreads) s.hist2[i] = 0;
     __syncthreads();
-    unsigned *h2 = multi ? sel.ghist2 + static_cast<int64_t>(n) * kHistBins : s.hist2;
     auto score_at = [&](int i) { return keep_local ? sloc[i - lo] : __ldcg(srow + i); };
-    classify_range(score_at, lo, hi, bstar, h2, s);   // lo = 0, hi = n_vis when G = 1
+    if (multi)   // the 16-bit boundary: list B is a handful of entries, ranked without a level 2
+        classify_range(score_at, lo, hi, bstar, nullptr, s, 32 - kFineBits);
+    else         // lo = 0, hi = n_vis
+        classify_range(score_at, lo, hi, bstar, s.hist2, s);
     __syncthreads();
     if (sel.rows && sel.slot_map) {   // warm L2 with the slot-map lines the expansion may read
         const unsigned la = min(s.n_a, static_cast<unsigned>(kMaxSelect));
@@ -403,9 +470,17 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     if (multi) {
         if (!merge_lists_multi(cnt, sel.words + static_cast<int64_t>(n) * kMaxSelCtas,
                                sel.alist + static_cast<int64_t>(n) * sel.list_cap,
-                               sel.blist + static_cast<int64_t>(n) * sel.list_cap, per,
-                               sel.ghist2 + static_cast<int64_t>(n) * kHistBins, G, nA, nB, b_complete, s))
+                               sel.blist + static_cast<int64_t>(n) * sel.list_cap, per, nullptr, G, nA, nB,
+                               b_complete, s))
             return;
+        const unsigned fb = static_cast<unsigned>(bstar < 0 ? 0 : bstar);
+        auto get_b = [&](int i) -> unsigned long long {   // list B straight from the scores
+            const uint32_t key = score_key(__ldcg(srow + i));
+            return (key >> (32 - kFineBits)) == fb ? compose(key, i) : 0ull;
+        };
+        finish_fine(count, nA, nB, b_complete, bstar, get_b, n_vis, s);
+        write_outputs(sel, n, b, valid_b, pb, seq_len, qp, count, s);
+        return;
     } else {
         nA = min(s.n_a, static_cast<unsigned>(kMaxSelect));
         nB = s.n_b;

@@ -18,14 +18,15 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
                                int32_t *n_pools, cudaStream_t stream, int num_sms,
                                int8_t *codes = nullptr, float *scales = nullptr);   // codes: INT8 state
 // Selection and expansion arguments of the fused index kernel; topk == nullptr: scores only.
-// The multi-CTA words (ghist, ghist2, counters: 2 kHistBins + kCntWords uint32 per query) must
-// be zero at launch when index_select_ctas() > 1.
+// The multi-CTA words (ghist, ghist2, counters, gfine: 2 kHistBins + kCntWords + kFineBins uint32
+// per query) must be zero at launch when index_select_ctas() > 1.
 struct IxSelectArgs {
     int select_k;
     int32_t *topk;                 // [n_q][select_k]
     int32_t *n_sel;                // [n_q] or null
     unsigned *ghist;               // [n_q][kHistBins] level-1 histograms
     unsigned *ghist2;              // [n_q][kHistBins] level-2 histograms
+    unsigned *gfine;               // [n_q][kFineBins] histograms of the top 16 key bits
     unsigned *counters;            // [n_q][kCntWords]
     unsigned *words;               // [n_q][kMaxSelCtas] list sizes of each CTA
     unsigned long long *alist;     // [n_q][list_cap] per-CTA regions of list A

@@ -26,6 +26,10 @@ namespace glm {
 constexpr int kBoundCap = 4096;                  // list B entries kept on chip
 constexpr int kSubCap = 256;                     // level-2 boundary entries ranked directly
 constexpr int kShift2 = 64 - 2 * kHistBitsTop;   // level-2 digit: composite bits 52..42
+constexpr int kFineBits = 16;                     // multi-CTA boundary: the top 16 key bits
+constexpr int kFineBins = 1 << kFineBits;
+constexpr int kFineSub = 1 << (kFineBits - kHistBitsTop);   // 16-bit bins per 11-bit bin (32)
+constexpr int kFineRankCap = 512;                 // boundary entries ranked directly
 constexpr uint32_t kSelWaitLimit = 1u << 21;     // polls of a cross-CTA wait before giving up
 
 __device__ __forceinline__ unsigned long long compose(uint32_t key, int id) {
@@ -45,6 +49,7 @@ struct SelShared {
     unsigned part[256];
     unsigned rh[256];                      // radix fallback digit histogram
     unsigned bin, above, count;            // result of block_find_bin / find_bin_warp
+    unsigned fbin, fabove, fcount;         // the 16-bit boundary bin, the count above it, its count
     unsigned n_a, n_b, n_s, n_up;
     unsigned last, flags, maxb;
     unsigned long long prefix;
@@ -203,14 +208,14 @@ __device__ __forceinline__ void warp_append2(bool ta, unsigned *ca, bool tb, uns
 // s.bnd (list B) with their level-2 digit counted in hist2 (shared or global memory).
 template <typename ScoreAt>
 __device__ __forceinline__ void classify_range(const ScoreAt &score_at, int lo, int hi, int bstar,
-                                               unsigned *hist2, SelShared &s) {
+                                               unsigned *hist2, SelShared &s, int shift = 32 - kHistBitsTop) {
     const int T = blockDim.x;
 #pragma unroll 1
     for (int b0 = lo; b0 < hi; b0 += T) {
         const int i = b0 + static_cast<int>(threadIdx.x);
         const bool ok = i < hi;
         const uint32_t key = ok ? score_key(score_at(i)) : 0u;
-        const int d = static_cast<int>(key >> (32 - kHistBitsTop));
+        const int d = static_cast<int>(key >> shift);
         const bool a = ok && (bstar < 0 || d > bstar);
         const bool b = ok && bstar >= 0 && d == bstar;
         if (!__any_sync(0xffffffffu, a || b)) continue;
@@ -220,7 +225,7 @@ __device__ __forceinline__ void classify_range(const ScoreAt &score_at, int lo, 
         if (a && ra < static_cast<unsigned>(kMaxSelect)) s.cand[ra] = c;
         if (b) {
             if (rb < static_cast<unsigned>(kBoundCap)) s.bnd[rb] = c;
-            atomicAdd(&hist2[(c >> kShift2) & (kHistBins - 1)], 1u);
+            if (hist2) atomicAdd(&hist2[(c >> kShift2) & (kHistBins - 1)], 1u);
         }
     }
 }
@@ -510,6 +515,70 @@ __device__ __forceinline__ void finish_selection(unsigned count, unsigned nA, un
     sort_selected(s.cand, static_cast<int>(count), s);
 }
 
+// Word of 16-bit bin d in a query's 65536-bin histogram: consecutive bins lie 33 words apart, so the
+// few hundred bins a query's scores fill sit on distinct 128-byte lines and no line serialises the
+// atomics of the query's CTAs (33 is odd: the map is a bijection of [0, 65536)).
+__device__ __forceinline__ unsigned fine_slot(unsigned d) { return (d * 33u) & static_cast<unsigned>(kFineBins - 1); }
+
+// The 16-bit boundary inside 11-bit bin bstar (warp 0 only; fine = the query's 65536-bin histogram
+// in global memory): the highest of its 32 sub-bins whose suffix count reaches k1 = the number
+// still needed from bin bstar. Writes s.fbin (16-bit bin), s.fabove (count above it within bstar)
+// and s.fcount (its count).
+__device__ __forceinline__ void find_fine_bin_warp(const unsigned *fine, int bstar, unsigned k1, SelShared &s) {
+    const int lane = threadIdx.x & 31;
+    const unsigned v = __ldcg(fine + fine_slot(static_cast<unsigned>(bstar * kFineSub + lane)));
+    unsigned suf = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const unsigned y = __shfl_down_sync(0xffffffffu, suf, o);
+        if (lane + o < 32) suf += y;
+    }
+    const unsigned above = suf - v;
+    if (above < k1 && k1 <= suf) {
+        s.fbin = static_cast<unsigned>(bstar * kFineSub + lane);
+        s.fabove = above;
+        s.fcount = v;
+    }
+}
+
+// Finish a multi-CTA selection with a 16-bit boundary bin fbin: s.cand[0 .. nA) holds every entry
+// above it, s.bnd[0 .. nB) the entries of fbin (when b_complete; else get_b over m_b entries returns
+// them, 0 elsewhere). The boundary entries are ranked directly (few: a 16-bit bin is narrow), or
+// by the radix selection when they are many (ties). Leaves the count selected composites sorted.
+template <typename GetB>
+__device__ __forceinline__ void finish_fine(unsigned count, unsigned nA, unsigned nB, bool b_complete, int fbin,
+                                            const GetB &get_b, int m_b, SelShared &s) {
+    const int tid = threadIdx.x;
+    const unsigned need = count > nA ? count - nA : 0u;
+    if (need > 0) {
+        const unsigned long long top = static_cast<unsigned long long>(fbin) << (64 - kFineBits);
+        if (b_complete && nB == need) {
+#pragma unroll 1
+            for (unsigned i = tid; i < nB; i += blockDim.x)
+                if (nA + i < static_cast<unsigned>(kMaxSelect)) s.cand[nA + i] = s.bnd[i];
+            __syncthreads();
+        } else if (b_complete && nB <= static_cast<unsigned>(kFineRankCap)) {
+#pragma unroll 1
+            for (unsigned i = tid; i < nB; i += blockDim.x) {   // rank among the boundary entries
+                const unsigned long long x = s.bnd[i];
+                unsigned rank = 0;
+#pragma unroll 4
+                for (unsigned j = 0; j < nB; j++) rank += s.bnd[j] > x;
+                if (rank < need && nA + rank < static_cast<unsigned>(kMaxSelect)) s.cand[nA + rank] = x;
+            }
+            __syncthreads();
+        } else if (b_complete) {
+            auto get = [&](int i) { return s.bnd[i]; };
+            radix_select(get, static_cast<int>(nB), need, kFineBits, top, s);
+            collect_from(get, static_cast<int>(nB), ~0ull << (64 - s.done), s.prefix, nA, s);
+        } else {
+            radix_select(get_b, m_b, need, kFineBits, top, s);
+            collect_from(get_b, m_b, ~0ull << (64 - s.done), s.prefix, nA, s);
+        }
+    }
+    sort_selected(s.cand, static_cast<int>(count), s);
+}
+
 // Multi-CTA selection, after every CTA of the query has classified its slice into s.cand /
 // s.bnd (level-2 digits counted straight into the global hist2): CTA g writes its lists to its
 // own regions (al / bl + g * stride) and its list sizes to words[g] -- no shared counters --,
@@ -576,7 +645,7 @@ __device__ __forceinline__ bool merge_lists_multi(unsigned *cnt, unsigned *words
             s.flags = flags;
             s.maxb = mx;
         }
-    } else {   // meanwhile the other warps fetch the level-2 histogram
+    } else if (ghist2) {   // meanwhile the other warps fetch the level-2 histogram
 #pragma unroll 1
         for (int i = tid - 32; i < kHistBins / 4; i += blockDim.x - 32)
             reinterpret_cast<uint4 *>(s.hist2)[i] = __ldcg(reinterpret_cast<const uint4 *>(ghist2) + i);

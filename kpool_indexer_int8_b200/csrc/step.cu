@@ -1,7 +1,7 @@
 // step.cu -- the first kernel of a fused decode step: the int8 store of the new latent rows
 // ("GLM-5.3 Kernels" README, 'Included': titan_kv.store_int8), the build of the new pools
 // ("Module glm5next_dsa_ref", pool_states) and the zeroing of the step's cross-CTA counters, as
-// three independent groups of CTAs of one launch (one warp per row, one warp per pool, 16 bytes
+// three independent groups of CTAs of one launch (one warp per row, one warp per pool, 64 bytes
 // per thread of zeros), so that the three short jobs overlap instead of following one another.
 #include "append.cuh"
 #include "kernels.cuh"
@@ -10,6 +10,7 @@ namespace glm {
 
 constexpr int kPrepThreads = 256;
 constexpr int kPrepWarps = kPrepThreads / 32;
+constexpr int kZeroPerThread = 4;   // 16-byte stores per thread of a zeroing CTA
 
 __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(StepPrepArgs a, int store_ctas, int pool_ctas) {
     pdl_begin();
@@ -32,15 +33,20 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(StepPrepArgs a,
         return;
     }
     cta -= pool_ctas;
-    const int64_t i = static_cast<int64_t>(cta) * kPrepThreads + threadIdx.x;
-    if (i < a.zero_n16) a.zero[i] = make_uint4(0u, 0u, 0u, 0u);
+    const int64_t i0 = static_cast<int64_t>(cta) * kPrepThreads * kZeroPerThread + threadIdx.x;
+#pragma unroll
+    for (int k = 0; k < kZeroPerThread; k++) {
+        const int64_t i = i0 + k * kPrepThreads;
+        if (i < a.zero_n16) a.zero[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
 }
 
 cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream) {
     const int64_t items = static_cast<int64_t>(a.batch) * a.max_new_pools;
     const int store_ctas = static_cast<int>((a.n_new + kPrepWarps - 1) / kPrepWarps);
     const int pool_ctas = static_cast<int>((items + kPrepWarps - 1) / kPrepWarps);
-    const int zero_ctas = static_cast<int>((a.zero_n16 + kPrepThreads - 1) / kPrepThreads);
+    const int zero_ctas =
+        static_cast<int>((a.zero_n16 + kPrepThreads * kZeroPerThread - 1) / (kPrepThreads * kZeroPerThread));
     const int total = store_ctas + pool_ctas + zero_ctas;
     if (total == 0) return cudaSuccess;
     launch_pdl(step_prep_kernel, dim3(static_cast<unsigned>(total)), dim3(kPrepThreads), 0, stream, a, store_ctas,

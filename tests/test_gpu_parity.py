@@ -256,11 +256,13 @@ _FUSED_CASES = [synth.TINY_DECODE, synth.PADDING_DECODE,
 
 
 @pytest.mark.parametrize("wl", _FUSED_CASES, ids=lambda w: w.name)
-@pytest.mark.parametrize("pattern", ["synth", "few", "equal"])
+@pytest.mark.parametrize("pattern", ["synth", "few", "equal", "signed", "wide"])
 def test_fused_select_expand_bit_exact_on_own_scores(cuda, wl, pattern):
     # the one-launch scores + selection + expansion: its top-k rows must be exactly the oracle's
     # selection of the scores it wrote, and its tokens / rows exactly the oracle's expansion of
-    # that selection ("few": 3 distinct pooled keys, "equal": one -- only pool ids decide)
+    # that selection ("few": 3 distinct pooled keys, "equal": one -- only pool ids decide;
+    # "signed": head weights of both signs, so scores of both signs; "wide": signed, and pooled
+    # keys scaled over 2^-60 .. 2^60, so a CTA's scores fill hundreds of 11-bit bins)
     inp = synth.generate(wl)
     b = sdev.allocate_for(inp, cuda, keep_scores=True)
     sdev.load(inp, b, build_prefix=True)
@@ -268,6 +270,11 @@ def test_fused_select_expand_bit_exact_on_own_scores(cuda, wl, pattern):
         b.pooled.copy_(b.pooled[:, torch.arange(b.pooled.shape[1], device=cuda) % 3])
     elif pattern == "equal":
         b.pooled.copy_(b.pooled[:, :1].expand_as(b.pooled))
+    if pattern in ("signed", "wide"):
+        b.w.mul_(torch.where(torch.arange(b.w.shape[1], device=cuda) % 3 == 0, -1.5, 1.0))
+    if pattern == "wide":
+        e = (torch.arange(b.pooled.shape[1], device=cuda) * 37 % 121 - 60).float()
+        b.pooled.mul_(torch.exp2(e)[None, :, None])
     for t in (b.topk, b.n_sel, b.tok, b.rows):
         t.fill_(4242)
     b.scores.fill_(7.0)
