@@ -27,10 +27,11 @@ int num_sms() {
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace of a selection (first in the workspace of both selection entry points): per query
-// two 2048-bin histograms of score keys, kCntWords counters and a 65536-bin histogram of the top
-// 16 key bits (all zeroed by one kernel before a selection that spans several CTAs; the selection
-// on given scores uses no 16-bit histogram), the list sizes of each CTA, and the per-CTA regions of
-// list A (candidates above the boundary bin) and list B (the boundary bin).
+// two 2048-bin histograms of score keys and kCntWords counters (zeroed by one kernel before a
+// selection that spans several CTAs), a 65536-bin histogram of the top 16 key bits (zeroed by the
+// fused index kernel itself; the selection on given scores uses none), the list sizes of each
+// CTA, and the per-CTA regions of list A (candidates above the boundary bin) and list B (the
+// boundary bin).
 struct SelWs {
     unsigned *hist;
     unsigned *hist2;
@@ -39,22 +40,19 @@ struct SelWs {
     unsigned *words;
     unsigned long long *alist;
     unsigned long long *blist;
-    size_t zero_bytes;        // everything above
-    size_t zero_bytes_small;  // without the 16-bit histograms
+    size_t zero_bytes;   // hist, hist2 and counters
 };
-size_t sel_small_zero_bytes(int n_q) {
+size_t sel_zero_bytes(int n_q) {
     return static_cast<size_t>(n_q) * (2 * glm::kHistBins + glm::kCntWords) * sizeof(unsigned);
 }
-size_t sel_zero_bytes(int n_q) {
-    return sel_small_zero_bytes(n_q) + static_cast<size_t>(n_q) * glm::kFineBins * sizeof(unsigned);
-}
+size_t sel_fine_bytes(int n_q) { return static_cast<size_t>(n_q) * glm::kFineBins * sizeof(unsigned); }
 size_t sel_list_bytes(int n_q, int64_t ld) {
     return align_up(static_cast<size_t>(n_q) * static_cast<size_t>(glm::sel_list_cap(ld)) *
                     sizeof(unsigned long long), 256);
 }
 size_t sel_words_bytes(int n_q) { return align_up(static_cast<size_t>(n_q) * glm::kMaxSelCtas * sizeof(unsigned), 256); }
 size_t sel_bytes(int n_q, int64_t ld) {
-    return align_up(sel_zero_bytes(n_q), 256) + sel_words_bytes(n_q) + 2 * sel_list_bytes(n_q, ld);
+    return align_up(sel_zero_bytes(n_q), 256) + sel_fine_bytes(n_q) + sel_words_bytes(n_q) + 2 * sel_list_bytes(n_q, ld);
 }
 SelWs sel_layout(void *base, int n_q, int64_t ld) {
     char *p = static_cast<char *>(base);
@@ -62,10 +60,10 @@ SelWs sel_layout(void *base, int n_q, int64_t ld) {
     w.hist = reinterpret_cast<unsigned *>(p);
     w.hist2 = w.hist + static_cast<size_t>(n_q) * glm::kHistBins;
     w.counters = w.hist2 + static_cast<size_t>(n_q) * glm::kHistBins;
-    w.fine = w.counters + static_cast<size_t>(n_q) * glm::kCntWords;
     w.zero_bytes = sel_zero_bytes(n_q);
-    w.zero_bytes_small = sel_small_zero_bytes(n_q);
     p += align_up(w.zero_bytes, 256);
+    w.fine = reinterpret_cast<unsigned *>(p);
+    p += sel_fine_bytes(n_q);
     w.words = reinterpret_cast<unsigned *>(p);
     p += sel_words_bytes(n_q);
     w.alist = reinterpret_cast<unsigned long long *>(p);
@@ -419,7 +417,7 @@ int glm_topk_pools(const float *scores, int64_t ld_scores, const int32_t *n_visi
     const SelWs sw = sel_layout(workspace, n_q, ld_scores);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const glm::NvisSource src{n_visible, nullptr, nullptr, nullptr, nullptr, 0, ld_scores};
-    int rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes_small, 16), st));
+    int rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
     if (rc != GLM_OK) return rc;
     rc = cuda_status(glm::launch_topk_hist(scores, src, n_q, sw.hist, st));
     if (rc != GLM_OK) return rc;

@@ -57,13 +57,22 @@ struct IxLayout {                                      // offsets from a 1024-by
     static constexpr int kW = kLocal + kIxLocalCap * 4;               // 32 fp32 head weights
     static constexpr int kBar = kW + kIdxHeads * 4;                   // 24 mbarriers
     static constexpr int kTmem = kBar + 24 * 8;
-    static constexpr int kFlag = kTmem + 16;
-    static constexpr int kBytes = kFlag + 16;
+    static constexpr int kFlag = kTmem + 16;                          // 8 words, see kFl*
+    static constexpr int kBytes = kFlag + 32;
     static constexpr int kAlloc = kBytes + 1024;                      // room to align the base
 };
 // The selection's working set overlays the tile buffers once scoring is over.
 // It stays clear of the staging slots, which hold the on-chip 16-bit histogram window.
 static_assert(sizeof(SelShared) <= IxLayout::kStage, "selection working set must fit the tile buffers");
+
+// words at IxLayout::kFlag
+constexpr int kFlBarrier = 0;   // the grid barrier gave up
+constexpr int kFlNegLo = 1;     // the CTA's nonzero 11-bit bins of negative scores: [lo, hi)
+constexpr int kFlNegHi = 2;
+constexpr int kFlPosLo = 3;     // ... of non-negative scores
+constexpr int kFlPosHi = 4;
+constexpr int kFlZeroed = 5;    // the wait for the zeroed 16-bit histogram gave up
+constexpr unsigned kMidBin = kHistBins / 2;   // keys below it: negative scores
 
 // mbarrier indices
 constexpr int kBarStFull = 0;     // [8] staging slot filled (producer, tx bytes)
@@ -214,6 +223,13 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     if (tid < kIdxHeads) ws[tid] = w[static_cast<int64_t>(n) * kIdxHeads + tid];
     if (select)
         for (int i = tid; i < kHistBins; i += kIxThreads) hist[i] = 0;
+    if (tid == 64) {
+        flag[kFlNegLo] = kMidBin;
+        flag[kFlNegHi] = 0;
+        flag[kFlPosLo] = kHistBins;
+        flag[kFlPosHi] = kMidBin;
+        flag[kFlZeroed] = 0;
+    }
     tc::fence_proxy_async();
     __syncthreads();
     tc::fence_after_sync();
@@ -266,6 +282,23 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                 tc::mma_commit(bar(kBarTmEmpty + tb));
                 tc::mma_commit(bar(kBarAccFull + tb));
             }
+        }
+    } else if (warp == 2) {
+        // ---------------- zeroing of the query's 16-bit histogram ----------------
+        // Every launch before this one on the stream has ended (this one starts once its
+        // predecessor has waited for its own), so the histogram is free; each CTA with a score
+        // range zeroes its share and arrives, and none adds to it before all have arrived.
+        if (multi) {
+            const int g_eff = (n_vis + per - 1) / per;   // CTAs with a score range
+            const int share = (kFineBins / 4 + g_eff - 1) / g_eff;
+            uint4 *gf4 = reinterpret_cast<uint4 *>(sel.gfine + static_cast<int64_t>(n) * kFineBins);
+            for (int i = g * share + lane; i < min((g + 1) * share, kFineBins / 4); i += 32)
+                gf4[i] = make_uint4(0u, 0u, 0u, 0u);
+            __threadfence();
+            __syncwarp();
+            if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // the counters are zeroed
+            if (lane == 0 && !grid_barrier(&sel.counters[static_cast<int64_t>(n) * kCntWords + kCntZeroed], g_eff))
+                flag[kFlZeroed] = 1;
         }
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue: TMEM lane quadrant (warp % 4), rows 16q .. 16q+15 ----------------
@@ -353,41 +386,33 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     }
     if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // before touching the zeroed words
     if (multi) {   // this CTA's histograms into the query's: the 11-bit one and the 16-bit one
+        static_assert(kHistBins == 4 * kIxThreads, "four 11-bit bins per thread");
+        const uint4 h4 = reinterpret_cast<const uint4 *>(hist)[tid];   // bins 4 tid .. 4 tid + 3
+        const unsigned b0 = 4u * static_cast<unsigned>(tid);
         unsigned *gh = sel.ghist + static_cast<int64_t>(n) * kHistBins;
-        for (int i = tid; i < kHistBins; i += kIxThreads)
-            if (hist[i]) atomicAdd(&gh[i], hist[i]);
+        if (h4.x) atomicAdd(&gh[b0], h4.x);
+        if (h4.y) atomicAdd(&gh[b0 + 1], h4.y);
+        if (h4.z) atomicAdd(&gh[b0 + 2], h4.z);
+        if (h4.w) atomicAdd(&gh[b0 + 3], h4.w);
+        // the CTA's range of nonzero 11-bit bins per score sign (a warp's bins share one sign)
+        const unsigned nzm = (h4.x != 0u ? 1u : 0u) | (h4.y != 0u ? 2u : 0u) | (h4.z != 0u ? 4u : 0u) |
+                             (h4.w != 0u ? 8u : 0u);
+        const bool neg = b0 < kMidBin;
+        const unsigned r_lo = __reduce_min_sync(0xffffffffu, nzm ? b0 + __ffs(nzm) - 1 : (neg ? kMidBin : kHistBins));
+        const unsigned r_hi = __reduce_max_sync(0xffffffffu, nzm ? b0 + 32 - __clz(nzm) : (neg ? 0u : kMidBin));
+        if (lane == 0) {
+            atomicMin(&flag[neg ? kFlNegLo : kFlPosLo], r_lo);
+            atomicMax(&flag[neg ? kFlNegHi : kFlPosHi], r_hi);
+        }
+        __syncthreads();
+        if (tid == 0 && flag[kFlZeroed] && status) atomicOr(status, 8);
         // the 16-bit histogram, counted on chip (in the free staging slots), then one atomic per
         // nonzero 16-bit bin: the query's CTAs meet on a few hundred words, not on every score.
-        // The counters cover the 16-bit bins under the CTA's range of nonzero 11-bit bins, one range
-        // per sign of the score (keys below / above the middle bin); one atomic per score when the
-        // two ranges are too wide for the 64 KB.
-        constexpr unsigned kMid = kHistBins / 2;
-        unsigned n_lo = kMid, n_hi = 0, p_lo = kHistBins, p_hi = kMid;   // [lo, hi] per half, empty
-        for (int i = tid; i < kHistBins; i += kIxThreads)
-            if (hist[i]) {
-                const unsigned u = static_cast<unsigned>(i);
-                if (u < kMid) { n_lo = min(n_lo, u); n_hi = max(n_hi, u + 1); }
-                else { p_lo = min(p_lo, u); p_hi = max(p_hi, u + 1); }
-            }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            n_lo = min(n_lo, __shfl_xor_sync(0xffffffffu, n_lo, o));
-            n_hi = max(n_hi, __shfl_xor_sync(0xffffffffu, n_hi, o));
-            p_lo = min(p_lo, __shfl_xor_sync(0xffffffffu, p_lo, o));
-            p_hi = max(p_hi, __shfl_xor_sync(0xffffffffu, p_hi, o));
-        }
-        if (lane == 0) { s.wsum[warp] = n_lo | (n_hi << 16); s.wcnt[warp] = p_lo | (p_hi << 16); }
-        __syncthreads();
-#pragma unroll 1
-        for (int w2 = 0; w2 < kIxThreads / 32; w2++) {
-            const unsigned a = s.wsum[w2], c = s.wcnt[w2];
-            n_lo = min(n_lo, a & 0xffffu);
-            n_hi = max(n_hi, a >> 16);
-            p_lo = min(p_lo, c & 0xffffu);
-            p_hi = max(p_hi, c >> 16);
-        }
+        // The counters cover the 16-bit bins under each sign's range of nonzero 11-bit bins; one
+        // atomic per score when the two ranges are too wide for the 64 KB.
+        const unsigned n_lo = flag[kFlNegLo], n_hi = flag[kFlNegHi], p_lo = flag[kFlPosLo], p_hi = flag[kFlPosHi];
         unsigned *gf = sel.gfine + static_cast<int64_t>(n) * kFineBins;
-        // window words: [0, wn) the negative half's range from bin fn, [wn, wn + wp) the positive one's from fp
+        // window words: [0, wn) the negative range's from bin fn, [wn, wn + wp) the non-negative one's from fp
         const unsigned fn = n_lo * kFineSub, fp = p_lo * kFineSub;
         const unsigned wn = n_hi > n_lo ? (n_hi - n_lo) * kFineSub : 0u;
         const unsigned wp = p_hi > p_lo ? (p_hi - p_lo) * kFineSub : 0u;
@@ -399,7 +424,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             __syncthreads();
             for (int i = lo + tid; i < hi; i += kIxThreads) {
                 const unsigned d = fine_of(i);
-                const unsigned x = d < kMid * kFineSub ? d - fn : wn + (d - fp);
+                const unsigned x = d < kMidBin * kFineSub ? d - fn : wn + (d - fp);
                 if (x < static_cast<unsigned>(nwin)) atomicAdd(&fw[x], 1u);   // always: its 11-bit bin is counted
             }
             __syncthreads();
@@ -421,11 +446,11 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     if (multi) {   // grid barrier of the query's CTAs, then the summed histogram
         __syncthreads();
         if (tid == 0) {   // release this CTA's histogram, arrive, wait (acquire) for the others
-            *flag = grid_barrier(&cnt[kCntArrive], G) ? 0u : 1u;
-            if (*flag && status) atomicOr(status, 8);
+            flag[kFlBarrier] = grid_barrier(&cnt[kCntArrive], G) ? 0u : 1u;
+            if (flag[kFlBarrier] && status) atomicOr(status, 8);
         }
         __syncthreads();
-        if (*flag) return;   // gave up waiting: the status word reports it
+        if (flag[kFlBarrier]) return;   // gave up waiting: the status word reports it
         const uint4 *gh = reinterpret_cast<const uint4 *>(sel.ghist + static_cast<int64_t>(n) * kHistBins);
         for (int i = tid; i < kHistBins / 4; i += kIxThreads) reinterpret_cast<uint4 *>(hist)[i] = __ldcg(gh + i);
         __syncthreads();

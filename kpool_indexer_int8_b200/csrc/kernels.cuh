@@ -18,8 +18,10 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
                                int32_t *n_pools, cudaStream_t stream, int num_sms,
                                int8_t *codes = nullptr, float *scales = nullptr);   // codes: INT8 state
 // Selection and expansion arguments of the fused index kernel; topk == nullptr: scores only.
-// The multi-CTA words (ghist, ghist2, counters, gfine: 2 kHistBins + kCntWords + kFineBins uint32
-// per query) must be zero at launch when index_select_ctas() > 1.
+// The multi-CTA words (ghist, ghist2, counters: 2 kHistBins + kCntWords uint32 per query) must be
+// zero at launch when index_select_ctas() > 1; gfine (kFineBins uint32 per query, 16-byte aligned)
+// needs no zeroing: the kernel zeroes it, and every launch before it on the stream must have ended
+// (or be the kernel that zeroes the words, launched before it).
 struct IxSelectArgs {
     int select_k;
     int32_t *topk;                 // [n_q][select_k]

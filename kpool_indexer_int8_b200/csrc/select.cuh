@@ -60,7 +60,7 @@ struct SelShared {
 };
 
 // Per-query words of a multi-CTA selection in global memory (zeroed before the launch).
-enum SelCounter { kCntArrive = 0, kCntTicket = 1, kCntWords = 8 };
+enum SelCounter { kCntArrive = 0, kCntTicket = 1, kCntZeroed = 2, kCntWords = 8 };
 constexpr int kMaxSelCtas = 256;   // CTAs of one query in a multi-CTA selection (per-CTA list words)
 
 // Bytes per query of the multi-CTA lists: each CTA g of a query writes its list A and list B at

@@ -49,6 +49,12 @@ cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream) {
         static_cast<int>((a.zero_n16 + kPrepThreads * kZeroPerThread - 1) / (kPrepThreads * kZeroPerThread));
     const int total = store_ctas + pool_ctas + zero_ctas;
     if (total == 0) return cudaSuccess;
+    // Keep the SMs that run these CTAs configured for the most shared memory: the fused index
+    // kernel's CTAs (one per SM, ~190 KB each) start beside them under programmatic dependent
+    // launch, which a smaller carve-out would hold back until these CTAs end.
+    cudaError_t e = cudaFuncSetAttribute(step_prep_kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                         cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
     launch_pdl(step_prep_kernel, dim3(static_cast<unsigned>(total)), dim3(kPrepThreads), 0, stream, a, store_ctas,
                pool_ctas);
     return cudaGetLastError();
