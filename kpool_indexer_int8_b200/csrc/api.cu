@@ -28,8 +28,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Workspace of a selection (first in the workspace of both selection entry points): per query
 // two 2048-bin histograms of score keys and kCntWords counters (zeroed by one kernel before a
-// selection that spans several CTAs), a 65536-bin histogram of the top 16 key bits (zeroed by the
-// fused index kernel itself; the selection on given scores uses none), the list sizes of each
+// selection that spans several CTAs), the sample keys the CTAs of the fused index kernel publish
+// (kSampleUnion per query; the selection on given scores uses none), the list sizes of each
 // CTA, and the per-CTA regions of list A (candidates above the boundary bin) and list B (the
 // boundary bin).
 struct SelWs {
@@ -45,7 +45,7 @@ struct SelWs {
 size_t sel_zero_bytes(int n_q) {
     return static_cast<size_t>(n_q) * (2 * glm::kHistBins + glm::kCntWords) * sizeof(unsigned);
 }
-size_t sel_fine_bytes(int n_q) { return static_cast<size_t>(n_q) * glm::kFineBins * sizeof(unsigned); }
+size_t sel_fine_bytes(int n_q) { return align_up(static_cast<size_t>(n_q) * glm::kSampleUnion * sizeof(unsigned), 256); }
 size_t sel_list_bytes(int n_q, int64_t ld) {
     return align_up(static_cast<size_t>(n_q) * static_cast<size_t>(glm::sel_list_cap(ld)) *
                     sizeof(unsigned long long), 256);
@@ -304,7 +304,7 @@ int enqueue_index_select(const void *q_idx, const float *w, const void *keys, co
     sel.n_sel = n_sel;
     sel.ghist = sw.hist;
     sel.ghist2 = sw.hist2;
-    sel.gfine = sw.fine;
+    sel.gsamp = sw.fine;
     sel.counters = sw.counters;
     sel.words = sw.words;
     sel.alist = sw.alist;

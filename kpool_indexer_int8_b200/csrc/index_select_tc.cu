@@ -15,14 +15,20 @@
 //     fp32 tensor-memory accumulators; with the bf16 query exact, the three terms reproduce q . x
 //     to fp32 accumulation accuracy;
 //   * epilogue (warps 4-7, one TMEM lane quadrant each): relu and head weights, the score (to
-//     global memory and, when the range is short enough, to shared memory), and its top-11-bit
-//     key digit counted in the CTA's histogram.
-// Phase 2, selection (select.cuh): with G > 1 the CTA histograms are summed in global memory and
-// the G CTAs of a query meet at a grid barrier (all CTAs are resident: at most one per SM; the wait
-// is bounded); every CTA then classifies its own scores against the boundary
-// bin, appends them to the query's global lists, and the last CTA to finish (ticket) completes
-// the selection, sorts it, and writes the top-k row, n_sel and the expanded token / row indices.
-// With G = 1 the one CTA does all of it on chip.
+//     global memory and, when the range is short enough, to shared memory), and (one CTA per
+//     query) its top-11-bit key digit counted in the CTA's histogram.
+// Selection with G = 1: the one CTA selects on chip (histogram boundary bin, lists, sort).
+// Selection with G > 1 -- a sample threshold, so that the query's CTAs meet while the keys still
+// stream: the first tiles of every CTA's range (about an eighth of it) are a sample of the
+// query's scores. While phase 1 runs, warp 2 of each CTA adds its sample to the query's 11-bit and
+// 16-bit key histograms in global memory (zeroed by the kernel before this one); the CTAs meet
+// (all are resident, at most one per SM; every wait is bounded), and each finds the 16-bit key
+// bin of the k_s-th largest sample score,
+// k_s = 1.5 select_k (sample size / visible pools) + 16. Scores whose key reaches that bin are
+// candidates (about 1.5 select_k of them): when phase 1 ends, each CTA writes its candidates to its
+// region of the query's list, and the last CTA to finish (ticket) gathers them, sorts them and
+// keeps the select_k largest. The threshold only prunes: if fewer than select_k scores (or more
+// than the list holds on chip) pass it, the last CTA selects exactly over every score of the row.
 // Phase 1 is HBM-bound: 512 bytes of pooled key per pool; the tensor cores run at a few percent.
 // With the INT8 indexer state ("GLM-5.3-Flash" pypto-lib page, 'What is quantized': the indexer
 // cache in INT8 with one FP32 scale per row) a pool is 128 code bytes plus its scale: 4 KB bulk
@@ -47,6 +53,8 @@ constexpr int kIxStageRegion = 4 * kIxChunk * kIdxDim * 4;   // 64 KB: 4 x 16 KB
 constexpr uint32_t kIxWaitLimit = 1u << 22;
 
 constexpr int kIxLocalCap = 4096;                      // scores of a CTA kept in shared memory
+constexpr int kIxSampleTiles = 8;                      // most tiles of a CTA's range in the sample
+constexpr int kIxSampleMax = kIxSampleTiles * kIxTile;
 
 struct IxLayout {                                      // offsets from a 1024-byte aligned base
     static constexpr int kTerms = 0;                                  // [2 buffers][3 terms][16 KB]
@@ -55,24 +63,21 @@ struct IxLayout {                                      // offsets from a 1024-by
     static constexpr int kHist = kQ + kIdxHeads * kIdxDim * 2;        // 2048 uint32
     static constexpr int kLocal = kHist + kHistBins * 4;              // kIxLocalCap fp32 scores
     static constexpr int kW = kLocal + kIxLocalCap * 4;               // 32 fp32 head weights
-    static constexpr int kBar = kW + kIdxHeads * 4;                   // 24 mbarriers
-    static constexpr int kTmem = kBar + 24 * 8;
+    static constexpr int kBar = kW + kIdxHeads * 4;                   // 25 mbarriers
+    static constexpr int kTmem = kBar + 25 * 8;
     static constexpr int kFlag = kTmem + 16;                          // 8 words, see kFl*
-    static constexpr int kBytes = kFlag + 32;
+    static constexpr int kSamp = (kFlag + 32 + 15) / 16 * 16;         // the CTA's sample keys
+    static constexpr int kScr = kSamp + kIxSampleMax * 4;             // the published keys, staged
+    static constexpr int kBytes = kScr + 16 * 4;
     static constexpr int kAlloc = kBytes + 1024;                      // room to align the base
 };
+static_assert(IxLayout::kScr % 16 == 0, "the threshold's staged keys are read as 16-byte vectors");
 // The selection's working set overlays the tile buffers once scoring is over.
-// It stays clear of the staging slots, which hold the on-chip 16-bit histogram window.
 static_assert(sizeof(SelShared) <= IxLayout::kStage, "selection working set must fit the tile buffers");
 
 // words at IxLayout::kFlag
-constexpr int kFlBarrier = 0;   // the grid barrier gave up
-constexpr int kFlNegLo = 1;     // the CTA's nonzero 11-bit bins of negative scores: [lo, hi)
-constexpr int kFlNegHi = 2;
-constexpr int kFlPosLo = 3;     // ... of non-negative scores
-constexpr int kFlPosHi = 4;
-constexpr int kFlZeroed = 5;    // the wait for the zeroed 16-bit histogram gave up
-constexpr unsigned kMidBin = kHistBins / 2;   // keys below it: negative scores
+constexpr int kFlThr = 0;       // the sample threshold: a candidate's key is at least this
+constexpr int kFlWait = 1;      // a wait of the threshold warp on the query's other CTAs gave up
 
 // mbarrier indices
 constexpr int kBarStFull = 0;     // [8] staging slot filled (producer, tx bytes)
@@ -81,6 +86,7 @@ constexpr int kBarTmFull = 16;    // [2] tile buffer written (8 warps x 2 chunk 
 constexpr int kBarTmEmpty = 18;   // [2] tile buffer read by the MMAs (commit)
 constexpr int kBarAccFull = 20;   // [2] accumulator ready (commit)
 constexpr int kBarAccEmpty = 22;  // [2] accumulator read (4 epilogue warps)
+constexpr int kBarSample = 24;    // the sample keys are in shared memory (4 epilogue warps)
 
 __device__ __forceinline__ uint32_t bf16_pair(float a, float b) {
     const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low half), .y = b
@@ -88,6 +94,112 @@ __device__ __forceinline__ uint32_t bf16_pair(float a, float b) {
 }
 __device__ __forceinline__ float bf16_lo_f(uint32_t p) { return __uint_as_float(p << 16); }
 __device__ __forceinline__ float bf16_hi_f(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
+
+// The k-th largest sample key of a query (warp 2 of each of its n_ctas CTAs): CTA g publishes
+// the r largest of its n_samp sample keys (r a multiple of 4; 0 where it has fewer) at gs + g r --
+// lane 0 stores them, then releases them as it arrives at the meeting word *ctr --, the CTAs meet,
+// and each reads the n_ctas r published keys (at most kSampleUnion, eight 16-byte loads per lane)
+// and finds the k-th largest, rounded down to its top kThrBits bits, by a binary search on the
+// key bits (stage: kPubMax words of shared memory). The published keys are a subset of the
+// sample, so the result is at most the sample's k-th largest key: a threshold that lets through
+// at least as many scores. Returns 0 -- every score passes -- when fewer than k keys are
+// published. ok turns false on lane 0 if the wait gave up.
+constexpr int kPubMax = 16;   // published keys per CTA, at most
+constexpr int kThrBits = 16;  // bits of the threshold key that are searched (the rest are 0)
+__device__ __noinline__ unsigned sample_threshold(const unsigned *samp, int n_samp, int r, unsigned k,
+                                                  unsigned *gs, int g, unsigned *ctr, int n_ctas,
+                                                  unsigned *stage, bool &ok) {
+    const int lane = threadIdx.x & 31;
+    // this CTA's r largest keys: r rounds of a warp-wide maximum over the lanes' own keys
+    unsigned kv[kIxSampleMax / 32];
+#pragma unroll
+    for (int j = 0; j < kIxSampleMax / 32; j++) {
+        const int i = j * 32 + lane;
+        kv[j] = i < n_samp ? samp[i] : 0u;
+    }
+    unsigned *top = stage;   // the r keys, largest first
+#pragma unroll 1
+    for (int q = 0; q < r; q++) {
+        unsigned m = 0u;
+#pragma unroll
+        for (int j = 0; j < kIxSampleMax / 32; j++) m = max(m, kv[j]);
+        const unsigned M = __reduce_max_sync(0xffffffffu, m);
+        if (lane == 0) top[q] = M;
+        const unsigned own = __ballot_sync(0xffffffffu, m == M);
+        if (lane == __ffs(own) - 1) {   // that lane drops one copy of M
+            bool done = false;
+#pragma unroll
+            for (int j = 0; j < kIxSampleMax / 32; j++)
+                if (!done && kv[j] == M) { kv[j] = 0u; done = true; }
+        }
+    }
+    if (lane == 0) {
+#pragma unroll 1
+        for (int q = 0; q < r; q += 4)
+            *reinterpret_cast<uint4 *>(gs + static_cast<int64_t>(g) * r + q) = *reinterpret_cast<const uint4 *>(top + q);
+        if (!grid_barrier(ctr, n_ctas)) ok = false;
+    }
+    __syncwarp();   // the other lanes wait for lane 0's acquire
+    const int U = n_ctas * r;
+    if (static_cast<unsigned>(U) < k) return 0u;
+    uint4 u[kSampleUnion / 128];
+#pragma unroll
+    for (int j = 0; j < kSampleUnion / 128; j++) {
+        const int i = j * 32 + lane;   // 16-byte piece: keys 4 i .. 4 i + 3
+        u[j] = 4 * i < U ? __ldcg(reinterpret_cast<const uint4 *>(gs) + i) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // the k-th largest published key, to 16 bits (rounded down: a threshold at most that key), by
+    // a binary search on its bits: keep each bit if at least k keys reach the prefix with it set
+    unsigned prefix = 0u;
+#pragma unroll 1
+    for (int bit = 31; bit >= 32 - kThrBits; bit--) {
+        const unsigned cand = prefix | (1u << bit);
+        unsigned c = 0u;
+#pragma unroll
+        for (int j = 0; j < kSampleUnion / 128; j++)   // (absent keys are 0 and never count)
+            c += (u[j].x >= cand) + (u[j].y >= cand) + (u[j].z >= cand) + (u[j].w >= cand);
+        if (__reduce_add_sync(0xffffffffu, c) >= k) prefix = cand;
+    }
+    return prefix;
+}
+
+// The last CTA of a multi-CTA selection gathers the candidates of the query's n_ctas CTAs into
+// s.bnd (count in s.n_b; entries past kBoundCap are counted but dropped): region c of the list
+// (at reg_q + c * stride) holds its count in slot 0 and its candidates from slot 1. One warp
+// reads 32 slots of each of its CTAs, all loads in flight together; longer regions are finished
+// 32 slots at a time.
+constexpr int kCandK = 10;   // CTAs per warp whose first 32 slots are loaded together
+__device__ __noinline__ void gather_candidates(const unsigned long long *reg_q, int stride, int n_ctas,
+                                               SelShared &s) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll 1
+    for (int c0 = 0; c0 < n_ctas; c0 += nw * kCandK) {
+        unsigned long long v[kCandK];
+#pragma unroll
+        for (int k = 0; k < kCandK; k++) {
+            const int c = c0 + warp + nw * k;
+            v[k] = c < n_ctas ? __ldcg(reg_q + static_cast<long long>(c) * stride + lane) : 0ull;
+        }
+#pragma unroll
+        for (int k = 0; k < kCandK; k++) {
+            const int c = c0 + warp + nw * k;
+            if (c >= n_ctas) break;
+            const unsigned cnt = min(static_cast<unsigned>(__shfl_sync(0xffffffffu, v[k], 0)),
+                                     static_cast<unsigned>(stride - 1));   // (a region holds stride - 1)
+            const bool take = lane >= 1 && static_cast<unsigned>(lane) <= cnt;
+            const unsigned pos = warp_append(take, &s.n_b);
+            if (take && pos < static_cast<unsigned>(kBoundCap)) s.bnd[pos] = v[k];
+#pragma unroll 1
+            for (unsigned j0 = 32; j0 <= cnt; j0 += 32) {
+                const unsigned j = j0 + lane;
+                const bool t = j <= cnt;
+                const unsigned long long x = t ? __ldcg(reg_q + static_cast<long long>(c) * stride + j) : 0ull;
+                const unsigned q = warp_append(t, &s.n_b);
+                if (t && q < static_cast<unsigned>(kBoundCap)) s.bnd[q] = x;
+            }
+        }
+    }
+}
 
 // Write the outputs of a query whose selection is final (s.cand[0 .. count) sorted): the top-k
 // row, n_sel, and the expansion into tokens / cache rows (the rules of expand_selection).
@@ -148,8 +260,10 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     constexpr int kStageBytes = kIxChunk * kIdxDim * kElem;       // one chunk of keys
     constexpr int kNumTerms = kQ8 ? 1 : 3;                        // bf16 terms per key
     static_assert(kStages * kStageBytes <= kIxStageRegion && kStages <= kIxMaxStages, "staging");
-    if (sel.early) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    else pdl_begin();
+    // The next kernel of the stream may launch only once this one's CTAs reach the selection (its
+    // CTAs then take the SMs the finished CTAs free). Early mode: wait for the preceding kernel
+    // only where its outputs are needed; otherwise at once.
+    if (!sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
     unsigned char *terms = smem + IxLayout::kTerms;
@@ -160,6 +274,8 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     float *ws = reinterpret_cast<float *>(smem + IxLayout::kW);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + IxLayout::kTmem);
     unsigned *flag = reinterpret_cast<unsigned *>(smem + IxLayout::kFlag);
+    unsigned *samp = reinterpret_cast<unsigned *>(smem + IxLayout::kSamp);
+    unsigned *scr = reinterpret_cast<unsigned *>(smem + IxLayout::kScr);
 
     const int n = blockIdx.y, g = blockIdx.x, G = gridDim.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -191,6 +307,18 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     const int lo = min(n_vis, g * per);
     const int hi = min(n_vis, lo + per);
     const bool keep_local = select && per <= kIxLocalCap;
+    const int g_eff = (n_vis + per - 1) / per;   // CTAs with a score range
+    // multi-CTA sample: the first n_st0 tiles of every CTA's range; m_all keys in all, and the
+    // threshold is the k_s-th largest of them (no threshold when the sample is that small)
+    const int n_st0 = min(kIxSampleTiles, max(1, (per + 8 * kIxTile - 1) / (8 * kIxTile)));
+    const int s0 = n_st0 * kIxTile;
+    const long long m_all = static_cast<long long>(g_eff - 1) * min(s0, per) + min(s0, n_vis - (g_eff - 1) * per);
+    const long long k_s = (3ll * sel.select_k * m_all + 2ll * n_vis - 1) / (2ll * n_vis) + 16;
+    const bool sample = multi && n_vis > sel.select_k && k_s < m_all;
+    // keys each CTA publishes for the threshold: enough that their union holds about 2 k_s, a
+    // multiple of 4, and at most kSampleUnion in all
+    const int r_pub = min(min(kPubMax, (kSampleUnion / max(g_eff, 1)) & ~3),
+                          max(4, static_cast<int>((2 * k_s + g_eff - 1) / max(g_eff, 1) + 3) & ~3));
     if (lo < hi) {
     const int n_chunks = (hi - lo + kIxChunk - 1) / kIxChunk;
     const int n_tiles = (hi - lo + kIxTile - 1) / kIxTile;
@@ -211,6 +339,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
         for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarTmEmpty + i), 1);
         for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccFull + i), 1);
         for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccEmpty + i), 4);
+        tc::mbar_init(bar(kBarSample), 4);
         tc::mbar_fence_init();
     }
     // query block (bf16 [32 x 128], core matrices: head group stride 2048 B, dim group 128 B)
@@ -221,14 +350,11 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             __ldg(reinterpret_cast<const uint4 *>(qn) + i);
     }
     if (tid < kIdxHeads) ws[tid] = w[static_cast<int64_t>(n) * kIdxHeads + tid];
-    if (select)
+    if (select && !multi)
         for (int i = tid; i < kHistBins; i += kIxThreads) hist[i] = 0;
     if (tid == 64) {
-        flag[kFlNegLo] = kMidBin;
-        flag[kFlNegHi] = 0;
-        flag[kFlPosLo] = kHistBins;
-        flag[kFlPosHi] = kMidBin;
-        flag[kFlZeroed] = 0;
+        flag[kFlThr] = 0;
+        flag[kFlWait] = 0;
     }
     tc::fence_proxy_async();
     __syncthreads();
@@ -284,25 +410,27 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             }
         }
     } else if (warp == 2) {
-        // ---------------- zeroing of the query's 16-bit histogram ----------------
-        // Every launch before this one on the stream has ended (this one starts once its
-        // predecessor has waited for its own), so the histogram is free; each CTA with a score
-        // range zeroes its share and arrives, and none adds to it before all have arrived.
-        if (multi) {
-            const int g_eff = (n_vis + per - 1) / per;   // CTAs with a score range
-            const int share = (kFineBins / 4 + g_eff - 1) / g_eff;
-            uint4 *gf4 = reinterpret_cast<uint4 *>(sel.gfine + static_cast<int64_t>(n) * kFineBins);
-            for (int i = g * share + lane; i < min((g + 1) * share, kFineBins / 4); i += 32)
-                gf4[i] = make_uint4(0u, 0u, 0u, 0u);
-            __threadfence();
+        // ---------------- the multi-CTA selection's sample threshold ----------------
+        // Once the epilogue has scored the sample tiles: publish this CTA's largest sample keys,
+        // meet the query's other CTAs, and select the threshold from all published keys.
+        if (sample) {
+            unsigned *cq = sel.counters + static_cast<int64_t>(n) * kCntWords;
+            if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // the meeting word is zeroed
+            bool waited = tc::mbar_wait(bar(kBarSample), 0, kIxWaitLimit);   // the sample keys are written
             __syncwarp();
-            if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // the counters are zeroed
-            if (lane == 0 && !grid_barrier(&sel.counters[static_cast<int64_t>(n) * kCntWords + kCntZeroed], g_eff))
-                flag[kFlZeroed] = 1;
+            const unsigned thr = sample_threshold(samp, min(s0, hi - lo), r_pub, static_cast<unsigned>(k_s),
+                                                  sel.gsamp + static_cast<int64_t>(n) * kSampleUnion, g,
+                                                  &cq[kCntSample], g_eff, scr, waited);
+            if (lane == 0) {
+                flag[kFlThr] = thr;
+                if (!waited) flag[kFlWait] = 1;
+            }
+            __syncwarp();
         }
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue: TMEM lane quadrant (warp % 4), rows 16q .. 16q+15 ----------------
         const int qd = warp & 3;
+        const int n_st = min(n_st0, n_tiles);   // tiles of the sample (multi-CTA selection)
         for (int t = 0; t < n_tiles; t++) {
             const int tb = t & 1;
             const int p = lo + t * kIxTile + qd * 16 + lane;
@@ -322,12 +450,18 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                 if (kQ8) sc *= ksc;   // relu(s q.c) = s relu(q.c) for the scale s > 0
                 srow[p] = sc;
                 if (keep_local) sloc[p - lo] = sc;
-                digit = score_key(sc) >> (32 - kHistBitsTop);
+                const uint32_t key = score_key(sc);
+                if (sample && t < n_st) samp[p - lo] = key;
+                digit = key >> (32 - kHistBitsTop);
             }
-            if (select && digit != 0xffffffffu) atomicAdd(&hist[digit], 1u);
+            if (select && !multi && digit != 0xffffffffu) atomicAdd(&hist[digit], 1u);
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(kBarAccEmpty + tb));
+            if (sample && t == n_st - 1) {   // the sample keys of this warp's rows are written
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(kBarSample));
+            }
         }
     } else if (warp >= 16 - kIxConv) {
         // ---------------- converters ----------------
@@ -384,101 +518,83 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, 64);
     }
-    if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // before touching the zeroed words
-    if (multi) {   // this CTA's histograms into the query's: the 11-bit one and the 16-bit one
-        static_assert(kHistBins == 4 * kIxThreads, "four 11-bit bins per thread");
-        const uint4 h4 = reinterpret_cast<const uint4 *>(hist)[tid];   // bins 4 tid .. 4 tid + 3
-        const unsigned b0 = 4u * static_cast<unsigned>(tid);
-        unsigned *gh = sel.ghist + static_cast<int64_t>(n) * kHistBins;
-        if (h4.x) atomicAdd(&gh[b0], h4.x);
-        if (h4.y) atomicAdd(&gh[b0 + 1], h4.y);
-        if (h4.z) atomicAdd(&gh[b0 + 2], h4.z);
-        if (h4.w) atomicAdd(&gh[b0 + 3], h4.w);
-        // the CTA's range of nonzero 11-bit bins per score sign (a warp's bins share one sign)
-        const unsigned nzm = (h4.x != 0u ? 1u : 0u) | (h4.y != 0u ? 2u : 0u) | (h4.z != 0u ? 4u : 0u) |
-                             (h4.w != 0u ? 8u : 0u);
-        const bool neg = b0 < kMidBin;
-        const unsigned r_lo = __reduce_min_sync(0xffffffffu, nzm ? b0 + __ffs(nzm) - 1 : (neg ? kMidBin : kHistBins));
-        const unsigned r_hi = __reduce_max_sync(0xffffffffu, nzm ? b0 + 32 - __clz(nzm) : (neg ? 0u : kMidBin));
-        if (lane == 0) {
-            atomicMin(&flag[neg ? kFlNegLo : kFlPosLo], r_lo);
-            atomicMax(&flag[neg ? kFlNegHi : kFlPosHi], r_hi);
-        }
-        __syncthreads();
-        if (tid == 0 && flag[kFlZeroed] && status) atomicOr(status, 8);
-        // the 16-bit histogram, counted on chip (in the free staging slots), then one atomic per
-        // nonzero 16-bit bin: the query's CTAs meet on a few hundred words, not on every score.
-        // The counters cover the 16-bit bins under each sign's range of nonzero 11-bit bins; one
-        // atomic per score when the two ranges are too wide for the 64 KB.
-        const unsigned n_lo = flag[kFlNegLo], n_hi = flag[kFlNegHi], p_lo = flag[kFlPosLo], p_hi = flag[kFlPosHi];
-        unsigned *gf = sel.gfine + static_cast<int64_t>(n) * kFineBins;
-        // window words: [0, wn) the negative range's from bin fn, [wn, wn + wp) the non-negative one's from fp
-        const unsigned fn = n_lo * kFineSub, fp = p_lo * kFineSub;
-        const unsigned wn = n_hi > n_lo ? (n_hi - n_lo) * kFineSub : 0u;
-        const unsigned wp = p_hi > p_lo ? (p_hi - p_lo) * kFineSub : 0u;
-        auto fine_of = [&](int i) { return score_key(keep_local ? sloc[i - lo] : __ldcg(srow + i)) >> (32 - kFineBits); };
-        if (wn + wp <= static_cast<unsigned>(kIxStageRegion / 4)) {
-            unsigned *fw = reinterpret_cast<unsigned *>(stage);
-            const int nwin = static_cast<int>(wn + wp);
-            for (int i = tid; i < nwin; i += kIxThreads) fw[i] = 0;
-            __syncthreads();
-            for (int i = lo + tid; i < hi; i += kIxThreads) {
-                const unsigned d = fine_of(i);
-                const unsigned x = d < kMidBin * kFineSub ? d - fn : wn + (d - fp);
-                if (x < static_cast<unsigned>(nwin)) atomicAdd(&fw[x], 1u);   // always: its 11-bit bin is counted
-            }
-            __syncthreads();
-            for (int i = tid; i < nwin; i += kIxThreads)
-                if (fw[i]) {
-                    const unsigned u = static_cast<unsigned>(i);
-                    atomicAdd(&gf[fine_slot(u < wn ? fn + u : fp + (u - wn))], fw[i]);
-                }
-        } else {   // scores over too wide a range for the counters
-            for (int i = lo + tid; i < hi; i += kIxThreads) atomicAdd(&gf[fine_slot(fine_of(i))], 1u);
-        }
-    }
     }   // lo < hi
-    if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // (CTAs without a score range)
+    if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (!select) return;
+    const unsigned count = static_cast<unsigned>(min(sel.select_k, n_vis));
+    auto score_at = [&](int i) { return keep_local ? sloc[i - lo] : __ldcg(srow + i); };
 
     // ---------------- phase 2: selection (every MMA and bulk copy of this CTA has completed) ----------------
     unsigned *cnt = sel.counters + static_cast<int64_t>(n) * kCntWords;
-    if (multi) {   // grid barrier of the query's CTAs, then the summed histogram
+    if (multi) {
+        if (lo >= hi) return;   // no score range: not part of the query's selection
+        if (tid == 0 && flag[kFlWait] && status) atomicOr(status, 8);
+        // this CTA's candidates (scores whose key reaches the sample threshold) to its region of
+        // the query's list: slot 0 the count, then the composites
+        const unsigned thr = flag[kFlThr];
+        const int stride = per + 1;
+        unsigned long long *reg_q = sel.alist + static_cast<int64_t>(n) * sel.list_cap;
+        unsigned long long *reg = reg_q + static_cast<int64_t>(g) * stride;
+        if (tid == 0) s.n_b = 0;
         __syncthreads();
-        if (tid == 0) {   // release this CTA's histogram, arrive, wait (acquire) for the others
-            flag[kFlBarrier] = grid_barrier(&cnt[kCntArrive], G) ? 0u : 1u;
-            if (flag[kFlBarrier] && status) atomicOr(status, 8);
+#pragma unroll 1
+        for (int b0 = lo; b0 < hi; b0 += kIxThreads) {
+            const int i = b0 + tid;
+            const uint32_t key = i < hi ? score_key(score_at(i)) : 0u;
+            const bool take = i < hi && key >= thr;
+            if (!__any_sync(0xffffffffu, take)) continue;
+            const unsigned pos = warp_append(take, &s.n_b);
+            if (take) {
+                reg[1 + pos] = compose(key, i);
+                const long long t0 = pb + static_cast<long long>(kKpool) * i;   // warm L2 for the expansion
+                if (sel.rows && sel.slot_map && t0 >= 0 && t0 + kKpool <= sel.ld_slot)
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(sel.slot_map + static_cast<int64_t>(b) * sel.ld_slot + t0));
+            }
         }
         __syncthreads();
-        if (flag[kFlBarrier]) return;   // gave up waiting: the status word reports it
-        const uint4 *gh = reinterpret_cast<const uint4 *>(sel.ghist + static_cast<int64_t>(n) * kHistBins);
-        for (int i = tid; i < kHistBins / 4; i += kIxThreads) reinterpret_cast<uint4 *>(hist)[i] = __ldcg(gh + i);
+        if (tid == 0) {   // release the region, take the ticket; the last CTA acquires every region
+            reg[0] = s.n_b;
+            s.last = take_ticket(&cnt[kCntTicket], g_eff) ? 1u : 0u;
+        }
         __syncthreads();
+        if (!s.last) return;
+        if (tid == 0) s.n_b = 0;
+        __syncthreads();
+        gather_candidates(reg_q, stride, g_eff, s);
+        __syncthreads();
+        const unsigned total = s.n_b;
+        if (total >= count && total <= static_cast<unsigned>(kBoundCap)) {
+            if (total <= static_cast<unsigned>(kMaxSelect)) {   // sort them all, keep the first count
+#pragma unroll 1
+                for (unsigned i = tid; i < total; i += kIxThreads) s.cand[i] = s.bnd[i];
+                __syncthreads();
+                sort_selected(s.cand, static_cast<int>(total), s);
+            } else {
+                auto get = [&](int i) { return s.bnd[i]; };
+                radix_select(get, static_cast<int>(total), count, 0, 0ull, s);
+                collect_from(get, static_cast<int>(total), ~0ull << (64 - s.done), s.prefix, 0u, s);
+                sort_selected(s.cand, static_cast<int>(count), s);
+            }
+        } else {   // the threshold let too few (or too many) through: exact over every score of the row
+            auto get = [&](int i) { return compose(score_key(__ldcg(srow + i)), i); };
+            radix_select(get, n_vis, count, 0, 0ull, s);
+            collect_from(get, n_vis, ~0ull << (64 - s.done), s.prefix, 0u, s);
+            sort_selected(s.cand, static_cast<int>(count), s);
+        }
+        write_outputs(sel, n, b, valid_b, pb, seq_len, qp, count, s);
+        return;
     }
-    const unsigned count = static_cast<unsigned>(min(sel.select_k, n_vis));
+    // one CTA: lo = 0, hi = n_vis, the histogram and the scores on chip
     int bstar = -1;   // every visible pool is selected
     if (n_vis > sel.select_k) {
         block_find_bin(hist, static_cast<unsigned>(sel.select_k), s);
         bstar = static_cast<int>(s.bin);
-        if (multi) {   // narrow the boundary to one of the 32 16-bit bins inside the 11-bit one
-            if (tid == 0) { s.fbin = static_cast<unsigned>(bstar) * kFineSub; s.fabove = 0; s.fcount = 0; }
-            __syncthreads();
-            if (warp == 0)
-                find_fine_bin_warp(sel.gfine + static_cast<int64_t>(n) * kFineBins, bstar,
-                                   static_cast<unsigned>(sel.select_k) - s.above, s);
-            __syncthreads();
-            bstar = static_cast<int>(s.fbin);
-        }
     }
     if (tid == 0) { s.n_a = 0; s.n_b = 0; }
-    if (!multi)
-        for (int i = tid; i < kHistBins; i += kIxThreads) s.hist2[i] = 0;
+    for (int i = tid; i < kHistBins; i += kIxThreads) s.hist2[i] = 0;
     __syncthreads();
-    auto score_at = [&](int i) { return keep_local ? sloc[i - lo] : __ldcg(srow + i); };
-    if (multi)   // the 16-bit boundary: list B is a handful of entries, ranked without a level 2
-        classify_range(score_at, lo, hi, bstar, nullptr, s, 32 - kFineBits);
-    else         // lo = 0, hi = n_vis
-        classify_range(score_at, lo, hi, bstar, s.hist2, s);
+    classify_range(score_at, lo, hi, bstar, s.hist2, s);
     __syncthreads();
     if (sel.rows && sel.slot_map) {   // warm L2 with the slot-map lines the expansion may read
         const unsigned la = min(s.n_a, static_cast<unsigned>(kMaxSelect));
@@ -490,27 +606,9 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                 asm volatile("prefetch.global.L2 [%0];" ::"l"(sel.slot_map + static_cast<int64_t>(b) * sel.ld_slot + t0));
         }
     }
-    unsigned nA, nB;
-    bool b_complete;
-    if (multi) {
-        if (!merge_lists_multi(cnt, sel.words + static_cast<int64_t>(n) * kMaxSelCtas,
-                               sel.alist + static_cast<int64_t>(n) * sel.list_cap,
-                               sel.blist + static_cast<int64_t>(n) * sel.list_cap, per, nullptr, G, nA, nB,
-                               b_complete, s))
-            return;
-        const unsigned fb = static_cast<unsigned>(bstar < 0 ? 0 : bstar);
-        auto get_b = [&](int i) -> unsigned long long {   // list B straight from the scores
-            const uint32_t key = score_key(__ldcg(srow + i));
-            return (key >> (32 - kFineBits)) == fb ? compose(key, i) : 0ull;
-        };
-        finish_fine(count, nA, nB, b_complete, bstar, get_b, n_vis, s);
-        write_outputs(sel, n, b, valid_b, pb, seq_len, qp, count, s);
-        return;
-    } else {
-        nA = min(s.n_a, static_cast<unsigned>(kMaxSelect));
-        nB = s.n_b;
-        b_complete = nB <= static_cast<unsigned>(kBoundCap);
-    }
+    const unsigned nA = min(s.n_a, static_cast<unsigned>(kMaxSelect));
+    const unsigned nB = s.n_b;
+    const bool b_complete = nB <= static_cast<unsigned>(kBoundCap);
     const unsigned long long top = static_cast<unsigned long long>(bstar < 0 ? 0 : bstar);
     auto get_b = [&](int i) -> unsigned long long {   // list B straight from the scores
         const uint32_t key = score_key(__ldcg(srow + i));

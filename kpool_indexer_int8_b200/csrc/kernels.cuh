@@ -18,17 +18,17 @@ cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_token
                                int32_t *n_pools, cudaStream_t stream, int num_sms,
                                int8_t *codes = nullptr, float *scales = nullptr);   // codes: INT8 state
 // Selection and expansion arguments of the fused index kernel; topk == nullptr: scores only.
-// The multi-CTA words (ghist, ghist2, counters: 2 kHistBins + kCntWords uint32 per query) must be
-// zero at launch when index_select_ctas() > 1; gfine (kFineBins uint32 per query, 16-byte aligned)
-// needs no zeroing: the kernel zeroes it, and every launch before it on the stream must have ended
-// (or be the kernel that zeroes the words, launched before it).
+// The multi-CTA counters (kCntWords uint32 per query) must be zero at launch when
+// index_select_ctas() > 1 (or be zeroed by the kernel launched just before it, which the kernel
+// waits for before it touches them); gsamp (kSampleUnion uint32 per query, 16-byte aligned) needs
+// no zeroing. ghist and ghist2 are not used by this kernel.
 struct IxSelectArgs {
     int select_k;
     int32_t *topk;                 // [n_q][select_k]
     int32_t *n_sel;                // [n_q] or null
     unsigned *ghist;               // [n_q][kHistBins] level-1 histograms
     unsigned *ghist2;              // [n_q][kHistBins] level-2 histograms
-    unsigned *gfine;               // [n_q][kFineBins] histograms of the top 16 key bits
+    unsigned *gsamp;               // [n_q][kSampleUnion] sample keys published by the CTAs
     unsigned *counters;            // [n_q][kCntWords]
     unsigned *words;               // [n_q][kMaxSelCtas] list sizes of each CTA
     unsigned long long *alist;     // [n_q][list_cap] per-CTA regions of list A

@@ -3,7 +3,7 @@
 //
 //   M = max_c m_c,  L = sum_c l_c e^{m_c - M},  out = (sum_c e^{m_c - M} acc_c) / L,
 //   lse = M + log L.
-// Chunks with l = 0 (no valid entry) are skipped without reading their accumulator.
+// Chunks with l = 0 (no valid entry) contribute nothing (their accumulators were never written).
 #include "common.cuh"
 #include "sparse_mla.cuh"
 
@@ -12,10 +12,21 @@ namespace glm {
 constexpr int kMaxCombineChunks = 1024;  // 65536 / 64
 constexpr int kCombineThreads = 512;
 constexpr int kChunkGroups = kCombineThreads / (kLatent / 4);   // 4 groups of 128 threads
+constexpr int kFirstLoads = 9;   // chunks per thread whose accumulators load with the (m, l) pairs
+
+__device__ __forceinline__ void fma4(float4 &a, float w, const float4 &v) {
+    a.x = fmaf(w, v.x, a.x);
+    a.y = fmaf(w, v.y, a.y);
+    a.z = fmaf(w, v.z, a.z);
+    a.w = fmaf(w, v.w, a.w);
+}
 
 // One CTA of 512 threads per (head, query): thread t owns output columns [4 (t % 128), +4) of
-// chunk group t / 128 (chunks c = group, group + 4, ...), all of its chunk loads in flight at
-// once; the 4 group sums are added in shared memory.
+// chunk group t / 128 (chunks c = group, group + 4, ...). The accumulators of its first
+// kFirstLoads chunks are loaded together with every chunk's (m, l), so that one round trip to L2
+// serves both; the weights follow from the (m, l) pairs, the rest of the chunks (if any) load 8 at
+// a time, and the 4 group sums are added in shared memory. A chunk without a valid entry (l = 0)
+// was never written: its accumulator is dropped, never multiplied.
 __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const float *__restrict__ part_acc,
                                                                       const float *__restrict__ part_ml,
                                                                       int n_heads, int n_chunks,
@@ -24,15 +35,27 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const floa
                                                                       float *__restrict__ lse) {
     pdl_begin();
     __shared__ float wgt[kMaxCombineChunks];
+    __shared__ float lsum[kMaxCombineChunks];
     __shared__ float red[kCombineThreads / 32];
     __shared__ float4 part[kChunkGroups - 1][kLatent / 4];
     const int h = blockIdx.x, n = blockIdx.y, t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int64_t base = static_cast<int64_t>(n) * n_chunks * n_heads + h;
-    // every chunk's (m, l) at once; M = the largest m of a chunk with an entry
+    const int col = t % (kLatent / 4), grp = t / (kLatent / 4);
+    auto acc_at = [&](int c) {
+        return __ldcg(reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(c) * n_heads) * kLatent) + col);
+    };
+    float4 v[kFirstLoads];
+#pragma unroll
+    for (int u = 0; u < kFirstLoads; u++) {
+        const int cu = grp + u * kChunkGroups;
+        v[u] = cu < n_chunks ? acc_at(cu) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // every chunk's (m, l); M = the largest m of a chunk with an entry
     float mx = -INFINITY;
     for (int c = t; c < n_chunks; c += kCombineThreads) {
-        const float2 ml = *reinterpret_cast<const float2 *>(part_ml + 2 * (base + static_cast<int64_t>(c) * n_heads));
+        const float2 ml = __ldcg(reinterpret_cast<const float2 *>(part_ml + 2 * (base + static_cast<int64_t>(c) * n_heads)));
         wgt[c] = ml.y > 0.0f ? ml.x : -INFINITY;
+        lsum[c] = ml.y;
         if (ml.y > 0.0f) mx = fmaxf(mx, ml.x);
     }
     mx = warp_max(mx);
@@ -46,42 +69,36 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const floa
         const float m = wgt[c];
         const float wc = (m == -INFINITY || M == -INFINITY) ? 0.0f : expf(m - M);
         wgt[c] = wc;
-        Lp = fmaf(part_ml[2 * (base + static_cast<int64_t>(c) * n_heads) + 1], wc, Lp);
+        Lp = fmaf(lsum[c], wc, Lp);
     }
     Lp = warp_sum(Lp);
     if (lane == 0) red[warp] = Lp;
     __syncthreads();
     float L = lane < kCombineThreads / 32 ? red[lane] : 0.0f;
     L = warp_sum(L);
-    // this thread's columns over its chunk group, eight chunk loads in flight
-    const int col = t % (kLatent / 4), grp = t / (kLatent / 4);
     float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-    int c = grp;
+#pragma unroll
+    for (int u = 0; u < kFirstLoads; u++) {
+        const int cu = grp + u * kChunkGroups;
+        if (cu < n_chunks && wgt[cu] > 0.0f) fma4(a, wgt[cu], v[u]);
+    }
+    int c = grp + kFirstLoads * kChunkGroups;
     for (; c + 7 * kChunkGroups < n_chunks; c += 8 * kChunkGroups) {
-        float4 v[8];
+        float4 r[8];
 #pragma unroll
         for (int u = 0; u < 8; u++) {
             const int cu = c + u * kChunkGroups;
-            v[u] = wgt[cu] > 0.0f ? reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(cu) * n_heads) * kLatent)[col]
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+            r[u] = wgt[cu] > 0.0f ? acc_at(cu) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int u = 0; u < 8; u++) {
             const float wc = wgt[c + u * kChunkGroups];
-            a.x = fmaf(wc, v[u].x, a.x);
-            a.y = fmaf(wc, v[u].y, a.y);
-            a.z = fmaf(wc, v[u].z, a.z);
-            a.w = fmaf(wc, v[u].w, a.w);
+            if (wc > 0.0f) fma4(a, wc, r[u]);
         }
     }
     for (; c < n_chunks; c += kChunkGroups) {
         const float wc = wgt[c];
-        if (!(wc > 0.0f)) continue;
-        const float4 v = reinterpret_cast<const float4 *>(part_acc + (base + static_cast<int64_t>(c) * n_heads) * kLatent)[col];
-        a.x = fmaf(wc, v.x, a.x);
-        a.y = fmaf(wc, v.y, a.y);
-        a.z = fmaf(wc, v.z, a.z);
-        a.w = fmaf(wc, v.w, a.w);
+        if (wc > 0.0f) fma4(a, wc, acc_at(c));
     }
     if (grp > 0) part[grp - 1][col] = a;
     __syncthreads();

@@ -26,10 +26,6 @@ namespace glm {
 constexpr int kBoundCap = 4096;                  // list B entries kept on chip
 constexpr int kSubCap = 256;                     // level-2 boundary entries ranked directly
 constexpr int kShift2 = 64 - 2 * kHistBitsTop;   // level-2 digit: composite bits 52..42
-constexpr int kFineBits = 16;                     // multi-CTA boundary: the top 16 key bits
-constexpr int kFineBins = 1 << kFineBits;
-constexpr int kFineSub = 1 << (kFineBits - kHistBitsTop);   // 16-bit bins per 11-bit bin (32)
-constexpr int kFineRankCap = 512;                 // boundary entries ranked directly
 constexpr uint32_t kSelWaitLimit = 1u << 21;     // polls of a cross-CTA wait before giving up
 
 __device__ __forceinline__ unsigned long long compose(uint32_t key, int id) {
@@ -60,13 +56,15 @@ struct SelShared {
 };
 
 // Per-query words of a multi-CTA selection in global memory (zeroed before the launch).
-enum SelCounter { kCntArrive = 0, kCntTicket = 1, kCntZeroed = 2, kCntWords = 8 };
+enum SelCounter { kCntArrive = 0, kCntTicket = 1, kCntSample = 2, kCntWords = 8 };
 constexpr int kMaxSelCtas = 256;   // CTAs of one query in a multi-CTA selection (per-CTA list words)
+constexpr int kSampleUnion = 1024; // sample keys the CTAs of one query publish (at most)
 
-// Bytes per query of the multi-CTA lists: each CTA g of a query writes its list A and list B at
-// g * stride (stride = the CTA's score range, >= 64) of regions of list_cap(ld) composites; with
-// G * stride <= n_vis + 64 G and 64 G <= ld + 63, 2 ld + 64 always suffices.
-__host__ __device__ constexpr long long sel_list_cap(long long ld) { return 2 * ld + 64; }
+// Composites per query of each multi-CTA list region: CTA g of a query writes at g * stride, where
+// stride is at most its score range per + 1 (per = max(ceil(n_vis / G), 64), G <= ceil(ld / 64) and
+// G <= 256): G * (per + 1) is at most ld + 2 G <= ld + 512 when per > 64, and 65 G <= 1.02 ld + 65
+// when per = 64, so 2 ld + 512 always suffices.
+__host__ __device__ constexpr long long sel_list_cap(long long ld) { return 2 * ld + 512; }
 
 __device__ __forceinline__ unsigned ld_acquire(const unsigned *p) {
     unsigned v;
@@ -237,7 +235,7 @@ template <typename Get>
 __device__ __noinline__ void radix_select(const Get &get, int m, unsigned k, int known_bits,
                                              unsigned long long prefix, SelShared &s) {
     const int tid = threadIdx.x;
-    unsigned long long mask = ~0ull << (64 - known_bits);
+    unsigned long long mask = known_bits > 0 ? ~0ull << (64 - known_bits) : 0ull;
     int bits = known_bits;
     while (bits < 64) {
         const int width = min(8, 64 - bits);
@@ -509,70 +507,6 @@ __device__ __forceinline__ void finish_selection(unsigned count, unsigned nA, un
             }
         } else {   // list B did not fit on chip: radix selection straight from its source
             radix_select(get_b, m_b, need, kHistBitsTop, top, s);
-            collect_from(get_b, m_b, ~0ull << (64 - s.done), s.prefix, nA, s);
-        }
-    }
-    sort_selected(s.cand, static_cast<int>(count), s);
-}
-
-// Word of 16-bit bin d in a query's 65536-bin histogram: consecutive bins lie 33 words apart, so the
-// few hundred bins a query's scores fill sit on distinct 128-byte lines and no line serialises the
-// atomics of the query's CTAs (33 is odd: the map is a bijection of [0, 65536)).
-__device__ __forceinline__ unsigned fine_slot(unsigned d) { return (d * 33u) & static_cast<unsigned>(kFineBins - 1); }
-
-// The 16-bit boundary inside 11-bit bin bstar (warp 0 only; fine = the query's 65536-bin histogram
-// in global memory): the highest of its 32 sub-bins whose suffix count reaches k1 = the number
-// still needed from bin bstar. Writes s.fbin (16-bit bin), s.fabove (count above it within bstar)
-// and s.fcount (its count).
-__device__ __forceinline__ void find_fine_bin_warp(const unsigned *fine, int bstar, unsigned k1, SelShared &s) {
-    const int lane = threadIdx.x & 31;
-    const unsigned v = __ldcg(fine + fine_slot(static_cast<unsigned>(bstar * kFineSub + lane)));
-    unsigned suf = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const unsigned y = __shfl_down_sync(0xffffffffu, suf, o);
-        if (lane + o < 32) suf += y;
-    }
-    const unsigned above = suf - v;
-    if (above < k1 && k1 <= suf) {
-        s.fbin = static_cast<unsigned>(bstar * kFineSub + lane);
-        s.fabove = above;
-        s.fcount = v;
-    }
-}
-
-// Finish a multi-CTA selection with a 16-bit boundary bin fbin: s.cand[0 .. nA) holds every entry
-// above it, s.bnd[0 .. nB) the entries of fbin (when b_complete; else get_b over m_b entries returns
-// them, 0 elsewhere). The boundary entries are ranked directly (few: a 16-bit bin is narrow), or
-// by the radix selection when they are many (ties). Leaves the count selected composites sorted.
-template <typename GetB>
-__device__ __forceinline__ void finish_fine(unsigned count, unsigned nA, unsigned nB, bool b_complete, int fbin,
-                                            const GetB &get_b, int m_b, SelShared &s) {
-    const int tid = threadIdx.x;
-    const unsigned need = count > nA ? count - nA : 0u;
-    if (need > 0) {
-        const unsigned long long top = static_cast<unsigned long long>(fbin) << (64 - kFineBits);
-        if (b_complete && nB == need) {
-#pragma unroll 1
-            for (unsigned i = tid; i < nB; i += blockDim.x)
-                if (nA + i < static_cast<unsigned>(kMaxSelect)) s.cand[nA + i] = s.bnd[i];
-            __syncthreads();
-        } else if (b_complete && nB <= static_cast<unsigned>(kFineRankCap)) {
-#pragma unroll 1
-            for (unsigned i = tid; i < nB; i += blockDim.x) {   // rank among the boundary entries
-                const unsigned long long x = s.bnd[i];
-                unsigned rank = 0;
-#pragma unroll 4
-                for (unsigned j = 0; j < nB; j++) rank += s.bnd[j] > x;
-                if (rank < need && nA + rank < static_cast<unsigned>(kMaxSelect)) s.cand[nA + rank] = x;
-            }
-            __syncthreads();
-        } else if (b_complete) {
-            auto get = [&](int i) { return s.bnd[i]; };
-            radix_select(get, static_cast<int>(nB), need, kFineBits, top, s);
-            collect_from(get, static_cast<int>(nB), ~0ull << (64 - s.done), s.prefix, nA, s);
-        } else {
-            radix_select(get_b, m_b, need, kFineBits, top, s);
             collect_from(get_b, m_b, ~0ull << (64 - s.done), s.prefix, nA, s);
         }
     }

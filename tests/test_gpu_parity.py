@@ -256,13 +256,16 @@ _FUSED_CASES = [synth.TINY_DECODE, synth.PADDING_DECODE,
 
 
 @pytest.mark.parametrize("wl", _FUSED_CASES, ids=lambda w: w.name)
-@pytest.mark.parametrize("pattern", ["synth", "few", "equal", "signed", "wide"])
+@pytest.mark.parametrize("pattern", ["synth", "few", "equal", "signed", "wide", "lead", "trend"])
 def test_fused_select_expand_bit_exact_on_own_scores(cuda, wl, pattern):
     # the one-launch scores + selection + expansion: its top-k rows must be exactly the oracle's
     # selection of the scores it wrote, and its tokens / rows exactly the oracle's expansion of
     # that selection ("few": 3 distinct pooled keys, "equal": one -- only pool ids decide;
     # "signed": head weights of both signs, so scores of both signs; "wide": signed, and pooled
-    # keys scaled over 2^-60 .. 2^60, so a CTA's scores fill hundreds of 11-bit bins)
+    # keys scaled over 2^-60 .. 2^60, so a CTA's scores fill hundreds of 11-bit bins; "lead": the
+    # first tile of every CTA's range scaled x8, so that the multi-CTA sample overstates the
+    # scores and its threshold lets too few through; "trend": keys scaled up along the sequence,
+    # so that the candidates crowd into the last CTAs' ranges)
     inp = synth.generate(wl)
     b = sdev.allocate_for(inp, cuda, keep_scores=True)
     sdev.load(inp, b, build_prefix=True)
@@ -275,6 +278,16 @@ def test_fused_select_expand_bit_exact_on_own_scores(cuda, wl, pattern):
     if pattern == "wide":
         e = (torch.arange(b.pooled.shape[1], device=cuda) * 37 % 121 - 60).float()
         b.pooled.mul_(torch.exp2(e)[None, :, None])
+    if pattern in ("lead", "trend"):
+        ld, n_q = b.pooled.shape[1], len(inp.q_pos)
+        G = min(max(1, torch.cuda.get_device_properties(cuda).multi_processor_count // n_q), -(-ld // 64))
+        p = torch.arange(ld, device=cuda)
+        for n in range(n_q):
+            s = int(inp.q_seq[n])
+            nv = max(1, oracle.n_visible_pools(inp.pad[s], inp.len[s], inp.q_pos[n]))
+            per = max(-(-nv // G), 64)
+            f = torch.where(p % per < 64, 8.0, 1.0) if pattern == "lead" else 1.0 + 3.0 * p.float() / nv
+            b.pooled[s].mul_(f[:, None])
     for t in (b.topk, b.n_sel, b.tok, b.rows):
         t.fill_(4242)
     b.scores.fill_(7.0)
