@@ -20,15 +20,16 @@
 // Selection with G = 1: the one CTA selects on chip (histogram boundary bin, lists, sort).
 // Selection with G > 1 -- a sample threshold, so that the query's CTAs meet while the keys still
 // stream: the first tiles of every CTA's range (about an eighth of it) are a sample of the
-// query's scores. While phase 1 runs, warp 2 of each CTA adds its sample to the query's 11-bit and
-// 16-bit key histograms in global memory (zeroed by the kernel before this one); the CTAs meet
-// (all are resident, at most one per SM; every wait is bounded), and each finds the 16-bit key
-// bin of the k_s-th largest sample score,
-// k_s = 1.5 select_k (sample size / visible pools) + 16. Scores whose key reaches that bin are
-// candidates (about 1.5 select_k of them): when phase 1 ends, each CTA writes its candidates to its
-// region of the query's list, and the last CTA to finish (ticket) gathers them, sorts them and
-// keeps the select_k largest. The threshold only prunes: if fewer than select_k scores (or more
-// than the list holds on chip) pass it, the last CTA selects exactly over every score of the row.
+// query's scores. While phase 1 runs, warp 2 of each CTA publishes its largest sample keys, the
+// CTAs meet (all are resident, at most one per SM; every wait is bounded), and each finds the
+// k_s-th largest published key (k_s = 1.5 select_k sample size / visible pools + 16), rounded down
+// to 16 bits: the threshold. Scores whose key reaches it are candidates (about 1.5 select_k of
+// them): when phase 1 ends, each CTA appends its candidates to the query's list (an offset from a
+// counter), the CTAs meet again, and every CTA loads the whole list, ranks its share of it exactly
+// (the number of larger composites) and writes the outputs of the select_k best; one CTA writes
+// the rest (padding, n_sel, the visible tail). The threshold only prunes: if fewer than select_k
+// scores (or more than the list holds on chip) pass it, one CTA selects exactly over every score
+// of the row.
 // Phase 1 is HBM-bound: 512 bytes of pooled key per pool; the tensor cores run at a few percent.
 // With the INT8 indexer state ("GLM-5.3-Flash" pypto-lib page, 'What is quantized': the indexer
 // cache in INT8 with one FP32 scale per row) a pool is 128 code bytes plus its scale: 4 KB bulk
@@ -77,7 +78,7 @@ static_assert(sizeof(SelShared) <= IxLayout::kStage, "selection working set must
 
 // words at IxLayout::kFlag
 constexpr int kFlThr = 0;       // the sample threshold: a candidate's key is at least this
-constexpr int kFlWait = 1;      // a wait of the threshold warp on the query's other CTAs gave up
+constexpr int kFlWait = 1;      // a wait on the query's other CTAs gave up
 
 // mbarrier indices
 constexpr int kBarStFull = 0;     // [8] staging slot filled (producer, tx bytes)
@@ -163,41 +164,47 @@ __device__ __noinline__ unsigned sample_threshold(const unsigned *samp, int n_sa
     return prefix;
 }
 
-// The last CTA of a multi-CTA selection gathers the candidates of the query's n_ctas CTAs into
-// s.bnd (count in s.n_b; entries past kBoundCap are counted but dropped): region c of the list
-// (at reg_q + c * stride) holds its count in slot 0 and its candidates from slot 1. One warp
-// reads 32 slots of each of its CTAs, all loads in flight together; longer regions are finished
-// 32 slots at a time.
-constexpr int kCandK = 10;   // CTAs per warp whose first 32 slots are loaded together
-__device__ __noinline__ void gather_candidates(const unsigned long long *reg_q, int stride, int n_ctas,
-                                               SelShared &s) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-#pragma unroll 1
-    for (int c0 = 0; c0 < n_ctas; c0 += nw * kCandK) {
-        unsigned long long v[kCandK];
-#pragma unroll
-        for (int k = 0; k < kCandK; k++) {
-            const int c = c0 + warp + nw * k;
-            v[k] = c < n_ctas ? __ldcg(reg_q + static_cast<long long>(c) * stride + lane) : 0ull;
-        }
-#pragma unroll
-        for (int k = 0; k < kCandK; k++) {
-            const int c = c0 + warp + nw * k;
-            if (c >= n_ctas) break;
-            const unsigned cnt = min(static_cast<unsigned>(__shfl_sync(0xffffffffu, v[k], 0)),
-                                     static_cast<unsigned>(stride - 1));   // (a region holds stride - 1)
-            const bool take = lane >= 1 && static_cast<unsigned>(lane) <= cnt;
-            const unsigned pos = warp_append(take, &s.n_b);
-            if (take && pos < static_cast<unsigned>(kBoundCap)) s.bnd[pos] = v[k];
-#pragma unroll 1
-            for (unsigned j0 = 32; j0 <= cnt; j0 += 32) {
-                const unsigned j = j0 + lane;
-                const bool t = j <= cnt;
-                const unsigned long long x = t ? __ldcg(reg_q + static_cast<long long>(c) * stride + j) : 0ull;
-                const unsigned q = warp_append(t, &s.n_b);
-                if (t && q < static_cast<unsigned>(kBoundCap)) s.bnd[q] = x;
-            }
-        }
+// The cache row of padded token t of sequence b (the slot map's entry; the token itself without a
+// slot map), -1 where there is none.
+__device__ __forceinline__ int32_t row_of(const IxSelectArgs &sel, int b, long long t) {
+    long long rv = t;
+    if (sel.slot_map) rv = (t >= 0 && t < sel.ld_slot) ? sel.slot_map[static_cast<int64_t>(b) * sel.ld_slot + t] : -1ll;
+    return (rv >= 0 && rv <= 0x7fffffffll) ? static_cast<int32_t>(rv) : GLM_INVALID;
+}
+
+// The outputs of the selected pool p of rank r (r < the selection's count): its top-k entry and
+// its kKpool expanded token / cache-row entries (the rules of expand_selection). Lanes 0 ..
+// kKpool of a warp write them.
+__device__ __forceinline__ void write_ranked(const IxSelectArgs &sel, int n, int b, int pb, unsigned r, int p,
+                                             int lane) {
+    if (lane == kKpool) sel.topk[static_cast<int64_t>(n) * sel.select_k + r] = p;
+    if (lane < kKpool) {
+        const int64_t j = static_cast<int64_t>(n) * sel.out_width + kKpool * static_cast<int64_t>(r) + lane;
+        const int t = pb + kKpool * p + lane;
+        if (sel.tok) sel.tok[j] = t;
+        if (sel.rows) sel.rows[j] = row_of(sel, b, t);
+    }
+}
+
+// The outputs no selected pool owns (one CTA of a query, count >= 1 pools selected): the top-k
+// row's -1 padding, n_sel, and the expanded entries past the selected pools -- the visible tail,
+// then -1 up to out_width.
+__device__ __forceinline__ void write_unranked(const IxSelectArgs &sel, int n, int b, int pb, int seq_len,
+                                               int qp, unsigned count) {
+    for (int x = static_cast<int>(count) + static_cast<int>(threadIdx.x); x < sel.select_k; x += blockDim.x)
+        sel.topk[static_cast<int64_t>(n) * sel.select_k + x] = GLM_INVALID;
+    if (threadIdx.x == 0 && sel.n_sel) sel.n_sel[n] = static_cast<int32_t>(count);
+    if (!sel.tok && !sel.rows) return;
+    const int nvx = visible_pools(pb, seq_len, qp, 0x7fffffffll);   // uncapped, as the expansion defines it
+    const int ns = min(static_cast<int>(count), nvx);
+    const int last = min(qp, pb + seq_len - 1);                     // the tail stops at the query or the end
+    const int tail = max(0, last - (pb + kKpool * nvx) + 1);
+    const int n_valid = kKpool * ns + tail;
+    for (int j = kKpool * ns + static_cast<int>(threadIdx.x); j < sel.out_width; j += blockDim.x) {
+        const int t = j < n_valid ? pb + kKpool * nvx + (j - kKpool * ns) : GLM_INVALID;
+        const int64_t o = static_cast<int64_t>(n) * sel.out_width + j;
+        if (sel.tok) sel.tok[o] = t;
+        if (sel.rows) sel.rows[o] = t >= 0 ? row_of(sel, b, t) : GLM_INVALID;
     }
 }
 
@@ -530,14 +537,22 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     if (multi) {
         if (lo >= hi) return;   // no score range: not part of the query's selection
         if (tid == 0 && flag[kFlWait] && status) atomicOr(status, 8);
-        // this CTA's candidates (scores whose key reaches the sample threshold) to its region of
-        // the query's list: slot 0 the count, then the composites
-        const unsigned thr = flag[kFlThr];
-        const int stride = per + 1;
-        unsigned long long *reg_q = sel.alist + static_cast<int64_t>(n) * sel.list_cap;
-        unsigned long long *reg = reg_q + static_cast<int64_t>(g) * stride;
-        if (tid == 0) s.n_b = 0;
+        const unsigned thr = flag[kFlThr];   // the sample threshold (0: every score is a candidate)
+        // this CTA's candidates (scores whose key reaches the sample threshold) go to the query's
+        // list at an offset taken from its counter: count them, take the offset, write them
+        unsigned long long *cand_q = sel.alist + static_cast<int64_t>(n) * sel.list_cap;   // holds n_vis
+        unsigned mine = 0u;
+#pragma unroll 1
+        for (int b0 = lo; b0 < hi; b0 += kIxThreads) {
+            const int i = b0 + tid;
+            mine += static_cast<unsigned>(__syncthreads_count(i < hi && score_key(score_at(i)) >= thr));
+        }
+        if (tid == 0) {
+            s.n_a = atomicAdd(&cnt[kCntTicket], mine);
+            s.n_b = 0;
+        }
         __syncthreads();
+        const unsigned base = s.n_a;
 #pragma unroll 1
         for (int b0 = lo; b0 < hi; b0 += kIxThreads) {
             const int i = b0 + tid;
@@ -546,43 +561,46 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             if (!__any_sync(0xffffffffu, take)) continue;
             const unsigned pos = warp_append(take, &s.n_b);
             if (take) {
-                reg[1 + pos] = compose(key, i);
+                cand_q[base + pos] = compose(key, i);
                 const long long t0 = pb + static_cast<long long>(kKpool) * i;   // warm L2 for the expansion
                 if (sel.rows && sel.slot_map && t0 >= 0 && t0 + kKpool <= sel.ld_slot)
                     asm volatile("prefetch.global.L2 [%0];" ::"l"(sel.slot_map + static_cast<int64_t>(b) * sel.ld_slot + t0));
             }
         }
         __syncthreads();
-        if (tid == 0) {   // release the region, take the ticket; the last CTA acquires every region
-            reg[0] = s.n_b;
-            s.last = take_ticket(&cnt[kCntTicket], g_eff) ? 1u : 0u;
+        if (tid == 0) {   // release the candidates, wait (acquire) for every CTA's
+            flag[kFlWait] = grid_barrier(&cnt[kCntArrive], g_eff) ? 0u : 1u;
+            if (flag[kFlWait] && status) atomicOr(status, 8);
         }
         __syncthreads();
-        if (!s.last) return;
-        if (tid == 0) s.n_b = 0;
-        __syncthreads();
-        gather_candidates(reg_q, stride, g_eff, s);
-        __syncthreads();
-        const unsigned total = s.n_b;
-        if (total >= count && total <= static_cast<unsigned>(kBoundCap)) {
-            if (total <= static_cast<unsigned>(kMaxSelect)) {   // sort them all, keep the first count
-#pragma unroll 1
-                for (unsigned i = tid; i < total; i += kIxThreads) s.cand[i] = s.bnd[i];
-                __syncthreads();
-                sort_selected(s.cand, static_cast<int>(total), s);
-            } else {
-                auto get = [&](int i) { return s.bnd[i]; };
-                radix_select(get, static_cast<int>(total), count, 0, 0ull, s);
-                collect_from(get, static_cast<int>(total), ~0ull << (64 - s.done), s.prefix, 0u, s);
-                sort_selected(s.cand, static_cast<int>(count), s);
-            }
-        } else {   // the threshold let too few (or too many) through: exact over every score of the row
+        if (flag[kFlWait]) return;   // gave up waiting: the status word reports it
+        const unsigned total = __ldcg(&cnt[kCntTicket]);
+        if (total < count || total > static_cast<unsigned>(kBoundCap)) {
+            // the threshold let too few (or too many) through: CTA 0 selects exactly over every
+            // score of the row and writes the outputs
+            if (g != 0) return;
             auto get = [&](int i) { return compose(score_key(__ldcg(srow + i)), i); };
             radix_select(get, n_vis, count, 0, 0ull, s);
             collect_from(get, n_vis, ~0ull << (64 - s.done), s.prefix, 0u, s);
             sort_selected(s.cand, static_cast<int>(count), s);
+            write_outputs(sel, n, b, valid_b, pb, seq_len, qp, count, s);
+            return;
         }
-        write_outputs(sel, n, b, valid_b, pb, seq_len, qp, count, s);
+        // every CTA: all candidates on chip, then the rank of its share of them -- the number of
+        // larger composites (they are unique) -- and, for the count best, their outputs
+#pragma unroll 1
+        for (unsigned i = tid; i < total; i += kIxThreads) s.bnd[i] = __ldcg(cand_q + i);
+        __syncthreads();
+#pragma unroll 1
+        for (unsigned j = static_cast<unsigned>(g + g_eff * warp); j < total; j += static_cast<unsigned>(g_eff * (kIxThreads / 32))) {
+            const unsigned long long c = s.bnd[j];
+            unsigned gt = 0u;
+#pragma unroll 4
+            for (unsigned i = lane; i < total; i += 32) gt += s.bnd[i] > c ? 1u : 0u;
+            const unsigned r = __reduce_add_sync(0xffffffffu, gt);
+            if (r < count) write_ranked(sel, n, b, pb, r, id_of(c), lane);
+        }
+        if (g == 0) write_unranked(sel, n, b, pb, seq_len, qp, count);
         return;
     }
     // one CTA: lo = 0, hi = n_vis, the histogram and the scores on chip

@@ -64,8 +64,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
     const uint16_t *__restrict__ q, int n_heads, const int8_t *__restrict__ cache, int64_t n_rows,
     const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks,
     float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status, int early_q) {
-    // early_q: the query block is an input no preceding kernel writes (the one-call step), so it is
-    // staged before waiting for the preceding kernel; only the row indices wait for it
+    // early_q: the query block is an input no preceding kernel writes (the one-call step), so its
+    // loads are issued before waiting for the preceding kernel; only the row indices wait for it
     if (early_q) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     else pdl_begin();
     using Lay = TcLayout<M>;
@@ -107,10 +107,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
             *reinterpret_cast<uint4 *>(Qs + hg * 8192 + dg * 128 + (h & 7) * 16) = qv[it];
         }
     };
-    if (early_q) {
-        store_q();
-        asm volatile("griddepcontrol.wait;" ::: "memory");
-    }
+    if (early_q) asm volatile("griddepcontrol.wait;" ::: "memory");   // (the query loads stay in flight)
 
     if (tid == 0) *flag = 0;
     __syncthreads();
@@ -173,7 +170,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
                                                                 codes_to_bf16x2(v[it].w, 0), codes_to_bf16x2(v[it].w, 16));
         }
         if (tid < kTcRows) scl[tid] = sc;
-        if (!early_q) store_q();
+        store_q();
     }
     tc::fence_proxy_async();
     __syncthreads();
