@@ -76,6 +76,14 @@ def _declare(L):
     L.oracle_topk_to_mask.restype = None
     L.oracle_masked_attention.argtypes = [_p, _i32, _p, _i64, _p, _i64, _p, _f64, _p, _p]
     L.oracle_masked_attention.restype = _i32
+    L.oracle_expand_kv.argtypes = [_p, _i64, _i32, _p, _i32, _i32, _i32, _p, _p]
+    L.oracle_expand_kv.restype = None
+    L.oracle_q_absorb.argtypes = [_p, _i32, _i32, _p, _i32, _i32, _p]
+    L.oracle_q_absorb.restype = None
+    L.oracle_v_up.argtypes = [_p, _i32, _i32, _p, _i32, _i32, _p]
+    L.oracle_v_up.restype = None
+    L.oracle_attention_f64.argtypes = [_p, _i32, _i32, _p, _p, _i64, _i32, _i32, _f64, _p]
+    L.oracle_attention_f64.restype = None
 
 
 def _c(a, dtype):
@@ -254,6 +262,59 @@ def masked_attention(q, cache, slot_map_row, mask, sm_scale):
     if rc != 0:
         raise ValueError("index past the end of the cache")
     return out, lse
+
+
+# ------------------------------------------------------------------------------------------------
+# the MLA up-projection ("Module glm5next_dsa_ref", expand_kv; kv_b_proj rows grouped per head,
+# the dk K rows of a head, then its dv V rows; weights as bf16 bits [Hm * (dk + dv), L])
+# ------------------------------------------------------------------------------------------------
+
+def _as_f64(a):
+    a = np.ascontiguousarray(a, dtype=np.float64)
+    return a, a.ctypes.data_as(C.c_void_p)
+
+
+def expand_kv(c, w_kv_b, n_heads, dk, dv):
+    """Per-head K [Hm, T, dk] and V [Hm, T, dv] of latent rows ``c`` float64 [T, L]."""
+    cc, cp = _as_f64(c)
+    w, wp = _c(w_kv_b, np.uint16)
+    T, L = cc.shape
+    k = np.empty((n_heads, T, dk), dtype=np.float64)
+    v = np.empty((n_heads, T, dv), dtype=np.float64)
+    lib().oracle_expand_kv(cp, T, L, wp, n_heads, dk, dv, k.ctypes.data_as(C.c_void_p),
+                           v.ctypes.data_as(C.c_void_p))
+    return k, v
+
+
+def q_absorb(q, w_kv_b, dk, dv, latent=LATENT):
+    """Latent-space queries [Hm, L] of per-head queries ``q`` float64 [Hm, dk]."""
+    qq, qp = _as_f64(q)
+    w, wp = _c(w_kv_b, np.uint16)
+    out = np.empty((qq.shape[0], latent), dtype=np.float64)
+    lib().oracle_q_absorb(qp, qq.shape[0], latent, wp, dk, dv, out.ctypes.data_as(C.c_void_p))
+    return out
+
+
+def v_up(o_lat, w_kv_b, dk, dv):
+    """The up-projection of latent-space outputs ``o_lat`` float64 [Hm, L] to [Hm, dv]."""
+    oo, op = _as_f64(o_lat)
+    w, wp = _c(w_kv_b, np.uint16)
+    out = np.empty((oo.shape[0], dv), dtype=np.float64)
+    lib().oracle_v_up(op, oo.shape[0], oo.shape[1], wp, dk, dv, out.ctypes.data_as(C.c_void_p))
+    return out
+
+
+def attention_f64(q, k, v, scale, shared):
+    """Softmax attention in fp64: ``q`` [Hm, dq]; ``k`` [Hm, T, dq] and ``v`` [Hm, T, dv] per head,
+    or [T, dq] and [T, dv] for every head when ``shared``. Returns [Hm, dv]."""
+    qq, qp = _as_f64(q)
+    kk, kp = _as_f64(k)
+    vv, vp = _as_f64(v)
+    T = kk.shape[-2]
+    out = np.empty((qq.shape[0], vv.shape[-1]), dtype=np.float64)
+    lib().oracle_attention_f64(qp, qq.shape[0], qq.shape[1], kp, vp, T, vv.shape[-1], 1 if shared else 0,
+                               float(scale), out.ctypes.data_as(C.c_void_p))
+    return out
 
 
 # ------------------------------------------------------------------------------------------------

@@ -429,3 +429,93 @@ int oracle_masked_attention(const uint16_t *q, int Hm, const int8_t *cache, int6
     free(c); free(m); free(l);
     return 0;
 }
+
+/* =============================================================================================
+ * The MLA up-projection (the step after the sparse attention; NEXT-3 of the build)
+ * [DSA-REF] "expand_kv: expand the compressed latent into per-head K and V", with kv_b_proj in
+ * the "linear: y = x @ w^T" layout (w is [out, in]); [GLM-5.3-Flash] 'Checkpoint shape':
+ * 64 heads, kv_lora_rank 512, qk_head_dim = v_head_dim = 256, qk_rope_head_dim 0.
+ * READING: the rows of kv_b_proj are grouped per head, the dk K rows of head h first, then its
+ * dv V rows: row h (dk + dv) + e. The weights are bf16 (the checkpoint's kv_b_proj dtype,
+ * [GLM-5.3-Flash] 'Open questions': "kv_b_proj is BF16 in the checkpoint").
+ * The absorbed form that the sparse MLA computes in latent space meets the expanded form through
+ *   q_h . K_h,t = (q_h W_k,h) . c_t        and        sum_t p_t V_h,t = (sum_t p_t c_t) W_v,h^T.
+ * ============================================================================================= */
+
+/* K[h][t][e] = sum_d c[t][d] W[h (dk+dv) + e][d];  V[h][t][e] = sum_d c[t][d] W[h (dk+dv) + dk + e][d].
+ * c is [T][L]; K is [Hm][T][dk], V is [Hm][T][dv]. */
+void oracle_expand_kv(const double *c, int64_t T, int L, const uint16_t *w, int Hm, int dk, int dv,
+                      double *k_out, double *v_out)
+{
+    for (int h = 0; h < Hm; h++) {
+        const uint16_t *wh = w + (size_t)h * (dk + dv) * L;
+        for (int64_t t = 0; t < T; t++) {
+            for (int e = 0; e < dk + dv; e++) {
+                double s = 0.0;
+                for (int d = 0; d < L; d++) s += c[(size_t)t * L + d] * bf16(wh[(size_t)e * L + d]);
+                if (e < dk) k_out[((size_t)h * T + t) * dk + e] = s;
+                else v_out[((size_t)h * T + t) * dv + (e - dk)] = s;
+            }
+        }
+    }
+}
+
+/* The latent-space query of the absorbed form: q_lat[h][d] = sum_e q[h][e] W[h (dk+dv) + e][d]
+ * for the dk K rows of head h (q is [Hm][dk], q_lat is [Hm][L]). */
+void oracle_q_absorb(const double *q, int Hm, int L, const uint16_t *w, int dk, int dv, double *q_lat)
+{
+    for (int h = 0; h < Hm; h++) {
+        const uint16_t *wh = w + (size_t)h * (dk + dv) * L;
+        for (int d = 0; d < L; d++) {
+            double s = 0.0;
+            for (int e = 0; e < dk; e++) s += q[(size_t)h * dk + e] * bf16(wh[(size_t)e * L + d]);
+            q_lat[(size_t)h * L + d] = s;
+        }
+    }
+}
+
+/* The up-projection epilogue of the absorbed form: out[h][e] = sum_d o_lat[h][d] W[h (dk+dv) + dk + e][d]
+ * for the dv V rows of head h (o_lat is [Hm][L], out is [Hm][dv]). */
+void oracle_v_up(const double *o_lat, int Hm, int L, const uint16_t *w, int dk, int dv, double *out)
+{
+    for (int h = 0; h < Hm; h++) {
+        const uint16_t *wv = w + ((size_t)h * (dk + dv) + dk) * L;
+        for (int e = 0; e < dv; e++) {
+            double s = 0.0;
+            for (int d = 0; d < L; d++) s += o_lat[(size_t)h * L + d] * bf16(wv[(size_t)e * L + d]);
+            out[(size_t)h * dv + e] = s;
+        }
+    }
+}
+
+/* Softmax attention of Hm queries over T keys in fp64 (the definition, max-subtracted):
+ *   out[h] = sum_t softmax_t(scale * q[h] . K[t]) V[t],
+ * with K, V per head ([Hm][T][dq] and [Hm][T][dvv]) when shared == 0, or one set for every head
+ * ([T][dq], [T][dvv]) when shared != 0 (the latent form: K = V = the latent rows). */
+void oracle_attention_f64(const double *q, int Hm, int dq, const double *k, const double *v, int64_t T,
+                          int dvv, int shared, double scale, double *out)
+{
+    double *s = malloc(sizeof(double) * (size_t)(T > 0 ? T : 1));
+    for (int h = 0; h < Hm; h++) {
+        const double *kh = shared ? k : k + (size_t)h * T * dq;
+        const double *vh = shared ? v : v + (size_t)h * T * dvv;
+        double *o = out + (size_t)h * dvv;
+        for (int e = 0; e < dvv; e++) o[e] = 0.0;
+        if (T == 0) continue;
+        double m = -INFINITY;
+        for (int64_t t = 0; t < T; t++) {
+            double dot = 0.0;
+            for (int d = 0; d < dq; d++) dot += q[(size_t)h * dq + d] * kh[(size_t)t * dq + d];
+            s[t] = scale * dot;
+            if (s[t] > m) m = s[t];
+        }
+        double l = 0.0;
+        for (int64_t t = 0; t < T; t++) {
+            const double p = exp(s[t] - m);
+            l += p;
+            for (int e = 0; e < dvv; e++) o[e] += p * vh[(size_t)t * dvv + e];
+        }
+        for (int e = 0; e < dvv; e++) o[e] /= l;
+    }
+    free(s);
+}
