@@ -84,6 +84,14 @@ def _declare(L):
     L.oracle_v_up.restype = None
     L.oracle_attention_f64.argtypes = [_p, _i32, _i32, _p, _p, _i64, _i32, _i32, _f64, _p]
     L.oracle_attention_f64.restype = None
+    L.oracle_e4m3_value.argtypes = [C.c_uint]
+    L.oracle_e4m3_value.restype = _f64
+    L.oracle_e4m3_encode.argtypes = [_f64]
+    L.oracle_e4m3_encode.restype = C.c_uint
+    L.oracle_store_fp8.argtypes = [_p, _p, _i64, _p, _i64]
+    L.oracle_store_fp8.restype = _i32
+    L.oracle_dequant_row_fp8.argtypes = [_p, _i64, _p]
+    L.oracle_dequant_row_fp8.restype = None
 
 
 def _c(a, dtype):
@@ -314,6 +322,37 @@ def attention_f64(q, k, v, scale, shared):
     out = np.empty((qq.shape[0], vv.shape[-1]), dtype=np.float64)
     lib().oracle_attention_f64(qp, qq.shape[0], qq.shape[1], kp, vp, T, vv.shape[-1], 1 if shared else 0,
                                float(scale), out.ctypes.data_as(C.c_void_p))
+    return out
+
+
+# ------------------------------------------------------------------------------------------------
+# the FP8 latent cache row (E4M3 codes, one fp32 scale per row, the INT8 row's 528-byte layout)
+# ------------------------------------------------------------------------------------------------
+
+def e4m3_value(code) -> float:
+    return lib().oracle_e4m3_value(int(code) & 0xFF)
+
+
+def e4m3_encode(x) -> int:
+    return int(lib().oracle_e4m3_encode(float(x)))
+
+
+def store_fp8(latent, slots, cache) -> None:
+    """Quantise ``latent`` (uint16 bf16 bits [n, 512]) into ``cache`` (uint8 [n_rows, 528]) in place."""
+    assert cache.dtype == np.uint8 and cache.flags.c_contiguous and cache.shape[-1] == ROW_BYTES
+    lat, lp = _c(latent, np.uint16)
+    sl, sp = _c(slots, np.int64)
+    assert lat.shape == (sl.shape[0], LATENT)
+    rc = lib().oracle_store_fp8(lp, sp, sl.shape[0], cache.ctypes.data_as(C.c_void_p), cache.shape[0])
+    if rc != 0:
+        raise ValueError("slot past the end of the cache")
+
+
+def dequant_rows_fp8(cache, rows) -> np.ndarray:
+    cache = np.ascontiguousarray(cache, dtype=np.uint8).reshape(-1, ROW_BYTES)
+    out = np.empty((len(rows), LATENT), dtype=np.float64)
+    for i, r in enumerate(rows):
+        lib().oracle_dequant_row_fp8(cache.ctypes.data_as(C.c_void_p), int(r), out[i].ctypes.data_as(C.c_void_p))
     return out
 
 

@@ -519,3 +519,81 @@ void oracle_attention_f64(const double *q, int Hm, int dq, const double *k, cons
     }
     free(s);
 }
+
+/* =============================================================================================
+ * The FP8 latent cache row (NEXT-4 of the build). [GLM on CUDA] names an opt-in "FP8 or 4-bit
+ * latent cache (--kv-dtype fp8 / fp4), lossy" and gives no format.
+ * READINGS: FP8 is E4M3 in its OCP "E4M3FN" form (exponent bias 7, subnormals, no infinities,
+ * S.1111.111 is NaN, largest finite value 448); the row is the INT8 row's layout and recipe with
+ * 448 in place of 127: scale = fl32(max(amax, floor) / 448), code = the E4M3 value nearest
+ * fl32(x / scale) with ties to the even code (even mantissa), saturating at +-448, the sign kept
+ * (-0 gives 0x80); bytes: 512 codes, the fp32 scale (little endian), 12 zero bytes. The
+ * dequantised value is value(code) * scale.
+ * ============================================================================================= */
+#define ORACLE_E4M3_MAX 448.0
+
+/* The value of an E4M3 code: (1 + m/8) 2^(e-7) for exponent field e >= 1, (m/8) 2^-6 for e = 0. */
+double oracle_e4m3_value(unsigned code)
+{
+    const int s = (int)((code >> 7) & 1u), e = (int)((code >> 3) & 15u), m = (int)(code & 7u);
+    if (e == 15 && m == 7) return NAN;
+    const double v = e == 0 ? ldexp((double)m, -9) : ldexp(8.0 + m, e - 10);
+    return s ? -v : v;
+}
+
+/* The E4M3 code nearest x (ties to the even code), saturating at +-448. */
+unsigned oracle_e4m3_encode(double x)
+{
+    if (x != x) return 0x7Fu;
+    const unsigned s = signbit(x) ? 0x80u : 0u;
+    const double a = fabs(x);
+    if (a >= ORACLE_E4M3_MAX) return s | 0x7Eu;
+    unsigned code;
+    if (a < ldexp(1.0, -6)) {                     /* subnormal range: steps of 2^-9; 8 is 2^-6 */
+        code = (unsigned)nearbyint(ldexp(a, 9));
+    } else {
+        int e;
+        frexp(a, &e);                             /* a in [2^(e-1), 2^e)                      */
+        const int E = e - 1;
+        unsigned m = (unsigned)nearbyint(ldexp(a, 3 - E));   /* in [8, 16]                    */
+        int field = E + 7;
+        if (m == 16u) { m = 8u; field++; }
+        code = ((unsigned)field << 3) | (m - 8u);
+        if (code > 0x7Eu) code = 0x7Eu;
+    }
+    return s | code;
+}
+
+/* store of FP8 rows: the store_int8 contract with E4M3 codes. Returns 0, or -1 if a slot is past
+ * the cache. */
+int oracle_store_fp8(const uint16_t *latent, const int64_t *slots, int64_t n, uint8_t *cache, int64_t n_rows)
+{
+    for (int64_t i = 0; i < n; i++) {
+        const int64_t slot = slots[i];
+        if (slot < 0) continue;
+        if (slot >= n_rows) return -1;
+        const uint16_t *x = latent + i * ORACLE_LATENT;
+        double amax = 0.0;
+        for (int j = 0; j < ORACLE_LATENT; j++) {
+            const double a = fabs(bf16(x[j]));
+            if (a > amax) amax = a;
+        }
+        if (amax < amax_floor()) amax = amax_floor();
+        const float scale = (float)(amax / ORACLE_E4M3_MAX);
+        unsigned char *row = cache + slot * ORACLE_ROW_BYTES;
+        for (int j = 0; j < ORACLE_LATENT; j++)
+            row[j] = (unsigned char)oracle_e4m3_encode((double)(float)(bf16(x[j]) / (double)scale));
+        memcpy(row + ORACLE_LATENT, &scale, 4);
+        memset(row + ORACLE_LATENT + 4, 0, ORACLE_ROW_BYTES - ORACLE_LATENT - 4);
+    }
+    return 0;
+}
+
+/* Dequantise one FP8 cache row into fp64 (value(code) * scale). */
+void oracle_dequant_row_fp8(const uint8_t *cache, int64_t row, double *out)
+{
+    const unsigned char *r = cache + row * ORACLE_ROW_BYTES;
+    float scale;
+    memcpy(&scale, r + ORACLE_LATENT, 4);
+    for (int j = 0; j < ORACLE_LATENT; j++) out[j] = oracle_e4m3_value(r[j]) * (double)scale;
+}
