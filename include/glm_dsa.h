@@ -94,6 +94,16 @@ int glm_last_cuda_error(void);
 int glm_kv_store_int8(const glm_dsa_dims *dims, const void *latent_dev, const int64_t *slots_dev,
                       int64_t n, int8_t *cache_dev, int64_t n_rows, void *stream);
 
+/*
+ * The FP8 latent cache ("GLM on CUDA": an opt-in FP8 latent cache, --kv-dtype fp8, lossy; the
+ * page gives no format). The row of glm_kv_store_int8 with E4M3 codes (OCP E4M3FN: exponent bias
+ * 7, subnormals, largest finite 448) in bytes [0,512): scale = max(amax, 1e-4f) / 448 (fp32), code =
+ * the E4M3 value nearest the IEEE fp32 quotient x / scale, ties to the even code, saturating at
+ * +-448, the sign kept. Arguments, slots and padding as glm_kv_store_int8; cache_dev uint8 [n_rows, 528].
+ */
+int glm_kv_store_fp8(const glm_dsa_dims *dims, const void *latent_dev, const int64_t *slots_dev,
+                     int64_t n, uint8_t *cache_dev, int64_t n_rows, void *stream);
+
 /* ------------------------------------------------------------------------------------------ */
 /* kpool_build                                                                                 */
 /* ------------------------------------------------------------------------------------------ */
@@ -276,6 +286,16 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q_dev, const int
                           int64_t n_rows, const int32_t *rows_dev, int32_t n_q, int32_t width,
                           float sm_scale, void *out_dev, float *lse_dev, float *out_f32_dev,
                           void *workspace_dev, size_t ws_bytes, void *stream);
+
+/*
+ * glm_sparse_mla_decode over FP8 rows (glm_kv_store_fp8): each entry's key and value is
+ * value(code) * scale, the E4M3 codes widened to bf16 exactly; everything else as
+ * glm_sparse_mla_decode (cache_dev uint8 [n_rows, 528], same workspace).
+ */
+int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q_dev, const uint8_t *cache_dev,
+                              int64_t n_rows, const int32_t *rows_dev, int32_t n_q, int32_t width,
+                              float sm_scale, void *out_dev, float *lse_dev, float *out_f32_dev,
+                              void *workspace_dev, size_t ws_bytes, void *stream);
 
 /*
  * The same sparse NoPE MLA decode without a workspace argument. The pages have no counterpart:

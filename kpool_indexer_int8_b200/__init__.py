@@ -38,7 +38,7 @@ EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv
            "glm_index_topk_expand", "glm_index_topk_expand_q8",
            "glm_dsa_decode_step",
            "glm_topk_pools", "glm_expand_selection",
-           "glm_sparse_mla_decode", "glm_dsa_workspace_size")
+           "glm_sparse_mla_decode", "glm_dsa_workspace_size", "glm_kv_store_fp8", "glm_sparse_mla_decode_fp8")
 
 
 class glm_dsa_dims(C.Structure):
@@ -109,6 +109,10 @@ lib.glm_expand_selection.argtypes = [_D, _P, _P, _P, _P, _P, _P, _I32, _I32, _I3
                                      _P, _P]
 lib.glm_expand_selection.restype = C.c_int
 lib.glm_sparse_mla_decode.argtypes = [_D, _P, _P, _I64, _P, _I32, _I32, _F32, _P, _P, _P, _P, _SZ, _P]
+lib.glm_sparse_mla_decode_fp8.argtypes = [_D, _P, _P, _I64, _P, _I32, _I32, _F32, _P, _P, _P, _P, _SZ, _P]
+lib.glm_sparse_mla_decode_fp8.restype = C.c_int
+lib.glm_kv_store_fp8.argtypes = [_D, _P, _P, _I64, _P, _I64, _P]
+lib.glm_kv_store_fp8.restype = C.c_int
 lib.glm_sparse_mla_decode.restype = C.c_int
 lib.glm_dsa_workspace_size.argtypes = [_D, _I32, _I32, _I64, _I32, _I32]
 lib.glm_dsa_workspace_size.restype = C.c_size_t
@@ -169,6 +173,16 @@ def glm_kv_store_int8(dims, latent, slots, cache, stream=None) -> None:
     n_rows = cache.numel() // GLM_ROW_BYTES
     _check(lib.glm_kv_store_int8(C.byref(dims), _ptr(latent), _ptr(slots), latent.shape[0],
                                  _ptr(cache), n_rows, _stream(stream)), "glm_kv_store_int8")
+
+
+def glm_kv_store_fp8(dims, latent, slots, cache, stream=None) -> None:
+    """The FP8 latent row: latent bf16 [n, 512], slots int64 [n], cache uint8 [n_rows, 528]."""
+    _dev(latent, torch.bfloat16, "latent", 2)
+    _dev(slots, torch.int64, "slots", 1)
+    _dev(cache, torch.uint8, "cache")
+    n_rows = cache.numel() // GLM_ROW_BYTES
+    _check(lib.glm_kv_store_fp8(C.byref(dims), _ptr(latent), _ptr(slots), latent.shape[0],
+                                _ptr(cache), n_rows, _stream(stream)), "glm_kv_store_fp8")
 
 
 def glm_kpool_build(dims, k, gate, ln_w, ln_b, ln_eps, pad, length, pooled, pool_begin=None,
@@ -371,6 +385,21 @@ def glm_sparse_mla_decode(dims, q, cache, rows, sm_scale, out, workspace, lse=No
                                      rows.shape[0], rows.shape[1], float(sm_scale), _ptr(out),
                                      _ptr(lse), _ptr(out_f32), _ptr(workspace), workspace.numel(),
                                      _stream(stream)), "glm_sparse_mla_decode")
+
+
+def glm_sparse_mla_decode_fp8(dims, q, cache, rows, sm_scale, out, workspace, lse=None, out_f32=None,
+                              stream=None) -> None:
+    """glm_sparse_mla_decode over FP8 rows: cache uint8 [n_rows, 528] (glm_kv_store_fp8)."""
+    for t, dt, nm in ((q, torch.bfloat16, "q"), (cache, torch.uint8, "cache"),
+                      (rows, torch.int32, "rows"), (out, torch.bfloat16, "out"),
+                      (workspace, torch.uint8, "workspace"), (lse, torch.float32, "lse"),
+                      (out_f32, torch.float32, "out_f32")):
+        _dev(t, dt, nm)
+    n_rows = cache.numel() // GLM_ROW_BYTES
+    _check(lib.glm_sparse_mla_decode_fp8(C.byref(dims), _ptr(q), _ptr(cache), n_rows, _ptr(rows),
+                                         rows.shape[0], rows.shape[1], float(sm_scale), _ptr(out),
+                                         _ptr(lse), _ptr(out_f32), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)), "glm_sparse_mla_decode_fp8")
 
 
 # ------------------------------------------------------------------------------------------------

@@ -180,6 +180,14 @@ int glm_kv_store_int8(const glm_dsa_dims *dims, const void *latent, const int64_
                                               static_cast<cudaStream_t>(stream), num_sms()));
 }
 
+int glm_kv_store_fp8(const glm_dsa_dims *dims, const void *latent, const int64_t *slots,
+                     int64_t n, uint8_t *cache, int64_t n_rows, void *stream) {
+    const int rc = check_store(dims, latent, slots, n, reinterpret_cast<int8_t *>(cache), n_rows);
+    if (rc != GLM_OK || n == 0) return rc;
+    return cuda_status(glm::launch_store_fp8(latent, slots, n, cache, n_rows,
+                                             static_cast<cudaStream_t>(stream), num_sms()));
+}
+
 int glm_kpool_build(const glm_dsa_dims *dims, const void *k, const void *gate, int64_t ld_tokens,
                     const float *ln_w, const float *ln_b, float ln_eps, const int32_t *pad,
                     const int32_t *len, const int32_t *pool_begin, int32_t batch,
@@ -467,6 +475,30 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = cuda_status(glm::launch_mla_split_tc(q, H, cache, n_rows, rows, n_q, width, sm_scale,
                                               part_acc, part_ml, status, st));
+    if (rc != GLM_OK) return rc;
+    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32, lse, st));
+}
+
+int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q, const uint8_t *cache,
+                              int64_t n_rows, const int32_t *rows, int32_t n_q, int32_t width,
+                              float sm_scale, void *out, float *lse, float *out_f32, void *workspace,
+                              size_t ws_bytes, void *stream) {
+    const int8_t *c8 = reinterpret_cast<const int8_t *>(cache);
+    int rc = check_mla(dims, q, c8, n_rows, rows, n_q, width, sm_scale, out, lse, out_f32);
+    if (rc != GLM_OK || n_q == 0) return rc;
+    const int H = dims->n_heads;
+    const size_t need = glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width);
+    if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
+    const int chunk = glm::mla_tc_chunk();
+    const int n_chunks = (width + chunk - 1) / chunk;
+    const size_t parts = mla_parts(n_q, H, width);
+    char *ws = static_cast<char *>(workspace);
+    float *part_acc = reinterpret_cast<float *>(ws);
+    float *part_ml = reinterpret_cast<float *>(ws + mla_acc_bytes(parts));
+    int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = cuda_status(glm::launch_mla_split_tc(q, H, c8, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml,
+                                              status, st, false, true));
     if (rc != GLM_OK) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32, lse, st));
 }

@@ -45,6 +45,48 @@ __device__ __forceinline__ void store_int8_row(const uint16_t *__restrict__ late
     if (lane == 0) dst[32] = make_uint4(__float_as_uint(scale), 0u, 0u, 0u);
 }
 
+// The E4M3 code of x (nearest value, ties to the even code, saturating at +-448; the hardware
+// conversion, given x twice so that the code's byte position is not in question).
+__device__ __forceinline__ uint32_t e4m3_code(float x) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(x), "f"(x));
+    return static_cast<uint32_t>(d) & 0xffu;
+}
+
+// The FP8 twin of store_int8_row (the FP8 latent cache of "GLM on CUDA", --kv-dtype fp8): the same
+// 528-byte row with E4M3 codes and scale = max(amax, 1e-4) / 448. One warp; every lane calls.
+__device__ __forceinline__ void store_fp8_row(const uint16_t *__restrict__ latent, const int64_t *__restrict__ slots,
+                                              int64_t row, uint8_t *__restrict__ cache, int64_t n_rows) {
+    const int lane = threadIdx.x & 31;
+    const int64_t slot = slots[row];
+    if (slot < 0 || slot >= n_rows) return;  // padding (or outside the contract): no write
+    const uint4 *src = reinterpret_cast<const uint4 *>(latent + row * kLatent) + lane * 2;
+    uint4 v0 = __ldcs(src), v1 = __ldcs(src + 1);
+    uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float x[16];
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        amax = fmaxf(amax, fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1])));
+    }
+    amax = warp_max(amax);
+    amax = fmaxf(amax, 1e-4f);
+    const float scale = __fdiv_rn(amax, 448.0f);
+    uint32_t packed[4];
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        uint32_t p = 0;
+#pragma unroll
+        for (int j = 0; j < 4; j++) p |= e4m3_code(__fdiv_rn(x[4 * i + j], scale)) << (8 * j);
+        packed[i] = p;
+    }
+    uint4 *dst = reinterpret_cast<uint4 *>(cache + slot * kRowBytes);
+    dst[lane] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    if (lane == 0) dst[32] = make_uint4(__float_as_uint(scale), 0u, 0u, 0u);
+}
+
 // Item `it` = (sequence b, i-th new pool) of a build (one warp; every lane calls). lw / lb: this
 // lane's four LayerNorm weights and biases.
 __device__ __forceinline__ void kpool_build_item(const uint16_t *__restrict__ k, const uint16_t *__restrict__ gate,

@@ -11,6 +11,8 @@ namespace glm {
 
 cudaError_t launch_store_int8(const void *latent, const int64_t *slots, int64_t n, int8_t *cache,
                               int64_t n_rows, cudaStream_t stream, int num_sms);
+cudaError_t launch_store_fp8(const void *latent, const int64_t *slots, int64_t n, uint8_t *cache,
+                             int64_t n_rows, cudaStream_t stream, int num_sms);
 cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_tokens,
                                const float *ln_w, const float *ln_b, float eps,
                                const int32_t *pad, const int32_t *len, const int32_t *pool_begin,

@@ -14,7 +14,8 @@ int mla_tc_chunk();
 cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
                                 const int32_t *rows, int n_q, int width, float sm_scale,
                                 float *part_acc, float *part_ml, int *status, cudaStream_t stream,
-                                bool early_q = false);   // early_q: stage q before waiting on the previous kernel
+                                bool early_q = false,    // early_q: stage q before waiting on the previous kernel
+                                bool fp8 = false);       // fp8: the rows hold E4M3 codes (the FP8 latent cache)
 cudaError_t launch_mla_combine(const float *part_acc, const float *part_ml, int n_q, int n_heads,
                                int n_chunks, void *out, float *out_f32, float *lse,
                                cudaStream_t stream);

@@ -5,8 +5,8 @@
 //
 // One CTA per (query, chunk of 64 index entries); heads are the MMA M dimension (M = 64 for up
 // to 64 heads, 128 above; missing heads are zero rows):
-//   1. gather: each entry's 512 int8 codes are widened to bf16 (exact: |code| <= 127) into a
-//      shared tile C[64 rows x 512] stored as 8x8 core matrices, its fp32 scale to a register
+//   1. gather: each entry's 512 int8 codes are widened to bf16 (exact: |code| <= 127; the E4M3
+//      codes of the FP8 row are exact in bf16 as well) into a shared tile C[64 rows x 512] stored as 8x8 core matrices, its fp32 scale to a register
 //      file in shared memory; the query block Q[heads x 512] goes to shared memory the same way.
 //   2. S = Q . C^T on tcgen05 (kind::f16, fp32 accumulator in tensor memory, 32 MMAs of K = 16).
 //      C is the K-major B operand here.
@@ -57,9 +57,22 @@ __device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w, int shift) {
     return (__float_as_uint(a) >> 16) | (__float_as_uint(b) & 0xffff0000u);
 }
 
+// One E4M3 code (OCP E4M3FN: bias 7, subnormals) as bf16 bits -- exact: 3 mantissa bits and
+// exponents 2^-9 .. 2^8 fit bf16. (Codes 0x7F / 0xFF, NaN, are never written by the store.)
+__device__ __forceinline__ uint32_t e4m3_bf16_bits(uint32_t b) {
+    const uint32_t s = (b & 0x80u) << 8, e = (b >> 3) & 15u, m = b & 7u;
+    if (e != 0u) return s | ((e + 120u) << 7) | (m << 4);   // 2^(e-7) (1 + m/8)
+    if (m == 0u) return s;
+    const uint32_t p = 31u - __clz(m);                          // m 2^-9 = 2^(p-9) (1 + frac)
+    return s | ((p + 118u) << 7) | (((m << (3u - p)) & 7u) << 4);
+}
+__device__ __forceinline__ uint32_t fp8_to_bf16x2(uint32_t w, int shift) {
+    return e4m3_bf16_bits((w >> shift) & 0xffu) | (e4m3_bf16_bits((w >> (shift + 8)) & 0xffu) << 16);
+}
+
 __device__ __forceinline__ uint16_t bf16_rn_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
 
-template <int M>
+template <int M, bool kFp8>
 __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
     const uint16_t *__restrict__ q, int n_heads, const int8_t *__restrict__ cache, int64_t n_rows,
     const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks,
@@ -164,10 +177,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
             const int j = (g & 7) * 8 + (t & 7);
             const int k = (g >> 3) * 4 + (t >> 3);
             unsigned char *line = Cs + (j >> 3) * 8192 + (2 * k) * 128 + (j & 7) * 16;
-            *reinterpret_cast<uint4 *>(line) = make_uint4(codes_to_bf16x2(v[it].x, 0), codes_to_bf16x2(v[it].x, 16),
-                                                          codes_to_bf16x2(v[it].y, 0), codes_to_bf16x2(v[it].y, 16));
-            *reinterpret_cast<uint4 *>(line + 128) = make_uint4(codes_to_bf16x2(v[it].z, 0), codes_to_bf16x2(v[it].z, 16),
-                                                                codes_to_bf16x2(v[it].w, 0), codes_to_bf16x2(v[it].w, 16));
+            auto cv = [&](uint32_t w, int shift) { return kFp8 ? fp8_to_bf16x2(w, shift) : codes_to_bf16x2(w, shift); };
+            *reinterpret_cast<uint4 *>(line) = make_uint4(cv(v[it].x, 0), cv(v[it].x, 16), cv(v[it].y, 0), cv(v[it].y, 16));
+            *reinterpret_cast<uint4 *>(line + 128) = make_uint4(cv(v[it].z, 0), cv(v[it].z, 16), cv(v[it].w, 0), cv(v[it].w, 16));
         }
         if (tid < kTcRows) scl[tid] = sc;
         store_q();
@@ -306,28 +318,33 @@ __global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
 
 int mla_tc_chunk() { return kTcRows; }
 
+template <int M, bool kFp8>
+cudaError_t launch_mla_split_tc_t(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
+                                  const int32_t *rows, int n_q, int width, float sm_scale,
+                                  float *part_acc, float *part_ml, int *status, cudaStream_t stream, bool early_q) {
+    const int n_chunks = (width + kTcRows - 1) / kTcRows;
+    const int smem = TcLayout<M>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(mla_split_tc_kernel<M, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(mla_split_tc_kernel<M, kFp8>, dim3(n_chunks, n_q), dim3(kTcThreads), smem, stream,
+                   static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
+                   part_acc, part_ml, status, early_q ? 1 : 0);
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
 cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
                                 const int32_t *rows, int n_q, int width, float sm_scale,
-                                float *part_acc, float *part_ml, int *status, cudaStream_t stream, bool early_q) {
-    const int n_chunks = (width + kTcRows - 1) / kTcRows;
-    dim3 grid(n_chunks, n_q);
-    cudaError_t e;
-    if (n_heads <= 64) {
-        const int smem = TcLayout<64>::kBytes;
-        e = cudaFuncSetAttribute(mla_split_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        e = launch_pdl(mla_split_tc_kernel<64>, dim3(grid), dim3(kTcThreads), smem, stream,
-                       static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
-                       part_acc, part_ml, status, early_q ? 1 : 0);
-    } else {
-        const int smem = TcLayout<128>::kBytes;
-        e = cudaFuncSetAttribute(mla_split_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-        if (e != cudaSuccess) return e;
-        e = launch_pdl(mla_split_tc_kernel<128>, dim3(grid), dim3(kTcThreads), smem, stream,
-                       static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
-                       part_acc, part_ml, status, early_q ? 1 : 0);
-    }
-    return e != cudaSuccess ? e : cudaGetLastError();
+                                float *part_acc, float *part_ml, int *status, cudaStream_t stream, bool early_q,
+                                bool fp8) {
+    if (n_heads <= 64)
+        return fp8 ? launch_mla_split_tc_t<64, true>(q, n_heads, cache, n_rows, rows, n_q, width, sm_scale, part_acc,
+                                                     part_ml, status, stream, early_q)
+                   : launch_mla_split_tc_t<64, false>(q, n_heads, cache, n_rows, rows, n_q, width, sm_scale, part_acc,
+                                                      part_ml, status, stream, early_q);
+    return fp8 ? launch_mla_split_tc_t<128, true>(q, n_heads, cache, n_rows, rows, n_q, width, sm_scale, part_acc,
+                                                  part_ml, status, stream, early_q)
+               : launch_mla_split_tc_t<128, false>(q, n_heads, cache, n_rows, rows, n_q, width, sm_scale, part_acc,
+                                                   part_ml, status, stream, early_q);
 }
 
 }  // namespace glm
