@@ -267,6 +267,7 @@ def config_of(wl, args):
             "out_width": wl.out_width, "kpool": 4, "index_heads": 32, "index_dim": 128,
             "latent": 512, "states": args.states,
             "pooled_keys": "int8 codes + fp32 scale per pool" if args.pooled == "int8" else "fp32",
+            "latent_cache": "fp8 (e4m3) rows" if args.cache == "fp8" else "int8 rows",
             "l2": f"rotates {args.states} independent states per rank (inputs >> 126 MB L2)",
             "launch": f"one cuda graph of {args.states} steps (one per state) per replay", "parallelism": f"replicas x{args.gpus}"}
 
@@ -298,7 +299,7 @@ def run_kernels(args, wl):
     inps, bufs = [], []
     for r, sid in enumerate(replica_state_ids(rank, R)):
         inp = synth.generate(wl, state=sid)
-        b = sdev.allocate_for(inp, dev, q8=args.pooled == "int8")
+        b = sdev.allocate_for(inp, dev, q8=args.pooled == "int8", fp8=args.cache == "fp8")
         sdev.load(inp, b)
         bufs.append(b)
         inps.append(inp if r == 0 else None)
@@ -470,7 +471,7 @@ def run_kernels(args, wl):
         "clocks": sampler.summary(),
     }
     line["achieved_hbm_frac_per_gpu"] = line["achieved_hbm_gbs_per_gpu"] / peak
-    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+    if world == 1 and rank == 0 and not args.no_cpu_baseline and args.cache == "int8":
         qps, done, el = oracle_decode_throughput(wl, budget_s=12.0)
         line["cpu_baseline"] = {"value": qps, "unit": "queries/s", "cores": 1, "kind": "oracle",
                                 "sample": f"{done} decode queries of {wl.name} state 0 ({el:.1f} s); oracle state built untimed"}
@@ -493,6 +494,8 @@ def main(argv=None):
     ap.add_argument("--states", type=int, default=8)
     ap.add_argument("--pooled", choices=["fp32", "int8"], default="fp32",
                     help="indexer state: fp32 pooled keys (the pages' path) or the INT8 variant")
+    ap.add_argument("--cache", choices=["int8", "fp8"], default="int8",
+                    help="latent cache rows: INT8 (the pages' path) or the FP8 variant")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     if args.warmup < 3:

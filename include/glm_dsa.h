@@ -376,6 +376,9 @@ typedef struct glm_dsa_step {
     /* the INT8 indexer state instead of pooled_dev (glm_kpool_build_q8), or NULL */
     int8_t *pooled_codes_dev;      /* int8 [batch, ld_pools, 128]        */
     float *pooled_scales_dev;      /* fp32 [batch, ld_pools]             */
+    /* nonzero: cache_dev holds FP8 rows (uint8 [n_rows, 528]); the store and the attention are
+     * glm_kv_store_fp8 and glm_sparse_mla_decode_fp8 */
+    int32_t cache_fp8;
 } glm_dsa_step;
 
 /*

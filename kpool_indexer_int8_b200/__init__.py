@@ -66,7 +66,7 @@ class glm_dsa_step(C.Structure):
                 ("tok_dev", C.c_void_p), ("rows_dev", C.c_void_p),
                 ("q_dev", C.c_void_p), ("sm_scale", C.c_float), ("out_dev", C.c_void_p),
                 ("lse_dev", C.c_void_p), ("out_f32_dev", C.c_void_p),
-                ("pooled_codes_dev", C.c_void_p), ("pooled_scales_dev", C.c_void_p)]
+                ("pooled_codes_dev", C.c_void_p), ("pooled_scales_dev", C.c_void_p), ("cache_fp8", C.c_int32)]
 
 
 def make_dims(n_heads: int, kv_lora_rank: int = 512, qk_rope_head_dim: int = 0,
@@ -294,10 +294,13 @@ def glm_index_topk_expand(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, sel
 def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_eps, pad, length, pool_begin,
                         max_new_pools, pooled, q_idx, w, q_seq, q_pos, select_k, out_width, slot_map, rows,
                         topk, q, sm_scale, out, workspace, n_sel=None, tok=None, scores=None, lse=None,
-                        out_f32=None, pooled_codes=None, pooled_scales=None, stream=None) -> None:
+                        out_f32=None, pooled_codes=None, pooled_scales=None, cache_fp8=False, stream=None) -> None:
     """The whole step in one call: the arguments of glm_kv_store_int8, glm_kpool_build,
-    glm_index_topk_expand and glm_sparse_mla_decode (same tensors and rules)."""
-    for t, dt, nm in ((latent, torch.bfloat16, "latent"), (slots, torch.int64, "slots"), (cache, torch.int8, "cache"),
+    glm_index_topk_expand and glm_sparse_mla_decode (same tensors and rules); with cache_fp8 the
+    cache holds FP8 rows (uint8) and the step stores and attends as glm_kv_store_fp8 and
+    glm_sparse_mla_decode_fp8."""
+    for t, dt, nm in ((latent, torch.bfloat16, "latent"), (slots, torch.int64, "slots"),
+                      (cache, torch.uint8 if cache_fp8 else torch.int8, "cache"),
                       (k, torch.bfloat16, "k"), (gate, torch.bfloat16, "gate"), (ln_w, torch.float32, "ln_w"),
                       (ln_b, torch.float32, "ln_b"), (pad, torch.int32, "pad"), (length, torch.int32, "len"),
                       (pool_begin, torch.int32, "pool_begin"), (pooled, torch.float32, "pooled"),
@@ -325,6 +328,7 @@ def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_e
     a.q_dev, a.sm_scale, a.out_dev = v(q), float(sm_scale), v(out)
     a.lse_dev, a.out_f32_dev = v(lse), v(out_f32)
     a.pooled_codes_dev, a.pooled_scales_dev = v(pooled_codes), v(pooled_scales)
+    a.cache_fp8 = 1 if cache_fp8 else 0
     ws_bytes = 0 if workspace is None else workspace.numel()
     _check(lib.glm_dsa_decode_step(C.byref(dims), C.byref(a), _ptr(workspace), ws_bytes, _stream(stream)),
            "glm_dsa_decode_step")

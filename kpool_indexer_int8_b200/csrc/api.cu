@@ -557,6 +557,7 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     p.codes = q8 ? a->pooled_codes_dev : nullptr;
     p.scales = q8 ? a->pooled_scales_dev : nullptr;
     p.ld_pools = a->ld_pools;
+    p.fp8 = a->cache_fp8 != 0 ? 1 : 0;
     p.zero = reinterpret_cast<uint4 *>(sw.hist);
     p.zero_n16 = idx_multi ? static_cast<int64_t>(align_up(sw.zero_bytes, 16) / 16) : 0;
     rc = cuda_status(glm::launch_step_prep(p, st));
@@ -575,7 +576,7 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     float *part_acc = reinterpret_cast<float *>(ws + L.mla);
     float *part_ml = reinterpret_cast<float *>(ws + L.mla + mla_acc_bytes(parts));
     rc = cuda_status(glm::launch_mla_split_tc(a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
-                                              a->sm_scale, part_acc, part_ml, status, st, true));
+                                              a->sm_scale, part_acc, part_ml, status, st, true, a->cache_fp8 != 0));
     if (rc != GLM_OK) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, n_chunks, a->out_dev, a->out_f32_dev,
                                                a->lse_dev, st));

@@ -78,6 +78,7 @@ struct StepPrepArgs {
     int64_t ld_pools;
     uint4 *zero;
     int64_t zero_n16;
+    int fp8;                       // the cache holds FP8 rows
 };
 cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream);
 

@@ -18,7 +18,10 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(StepPrepArgs a,
     int cta = blockIdx.x;
     if (cta < store_ctas) {
         const int64_t row = static_cast<int64_t>(cta) * kPrepWarps + warp;
-        if (row < a.n_new) store_int8_row(a.latent, a.slots, row, a.cache, a.n_rows);
+        if (row < a.n_new) {
+            if (a.fp8) store_fp8_row(a.latent, a.slots, row, reinterpret_cast<uint8_t *>(a.cache), a.n_rows);
+            else store_int8_row(a.latent, a.slots, row, a.cache, a.n_rows);
+        }
         return;
     }
     cta -= store_ctas;

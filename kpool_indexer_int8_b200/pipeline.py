@@ -21,8 +21,8 @@ import torch
 
 from . import (GLM_OP_DECODE_STEP, GLM_OP_INDEX_SCORES_TOPK, GLM_OP_SPARSE_MLA, GLM_ROW_BYTES,
                glm_dsa_decode_step, glm_dsa_workspace_size, glm_expand_selection, glm_index_scores_topk,
-               glm_index_topk_expand, glm_index_topk_expand_q8, glm_kpool_build, glm_kpool_build_q8, glm_kv_store_int8,
-               glm_sparse_mla_decode, make_dims)
+               glm_index_topk_expand, glm_index_topk_expand_q8, glm_kpool_build, glm_kpool_build_q8, glm_kv_store_fp8,
+               glm_kv_store_int8, glm_sparse_mla_decode, glm_sparse_mla_decode_fp8, make_dims)
 
 LATENT = 512
 IDX_HEADS = 32
@@ -72,11 +72,13 @@ class DecodeBuffers:
     out_f32: Optional[torch.Tensor] = None
     pooled_codes: Optional[torch.Tensor] = None   # INT8 indexer state: int8 [B, ld_pools, 128]
     pooled_scales: Optional[torch.Tensor] = None  #                       fp32 [B, ld_pools]
+    fp8: bool = False                             # the cache holds FP8 rows (uint8)
 
 
 def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_new: int,
              select_k: int, out_width: int, sm_scale: float, ln_eps: float, max_new_pools: int,
-             device, keep_scores: bool = False, keep_f32: bool = False, q8: bool = False) -> DecodeBuffers:
+             device, keep_scores: bool = False, keep_f32: bool = False, q8: bool = False,
+             fp8: bool = False) -> DecodeBuffers:
     dims = make_dims(n_heads)
     ld_pools = max(1, ld_tokens // KPOOL)
     f = dict(device=device)
@@ -85,7 +87,8 @@ def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_
     ws_s = glm_dsa_workspace_size(dims, GLM_OP_DECODE_STEP, n_q, ld_pools, select_k, out_width)
     return DecodeBuffers(
         dims=dims, select_k=select_k, out_width=out_width, sm_scale=sm_scale, ln_eps=ln_eps,
-        cache=torch.zeros(n_rows, GLM_ROW_BYTES, dtype=torch.int8, **f),
+        cache=torch.zeros(n_rows, GLM_ROW_BYTES, dtype=torch.uint8 if fp8 else torch.int8, **f),
+        fp8=fp8,
         pooled=torch.zeros(batch, ld_pools, IDX_DIM, dtype=torch.float32, **f),
         k=torch.zeros(batch, ld_tokens, IDX_DIM, dtype=torch.bfloat16, **f),
         gate=torch.zeros(batch, ld_tokens, IDX_DIM, dtype=torch.bfloat16, **f),
@@ -120,6 +123,9 @@ def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_
 
 
 def store(b: DecodeBuffers, stream=None) -> None:
+    if b.fp8:
+        glm_kv_store_fp8(b.dims, b.new_latent, b.new_slots, b.cache, stream=stream)
+        return
     glm_kv_store_int8(b.dims, b.new_latent, b.new_slots, b.cache, stream=stream)
 
 
@@ -161,6 +167,10 @@ def index_topk_expand(b: DecodeBuffers, stream=None) -> None:
 
 
 def attend(b: DecodeBuffers, stream=None) -> None:
+    if b.fp8:
+        glm_sparse_mla_decode_fp8(b.dims, b.q, b.cache, b.rows, b.sm_scale, b.out, b.ws_mla, lse=b.lse,
+                                  out_f32=b.out_f32, stream=stream)
+        return
     glm_sparse_mla_decode(b.dims, b.q, b.cache, b.rows, b.sm_scale, b.out, b.ws_mla, lse=b.lse,
                           out_f32=b.out_f32, stream=stream)
 
@@ -184,4 +194,4 @@ def run_step(b: DecodeBuffers, stream=None) -> None:
                         slot_map=b.slot_map, rows=b.rows, topk=b.topk, q=b.q, sm_scale=b.sm_scale, out=b.out,
                         workspace=b.ws_step, n_sel=b.n_sel, tok=b.tok, scores=b.scores, lse=b.lse,
                         out_f32=b.out_f32, pooled_codes=b.pooled_codes, pooled_scales=b.pooled_scales,
-                        stream=stream)
+                        cache_fp8=b.fp8, stream=stream)

@@ -83,3 +83,31 @@ def test_sparse_mla_fp8_matches_oracle(cuda, n_heads, W, n_valid, n_rows):
         want = oracle.attention_f64(qf[n], c, c, sm, shared=True)
         assert_attention_close(g32[n], want, "fp8")
         assert_bf16_is_rounded_f32(gb[n], g32[n])
+
+
+def test_fp8_step_equals_separate_calls_and_stores_the_oracles_rows(cuda):
+    # the one-call step on an FP8 cache against the separate entry points (identical integers and
+    # attention), its cache against the oracle's FP8 store of every token, and its attention
+    # against the oracle's over the rows it selected
+    from kpool_indexer_int8_b200 import pipeline as P
+    from synth import device as sdev
+    inp = synth.generate(synth.PADDING_DECODE)
+    outs = []
+    for runner in (P.run_stages, P.run_step):
+        b = sdev.allocate_for(inp, cuda, keep_scores=True, keep_f32=True, fp8=True)
+        sdev.load(inp, b, build_prefix=True)
+        runner(b)
+        torch.cuda.synchronize()
+        outs.append(b)
+    a, c = outs
+    for name in ("cache", "pooled", "scores", "topk", "n_sel", "tok", "rows", "out_f32", "lse"):
+        assert torch.equal(getattr(a, name), getattr(c, name)), name
+    want = np.zeros(tuple(c.cache.shape), np.uint8)
+    oracle.store_fp8(inp.latent, inp.slots, want)
+    assert np.array_equal(np_(c.cache), want)
+    rows, o32 = np_(c.rows), np_(c.out_f32)
+    qf = synth.bf16_bits_to_f32(inp.q).astype(np.float64)
+    for n in range(len(inp.q_pos)):
+        valid = rows[n][rows[n] >= 0]
+        cr = oracle.dequant_rows_fp8(want, valid)
+        assert_attention_close(o32[n], oracle.attention_f64(qf[n], cr, cr, inp.sm_scale, shared=True), n)
