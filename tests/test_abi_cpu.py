@@ -148,3 +148,36 @@ def test_step_argument_checks():
     a.n_new = 0
     need = kp.glm_dsa_workspace_size(kp.make_dims(64), kp.GLM_OP_DECODE_STEP, 0, 16, 512, 2051)
     assert L.glm_dsa_decode_step(d, C.byref(a), FAKE, need - 1, None) == kp.GLM_ERR_WORKSPACE
+
+
+def test_fp8_entry_points_reject_before_launch():
+    L = kp.lib
+    d = C.byref(kp.make_dims(64))
+    bad = C.byref(kp.make_dims(64, qk_rope_head_dim=64))
+    assert L.glm_kv_store_fp8(bad, FAKE, FAKE, 1, FAKE, 1, None) == kp.GLM_ERR_UNSUPPORTED
+    assert L.glm_kv_store_fp8(d, None, FAKE, 1, FAKE, 1, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kv_store_fp8(d, FAKE, FAKE, 1, MIS, 1, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kv_store_fp8(d, None, None, 0, None, 0, None) == kp.GLM_OK        # n == 0: no-op
+    assert L.glm_sparse_mla_decode_fp8(bad, FAKE, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None, FAKE,
+                                       1 << 30, None) == kp.GLM_ERR_UNSUPPORTED
+    assert L.glm_sparse_mla_decode_fp8(d, FAKE, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None, FAKE, 16,
+                                       None) == kp.GLM_ERR_WORKSPACE
+    assert L.glm_sparse_mla_decode_fp8(d, FAKE, FAKE, 10, FAKE, 1, 0, 0.04, FAKE, None, None, FAKE,
+                                       1 << 30, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_sparse_mla_decode_fp8(d, MIS, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None, FAKE,
+                                       1 << 30, None) == kp.GLM_ERR_INVALID_ARG
+
+
+def test_algorithmic_bytes_of_the_tiny_decode():
+    # by hand: 128 visible pools x 512 B + q_idx 8,192 B + w 128 B + 16 top-k ids x 4 B; 64 gathered
+    # rows x 528 B + q and out 2 x 16 heads x 1,024 B + 80 indices x 4 B; one new row (1,024 B in,
+    # 528 B out, 8 B slot); one completed pool (4 x 512 B of k and gate in, 512 B out)
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    ab = bench.algorithmic_bytes(synth.generate(synth.TINY_DECODE))
+    assert ab["index"] == 128 * 512 + 8192 + 128 + 16 * 4
+    assert ab["mla"] == 64 * 528 + 2 * 16 * 1024 + 80 * 4
+    assert ab["store"] == 1560 and ab["kpool"] == 2560 and ab["gathered"] == 64
+    assert ab["total"] == ab["index"] + ab["mla"] + ab["store"] + ab["kpool"] == 144920
