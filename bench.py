@@ -455,7 +455,8 @@ def run_kernels(args, wl):
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "int8/bf16 in, f32 math", "data": "synthetic", "config": config_of(wl, args),
+        "dtype": "f32", "precision": "int8 (or fp8) cache rows and bf16 tensor-core operands, fp32 accumulation",
+        "data": "synthetic", "config": config_of(wl, args),
         "achieved_hbm_gbs_per_gpu": ab["total"] / (ms_per_step / 1e3) / 1e9,
         "algorithmic_bytes_per_step": ab["total"],
         "tokens_gathered_per_s": ab["gathered"] * args.steps * world / (ms / 1e3),
