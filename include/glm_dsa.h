@@ -279,8 +279,10 @@ int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk_dev,
  *               256-byte aligned. Its last 256 bytes start with a status word that the kernels set
  *               nonzero if a wait on the tensor cores gave up (the outputs are then invalid); it is
  *               never cleared by the library, so a caller that checks it zeroes it first.
- * 1 <= width <= 65536. The contractions run on the tensor cores (bf16 operands: the int8 codes and
- * the bf16 queries exactly; the softmax weights as a two-term bf16 split), accumulating in fp32.
+ * 1 <= width <= 65536. The contractions run on the tensor cores with fp16 operands, accumulating
+ * in fp32: the int8 codes exactly, each query head exactly after scaling it by a power of two
+ * (values below 2^-17 of the head's scaled range aside), the softmax weights as a two-term fp16
+ * split of p * scale_row / (the chunk's largest row scale).
  */
 int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q_dev, const int8_t *cache_dev,
                           int64_t n_rows, const int32_t *rows_dev, int32_t n_q, int32_t width,
@@ -309,12 +311,14 @@ int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q_dev, const
  *     2,056 bytes each, each region rounded up to 256 bytes, plus 256 bytes -- returns
  *     GLM_ERR_WORKSPACE before anything is enqueued (one 64-head query of width 2,176 needs about
  *     4.5 MiB, one 128-head query about 9 MiB).
- *   - The first call on a device looks up the scratch's device address for that device (the
- *     device current at the call); make that first call before any stream capture.
+ *   - Every call looks up the scratch's device address on the device current at the call; the
+ *     first call on a device also loads the library's device code there, so make that first call
+ *     before any stream capture.
  *   - Every call shares the one array, and the status word is cleared at the start of each call:
  *     calls that overlap on the GPU (other streams, other host threads) race on it and must be
  *     serialised by the caller.
- *   - GLM_ERR_CUDA does not update glm_last_cuda_error().
+ *   - The caller cannot read the scratch's status word; if a wait on the tensor cores gave up, the
+ *     call's outputs (out, lse, out_f32) are NaN instead.
  */
 #define GLM_NOALLOC_SCRATCH_BYTES (16u << 20)
 int glm_sparse_mla_decode_noalloc(const glm_dsa_dims *dims, const void *q_dev,

@@ -7,10 +7,12 @@
 #include "select.cuh"
 
 namespace {
-
 thread_local int g_last_cuda_error = 0;
-
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+}  // namespace
+
+namespace glm {
+namespace abi {
 
 int cuda_status(cudaError_t e) {
     if (e == cudaSuccess) return GLM_OK;
@@ -23,6 +25,28 @@ int num_sms() {
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     return sms > 0 ? sms : 148;
 }
+
+int check_mla(const glm_dsa_dims *dims, const void *q, const int8_t *cache, int64_t n_rows, const int32_t *rows,
+              int32_t n_q, int32_t width, float sm_scale, const void *out, const float *lse, const float *out_f32) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_q < 0 || n_rows < 0 || width < 1 || width > 65536 || n_q > 65535) return GLM_ERR_INVALID_ARG;
+    if (!(sm_scale == sm_scale)) return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (!q || !rows || !out || (n_rows > 0 && !cache)) return GLM_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || (cache && !aligned(cache, 16)) || !aligned(rows, 4) || !aligned(out, 16) ||
+        (lse && !aligned(lse, 4)) || (out_f32 && !aligned(out_f32, 16)))
+        return GLM_ERR_INVALID_ARG;
+    return GLM_OK;
+}
+
+}  // namespace abi
+}  // namespace glm
+
+namespace {
+using glm::abi::check_mla;
+using glm::abi::cuda_status;
+using glm::abi::num_sms;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
@@ -107,20 +131,6 @@ int check_kpool(const glm_dsa_dims *dims, const void *k, const void *gate, int64
         (pool_begin && !aligned(pool_begin, 4)) || (n_pools && !aligned(n_pools, 4)))
         return GLM_ERR_INVALID_ARG;
     if (static_cast<int64_t>(batch) * max_new_pools > (int64_t(1) << 40)) return GLM_ERR_INVALID_ARG;
-    return GLM_OK;
-}
-
-int check_mla(const glm_dsa_dims *dims, const void *q, const int8_t *cache, int64_t n_rows, const int32_t *rows,
-              int32_t n_q, int32_t width, float sm_scale, const void *out, const float *lse, const float *out_f32) {
-    int rc = glm_check_dims(dims);
-    if (rc != GLM_OK) return rc;
-    if (n_q < 0 || n_rows < 0 || width < 1 || width > 65536 || n_q > 65535) return GLM_ERR_INVALID_ARG;
-    if (!(sm_scale == sm_scale)) return GLM_ERR_INVALID_ARG;
-    if (n_q == 0) return GLM_OK;
-    if (!q || !rows || !out || (n_rows > 0 && !cache)) return GLM_ERR_INVALID_ARG;
-    if (!aligned(q, 16) || (cache && !aligned(cache, 16)) || !aligned(rows, 4) || !aligned(out, 16) ||
-        (lse && !aligned(lse, 4)) || (out_f32 && !aligned(out_f32, 16)))
-        return GLM_ERR_INVALID_ARG;
     return GLM_OK;
 }
 
@@ -465,18 +475,17 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t 
     const int H = dims->n_heads;
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
-    const int chunk = glm::mla_tc_chunk();
-    const int n_chunks = (width + chunk - 1) / chunk;
+    const glm::MlaPlan plan = glm::mla_plan(n_q, H, width, num_sms());
     const size_t parts = mla_parts(n_q, H, width);
     char *ws = static_cast<char *>(workspace);
     float *part_acc = reinterpret_cast<float *>(ws);
     float *part_ml = reinterpret_cast<float *>(ws + mla_acc_bytes(parts));
     int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = cuda_status(glm::launch_mla_split_tc(q, H, cache, n_rows, rows, n_q, width, sm_scale,
+    rc = cuda_status(glm::launch_mla_split_tc(plan, q, H, cache, n_rows, rows, n_q, width, sm_scale,
                                               part_acc, part_ml, status, st));
     if (rc != GLM_OK) return rc;
-    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32, lse, st));
+    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32, lse, st));
 }
 
 int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q, const uint8_t *cache,
@@ -489,18 +498,17 @@ int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q, const uin
     const int H = dims->n_heads;
     const size_t need = glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width);
     if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
-    const int chunk = glm::mla_tc_chunk();
-    const int n_chunks = (width + chunk - 1) / chunk;
+    const glm::MlaPlan plan = glm::mla_plan(n_q, H, width, num_sms());
     const size_t parts = mla_parts(n_q, H, width);
     char *ws = static_cast<char *>(workspace);
     float *part_acc = reinterpret_cast<float *>(ws);
     float *part_ml = reinterpret_cast<float *>(ws + mla_acc_bytes(parts));
     int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = cuda_status(glm::launch_mla_split_tc(q, H, c8, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml,
+    rc = cuda_status(glm::launch_mla_split_tc(plan, q, H, c8, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml,
                                               status, st, false, true));
     if (rc != GLM_OK) return rc;
-    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32, lse, st));
+    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32, lse, st));
 }
 
 int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *workspace, size_t ws_bytes,
@@ -570,15 +578,14 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
                               a->batch > 0 ? a->max_new_pools : 0);
     if (rc != GLM_OK) return rc;
     const int H = dims->n_heads;
-    const int chunk = glm::mla_tc_chunk();
-    const int n_chunks = (a->out_width + chunk - 1) / chunk;
+    const glm::MlaPlan plan = glm::mla_plan(a->n_q, H, a->out_width, sms);
     const size_t parts = mla_parts(a->n_q, H, a->out_width);
     float *part_acc = reinterpret_cast<float *>(ws + L.mla);
     float *part_ml = reinterpret_cast<float *>(ws + L.mla + mla_acc_bytes(parts));
-    rc = cuda_status(glm::launch_mla_split_tc(a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
+    rc = cuda_status(glm::launch_mla_split_tc(plan, a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
                                               a->sm_scale, part_acc, part_ml, status, st, true, a->cache_fp8 != 0));
     if (rc != GLM_OK) return rc;
-    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, n_chunks, a->out_dev, a->out_f32_dev,
+    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, plan.n_chunks, a->out_dev, a->out_f32_dev,
                                                a->lse_dev, st));
 }
 

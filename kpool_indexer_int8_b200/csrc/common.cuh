@@ -9,6 +9,40 @@
 
 #include "glm_dsa.h"
 
+// Phase stamps of a timeline build (compiled with -DGLM_TIMELINE; they compile to nothing
+// otherwise): thread t of a CTA records %globaltimer into slot k of the CTA's row of a per-kernel
+// table, read back through <table>_read(host buffer of 2048 x 16 uint64).
+#ifdef GLM_TIMELINE
+#define GLM_TL_TABLE(name)                                                            \
+    __device__ unsigned long long name[2048][16];                                     \
+    extern "C" int name##_read(void *h) { return (int)cudaMemcpyFromSymbol(h, name, sizeof(name)); }
+#define GLM_TL_AT(name, k, t)                                                         \
+    do {                                                                              \
+        if (threadIdx.x == (t)) {                                                     \
+            unsigned long long t_;                                                    \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_)::"memory");          \
+            name[(blockIdx.y * gridDim.x + blockIdx.x) & 2047][k] = t_;               \
+        }                                                                             \
+    } while (0)
+#define GLM_TL_SMID(name)                                                             \
+    do {                                                                              \
+        if (threadIdx.x == 0) {                                                       \
+            unsigned s_;                                                              \
+            asm volatile("mov.u32 %0, %%smid;" : "=r"(s_));                          \
+            name[(blockIdx.y * gridDim.x + blockIdx.x) & 2047][15] = s_;              \
+        }                                                                             \
+    } while (0)
+#else
+#define GLM_TL_TABLE(name)
+#define GLM_TL_AT(name, k, t) \
+    do {                      \
+    } while (0)
+#define GLM_TL_SMID(name) \
+    do {                  \
+    } while (0)
+#endif
+#define GLM_TL(name, k) GLM_TL_AT(name, k, 0)
+
 namespace glm {
 
 constexpr int kLatent = 512;        // kv_lora_rank

@@ -4,10 +4,19 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "glm_dsa.h"
 #include "sparse_mla.cuh"
 #include "topk.cuh"
 
 namespace glm {
+
+// Host helpers of the C ABI shared by its source files.
+namespace abi {
+int cuda_status(cudaError_t e);   // GLM_OK, or GLM_ERR_CUDA with e kept for glm_last_cuda_error()
+int num_sms();                    // SMs of the current device
+int check_mla(const glm_dsa_dims *dims, const void *q, const int8_t *cache, int64_t n_rows, const int32_t *rows,
+              int32_t n_q, int32_t width, float sm_scale, const void *out, const float *lse, const float *out_f32);
+}  // namespace abi
 
 cudaError_t launch_store_int8(const void *latent, const int64_t *slots, int64_t n, int8_t *cache,
                               int64_t n_rows, cudaStream_t stream, int num_sms);

@@ -9,6 +9,8 @@
 
 namespace glm {
 
+GLM_TL_TABLE(glm_tl_combine)
+
 constexpr int kMaxCombineChunks = 1024;  // 65536 / 64
 constexpr int kCombineThreads = 512;
 constexpr int kChunkGroups = kCombineThreads / (kLatent / 4);   // 4 groups of 128 threads
@@ -32,8 +34,21 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const floa
                                                                       int n_heads, int n_chunks,
                                                                       uint16_t *__restrict__ out,
                                                                       float *__restrict__ out_f32,
-                                                                      float *__restrict__ lse) {
+                                                                      float *__restrict__ lse,
+                                                                      const int *__restrict__ poison) {
+    GLM_TL(glm_tl_combine, 0);
+    GLM_TL_SMID(glm_tl_combine);
     pdl_begin();
+    GLM_TL(glm_tl_combine, 1);
+    if (poison && __ldcg(poison) != 0) {   // a split CTA gave up a wait: its partial is missing
+        const int64_t ob = (static_cast<int64_t>(blockIdx.y) * n_heads + blockIdx.x) * kLatent;
+        for (int i = threadIdx.x; i < kLatent; i += blockDim.x) {
+            out[ob + i] = 0x7fc0u;   // bf16 NaN
+            if (out_f32) out_f32[ob + i] = __int_as_float(0x7fc00000);
+        }
+        if (lse && threadIdx.x == 0) lse[static_cast<int64_t>(blockIdx.y) * n_heads + blockIdx.x] = __int_as_float(0x7fc00000);
+        return;
+    }
     __shared__ float wgt[kMaxCombineChunks];
     __shared__ float lsum[kMaxCombineChunks];
     __shared__ float red[kCombineThreads / 32];
@@ -120,15 +135,16 @@ __global__ void __launch_bounds__(kCombineThreads) mla_combine_kernel(const floa
                   (static_cast<uint32_t>(__bfloat16_as_ushort(__float2bfloat16_rn(o[3]))) << 16);
     *reinterpret_cast<uint2 *>(out + ob) = make_uint2(lo, hi);
     if (out_f32) *reinterpret_cast<float4 *>(out_f32 + ob) = make_float4(o[0], o[1], o[2], o[3]);
+    GLM_TL(glm_tl_combine, 2);
     if (lse && t == 0) lse[static_cast<int64_t>(n) * n_heads + h] = L > 0.0f ? M + logf(L) : -INFINITY;
 }
 
 cudaError_t launch_mla_combine(const float *part_acc, const float *part_ml, int n_q, int n_heads,
                                int n_chunks, void *out, float *out_f32, float *lse,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, const int *poison) {
     dim3 grid(n_heads, n_q);
     launch_pdl(mla_combine_kernel, dim3(grid), dim3(kCombineThreads), 0, stream, part_acc, part_ml, n_heads,
-               n_chunks, static_cast<uint16_t *>(out), out_f32, lse);
+               n_chunks, static_cast<uint16_t *>(out), out_f32, lse, poison);
     return cudaGetLastError();
 }
 

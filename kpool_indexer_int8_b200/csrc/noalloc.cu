@@ -8,10 +8,11 @@
 // into the library. Every GPU that loads the library holds this array until the process exits.
 //
 // The computation is exactly glm_sparse_mla_decode's: the same split and combine kernels run on
-// the same data, only the scratch lives here instead of in a caller buffer.
-#include <mutex>
-
+// the same data with the same plan, only the scratch lives here instead of in a caller buffer.
+// The caller cannot read the scratch's status word, so a timed-out wait shows in the outputs
+// instead: the combine then writes NaN to every output of the call.
 #include "common.cuh"
+#include "kernels.cuh"
 #include "sparse_mla.cuh"
 
 namespace {
@@ -20,30 +21,7 @@ namespace {
 // stands for the symbol; its device address comes from cudaGetSymbolAddress below.
 static __device__ __align__(256) unsigned char g_mla_scratch[GLM_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_scratch_mutex;
-void *g_scratch_addr[kMaxDevices] = {};
-
 size_t round256(size_t x) { return (x + 255) / 256 * 256; }
-
-// Device address of the scratch on the current device, looked up once per device.
-cudaError_t scratch_address(void **out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (g_scratch_addr[dev] == nullptr) {
-        void *p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_mla_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_addr[dev] = p;
-    }
-    *out = g_scratch_addr[dev];
-    return cudaSuccess;
-}
-
-int noalloc_cuda_status(cudaError_t e) { return e == cudaSuccess ? GLM_OK : GLM_ERR_CUDA; }
 
 }  // namespace
 
@@ -52,28 +30,22 @@ extern "C" int glm_sparse_mla_decode_noalloc(const glm_dsa_dims *dims, const voi
                                              const int32_t *rows, int32_t n_q, int32_t width,
                                              float sm_scale, void *out, float *lse,
                                              float *out_f32, void *stream) {
-    int rc = glm_check_dims(dims);
-    if (rc != GLM_OK) return rc;
-    if (n_q < 0 || n_rows < 0 || width < 1 || width > 65536 || n_q > 65535) return GLM_ERR_INVALID_ARG;
-    if (!(sm_scale == sm_scale)) return GLM_ERR_INVALID_ARG;
-    if (n_q == 0) return GLM_OK;
-    if (!q || !rows || !out || (n_rows > 0 && !cache)) return GLM_ERR_INVALID_ARG;
-    const uintptr_t a16 = 15;
-    if ((reinterpret_cast<uintptr_t>(q) & a16) || (cache && (reinterpret_cast<uintptr_t>(cache) & a16)) ||
-        (reinterpret_cast<uintptr_t>(rows) & 3) || (reinterpret_cast<uintptr_t>(out) & a16) ||
-        (lse && (reinterpret_cast<uintptr_t>(lse) & 3)) || (out_f32 && (reinterpret_cast<uintptr_t>(out_f32) & a16)))
-        return GLM_ERR_INVALID_ARG;
-    // size of this call's scratch; larger requests are refused before anything is enqueued
+    int rc = glm::abi::check_mla(dims, q, cache, n_rows, rows, n_q, width, sm_scale, out, lse, out_f32);
+    if (rc != GLM_OK || n_q == 0) return rc;
+    // size of this call's scratch, for the smallest chunk any plan uses; larger requests are
+    // refused before anything is enqueued
     const int H = dims->n_heads;
     const int chunk = glm::mla_tc_chunk();
-    const int n_chunks = (width + chunk - 1) / chunk;
-    const size_t parts = static_cast<size_t>(n_q) * static_cast<size_t>(n_chunks) * static_cast<size_t>(H);
+    const size_t parts = static_cast<size_t>(n_q) * static_cast<size_t>((width + chunk - 1) / chunk) *
+                         static_cast<size_t>(H);
     const size_t acc_bytes = round256(parts * glm::kLatent * sizeof(float));
     const size_t ml_bytes = round256(parts * 2 * sizeof(float));
     if (acc_bytes + ml_bytes + 256 > GLM_NOALLOC_SCRATCH_BYTES) return GLM_ERR_WORKSPACE;
 
+    // the scratch's device address on the current device, looked up on every call (a host-side
+    // query; the first one on a device loads the library's device code there)
     void *base = nullptr;
-    rc = noalloc_cuda_status(scratch_address(&base));
+    rc = glm::abi::cuda_status(cudaGetSymbolAddress(&base, g_mla_scratch));
     if (rc != GLM_OK) return rc;
     char *ws = static_cast<char *>(base);
     float *part_acc = reinterpret_cast<float *>(ws);
@@ -81,11 +53,12 @@ extern "C" int glm_sparse_mla_decode_noalloc(const glm_dsa_dims *dims, const voi
     int *status = reinterpret_cast<int *>(ws + acc_bytes + ml_bytes);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the status word keeps the previous call's value: clear it for this call
-    rc = noalloc_cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st));
+    rc = glm::abi::cuda_status(cudaMemsetAsync(status, 0, sizeof(int), st));
     if (rc != GLM_OK) return rc;
-    rc = noalloc_cuda_status(glm::launch_mla_split_tc(q, H, cache, n_rows, rows, n_q, width, sm_scale,
-                                                      part_acc, part_ml, status, st));
+    const glm::MlaPlan plan = glm::mla_plan(n_q, H, width, glm::abi::num_sms());
+    rc = glm::abi::cuda_status(glm::launch_mla_split_tc(plan, q, H, cache, n_rows, rows, n_q, width, sm_scale,
+                                                        part_acc, part_ml, status, st));
     if (rc != GLM_OK) return rc;
-    return noalloc_cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, n_chunks, out, out_f32,
-                                                       lse, st));
+    return glm::abi::cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32,
+                                                         lse, st, status));
 }

@@ -3,348 +3,487 @@
 // dequantisation fused in, the shared 512-d latent is both K and V, split-KV decode, fp32
 // softmax and accumulation; 'The tested MLA contract': one KV head, negative index padding).
 //
-// One CTA per (query, chunk of 64 index entries); heads are the MMA M dimension (M = 64 for up
-// to 64 heads, 128 above; missing heads are zero rows):
-//   1. gather: each entry's 512 int8 codes are widened to bf16 (exact: |code| <= 127; the E4M3
-//      codes of the FP8 row are exact in bf16 as well) into a shared tile C[64 rows x 512] stored as 8x8 core matrices, its fp32 scale to a register
-//      file in shared memory; the query block Q[heads x 512] goes to shared memory the same way.
-//   2. S = Q . C^T on tcgen05 (kind::f16, fp32 accumulator in tensor memory, 32 MMAs of K = 16).
-//      C is the K-major B operand here.
-//   3. softmax of the chunk, two threads per head (one TMEM lane, half of the entries each, the
-//      halves' maxima and sums exchanged in shared memory): s = S * scale_j * sm_scale, m = max,
-//      p = exp(s - m), l = sum p; P' = p * scale_j (the V dequantisation scale folded in) is split
-//      into bf16 hi + lo so that the PV product keeps ~16 mantissa bits of P'.
-//   4. O^T = C^T . P'^T: the 512 latent dims are the M dimension (4 tiles of M = 128) and the heads
-//      the N dimension, so that in tensor memory one lane holds one latent dim of every head. The
-//      same tile C is now the MN-major A operand (a core matrix of 8 rows x 8 dims serves both
-//      products) and P' the K-major B operand; 2 terms x 4 K-steps x 4 tiles = 32 MMAs.
-//   5. (m, l) and the unnormalised O of every head go to the workspace (one lane per latent dim:
-//      each warp store is 32 consecutive floats of one head); the combine kernel merges the
+// One CTA per (query, chunk of ROWS index entries, group of NH heads); the rows of a chunk are
+// the MMA M dimension, the heads the N dimension:
+//   1. the query block of the head group goes to shared memory as fp16, each head scaled by the
+//      power of two 2^e_h that puts its largest magnitude in [2^14, 2^15) (every bf16 value of
+//      magnitude >= 2^-17 after scaling is exact in fp16; the scores are multiplied back by
+//      2^-e_h); in the one-call step this happens before the kernel waits for the index lists;
+//   2. gather: one 1-D bulk copy per valid entry brings its whole 528-byte row (codes, fp32
+//      scale, zero pad) into shared memory, all completing on one mbarrier; the codes are then
+//      widened to fp16 (exact: |code| <= 127; E4M3 codes are exact in fp16 as well) into a tile
+//      C[ROWS x 512] of 8x8 core matrices -- the int8 codes through byte permutes and one packed
+//      subtraction (1024 + code + 128 built as fp16 bits, minus 1152), no integer conversions;
+//   3. S^T = C . Q^T on tcgen05 (kind::f16, fp32 accumulator in tensor memory: lane = row,
+//      column = head), 32 MMAs of K = 16;
+//   4. softmax over the chunk's rows for each head: one thread per row and half of the heads;
+//      per-head maxima and sums by a transposing warp butterfly (V - 1 + log shuffles for V
+//      values) and four quadrant partials in shared memory; p = exp2(s - m) with
+//      s = S * scale_row * sm_scale * log2(e) * 2^-e_h; P' = p * scale_row / scale_max (the
+//      chunk's largest row scale, so P' <= 1) as an fp16 hi + lo pair;
+//   5. O^T = C^T . [P'_hi | P'_lo]^T: the 512 latent dims are M (4 tiles of 128), the hi and lo
+//      heads side by side are N = 2 NH, K = ROWS; the tile C is now the MN-major A operand (one
+//      core matrix of 8 rows x 8 dims serves both products);
+//   6. acc = scale_max * (O_hi + O_lo) and (m, l) of each head go to the workspace (lane = latent
+//      dim: every warp store is 32 consecutive floats of one head); the combine kernel merges the
 //      chunks by log-sum-exp.
-// Tensor memory: 512 columns (S in columns 0..M-1, then the 4 O^T tiles of M columns each over
-// columns 0..4M-1 once S has been read).
-// Every wait on the tensor cores is bounded; a timeout sets a status word and the CTA still
-// frees its tensor memory and exits.
+// Every wait is bounded; a timeout sets a status bit, waits (bounded) for this CTA's copies and
+// MMAs still in flight, frees the tensor memory and leaves the partial unwritten.
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 #include "sparse_mla.cuh"
 #include "tc.cuh"
 
 namespace glm {
 
-constexpr int kTcRows = 64;
-constexpr int kTcThreads = 256;
-constexpr uint32_t kWaitLimit = 1u << 22;
+GLM_TL_TABLE(glm_tl_split)
 
-template <int M>
-struct TcLayout {
-    static constexpr int kQ = 0;                     // M/8 head groups x 64 dim groups x 128 B
-    static constexpr int kC = kQ + M * 1024;         // 8 row groups x 64 dim groups x 128 B
-    static constexpr int kPhi = kC + 64 * 1024;      // M/8 head groups x 8 row groups x 128 B
-    static constexpr int kPlo = kPhi + M * 128;
-    static constexpr int kScl = kPlo + M * 128;      // 64 fp32 scales
-    static constexpr int kRow = kScl + 256;          // 64 row indices
-    static constexpr int kBar = kRow + 256;          // 2 mbarriers
-    static constexpr int kTmem = kBar + 16;          // tensor-memory base address
-    static constexpr int kFlag = kTmem + 16;
-    static constexpr int kPmax = kFlag + 16;         // [2 column halves][128 heads] partial maxima
-    static constexpr int kPl = kPmax + 2 * 128 * 4;  // [2][128] partial sums
-    static constexpr int kBytes = kPl + 2 * 128 * 4;
+constexpr int kMlaThreads = 256;
+constexpr uint32_t kMlaWaitLimit = 1u << 22;
+
+template <int ROWS, int NH>
+struct MlaLayout {
+    static constexpr int kPBytes = ROWS * 4 * NH;                     // ROWS x 2 NH fp16 (hi | lo)
+    static constexpr int kRawBytes = ROWS * kRowBytes;
+    static constexpr int kC = 0;                                      // ROWS/8 row groups x 64 dim groups x 128 B
+    static constexpr int kRaw = kC + ROWS * 1024;                     // gathered rows, 528 B apart; then P'
+    static constexpr int kQ = kRaw + (kRawBytes > kPBytes ? kRawBytes : kPBytes);   // NH/8 x 64 x 128 B
+    static constexpr int kScl = kQ + NH * 1024;                       // ROWS fp32 row scales
+    static constexpr int kRow = kScl + ROWS * 4;                      // ROWS row indices
+    static constexpr int kRed = kRow + ROWS * 4;                      // [4 quadrants][NH] partial maxima
+    static constexpr int kRed2 = kRed + 4 * NH * 4;                   // [4][NH] partial sums
+    static constexpr int kQk = kRed2 + 4 * NH * 4;                    // NH fp32 score factors
+    static constexpr int kQmax = kQk + NH * 4;                        // NH uint32 |q| maxima (bf16 bits)
+    static constexpr int kWords = kQmax + NH * 4;                     // [0] scale max bits, [1] tmem base
+    static constexpr int kBar = kWords + 16;                          // 3 mbarriers
+    static constexpr int kBytes = kBar + 3 * 8;
+    static_assert(kQ % 16 == 0 && kRaw % 16 == 0 && kBar % 8 == 0, "alignment");
 };
 
-__device__ __forceinline__ uint32_t codes_to_bf16x2(uint32_t w, int shift) {
-    const float a = static_cast<float>(static_cast<int8_t>((w >> shift) & 0xffu));
-    const float b = static_cast<float>(static_cast<int8_t>((w >> (shift + 8)) & 0xffu));
-    return (__float_as_uint(a) >> 16) | (__float_as_uint(b) & 0xffff0000u);
+// Four int8 codes (one little-endian word) as four exact fp16 values (two fp16x2 words).
+__device__ __forceinline__ void codes_to_f16x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    const uint32_t t = w ^ 0x80808080u;                          // each code c as the byte c + 128
+    const uint32_t a = __byte_perm(t, 0x64646464u, 0x5140u);     // fp16 bits 0x64bb = 1024 + c + 128
+    const uint32_t b = __byte_perm(t, 0x64646464u, 0x5342u);
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x64806480u));   // - 1152 (exact)
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x64806480u));
+}
+// Four E4M3 codes as four exact fp16 values (hardware conversion of code pairs).
+__device__ __forceinline__ void fp8_to_f16x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xffffu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+    lo = static_cast<uint32_t>(a.x) | (static_cast<uint32_t>(a.y) << 16);
+    hi = static_cast<uint32_t>(b.x) | (static_cast<uint32_t>(b.y) << 16);
 }
 
-// One E4M3 code (OCP E4M3FN: bias 7, subnormals) as bf16 bits -- exact: 3 mantissa bits and
-// exponents 2^-9 .. 2^8 fit bf16. (Codes 0x7F / 0xFF, NaN, are never written by the store.)
-__device__ __forceinline__ uint32_t e4m3_bf16_bits(uint32_t b) {
-    const uint32_t s = (b & 0x80u) << 8, e = (b >> 3) & 15u, m = b & 7u;
-    if (e != 0u) return s | ((e + 120u) << 7) | (m << 4);   // 2^(e-7) (1 + m/8)
-    if (m == 0u) return s;
-    const uint32_t p = 31u - __clz(m);                          // m 2^-9 = 2^(p-9) (1 + frac)
-    return s | ((p + 118u) << 7) | (((m << (3u - p)) & 7u) << 4);
+__device__ __forceinline__ uint32_t f16x2_rn(float a, float b) {   // .x = a (low half)
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
 }
-__device__ __forceinline__ uint32_t fp8_to_bf16x2(uint32_t w, int shift) {
-    return e4m3_bf16_bits((w >> shift) & 0xffu) | (e4m3_bf16_bits((w >> (shift + 8)) & 0xffu) << 16);
+__device__ __forceinline__ float f16_lo_f(uint32_t p) { return __half2float(__ushort_as_half(static_cast<unsigned short>(p & 0xffffu))); }
+__device__ __forceinline__ float f16_hi_f(uint32_t p) { return __half2float(__ushort_as_half(static_cast<unsigned short>(p >> 16))); }
+
+template <int V>
+__device__ __forceinline__ void tmem_ld_v(uint32_t taddr, uint32_t (&r)[V]) {
+    if constexpr (V == 8) tc::tmem_ld8(taddr, r);
+    else if constexpr (V == 16) tc::tmem_ld16(taddr, r);
+    else tc::tmem_ld32(taddr, r);
 }
 
-__device__ __forceinline__ uint16_t bf16_rn_bits(float x) { return __bfloat16_as_ushort(__float2bfloat16_rn(x)); }
+// Reduce V values per lane (V a power of two <= 32) across the warp's 32 lanes with max (kMax) or
+// sum: halving steps hand half of the values to the partner lane, so that after log2(V) steps lane
+// l holds value index (l >> (5 - log2 V)) & (V - 1), reduced over the lanes that differ from l in
+// the bits already used; the remaining steps finish the reduction over the other bits. Returns the
+// lane's value (every lane with the same index holds the same result).
+template <int V, bool kMax>
+__device__ __forceinline__ float butterfly(float (&v)[V]) {
+    const int lane = threadIdx.x & 31;
+    auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+#pragma unroll
+    for (int half = V / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int i = 0; i < half; i++) {
+            const float send = up ? v[i] : v[i + half];
+            const float keep = up ? v[i + half] : v[i];
+            v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, bit));
+        }
+    }
+    float r = v[0];
+    constexpr int kRest = (V == 32) ? 0 : (V == 16) ? 1 : (V == 8) ? 2 : (V == 4) ? 3 : (V == 2) ? 4 : 5;
+#pragma unroll
+    for (int k = 0; k < kRest; k++) r = op(r, __shfl_xor_sync(0xffffffffu, r, 1 << (kRest - 1 - k)));
+    return r;
+}
 
-template <int M, bool kFp8>
-__global__ void __launch_bounds__(kTcThreads, 1) mla_split_tc_kernel(
-    const uint16_t *__restrict__ q, int n_heads, const int8_t *__restrict__ cache, int64_t n_rows,
-    const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks,
+template <int ROWS, int NH, bool kFp8>
+__global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
+    const uint16_t *__restrict__ q, int n_heads, const uint8_t *__restrict__ cache, int64_t n_rows,
+    const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks, int n_hg,
     float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status, int early_q) {
-    // early_q: the query block is an input no preceding kernel writes (the one-call step), so its
-    // loads are issued before waiting for the preceding kernel; only the row indices wait for it
+    using L = MlaLayout<ROWS, NH>;
+    constexpr int V = NH / 2;             // heads per softmax thread
+    constexpr int kLboP = 32 * NH;        // P': bytes between row groups (2 NH / 8 head groups x 128 B)
+    // early_q: the query block is an input no preceding kernel writes (the one-call step), so it is
+    // staged before waiting for the preceding kernel; only the row indices wait for it
     if (early_q) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     else pdl_begin();
-    using Lay = TcLayout<M>;
     extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char *Qs = smem + Lay::kQ;
-    unsigned char *Cs = smem + Lay::kC;
-    unsigned char *Phi = smem + Lay::kPhi;
-    unsigned char *Plo = smem + Lay::kPlo;
-    float *scl = reinterpret_cast<float *>(smem + Lay::kScl);
-    int *ridx = reinterpret_cast<int *>(smem + Lay::kRow);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + Lay::kBar);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + Lay::kTmem);
-    int *flag = reinterpret_cast<int *>(smem + Lay::kFlag);
+    unsigned char *Cs = smem + L::kC;
+    unsigned char *raw = smem + L::kRaw;
+    unsigned char *Ps = smem + L::kRaw;
+    unsigned char *Qs = smem + L::kQ;
+    float *scl = reinterpret_cast<float *>(smem + L::kScl);
+    int *ridx = reinterpret_cast<int *>(smem + L::kRow);
+    float *red = reinterpret_cast<float *>(smem + L::kRed);
+    float *red2 = reinterpret_cast<float *>(smem + L::kRed2);
+    float *qk = reinterpret_cast<float *>(smem + L::kQk);
+    unsigned *qmax = reinterpret_cast<unsigned *>(smem + L::kQmax);
+    unsigned *words = reinterpret_cast<unsigned *>(smem + L::kWords);
+    const uint32_t bar0 = tc::smem_addr(smem + L::kBar);
+    const uint32_t bar_g = bar0, bar_s = bar0 + 8, bar_o = bar0 + 16;
 
-    const int n = blockIdx.y, c = blockIdx.x, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t ml_base = (static_cast<int64_t>(n) * n_chunks + c) * n_heads;
+    const int n = blockIdx.y, c = blockIdx.x / n_hg, hg = blockIdx.x % n_hg;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h0 = hg * NH;
+    const int nh_real = min(NH, n_heads - h0);
+    const int64_t ml_base = (static_cast<int64_t>(n) * n_chunks + c) * n_heads + h0;
+    GLM_TL(glm_tl_split, 0);
+    GLM_TL_SMID(glm_tl_split);
 
-    // the query block (bf16 [heads x 512] as core matrices: head group stride 8192 B, dim group 128 B)
-    constexpr int kQIters = M * 64 / kTcThreads;           // 16-byte query pieces per thread
-    const uint16_t *qn = q + static_cast<int64_t>(n) * n_heads * kLatent;
-    uint4 qv[kQIters];
+    // 1. the query block: thread t holds head qh = 8 ((t >> 3) % (NH/8)) + (t & 7), dim groups
+    //    qd0 + i (256/NH) (8 consecutive heads of one dim group per 8 lanes: conflict-free stores)
+    constexpr int kQPieces = NH * 64 / kMlaThreads;
+    constexpr int kQStride = kMlaThreads / NH;
+    const int qh = ((tid >> 3) % (NH / 8)) * 8 + (tid & 7);
+    const int qd0 = (tid >> 3) / (NH / 8);
+    const bool qreal = qh < nh_real;
+    if (tid < NH) qmax[tid] = 0u;
+    if (tid == 0) words[0] = 0u;
+    uint4 qv[kQPieces];
+    {
+        const uint4 *qn = reinterpret_cast<const uint4 *>(q + (static_cast<int64_t>(n) * n_heads + h0 + (qreal ? qh : 0)) * kLatent);
 #pragma unroll
-    for (int it = 0; it < kQIters; it++) {
-        const int i = it * kTcThreads + tid;
-        const int g = i >> 5, t = i & 31;
-        const int h = (g % (M / 8)) * 8 + (t & 7);
-        const int dg = (g / (M / 8)) * 4 + (t >> 3);
-        qv[it] = h < n_heads ? __ldg(reinterpret_cast<const uint4 *>(qn + static_cast<int64_t>(h) * kLatent) + dg)
-                             : make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < kQPieces; i++) qv[i] = qreal ? __ldg(qn + qd0 + i * kQStride) : make_uint4(0u, 0u, 0u, 0u);
     }
-    auto store_q = [&]() {
+    unsigned mx = 0u;   // largest |q| of the thread's pieces, as bf16 magnitude bits (ordered as integers)
 #pragma unroll
-        for (int it = 0; it < kQIters; it++) {
-            const int i = it * kTcThreads + tid;
-            const int g = i >> 5, t = i & 31;
-            const int hg = g % (M / 8);
-            const int h = hg * 8 + (t & 7);
-            const int dg = (g / (M / 8)) * 4 + (t >> 3);
-            *reinterpret_cast<uint4 *>(Qs + hg * 8192 + dg * 128 + (h & 7) * 16) = qv[it];
+    for (int i = 0; i < kQPieces; i++) {
+        const uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+#pragma unroll
+        for (int e = 0; e < 4; e++) mx = max(mx, max(w4[e] & 0x7fffu, (w4[e] >> 16) & 0x7fffu));
+    }
+    __syncthreads();
+    if (qreal) atomicMax(&qmax[qh], mx);
+    __syncthreads();
+    {
+        const unsigned m = qmax[qh];
+        int e = 0;
+        if (m != 0u) {
+            const int E = static_cast<int>(m >> 7) - 127;   // exponent of the largest magnitude
+            e = min(120, max(-120, 14 - E));
         }
-    };
-    if (early_q) asm volatile("griddepcontrol.wait;" ::: "memory");   // (the query loads stay in flight)
-
-    if (tid == 0) *flag = 0;
-    __syncthreads();
-    if (tid < kTcRows) {
-        const int j = c * kTcRows + tid;
-        const int r = j < width ? rows[static_cast<int64_t>(n) * width + j] : -1;
-        const bool ok = r >= 0 && r < n_rows;
-        ridx[tid] = ok ? r : -1;
-        if (ok) atomicOr(flag, 1);
+        const float f = __uint_as_float(static_cast<uint32_t>(e + 127) << 23);   // 2^e, exact
+        if (tid < NH) {
+            const unsigned mt = qmax[tid];
+            int et = 0;
+            if (mt != 0u) et = min(120, max(-120, 14 - (static_cast<int>(mt >> 7) - 127)));
+            qk[tid] = sm_scale * 1.4426950408889634f * __uint_as_float(static_cast<uint32_t>(127 - et) << 23);
+        }
+#pragma unroll
+        for (int i = 0; i < kQPieces; i++) {
+            const uint32_t w4[4] = {qv[i].x, qv[i].y, qv[i].z, qv[i].w};
+            uint32_t o[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++)
+                o[k] = f16x2_rn(__uint_as_float(w4[k] << 16) * f, __uint_as_float(w4[k] & 0xffff0000u) * f);
+            const int dg = qd0 + i * kQStride;
+            *reinterpret_cast<uint4 *>(Qs + (qh >> 3) * 8192 + dg * 128 + (qh & 7) * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
     }
-    __syncthreads();
-    if (*flag == 0) {  // no valid entry in this chunk: an empty partial
-        for (int h = tid; h < n_heads; h += blockDim.x) {
-            part_ml[2 * (ml_base + h)] = -INFINITY;
-            part_ml[2 * (ml_base + h) + 1] = 0.0f;
+    GLM_TL(glm_tl_split, 1);
+    if (early_q) asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("fence.proxy.async.global;" ::: "memory");   // rows written before this kernel are read by bulk copies
+
+    // 2. the chunk's row indices (entries past width or outside [0, n_rows) are padding)
+    int myrow = -1;
+    if (tid < ROWS) {
+        const int j = c * ROWS + tid;
+        const int r = j < width ? rows[static_cast<int64_t>(n) * width + j] : -1;
+        myrow = (r >= 0 && r < n_rows) ? r : -1;
+        ridx[tid] = myrow;
+    }
+    const int n_valid = __syncthreads_count(myrow >= 0);
+    GLM_TL(glm_tl_split, 2);
+    if (n_valid == 0) {   // no valid entry in this chunk: an empty partial
+        if (tid < nh_real) {
+            part_ml[2 * (ml_base + tid)] = -INFINITY;
+            part_ml[2 * (ml_base + tid) + 1] = 0.0f;
         }
         return;
     }
     if (warp == 0) {
-        tc::tmem_alloc(tc::smem_addr(tmem_slot), 512);
+        tc::tmem_alloc(tc::smem_addr(&words[1]), 8 * NH);
         tc::tmem_relinquish();
         tc::fence_before_sync();
     }
-    if (tid == 32) {
-        tc::mbar_init(tc::smem_addr(&bar[0]), 1);
-        tc::mbar_init(tc::smem_addr(&bar[1]), 1);
-        tc::mbar_fence_init();
+    if (warp == 1) {
+        if (lane == 0) {
+            tc::mbar_init(bar_g, 1);
+            tc::mbar_init(bar_s, 1);
+            tc::mbar_init(bar_o, 1);
+            tc::mbar_fence_init();
+            tc::mbar_arrive_expect_tx(bar_g, static_cast<uint32_t>(n_valid) * kRowBytes);
+        }
+        __syncwarp();
+        // every valid entry's whole row: one bulk copy each (528 = 33 x 16 bytes, 16-byte aligned)
+        const uint32_t raw_addr = tc::smem_addr(raw);
+#pragma unroll
+        for (int j = lane; j < ROWS; j += 32) {
+            const int r = ridx[j];
+            if (r >= 0) tc::bulk_g2s(raw_addr + j * kRowBytes, cache + static_cast<int64_t>(r) * kRowBytes, kRowBytes, bar_g);
+        }
+    }
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = words[1];
+    bool ok = tc::mbar_wait(bar_g, 0, kMlaWaitLimit);
+    GLM_TL(glm_tl_split, 3);
+    if (!__syncthreads_and(ok)) {   // the rows did not arrive: wait once more, then give up
+        if (tid == 0) atomicOr(status, 16);
+        tc::mbar_wait(bar_g, 0, kMlaWaitLimit);
+        __syncthreads();
+        goto done;
     }
 
-    // 1. gather the chunk's rows (codes widened to bf16) and its scales; every global load of a
-    //    thread is issued before any of them is used, so the CTA waits for one round trip
-    constexpr int kRowIters = kTcRows * 32 / kTcThreads;   // 16-byte code pieces per thread
+    // 3. row scales, their maximum, and the codes widened to fp16 core matrices
+    if (tid < ROWS) {
+        const float s = myrow >= 0 ? *reinterpret_cast<const float *>(raw + tid * kRowBytes + kLatent) : 0.0f;
+        scl[tid] = s;
+        const unsigned sm = __reduce_max_sync(0xffffffffu, __float_as_uint(s));   // scales are >= 0
+        if (lane == 0) atomicMax(&words[0], sm);
+    }
     {
-        uint4 v[kRowIters];
+        constexpr int kCvt = ROWS * 32 / kMlaThreads;   // 16-code pieces per thread
 #pragma unroll
-        for (int it = 0; it < kRowIters; it++) {
-            const int i = it * kTcThreads + tid;
-            const int g = i >> 5, t = i & 31;
-            const int j = (g & 7) * 8 + (t & 7);     // entry (row) of the chunk
-            const int k = (g >> 3) * 4 + (t >> 3);   // 16-byte piece of its codes (dims 16k .. 16k+15)
-            const int r = ridx[j];
-            v[it] = r >= 0 ? __ldg(reinterpret_cast<const uint4 *>(cache + static_cast<int64_t>(r) * kRowBytes) + k)
-                           : make_uint4(0u, 0u, 0u, 0u);
+        for (int it = 0; it < kCvt; it++) {
+            const int P = it * kMlaThreads + tid;
+            const int jl = P & 7, klo = (P >> 3) & 3, rest = P >> 5;
+            const int rg = rest % (ROWS / 8), k = (rest / (ROWS / 8)) * 4 + klo;
+            const int j = rg * 8 + jl;
+            uint4 w = make_uint4(0u, 0u, 0u, 0u);
+            if (ridx[j] >= 0) w = *reinterpret_cast<const uint4 *>(raw + j * kRowBytes + k * 16);
+            uint32_t o[8];
+            if (kFp8) {
+                fp8_to_f16x4(w.x, o[0], o[1]);
+                fp8_to_f16x4(w.y, o[2], o[3]);
+                fp8_to_f16x4(w.z, o[4], o[5]);
+                fp8_to_f16x4(w.w, o[6], o[7]);
+            } else {
+                codes_to_f16x4(w.x, o[0], o[1]);
+                codes_to_f16x4(w.y, o[2], o[3]);
+                codes_to_f16x4(w.z, o[4], o[5]);
+                codes_to_f16x4(w.w, o[6], o[7]);
+            }
+            unsigned char *line = Cs + rg * 8192 + (2 * k) * 128 + jl * 16;
+            *reinterpret_cast<uint4 *>(line) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4 *>(line + 128) = make_uint4(o[4], o[5], o[6], o[7]);
         }
-        float sc = 0.0f;
-        if (tid < kTcRows) {
-            const int r = ridx[tid];
-            if (r >= 0) sc = __ldg(reinterpret_cast<const float *>(cache + static_cast<int64_t>(r) * kRowBytes + kLatent));
-        }
-#pragma unroll
-        for (int it = 0; it < kRowIters; it++) {
-            const int i = it * kTcThreads + tid;
-            const int g = i >> 5, t = i & 31;
-            const int j = (g & 7) * 8 + (t & 7);
-            const int k = (g >> 3) * 4 + (t >> 3);
-            unsigned char *line = Cs + (j >> 3) * 8192 + (2 * k) * 128 + (j & 7) * 16;
-            auto cv = [&](uint32_t w, int shift) { return kFp8 ? fp8_to_bf16x2(w, shift) : codes_to_bf16x2(w, shift); };
-            *reinterpret_cast<uint4 *>(line) = make_uint4(cv(v[it].x, 0), cv(v[it].x, 16), cv(v[it].y, 0), cv(v[it].y, 16));
-            *reinterpret_cast<uint4 *>(line + 128) = make_uint4(cv(v[it].z, 0), cv(v[it].z, 16), cv(v[it].w, 0), cv(v[it].w, 16));
-        }
-        if (tid < kTcRows) scl[tid] = sc;
-        store_q();
     }
     tc::fence_proxy_async();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = *tmem_slot;
 
-    // 2. S = Q . C^T
+    GLM_TL(glm_tl_split, 4);
+    // 4. S^T = C . Q^T (M = ROWS rows, N = NH heads, K = 512)
     if (tid == 0) {
-        const uint32_t idesc = tc::idesc_bf16(M, kTcRows, false, false);
-        const uint32_t qa = tc::smem_addr(Qs), ca = tc::smem_addr(Cs);
+        const uint32_t idesc = tc::idesc_f16(ROWS, NH, false, false);
+        const uint32_t ca = tc::smem_addr(Cs), qa = tc::smem_addr(Qs);
 #pragma unroll 4
         for (int ks = 0; ks < kLatent / 16; ks++)
-            tc::mma_bf16(tmem, tc::desc(qa + ks * 256, 128, 8192), tc::desc(ca + ks * 256, 128, 8192), idesc,
+            tc::mma_bf16(tmem, tc::desc(ca + ks * 256, 128, 8192), tc::desc(qa + ks * 256, 128, 8192), idesc,
                          ks > 0 ? 1u : 0u);
-        tc::mma_commit(tc::smem_addr(&bar[0]));
+        tc::mma_commit(bar_s);
     }
-
-    // 3. softmax of the chunk on all 8 warps: warp w reads TMEM lane quadrant w % 4 (lane = head)
-    //    and the columns (entries) [32 (w / 4), +32); the two halves of a head exchange their
-    //    maxima and sums through shared memory
-    {
-        float *pmax = reinterpret_cast<float *>(smem + Lay::kPmax);
-        float *pl = reinterpret_cast<float *>(smem + Lay::kPl);
-        const int quad = warp & 3, hf = warp >> 2;
-        if (!tc::mbar_wait(tc::smem_addr(&bar[0]), 0, kWaitLimit)) atomicOr(status, 1);
-        __syncwarp();  // thread 0 arrives here after issuing the MMAs: reconverge for tcgen05.ld
-        tc::fence_after_sync();
-        uint32_t r[32];
-        tc::tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + hf * 32, r);
-        tc::tmem_wait_ld();
-        const int head = (M == 128) ? quad * 32 + lane : (lane < 16 ? quad * 16 + lane : -1);
-        const float k2 = sm_scale * 1.4426950408889634f;  // scores in log2 units
-        float sv[32];
-        float mx = -INFINITY;
-#pragma unroll
-        for (int jj = 0; jj < 32; jj++) {
-            const int j = hf * 32 + jj;
-            sv[jj] = ridx[j] >= 0 ? __uint_as_float(r[jj]) * scl[j] * k2 : -INFINITY;
-            mx = fmaxf(mx, sv[jj]);
-        }
-        if (head >= 0) pmax[hf * 128 + head] = mx;
+    ok = tc::mbar_wait(bar_s, 0, kMlaWaitLimit);
+    if (!__syncthreads_and(ok)) {
+        if (tid == 0) atomicOr(status, 1);
+        tc::mbar_wait(bar_s, 0, kMlaWaitLimit);
         __syncthreads();
-        if (head >= 0) {
-            mx = fmaxf(pmax[head], pmax[128 + head]);
-            float l = 0.0f;
-            const bool real = head < n_heads;
+        goto done;
+    }
+    tc::fence_after_sync();
+    GLM_TL(glm_tl_split, 5);
+
+    // 5. softmax: warp w reads TMEM lane quadrant w % 4 (one row per lane) and heads [V (w / 4), +V)
+    {
+        const int quad = warp & 3, hh = warp >> 2;
+        const int j = (ROWS == 128) ? quad * 32 + lane : (lane < 16 ? quad * 16 + lane : -1);
+        uint32_t r[V];
+        tmem_ld_v<V>(tmem + (static_cast<uint32_t>(quad * 32) << 16) + hh * V, r);
+        tc::tmem_wait_ld();
+        const bool rv = j >= 0 && ridx[j] >= 0;
+        const float sc = rv ? scl[j] : 0.0f;
+        float s[V], t[V];
 #pragma unroll
-            for (int rq = 0; rq < 4; rq++) {
-                const int rg = hf * 4 + rq;   // row group of 8 entries
-                uint32_t hi[4], lo[4];
+        for (int i = 0; i < V; i++) {
+            s[i] = rv ? __uint_as_float(r[i]) * sc * qk[hh * V + i] : -INFINITY;
+            t[i] = s[i];
+        }
+        constexpr int kLow = (V == 32) ? 0 : (V == 16) ? 1 : 3;   // lane bits that repeat a head index
+        constexpr int kShift = (V == 32) ? 0 : (V == 16) ? 1 : 2;
+        float bm = butterfly<V, true>(t);
+        if ((lane & kLow) == 0) red[quad * NH + hh * V + ((lane >> kShift) & (V - 1))] = bm;
+        __syncthreads();
+        const float smax = __uint_as_float(words[0]);
+        const float ratio = rv ? __fdiv_rn(sc, smax) : 0.0f;   // scale_row / scale_max, in (0, 1]
+#pragma unroll
+        for (int i = 0; i < V; i++) {
+            const int h = hh * V + i;
+            const float m = fmaxf(fmaxf(red[h], red[NH + h]), fmaxf(red[2 * NH + h], red[3 * NH + h]));
+            const float p = (rv && m != -INFINITY) ? exp2f(s[i] - m) : 0.0f;
+            s[i] = p;
+            t[i] = p;
+        }
+        float bl = butterfly<V, false>(t);
+        if ((lane & kLow) == 0) red2[quad * NH + hh * V + ((lane >> kShift) & (V - 1))] = bl;
+        if (j >= 0) {   // P' of this row as fp16 hi + lo, 8 heads per 16-byte line
+#pragma unroll
+            for (int g = 0; g < V / 8; g++) {
+                uint32_t hi4[4], lo4[4];
 #pragma unroll
                 for (int e = 0; e < 4; e++) {
-                    uint32_t hb[2], lb[2];
-#pragma unroll
-                    for (int u = 0; u < 2; u++) {
-                        const int jj = rq * 8 + 2 * e + u, j = hf * 32 + jj;
-                        const float p = ridx[j] >= 0 ? exp2f(sv[jj] - mx) : 0.0f;
-                        l += p;
-                        const float pp = real ? p * scl[j] : 0.0f;
-                        const uint16_t h16 = bf16_rn_bits(pp);
-                        hb[u] = h16;
-                        lb[u] = bf16_rn_bits(pp - __uint_as_float(static_cast<uint32_t>(h16) << 16));
-                    }
-                    hi[e] = hb[0] | (hb[1] << 16);
-                    lo[e] = lb[0] | (lb[1] << 16);
+                    const float a = s[8 * g + 2 * e] * ratio, b = s[8 * g + 2 * e + 1] * ratio;
+                    hi4[e] = f16x2_rn(a, b);
+                    lo4[e] = f16x2_rn(a - f16_lo_f(hi4[e]), b - f16_hi_f(hi4[e]));
                 }
-                const int off = (head >> 3) * 1024 + rg * 128 + (head & 7) * 16;
-                *reinterpret_cast<uint4 *>(Phi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4 *>(Plo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                const int G = hh * (V / 8) + g;
+                unsigned char *line = Ps + (j >> 3) * kLboP + G * 128 + (j & 7) * 16;
+                *reinterpret_cast<uint4 *>(line) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+                *reinterpret_cast<uint4 *>(line + (NH / 8) * 128) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
             }
-            pl[hf * 128 + head] = l;
-            pmax[hf * 128 + head] = mx;   // (same value in both halves)
         }
         tc::fence_before_sync();
     }
     tc::fence_proxy_async();
     __syncthreads();
-    if (warp < 4) {   // (m, l) of each head, natural-log units
-        const float *pmax = reinterpret_cast<const float *>(smem + Lay::kPmax);
-        const float *pl = reinterpret_cast<const float *>(smem + Lay::kPl);
-        const int head = (M == 128) ? warp * 32 + lane : (lane < 16 ? warp * 16 + lane : -1);
-        if (head >= 0 && head < n_heads) {
-            part_ml[2 * (ml_base + head)] = pmax[head] * 0.6931471805599453f;
-            part_ml[2 * (ml_base + head) + 1] = pl[head] + pl[128 + head];
-        }
+    if (tid < nh_real) {   // (m, l) of each head, natural-log units
+        const float m = fmaxf(fmaxf(red[tid], red[NH + tid]), fmaxf(red[2 * NH + tid], red[3 * NH + tid]));
+        const float l = (red2[tid] + red2[NH + tid]) + (red2[2 * NH + tid] + red2[3 * NH + tid]);
+        part_ml[2 * (ml_base + tid)] = m * 0.6931471805599453f;
+        part_ml[2 * (ml_base + tid) + 1] = l;
     }
 
-    // 4. O^T = C^T . P'^T (hi and lo terms accumulate into the same columns)
+    GLM_TL(glm_tl_split, 6);
+    // 6. O^T = C^T . P'^T (hi and lo heads side by side: N = 2 NH)
     if (tid == 0) {
         tc::fence_after_sync();
-        const uint32_t idesc = tc::idesc_bf16(128, M, true, false);
-        const uint32_t ph = tc::smem_addr(Phi), pl = tc::smem_addr(Plo), ca = tc::smem_addr(Cs);
+        const uint32_t idesc = tc::idesc_f16(128, 2 * NH, true, true);
+        const uint32_t pa = tc::smem_addr(Ps), ca = tc::smem_addr(Cs);
 #pragma unroll
-        for (int mt = 0; mt < kLatent / 128; mt++) {
+        for (int ks = 0; ks < ROWS / 16; ks++) {
 #pragma unroll
-            for (int ks = 0; ks < kTcRows / 16; ks++) {
-                const uint64_t a = tc::desc(ca + ks * 2 * 8192 + mt * 16 * 128, 8192, 128);
-                tc::mma_bf16(tmem + mt * M, a, tc::desc(ph + ks * 256, 128, 1024), idesc, ks > 0 ? 1u : 0u);
-                tc::mma_bf16(tmem + mt * M, a, tc::desc(pl + ks * 256, 128, 1024), idesc, 1u);
-            }
+            for (int mt = 0; mt < kLatent / 128; mt++)
+                tc::mma_bf16(tmem + mt * 2 * NH, tc::desc(ca + ks * 2 * 8192 + mt * 16 * 128, 8192, 128),
+                             tc::desc(pa + ks * 2 * kLboP, kLboP, 128), idesc, ks > 0 ? 1u : 0u);
         }
-        tc::mma_commit(tc::smem_addr(&bar[1]));
+        tc::mma_commit(bar_o);
     }
+    ok = tc::mbar_wait(bar_o, 0, kMlaWaitLimit);
+    if (!__syncthreads_and(ok)) {
+        if (tid == 0) atomicOr(status, 2);
+        tc::mbar_wait(bar_o, 0, kMlaWaitLimit);
+        __syncthreads();
+        goto done;
+    }
+    tc::fence_after_sync();
+    GLM_TL(glm_tl_split, 7);
 
-    // 5. unnormalised O to the workspace: tile mt, lane quadrant q (latent dims 128 mt + 32 q + lane)
+    // 7. acc = scale_max (O_hi + O_lo): tile mt, lane quadrant q (latent dims 128 mt + 32 q + lane)
     {
-        if (!tc::mbar_wait(tc::smem_addr(&bar[1]), 0, kWaitLimit)) atomicOr(status, 2);
-        __syncwarp();
-        tc::fence_after_sync();
         const int quad = warp & 3;
+        const float smax = __uint_as_float(words[0]);
 #pragma unroll 1
         for (int mt = warp >> 2; mt < kLatent / 128; mt += 2) {
             const int dim = mt * 128 + quad * 32 + lane;
-            const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + mt * M;
+            const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + mt * 2 * NH;
 #pragma unroll 1
-            for (int hb = 0; hb < M; hb += 32) {
-                uint32_t r[32];
-                tc::tmem_ld32(ta + hb, r);
+            for (int hb = 0; hb < NH; hb += 16) {
+                uint32_t hi[16], lo[16];
+                tc::tmem_ld16(ta + hb, hi);
+                tc::tmem_ld16(ta + NH + hb, lo);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; e++)
-                    if (hb + e < n_heads) part_acc[(ml_base + hb + e) * kLatent + dim] = __uint_as_float(r[e]);
+                for (int e = 0; e < 16; e++)
+                    if (hb + e < nh_real)
+                        part_acc[(ml_base + hb + e) * kLatent + dim] =
+                            smax * (__uint_as_float(hi[e]) + __uint_as_float(lo[e]));
             }
         }
     }
+done:
     tc::fence_before_sync();
     __syncthreads();
+    GLM_TL(glm_tl_split, 8);
     if (warp == 0) {
         tc::fence_after_sync();
-        tc::tmem_dealloc(tmem, 512);
+        tc::tmem_dealloc(tmem, 8 * NH);
     }
 }
 
-int mla_tc_chunk() { return kTcRows; }
+int mla_tc_chunk() { return 64; }
 
-template <int M, bool kFp8>
-cudaError_t launch_mla_split_tc_t(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
-                                  const int32_t *rows, int n_q, int width, float sm_scale,
-                                  float *part_acc, float *part_ml, int *status, cudaStream_t stream, bool early_q) {
-    const int n_chunks = (width + kTcRows - 1) / kTcRows;
-    const int smem = TcLayout<M>::kBytes;
-    cudaError_t e = cudaFuncSetAttribute(mla_split_tc_kernel<M, kFp8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+MlaPlan mla_plan(int n_q, int n_heads, int width, int num_sms) {
+    // 128-row chunks of 16 heads while they fill the SMs about twice; otherwise 64-row chunks of
+    // 64 heads (no head group gathers a row another group of its chunk gathers again)
+    MlaPlan p{};
+    const long long ctas128 = static_cast<long long>(n_q) * ((width + 127) / 128) * ((n_heads + 15) / 16);
+    if (ctas128 <= 2ll * num_sms) {
+        p.rows = 128;
+        p.heads = 16;
+    } else {
+        p.rows = 64;
+        p.heads = 64;
+    }
+    p.n_chunks = (width + p.rows - 1) / p.rows;
+    p.n_hg = (n_heads + p.heads - 1) / p.heads;
+    return p;
+}
+
+template <int ROWS, int NH, bool kFp8>
+cudaError_t launch_t(const MlaPlan &p, const void *q, int n_heads, const uint8_t *cache, int64_t n_rows,
+                     const int32_t *rows, int n_q, int width, float sm_scale, float *part_acc, float *part_ml,
+                     int *status, cudaStream_t stream, bool early_q) {
+    auto kernel = mla_split_tc_kernel<ROWS, NH, kFp8>;
+    const int smem = MlaLayout<ROWS, NH>::kBytes;
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(mla_split_tc_kernel<M, kFp8>, dim3(n_chunks, n_q), dim3(kTcThreads), smem, stream,
-                   static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, n_chunks,
-                   part_acc, part_ml, status, early_q ? 1 : 0);
+    e = launch_pdl(kernel, dim3(p.n_chunks * p.n_hg, n_q), dim3(kMlaThreads), smem, stream,
+                   static_cast<const uint16_t *>(q), n_heads, cache, n_rows, rows, width, sm_scale, p.n_chunks,
+                   p.n_hg, part_acc, part_ml, status, early_q ? 1 : 0);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
-cudaError_t launch_mla_split_tc(const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
+cudaError_t launch_mla_split_tc(const MlaPlan &p, const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
                                 const int32_t *rows, int n_q, int width, float sm_scale,
                                 float *part_acc, float *part_ml, int *status, cudaStream_t stream, bool early_q,
                                 bool fp8) {
-    if (n_heads <= 64)
-        return fp8 ? launch_mla_split_tc_t<64, true>(q, n_heads, cache, n_rows, rows, n_q, width, sm_scale, part_acc,
-                                                     part_ml, status, stream, early_q)
-                   : launch_mla_split_tc_t<64, false>(q, n_heads, cache, n_rows, rows, n_q, width, sm_scale, part_acc,
-                                                      part_ml, status, stream, early_q);
-    return fp8 ? launch_mla_split_tc_t<128, true>(q, n_heads, cache, n_rows, rows, n_q, width, sm_scale, part_acc,
-                                                  part_ml, status, stream, early_q)
-               : launch_mla_split_tc_t<128, false>(q, n_heads, cache, n_rows, rows, n_q, width, sm_scale, part_acc,
-                                                   part_ml, status, stream, early_q);
+    const uint8_t *c8 = reinterpret_cast<const uint8_t *>(cache);
+#define GLM_MLA_LAUNCH(R, H)                                                                                       \
+    if (p.rows == R && p.heads == H)                                                                             \
+        return fp8 ? launch_t<R, H, true>(p, q, n_heads, c8, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml, \
+                                          status, stream, early_q)                                               \
+                   : launch_t<R, H, false>(p, q, n_heads, c8, n_rows, rows, n_q, width, sm_scale, part_acc,         \
+                                           part_ml, status, stream, early_q);
+    GLM_MLA_LAUNCH(128, 16)
+    GLM_MLA_LAUNCH(64, 16)
+    GLM_MLA_LAUNCH(64, 32)
+    GLM_MLA_LAUNCH(64, 64)
+#undef GLM_MLA_LAUNCH
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace glm

@@ -8,12 +8,17 @@
 
 namespace glm {
 
+GLM_TL_TABLE(glm_tl_prep)
+
 constexpr int kPrepThreads = 256;
 constexpr int kPrepWarps = kPrepThreads / 32;
 constexpr int kZeroPerThread = 4;   // 16-byte stores per thread of a zeroing CTA
 
 __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(StepPrepArgs a, int store_ctas, int pool_ctas) {
+    GLM_TL(glm_tl_prep, 0);
+    GLM_TL_SMID(glm_tl_prep);
     pdl_begin();
+    GLM_TL(glm_tl_prep, 1);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     int cta = blockIdx.x;
     if (cta < store_ctas) {

@@ -168,6 +168,34 @@ def test_fp8_entry_points_reject_before_launch():
                                        1 << 30, None) == kp.GLM_ERR_INVALID_ARG
 
 
+def test_noalloc_entry_rejects_before_launch():
+    # the allocation-free MLA entry point runs the workspace entry's checks: every rejection below
+    # happens on the host, before its scratch is looked up or anything is enqueued
+    L = kp.lib
+    d = C.byref(kp.make_dims(64))
+    bad = C.byref(kp.make_dims(64, qk_rope_head_dim=64))
+    assert L.glm_sparse_mla_decode_noalloc(bad, FAKE, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None,
+                                           None) == kp.GLM_ERR_UNSUPPORTED
+    assert L.glm_sparse_mla_decode_noalloc(d, FAKE, FAKE, 10, FAKE, 1, 0, 0.04, FAKE, None, None,
+                                           None) == kp.GLM_ERR_INVALID_ARG        # width 0
+    assert L.glm_sparse_mla_decode_noalloc(d, FAKE, FAKE, 10, FAKE, -1, 64, 0.04, FAKE, None, None,
+                                           None) == kp.GLM_ERR_INVALID_ARG        # n_q < 0
+    assert L.glm_sparse_mla_decode_noalloc(d, None, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None,
+                                           None) == kp.GLM_ERR_INVALID_ARG        # null q
+    assert L.glm_sparse_mla_decode_noalloc(d, FAKE, FAKE, 10, None, 1, 64, 0.04, FAKE, None, None,
+                                           None) == kp.GLM_ERR_INVALID_ARG        # null rows
+    assert L.glm_sparse_mla_decode_noalloc(d, MIS, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None,
+                                           None) == kp.GLM_ERR_INVALID_ARG        # misaligned q
+    assert L.glm_sparse_mla_decode_noalloc(d, FAKE, FAKE, 10, FAKE, 1, 64, C.c_float(float("nan")), FAKE,
+                                           None, None, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_sparse_mla_decode_noalloc(d, None, None, 0, None, 0, 64, 0.04, None, None, None,
+                                           None) == kp.GLM_OK                     # n_q == 0: no-op
+    # more partials than the scratch holds: refused before any CUDA call
+    d128 = C.byref(kp.make_dims(128))
+    assert L.glm_sparse_mla_decode_noalloc(d128, FAKE, FAKE, 10, FAKE, 8, 65536, 0.04, FAKE, None, None,
+                                           None) == kp.GLM_ERR_WORKSPACE
+
+
 def test_algorithmic_bytes_of_the_tiny_decode():
     # by hand: 128 visible pools x 512 B + q_idx 8,192 B + w 128 B + 16 top-k ids x 4 B; 64 gathered
     # rows x 528 B + q and out 2 x 16 heads x 1,024 B + 80 indices x 4 B; one new row (1,024 B in,
