@@ -24,7 +24,6 @@ import hashlib
 import json
 import os
 import re
-import subprocess
 import sys
 import threading
 import time
@@ -36,10 +35,10 @@ sys.path.insert(0, ROOT)
 
 import synth  # noqa: E402
 
-def kernel_launches_per_step(wl, num_sms: int) -> int:
-    """Kernels of one glm_dsa_decode_step: store + pool build + zeroing of the selection words,
-    scores + top-k + expansion, MLA split, MLA combine."""
-    return 4
+# Kernels of one glm_dsa_decode_step: store + pool build + zeroing of the selection words, scores +
+# top-k + expansion, MLA split, MLA combine.
+KERNELS_PER_STEP = 4
+STEP_KERNELS = ("step_prep", "index_select_tc", "mla_split_tc", "mla_combine")
 
 
 def algorithmic_bytes(inp, key_bytes: int = 512) -> dict:
@@ -360,32 +359,35 @@ def run_kernels(args, wl):
     ms_per_step = ms / args.steps
     value = whole_job_throughput(wl.n_queries, args.steps, world, ms)
 
-    # per-stage device time (same kernels, same buffers, direct launches queued behind a sleep so
-    # the host never starves the GPU; events on the launching stream). "index_scores" is the
-    # same index kernel with the selection switched off (scores only), timed for comparison.
-    stage_names = [nm for nm, _ in P.STAGES] + ["index_scores"]
+    # per-kernel cost inside the step: the same graphs of R steps cut after the step's first k
+    # kernels (glm_dsa_decode_step's stop_after = k), timed the same way; kernel k's cost is the
+    # difference of consecutive prefixes, so the costs add up to the whole step
+    def time_graph(fn, reps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            for b in bufs:
+                fn(b)
+            stream.synchronize()
+            with torch.cuda.graph(g, stream=stream):
+                for b in bufs:
+                    fn(b)
+            for _ in range(max(3, args.warmup // R + 1)):
+                g.replay()
+            a0 = torch.cuda.Event(enable_timing=True)
+            a1 = torch.cuda.Event(enable_timing=True)
+            a0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            a1.record(stream)
+        stream.synchronize()
+        t = a0.elapsed_time(a1) / (reps * R)
+        del g
+        return t
 
-    def stage_calls(b):
-        nq, ld = b.q_idx.shape[0], b.pooled.shape[1]
-        scratch = b.ws_index.view(torch.float32)[:nq * ld].view(nq, ld)
-        return [lambda fn=fn: fn(b) for _, fn in P.STAGES] + [
-            lambda: kp.glm_index_scores(b.dims, b.q_idx, b.w, b.pooled, b.q_seq, b.q_pos, b.pad,
-                                        b.len, scratch)]
-
-    n_stage_steps = max(1, min(args.steps, 200))
-    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in stage_names] for _ in range(n_stage_steps)]
-    with torch.cuda.stream(stream):
-        calls = [stage_calls(b) for b in bufs]
-        torch.cuda._sleep(int(1.5e6 * n_stage_steps))      # ~0.75 ms of GPU time per step queued
-        for i in range(n_stage_steps):
-            for j, c in enumerate(calls[i % R]):
-                ev[i][j][0].record(stream)
-                c()
-                ev[i][j][1].record(stream)
-    stream.synchronize()
-    stage_ms = {nm: float(np.mean([ev[i][j][0].elapsed_time(ev[i][j][1]) for i in range(n_stage_steps)]))
-                for j, nm in enumerate(stage_names)}
+    reps = max(2, args.steps // R)
+    prefix_ms = [time_graph(lambda b, k=k: P.run_step(b, stop_after=k), reps) for k in (1, 2, 3)]
+    prefix_ms.append(time_graph(P.run_step, reps))
+    kernel_ms = [prefix_ms[0]] + [prefix_ms[i] - prefix_ms[i - 1] for i in range(1, 4)]
 
     # the dominant kernel on its own: back-to-back launches of the fused scores + top-k + expansion
     # entry over the rotating states (queued behind a sleep, events on the launching stream); each
@@ -402,48 +404,73 @@ def run_kernels(args, wl):
     stream.synchronize()
     idx_launch_ms = i0.elapsed_time(i1) / n_idx
 
-    # end to end through the public API with host buffers: per step the new token's latent, its
-    # k/gate rows, q_idx, w, q (and positions) go host->device from pinned memory, the step runs
-    # through the C-ABI calls, and the output comes back device->host
-    b = bufs[0]
-    inp0 = inps[0]
-    pin = lambda a: a.pin_memory()  # noqa: E731
-    h_lat = pin(b.new_latent.cpu())
-    h_slots = pin(b.new_slots.cpu())
-    h_qidx, h_w, h_q = pin(b.q_idx.cpu()), pin(b.w.cpu()), pin(b.q.cpu())
-    h_qpos, h_qseq, h_pb = pin(b.q_pos.cpu()), pin(b.q_seq.cpu()), pin(b.pool_begin.cpu())
-    kg_ranges = []
-    for sq in sorted(set(int(v) for v in inp0.q_seq)):
-        pos = inp0.q_pos[inp0.q_seq == sq]
-        kg_ranges.append((sq, int(pos.min()), int(pos.max()) + 1))
-    h_k = [pin(b.k[sq, lo:hi].cpu()) for sq, lo, hi in kg_ranges]
-    h_g = [pin(b.gate[sq, lo:hi].cpu()) for sq, lo, hi in kg_ranges]
-    h_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (h_lat, h_slots, h_qidx, h_w, h_q, h_qpos, h_qseq, h_pb, *h_k, *h_g))
-    d2h = h_out.numel() * h_out.element_size()
-    n_e2e = max(1, min(args.steps, 200))
+    # end to end through the public API with host buffers: per step, one host->device copy of the
+    # step's packed inputs (new latent rows and slots, q_idx, w, q, positions, pool begins) from
+    # pinned memory, the new tokens' k and gate rows (one copy each per sequence), the one-call
+    # step, and the output copied back device->host, then a synchronisation. Each state's copies
+    # and step are captured as one CUDA graph, replayed in turn (the states rotate as above).
+    import dataclasses
+    e2e_fields = ("new_latent", "new_slots", "q_idx", "w", "q", "q_pos", "q_seq", "pool_begin")
+    e2e = []
+    for r, b in enumerate(bufs):
+        srcs = [getattr(b, f) for f in e2e_fields]
+        offs, total = [], 0
+        for t in srcs:
+            offs.append(total)
+            total += (t.numel() * t.element_size() + 15) // 16 * 16
+        d_pack = torch.empty(total, dtype=torch.uint8, device=dev)
+        h_pack = torch.empty(total, dtype=torch.uint8).pin_memory()
+        views = {}
+        for f, t, o in zip(e2e_fields, srcs, offs):
+            nb = t.numel() * t.element_size()
+            views[f] = d_pack[o:o + nb].view(t.dtype).view(t.shape)
+            h_pack[o:o + nb].copy_(t.reshape(-1).view(torch.uint8).cpu())
+        b2 = dataclasses.replace(b, **views)
+        q_seq_h, q_pos_h = b.q_seq.cpu().numpy(), b.q_pos.cpu().numpy()
+        kg = []
+        for sq in sorted(set(int(v) for v in q_seq_h)):
+            pos = q_pos_h[q_seq_h == sq]
+            lo_t, hi_t = int(pos.min()), int(pos.max()) + 1
+            kg.append((b.k[sq, lo_t:hi_t], b.k[sq, lo_t:hi_t].cpu().pin_memory(),
+                       b.gate[sq, lo_t:hi_t], b.gate[sq, lo_t:hi_t].cpu().pin_memory()))
+        h_out = torch.empty(b.out.shape, dtype=b.out.dtype).pin_memory()
+        e2e.append((b2, d_pack, h_pack, kg, h_out))
+    h2d = e2e[0][1].numel() + sum(hk.numel() * hk.element_size() + hg.numel() * hg.element_size()
+                                  for _, hk, _, hg in e2e[0][3])
+    d2h = e2e[0][4].numel() * e2e[0][4].element_size()
+
+    def e2e_step(item):
+        b2, d_pack, h_pack, kg, h_out = item
+        d_pack.copy_(h_pack, non_blocking=True)
+        for dk, hk, dg, hg in kg:
+            dk.copy_(hk, non_blocking=True)
+            dg.copy_(hg, non_blocking=True)
+        P.run_step(b2)
+        h_out.copy_(b2.out, non_blocking=True)
+
+    e2e_graphs = []
     with torch.cuda.stream(stream):
-        for _ in range(2):
-            P.run_step(b)
+        for item in e2e:
+            e2e_step(item)
         stream.synchronize()
+        for item in e2e:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                e2e_step(item)
+            e2e_graphs.append(g)
+        for g in e2e_graphs:
+            g.replay()
+        stream.synchronize()
+    n_e2e = max(R, min(args.steps, 400))
+    with torch.cuda.stream(stream):              # replays go to the stream the graphs were captured on
         t0 = time.perf_counter()
-        for _ in range(n_e2e):
-            b.new_latent.copy_(h_lat, non_blocking=True)
-            b.new_slots.copy_(h_slots, non_blocking=True)
-            b.q_idx.copy_(h_qidx, non_blocking=True)
-            b.w.copy_(h_w, non_blocking=True)
-            b.q.copy_(h_q, non_blocking=True)
-            b.q_pos.copy_(h_qpos, non_blocking=True)
-            b.q_seq.copy_(h_qseq, non_blocking=True)
-            b.pool_begin.copy_(h_pb, non_blocking=True)
-            for i, (sq, lo, hi) in enumerate(kg_ranges):
-                b.k[sq, lo:hi].copy_(h_k[i], non_blocking=True)
-                b.gate[sq, lo:hi].copy_(h_g[i], non_blocking=True)
-            P.run_step(b)
-            h_out.copy_(b.out, non_blocking=True)
+        for i in range(n_e2e):
+            e2e_graphs[i % R].replay()
             stream.synchronize()
         e2e_s = time.perf_counter() - t0
+    assert torch.equal(e2e[(n_e2e - 1) % R][4], e2e[(n_e2e - 1) % R][0].out.cpu())   # the copy is the output
     e2e_qps = whole_job_throughput(wl.n_queries, n_e2e, world, reduce_max(e2e_s * 1e3, world, dev))
+    del e2e_graphs
 
     peak, peak_kind = measured_peaks()
     # dominant kernel: the fused scores + selection + expansion launch (each timed launch also
@@ -460,15 +487,20 @@ def run_kernels(args, wl):
         "achieved_hbm_gbs_per_gpu": ab["total"] / (ms_per_step / 1e3) / 1e9,
         "algorithmic_bytes_per_step": ab["total"],
         "tokens_gathered_per_s": ab["gathered"] * args.steps * world / (ms / 1e3),
-        "stage_us": {k: v * 1e3 for k, v in stage_ms.items()},
+        "kernel_us_in_step": {nm: v * 1e3 for nm, v in zip(STEP_KERNELS, kernel_ms)},
+        "kernel_us_method": "step prefixes (stop_after = 1, 2, 3, whole) as graphs of the rotating states; "
+                            "each kernel = difference of consecutive prefixes; their sum is the whole step "
+                            f"timed the same way ({prefix_ms[3] * 1e3:.2f} us)",
         "roofline": {"kernel": "index_select_tc (scores + top-k + expansion)", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
                      "traffic": traffic, "algorithmic_bytes_per_launch": ab["index"],
                      "launch_us": idx_ms * 1e3},
         "e2e": {"value": e2e_qps, "unit": "queries/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
-                "api": "C ABI via kpool_indexer_int8_b200 binding, host pinned buffers, sync per step"},
-        "gpu_launches": kernel_launches_per_step(wl, torch.cuda.get_device_properties(dev).multi_processor_count) * args.steps,
+                "api": "glm_dsa_decode_step through the binding with its host copies (pinned, one packed "
+                       "H2D of the step inputs + the new k/gate rows, one D2H of out) captured per state "
+                       "as a CUDA graph, replayed per step with a host synchronisation per step"},
+        "gpu_launches": KERNELS_PER_STEP * args.steps,
         "clocks": sampler.summary(),
     }
     line["achieved_hbm_frac_per_gpu"] = line["achieved_hbm_gbs_per_gpu"] / peak

@@ -327,6 +327,42 @@ int glm_sparse_mla_decode_noalloc(const glm_dsa_dims *dims, const void *q_dev,
                                   float *lse_dev, float *out_f32_dev, void *stream);
 
 /* ------------------------------------------------------------------------------------------ */
+/* up-projection of the attention output                                                       */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * "Module glm5next_dsa_ref", expand_kv (kv_b_proj maps the 512-d latent to per-head K and V) and
+ * "GLM-5.3-Flash" pypto-lib page, 'Checkpoint shape' (qk_head_dim / v_head_dim 256) and 'Open
+ * questions an owner will hit' (kv_b_proj is BF16): the latent-space attention output of each head
+ * taken to that head's value space,
+ *     out_v[n][h][e] = sum_d o_lat[n][h][d] * W[h (dk + dv) + dk + e][d],   e < dv, d < 512,
+ * which with the absorbed query (q_lat[h] = W_K,h^T q_h) equals attention over the expanded K and V.
+ *   o_lat_dev    bf16 [n_q, n_heads, 512]   (the out_dev of glm_sparse_mla_decode)
+ *   w_kv_b_dev   bf16 [n_heads * (dk + dv), 512], torch Linear layout: per head dk K rows, then dv V rows
+ *   out_v_dev    bf16 [n_q, n_heads, dv]    out_v_f32_dev fp32 [n_q, n_heads, dv] or NULL
+ * dk = qk_nope_head_dim >= 0, dv = v_head_dim a multiple of 128 (<= 4096). Pointers 16-byte aligned.
+ * Tensor cores (bf16 operands, fp32 accumulation); W is read once per 128 queries. If a bounded wait
+ * gives up, the affected outputs are NaN. Returns GLM_OK, GLM_ERR_INVALID_ARG / _UNSUPPORTED (before
+ * anything is enqueued) or GLM_ERR_CUDA.
+ */
+int glm_mla_v_up(const glm_dsa_dims *dims, const void *o_lat_dev, const void *w_kv_b_dev,
+                 int32_t qk_nope_head_dim, int32_t v_head_dim, int32_t n_q, void *out_v_dev,
+                 float *out_v_f32_dev, void *stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* testing                                                                                    */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * The number of polls after which a wait of the fused index kernel's CTAs on one another (the
+ * sample meeting, the candidate meeting) gives up, on the current device: GLM_CROSS_CTA_WAIT_LIMIT
+ * by default. A test lowers it (0: every such wait gives up at once) to check the give-up path
+ * without a fault: the kernel sets bit 8 of the status word, leaves its selection outputs
+ * unwritten and returns; restore the default afterwards. Not for use while kernels of the
+ * library run on the device. Returns GLM_OK or GLM_ERR_CUDA.
+ */
+#define GLM_CROSS_CTA_WAIT_LIMIT (1u << 21)
+int glm_debug_set_cross_cta_wait_limit(uint32_t polls);
+
+/* ------------------------------------------------------------------------------------------ */
 /* the whole decode step in one call                                                           */
 /* ------------------------------------------------------------------------------------------ */
 /*
@@ -383,6 +419,10 @@ typedef struct glm_dsa_step {
     /* nonzero: cache_dev holds FP8 rows (uint8 [n_rows, 528]); the store and the attention are
      * glm_kv_store_fp8 and glm_sparse_mla_decode_fp8 */
     int32_t cache_fp8;
+    /* 0: the whole step. k = 1, 2, 3: only the step's first k kernels (1: store, pool build and
+     * counter zeroing; 2: + scoring, selection and expansion; 3: + the attention's split), for
+     * timing a prefix of the step; the outputs of the later kernels are then not written. */
+    int32_t stop_after;
 } glm_dsa_step;
 
 /*

@@ -38,7 +38,8 @@ EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv
            "glm_index_topk_expand", "glm_index_topk_expand_q8",
            "glm_dsa_decode_step",
            "glm_topk_pools", "glm_expand_selection",
-           "glm_sparse_mla_decode", "glm_dsa_workspace_size", "glm_kv_store_fp8", "glm_sparse_mla_decode_fp8")
+           "glm_sparse_mla_decode", "glm_dsa_workspace_size", "glm_kv_store_fp8", "glm_sparse_mla_decode_fp8",
+           "glm_debug_set_cross_cta_wait_limit", "glm_mla_v_up")
 
 
 class glm_dsa_dims(C.Structure):
@@ -66,7 +67,8 @@ class glm_dsa_step(C.Structure):
                 ("tok_dev", C.c_void_p), ("rows_dev", C.c_void_p),
                 ("q_dev", C.c_void_p), ("sm_scale", C.c_float), ("out_dev", C.c_void_p),
                 ("lse_dev", C.c_void_p), ("out_f32_dev", C.c_void_p),
-                ("pooled_codes_dev", C.c_void_p), ("pooled_scales_dev", C.c_void_p), ("cache_fp8", C.c_int32)]
+                ("pooled_codes_dev", C.c_void_p), ("pooled_scales_dev", C.c_void_p), ("cache_fp8", C.c_int32),
+                ("stop_after", C.c_int32)]
 
 
 def make_dims(n_heads: int, kv_lora_rank: int = 512, qk_rope_head_dim: int = 0,
@@ -294,11 +296,12 @@ def glm_index_topk_expand(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, sel
 def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_eps, pad, length, pool_begin,
                         max_new_pools, pooled, q_idx, w, q_seq, q_pos, select_k, out_width, slot_map, rows,
                         topk, q, sm_scale, out, workspace, n_sel=None, tok=None, scores=None, lse=None,
-                        out_f32=None, pooled_codes=None, pooled_scales=None, cache_fp8=False, stream=None) -> None:
+                        out_f32=None, pooled_codes=None, pooled_scales=None, cache_fp8=False, stop_after=0,
+                        stream=None) -> None:
     """The whole step in one call: the arguments of glm_kv_store_int8, glm_kpool_build,
     glm_index_topk_expand and glm_sparse_mla_decode (same tensors and rules); with cache_fp8 the
     cache holds FP8 rows (uint8) and the step stores and attends as glm_kv_store_fp8 and
-    glm_sparse_mla_decode_fp8."""
+    glm_sparse_mla_decode_fp8. stop_after = k (1..3) runs only the step's first k kernels."""
     for t, dt, nm in ((latent, torch.bfloat16, "latent"), (slots, torch.int64, "slots"),
                       (cache, torch.uint8 if cache_fp8 else torch.int8, "cache"),
                       (k, torch.bfloat16, "k"), (gate, torch.bfloat16, "gate"), (ln_w, torch.float32, "ln_w"),
@@ -329,6 +332,7 @@ def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_e
     a.lse_dev, a.out_f32_dev = v(lse), v(out_f32)
     a.pooled_codes_dev, a.pooled_scales_dev = v(pooled_codes), v(pooled_scales)
     a.cache_fp8 = 1 if cache_fp8 else 0
+    a.stop_after = int(stop_after)
     ws_bytes = 0 if workspace is None else workspace.numel()
     _check(lib.glm_dsa_decode_step(C.byref(dims), C.byref(a), _ptr(workspace), ws_bytes, _stream(stream)),
            "glm_dsa_decode_step")
@@ -427,3 +431,29 @@ def glm_sparse_mla_decode_noalloc(dims, q, cache, rows, sm_scale, out, lse=None,
                                              rows.shape[0], rows.shape[1], float(sm_scale), _ptr(out),
                                              _ptr(lse), _ptr(out_f32), _stream(stream)),
            "glm_sparse_mla_decode_noalloc")
+
+
+lib.glm_debug_set_cross_cta_wait_limit.argtypes = [C.c_uint32]
+lib.glm_debug_set_cross_cta_wait_limit.restype = C.c_int
+GLM_CROSS_CTA_WAIT_LIMIT = 1 << 21
+
+
+def glm_debug_set_cross_cta_wait_limit(polls: int) -> None:
+    """Polls before a wait of the fused index kernel's CTAs on one another gives up (tests only;
+    GLM_CROSS_CTA_WAIT_LIMIT restores the default)."""
+    _check(lib.glm_debug_set_cross_cta_wait_limit(int(polls)), "glm_debug_set_cross_cta_wait_limit")
+
+
+lib.glm_mla_v_up.argtypes = [_D, _P, _P, _I32, _I32, _I32, _P, _P, _P]
+lib.glm_mla_v_up.restype = C.c_int
+
+
+def glm_mla_v_up(dims, o_lat, w_kv_b, qk_nope_head_dim, v_head_dim, out_v, out_v_f32=None, stream=None) -> None:
+    """Up-projection of the latent attention output: o_lat bf16 [n_q, n_heads, 512], w_kv_b bf16
+    [n_heads * (dk + dv), 512] -> out_v bf16 [n_q, n_heads, dv] (and fp32 if out_v_f32 is given)."""
+    for t, dt, nm in ((o_lat, torch.bfloat16, "o_lat"), (w_kv_b, torch.bfloat16, "w_kv_b"),
+                      (out_v, torch.bfloat16, "out_v"), (out_v_f32, torch.float32, "out_v_f32")):
+        _dev(t, dt, nm)
+    n_q = o_lat.shape[0]
+    _check(lib.glm_mla_v_up(C.byref(dims), _ptr(o_lat), _ptr(w_kv_b), int(qk_nope_head_dim), int(v_head_dim), n_q,
+                            _ptr(out_v), _ptr(out_v_f32), _stream(stream)), "glm_mla_v_up")

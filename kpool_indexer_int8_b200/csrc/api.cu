@@ -182,6 +182,10 @@ const char *glm_status_string(int s) {
 
 int glm_last_cuda_error(void) { return g_last_cuda_error; }
 
+int glm_debug_set_cross_cta_wait_limit(uint32_t polls) {
+    return cuda_status(glm::set_cross_cta_wait_limit(polls));
+}
+
 int glm_kv_store_int8(const glm_dsa_dims *dims, const void *latent, const int64_t *slots,
                       int64_t n, int8_t *cache, int64_t n_rows, void *stream) {
     const int rc = check_store(dims, latent, slots, n, cache, n_rows);
@@ -511,6 +515,23 @@ int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q, const uin
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32, lse, st));
 }
 
+int glm_mla_v_up(const glm_dsa_dims *dims, const void *o_lat, const void *w_kv_b, int32_t qk_nope_head_dim,
+                 int32_t v_head_dim, int32_t n_q, void *out_v, float *out_v_f32, void *stream) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_q < 0 || n_q > 65535 * 128 || qk_nope_head_dim < 0 || v_head_dim < 128 || v_head_dim % 128 != 0 ||
+        v_head_dim > 4096 || qk_nope_head_dim > 4096)
+        return GLM_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(dims->n_heads) * (qk_nope_head_dim + v_head_dim) > (int64_t(1) << 31))
+        return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (!o_lat || !w_kv_b || !out_v) return GLM_ERR_INVALID_ARG;
+    if (!aligned(o_lat, 16) || !aligned(w_kv_b, 16) || !aligned(out_v, 16) || (out_v_f32 && !aligned(out_v_f32, 16)))
+        return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_mla_vup(o_lat, w_kv_b, dims->n_heads, qk_nope_head_dim, v_head_dim, n_q, out_v,
+                                           out_v_f32, static_cast<cudaStream_t>(stream)));
+}
+
 int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *workspace, size_t ws_bytes,
                         void *stream) {
     if (a == nullptr) return GLM_ERR_INVALID_ARG;
@@ -568,15 +589,16 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     p.fp8 = a->cache_fp8 != 0 ? 1 : 0;
     p.zero = reinterpret_cast<uint4 *>(sw.hist);
     p.zero_n16 = idx_multi ? static_cast<int64_t>(align_up(sw.zero_bytes, 16) / 16) : 0;
+    if (a->stop_after < 0 || a->stop_after > 3) return GLM_ERR_INVALID_ARG;
     rc = cuda_status(glm::launch_step_prep(p, st));
-    if (rc != GLM_OK || a->n_q == 0) return rc;
+    if (rc != GLM_OK || a->n_q == 0 || a->stop_after == 1) return rc;
     rc = enqueue_index_select(a->q_idx_dev, a->w_dev, keys, q8 ? a->pooled_scales_dev : nullptr, a->ld_pools,
                               a->q_seq_dev, a->q_pos_dev,
                               a->pad_dev, a->len_dev, a->batch, a->n_q, a->select_k, a->slot_map_dev, a->ld_slot,
                               a->out_width, a->scores_dev, a->topk_dev, a->n_sel_dev, a->tok_dev, a->rows_dev,
                               ws + L.idx, status, false, sms, st, a->pool_begin_dev,
                               a->batch > 0 ? a->max_new_pools : 0);
-    if (rc != GLM_OK) return rc;
+    if (rc != GLM_OK || a->stop_after == 2) return rc;
     const int H = dims->n_heads;
     const glm::MlaPlan plan = glm::mla_plan(a->n_q, H, a->out_width, sms);
     const size_t parts = mla_parts(a->n_q, H, a->out_width);
@@ -584,7 +606,7 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     float *part_ml = reinterpret_cast<float *>(ws + L.mla + mla_acc_bytes(parts));
     rc = cuda_status(glm::launch_mla_split_tc(plan, a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
                                               a->sm_scale, part_acc, part_ml, status, st, true, a->cache_fp8 != 0));
-    if (rc != GLM_OK) return rc;
+    if (rc != GLM_OK || a->stop_after == 3) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, plan.n_chunks, a->out_dev, a->out_f32_dev,
                                                a->lse_dev, st));
 }

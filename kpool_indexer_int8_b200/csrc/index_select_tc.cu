@@ -42,6 +42,8 @@
 
 namespace glm {
 
+GLM_TL_TABLE(glm_tl_index)
+
 constexpr int kIxThreads = 512;                        // 16 warps, see the roles above
 constexpr int kIxTile = 64;                            // pools per tile (UMMA M)
 constexpr int kIxChunk = 32;                           // pools per bulk copy (2 per tile)
@@ -139,6 +141,7 @@ __device__ __noinline__ unsigned sample_threshold(const unsigned *samp, int n_sa
         for (int q = 0; q < r; q += 4)
             *reinterpret_cast<uint4 *>(gs + static_cast<int64_t>(g) * r + q) = *reinterpret_cast<const uint4 *>(top + q);
         if (!grid_barrier(ctr, n_ctas)) ok = false;
+        GLM_TL_AT(glm_tl_index, 14, 64);
     }
     __syncwarp();   // the other lanes wait for lane 0's acquire
     const int U = n_ctas * r;
@@ -296,6 +299,8 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     const bool select = sel.topk != nullptr;
     const bool multi = select && G > 1;
     SelShared &s = *reinterpret_cast<SelShared *>(terms);
+    GLM_TL(glm_tl_index, 0);
+    GLM_TL_SMID(glm_tl_index);
 
     if (fill_invisible) {  // entries past the visible pools are -inf (split over the CTAs)
         const int64_t rest = ld_pools - n_vis;
@@ -368,6 +373,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     tc::fence_after_sync();
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
+    GLM_TL(glm_tl_index, 1);
 
     if (warp == 0) {
         // ---------------- producer ----------------
@@ -415,6 +421,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                 tc::mma_commit(bar(kBarTmEmpty + tb));
                 tc::mma_commit(bar(kBarAccFull + tb));
             }
+            GLM_TL_AT(glm_tl_index, 2, 32);
         }
     } else if (warp == 2) {
         // ---------------- the multi-CTA selection's sample threshold ----------------
@@ -425,9 +432,11 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");   // the meeting word is zeroed
             bool waited = tc::mbar_wait(bar(kBarSample), 0, kIxWaitLimit);   // the sample keys are written
             __syncwarp();
+            GLM_TL_AT(glm_tl_index, 13, 64);
             const unsigned thr = sample_threshold(samp, min(s0, hi - lo), r_pub, static_cast<unsigned>(k_s),
                                                   sel.gsamp + static_cast<int64_t>(n) * kSampleUnion, g,
                                                   &cq[kCntSample], g_eff, scr, waited);
+            GLM_TL_AT(glm_tl_index, 5, 64);
             if (lane == 0) {
                 flag[kFlThr] = thr;
                 if (!waited) flag[kFlWait] = 1;
@@ -465,11 +474,13 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(kBarAccEmpty + tb));
+            if (t == 0) GLM_TL_AT(glm_tl_index, 12, 128);
             if (sample && t == n_st - 1) {   // the sample keys of this warp's rows are written
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar(kBarSample));
             }
         }
+        GLM_TL_AT(glm_tl_index, 3, 128);
     } else if (warp >= 16 - kIxConv) {
         // ---------------- converters ----------------
         const int cw = warp - (16 - kIxConv);
@@ -517,6 +528,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                 if (lane == 0) tc::mbar_arrive(bar(kBarTmFull + tb));
             }
         }
+        GLM_TL_AT(glm_tl_index, 4, 256);
     }
     if (!ok && status) atomicOr(status, 4);
     tc::fence_before_sync();
@@ -528,6 +540,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     }   // lo < hi
     if (sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    GLM_TL(glm_tl_index, 6);
     if (!select) return;
     const unsigned count = static_cast<unsigned>(min(sel.select_k, n_vis));
     auto score_at = [&](int i) { return keep_local ? sloc[i - lo] : __ldcg(srow + i); };
@@ -553,6 +566,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
         }
         __syncthreads();
         const unsigned base = s.n_a;
+        GLM_TL(glm_tl_index, 7);
 #pragma unroll 1
         for (int b0 = lo; b0 < hi; b0 += kIxThreads) {
             const int i = b0 + tid;
@@ -568,12 +582,14 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             }
         }
         __syncthreads();
+        GLM_TL(glm_tl_index, 8);
         if (tid == 0) {   // release the candidates, wait (acquire) for every CTA's
             flag[kFlWait] = grid_barrier(&cnt[kCntArrive], g_eff) ? 0u : 1u;
             if (flag[kFlWait] && status) atomicOr(status, 8);
         }
         __syncthreads();
         if (flag[kFlWait]) return;   // gave up waiting: the status word reports it
+        GLM_TL(glm_tl_index, 9);
         const unsigned total = __ldcg(&cnt[kCntTicket]);
         if (total < count || total > static_cast<unsigned>(kBoundCap)) {
             // the threshold let too few (or too many) through: CTA 0 selects exactly over every
@@ -591,6 +607,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
 #pragma unroll 1
         for (unsigned i = tid; i < total; i += kIxThreads) s.bnd[i] = __ldcg(cand_q + i);
         __syncthreads();
+        GLM_TL(glm_tl_index, 10);
 #pragma unroll 1
         for (unsigned j = static_cast<unsigned>(g + g_eff * warp); j < total; j += static_cast<unsigned>(g_eff * (kIxThreads / 32))) {
             const unsigned long long c = s.bnd[j];
@@ -601,6 +618,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             if (r < count) write_ranked(sel, n, b, pb, r, id_of(c), lane);
         }
         if (g == 0) write_unranked(sel, n, b, pb, seq_len, qp, count);
+        GLM_TL(glm_tl_index, 11);
         return;
     }
     // one CTA: lo = 0, hi = n_vis, the histogram and the scores on chip
@@ -634,6 +652,10 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     };
     finish_selection(count, nA, nB, b_complete, bstar, s.hist2, get_b, n_vis, s);
     write_outputs(sel, n, b, valid_b, pb, seq_len, qp, count, s);
+}
+
+cudaError_t set_cross_cta_wait_limit(uint32_t polls) {
+    return cudaMemcpyToSymbol(g_cross_cta_wait_limit, &polls, sizeof(polls));
 }
 
 int index_select_ctas(int n_q, int64_t ld_pools, int num_sms) {

@@ -58,6 +58,7 @@ struct IxSelectArgs {
     int new_pools;
 };
 int index_select_ctas(int n_q, int64_t ld_pools, int num_sms);
+cudaError_t set_cross_cta_wait_limit(uint32_t polls);   // the index kernel's meetings (current device)
 cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const void *keys,
                                    const float *key_scales, int64_t ld_pools, const int32_t *q_seq,
                                    const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
@@ -90,6 +91,10 @@ struct StepPrepArgs {
     int fp8;                       // the cache holds FP8 rows
 };
 cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream);
+
+// The up-projection after the absorbed MLA (mla_vup.cu): out_v = o_lat . W_v,h^T per head.
+cudaError_t launch_mla_vup(const void *o_lat, const void *w_kv_b, int n_heads, int dk, int dv, int n_q, void *out_v,
+                           float *out_f32, cudaStream_t stream);
 
 cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32_t *q_seq,
                           const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,

@@ -27,6 +27,9 @@ constexpr int kBoundCap = 4096;                  // list B entries kept on chip
 constexpr int kSubCap = 256;                     // level-2 boundary entries ranked directly
 constexpr int kShift2 = 64 - 2 * kHistBitsTop;   // level-2 digit: composite bits 52..42
 constexpr uint32_t kSelWaitLimit = 1u << 21;     // polls of a cross-CTA wait before giving up
+// The limit the waits use: kSelWaitLimit unless a test lowers it (glm_debug_set_cross_cta_wait_limit)
+// to make a wait run out on purpose. One copy per translation unit that waits across CTAs.
+static __device__ uint32_t g_cross_cta_wait_limit = kSelWaitLimit;
 
 __device__ __forceinline__ unsigned long long compose(uint32_t key, int id) {
     return (static_cast<unsigned long long>(key) << 32) |
@@ -85,7 +88,8 @@ __device__ __forceinline__ bool take_ticket(unsigned *ctr, int n_ctas) {
 // wait gave up after kSelWaitLimit polls.
 __device__ __forceinline__ bool grid_barrier(unsigned *ctr, int n_ctas) {
     asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ctr) : "memory");
-    for (uint32_t it = 0; it < kSelWaitLimit; it++) {
+    const uint32_t limit = *static_cast<volatile uint32_t *>(&g_cross_cta_wait_limit);
+    for (uint32_t it = 0; it < limit; it++) {
         if (ld_acquire(ctr) >= static_cast<unsigned>(n_ctas)) return true;
         __nanosleep(32);
     }

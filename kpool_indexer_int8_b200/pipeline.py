@@ -185,8 +185,8 @@ def run_stages(b: DecodeBuffers, stream=None) -> None:
         fn(b, stream=stream)
 
 
-def run_step(b: DecodeBuffers, stream=None) -> None:
-    """One whole step through the one-call entry point."""
+def run_step(b: DecodeBuffers, stream=None, stop_after: int = 0) -> None:
+    """One whole step through the one-call entry point (stop_after = k: its first k kernels only)."""
     glm_dsa_decode_step(b.dims, latent=b.new_latent, slots=b.new_slots, cache=b.cache, k=b.k, gate=b.gate,
                         ln_w=b.ln_w, ln_b=b.ln_b, ln_eps=b.ln_eps, pad=b.pad, length=b.len,
                         pool_begin=b.pool_begin, max_new_pools=b.max_new_pools, pooled=b.pooled, q_idx=b.q_idx,
@@ -194,4 +194,4 @@ def run_step(b: DecodeBuffers, stream=None) -> None:
                         slot_map=b.slot_map, rows=b.rows, topk=b.topk, q=b.q, sm_scale=b.sm_scale, out=b.out,
                         workspace=b.ws_step, n_sel=b.n_sel, tok=b.tok, scores=b.scores, lse=b.lse,
                         out_f32=b.out_f32, pooled_codes=b.pooled_codes, pooled_scales=b.pooled_scales,
-                        cache_fp8=b.fp8, stream=stream)
+                        cache_fp8=b.fp8, stop_after=stop_after, stream=stream)
