@@ -69,6 +69,32 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
+// Reduce V values per lane (V a power of two <= 32) across the warp's 32 lanes with max (kMax) or
+// sum: halving steps hand half of the values to the partner lane, so that after log2(V) steps lane
+// l holds value index (l >> (5 - log2 V)) & (V - 1), reduced over the lanes that differ from l in
+// the bits already used; the remaining steps finish the reduction over the other bits. Returns the
+// lane's value (every lane with the same index holds the same result).
+template <int V, bool kMax>
+__device__ __forceinline__ float butterfly(float (&v)[V]) {
+    const int lane = threadIdx.x & 31;
+    auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
+#pragma unroll
+    for (int half = V / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
+        const bool up = (lane & bit) != 0;
+#pragma unroll
+        for (int i = 0; i < half; i++) {
+            const float send = up ? v[i] : v[i + half];
+            const float keep = up ? v[i + half] : v[i];
+            v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, bit));
+        }
+    }
+    float r = v[0];
+    constexpr int kRest = (V == 32) ? 0 : (V == 16) ? 1 : (V == 8) ? 2 : (V == 4) ? 3 : (V == 2) ? 4 : 5;
+#pragma unroll
+    for (int k = 0; k < kRest; k++) r = op(r, __shfl_xor_sync(0xffffffffu, r, 1 << (kRest - 1 - k)));
+    return r;
+}
+
 // Order-preserving map of an fp32 score to an unsigned key (larger score -> larger key);
 // -0.0 is folded onto +0.0 first so that the two compare equal.
 __device__ __forceinline__ uint32_t score_key(float s) {

@@ -8,12 +8,14 @@
 //   1. the query block of the head group goes to shared memory as fp16, each head scaled by the
 //      power of two 2^e_h that puts its largest magnitude in [2^14, 2^15) (every bf16 value of
 //      magnitude >= 2^-17 after scaling is exact in fp16; the scores are multiplied back by
-//      2^-e_h); in the one-call step this happens before the kernel waits for the index lists;
-//   2. gather: one 1-D bulk copy per valid entry brings its whole 528-byte row (codes, fp32
-//      scale, zero pad) into shared memory, all completing on one mbarrier; the codes are then
-//      widened to fp16 (exact: |code| <= 127; E4M3 codes are exact in fp16 as well) into a tile
-//      C[ROWS x 512] of 8x8 core matrices -- the int8 codes through byte permutes and one packed
-//      subtraction (1024 + code + 128 built as fp16 bits, minus 1152), no integer conversions;
+//      2^-e_h); in the one-call step its loads are issued before the kernel waits for the index
+//      lists;
+//   2. gather: every thread requests its 16-byte pieces of the chunk's rows at once (all of a
+//      chunk's loads in flight together: one round trip), and the row scales; while they are in
+//      flight the query block is staged; the codes are then widened in registers to fp16 (exact:
+//      |code| <= 127; E4M3 codes are exact in fp16 as well) and stored as a tile C[ROWS x 512] of
+//      8x8 core matrices -- the int8 codes through byte permutes and one packed subtraction
+//      (1024 + code + 128 built as fp16 bits, minus 1152), no integer conversions;
 //   3. S^T = C . Q^T on tcgen05 (kind::f16, fp32 accumulator in tensor memory: lane = row,
 //      column = head), 32 MMAs of K = 16;
 //   4. softmax over the chunk's rows for each head: one thread per row and half of the heads;
@@ -27,8 +29,8 @@
 //   6. acc = scale_max * (O_hi + O_lo) and (m, l) of each head go to the workspace (lane = latent
 //      dim: every warp store is 32 consecutive floats of one head); the combine kernel merges the
 //      chunks by log-sum-exp.
-// Every wait is bounded; a timeout sets a status bit, waits (bounded) for this CTA's copies and
-// MMAs still in flight, frees the tensor memory and leaves the partial unwritten.
+// Every wait on the tensor cores is bounded; a timeout sets a status bit, waits (bounded) for this
+// CTA's MMAs still in flight, frees the tensor memory and leaves the partial unwritten.
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
@@ -46,10 +48,9 @@ constexpr uint32_t kMlaWaitLimit = 1u << 22;
 template <int ROWS, int NH>
 struct MlaLayout {
     static constexpr int kPBytes = ROWS * 4 * NH;                     // ROWS x 2 NH fp16 (hi | lo)
-    static constexpr int kRawBytes = ROWS * kRowBytes;
     static constexpr int kC = 0;                                      // ROWS/8 row groups x 64 dim groups x 128 B
-    static constexpr int kRaw = kC + ROWS * 1024;                     // gathered rows, 528 B apart; then P'
-    static constexpr int kQ = kRaw + (kRawBytes > kPBytes ? kRawBytes : kPBytes);   // NH/8 x 64 x 128 B
+    static constexpr int kP = kC + ROWS * 1024;                       // P', core matrices of 8 rows x 8 heads
+    static constexpr int kQ = kP + kPBytes;                           // NH/8 x 64 x 128 B
     static constexpr int kScl = kQ + NH * 1024;                       // ROWS fp32 row scales
     static constexpr int kRow = kScl + ROWS * 4;                      // ROWS row indices
     static constexpr int kRed = kRow + ROWS * 4;                      // [4 quadrants][NH] partial maxima
@@ -57,9 +58,9 @@ struct MlaLayout {
     static constexpr int kQk = kRed2 + 4 * NH * 4;                    // NH fp32 score factors
     static constexpr int kQmax = kQk + NH * 4;                        // NH uint32 |q| maxima (bf16 bits)
     static constexpr int kWords = kQmax + NH * 4;                     // [0] scale max bits, [1] tmem base
-    static constexpr int kBar = kWords + 16;                          // 3 mbarriers
-    static constexpr int kBytes = kBar + 3 * 8;
-    static_assert(kQ % 16 == 0 && kRaw % 16 == 0 && kBar % 8 == 0, "alignment");
+    static constexpr int kBar = kWords + 16;                          // 2 mbarriers
+    static constexpr int kBytes = kBar + 2 * 8;
+    static_assert(kQ % 16 == 0 && kP % 16 == 0 && kBar % 8 == 0, "alignment");
 };
 
 // Four int8 codes (one little-endian word) as four exact fp16 values (two fp16x2 words).
@@ -93,32 +94,6 @@ __device__ __forceinline__ void tmem_ld_v(uint32_t taddr, uint32_t (&r)[V]) {
     else tc::tmem_ld32(taddr, r);
 }
 
-// Reduce V values per lane (V a power of two <= 32) across the warp's 32 lanes with max (kMax) or
-// sum: halving steps hand half of the values to the partner lane, so that after log2(V) steps lane
-// l holds value index (l >> (5 - log2 V)) & (V - 1), reduced over the lanes that differ from l in
-// the bits already used; the remaining steps finish the reduction over the other bits. Returns the
-// lane's value (every lane with the same index holds the same result).
-template <int V, bool kMax>
-__device__ __forceinline__ float butterfly(float (&v)[V]) {
-    const int lane = threadIdx.x & 31;
-    auto op = [](float a, float b) { return kMax ? fmaxf(a, b) : a + b; };
-#pragma unroll
-    for (int half = V / 2, bit = 16; half >= 1; half >>= 1, bit >>= 1) {
-        const bool up = (lane & bit) != 0;
-#pragma unroll
-        for (int i = 0; i < half; i++) {
-            const float send = up ? v[i] : v[i + half];
-            const float keep = up ? v[i + half] : v[i];
-            v[i] = op(keep, __shfl_xor_sync(0xffffffffu, send, bit));
-        }
-    }
-    float r = v[0];
-    constexpr int kRest = (V == 32) ? 0 : (V == 16) ? 1 : (V == 8) ? 2 : (V == 4) ? 3 : (V == 2) ? 4 : 5;
-#pragma unroll
-    for (int k = 0; k < kRest; k++) r = op(r, __shfl_xor_sync(0xffffffffu, r, 1 << (kRest - 1 - k)));
-    return r;
-}
-
 template <int ROWS, int NH, bool kFp8>
 __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
     const uint16_t *__restrict__ q, int n_heads, const uint8_t *__restrict__ cache, int64_t n_rows,
@@ -127,14 +102,13 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
     using L = MlaLayout<ROWS, NH>;
     constexpr int V = NH / 2;             // heads per softmax thread
     constexpr int kLboP = 32 * NH;        // P': bytes between row groups (2 NH / 8 head groups x 128 B)
-    // early_q: the query block is an input no preceding kernel writes (the one-call step), so it is
-    // staged before waiting for the preceding kernel; only the row indices wait for it
+    // early_q: the query block is an input no preceding kernel writes (the one-call step), so its
+    // loads are issued before waiting for the preceding kernel; the row indices wait for it
     if (early_q) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     else pdl_begin();
     extern __shared__ __align__(128) unsigned char smem[];
     unsigned char *Cs = smem + L::kC;
-    unsigned char *raw = smem + L::kRaw;
-    unsigned char *Ps = smem + L::kRaw;
+    unsigned char *Ps = smem + L::kP;
     unsigned char *Qs = smem + L::kQ;
     float *scl = reinterpret_cast<float *>(smem + L::kScl);
     int *ridx = reinterpret_cast<int *>(smem + L::kRow);
@@ -144,7 +118,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
     unsigned *qmax = reinterpret_cast<unsigned *>(smem + L::kQmax);
     unsigned *words = reinterpret_cast<unsigned *>(smem + L::kWords);
     const uint32_t bar0 = tc::smem_addr(smem + L::kBar);
-    const uint32_t bar_g = bar0, bar_s = bar0 + 8, bar_o = bar0 + 16;
+    const uint32_t bar_s = bar0, bar_o = bar0 + 8;
 
     const int n = blockIdx.y, c = blockIdx.x / n_hg, hg = blockIdx.x % n_hg;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -154,8 +128,8 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
     GLM_TL(glm_tl_split, 0);
     GLM_TL_SMID(glm_tl_split);
 
-    // 1. the query block: thread t holds head qh = 8 ((t >> 3) % (NH/8)) + (t & 7), dim groups
-    //    qd0 + i (256/NH) (8 consecutive heads of one dim group per 8 lanes: conflict-free stores)
+    // 1. the query block's loads: thread t holds head qh = 8 ((t >> 3) % (NH/8)) + (t & 7), dim
+    //    groups qd0 + i (256/NH) (8 consecutive heads of one dim group per 8 lanes: conflict-free stores)
     constexpr int kQPieces = NH * 64 / kMlaThreads;
     constexpr int kQStride = kMlaThreads / NH;
     const int qh = ((tid >> 3) % (NH / 8)) * 8 + (tid & 7);
@@ -169,6 +143,54 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
 #pragma unroll
         for (int i = 0; i < kQPieces; i++) qv[i] = qreal ? __ldg(qn + qd0 + i * kQStride) : make_uint4(0u, 0u, 0u, 0u);
     }
+    if (early_q) asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    // 2. the chunk's row indices (entries past width or outside [0, n_rows) are padding)
+    int myrow = -1;
+    if (tid < ROWS) {
+        const int j = c * ROWS + tid;
+        const int r = j < width ? rows[static_cast<int64_t>(n) * width + j] : -1;
+        myrow = (r >= 0 && r < n_rows) ? r : -1;
+        ridx[tid] = myrow;
+    }
+    const int n_valid = __syncthreads_count(myrow >= 0);
+    GLM_TL(glm_tl_split, 2);
+    if (n_valid == 0) {   // no valid entry in this chunk: an empty partial
+        if (tid < nh_real) {
+            part_ml[2 * (ml_base + tid)] = -INFINITY;
+            part_ml[2 * (ml_base + tid) + 1] = 0.0f;
+        }
+        return;
+    }
+
+    // 3. gather: every 16-code piece of the chunk's rows and every row scale is requested at once
+    //    (piece P: row 8 rg + (P & 7), codes 16 k .. 16 k + 15; eight lanes hold eight rows of one
+    //    piece index, so that the widened lines they store are 128 contiguous bytes)
+    constexpr int kCvt = ROWS * 32 / kMlaThreads;
+    uint4 gv[kCvt];
+#pragma unroll
+    for (int it = 0; it < kCvt; it++) {
+        const int P = it * kMlaThreads + tid;
+        const int jl = P & 7, klo = (P >> 3) & 3, rest = P >> 5;
+        const int rg = rest % (ROWS / 8), k = (rest / (ROWS / 8)) * 4 + klo;
+        const int r = ridx[rg * 8 + jl];
+        gv[it] = r >= 0 ? __ldg(reinterpret_cast<const uint4 *>(cache + static_cast<int64_t>(r) * kRowBytes) + k)
+                        : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const float my_scale = myrow >= 0 ? __ldg(reinterpret_cast<const float *>(cache + static_cast<int64_t>(myrow) * kRowBytes + kLatent)) : 0.0f;
+    if (warp == 0) {
+        tc::tmem_alloc(tc::smem_addr(&words[1]), 8 * NH);
+        tc::tmem_relinquish();
+        tc::fence_before_sync();
+    }
+    if (tid == 32) {
+        tc::mbar_init(bar_s, 1);
+        tc::mbar_init(bar_o, 1);
+        tc::mbar_fence_init();
+    }
+
+    // 4. while the rows are in flight: the query block as fp16, each head scaled by the power of two
+    //    2^e_h that puts its largest magnitude in [2^14, 2^15) (exact: bf16 mantissas fit fp16)
     unsigned mx = 0u;   // largest |q| of the thread's pieces, as bf16 magnitude bits (ordered as integers)
 #pragma unroll
     for (int i = 0; i < kQPieces; i++) {
@@ -176,7 +198,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
 #pragma unroll
         for (int e = 0; e < 4; e++) mx = max(mx, max(w4[e] & 0x7fffu, (w4[e] >> 16) & 0x7fffu));
     }
-    __syncthreads();
     if (qreal) atomicMax(&qmax[qh], mx);
     __syncthreads();
     {
@@ -205,97 +226,41 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
         }
     }
     GLM_TL(glm_tl_split, 1);
-    if (early_q) asm volatile("griddepcontrol.wait;" ::: "memory");
-    asm volatile("fence.proxy.async.global;" ::: "memory");   // rows written before this kernel are read by bulk copies
 
-    // 2. the chunk's row indices (entries past width or outside [0, n_rows) are padding)
-    int myrow = -1;
+    // 5. row scales, their maximum, and the codes widened to fp16 core matrices
     if (tid < ROWS) {
-        const int j = c * ROWS + tid;
-        const int r = j < width ? rows[static_cast<int64_t>(n) * width + j] : -1;
-        myrow = (r >= 0 && r < n_rows) ? r : -1;
-        ridx[tid] = myrow;
-    }
-    const int n_valid = __syncthreads_count(myrow >= 0);
-    GLM_TL(glm_tl_split, 2);
-    if (n_valid == 0) {   // no valid entry in this chunk: an empty partial
-        if (tid < nh_real) {
-            part_ml[2 * (ml_base + tid)] = -INFINITY;
-            part_ml[2 * (ml_base + tid) + 1] = 0.0f;
-        }
-        return;
-    }
-    if (warp == 0) {
-        tc::tmem_alloc(tc::smem_addr(&words[1]), 8 * NH);
-        tc::tmem_relinquish();
-        tc::fence_before_sync();
-    }
-    if (warp == 1) {
-        if (lane == 0) {
-            tc::mbar_init(bar_g, 1);
-            tc::mbar_init(bar_s, 1);
-            tc::mbar_init(bar_o, 1);
-            tc::mbar_fence_init();
-            tc::mbar_arrive_expect_tx(bar_g, static_cast<uint32_t>(n_valid) * kRowBytes);
-        }
-        __syncwarp();
-        // every valid entry's whole row: one bulk copy each (528 = 33 x 16 bytes, 16-byte aligned)
-        const uint32_t raw_addr = tc::smem_addr(raw);
-#pragma unroll
-        for (int j = lane; j < ROWS; j += 32) {
-            const int r = ridx[j];
-            if (r >= 0) tc::bulk_g2s(raw_addr + j * kRowBytes, cache + static_cast<int64_t>(r) * kRowBytes, kRowBytes, bar_g);
-        }
-    }
-    __syncthreads();
-    tc::fence_after_sync();
-    const uint32_t tmem = words[1];
-    bool ok = tc::mbar_wait(bar_g, 0, kMlaWaitLimit);
-    GLM_TL(glm_tl_split, 3);
-    if (!__syncthreads_and(ok)) {   // the rows did not arrive: wait once more, then give up
-        if (tid == 0) atomicOr(status, 16);
-        tc::mbar_wait(bar_g, 0, kMlaWaitLimit);
-        __syncthreads();
-        goto done;
-    }
-
-    // 3. row scales, their maximum, and the codes widened to fp16 core matrices
-    if (tid < ROWS) {
-        const float s = myrow >= 0 ? *reinterpret_cast<const float *>(raw + tid * kRowBytes + kLatent) : 0.0f;
-        scl[tid] = s;
-        const unsigned sm = __reduce_max_sync(0xffffffffu, __float_as_uint(s));   // scales are >= 0
+        scl[tid] = my_scale;
+        const unsigned sm = __reduce_max_sync(0xffffffffu, __float_as_uint(my_scale));   // scales are >= 0
         if (lane == 0) atomicMax(&words[0], sm);
     }
-    {
-        constexpr int kCvt = ROWS * 32 / kMlaThreads;   // 16-code pieces per thread
 #pragma unroll
-        for (int it = 0; it < kCvt; it++) {
-            const int P = it * kMlaThreads + tid;
-            const int jl = P & 7, klo = (P >> 3) & 3, rest = P >> 5;
-            const int rg = rest % (ROWS / 8), k = (rest / (ROWS / 8)) * 4 + klo;
-            const int j = rg * 8 + jl;
-            uint4 w = make_uint4(0u, 0u, 0u, 0u);
-            if (ridx[j] >= 0) w = *reinterpret_cast<const uint4 *>(raw + j * kRowBytes + k * 16);
-            uint32_t o[8];
-            if (kFp8) {
-                fp8_to_f16x4(w.x, o[0], o[1]);
-                fp8_to_f16x4(w.y, o[2], o[3]);
-                fp8_to_f16x4(w.z, o[4], o[5]);
-                fp8_to_f16x4(w.w, o[6], o[7]);
-            } else {
-                codes_to_f16x4(w.x, o[0], o[1]);
-                codes_to_f16x4(w.y, o[2], o[3]);
-                codes_to_f16x4(w.z, o[4], o[5]);
-                codes_to_f16x4(w.w, o[6], o[7]);
-            }
-            unsigned char *line = Cs + rg * 8192 + (2 * k) * 128 + jl * 16;
-            *reinterpret_cast<uint4 *>(line) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4 *>(line + 128) = make_uint4(o[4], o[5], o[6], o[7]);
+    for (int it = 0; it < kCvt; it++) {
+        const int P = it * kMlaThreads + tid;
+        const int jl = P & 7, klo = (P >> 3) & 3, rest = P >> 5;
+        const int rg = rest % (ROWS / 8), k = (rest / (ROWS / 8)) * 4 + klo;
+        const uint4 w = gv[it];
+        uint32_t o[8];
+        if (kFp8) {
+            fp8_to_f16x4(w.x, o[0], o[1]);
+            fp8_to_f16x4(w.y, o[2], o[3]);
+            fp8_to_f16x4(w.z, o[4], o[5]);
+            fp8_to_f16x4(w.w, o[6], o[7]);
+        } else {
+            codes_to_f16x4(w.x, o[0], o[1]);
+            codes_to_f16x4(w.y, o[2], o[3]);
+            codes_to_f16x4(w.z, o[4], o[5]);
+            codes_to_f16x4(w.w, o[6], o[7]);
         }
+        unsigned char *line = Cs + rg * 8192 + (2 * k) * 128 + jl * 16;
+        *reinterpret_cast<uint4 *>(line) = make_uint4(o[0], o[1], o[2], o[3]);
+        *reinterpret_cast<uint4 *>(line + 128) = make_uint4(o[4], o[5], o[6], o[7]);
     }
+    GLM_TL(glm_tl_split, 3);
     tc::fence_proxy_async();
     __syncthreads();
     tc::fence_after_sync();
+    const uint32_t tmem = words[1];
+    bool ok;
 
     GLM_TL(glm_tl_split, 4);
     // 4. S^T = C . Q^T (M = ROWS rows, N = NH heads, K = 512)
@@ -437,17 +402,13 @@ done:
 int mla_tc_chunk() { return 64; }
 
 MlaPlan mla_plan(int n_q, int n_heads, int width, int num_sms) {
-    // 128-row chunks of 16 heads while they fill the SMs about twice; otherwise 64-row chunks of
-    // 64 heads (no head group gathers a row another group of its chunk gathers again)
+    // 64-row chunks of 16 heads while they fill the SMs about one and a half times; otherwise
+    // 64-row chunks of all 64 heads (no head group gathers a row another group of its chunk
+    // gathers again)
     MlaPlan p{};
-    const long long ctas128 = static_cast<long long>(n_q) * ((width + 127) / 128) * ((n_heads + 15) / 16);
-    if (ctas128 <= 2ll * num_sms) {
-        p.rows = 128;
-        p.heads = 16;
-    } else {
-        p.rows = 64;
-        p.heads = 64;
-    }
+    const long long ctas16 = static_cast<long long>(n_q) * ((width + 63) / 64) * ((n_heads + 15) / 16);
+    p.rows = 64;
+    p.heads = (2 * ctas16 <= 3ll * num_sms) ? 16 : 64;
     p.n_chunks = (width + p.rows - 1) / p.rows;
     p.n_hg = (n_heads + p.heads - 1) / p.heads;
     return p;
@@ -478,9 +439,7 @@ cudaError_t launch_mla_split_tc(const MlaPlan &p, const void *q, int n_heads, co
                                           status, stream, early_q)                                               \
                    : launch_t<R, H, false>(p, q, n_heads, c8, n_rows, rows, n_q, width, sm_scale, part_acc,         \
                                            part_ml, status, stream, early_q);
-    GLM_MLA_LAUNCH(128, 16)
     GLM_MLA_LAUNCH(64, 16)
-    GLM_MLA_LAUNCH(64, 32)
     GLM_MLA_LAUNCH(64, 64)
 #undef GLM_MLA_LAUNCH
     return cudaErrorInvalidValue;
