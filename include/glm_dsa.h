@@ -349,6 +349,40 @@ int glm_mla_v_up(const glm_dsa_dims *dims, const void *o_lat_dev, const void *w_
                  float *out_v_f32_dev, void *stream);
 
 /* ------------------------------------------------------------------------------------------ */
+/* context parallelism: one sequence's pools and rows over several ranks                        */
+/* ------------------------------------------------------------------------------------------ */
+/*
+ * TensorFold issue #402, 'Credit': tokens are interleaved over the ranks, local candidates are
+ * merged into the global top-k, and attention partials are merged by log-sum-exp in rank order.
+ * Here the unit is the pool: rank r of `world` holds the pools p = r + world i (stored at local
+ * index i, with the cache rows of their tokens) and the visible tail when it would own the next
+ * pool. Each rank selects its local top-k (glm_index_scores_topk, keeping the scores), turns it into
+ * (score, global pool id) candidates, the ranks exchange them (a collective of the caller's), and
+ * every rank runs the same merge, which equals the selection over all pools; each rank then
+ * attends over the selected rows it holds and the ranks exchange and merge those results.
+ *
+ * glm_cp_candidates: cand_scores[n][x] = scores[n][topk[n][x]], cand_ids[n][x] = topk[n][x] * world
+ *   + rank (-1 where topk is -1 or past ld_scores).  scores fp32 [n_q, ld_scores], topk int32
+ *   [n_q, select_k] (local indices), cand_* [n_q, select_k].
+ * glm_merge_topk: over the candidates of n_parts parts, laid out [n_parts][n_q][per_part] (what an
+ *   all-gather of every rank's [n_q][per_part] arrays gives), the select_k best (score descending,
+ *   then the lower id; ids must be distinct) per query into topk [n_q, select_k] (-1 padded) and
+ *   n_sel [n_q] (or NULL).
+ * glm_lse_merge: out_parts fp32 [n_parts][n_q][n_heads][512] (normalised attention outputs over
+ *   disjoint row sets) and lse_parts fp32 [n_parts][n_q][n_heads] -> LSE = log sum_r e^{lse_r},
+ *   out = sum_r e^{lse_r - LSE} out_r (bf16 [n_q][n_heads][512], fp32 copy and lse optional),
+ *   parts taken in order; a part with lse = -inf contributes nothing.
+ * All return GLM_OK, GLM_ERR_INVALID_ARG (before anything is enqueued) or GLM_ERR_CUDA.
+ */
+int glm_cp_candidates(const float *scores_dev, int64_t ld_scores, const int32_t *topk_dev, int32_t n_q,
+                      int32_t select_k, int32_t rank, int32_t world, float *cand_scores_dev,
+                      int32_t *cand_ids_dev, void *stream);
+int glm_merge_topk(const float *cand_scores_dev, const int32_t *cand_ids_dev, int32_t n_parts, int32_t n_q,
+                   int32_t per_part, int32_t select_k, int32_t *topk_dev, int32_t *n_sel_dev, void *stream);
+int glm_lse_merge(const glm_dsa_dims *dims, const float *out_parts_dev, const float *lse_parts_dev,
+                  int32_t n_parts, int32_t n_q, void *out_dev, float *out_f32_dev, float *lse_dev, void *stream);
+
+/* ------------------------------------------------------------------------------------------ */
 /* testing                                                                                    */
 /* ------------------------------------------------------------------------------------------ */
 /*

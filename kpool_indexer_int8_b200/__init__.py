@@ -39,7 +39,8 @@ EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv
            "glm_dsa_decode_step",
            "glm_topk_pools", "glm_expand_selection",
            "glm_sparse_mla_decode", "glm_dsa_workspace_size", "glm_kv_store_fp8", "glm_sparse_mla_decode_fp8",
-           "glm_debug_set_cross_cta_wait_limit", "glm_mla_v_up")
+           "glm_debug_set_cross_cta_wait_limit", "glm_mla_v_up", "glm_cp_candidates", "glm_merge_topk",
+           "glm_lse_merge")
 
 
 class glm_dsa_dims(C.Structure):
@@ -457,3 +458,41 @@ def glm_mla_v_up(dims, o_lat, w_kv_b, qk_nope_head_dim, v_head_dim, out_v, out_v
     n_q = o_lat.shape[0]
     _check(lib.glm_mla_v_up(C.byref(dims), _ptr(o_lat), _ptr(w_kv_b), int(qk_nope_head_dim), int(v_head_dim), n_q,
                             _ptr(out_v), _ptr(out_v_f32), _stream(stream)), "glm_mla_v_up")
+
+
+lib.glm_cp_candidates.argtypes = [_P, _I64, _P, _I32, _I32, _I32, _I32, _P, _P, _P]
+lib.glm_cp_candidates.restype = C.c_int
+lib.glm_merge_topk.argtypes = [_P, _P, _I32, _I32, _I32, _I32, _P, _P, _P]
+lib.glm_merge_topk.restype = C.c_int
+lib.glm_lse_merge.argtypes = [_D, _P, _P, _I32, _I32, _P, _P, _P, _P]
+lib.glm_lse_merge.restype = C.c_int
+
+
+def glm_cp_candidates(scores, topk, rank, world, cand_scores, cand_ids, stream=None) -> None:
+    """A rank's local selection as (score, global pool id) candidates: scores fp32 [n_q, ld], topk
+    int32 [n_q, select_k] (local indices) -> cand_scores fp32 / cand_ids int32 [n_q, select_k]."""
+    for t, dt, nm in ((scores, torch.float32, "scores"), (topk, torch.int32, "topk"),
+                      (cand_scores, torch.float32, "cand_scores"), (cand_ids, torch.int32, "cand_ids")):
+        _dev(t, dt, nm)
+    _check(lib.glm_cp_candidates(_ptr(scores), scores.shape[1], _ptr(topk), topk.shape[0], topk.shape[1], int(rank),
+                                 int(world), _ptr(cand_scores), _ptr(cand_ids), _stream(stream)), "glm_cp_candidates")
+
+
+def glm_merge_topk(cand_scores, cand_ids, select_k, topk, n_sel=None, stream=None) -> None:
+    """The global top-k of every part's candidates, laid out [n_parts, n_q, per_part]."""
+    for t, dt, nm in ((cand_scores, torch.float32, "cand_scores"), (cand_ids, torch.int32, "cand_ids"),
+                      (topk, torch.int32, "topk"), (n_sel, torch.int32, "n_sel")):
+        _dev(t, dt, nm)
+    n_parts, n_q, per = cand_ids.shape
+    _check(lib.glm_merge_topk(_ptr(cand_scores), _ptr(cand_ids), n_parts, n_q, per, int(select_k), _ptr(topk),
+                              _ptr(n_sel), _stream(stream)), "glm_merge_topk")
+
+
+def glm_lse_merge(dims, out_parts, lse_parts, out, out_f32=None, lse=None, stream=None) -> None:
+    """Log-sum-exp merge of attention parts: out_parts fp32 [n_parts, n_q, n_heads, 512], lse_parts
+    fp32 [n_parts, n_q, n_heads] -> out bf16 [n_q, n_heads, 512] (fp32 copy and lse optional)."""
+    for t, dt, nm in ((out_parts, torch.float32, "out_parts"), (lse_parts, torch.float32, "lse_parts"),
+                      (out, torch.bfloat16, "out"), (out_f32, torch.float32, "out_f32"), (lse, torch.float32, "lse")):
+        _dev(t, dt, nm)
+    _check(lib.glm_lse_merge(C.byref(dims), _ptr(out_parts), _ptr(lse_parts), out_parts.shape[0], out_parts.shape[1],
+                             _ptr(out), _ptr(out_f32), _ptr(lse), _stream(stream)), "glm_lse_merge")

@@ -515,6 +515,47 @@ int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q, const uin
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32, lse, st));
 }
 
+int glm_cp_candidates(const float *scores, int64_t ld_scores, const int32_t *topk, int32_t n_q, int32_t select_k,
+                      int32_t rank, int32_t world, float *cand_scores, int32_t *cand_ids, void *stream) {
+    if (n_q < 0 || n_q > 65535 || ld_scores < 0 || select_k < 1 || select_k > glm::kMaxSelect || world < 1 ||
+        rank < 0 || rank >= world || ld_scores > (int64_t(1) << 31) / world)
+        return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if ((ld_scores > 0 && !scores) || !topk || !cand_scores || !cand_ids) return GLM_ERR_INVALID_ARG;
+    if ((scores && !aligned(scores, 4)) || !aligned(topk, 4) || !aligned(cand_scores, 4) || !aligned(cand_ids, 4))
+        return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_cp_candidates(scores, ld_scores, topk, n_q, select_k, rank, world, cand_scores,
+                                                 cand_ids, static_cast<cudaStream_t>(stream)));
+}
+
+int glm_merge_topk(const float *cand_scores, const int32_t *cand_ids, int32_t n_parts, int32_t n_q, int32_t per_part,
+                   int32_t select_k, int32_t *topk, int32_t *n_sel, void *stream) {
+    if (n_parts < 1 || n_q < 0 || n_q > 65535 || per_part < 0 || select_k < 1 || select_k > glm::kMaxSelect ||
+        static_cast<int64_t>(n_parts) * per_part > (int64_t(1) << 24))
+        return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (!topk || (per_part > 0 && (!cand_scores || !cand_ids))) return GLM_ERR_INVALID_ARG;
+    if ((cand_scores && !aligned(cand_scores, 4)) || (cand_ids && !aligned(cand_ids, 4)) || !aligned(topk, 4) ||
+        (n_sel && !aligned(n_sel, 4)))
+        return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_merge_topk(cand_scores, cand_ids, n_parts, n_q, per_part, select_k, topk, n_sel,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int glm_lse_merge(const glm_dsa_dims *dims, const float *out_parts, const float *lse_parts, int32_t n_parts,
+                  int32_t n_q, void *out, float *out_f32, float *lse, void *stream) {
+    int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_parts < 1 || n_q < 0 || n_q > 65535) return GLM_ERR_INVALID_ARG;
+    if (n_q == 0) return GLM_OK;
+    if (!out_parts || !lse_parts || !out) return GLM_ERR_INVALID_ARG;
+    if (!aligned(out_parts, 16) || !aligned(lse_parts, 4) || !aligned(out, 16) || (out_f32 && !aligned(out_f32, 16)) ||
+        (lse && !aligned(lse, 4)))
+        return GLM_ERR_INVALID_ARG;
+    return cuda_status(glm::launch_lse_merge(out_parts, lse_parts, n_parts, n_q, dims->n_heads, out, out_f32, lse,
+                                             static_cast<cudaStream_t>(stream)));
+}
+
 int glm_mla_v_up(const glm_dsa_dims *dims, const void *o_lat, const void *w_kv_b, int32_t qk_nope_head_dim,
                  int32_t v_head_dim, int32_t n_q, void *out_v, float *out_v_f32, void *stream) {
     int rc = glm_check_dims(dims);

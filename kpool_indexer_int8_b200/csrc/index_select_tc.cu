@@ -5,18 +5,23 @@
 //     score[n][p] = sum_h w[n][h] * max(0, sum_d q_idx[n][h][d] * pooled[b][p][d])
 //
 // Grid (G, n_q): CTA g of query n owns a contiguous range of the query's visible pools.
-// Phase 1, scoring -- a warp-specialised pipeline, every hand-off an mbarrier:
-//   * producer (warp 0): 1-D bulk copies of 32 pools (16 KB, contiguous) into 4 staging slots;
-//   * converters (warps 8-15): split each fp32 value x exactly into three bf16 terms
-//     (hi = rn(x), mid = rn(x - hi), lo = rn(x - hi - mid)) written as K-major tiles of 64 pools in
-//     the 128-byte swizzle layout (lane reads 16 consecutive bytes of a pool row, writes 8 bytes of
-//     a swizzled 128-byte row: no bank conflicts); two tile buffers;
-//   * MMA issuer (warp 1): per term 8 UMMAs (M = 64 pools, N = 32 heads, K = 16) into one of two
-//     fp32 tensor-memory accumulators; with the bf16 query exact, the three terms reproduce q . x
-//     to fp32 accumulation accuracy;
-//   * epilogue (warps 4-7, one TMEM lane quadrant each): relu and head weights, the score (to
-//     global memory and, when the range is short enough, to shared memory), and (one CTA per
-//     query) its top-11-bit key digit counted in the CTA's histogram.
+// Phase 1, scoring -- a warp-specialised pipeline over chunks of 64 pools, every hand-off an mbarrier:
+//   * producer (warp 0): one 1-D bulk copy per chunk (64 pool rows, 32 KB, contiguous) into a ring
+//     of 5 slots (up to ~128 KB per SM in flight);
+//   * converters (warps 8-15, 8 pool rows of a chunk each): every warp first reads its rows into
+//     registers (lane l: dims 4 l .. 4 l + 3 of a row), the warps meet on an mbarrier, and each
+//     then rewrites its rows in place as two fp16 terms in the 128-byte swizzle layout: the row
+//     scaled by the power of two 2^e_p that puts its largest magnitude in [2^14, 2^15), hi =
+//     rn_fp16(x 2^e_p), lo = rn_fp16(x 2^e_p - hi) -- together x to 2^-23 relative --, and 2^-e_p
+//     kept for the epilogue. Shared memory sees one copy write, one read and one write of a pool
+//     row before the MMA reads: ~2.2 KB per pool;
+//   * MMA issuer (warp 1): per term 8 UMMAs (M = 64 pools, N = 32 heads, K = 16, fp16 operands)
+//     into one of two fp32 tensor-memory accumulators; the query block is fp16 with each head
+//     scaled by its own power of two (exact for the bf16 query), folded back into the head weight;
+//   * epilogue (warps 4-7, one TMEM lane quadrant each): relu and head weights, the pool's 2^-e_p
+//     (both exact powers of two), the score (to global memory and, when the range is short enough,
+//     to shared memory), and (one CTA per query) its top-11-bit key digit counted in the CTA's
+//     histogram.
 // Selection with G = 1: the one CTA selects on chip (histogram boundary bin, lists, sort).
 // Selection with G > 1 -- a sample threshold, so that the query's CTAs meet while the keys still
 // stream: the first tiles of every CTA's range (about an eighth of it) are a sample of the
@@ -32,41 +37,43 @@
 // of the row.
 // Phase 1 is HBM-bound: 512 bytes of pooled key per pool; the tensor cores run at a few percent.
 // With the INT8 indexer state ("GLM-5.3-Flash" pypto-lib page, 'What is quantized': the indexer
-// cache in INT8 with one FP32 scale per row) a pool is 128 code bytes plus its scale: 4 KB bulk
-// copies into 8 slots, one exact bf16 term (|code| <= 127), the score multiplied by the pool scale.
+// cache in INT8 with one FP32 scale per row) a pool is 128 code bytes plus its scale: a chunk is an
+// 8 KB copy, the codes are widened to one exact fp16 term beside them in the slot, and the score is
+// multiplied by the pool's scale.
 #include "common.cuh"
 #include "tc.cuh"
 #include "kernels.cuh"
 #include "select.cuh"
 #include "topk.cuh"
 
+#include <cuda_fp16.h>
+
 namespace glm {
 
 GLM_TL_TABLE(glm_tl_index)
 
 constexpr int kIxThreads = 512;                        // 16 warps, see the roles above
-constexpr int kIxTile = 64;                            // pools per tile (UMMA M)
-constexpr int kIxChunk = 32;                           // pools per bulk copy (2 per tile)
-constexpr int kIxMaxStages = 8;                        // staging slots (fp32 keys use 4, int8 keys 8)
-constexpr int kIxConv = 8;                             // converter warps
-constexpr int kIxAtomBytes = kIxTile * 128;            // 64 rows x 128 bytes (64 dims): 8 KB
-constexpr int kIxTermBytes = 2 * kIxAtomBytes;         // one bf16 term of a tile: 16 KB
-constexpr int kIxBufBytes = 3 * kIxTermBytes;          // three terms: 48 KB
-constexpr int kIxStageRegion = 4 * kIxChunk * kIdxDim * 4;   // 64 KB: 4 x 16 KB fp32 or 8 x 4 KB int8
+constexpr int kIxTile = 64;                            // pools per chunk (UMMA M)
+constexpr int kIxSlots = 5;                            // staging slots, converted in place
+constexpr int kIxSlotBytes = kIxTile * kIdxDim * 4;    // 32 KB: 64 fp32 pool rows
+constexpr int kIxConv = 8;                             // converter warps (8 rows of a chunk each)
+constexpr int kIxAtomBytes = kIxTile * 128;            // 8 KB: one 64-dim K atom of an fp16 term
+constexpr int kIxTermBytes = 2 * kIxAtomBytes;         // 16 KB: one fp16 term of a chunk
+constexpr int kIxPsDepth = kIxSlots + 2;               // ring of the pools' score factors (see converters)
 constexpr uint32_t kIxWaitLimit = 1u << 22;
 
-constexpr int kIxLocalCap = 4096;                      // scores of a CTA kept in shared memory
-constexpr int kIxSampleTiles = 8;                      // most tiles of a CTA's range in the sample
+constexpr int kIxLocalCap = 2048;                      // scores of a CTA kept in shared memory
+constexpr int kIxSampleTiles = 8;                      // most chunks of a CTA's range in the sample
 constexpr int kIxSampleMax = kIxSampleTiles * kIxTile;
 
 struct IxLayout {                                      // offsets from a 1024-byte aligned base
-    static constexpr int kTerms = 0;                                  // [2 buffers][3 terms][16 KB]
-    static constexpr int kStage = kTerms + 2 * kIxBufBytes;           // staging slots
-    static constexpr int kQ = kStage + kIxStageRegion;                // 32 heads x 128 dims bf16
+    static constexpr int kSlots = 0;                                  // [5][32 KB]
+    static constexpr int kQ = kSlots + kIxSlots * kIxSlotBytes;       // 32 heads x 128 dims fp16
     static constexpr int kHist = kQ + kIdxHeads * kIdxDim * 2;        // 2048 uint32
     static constexpr int kLocal = kHist + kHistBins * 4;              // kIxLocalCap fp32 scores
-    static constexpr int kW = kLocal + kIxLocalCap * 4;               // 32 fp32 head weights
-    static constexpr int kBar = kW + kIdxHeads * 4;                   // 25 mbarriers
+    static constexpr int kW = kLocal + kIxLocalCap * 4;               // 32 fp32 head weights (scaled)
+    static constexpr int kPs = kW + kIdxHeads * 4;                    // [kIxPsDepth][64] fp32 score factors
+    static constexpr int kBar = kPs + kIxPsDepth * kIxTile * 4;       // 25 mbarriers
     static constexpr int kTmem = kBar + 25 * 8;
     static constexpr int kFlag = kTmem + 16;                          // 8 words, see kFl*
     static constexpr int kSamp = (kFlag + 32 + 15) / 16 * 16;         // the CTA's sample keys
@@ -75,28 +82,47 @@ struct IxLayout {                                      // offsets from a 1024-by
     static constexpr int kAlloc = kBytes + 1024;                      // room to align the base
 };
 static_assert(IxLayout::kScr % 16 == 0, "the threshold's staged keys are read as 16-byte vectors");
-// The selection's working set overlays the tile buffers once scoring is over.
-static_assert(sizeof(SelShared) <= IxLayout::kStage, "selection working set must fit the tile buffers");
+static_assert(IxLayout::kAlloc <= 232448, "shared memory of one CTA");
+// The selection's working set overlays the staging slots once scoring is over.
+static_assert(sizeof(SelShared) <= IxLayout::kQ, "selection working set must fit the staging slots");
 
 // words at IxLayout::kFlag
 constexpr int kFlThr = 0;       // the sample threshold: a candidate's key is at least this
 constexpr int kFlWait = 1;      // a wait on the query's other CTAs gave up
 
 // mbarrier indices
-constexpr int kBarStFull = 0;     // [8] staging slot filled (producer, tx bytes)
-constexpr int kBarStEmpty = 8;    // [8] staging slot read (8 converter warps)
-constexpr int kBarTmFull = 16;    // [2] tile buffer written (8 warps x 2 chunk slots)
-constexpr int kBarTmEmpty = 18;   // [2] tile buffer read by the MMAs (commit)
+constexpr int kBarStFull = 0;     // [5] slot filled (producer, tx bytes)
+constexpr int kBarStRead = 5;     // [5] slot read into registers (8 converter warps)
+constexpr int kBarStConv = 10;    // [5] slot converted in place (8 converter warps)
+constexpr int kBarStEmpty = 15;   // [5] slot read by the MMAs (commit)
 constexpr int kBarAccFull = 20;   // [2] accumulator ready (commit)
 constexpr int kBarAccEmpty = 22;  // [2] accumulator read (4 epilogue warps)
 constexpr int kBarSample = 24;    // the sample keys are in shared memory (4 epilogue warps)
 
-__device__ __forceinline__ uint32_t bf16_pair(float a, float b) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(a, b);  // .x = a (low half), .y = b
-    return *reinterpret_cast<const uint32_t *>(&v);
+__device__ __forceinline__ uint32_t f16x2_rn(float a, float b) {   // .x = a (low half)
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(b), "f"(a));
+    return r;
 }
-__device__ __forceinline__ float bf16_lo_f(uint32_t p) { return __uint_as_float(p << 16); }
-__device__ __forceinline__ float bf16_hi_f(uint32_t p) { return __uint_as_float(p & 0xffff0000u); }
+__device__ __forceinline__ float f16_lo_f(uint32_t p) { return __half2float(__ushort_as_half(static_cast<unsigned short>(p & 0xffffu))); }
+__device__ __forceinline__ float f16_hi_f(uint32_t p) { return __half2float(__ushort_as_half(static_cast<unsigned short>(p >> 16))); }
+// Four int8 codes as four exact fp16 values (1024 + code + 128 built as fp16 bits, minus 1152).
+__device__ __forceinline__ uint2 codes_to_f16x4(uint32_t w) {
+    const uint32_t t = w ^ 0x80808080u;
+    const uint32_t a = __byte_perm(t, 0x64646464u, 0x5140u), b = __byte_perm(t, 0x64646464u, 0x5342u);
+    uint2 r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r.x) : "r"(a), "r"(0x64806480u));
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r.y) : "r"(b), "r"(0x64806480u));
+    return r;
+}
+// The exponent e that puts a nonzero magnitude m in [2^14, 2^15) once scaled by 2^e (clamped so
+// that 2^e and 2^-e are normal floats); 0 for m = 0.
+__device__ __forceinline__ int pow2_exponent(float m) {
+    if (!(m > 0.0f)) return 0;
+    const int E = static_cast<int>((__float_as_uint(m) >> 23) & 0xffu) - 127;
+    return min(120, max(-120, 14 - E));
+}
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float(static_cast<uint32_t>(e + 127) << 23); }
 
 // The k-th largest sample key of a query (warp 2 of each of its n_ctas CTAs): CTA g publishes
 // the r largest of its n_samp sample keys (r a multiple of 4; 0 where it has fewer) at gs + g r --
@@ -265,20 +291,17 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     const int32_t *__restrict__ q_pos, const int32_t *__restrict__ pad,
     const int32_t *__restrict__ len, int batch, float *__restrict__ scores, int fill_invisible,
     IxSelectArgs sel, int *__restrict__ status) {
-    constexpr int kStages = kQ8 ? 8 : 4;                          // staging slots
     constexpr int kElem = kQ8 ? 1 : 4;                            // bytes per key element
-    constexpr int kStageBytes = kIxChunk * kIdxDim * kElem;       // one chunk of keys
-    constexpr int kNumTerms = kQ8 ? 1 : 3;                        // bf16 terms per key
-    static_assert(kStages * kStageBytes <= kIxStageRegion && kStages <= kIxMaxStages, "staging");
+    constexpr int kNumTerms = kQ8 ? 1 : 2;                        // fp16 terms per key
     // The next kernel of the stream may launch only once this one's CTAs reach the selection (its
     // CTAs then take the SMs the finished CTAs free). Early mode: wait for the preceding kernel
     // only where its outputs are needed; otherwise at once.
     if (!sel.early) asm volatile("griddepcontrol.wait;" ::: "memory");
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char *smem = smem_raw + ((1024u - (tc::smem_addr(smem_raw) & 1023u)) & 1023u);
-    unsigned char *terms = smem + IxLayout::kTerms;
-    unsigned char *stage = smem + IxLayout::kStage;
+    unsigned char *slots = smem + IxLayout::kSlots;
     unsigned char *Qs = smem + IxLayout::kQ;
+    float *ps_ring = reinterpret_cast<float *>(smem + IxLayout::kPs);
     unsigned *hist = reinterpret_cast<unsigned *>(smem + IxLayout::kHist);
     float *sloc = reinterpret_cast<float *>(smem + IxLayout::kLocal);
     float *ws = reinterpret_cast<float *>(smem + IxLayout::kW);
@@ -298,7 +321,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     float *srow = scores + static_cast<int64_t>(n) * ld_pools;
     const bool select = sel.topk != nullptr;
     const bool multi = select && G > 1;
-    SelShared &s = *reinterpret_cast<SelShared *>(terms);
+    SelShared &s = *reinterpret_cast<SelShared *>(slots);
     GLM_TL(glm_tl_index, 0);
     GLM_TL_SMID(glm_tl_index);
 
@@ -332,8 +355,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     const int r_pub = min(min(kPubMax, (kSampleUnion / max(g_eff, 1)) & ~3),
                           max(4, static_cast<int>((2 * k_s + g_eff - 1) / max(g_eff, 1) + 3) & ~3));
     if (lo < hi) {
-    const int n_chunks = (hi - lo + kIxChunk - 1) / kIxChunk;
-    const int n_tiles = (hi - lo + kIxTile - 1) / kIxTile;
+    const int n_chunks = (hi - lo + kIxTile - 1) / kIxTile;
     const unsigned char *src = static_cast<const unsigned char *>(keys) +
                                (static_cast<int64_t>(b) * ld_pools + lo) * kIdxDim * kElem;
 
@@ -345,23 +367,39 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
         tc::fence_before_sync();
     }
     if (tid == 32) {
-        for (int i = 0; i < kStages; i++) tc::mbar_init(bar(kBarStFull + i), 1);
-        for (int i = 0; i < kStages; i++) tc::mbar_init(bar(kBarStEmpty + i), kIxConv);
-        for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarTmFull + i), 2 * kIxConv);
-        for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarTmEmpty + i), 1);
+        for (int i = 0; i < kIxSlots; i++) {
+            tc::mbar_init(bar(kBarStFull + i), 1);
+            tc::mbar_init(bar(kBarStRead + i), kIxConv);
+            tc::mbar_init(bar(kBarStConv + i), kIxConv);
+            tc::mbar_init(bar(kBarStEmpty + i), 1);
+        }
         for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccFull + i), 1);
         for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccEmpty + i), 4);
         tc::mbar_init(bar(kBarSample), 4);
         tc::mbar_fence_init();
     }
-    // query block (bf16 [32 x 128], core matrices: head group stride 2048 B, dim group 128 B)
+    // query block as fp16 (core matrices: head group stride 2048 B, dim group 128 B), each head
+    // scaled by the power of two 2^f_h that puts its largest magnitude in [2^14, 2^15) -- exact
+    // for bf16 values -- and its head weight by 2^-f_h, so that w_h relu(q_h . x) is unchanged:
+    // thread t holds dims 8 (t % 16) .. + 7 of head t / 16 (a head's 16 threads share a half-warp)
     {
         const uint16_t *qn = q_idx + static_cast<int64_t>(n) * kIdxHeads * kIdxDim;
-        const int i = tid, h = i >> 4, dg = i & 15;   // 512 pieces of 16 bytes, one per thread
-        *reinterpret_cast<uint4 *>(Qs + (h >> 3) * 2048 + dg * 128 + (h & 7) * 16) =
-            __ldg(reinterpret_cast<const uint4 *>(qn) + i);
+        const int h = tid >> 4, dg = tid & 15;
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(qn) + tid);
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        unsigned mb = 0u;   // largest |q| bits (bf16 magnitudes order as integers)
+#pragma unroll
+        for (int e = 0; e < 4; e++) mb = max(mb, max(w4[e] & 0x7fffu, (w4[e] >> 16) & 0x7fffu));
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) mb = max(mb, __shfl_xor_sync(0xffffffffu, mb, o));
+        const int f = pow2_exponent(__uint_as_float(mb << 16));
+        const float sc = pow2f(f);
+        uint32_t o4[4];
+#pragma unroll
+        for (int e = 0; e < 4; e++) o4[e] = f16x2_rn(__uint_as_float(w4[e] << 16) * sc, __uint_as_float(w4[e] & 0xffff0000u) * sc);
+        *reinterpret_cast<uint4 *>(Qs + (h >> 3) * 2048 + dg * 128 + (h & 7) * 16) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        if (dg == 0) ws[h] = w[static_cast<int64_t>(n) * kIdxHeads + h] * pow2f(-f);
     }
-    if (tid < kIdxHeads) ws[tid] = w[static_cast<int64_t>(n) * kIdxHeads + tid];
     if (select && !multi)
         for (int i = tid; i < kHistBins; i += kIxThreads) hist[i] = 0;
     if (tid == 64) {
@@ -374,58 +412,58 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
     GLM_TL(glm_tl_index, 1);
+    const uint32_t slots_addr = tc::smem_addr(slots);
 
     if (warp == 0) {
         // ---------------- producer ----------------
         if (lane == 0) {
-            const uint32_t stage_addr = tc::smem_addr(stage);
             bool waited = !sel.early;
             for (int c = 0; c < n_chunks; c++) {
-                const int slot = c % kStages;
-                const int c0 = lo + c * kIxChunk;
-                if (!waited && c0 + kIxChunk > first_new && c0 < first_new + sel.new_pools) {
+                const int slot = c % kIxSlots;
+                const int c0 = lo + c * kIxTile;
+                if (!waited && c0 + kIxTile > first_new && c0 < first_new + sel.new_pools) {
                     // this chunk holds a pool the preceding kernel writes: wait for it first
                     asm volatile("griddepcontrol.wait;" ::: "memory");
                     asm volatile("fence.proxy.async.global;" ::: "memory");
                     waited = true;
                 }
-                if (c >= kStages && !tc::mbar_wait(bar(kBarStEmpty + slot), ((c / kStages) - 1) & 1, kIxWaitLimit))
+                if (c >= kIxSlots && !tc::mbar_wait(bar(kBarStEmpty + slot), ((c / kIxSlots) - 1) & 1, kIxWaitLimit))
                     ok = false;
-                const uint32_t bytes = static_cast<uint32_t>(min(kIxChunk, hi - lo - c * kIxChunk)) * kIdxDim * kElem;
+                const uint32_t bytes = static_cast<uint32_t>(min(kIxTile, hi - c0)) * kIdxDim * kElem;
                 tc::mbar_arrive_expect_tx(bar(kBarStFull + slot), bytes);
-                tc::bulk_g2s(stage_addr + slot * kStageBytes, src + static_cast<int64_t>(c) * kStageBytes, bytes,
-                             bar(kBarStFull + slot));
+                tc::bulk_g2s(slots_addr + slot * kIxSlotBytes, src + static_cast<int64_t>(c) * kIxTile * kIdxDim * kElem,
+                             bytes, bar(kBarStFull + slot));
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            const uint32_t idesc = tc::idesc_bf16(kIxTile, kIdxHeads, false, false);
-            const uint32_t terms_addr = tc::smem_addr(terms), q_addr = tc::smem_addr(Qs);
-            for (int t = 0; t < n_tiles; t++) {
-                const int tb = t & 1;
-                if (!tc::mbar_wait(bar(kBarTmFull + tb), (t >> 1) & 1, kIxWaitLimit)) ok = false;
-                if (t >= 2 && !tc::mbar_wait(bar(kBarAccEmpty + tb), ((t >> 1) - 1) & 1, kIxWaitLimit)) ok = false;
+            const uint32_t idesc = tc::idesc_f16(kIxTile, kIdxHeads, false, false);
+            const uint32_t q_addr = tc::smem_addr(Qs);
+            for (int c = 0; c < n_chunks; c++) {
+                const int slot = c % kIxSlots, tb = c & 1;
+                if (!tc::mbar_wait(bar(kBarStConv + slot), (c / kIxSlots) & 1, kIxWaitLimit)) ok = false;
+                if (c >= 2 && !tc::mbar_wait(bar(kBarAccEmpty + tb), ((c >> 1) - 1) & 1, kIxWaitLimit)) ok = false;
                 tc::fence_after_sync();
                 const uint32_t d = tmem + tb * 32;
+                const uint32_t t0 = slots_addr + slot * kIxSlotBytes + (kQ8 ? kIxTermBytes : 0);
 #pragma unroll
                 for (int term = 0; term < kNumTerms; term++) {
 #pragma unroll
                     for (int ks = 0; ks < kIdxDim / 16; ks++) {
-                        const uint32_t a = terms_addr + tb * kIxBufBytes + term * kIxTermBytes +
-                                           (ks >> 2) * kIxAtomBytes + (ks & 3) * 32;
+                        const uint32_t a = t0 + term * kIxTermBytes + (ks >> 2) * kIxAtomBytes + (ks & 3) * 32;
                         tc::mma_bf16(d, tc::desc_sw128(a, 1024), tc::desc(q_addr + ks * 256, 128, 2048), idesc,
                                      (term > 0 || ks > 0) ? 1u : 0u);
                     }
                 }
-                tc::mma_commit(bar(kBarTmEmpty + tb));
+                tc::mma_commit(bar(kBarStEmpty + slot));
                 tc::mma_commit(bar(kBarAccFull + tb));
             }
             GLM_TL_AT(glm_tl_index, 2, 32);
         }
     } else if (warp == 2) {
         // ---------------- the multi-CTA selection's sample threshold ----------------
-        // Once the epilogue has scored the sample tiles: publish this CTA's largest sample keys,
+        // Once the epilogue has scored the sample chunks: publish this CTA's largest sample keys,
         // meet the query's other CTAs, and select the threshold from all published keys.
         if (sample) {
             unsigned *cq = sel.counters + static_cast<int64_t>(n) * kCntWords;
@@ -446,87 +484,95 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     } else if (warp >= 4 && warp < 8) {
         // ---------------- epilogue: TMEM lane quadrant (warp % 4), rows 16q .. 16q+15 ----------------
         const int qd = warp & 3;
-        const int n_st = min(n_st0, n_tiles);   // tiles of the sample (multi-CTA selection)
-        for (int t = 0; t < n_tiles; t++) {
-            const int tb = t & 1;
-            const int p = lo + t * kIxTile + qd * 16 + lane;
+        const int n_st = min(n_st0, n_chunks);   // chunks of the sample (multi-CTA selection)
+        for (int c = 0; c < n_chunks; c++) {
+            const int tb = c & 1;
+            const int r = qd * 16 + lane;          // row of the chunk (lanes 0-15)
+            const int p = lo + c * kIxTile + r;
             float ksc = 1.0f;   // the pool's int8 scale (loaded before the wait)
             if (kQ8 && lane < 16 && p < hi) ksc = __ldg(key_scales + static_cast<int64_t>(b) * ld_pools + p);
-            if (!tc::mbar_wait(bar(kBarAccFull + tb), (t >> 1) & 1, kIxWaitLimit)) ok = false;
+            if (!tc::mbar_wait(bar(kBarAccFull + tb), (c >> 1) & 1, kIxWaitLimit)) ok = false;
             __syncwarp();
             tc::fence_after_sync();
-            uint32_t r[32];
-            tc::tmem_ld32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + tb * 32, r);
+            uint32_t rr[32];
+            tc::tmem_ld32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + tb * 32, rr);
             tc::tmem_wait_ld();
             uint32_t digit = 0xffffffffu;
             if (lane < 16 && p < hi) {
                 float sc = 0.0f;
 #pragma unroll
-                for (int h2 = 0; h2 < kIdxHeads; h2++) sc = fmaf(ws[h2], fmaxf(__uint_as_float(r[h2]), 0.0f), sc);
-                if (kQ8) sc *= ksc;   // relu(s q.c) = s relu(q.c) for the scale s > 0
+                for (int h2 = 0; h2 < kIdxHeads; h2++) sc = fmaf(ws[h2], fmaxf(__uint_as_float(rr[h2]), 0.0f), sc);
+                // relu(s y) = s relu(y) for s > 0: the int8 scale, or the row's 2^-e_p (exact)
+                sc *= kQ8 ? ksc : ps_ring[(c % kIxPsDepth) * kIxTile + r];
                 srow[p] = sc;
                 if (keep_local) sloc[p - lo] = sc;
                 const uint32_t key = score_key(sc);
-                if (sample && t < n_st) samp[p - lo] = key;
+                if (sample && c < n_st) samp[p - lo] = key;
                 digit = key >> (32 - kHistBitsTop);
             }
             if (select && !multi && digit != 0xffffffffu) atomicAdd(&hist[digit], 1u);
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(kBarAccEmpty + tb));
-            if (t == 0) GLM_TL_AT(glm_tl_index, 12, 128);
-            if (sample && t == n_st - 1) {   // the sample keys of this warp's rows are written
+            if (c == 0) GLM_TL_AT(glm_tl_index, 12, 128);
+            if (sample && c == n_st - 1) {   // the sample keys of this warp's rows are written
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar(kBarSample));
             }
         }
         GLM_TL_AT(glm_tl_index, 3, 128);
     } else if (warp >= 16 - kIxConv) {
-        // ---------------- converters ----------------
+        // ---------------- converters: rows 8 cw .. 8 cw + 7 of each chunk, in place ----------------
         const int cw = warp - (16 - kIxConv);
-        for (int t = 0; t < n_tiles; t++) {
-            const int tb = t & 1;
-            if (t >= 2 && !tc::mbar_wait(bar(kBarTmEmpty + tb), ((t >> 1) - 1) & 1, kIxWaitLimit)) ok = false;
-            unsigned char *buf = terms + tb * kIxBufBytes;
-            for (int half = 0; half < 2; half++) {
-                const int c = 2 * t + half;
-                if (c < n_chunks) {
-                    const int slot = c % kStages;
-                    if (!tc::mbar_wait(bar(kBarStFull + slot), (c / kStages) & 1, kIxWaitLimit)) ok = false;
-                    const unsigned char *st = stage + slot * kStageBytes;
+        for (int c = 0; c < n_chunks; c++) {
+            const int slot = c % kIxSlots;
+            const uint32_t ph = (c / kIxSlots) & 1;
+            const int rows_c = min(kIxTile, hi - (lo + c * kIxTile));
+            unsigned char *st = slots + slot * kIxSlotBytes;
+            if (!tc::mbar_wait(bar(kBarStFull + slot), ph, kIxWaitLimit)) ok = false;
+            if constexpr (kQ8) {   // four int8 codes -> four exact fp16, beside the codes in the slot
 #pragma unroll
-                    for (int pi = 0; pi < kIxChunk / kIxConv; pi++) {
-                        const int pc = cw * (kIxChunk / kIxConv) + pi;   // pool within the chunk
-                        const int r = half * kIxChunk + pc;              // row within the tile
-                        const int off = (lane >> 4) * kIxAtomBytes + r * 128 +
-                                        ((((lane & 15) >> 1) ^ (r & 7)) << 4) + (lane & 1) * 8;
-                        if (kQ8) {   // four int8 codes -> four bf16 (exact: |code| <= 127)
-                            const uint32_t v = *reinterpret_cast<const uint32_t *>(st + pc * kIdxDim + lane * 4);
-                            const float c0 = static_cast<float>(static_cast<int8_t>(v & 0xffu));
-                            const float c1 = static_cast<float>(static_cast<int8_t>((v >> 8) & 0xffu));
-                            const float c2 = static_cast<float>(static_cast<int8_t>((v >> 16) & 0xffu));
-                            const float c3 = static_cast<float>(static_cast<int8_t>(v >> 24));
-                            *reinterpret_cast<uint2 *>(buf + off) = make_uint2(bf16_pair(c0, c1), bf16_pair(c2, c3));
-                            continue;
-                        }
-                        const float4 x = *reinterpret_cast<const float4 *>(st + pc * (kIdxDim * 4) + lane * 16);
-                        const uint32_t h0 = bf16_pair(x.x, x.y), h1 = bf16_pair(x.z, x.w);
-                        const float r0 = x.x - bf16_lo_f(h0), r1 = x.y - bf16_hi_f(h0);
-                        const float r2 = x.z - bf16_lo_f(h1), r3 = x.w - bf16_hi_f(h1);
-                        const uint32_t m0 = bf16_pair(r0, r1), m1 = bf16_pair(r2, r3);
-                        const uint32_t l0 = bf16_pair(r0 - bf16_lo_f(m0), r1 - bf16_hi_f(m0));
-                        const uint32_t l1 = bf16_pair(r2 - bf16_lo_f(m1), r3 - bf16_hi_f(m1));
-                        *reinterpret_cast<uint2 *>(buf + off) = make_uint2(h0, h1);
-                        *reinterpret_cast<uint2 *>(buf + kIxTermBytes + off) = make_uint2(m0, m1);
-                        *reinterpret_cast<uint2 *>(buf + 2 * kIxTermBytes + off) = make_uint2(l0, l1);
-                    }
-                    __syncwarp();
-                    if (lane == 0) tc::mbar_arrive(bar(kBarStEmpty + slot));
+                for (int i = 0; i < 8; i++) {
+                    const int r = cw * 8 + i;
+                    const uint32_t v = r < rows_c ? *reinterpret_cast<const uint32_t *>(st + r * kIdxDim + lane * 4) : 0u;
+                    const int off = (lane >> 4) * kIxAtomBytes + r * 128 + ((((lane & 15) >> 1) ^ (r & 7)) << 4) + (lane & 1) * 8;
+                    *reinterpret_cast<uint2 *>(st + kIxTermBytes + off) = codes_to_f16x4(v);
                 }
-                tc::fence_proxy_async();
+            } else {
+                float4 x[8];
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int r = cw * 8 + i;
+                    x[i] = r < rows_c ? *reinterpret_cast<const float4 *>(st + r * (kIdxDim * 4) + lane * 16)
+                                      : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+                // every warp has read its rows before any rewrites the slot
                 __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bar(kBarTmFull + tb));
+                if (lane == 0) tc::mbar_arrive(bar(kBarStRead + slot));
+                float m[8];
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    m[i] = fmaxf(fmaxf(fabsf(x[i].x), fabsf(x[i].y)), fmaxf(fabsf(x[i].z), fabsf(x[i].w)));
+                const float mrow = butterfly<8, true>(m);   // lane l: max of row (l >> 2) & 7
+                if (!tc::mbar_wait(bar(kBarStRead + slot), ph, kIxWaitLimit)) ok = false;
+#pragma unroll
+                for (int i = 0; i < 8; i++) {
+                    const int r = cw * 8 + i;
+                    const int e = pow2_exponent(__shfl_sync(0xffffffffu, mrow, 4 * i));
+                    const float f = pow2f(e);
+                    const float4 y = make_float4(x[i].x * f, x[i].y * f, x[i].z * f, x[i].w * f);
+                    const uint32_t h0 = f16x2_rn(y.x, y.y), h1 = f16x2_rn(y.z, y.w);
+                    const uint32_t l0 = f16x2_rn(y.x - f16_lo_f(h0), y.y - f16_hi_f(h0));
+                    const uint32_t l1 = f16x2_rn(y.z - f16_lo_f(h1), y.w - f16_hi_f(h1));
+                    const int off = (lane >> 4) * kIxAtomBytes + r * 128 + ((((lane & 15) >> 1) ^ (r & 7)) << 4) + (lane & 1) * 8;
+                    *reinterpret_cast<uint2 *>(st + off) = make_uint2(h0, h1);
+                    *reinterpret_cast<uint2 *>(st + kIxTermBytes + off) = make_uint2(l0, l1);
+                    if (lane == i) ps_ring[(c % kIxPsDepth) * kIxTile + r] = pow2f(-e);
+                }
             }
+            tc::fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bar(kBarStConv + slot));
         }
         GLM_TL_AT(glm_tl_index, 4, 256);
     }

@@ -96,6 +96,15 @@ cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream);
 cudaError_t launch_mla_vup(const void *o_lat, const void *w_kv_b, int n_heads, int dk, int dv, int n_q, void *out_v,
                            float *out_f32, cudaStream_t stream);
 
+// Context parallelism: a rank's selection as (score, global pool id) candidates; the global top-k
+// of every rank's candidates ([n_parts][n_q][per_part]); the log-sum-exp merge of attention parts.
+cudaError_t launch_cp_candidates(const float *scores, int64_t ld, const int32_t *topk, int n_q, int select_k,
+                                 int rank, int world, float *cand_scores, int32_t *cand_ids, cudaStream_t stream);
+cudaError_t launch_merge_topk(const float *cand_scores, const int32_t *cand_ids, int n_parts, int n_q, int per_part,
+                              int select_k, int32_t *topk, int32_t *n_sel, cudaStream_t stream);
+cudaError_t launch_lse_merge(const float *out_parts, const float *lse_parts, int n_parts, int n_q, int n_heads,
+                             void *out, float *out_f32, float *lse, cudaStream_t stream);
+
 cudaError_t launch_expand(const int32_t *topk, const int32_t *n_sel, const int32_t *q_seq,
                           const int32_t *q_pos, const int32_t *pad, const int32_t *len, int batch,
                           int n_q, int select_k, const int64_t *slot_map, int64_t ld_slot, int out_width,

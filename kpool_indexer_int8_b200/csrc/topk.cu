@@ -168,3 +168,79 @@ cudaError_t launch_topk_collect(const float *scores, const NvisSource &src, cons
 }
 
 }  // namespace glm
+
+namespace glm {
+
+// Context parallelism (TensorFold issue #402, 'Credit': "local candidates are merged into the
+// global top-k"): rank r of `world` holds the pools p = r + world i; its index kernel selected the
+// select_k best of them by local index i. cp_candidates turns that selection into (score, global
+// pool id) pairs; merge_topk selects the select_k best of every rank's pairs, by score descending
+// and then the lower global id -- exactly the selection over all pools, because each pool of the
+// global selection is among its own rank's select_k best.
+__global__ void __launch_bounds__(256) cp_candidates_kernel(const float *__restrict__ scores, int64_t ld,
+                                                            const int32_t *__restrict__ topk, int select_k,
+                                                            int rank, int world, float *__restrict__ cand_scores,
+                                                            int32_t *__restrict__ cand_ids) {
+    pdl_begin();
+    const int n = blockIdx.y;
+    const int x = blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= select_k) return;
+    const int64_t o = static_cast<int64_t>(n) * select_k + x;
+    const int i = topk[o];
+    const bool ok = i >= 0 && i < ld;
+    cand_scores[o] = ok ? scores[static_cast<int64_t>(n) * ld + i] : 0.0f;
+    cand_ids[o] = ok ? i * world + rank : GLM_INVALID;
+}
+
+// One CTA per query over the candidates of n_parts parts laid out [n_parts][n_q][per_part]
+// (per_part = n_cand / n_parts): radix selection of the count best composites, bitonic sort,
+// then the top-k row (-1 padded) and n_sel.
+__global__ void __launch_bounds__(kCollectThreads) merge_topk_kernel(const float *__restrict__ cand_scores,
+                                                                     const int32_t *__restrict__ cand_ids,
+                                                                     int n_parts, int n_q, int per_part,
+                                                                     int select_k, int32_t *__restrict__ topk,
+                                                                     int32_t *__restrict__ n_sel) {
+    pdl_begin();
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    SelShared &s = *reinterpret_cast<SelShared *>(smem_raw);
+    const int n = blockIdx.x;
+    const int m = n_parts * per_part;
+    auto at = [&](int i) { return (static_cast<int64_t>(i / per_part) * n_q + n) * per_part + (i % per_part); };
+    auto get = [&](int i) -> unsigned long long {
+        const int32_t id = cand_ids[at(i)];
+        return id >= 0 ? compose(score_key(cand_scores[at(i)]), id) : 0ull;
+    };
+    unsigned valid = 0u;
+    for (int b0 = 0; b0 < m; b0 += blockDim.x) {
+        const int i = b0 + static_cast<int>(threadIdx.x);
+        valid += static_cast<unsigned>(__syncthreads_count(i < m && cand_ids[at(i)] >= 0));
+    }
+    const unsigned count = min(static_cast<unsigned>(select_k), valid);
+    if (count > 0) {
+        radix_select(get, m, count, 0, 0ull, s);
+        collect_from(get, m, ~0ull << (64 - s.done), s.prefix, 0u, s);
+        sort_selected(s.cand, static_cast<int>(count), s);
+    }
+    write_selection(topk + static_cast<int64_t>(n) * select_k, select_k, count, s);
+    if (threadIdx.x == 0 && n_sel) n_sel[n] = static_cast<int32_t>(count);
+}
+
+cudaError_t launch_cp_candidates(const float *scores, int64_t ld, const int32_t *topk, int n_q, int select_k,
+                                 int rank, int world, float *cand_scores, int32_t *cand_ids, cudaStream_t stream) {
+    const dim3 grid(static_cast<unsigned>((select_k + 255) / 256), static_cast<unsigned>(n_q));
+    launch_pdl(cp_candidates_kernel, grid, dim3(256), 0, stream, scores, ld, topk, select_k, rank, world, cand_scores,
+               cand_ids);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_merge_topk(const float *cand_scores, const int32_t *cand_ids, int n_parts, int n_q, int per_part,
+                              int select_k, int32_t *topk, int32_t *n_sel, cudaStream_t stream) {
+    const int smem = static_cast<int>(sizeof(SelShared));
+    cudaError_t e = cudaFuncSetAttribute(merge_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    launch_pdl(merge_topk_kernel, dim3(static_cast<unsigned>(n_q)), dim3(kCollectThreads), smem, stream, cand_scores,
+               cand_ids, n_parts, n_q, per_part, select_k, topk, n_sel);
+    return cudaGetLastError();
+}
+
+}  // namespace glm

@@ -399,3 +399,38 @@ def decode_query(inp, n, cache, pools, select_k=None, out_width=None, pooled_ove
     if attend:
         res["out"], res["lse"] = sparse_mla(inp.q[n], cache, rows, inp.sm_scale)
     return res
+
+
+# ------------------------------------------------------------------------------------------------
+# context parallelism (TensorFold issue #402, 'Credit': local candidates merged into the global
+# top-k; attention partials merged by log-sum-exp in rank order) -- definitions, in numpy fp64
+# ------------------------------------------------------------------------------------------------
+
+def merge_topk(cand_scores, cand_ids, select_k):
+    """The select_k best of (score, id) candidates with distinct ids, by score descending and then
+    the lower id (the order of topk_pools); -1 padded. Returns (ids int32 [select_k], count)."""
+    s = np.asarray(cand_scores, dtype=np.float64).ravel()
+    i = np.asarray(cand_ids, dtype=np.int64).ravel()
+    keep = i >= 0
+    s, i = s[keep], i[keep]
+    s = np.where(s == 0.0, 0.0, s)                      # -0.0 ranks as +0.0
+    order = np.lexsort((i, -s))                         # primary: score descending; then id
+    n = min(int(select_k), len(order))
+    out = np.full(int(select_k), INVALID, dtype=np.int32)
+    out[:n] = i[order[:n]]
+    return out, n
+
+
+def lse_merge(outs, lses):
+    """Attention over the union of disjoint row sets from each set's result: out_r [Hm, L] and
+    lse_r [Hm] of parts r (taken in order; lse = -inf marks an empty part) ->
+    LSE = log sum_r e^{lse_r}, out = sum_r e^{lse_r - LSE} out_r."""
+    o = np.asarray(outs, dtype=np.float64)
+    l = np.asarray(lses, dtype=np.float64)
+    m = np.max(l, axis=0)
+    safe = np.where(np.isfinite(m), m, 0.0)
+    wgt = np.where(np.isfinite(l), np.exp(l - safe), 0.0)       # [parts, Hm]
+    tot = wgt.sum(axis=0)
+    out = np.einsum("rh,rhd->hd", wgt, o) / np.where(tot > 0, tot, 1.0)[:, None]
+    lse = np.where(tot > 0, safe + np.log(np.where(tot > 0, tot, 1.0)), -np.inf)
+    return out, lse
