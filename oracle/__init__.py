@@ -92,6 +92,14 @@ def _declare(L):
     L.oracle_store_fp8.restype = _i32
     L.oracle_dequant_row_fp8.argtypes = [_p, _i64, _p]
     L.oracle_dequant_row_fp8.restype = None
+    L.oracle_e2m1_value.argtypes = [C.c_uint]
+    L.oracle_e2m1_value.restype = _f64
+    L.oracle_e2m1_encode.argtypes = [_f64]
+    L.oracle_e2m1_encode.restype = C.c_uint
+    L.oracle_store_fp4.argtypes = [_p, _p, _i64, _p, _i64]
+    L.oracle_store_fp4.restype = _i32
+    L.oracle_dequant_row_fp4.argtypes = [_p, _i64, _p]
+    L.oracle_dequant_row_fp4.restype = None
 
 
 def _c(a, dtype):
@@ -353,6 +361,41 @@ def dequant_rows_fp8(cache, rows) -> np.ndarray:
     out = np.empty((len(rows), LATENT), dtype=np.float64)
     for i, r in enumerate(rows):
         lib().oracle_dequant_row_fp8(cache.ctypes.data_as(C.c_void_p), int(r), out[i].ctypes.data_as(C.c_void_p))
+    return out
+
+
+# ------------------------------------------------------------------------------------------------
+# the 4-bit latent cache row (E2M1 codes, an E4M3 scale per 16 values, an fp32 scale per row;
+# 304 bytes)
+# ------------------------------------------------------------------------------------------------
+
+FP4_ROW_BYTES = 304
+
+
+def e2m1_value(code) -> float:
+    return lib().oracle_e2m1_value(int(code) & 0xF)
+
+
+def e2m1_encode(x) -> int:
+    return int(lib().oracle_e2m1_encode(float(x)))
+
+
+def store_fp4(latent, slots, cache) -> None:
+    """Quantise ``latent`` (uint16 bf16 bits [n, 512]) into ``cache`` (uint8 [n_rows, 304]) in place."""
+    assert cache.dtype == np.uint8 and cache.flags.c_contiguous and cache.shape[-1] == FP4_ROW_BYTES
+    lat, lp = _c(latent, np.uint16)
+    sl, sp = _c(slots, np.int64)
+    assert lat.shape == (sl.shape[0], LATENT)
+    rc = lib().oracle_store_fp4(lp, sp, sl.shape[0], cache.ctypes.data_as(C.c_void_p), cache.shape[0])
+    if rc != 0:
+        raise ValueError("slot past the end of the cache")
+
+
+def dequant_rows_fp4(cache, rows) -> np.ndarray:
+    cache = np.ascontiguousarray(cache, dtype=np.uint8).reshape(-1, FP4_ROW_BYTES)
+    out = np.empty((len(rows), LATENT), dtype=np.float64)
+    for i, r in enumerate(rows):
+        lib().oracle_dequant_row_fp4(cache.ctypes.data_as(C.c_void_p), int(r), out[i].ctypes.data_as(C.c_void_p))
     return out
 
 

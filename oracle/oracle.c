@@ -597,3 +597,108 @@ void oracle_dequant_row_fp8(const uint8_t *cache, int64_t row, double *out)
     memcpy(&scale, r + ORACLE_LATENT, 4);
     for (int j = 0; j < ORACLE_LATENT; j++) out[j] = oracle_e4m3_value(r[j]) * (double)scale;
 }
+
+/* =============================================================================================
+ * The 4-bit latent cache row (NEXT-4 of the build). [GLM on CUDA] names the opt-in "--kv-dtype
+ * fp4" latent cache and gives no layout.
+ * READINGS: FP4 is E2M1 (sign bit, two exponent bits with bias 1, one mantissa bit: magnitudes
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6) with two levels of scale, one E4M3 scale for every 16 consecutive
+ * values and one fp32 scale for the row (the block-scaled FP4 form of the sm_100 tensor cores):
+ *   s_row = fl32(max(amax, floor) / 2688)     2688 = 6 * 448, the largest code times the
+ *                                             largest block scale
+ *   e_k   = the E4M3 code nearest fl32(bmax_k / fl32(6 s_row)) (bmax_k the largest |x| of block
+ *           k; ties to the even code, saturating at 448)
+ *   d_k   = fl32(value(e_k) s_row)
+ *   code  = the E2M1 code nearest fl32(x / d_k), ties to the even code, saturating at +-6, the
+ *           sign kept; 0 where d_k = 0
+ * bytes: [0, 256) code pairs (byte i holds dim 2i in its low nibble and dim 2i + 1 in its high
+ * one), [256, 288) the 32 block scales, [288, 292) s_row (little endian), [292, 304) zeros. The
+ * dequantised value is value(code) value(e_k) s_row.
+ * ============================================================================================= */
+#define ORACLE_FP4_ROW_BYTES 304
+#define ORACLE_FP4_BLOCK 16
+#define ORACLE_FP4_SCALES_AT 256
+#define ORACLE_FP4_ROW_SCALE_AT 288
+#define ORACLE_E2M1_MAX 6.0
+
+/* The value of an E2M1 code: (1 + m/2) 2^(e-1) for exponent field e >= 1, m/2 for e = 0. */
+double oracle_e2m1_value(unsigned code)
+{
+    const int s = (int)((code >> 3) & 1u), e = (int)((code >> 1) & 3u), m = (int)(code & 1u);
+    const double v = e == 0 ? 0.5 * m : ldexp(2.0 + m, e - 2);
+    return s ? -v : v;
+}
+
+/* The E2M1 code nearest x (ties to the even code), saturating at +-6, the sign kept. */
+unsigned oracle_e2m1_encode(double x)
+{
+    const unsigned s = signbit(x) ? 8u : 0u;
+    const double a = fabs(x);
+    if (a >= ORACLE_E2M1_MAX) return s | 7u;
+    unsigned code;
+    if (a < 1.0) {                                /* subnormal range: steps of 0.5; 2 is 1.0   */
+        code = (unsigned)nearbyint(2.0 * a);
+    } else {
+        int e;
+        frexp(a, &e);                             /* a in [2^(e-1), 2^e)                      */
+        const int E = e - 1;
+        unsigned m = (unsigned)nearbyint(ldexp(a, 1 - E));   /* in [2, 4]                     */
+        int field = E + 1;
+        if (m == 4u) { m = 2u; field++; }
+        code = ((unsigned)field << 1) | (m - 2u);
+        if (code > 7u) code = 7u;
+    }
+    return s | code;
+}
+
+/* store of 4-bit rows (uint8 [n_rows, 304]). Returns 0, or -1 if a slot is past the cache. */
+int oracle_store_fp4(const uint16_t *latent, const int64_t *slots, int64_t n, uint8_t *cache, int64_t n_rows)
+{
+    for (int64_t i = 0; i < n; i++) {
+        const int64_t slot = slots[i];
+        if (slot < 0) continue;
+        if (slot >= n_rows) return -1;
+        const uint16_t *x = latent + i * ORACLE_LATENT;
+        double amax = 0.0;
+        for (int j = 0; j < ORACLE_LATENT; j++) {
+            const double a = fabs(bf16(x[j]));
+            if (a > amax) amax = a;
+        }
+        if (amax < amax_floor()) amax = amax_floor();
+        const float s_row = (float)(amax / (6.0 * ORACLE_E4M3_MAX));
+        const float u = (float)(6.0 * (double)s_row);
+        unsigned char *row = cache + slot * ORACLE_FP4_ROW_BYTES;
+        memset(row, 0, ORACLE_FP4_ROW_BYTES);
+        for (int k = 0; k < ORACLE_LATENT / ORACLE_FP4_BLOCK; k++) {
+            const uint16_t *xb = x + k * ORACLE_FP4_BLOCK;
+            double bmax = 0.0;
+            for (int j = 0; j < ORACLE_FP4_BLOCK; j++) {
+                const double a = fabs(bf16(xb[j]));
+                if (a > bmax) bmax = a;
+            }
+            const unsigned e = oracle_e4m3_encode((double)(float)(bmax / (double)u));
+            const float d = (float)(oracle_e4m3_value(e) * (double)s_row);
+            row[ORACLE_FP4_SCALES_AT + k] = (unsigned char)e;
+            for (int j = 0; j < ORACLE_FP4_BLOCK; j++) {
+                const unsigned c = d > 0.0f ? oracle_e2m1_encode((double)(float)(bf16(xb[j]) / (double)d)) : 0u;
+                const int dim = k * ORACLE_FP4_BLOCK + j;
+                row[dim / 2] |= (unsigned char)((dim & 1) ? c << 4 : c);
+            }
+        }
+        memcpy(row + ORACLE_FP4_ROW_SCALE_AT, &s_row, 4);
+    }
+    return 0;
+}
+
+/* Dequantise one 4-bit cache row into fp64 (value(code) value(e_k) s_row). */
+void oracle_dequant_row_fp4(const uint8_t *cache, int64_t row, double *out)
+{
+    const unsigned char *r = cache + row * ORACLE_FP4_ROW_BYTES;
+    float s_row;
+    memcpy(&s_row, r + ORACLE_FP4_ROW_SCALE_AT, 4);
+    for (int j = 0; j < ORACLE_LATENT; j++) {
+        const unsigned c = (j & 1) ? (r[j / 2] >> 4) & 15u : r[j / 2] & 15u;
+        const unsigned e = r[ORACLE_FP4_SCALES_AT + j / ORACLE_FP4_BLOCK];
+        out[j] = oracle_e2m1_value(c) * oracle_e4m3_value(e) * (double)s_row;
+    }
+}
