@@ -13,15 +13,19 @@
 //     then rewrites its rows in place as two fp16 terms in the 128-byte swizzle layout: the row
 //     scaled by the power of two 2^e_p that puts its largest magnitude in [2^14, 2^15), hi =
 //     rn_fp16(x 2^e_p), lo = rn_fp16(x 2^e_p - hi) -- together x to 2^-23 relative --, and 2^-e_p
-//     kept for the epilogue. Shared memory sees one copy write, one read and one write of a pool
-//     row before the MMA reads: ~2.2 KB per pool;
-//   * MMA issuer (warp 1): per term 8 UMMAs (M = 64 pools, N = 32 heads, K = 16, fp16 operands)
-//     into one of two fp32 tensor-memory accumulators; the query block is fp16 with each head
-//     scaled by its own power of two (exact for the bf16 query), folded back into the head weight;
-//   * epilogue (warps 4-7, one TMEM lane quadrant each): relu and head weights, the pool's 2^-e_p
-//     (both exact powers of two), the score (to global memory and, when the range is short enough,
-//     to shared memory), and (one CTA per query) its top-11-bit key digit counted in the CTA's
-//     histogram.
+//     kept for the epilogue. The two terms of each 64-dim K atom sit one above the other (hi rows
+//     0-63, lo rows 64-127), so that one MMA of M = 128 covers both. Shared memory sees one copy
+//     write, one read and one write of a pool row before the MMA reads: ~2.2 KB per pool;
+//   * MMA issuer (warp 1): 8 UMMAs per chunk (M = 128 = the chunk's hi and lo rows, N = 32 heads,
+//     K = 16, fp16 operands) into one of two fp32 tensor-memory accumulators -- each tcgen05.mma
+//     costs about the same whatever its size here, so the count is what matters; the query block
+//     is fp16 with each head scaled by its own power of two (exact for the bf16 query), folded back
+//     into the head weight;
+//   * epilogue (warps 4-7, one TMEM lane quadrant each): warps 6-7 hold the lo halves of the dots
+//     and hand them over through shared memory; warps 4-5 add them to the hi halves, then relu and
+//     head weights, the pool's 2^-e_p (both exact powers of two), the score (to global memory and,
+//     when the range is short enough, to shared memory), and (one CTA per query) its top-11-bit key
+//     digit counted in the CTA's histogram.
 // Selection with G = 1: the one CTA selects on chip (histogram boundary bin, lists, sort).
 // Selection with G > 1 -- a sample threshold, so that the query's CTAs meet while the keys still
 // stream: the first tiles of every CTA's range (about an eighth of it) are a sample of the
@@ -73,8 +77,9 @@ struct IxLayout {                                      // offsets from a 1024-by
     static constexpr int kLocal = kHist + kHistBins * 4;              // kIxLocalCap fp32 scores
     static constexpr int kW = kLocal + kIxLocalCap * 4;               // 32 fp32 head weights (scaled)
     static constexpr int kPs = kW + kIdxHeads * 4;                    // [kIxPsDepth][64] fp32 score factors
-    static constexpr int kBar = kPs + kIxPsDepth * kIxTile * 4;       // 25 mbarriers
-    static constexpr int kTmem = kBar + 25 * 8;
+    static constexpr int kXch = kPs + kIxPsDepth * kIxTile * 4;       // [2][64 pools][32 heads] fp32 lo dots
+    static constexpr int kBar = kXch + 2 * kIxTile * kIdxHeads * 4;   // 27 mbarriers
+    static constexpr int kTmem = kBar + 27 * 8;
     static constexpr int kFlag = kTmem + 16;                          // 8 words, see kFl*
     static constexpr int kSamp = (kFlag + 32 + 15) / 16 * 16;         // the CTA's sample keys
     static constexpr int kScr = kSamp + kIxSampleMax * 4;             // the published keys, staged
@@ -97,7 +102,8 @@ constexpr int kBarStConv = 10;    // [5] slot converted in place (8 converter wa
 constexpr int kBarStEmpty = 15;   // [5] slot read by the MMAs (commit)
 constexpr int kBarAccFull = 20;   // [2] accumulator ready (commit)
 constexpr int kBarAccEmpty = 22;  // [2] accumulator read (4 epilogue warps)
-constexpr int kBarSample = 24;    // the sample keys are in shared memory (4 epilogue warps)
+constexpr int kBarSample = 24;    // the sample keys are in shared memory (2 epilogue warps)
+constexpr int kBarXch = 25;       // [2] the lo dots of an accumulator are in the exchange buffer (2 warps)
 
 __device__ __forceinline__ uint32_t f16x2_rn(float a, float b) {   // .x = a (low half)
     uint32_t r;
@@ -292,7 +298,6 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     const int32_t *__restrict__ len, int batch, float *__restrict__ scores, int fill_invisible,
     IxSelectArgs sel, int *__restrict__ status) {
     constexpr int kElem = kQ8 ? 1 : 4;                            // bytes per key element
-    constexpr int kNumTerms = kQ8 ? 1 : 2;                        // fp16 terms per key
     // The next kernel of the stream may launch only once this one's CTAs reach the selection (its
     // CTAs then take the SMs the finished CTAs free). Early mode: wait for the preceding kernel
     // only where its outputs are needed; otherwise at once.
@@ -361,32 +366,56 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
 
     const uint32_t bar0 = tc::smem_addr(smem + IxLayout::kBar);
     auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+    const uint32_t slots_addr = tc::smem_addr(slots);
+    bool waited_new = !sel.early;   // (producer) the preceding kernel's pools are safe to read
+    // the producer's copy of chunk c (waits first for the preceding kernel when the chunk holds a
+    // pool it writes)
+    auto issue = [&](int c) {
+        const int slot = c % kIxSlots;
+        const int c0 = lo + c * kIxTile;
+        if (!waited_new && c0 + kIxTile > first_new && c0 < first_new + sel.new_pools) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            waited_new = true;
+        }
+        const uint32_t bytes = static_cast<uint32_t>(min(kIxTile, hi - c0)) * kIdxDim * kElem;
+        tc::mbar_arrive_expect_tx(bar(kBarStFull + slot), bytes);
+        tc::bulk_g2s(slots_addr + slot * kIxSlotBytes, src + static_cast<int64_t>(c) * kIxTile * kIdxDim * kElem,
+                     bytes, bar(kBarStFull + slot));
+    };
+    // the query block's and head weights' loads go out before the first key copies, which would
+    // otherwise queue them behind the whole burst of the query's CTAs
+    const uint16_t *qn = q_idx + static_cast<int64_t>(n) * kIdxHeads * kIdxDim;
+    const uint4 qv = __ldg(reinterpret_cast<const uint4 *>(qn) + tid);
+    const float wv = (tid & 15) == 0 ? __ldg(w + static_cast<int64_t>(n) * kIdxHeads + (tid >> 4)) : 0.0f;
     if (warp == 0) {
         tc::tmem_alloc(tc::smem_addr(tmem_slot), 64);
         tc::tmem_relinquish();
         tc::fence_before_sync();
-    }
-    if (tid == 32) {
-        for (int i = 0; i < kIxSlots; i++) {
-            tc::mbar_init(bar(kBarStFull + i), 1);
-            tc::mbar_init(bar(kBarStRead + i), kIxConv);
-            tc::mbar_init(bar(kBarStConv + i), kIxConv);
-            tc::mbar_init(bar(kBarStEmpty + i), 1);
+        if (lane == 0) {   // the barriers, then the first copies: the stream starts before the set-up ends
+            for (int i = 0; i < kIxSlots; i++) {
+                tc::mbar_init(bar(kBarStFull + i), 1);
+                tc::mbar_init(bar(kBarStRead + i), kIxConv);
+                tc::mbar_init(bar(kBarStConv + i), kIxConv);
+                tc::mbar_init(bar(kBarStEmpty + i), 1);
+            }
+            for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccFull + i), 1);
+            for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccEmpty + i), 4);
+            for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarXch + i), 2);
+            tc::mbar_init(bar(kBarSample), kQ8 ? 4 : 2);
+            tc::mbar_fence_init();
         }
-        for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccFull + i), 1);
-        for (int i = 0; i < 2; i++) tc::mbar_init(bar(kBarAccEmpty + i), 4);
-        tc::mbar_init(bar(kBarSample), 4);
-        tc::mbar_fence_init();
     }
+    __syncthreads();   // (the loads above are issued by every thread; the barriers are initialised)
+    if (warp == 0 && lane == 0)
+        for (int c = 0; c < min(kIxSlots, n_chunks); c++) issue(c);
     // query block as fp16 (core matrices: head group stride 2048 B, dim group 128 B), each head
     // scaled by the power of two 2^f_h that puts its largest magnitude in [2^14, 2^15) -- exact
     // for bf16 values -- and its head weight by 2^-f_h, so that w_h relu(q_h . x) is unchanged:
     // thread t holds dims 8 (t % 16) .. + 7 of head t / 16 (a head's 16 threads share a half-warp)
     {
-        const uint16_t *qn = q_idx + static_cast<int64_t>(n) * kIdxHeads * kIdxDim;
         const int h = tid >> 4, dg = tid & 15;
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(qn) + tid);
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+        const uint32_t w4[4] = {qv.x, qv.y, qv.z, qv.w};
         unsigned mb = 0u;   // largest |q| bits (bf16 magnitudes order as integers)
 #pragma unroll
         for (int e = 0; e < 4; e++) mb = max(mb, max(w4[e] & 0x7fffu, (w4[e] >> 16) & 0x7fffu));
@@ -398,7 +427,7 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
 #pragma unroll
         for (int e = 0; e < 4; e++) o4[e] = f16x2_rn(__uint_as_float(w4[e] << 16) * sc, __uint_as_float(w4[e] & 0xffff0000u) * sc);
         *reinterpret_cast<uint4 *>(Qs + (h >> 3) * 2048 + dg * 128 + (h & 7) * 16) = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-        if (dg == 0) ws[h] = w[static_cast<int64_t>(n) * kIdxHeads + h] * pow2f(-f);
+        if (dg == 0) ws[h] = wv * pow2f(-f);
     }
     if (select && !multi)
         for (int i = tid; i < kHistBins; i += kIxThreads) hist[i] = 0;
@@ -412,33 +441,22 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
     const uint32_t tmem = *tmem_slot;
     bool ok = true;
     GLM_TL(glm_tl_index, 1);
-    const uint32_t slots_addr = tc::smem_addr(slots);
 
     if (warp == 0) {
-        // ---------------- producer ----------------
+        // ---------------- producer (the first kIxSlots copies were issued during the set-up) ----------------
         if (lane == 0) {
-            bool waited = !sel.early;
-            for (int c = 0; c < n_chunks; c++) {
+            for (int c = kIxSlots; c < n_chunks; c++) {
                 const int slot = c % kIxSlots;
-                const int c0 = lo + c * kIxTile;
-                if (!waited && c0 + kIxTile > first_new && c0 < first_new + sel.new_pools) {
-                    // this chunk holds a pool the preceding kernel writes: wait for it first
-                    asm volatile("griddepcontrol.wait;" ::: "memory");
-                    asm volatile("fence.proxy.async.global;" ::: "memory");
-                    waited = true;
-                }
-                if (c >= kIxSlots && !tc::mbar_wait(bar(kBarStEmpty + slot), ((c / kIxSlots) - 1) & 1, kIxWaitLimit))
-                    ok = false;
-                const uint32_t bytes = static_cast<uint32_t>(min(kIxTile, hi - c0)) * kIdxDim * kElem;
-                tc::mbar_arrive_expect_tx(bar(kBarStFull + slot), bytes);
-                tc::bulk_g2s(slots_addr + slot * kIxSlotBytes, src + static_cast<int64_t>(c) * kIxTile * kIdxDim * kElem,
-                             bytes, bar(kBarStFull + slot));
+                if (!tc::mbar_wait(bar(kBarStEmpty + slot), ((c / kIxSlots) - 1) & 1, kIxWaitLimit)) ok = false;
+                issue(c);
             }
         }
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            const uint32_t idesc = tc::idesc_f16(kIxTile, kIdxHeads, false, false);
+            // fp32 keys: M = 128, the chunk's hi rows over its lo rows (one K atom = 16 KB); int8 keys:
+            // M = 64, the one term at the slot's upper half (one K atom = 8 KB)
+            const uint32_t idesc = tc::idesc_f16(kQ8 ? kIxTile : 2 * kIxTile, kIdxHeads, false, false);
             const uint32_t q_addr = tc::smem_addr(Qs);
             for (int c = 0; c < n_chunks; c++) {
                 const int slot = c % kIxSlots, tb = c & 1;
@@ -448,13 +466,10 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                 const uint32_t d = tmem + tb * 32;
                 const uint32_t t0 = slots_addr + slot * kIxSlotBytes + (kQ8 ? kIxTermBytes : 0);
 #pragma unroll
-                for (int term = 0; term < kNumTerms; term++) {
-#pragma unroll
-                    for (int ks = 0; ks < kIdxDim / 16; ks++) {
-                        const uint32_t a = t0 + term * kIxTermBytes + (ks >> 2) * kIxAtomBytes + (ks & 3) * 32;
-                        tc::mma_bf16(d, tc::desc_sw128(a, 1024), tc::desc(q_addr + ks * 256, 128, 2048), idesc,
-                                     (term > 0 || ks > 0) ? 1u : 0u);
-                    }
+                for (int ks = 0; ks < kIdxDim / 16; ks++) {
+                    const uint32_t a = t0 + (ks >> 2) * (kQ8 ? kIxAtomBytes : 2 * kIxAtomBytes) + (ks & 3) * 32;
+                    tc::mma_bf16(d, tc::desc_sw128(a, 1024), tc::desc(q_addr + ks * 256, 128, 2048), idesc,
+                                 ks > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(bar(kBarStEmpty + slot));
                 tc::mma_commit(bar(kBarAccFull + tb));
@@ -482,40 +497,60 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
             __syncwarp();
         }
     } else if (warp >= 4 && warp < 8) {
-        // ---------------- epilogue: TMEM lane quadrant (warp % 4), rows 16q .. 16q+15 ----------------
+        // ---------------- epilogue: TMEM lane quadrant (warp % 4) ----------------
+        // fp32 keys: quadrants 0-1 hold the hi dots of pools 32 q + lane, quadrants 2-3 the lo dots
+        // of pools 32 (q - 2) + lane, handed over through the exchange buffer ([head][pool]: lanes
+        // write consecutive words). int8 keys: rows 16 q + lane (lanes 0-15) of an M = 64 tile.
         const int qd = warp & 3;
         const int n_st = min(n_st0, n_chunks);   // chunks of the sample (multi-CTA selection)
+        float *xch = reinterpret_cast<float *>(smem + IxLayout::kXch);
+        const bool scorer = kQ8 || qd < 2;
         for (int c = 0; c < n_chunks; c++) {
             const int tb = c & 1;
-            const int r = qd * 16 + lane;          // row of the chunk (lanes 0-15)
+            const int r = kQ8 ? qd * 16 + lane : (qd & 1) * 32 + lane;   // row of the chunk
+            const bool has_row = kQ8 ? lane < 16 : true;
             const int p = lo + c * kIxTile + r;
             float ksc = 1.0f;   // the pool's int8 scale (loaded before the wait)
-            if (kQ8 && lane < 16 && p < hi) ksc = __ldg(key_scales + static_cast<int64_t>(b) * ld_pools + p);
+            if (kQ8 && has_row && p < hi) ksc = __ldg(key_scales + static_cast<int64_t>(b) * ld_pools + p);
             if (!tc::mbar_wait(bar(kBarAccFull + tb), (c >> 1) & 1, kIxWaitLimit)) ok = false;
             __syncwarp();
             tc::fence_after_sync();
             uint32_t rr[32];
             tc::tmem_ld32(tmem + (static_cast<uint32_t>(qd * 32) << 16) + tb * 32, rr);
             tc::tmem_wait_ld();
-            uint32_t digit = 0xffffffffu;
-            if (lane < 16 && p < hi) {
-                float sc = 0.0f;
+            float *xb = xch + tb * (kIxTile * kIdxHeads);
+            if (!scorer) {   // lo dots: to the exchange buffer for the warp holding the same pools' hi dots
 #pragma unroll
-                for (int h2 = 0; h2 < kIdxHeads; h2++) sc = fmaf(ws[h2], fmaxf(__uint_as_float(rr[h2]), 0.0f), sc);
-                // relu(s y) = s relu(y) for s > 0: the int8 scale, or the row's 2^-e_p (exact)
-                sc *= kQ8 ? ksc : ps_ring[(c % kIxPsDepth) * kIxTile + r];
-                srow[p] = sc;
-                if (keep_local) sloc[p - lo] = sc;
-                const uint32_t key = score_key(sc);
-                if (sample && c < n_st) samp[p - lo] = key;
-                digit = key >> (32 - kHistBitsTop);
+                for (int h2 = 0; h2 < kIdxHeads; h2++) xb[h2 * kIxTile + r] = __uint_as_float(rr[h2]);
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bar(kBarXch + tb));
+            } else {
+                if (!kQ8) {
+                    if (!tc::mbar_wait(bar(kBarXch + tb), (c >> 1) & 1, kIxWaitLimit)) ok = false;
+#pragma unroll
+                    for (int h2 = 0; h2 < kIdxHeads; h2++)
+                        rr[h2] = __float_as_uint(__uint_as_float(rr[h2]) + xb[h2 * kIxTile + r]);
+                }
+                uint32_t digit = 0xffffffffu;
+                if (has_row && p < hi) {
+                    float sc = 0.0f;
+#pragma unroll
+                    for (int h2 = 0; h2 < kIdxHeads; h2++) sc = fmaf(ws[h2], fmaxf(__uint_as_float(rr[h2]), 0.0f), sc);
+                    // relu(s y) = s relu(y) for s > 0: the int8 scale, or the row's 2^-e_p (exact)
+                    sc *= kQ8 ? ksc : ps_ring[(c % kIxPsDepth) * kIxTile + r];
+                    srow[p] = sc;
+                    if (keep_local) sloc[p - lo] = sc;
+                    const uint32_t key = score_key(sc);
+                    if (sample && c < n_st) samp[p - lo] = key;
+                    digit = key >> (32 - kHistBitsTop);
+                }
+                if (select && !multi && digit != 0xffffffffu) atomicAdd(&hist[digit], 1u);
             }
-            if (select && !multi && digit != 0xffffffffu) atomicAdd(&hist[digit], 1u);
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bar(kBarAccEmpty + tb));
             if (c == 0) GLM_TL_AT(glm_tl_index, 12, 128);
-            if (sample && c == n_st - 1) {   // the sample keys of this warp's rows are written
+            if (scorer && sample && c == n_st - 1) {   // the sample keys of this warp's rows are written
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bar(kBarSample));
             }
@@ -564,9 +599,10 @@ __global__ void __maxnreg__(96) index_select_tc_kernel(
                     const uint32_t h0 = f16x2_rn(y.x, y.y), h1 = f16x2_rn(y.z, y.w);
                     const uint32_t l0 = f16x2_rn(y.x - f16_lo_f(h0), y.y - f16_hi_f(h0));
                     const uint32_t l1 = f16x2_rn(y.z - f16_lo_f(h1), y.w - f16_hi_f(h1));
-                    const int off = (lane >> 4) * kIxAtomBytes + r * 128 + ((((lane & 15) >> 1) ^ (r & 7)) << 4) + (lane & 1) * 8;
+                    // K atom (lane / 16) holds the hi rows at +0 and the lo rows at +8 KB
+                    const int off = (lane >> 4) * (2 * kIxAtomBytes) + r * 128 + ((((lane & 15) >> 1) ^ (r & 7)) << 4) + (lane & 1) * 8;
                     *reinterpret_cast<uint2 *>(st + off) = make_uint2(h0, h1);
-                    *reinterpret_cast<uint2 *>(st + kIxTermBytes + off) = make_uint2(l0, l1);
+                    *reinterpret_cast<uint2 *>(st + kIxAtomBytes + off) = make_uint2(l0, l1);
                     if (lane == i) ps_ring[(c % kIxPsDepth) * kIxTile + r] = pow2f(-e);
                 }
             }
