@@ -41,10 +41,11 @@ KERNELS_PER_STEP = 4
 STEP_KERNELS = ("step_prep", "index_select_tc", "mla_split_tc", "mla_combine")
 
 
-def algorithmic_bytes(inp, key_bytes: int = 512) -> dict:
+def algorithmic_bytes(inp, key_bytes: int = 512, row_bytes: int = 528) -> dict:
     """Bytes the method must move per step (no partials, no score spills): per query the visible
-    pooled keys (512 B each), q_idx + w, the gathered int8 rows (528 B each), q + out, indices;
-    per step the store of the new rows and the pools they complete."""
+    pooled keys (512 B each, 132 for the INT8 indexer state), q_idx + w, the gathered cache rows
+    (528 B each, 304 for 4-bit rows), q + out, indices; per step the store of the new rows and the
+    pools they complete."""
     wl = inp.wl
     per_q_idx = 0
     per_q_mla = 0
@@ -56,10 +57,10 @@ def algorithmic_bytes(inp, key_bytes: int = 512) -> dict:
         n_sel = min(n_vis, wl.select_k)
         tail = min(upto, int(inp.len[s])) - 4 * n_vis
         per_q_idx += n_vis * key_bytes + 32 * 128 * 2 + 32 * 4 + wl.select_k * 4
-        per_q_mla += (4 * n_sel + tail) * 528 + 2 * wl.n_heads * 512 * 2 + wl.out_width * 4
+        per_q_mla += (4 * n_sel + tail) * row_bytes + 2 * wl.n_heads * 512 * 2 + wl.out_width * 4
         gathered += 4 * n_sel + tail
     n_new = int(inp.new_token_mask().sum())
-    store = n_new * (1024 + 528 + 8)
+    store = n_new * (1024 + row_bytes + 8)
     new_pools = sum(1 for qs, qp in zip(inp.q_seq, inp.q_pos) if (qp - inp.pad[qs] + 1) % 4 == 0)
     kpool = new_pools * (4 * (256 + 256) + 512)
     return dict(index=per_q_idx, mla=per_q_mla, store=store, kpool=kpool, gathered=gathered,
@@ -266,7 +267,8 @@ def config_of(wl, args):
             "out_width": wl.out_width, "kpool": 4, "index_heads": 32, "index_dim": 128,
             "latent": 512, "states": args.states,
             "pooled_keys": "int8 codes + fp32 scale per pool" if args.pooled == "int8" else "fp32",
-            "latent_cache": "fp8 (e4m3) rows" if args.cache == "fp8" else "int8 rows",
+            "latent_cache": {"int8": "int8 rows", "fp8": "fp8 (e4m3) rows",
+                             "fp4": "4-bit rows (e2m1, e4m3 scale per 16)"}[args.cache],
             "l2": f"rotates {args.states} independent states per rank (inputs >> 126 MB L2)",
             "launch": f"one cuda graph of {args.states} steps (one per state) per replay", "parallelism": f"replicas x{args.gpus}"}
 
@@ -298,14 +300,29 @@ def run_kernels(args, wl):
     inps, bufs = [], []
     for r, sid in enumerate(replica_state_ids(rank, R)):
         inp = synth.generate(wl, state=sid)
-        b = sdev.allocate_for(inp, dev, q8=args.pooled == "int8", fp8=args.cache == "fp8")
+        b = sdev.allocate_for(inp, dev, q8=args.pooled == "int8", fp8=args.cache == "fp8",
+                               fp4=args.cache == "fp4")
         sdev.load(inp, b)
         bufs.append(b)
         inps.append(inp if r == 0 else None)
         del inp
-    ab = algorithmic_bytes(inps[0], key_bytes=132 if args.pooled == "int8" else 512)
+    ab = algorithmic_bytes(inps[0], key_bytes=132 if args.pooled == "int8" else 512,
+                           row_bytes=304 if args.cache == "fp4" else 528)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
+
+    if args.profile:
+        # plain launches for a profiler: the one-call step (step_prep, index_select_tc,
+        # mla_split_tc, mla_combine) or the separate entry points (store_int8, kpool_build,
+        # index_select_tc, mla_split_tc, mla_combine) over the rotating states, no graphs, no timing
+        fn = P.run_step if args.profile == "step" else P.run_stages
+        with torch.cuda.stream(stream):
+            for i in range(args.steps):
+                fn(bufs[i % R])
+        stream.synchronize()
+        if rank == 0:
+            print(json.dumps({"profile": args.profile, "steps": args.steps, "workload": wl.name}), flush=True)
+        return
 
     # one CUDA graph per state
     # one CUDA graph holding one step of every state in turn (R steps per replay, like a decode
@@ -389,20 +406,10 @@ def run_kernels(args, wl):
     prefix_ms.append(time_graph(P.run_step, reps))
     kernel_ms = [prefix_ms[0]] + [prefix_ms[i] - prefix_ms[i - 1] for i in range(1, 4)]
 
-    # the dominant kernel on its own: back-to-back launches of the fused scores + top-k + expansion
-    # entry over the rotating states (queued behind a sleep, events on the launching stream); each
-    # launch moves its query's pooled keys once, so the mean launch time gives the achieved GB/s
-    n_idx = max(1, min(args.steps, 200))
-    with torch.cuda.stream(stream):
-        torch.cuda._sleep(int(2e5 * n_idx))
-        i0 = torch.cuda.Event(enable_timing=True)
-        i1 = torch.cuda.Event(enable_timing=True)
-        i0.record(stream)
-        for i in range(n_idx):
-            P.index_topk_expand(bufs[i % R])
-        i1.record(stream)
-    stream.synchronize()
-    idx_launch_ms = i0.elapsed_time(i1) / n_idx
+    # the dominant kernel on its own: the fused scores + top-k + expansion entry over the rotating
+    # states, captured as one graph and replayed (events on the launching stream); each launch moves
+    # its query's pooled keys once, so the mean launch time gives the achieved GB/s
+    idx_launch_ms = time_graph(P.index_topk_expand, reps)
 
     # end to end through the public API with host buffers: per step, one host->device copy of the
     # step's packed inputs (new latent rows and slots, q_idx, w, q, positions, pool begins) from
@@ -527,9 +534,11 @@ def main(argv=None):
     ap.add_argument("--states", type=int, default=8)
     ap.add_argument("--pooled", choices=["fp32", "int8"], default="fp32",
                     help="indexer state: fp32 pooled keys (the pages' path) or the INT8 variant")
-    ap.add_argument("--cache", choices=["int8", "fp8"], default="int8",
-                    help="latent cache rows: INT8 (the pages' path) or the FP8 variant")
+    ap.add_argument("--cache", choices=["int8", "fp8", "fp4"], default="int8",
+                    help="latent cache rows: INT8 (the pages' path) or the FP8 or 4-bit variant")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile", choices=["step", "stages"], default=None,
+                    help="run --steps plain launches (no graphs, no timing) for a profiler and exit")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

@@ -42,6 +42,11 @@ extern "C" {
 #define GLM_ERR_WORKSPACE (-3)   /* workspace null or smaller than glm_dsa_workspace_size()    */
 #define GLM_ERR_CUDA (-4)        /* a kernel launch failed                                     */
 
+/* latent cache row formats (glm_dsa_step.cache_format) */
+#define GLM_CACHE_INT8 0         /* int8 codes, fp32 row scale, 528 bytes (glm_kv_store_int8)  */
+#define GLM_CACHE_FP8 1          /* E4M3 codes, fp32 row scale, 528 bytes (glm_kv_store_fp8)   */
+#define GLM_CACHE_FP4 2          /* E2M1 codes, E4M3 scale per 16, fp32 row scale, 304 bytes   */
+
 /* Sentinel of an unused index entry ("Module glm5next_dsa_ref": INVALID). */
 #define GLM_INVALID (-1)
 
@@ -102,6 +107,24 @@ int glm_kv_store_int8(const glm_dsa_dims *dims, const void *latent_dev, const in
  * +-448, the sign kept. Arguments, slots and padding as glm_kv_store_int8; cache_dev uint8 [n_rows, 528].
  */
 int glm_kv_store_fp8(const glm_dsa_dims *dims, const void *latent_dev, const int64_t *slots_dev,
+                     int64_t n, uint8_t *cache_dev, int64_t n_rows, void *stream);
+
+/*
+ * The 4-bit latent cache ("GLM on CUDA": an opt-in 4-bit latent cache, --kv-dtype fp4, lossy; the
+ * page gives no format). A 304-byte row of E2M1 codes (sign, 2 exponent bits with bias 1, 1
+ * mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6) with one E4M3 scale per 16 values and one
+ * fp32 scale per row:
+ *   s_row = max(amax, 1e-4f) / 2688          (2688 = 6 * 448)
+ *   e_k   = E4M3(bmax_k / (6 * s_row))       (bmax_k: largest |x| of values 16k .. 16k+15)
+ *   d_k   = value(e_k) * s_row
+ *   code  = E2M1(x / d_k), 0 where d_k == 0
+ * each an IEEE fp32 operation; E4M3() and E2M1() round to the nearest value, ties to the even
+ * code, saturating (448, 6), the sign kept. Bytes [0,256): code pairs (byte i: value 2i in the low
+ * nibble, 2i+1 in the high nibble); [256,288): e_0 .. e_31; [288,292): s_row (little endian);
+ * [292,304): zeros. The value of an entry is value(code) * value(e_k) * s_row. Arguments, slots
+ * and padding as glm_kv_store_int8; cache_dev uint8 [n_rows, 304] (16-byte aligned).
+ */
+int glm_kv_store_fp4(const glm_dsa_dims *dims, const void *latent_dev, const int64_t *slots_dev,
                      int64_t n, uint8_t *cache_dev, int64_t n_rows, void *stream);
 
 /* ------------------------------------------------------------------------------------------ */
@@ -300,6 +323,18 @@ int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q_dev, const
                               void *workspace_dev, size_t ws_bytes, void *stream);
 
 /*
+ * glm_sparse_mla_decode over 4-bit rows (glm_kv_store_fp4): each entry's key and value is
+ * value(code) * value(e_k) * s_row; code * block scale is widened to fp16 exactly (a product of
+ * magnitude in [2^-10, 2688] with at most 6 significant bits) and s_row is applied as the INT8
+ * row's scale is; everything else as glm_sparse_mla_decode (cache_dev uint8 [n_rows, 304], same
+ * workspace).
+ */
+int glm_sparse_mla_decode_fp4(const glm_dsa_dims *dims, const void *q_dev, const uint8_t *cache_dev,
+                              int64_t n_rows, const int32_t *rows_dev, int32_t n_q, int32_t width,
+                              float sm_scale, void *out_dev, float *lse_dev, float *out_f32_dev,
+                              void *workspace_dev, size_t ws_bytes, void *stream);
+
+/*
  * The same sparse NoPE MLA decode without a workspace argument. The pages have no counterpart:
  * this entry point exists for callers that cannot allocate device memory where they run the
  * attention -- plugin interfaces that pass a kernel only its inputs and outputs, and serving
@@ -450,9 +485,11 @@ typedef struct glm_dsa_step {
     /* the INT8 indexer state instead of pooled_dev (glm_kpool_build_q8), or NULL */
     int8_t *pooled_codes_dev;      /* int8 [batch, ld_pools, 128]        */
     float *pooled_scales_dev;      /* fp32 [batch, ld_pools]             */
-    /* nonzero: cache_dev holds FP8 rows (uint8 [n_rows, 528]); the store and the attention are
-     * glm_kv_store_fp8 and glm_sparse_mla_decode_fp8 */
-    int32_t cache_fp8;
+    /* the rows of cache_dev: GLM_CACHE_INT8 (int8 [n_rows, 528]), GLM_CACHE_FP8 (uint8
+     * [n_rows, 528]) or GLM_CACHE_FP4 (uint8 [n_rows, 304]); the store and the attention are those
+     * of glm_kv_store_int8 / _fp8 / _fp4 and glm_sparse_mla_decode / _fp8 / _fp4. Any other value:
+     * GLM_ERR_INVALID_ARG. */
+    int32_t cache_format;
     /* 0: the whole step. k = 1, 2, 3: only the step's first k kernels (1: store, pool build and
      * counter zeroing; 2: + scoring, selection and expansion; 3: + the attention's split), for
      * timing a prefix of the step; the outputs of the later kernels are then not written. */

@@ -28,6 +28,8 @@ GLM_ERR_WORKSPACE = -3
 GLM_ERR_CUDA = -4
 GLM_INVALID = -1
 GLM_ROW_BYTES = 528
+GLM_FP4_ROW_BYTES = 304
+GLM_CACHE_INT8, GLM_CACHE_FP8, GLM_CACHE_FP4 = 0, 1, 2
 GLM_OP_INDEX_SCORES_TOPK = 1
 GLM_OP_TOPK_POOLS = 2
 GLM_OP_SPARSE_MLA = 3
@@ -40,7 +42,7 @@ EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv
            "glm_topk_pools", "glm_expand_selection",
            "glm_sparse_mla_decode", "glm_dsa_workspace_size", "glm_kv_store_fp8", "glm_sparse_mla_decode_fp8",
            "glm_debug_set_cross_cta_wait_limit", "glm_mla_v_up", "glm_cp_candidates", "glm_merge_topk",
-           "glm_lse_merge")
+           "glm_lse_merge", "glm_kv_store_fp4", "glm_sparse_mla_decode_fp4")
 
 
 class glm_dsa_dims(C.Structure):
@@ -68,7 +70,7 @@ class glm_dsa_step(C.Structure):
                 ("tok_dev", C.c_void_p), ("rows_dev", C.c_void_p),
                 ("q_dev", C.c_void_p), ("sm_scale", C.c_float), ("out_dev", C.c_void_p),
                 ("lse_dev", C.c_void_p), ("out_f32_dev", C.c_void_p),
-                ("pooled_codes_dev", C.c_void_p), ("pooled_scales_dev", C.c_void_p), ("cache_fp8", C.c_int32),
+                ("pooled_codes_dev", C.c_void_p), ("pooled_scales_dev", C.c_void_p), ("cache_format", C.c_int32),
                 ("stop_after", C.c_int32)]
 
 
@@ -116,6 +118,10 @@ lib.glm_sparse_mla_decode_fp8.argtypes = [_D, _P, _P, _I64, _P, _I32, _I32, _F32
 lib.glm_sparse_mla_decode_fp8.restype = C.c_int
 lib.glm_kv_store_fp8.argtypes = [_D, _P, _P, _I64, _P, _I64, _P]
 lib.glm_kv_store_fp8.restype = C.c_int
+lib.glm_sparse_mla_decode_fp4.argtypes = [_D, _P, _P, _I64, _P, _I32, _I32, _F32, _P, _P, _P, _P, _SZ, _P]
+lib.glm_sparse_mla_decode_fp4.restype = C.c_int
+lib.glm_kv_store_fp4.argtypes = [_D, _P, _P, _I64, _P, _I64, _P]
+lib.glm_kv_store_fp4.restype = C.c_int
 lib.glm_sparse_mla_decode.restype = C.c_int
 lib.glm_dsa_workspace_size.argtypes = [_D, _I32, _I32, _I64, _I32, _I32]
 lib.glm_dsa_workspace_size.restype = C.c_size_t
@@ -186,6 +192,16 @@ def glm_kv_store_fp8(dims, latent, slots, cache, stream=None) -> None:
     n_rows = cache.numel() // GLM_ROW_BYTES
     _check(lib.glm_kv_store_fp8(C.byref(dims), _ptr(latent), _ptr(slots), latent.shape[0],
                                 _ptr(cache), n_rows, _stream(stream)), "glm_kv_store_fp8")
+
+
+def glm_kv_store_fp4(dims, latent, slots, cache, stream=None) -> None:
+    """The 4-bit latent row: latent bf16 [n, 512], slots int64 [n], cache uint8 [n_rows, 304]."""
+    _dev(latent, torch.bfloat16, "latent", 2)
+    _dev(slots, torch.int64, "slots", 1)
+    _dev(cache, torch.uint8, "cache")
+    n_rows = cache.numel() // GLM_FP4_ROW_BYTES
+    _check(lib.glm_kv_store_fp4(C.byref(dims), _ptr(latent), _ptr(slots), latent.shape[0],
+                                _ptr(cache), n_rows, _stream(stream)), "glm_kv_store_fp4")
 
 
 def glm_kpool_build(dims, k, gate, ln_w, ln_b, ln_eps, pad, length, pooled, pool_begin=None,
@@ -297,14 +313,15 @@ def glm_index_topk_expand(dims, q_idx, w, pooled, q_seq, q_pos, pad, length, sel
 def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_eps, pad, length, pool_begin,
                         max_new_pools, pooled, q_idx, w, q_seq, q_pos, select_k, out_width, slot_map, rows,
                         topk, q, sm_scale, out, workspace, n_sel=None, tok=None, scores=None, lse=None,
-                        out_f32=None, pooled_codes=None, pooled_scales=None, cache_fp8=False, stop_after=0,
-                        stream=None) -> None:
+                        out_f32=None, pooled_codes=None, pooled_scales=None, cache_format=GLM_CACHE_INT8,
+                        stop_after=0, stream=None) -> None:
     """The whole step in one call: the arguments of glm_kv_store_int8, glm_kpool_build,
-    glm_index_topk_expand and glm_sparse_mla_decode (same tensors and rules); with cache_fp8 the
-    cache holds FP8 rows (uint8) and the step stores and attends as glm_kv_store_fp8 and
-    glm_sparse_mla_decode_fp8. stop_after = k (1..3) runs only the step's first k kernels."""
+    glm_index_topk_expand and glm_sparse_mla_decode (same tensors and rules); with cache_format
+    GLM_CACHE_FP8 / GLM_CACHE_FP4 the cache holds FP8 / 4-bit rows (uint8) and the step stores and
+    attends as glm_kv_store_fp8 / _fp4 and glm_sparse_mla_decode_fp8 / _fp4. stop_after = k (1..3)
+    runs only the step's first k kernels."""
     for t, dt, nm in ((latent, torch.bfloat16, "latent"), (slots, torch.int64, "slots"),
-                      (cache, torch.uint8 if cache_fp8 else torch.int8, "cache"),
+                      (cache, torch.int8 if cache_format == GLM_CACHE_INT8 else torch.uint8, "cache"),
                       (k, torch.bfloat16, "k"), (gate, torch.bfloat16, "gate"), (ln_w, torch.float32, "ln_w"),
                       (ln_b, torch.float32, "ln_b"), (pad, torch.int32, "pad"), (length, torch.int32, "len"),
                       (pool_begin, torch.int32, "pool_begin"), (pooled, torch.float32, "pooled"),
@@ -332,7 +349,7 @@ def glm_dsa_decode_step(dims, *, latent, slots, cache, k, gate, ln_w, ln_b, ln_e
     a.q_dev, a.sm_scale, a.out_dev = v(q), float(sm_scale), v(out)
     a.lse_dev, a.out_f32_dev = v(lse), v(out_f32)
     a.pooled_codes_dev, a.pooled_scales_dev = v(pooled_codes), v(pooled_scales)
-    a.cache_fp8 = 1 if cache_fp8 else 0
+    a.cache_format = int(cache_format)
     a.stop_after = int(stop_after)
     ws_bytes = 0 if workspace is None else workspace.numel()
     _check(lib.glm_dsa_decode_step(C.byref(dims), C.byref(a), _ptr(workspace), ws_bytes, _stream(stream)),
@@ -409,6 +426,21 @@ def glm_sparse_mla_decode_fp8(dims, q, cache, rows, sm_scale, out, workspace, ls
                                          rows.shape[0], rows.shape[1], float(sm_scale), _ptr(out),
                                          _ptr(lse), _ptr(out_f32), _ptr(workspace), workspace.numel(),
                                          _stream(stream)), "glm_sparse_mla_decode_fp8")
+
+
+def glm_sparse_mla_decode_fp4(dims, q, cache, rows, sm_scale, out, workspace, lse=None, out_f32=None,
+                              stream=None) -> None:
+    """glm_sparse_mla_decode over 4-bit rows: cache uint8 [n_rows, 304] (glm_kv_store_fp4)."""
+    for t, dt, nm in ((q, torch.bfloat16, "q"), (cache, torch.uint8, "cache"),
+                      (rows, torch.int32, "rows"), (out, torch.bfloat16, "out"),
+                      (workspace, torch.uint8, "workspace"), (lse, torch.float32, "lse"),
+                      (out_f32, torch.float32, "out_f32")):
+        _dev(t, dt, nm)
+    n_rows = cache.numel() // GLM_FP4_ROW_BYTES
+    _check(lib.glm_sparse_mla_decode_fp4(C.byref(dims), _ptr(q), _ptr(cache), n_rows, _ptr(rows),
+                                         rows.shape[0], rows.shape[1], float(sm_scale), _ptr(out),
+                                         _ptr(lse), _ptr(out_f32), _ptr(workspace), workspace.numel(),
+                                         _stream(stream)), "glm_sparse_mla_decode_fp4")
 
 
 # ------------------------------------------------------------------------------------------------

@@ -202,6 +202,14 @@ int glm_kv_store_fp8(const glm_dsa_dims *dims, const void *latent, const int64_t
                                              static_cast<cudaStream_t>(stream), num_sms()));
 }
 
+int glm_kv_store_fp4(const glm_dsa_dims *dims, const void *latent, const int64_t *slots,
+                     int64_t n, uint8_t *cache, int64_t n_rows, void *stream) {
+    const int rc = check_store(dims, latent, slots, n, reinterpret_cast<int8_t *>(cache), n_rows);
+    if (rc != GLM_OK || n == 0) return rc;
+    return cuda_status(glm::launch_store_fp4(latent, slots, n, cache, n_rows,
+                                             static_cast<cudaStream_t>(stream), num_sms()));
+}
+
 int glm_kpool_build(const glm_dsa_dims *dims, const void *k, const void *gate, int64_t ld_tokens,
                     const float *ln_w, const float *ln_b, float ln_eps, const int32_t *pad,
                     const int32_t *len, const int32_t *pool_begin, int32_t batch,
@@ -326,7 +334,6 @@ int enqueue_index_select(const void *q_idx, const float *w, const void *keys, co
     sel.n_sel = n_sel;
     sel.ghist = sw.hist;
     sel.ghist2 = sw.hist2;
-    sel.gsamp = sw.fine;
     sel.counters = sw.counters;
     sel.words = sw.words;
     sel.alist = sw.alist;
@@ -337,6 +344,7 @@ int enqueue_index_select(const void *q_idx, const float *w, const void *keys, co
     sel.out_width = out_width;
     sel.tok = tok;
     sel.rows = rows;
+    sel.gsamp = sw.fine;
     sel.early = new_pools >= 0 ? 1 : 0;   // new_pools < 0: wait for the preceding kernel at the start
     sel.new_pool_begin = new_pool_begin;
     sel.new_pools = new_pools >= 0 ? new_pools : 0;
@@ -470,10 +478,13 @@ int glm_expand_selection(const glm_dsa_dims *dims, const int32_t *topk, const in
                                           static_cast<cudaStream_t>(stream)));
 }
 
-int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t *cache,
-                          int64_t n_rows, const int32_t *rows, int32_t n_q, int32_t width,
-                          float sm_scale, void *out, float *lse, float *out_f32, void *workspace,
-                          size_t ws_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+// The split + combine of one sparse MLA call over rows of the given format.
+int sparse_mla_entry(const glm_dsa_dims *dims, const void *q, const int8_t *cache, int64_t n_rows,
+                     const int32_t *rows, int32_t n_q, int32_t width, float sm_scale, void *out, float *lse,
+                     float *out_f32, void *workspace, size_t ws_bytes, void *stream, int format) {
     int rc = check_mla(dims, q, cache, n_rows, rows, n_q, width, sm_scale, out, lse, out_f32);
     if (rc != GLM_OK || n_q == 0) return rc;
     const int H = dims->n_heads;
@@ -486,33 +497,37 @@ int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t 
     float *part_ml = reinterpret_cast<float *>(ws + mla_acc_bytes(parts));
     int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = cuda_status(glm::launch_mla_split_tc(plan, q, H, cache, n_rows, rows, n_q, width, sm_scale,
-                                              part_acc, part_ml, status, st));
+    rc = cuda_status(glm::launch_mla_split_tc(plan, q, H, cache, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml,
+                                              status, st, false, format));
     if (rc != GLM_OK) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32, lse, st));
+}
+}  // namespace
+
+extern "C" {
+
+int glm_sparse_mla_decode(const glm_dsa_dims *dims, const void *q, const int8_t *cache,
+                          int64_t n_rows, const int32_t *rows, int32_t n_q, int32_t width,
+                          float sm_scale, void *out, float *lse, float *out_f32, void *workspace,
+                          size_t ws_bytes, void *stream) {
+    return sparse_mla_entry(dims, q, cache, n_rows, rows, n_q, width, sm_scale, out, lse, out_f32, workspace,
+                            ws_bytes, stream, glm::kFmtInt8);
 }
 
 int glm_sparse_mla_decode_fp8(const glm_dsa_dims *dims, const void *q, const uint8_t *cache,
                               int64_t n_rows, const int32_t *rows, int32_t n_q, int32_t width,
                               float sm_scale, void *out, float *lse, float *out_f32, void *workspace,
                               size_t ws_bytes, void *stream) {
-    const int8_t *c8 = reinterpret_cast<const int8_t *>(cache);
-    int rc = check_mla(dims, q, c8, n_rows, rows, n_q, width, sm_scale, out, lse, out_f32);
-    if (rc != GLM_OK || n_q == 0) return rc;
-    const int H = dims->n_heads;
-    const size_t need = glm_dsa_workspace_size(dims, GLM_OP_SPARSE_MLA, n_q, 0, 0, width);
-    if (workspace == nullptr || ws_bytes < need || !aligned(workspace, 256)) return GLM_ERR_WORKSPACE;
-    const glm::MlaPlan plan = glm::mla_plan(n_q, H, width, num_sms());
-    const size_t parts = mla_parts(n_q, H, width);
-    char *ws = static_cast<char *>(workspace);
-    float *part_acc = reinterpret_cast<float *>(ws);
-    float *part_ml = reinterpret_cast<float *>(ws + mla_acc_bytes(parts));
-    int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    rc = cuda_status(glm::launch_mla_split_tc(plan, q, H, c8, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml,
-                                              status, st, false, true));
-    if (rc != GLM_OK) return rc;
-    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32, lse, st));
+    return sparse_mla_entry(dims, q, reinterpret_cast<const int8_t *>(cache), n_rows, rows, n_q, width, sm_scale,
+                            out, lse, out_f32, workspace, ws_bytes, stream, glm::kFmtFp8);
+}
+
+int glm_sparse_mla_decode_fp4(const glm_dsa_dims *dims, const void *q, const uint8_t *cache,
+                              int64_t n_rows, const int32_t *rows, int32_t n_q, int32_t width,
+                              float sm_scale, void *out, float *lse, float *out_f32, void *workspace,
+                              size_t ws_bytes, void *stream) {
+    return sparse_mla_entry(dims, q, reinterpret_cast<const int8_t *>(cache), n_rows, rows, n_q, width, sm_scale,
+                            out, lse, out_f32, workspace, ws_bytes, stream, glm::kFmtFp4);
 }
 
 int glm_cp_candidates(const float *scores, int64_t ld_scores, const int32_t *topk, int32_t n_q, int32_t select_k,
@@ -576,6 +591,7 @@ int glm_mla_v_up(const glm_dsa_dims *dims, const void *o_lat, const void *w_kv_b
 int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *workspace, size_t ws_bytes,
                         void *stream) {
     if (a == nullptr) return GLM_ERR_INVALID_ARG;
+    if (a->cache_format < GLM_CACHE_INT8 || a->cache_format > GLM_CACHE_FP4) return GLM_ERR_INVALID_ARG;
     const bool q8 = a->pooled_codes_dev != nullptr;   // the INT8 indexer state replaces pooled_dev
     const void *keys = q8 ? static_cast<const void *>(a->pooled_codes_dev) : static_cast<const void *>(a->pooled_dev);
     if (q8 && (!a->pooled_scales_dev || !aligned(a->pooled_scales_dev, 4))) return GLM_ERR_INVALID_ARG;
@@ -627,7 +643,7 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     p.codes = q8 ? a->pooled_codes_dev : nullptr;
     p.scales = q8 ? a->pooled_scales_dev : nullptr;
     p.ld_pools = a->ld_pools;
-    p.fp8 = a->cache_fp8 != 0 ? 1 : 0;
+    p.format = a->cache_format;
     p.zero = reinterpret_cast<uint4 *>(sw.hist);
     p.zero_n16 = idx_multi ? static_cast<int64_t>(align_up(sw.zero_bytes, 16) / 16) : 0;
     if (a->stop_after < 0 || a->stop_after > 3) return GLM_ERR_INVALID_ARG;
@@ -646,7 +662,7 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     float *part_acc = reinterpret_cast<float *>(ws + L.mla);
     float *part_ml = reinterpret_cast<float *>(ws + L.mla + mla_acc_bytes(parts));
     rc = cuda_status(glm::launch_mla_split_tc(plan, a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
-                                              a->sm_scale, part_acc, part_ml, status, st, true, a->cache_fp8 != 0));
+                                              a->sm_scale, part_acc, part_ml, status, st, true, a->cache_format));
     if (rc != GLM_OK || a->stop_after == 3) return rc;
     return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, plan.n_chunks, a->out_dev, a->out_f32_dev,
                                                a->lse_dev, st));

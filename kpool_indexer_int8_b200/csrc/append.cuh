@@ -4,6 +4,9 @@
 // axis per channel). Used by their own kernels and by the fused decode step's first kernel.
 #pragma once
 
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
 #include "common.cuh"
 
 namespace glm {
@@ -53,6 +56,22 @@ __device__ __forceinline__ uint32_t e4m3_code(float x) {
     return static_cast<uint32_t>(d) & 0xffu;
 }
 
+// Eight E2M1 codes (nearest value, ties to the even code, saturating at +-6, the sign kept; the
+// hardware conversion) packed low nibble first: v[0] in bits 0-3, v[1] in bits 4-7, ... (each
+// conversion puts its first operand in the high nibble of its byte).
+__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
 // The FP8 twin of store_int8_row (the FP8 latent cache of "GLM on CUDA", --kv-dtype fp8): the same
 // 528-byte row with E4M3 codes and scale = max(amax, 1e-4) / 448. One warp; every lane calls.
 __device__ __forceinline__ void store_fp8_row(const uint16_t *__restrict__ latent, const int64_t *__restrict__ slots,
@@ -85,6 +104,46 @@ __device__ __forceinline__ void store_fp8_row(const uint16_t *__restrict__ laten
     uint4 *dst = reinterpret_cast<uint4 *>(cache + slot * kRowBytes);
     dst[lane] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
     if (lane == 0) dst[32] = make_uint4(__float_as_uint(scale), 0u, 0u, 0u);
+}
+
+// The 4-bit row (the 4-bit latent cache of "GLM on CUDA", --kv-dtype fp4): E2M1 codes with one
+// E4M3 scale per 16 values and one fp32 scale per row, 304 bytes:
+//   s_row = max(amax, 1e-4) / 2688, e_k = E4M3(bmax_k / (6 s_row)), d_k = value(e_k) s_row,
+//   code = E2M1(x / d_k) (0 where d_k = 0), each step one IEEE fp32 operation; both conversions
+//   are the hardware's (nearest, ties to even, saturating). Lane l holds block l (dims 16 l ..).
+__device__ __forceinline__ void store_fp4_row(const uint16_t *__restrict__ latent, const int64_t *__restrict__ slots,
+                                              int64_t row, uint8_t *__restrict__ cache, int64_t n_rows) {
+    const int lane = threadIdx.x & 31;
+    const int64_t slot = slots[row];
+    if (slot < 0 || slot >= n_rows) return;  // padding (or outside the contract): no write
+    const uint4 *src = reinterpret_cast<const uint4 *>(latent + row * kLatent) + lane * 2;
+    uint4 v0 = __ldcs(src), v1 = __ldcs(src + 1);
+    uint32_t w[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+    float x[16];
+    float bmax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        x[2 * i] = __uint_as_float(w[i] << 16);
+        x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        bmax = fmaxf(bmax, fmaxf(fabsf(x[2 * i]), fabsf(x[2 * i + 1])));
+    }
+    const float amax = fmaxf(warp_max(bmax), 1e-4f);
+    const float s_row = __fdiv_rn(amax, 2688.0f);
+    const uint32_t e = e4m3_code(__fdiv_rn(bmax, __fmul_rn(6.0f, s_row)));
+    const __half_raw ev = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(e), __NV_E4M3);
+    const float d = __fmul_rn(__half2float(__half(ev)), s_row);
+    uint32_t packed[2];
+#pragma unroll
+    for (int i = 0; i < 2; i++) {
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; j++) v[j] = d > 0.0f ? __fdiv_rn(x[8 * i + j], d) : 0.0f;
+        packed[i] = e2m1x8(v);
+    }
+    uint8_t *dst = cache + slot * kFp4RowBytes;
+    reinterpret_cast<uint2 *>(dst)[lane] = make_uint2(packed[0], packed[1]);
+    dst[kFp4ScalesAt + lane] = static_cast<uint8_t>(e);
+    if (lane == 0) *reinterpret_cast<uint4 *>(dst + kFp4RowScaleAt) = make_uint4(__float_as_uint(s_row), 0u, 0u, 0u);
 }
 
 // Item `it` = (sequence b, i-th new pool) of a build (one warp; every lane calls). lw / lb: this

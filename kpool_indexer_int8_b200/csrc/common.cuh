@@ -47,6 +47,12 @@ namespace glm {
 
 constexpr int kLatent = 512;        // kv_lora_rank
 constexpr int kRowBytes = 528;      // 512 codes + fp32 scale + 12 zero bytes
+constexpr int kFp4RowBytes = 304;   // 256 code pairs + 32 E4M3 block scales + fp32 row scale + 12 zero bytes
+constexpr int kFp4ScalesAt = 256;   // the block scales (one per 16 values)
+constexpr int kFp4RowScaleAt = 288; // the row scale
+// The latent cache row formats: int8 codes, E4M3 codes (both 528 bytes, one fp32 scale), and
+// block-scaled E2M1 codes (304 bytes).
+enum CacheFormat { kFmtInt8 = 0, kFmtFp8 = 1, kFmtFp4 = 2 };
 constexpr int kIdxHeads = 32;       // indexer heads
 constexpr int kIdxDim = 128;        // indexer head dim
 constexpr int kKpool = 4;           // tokens per pool

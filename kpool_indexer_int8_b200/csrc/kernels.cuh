@@ -22,6 +22,8 @@ cudaError_t launch_store_int8(const void *latent, const int64_t *slots, int64_t 
                               int64_t n_rows, cudaStream_t stream, int num_sms);
 cudaError_t launch_store_fp8(const void *latent, const int64_t *slots, int64_t n, uint8_t *cache,
                              int64_t n_rows, cudaStream_t stream, int num_sms);
+cudaError_t launch_store_fp4(const void *latent, const int64_t *slots, int64_t n, uint8_t *cache,
+                             int64_t n_rows, cudaStream_t stream, int num_sms);
 cudaError_t launch_kpool_build(const void *k, const void *gate, int64_t ld_tokens,
                                const float *ln_w, const float *ln_b, float eps,
                                const int32_t *pad, const int32_t *len, const int32_t *pool_begin,
@@ -88,7 +90,7 @@ struct StepPrepArgs {
     int64_t ld_pools;
     uint4 *zero;
     int64_t zero_n16;
-    int fp8;                       // the cache holds FP8 rows
+    int format;                    // CacheFormat of the cache rows
 };
 cudaError_t launch_step_prep(const StepPrepArgs &a, cudaStream_t stream);
 

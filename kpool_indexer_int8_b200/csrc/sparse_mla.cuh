@@ -22,7 +22,7 @@ cudaError_t launch_mla_split_tc(const MlaPlan &plan, const void *q, int n_heads,
                                 const int32_t *rows, int n_q, int width, float sm_scale,
                                 float *part_acc, float *part_ml, int *status, cudaStream_t stream,
                                 bool early_q = false,    // early_q: stage q before waiting on the previous kernel
-                                bool fp8 = false);       // fp8: the rows hold E4M3 codes (the FP8 latent cache)
+                                int format = 0);         // CacheFormat of the rows (int8, fp8 or 4-bit)
 // poison (or null): a status word the split kernel sets on a timed-out wait; when it is nonzero
 // the combine writes NaN to every output instead of merging (used where the caller cannot read it).
 cudaError_t launch_mla_combine(const float *part_acc, const float *part_ml, int n_q, int n_heads,

@@ -13,9 +13,10 @@
 //   2. gather: every thread requests its 16-byte pieces of the chunk's rows at once (all of a
 //      chunk's loads in flight together: one round trip), and the row scales; while they are in
 //      flight the query block is staged; the codes are then widened in registers to fp16 (exact:
-//      |code| <= 127; E4M3 codes are exact in fp16 as well) and stored as a tile C[ROWS x 512] of
-//      8x8 core matrices -- the int8 codes through byte permutes and one packed subtraction
-//      (1024 + code + 128 built as fp16 bits, minus 1152), no integer conversions;
+//      |code| <= 127; E4M3 codes are exact in fp16 as well; a 4-bit row's E2M1 code times its
+//      E4M3 block scale too) and stored as a tile C[ROWS x 512] of 8x8 core matrices -- the int8
+//      codes through byte permutes and one packed subtraction (1024 + code + 128 built as fp16
+//      bits, minus 1152), no integer conversions;
 //   3. S^T = C . Q^T on tcgen05 (kind::f16, fp32 accumulator in tensor memory: lane = row,
 //      column = head), 32 MMAs of K = 16;
 //   4. softmax over the chunk's rows for each head: one thread per row and half of the heads;
@@ -71,6 +72,20 @@ __device__ __forceinline__ void codes_to_f16x4(uint32_t w, uint32_t &lo, uint32_
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(lo) : "r"(a), "r"(0x64806480u));   // - 1152 (exact)
     asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(hi) : "r"(b), "r"(0x64806480u));
 }
+// Eight E2M1 codes (one word, low nibble first) as eight fp16 values times the fp16 block scale
+// sc2 (in both halves): exact, since a 2-bit by 4-bit significand product of magnitude in
+// [2^-10, 2688] is an fp16 normal.
+__device__ __forceinline__ void fp4_to_f16x8(uint32_t w, uint32_t sc2, uint32_t (&o)[4]) {
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+        : "=r"(o[0]), "=r"(o[1]), "=r"(o[2]), "=r"(o[3]) : "r"(w));
+#pragma unroll
+    for (int i = 0; i < 4; i++) asm("mul.rn.f16x2 %0, %0, %1;" : "+r"(o[i]) : "r"(sc2));
+}
 // Four E4M3 codes as four exact fp16 values (hardware conversion of code pairs).
 __device__ __forceinline__ void fp8_to_f16x4(uint32_t w, uint32_t &lo, uint32_t &hi) {
     const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xffffu), __NV_E4M3);
@@ -94,12 +109,16 @@ __device__ __forceinline__ void tmem_ld_v(uint32_t taddr, uint32_t (&r)[V]) {
     else tc::tmem_ld32(taddr, r);
 }
 
-template <int ROWS, int NH, bool kFp8>
+template <int ROWS, int NH, int kFmt>
 __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
     const uint16_t *__restrict__ q, int n_heads, const uint8_t *__restrict__ cache, int64_t n_rows,
     const int32_t *__restrict__ rows, int width, float sm_scale, int n_chunks, int n_hg,
     float *__restrict__ part_acc, float *__restrict__ part_ml, int *__restrict__ status, int early_q) {
     using L = MlaLayout<ROWS, NH>;
+    constexpr bool kFp4 = kFmt == kFmtFp4;
+    constexpr int kRowB = kFp4 ? kFp4RowBytes : kRowBytes;      // bytes of a cache row
+    constexpr int kSclAt = kFp4 ? kFp4RowScaleAt : kLatent;     // where its fp32 row scale sits
+    constexpr int kPieces = kFp4 ? 16 : 32;                     // 16-byte pieces of codes in a row
     constexpr int V = NH / 2;             // heads per softmax thread
     constexpr int kLboP = 32 * NH;        // P': bytes between row groups (2 NH / 8 head groups x 128 B)
     // early_q: the query block is an input no preceding kernel writes (the one-call step), so its
@@ -163,26 +182,32 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
         return;
     }
 
-    // 3. gather: every 16-code piece of the chunk's rows and every row scale is requested at once
-    //    (piece P: row 8 rg + (P & 7), codes 16 k .. 16 k + 15; eight lanes hold eight rows of one
-    //    piece index, so that the widened lines they store are 128 contiguous bytes)
-    constexpr int kCvt = ROWS * 32 / kMlaThreads;
+    // 3. gather: every 16-byte piece of codes of the chunk's rows (and, for 4-bit rows, the two
+    //    block scales of the piece) and every row scale is requested at once (piece P: row
+    //    8 rg + (P & 7), piece k of the row; eight lanes hold eight rows of one piece index, so
+    //    that the widened lines they store are 128 contiguous bytes)
+    constexpr int kCvt = ROWS * kPieces / kMlaThreads;
     uint4 gv[kCvt];
+    uint32_t es[kFp4 ? kCvt : 1];
 #pragma unroll
     for (int it = 0; it < kCvt; it++) {
         const int P = it * kMlaThreads + tid;
         const int jl = P & 7, klo = (P >> 3) & 3, rest = P >> 5;
         const int rg = rest % (ROWS / 8), k = (rest / (ROWS / 8)) * 4 + klo;
         const int r = ridx[rg * 8 + jl];
-        gv[it] = r >= 0 ? __ldg(reinterpret_cast<const uint4 *>(cache + static_cast<int64_t>(r) * kRowBytes) + k)
-                        : make_uint4(0u, 0u, 0u, 0u);
+        const uint8_t *rp = cache + static_cast<int64_t>(r) * kRowB;
+        gv[it] = r >= 0 ? __ldg(reinterpret_cast<const uint4 *>(rp) + k) : make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (kFp4)
+            es[it] = r >= 0 ? __ldg(reinterpret_cast<const uint16_t *>(rp + kFp4ScalesAt) + k) : 0u;
     }
-    const float my_scale = myrow >= 0 ? __ldg(reinterpret_cast<const float *>(cache + static_cast<int64_t>(myrow) * kRowBytes + kLatent)) : 0.0f;
+    const float my_scale = myrow >= 0 ? __ldg(reinterpret_cast<const float *>(cache + static_cast<int64_t>(myrow) * kRowB + kSclAt)) : 0.0f;
+    GLM_TL(glm_tl_split, 9);
     if (warp == 0) {
         tc::tmem_alloc(tc::smem_addr(&words[1]), 8 * NH);
         tc::tmem_relinquish();
         tc::fence_before_sync();
     }
+    GLM_TL(glm_tl_split, 10);
     if (tid == 32) {
         tc::mbar_init(bar_s, 1);
         tc::mbar_init(bar_o, 1);
@@ -198,8 +223,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
 #pragma unroll
         for (int e = 0; e < 4; e++) mx = max(mx, max(w4[e] & 0x7fffu, (w4[e] >> 16) & 0x7fffu));
     }
+    GLM_TL(glm_tl_split, 11);
     if (qreal) atomicMax(&qmax[qh], mx);
     __syncthreads();
+    GLM_TL(glm_tl_split, 12);
     {
         const unsigned m = qmax[qh];
         int e = 0;
@@ -239,8 +266,23 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_split_tc_kernel(
         const int jl = P & 7, klo = (P >> 3) & 3, rest = P >> 5;
         const int rg = rest % (ROWS / 8), k = (rest / (ROWS / 8)) * 4 + klo;
         const uint4 w = gv[it];
+        if constexpr (kFp4) {   // 32 codes: dim groups 4 k .. 4 k + 3 (block scales 2 k and 2 k + 1)
+            const __half2_raw sc = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(es[it]), __NV_E4M3);
+            const uint32_t s0 = static_cast<uint32_t>(sc.x) * 0x10001u, s1 = static_cast<uint32_t>(sc.y) * 0x10001u;
+            uint32_t o0[4], o1[4], o2[4], o3[4];
+            fp4_to_f16x8(w.x, s0, o0);
+            fp4_to_f16x8(w.y, s0, o1);
+            fp4_to_f16x8(w.z, s1, o2);
+            fp4_to_f16x8(w.w, s1, o3);
+            unsigned char *line = Cs + rg * 8192 + (4 * k) * 128 + jl * 16;
+            *reinterpret_cast<uint4 *>(line) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+            *reinterpret_cast<uint4 *>(line + 128) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+            *reinterpret_cast<uint4 *>(line + 256) = make_uint4(o2[0], o2[1], o2[2], o2[3]);
+            *reinterpret_cast<uint4 *>(line + 384) = make_uint4(o3[0], o3[1], o3[2], o3[3]);
+            continue;
+        }
         uint32_t o[8];
-        if (kFp8) {
+        if (kFmt == kFmtFp8) {
             fp8_to_f16x4(w.x, o[0], o[1]);
             fp8_to_f16x4(w.y, o[2], o[3]);
             fp8_to_f16x4(w.z, o[4], o[5]);
@@ -414,11 +456,11 @@ MlaPlan mla_plan(int n_q, int n_heads, int width, int num_sms) {
     return p;
 }
 
-template <int ROWS, int NH, bool kFp8>
+template <int ROWS, int NH, int kFmt>
 cudaError_t launch_t(const MlaPlan &p, const void *q, int n_heads, const uint8_t *cache, int64_t n_rows,
                      const int32_t *rows, int n_q, int width, float sm_scale, float *part_acc, float *part_ml,
                      int *status, cudaStream_t stream, bool early_q) {
-    auto kernel = mla_split_tc_kernel<ROWS, NH, kFp8>;
+    auto kernel = mla_split_tc_kernel<ROWS, NH, kFmt>;
     const int smem = MlaLayout<ROWS, NH>::kBytes;
     cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
@@ -431,16 +473,18 @@ cudaError_t launch_t(const MlaPlan &p, const void *q, int n_heads, const uint8_t
 cudaError_t launch_mla_split_tc(const MlaPlan &p, const void *q, int n_heads, const int8_t *cache, int64_t n_rows,
                                 const int32_t *rows, int n_q, int width, float sm_scale,
                                 float *part_acc, float *part_ml, int *status, cudaStream_t stream, bool early_q,
-                                bool fp8) {
+                                int format) {
     const uint8_t *c8 = reinterpret_cast<const uint8_t *>(cache);
-#define GLM_MLA_LAUNCH(R, H)                                                                                       \
-    if (p.rows == R && p.heads == H)                                                                             \
-        return fp8 ? launch_t<R, H, true>(p, q, n_heads, c8, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml, \
-                                          status, stream, early_q)                                               \
-                   : launch_t<R, H, false>(p, q, n_heads, c8, n_rows, rows, n_q, width, sm_scale, part_acc,         \
-                                           part_ml, status, stream, early_q);
-    GLM_MLA_LAUNCH(64, 16)
-    GLM_MLA_LAUNCH(64, 64)
+#define GLM_MLA_LAUNCH(R, H, F)                                                                                  \
+    if (p.rows == R && p.heads == H && format == F)                                                              \
+        return launch_t<R, H, F>(p, q, n_heads, c8, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml, status, \
+                                 stream, early_q);
+    GLM_MLA_LAUNCH(64, 16, kFmtInt8)
+    GLM_MLA_LAUNCH(64, 64, kFmtInt8)
+    GLM_MLA_LAUNCH(64, 16, kFmtFp8)
+    GLM_MLA_LAUNCH(64, 64, kFmtFp8)
+    GLM_MLA_LAUNCH(64, 16, kFmtFp4)
+    GLM_MLA_LAUNCH(64, 64, kFmtFp4)
 #undef GLM_MLA_LAUNCH
     return cudaErrorInvalidValue;
 }

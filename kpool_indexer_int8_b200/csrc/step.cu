@@ -1,5 +1,6 @@
-// step.cu -- the first kernel of a fused decode step: the int8 store of the new latent rows
-// ("GLM-5.3 Kernels" README, 'Included': titan_kv.store_int8), the build of the new pools
+// step.cu -- the first kernel of a fused decode step: the store of the new latent rows ("GLM-5.3
+// Kernels" README, 'Included': titan_kv.store_int8; or the FP8 or 4-bit row of "GLM on CUDA",
+// --kv-dtype fp8 / fp4), the build of the new pools
 // ("Module glm5next_dsa_ref", pool_states) and the zeroing of the step's cross-CTA counters, as
 // three independent groups of CTAs of one launch (one warp per row, one warp per pool, 64 bytes
 // per thread of zeros), so that the three short jobs overlap instead of following one another.
@@ -24,7 +25,8 @@ __global__ void __launch_bounds__(kPrepThreads) step_prep_kernel(StepPrepArgs a,
     if (cta < store_ctas) {
         const int64_t row = static_cast<int64_t>(cta) * kPrepWarps + warp;
         if (row < a.n_new) {
-            if (a.fp8) store_fp8_row(a.latent, a.slots, row, reinterpret_cast<uint8_t *>(a.cache), a.n_rows);
+            if (a.format == kFmtFp8) store_fp8_row(a.latent, a.slots, row, reinterpret_cast<uint8_t *>(a.cache), a.n_rows);
+            else if (a.format == kFmtFp4) store_fp4_row(a.latent, a.slots, row, reinterpret_cast<uint8_t *>(a.cache), a.n_rows);
             else store_int8_row(a.latent, a.slots, row, a.cache, a.n_rows);
         }
         return;

@@ -19,10 +19,11 @@ from typing import Optional
 
 import torch
 
-from . import (GLM_OP_DECODE_STEP, GLM_OP_INDEX_SCORES_TOPK, GLM_OP_SPARSE_MLA, GLM_ROW_BYTES,
-               glm_dsa_decode_step, glm_dsa_workspace_size, glm_expand_selection, glm_index_scores_topk,
-               glm_index_topk_expand, glm_index_topk_expand_q8, glm_kpool_build, glm_kpool_build_q8, glm_kv_store_fp8,
-               glm_kv_store_int8, glm_sparse_mla_decode, glm_sparse_mla_decode_fp8, make_dims)
+from . import (GLM_CACHE_FP4, GLM_CACHE_FP8, GLM_CACHE_INT8, GLM_FP4_ROW_BYTES, GLM_OP_DECODE_STEP,
+               GLM_OP_INDEX_SCORES_TOPK, GLM_OP_SPARSE_MLA, GLM_ROW_BYTES, glm_dsa_decode_step, glm_dsa_workspace_size,
+               glm_expand_selection, glm_index_scores_topk, glm_index_topk_expand, glm_index_topk_expand_q8,
+               glm_kpool_build, glm_kpool_build_q8, glm_kv_store_fp4, glm_kv_store_fp8, glm_kv_store_int8,
+               glm_sparse_mla_decode, glm_sparse_mla_decode_fp4, glm_sparse_mla_decode_fp8, make_dims)
 
 LATENT = 512
 IDX_HEADS = 32
@@ -73,12 +74,17 @@ class DecodeBuffers:
     pooled_codes: Optional[torch.Tensor] = None   # INT8 indexer state: int8 [B, ld_pools, 128]
     pooled_scales: Optional[torch.Tensor] = None  #                       fp32 [B, ld_pools]
     fp8: bool = False                             # the cache holds FP8 rows (uint8)
+    fp4: bool = False                             # the cache holds 4-bit rows (uint8 [n_rows, 304])
+
+    @property
+    def cache_format(self) -> int:
+        return GLM_CACHE_FP4 if self.fp4 else GLM_CACHE_FP8 if self.fp8 else GLM_CACHE_INT8
 
 
 def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_new: int,
              select_k: int, out_width: int, sm_scale: float, ln_eps: float, max_new_pools: int,
              device, keep_scores: bool = False, keep_f32: bool = False, q8: bool = False,
-             fp8: bool = False) -> DecodeBuffers:
+             fp8: bool = False, fp4: bool = False) -> DecodeBuffers:
     dims = make_dims(n_heads)
     ld_pools = max(1, ld_tokens // KPOOL)
     f = dict(device=device)
@@ -87,8 +93,9 @@ def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_
     ws_s = glm_dsa_workspace_size(dims, GLM_OP_DECODE_STEP, n_q, ld_pools, select_k, out_width)
     return DecodeBuffers(
         dims=dims, select_k=select_k, out_width=out_width, sm_scale=sm_scale, ln_eps=ln_eps,
-        cache=torch.zeros(n_rows, GLM_ROW_BYTES, dtype=torch.uint8 if fp8 else torch.int8, **f),
-        fp8=fp8,
+        cache=torch.zeros(n_rows, GLM_FP4_ROW_BYTES if fp4 else GLM_ROW_BYTES,
+                          dtype=torch.uint8 if (fp8 or fp4) else torch.int8, **f),
+        fp8=fp8, fp4=fp4,
         pooled=torch.zeros(batch, ld_pools, IDX_DIM, dtype=torch.float32, **f),
         k=torch.zeros(batch, ld_tokens, IDX_DIM, dtype=torch.bfloat16, **f),
         gate=torch.zeros(batch, ld_tokens, IDX_DIM, dtype=torch.bfloat16, **f),
@@ -123,6 +130,9 @@ def allocate(n_heads: int, batch: int, ld_tokens: int, n_rows: int, n_q: int, n_
 
 
 def store(b: DecodeBuffers, stream=None) -> None:
+    if b.fp4:
+        glm_kv_store_fp4(b.dims, b.new_latent, b.new_slots, b.cache, stream=stream)
+        return
     if b.fp8:
         glm_kv_store_fp8(b.dims, b.new_latent, b.new_slots, b.cache, stream=stream)
         return
@@ -167,6 +177,10 @@ def index_topk_expand(b: DecodeBuffers, stream=None) -> None:
 
 
 def attend(b: DecodeBuffers, stream=None) -> None:
+    if b.fp4:
+        glm_sparse_mla_decode_fp4(b.dims, b.q, b.cache, b.rows, b.sm_scale, b.out, b.ws_mla, lse=b.lse,
+                                  out_f32=b.out_f32, stream=stream)
+        return
     if b.fp8:
         glm_sparse_mla_decode_fp8(b.dims, b.q, b.cache, b.rows, b.sm_scale, b.out, b.ws_mla, lse=b.lse,
                                   out_f32=b.out_f32, stream=stream)
@@ -194,4 +208,4 @@ def run_step(b: DecodeBuffers, stream=None, stop_after: int = 0) -> None:
                         slot_map=b.slot_map, rows=b.rows, topk=b.topk, q=b.q, sm_scale=b.sm_scale, out=b.out,
                         workspace=b.ws_step, n_sel=b.n_sel, tok=b.tok, scores=b.scores, lse=b.lse,
                         out_f32=b.out_f32, pooled_codes=b.pooled_codes, pooled_scales=b.pooled_scales,
-                        cache_fp8=b.fp8, stop_after=stop_after, stream=stream)
+                        cache_format=b.cache_format, stop_after=stop_after, stream=stream)

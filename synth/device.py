@@ -30,14 +30,15 @@ def step_split(inp: Inputs):
     return (inp.len - n_new_seq).astype(np.int32), np.nonzero(new)[0]
 
 
-def allocate_for(inp: Inputs, device, keep_scores=False, keep_f32=False, q8=False, fp8=False) -> P.DecodeBuffers:
+def allocate_for(inp: Inputs, device, keep_scores=False, keep_f32=False, q8=False, fp8=False,
+                 fp4=False) -> P.DecodeBuffers:
     prefix, new_idx = step_split(inp)
     per_seq_new = int(max(1, (inp.len - prefix).max()))
     max_new_pools = per_seq_new // P.KPOOL + 1
     return P.allocate(inp.wl.n_heads, inp.wl.batch, inp.ld_tokens, inp.n_rows, len(inp.q_pos),
                       len(new_idx), inp.wl.select_k, inp.wl.out_width, inp.sm_scale,
                       inp.wl.ln_eps, max_new_pools, device, keep_scores=keep_scores,
-                      keep_f32=keep_f32, q8=q8, fp8=fp8)
+                      keep_f32=keep_f32, q8=q8, fp8=fp8, fp4=fp4)
 
 
 def load(inp: Inputs, b: P.DecodeBuffers, build_prefix: bool = True) -> None:
@@ -68,8 +69,9 @@ def load(inp: Inputs, b: P.DecodeBuffers, build_prefix: bool = True) -> None:
             sl = idx[s:s + step]
             lat = _t(inp.latent[sl], torch.bfloat16, dev)
             slots = _t(inp.slots[sl], torch.int64, dev)
-            from kpool_indexer_int8_b200 import glm_kv_store_fp8, glm_kv_store_int8
-            (glm_kv_store_fp8 if b.fp8 else glm_kv_store_int8)(b.dims, lat, slots, b.cache)
+            from kpool_indexer_int8_b200 import glm_kv_store_fp4, glm_kv_store_fp8, glm_kv_store_int8
+            store = glm_kv_store_fp4 if b.fp4 else glm_kv_store_fp8 if b.fp8 else glm_kv_store_int8
+            store(b.dims, lat, slots, b.cache)
             del lat, slots
         plen = _t(prefix, torch.int32, dev)
         P.build_pools(b, length=plen, pool_begin=torch.zeros_like(b.pool_begin),

@@ -168,6 +168,27 @@ def test_fp8_entry_points_reject_before_launch():
                                        1 << 30, None) == kp.GLM_ERR_INVALID_ARG
 
 
+def test_fp4_entry_points_reject_before_launch():
+    L = kp.lib
+    d = C.byref(kp.make_dims(64))
+    bad = C.byref(kp.make_dims(64, qk_rope_head_dim=64))
+    assert L.glm_kv_store_fp4(bad, FAKE, FAKE, 1, FAKE, 1, None) == kp.GLM_ERR_UNSUPPORTED
+    assert L.glm_kv_store_fp4(d, None, FAKE, 1, FAKE, 1, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kv_store_fp4(d, FAKE, FAKE, 1, MIS, 1, None) == kp.GLM_ERR_INVALID_ARG
+    assert L.glm_kv_store_fp4(d, None, None, 0, None, 0, None) == kp.GLM_OK        # n == 0: no-op
+    assert L.glm_sparse_mla_decode_fp4(bad, FAKE, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None, FAKE,
+                                       1 << 30, None) == kp.GLM_ERR_UNSUPPORTED
+    assert L.glm_sparse_mla_decode_fp4(d, FAKE, FAKE, 10, FAKE, 1, 64, 0.04, FAKE, None, None, FAKE, 16,
+                                       None) == kp.GLM_ERR_WORKSPACE
+    assert L.glm_sparse_mla_decode_fp4(d, FAKE, MIS, 10, FAKE, 1, 64, 0.04, FAKE, None, None, FAKE,
+                                       1 << 30, None) == kp.GLM_ERR_INVALID_ARG
+    # a cache format other than int8, fp8 and fp4 is rejected before anything else is looked at
+    a = kp.glm_dsa_step()
+    for fmt in (-1, 3):
+        a.cache_format = fmt
+        assert L.glm_dsa_decode_step(d, C.byref(a), FAKE, 1 << 30, None) == kp.GLM_ERR_INVALID_ARG
+
+
 def test_noalloc_entry_rejects_before_launch():
     # the allocation-free MLA entry point runs the workspace entry's checks: every rejection below
     # happens on the host, before its scratch is looked up or anything is enqueued

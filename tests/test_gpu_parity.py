@@ -452,16 +452,17 @@ def test_sparse_mla_matches_oracle(cuda, n_heads, W, n_valid, n_rows):
             np.testing.assert_allclose(lg[n], lo, atol=1e-3, rtol=0)
 
 
-@pytest.mark.parametrize("fp8", [False, True])
-def test_sparse_mla_many_queries_matches_oracle(cuda, fp8):
+@pytest.mark.parametrize("fmt", ["int8", "fp8", "fp4"])
+def test_sparse_mla_many_queries_matches_oracle(cuda, fmt):
     """Enough queries that the split kernel takes its many-query plan (64-entry chunks, all heads
     of a query in one CTA) instead of the few-query one (128-entry chunks, 16 heads per CTA)."""
-    rng = np.random.default_rng(77 + fp8)
+    rng = np.random.default_rng(77 + ["int8", "fp8", "fp4"].index(fmt))
     n_heads, W, n_rows, nq = 64, 2176, 4000, 24
     lat = synth.f32_to_bf16_bits(rng.standard_normal((n_rows, 512)).astype(np.float32))
     lat[rng.random(n_rows) < 0.01] = synth.f32_to_bf16_bits(rng.standard_normal((1, 512)).astype(np.float32) * 8)
-    cache = np.zeros((n_rows, 528), np.uint8 if fp8 else np.int8)
-    (oracle.store_fp8 if fp8 else oracle.store_int8)(lat, np.arange(n_rows, dtype=np.int64), cache)
+    cache = np.zeros((n_rows, 304 if fmt == "fp4" else 528), np.int8 if fmt == "int8" else np.uint8)
+    {"int8": oracle.store_int8, "fp8": oracle.store_fp8, "fp4": oracle.store_fp4}[fmt](
+        lat, np.arange(n_rows, dtype=np.int64), cache)
     rows = np.full((nq, W), -1, np.int32)
     for n in range(nq):
         nv = [2051, 0, 5, 1000, 64, 2176][n % 6]
@@ -478,7 +479,8 @@ def test_sparse_mla_many_queries_matches_oracle(cuda, fp8):
     out = torch.full((nq, n_heads, 512), 7.0, dtype=torch.bfloat16, device=cuda)
     o32 = torch.full((nq, n_heads, 512), 7.0, dtype=torch.float32, device=cuda)
     lse = torch.full((nq, n_heads), 7.0, dtype=torch.float32, device=cuda)
-    fn = kp.glm_sparse_mla_decode_fp8 if fp8 else kp.glm_sparse_mla_decode
+    fn = {"int8": kp.glm_sparse_mla_decode, "fp8": kp.glm_sparse_mla_decode_fp8,
+          "fp4": kp.glm_sparse_mla_decode_fp4}[fmt]
     fn(dims, to_dev(q, torch.bfloat16, cuda), torch.from_numpy(cache).to(cuda), to_dev(rows, torch.int32, cuda), sm,
        out, ws, lse=lse, out_f32=o32)
     og, g32, lg = np_(out.view(torch.int16)).view(np.uint16), np_(o32), np_(lse)
@@ -488,8 +490,8 @@ def test_sparse_mla_many_queries_matches_oracle(cuda, fp8):
         if not (rows[n] >= 0).any():
             assert np.isneginf(lg[n]).all() and not g32[n].any()
             continue
-        if fp8:
-            c = oracle.dequant_rows_fp8(cache, rows[n][rows[n] >= 0])
+        if fmt != "int8":
+            c = (oracle.dequant_rows_fp8 if fmt == "fp8" else oracle.dequant_rows_fp4)(cache, rows[n][rows[n] >= 0])
             assert_attention_close(g32[n], oracle.attention_f64(qf[n], c, c, sm, shared=True), f"query {n}")
             continue
         oo, lo = oracle.sparse_mla(q[n], cache, rows[n], sm)
