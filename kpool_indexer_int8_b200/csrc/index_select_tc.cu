@@ -7,7 +7,8 @@
 // Grid (G, n_q): CTA g of query n owns a contiguous range of the query's visible pools.
 // Phase 1, scoring -- a warp-specialised pipeline over chunks of 64 pools, every hand-off an mbarrier:
 //   * producer (warp 0): one 1-D bulk copy per chunk (64 pool rows, 32 KB, contiguous) into a ring
-//     of 5 slots (up to ~128 KB per SM in flight);
+//     of 4 slots (128 KB per SM in flight: a fifth slot streamed no faster and made the CTAs'
+//     later round trips, which queue behind the bulk data bound for the same SM, slower);
 //   * converters (warps 8-15, 8 pool rows of a chunk each): every warp first reads its rows into
 //     registers (lane l: dims 4 l .. 4 l + 3 of a row), the warps meet on an mbarrier, and each
 //     then rewrites its rows in place as two fp16 terms in the 128-byte swizzle layout: the row
@@ -58,11 +59,12 @@ GLM_TL_TABLE(glm_tl_index)
 
 constexpr int kIxThreads = 512;                        // 16 warps, see the roles above
 constexpr int kIxTile = 64;                            // pools per chunk (UMMA M)
-constexpr int kIxSlots = 5;                            // staging slots, converted in place
+constexpr int kIxSlots = 4;                            // staging slots, converted in place
 constexpr int kIxSlotBytes = kIxTile * kIdxDim * 4;    // 32 KB: 64 fp32 pool rows
 constexpr int kIxConv = 8;                             // converter warps (8 rows of a chunk each)
 constexpr int kIxAtomBytes = kIxTile * 128;            // 8 KB: one 64-dim K atom of an fp16 term
 constexpr int kIxTermBytes = 2 * kIxAtomBytes;         // 16 KB: one fp16 term of a chunk
+static_assert(kIxSlots <= 5, "the barrier table holds five slots");
 constexpr int kIxPsDepth = kIxSlots + 2;               // ring of the pools' score factors (see converters)
 constexpr uint32_t kIxWaitLimit = 1u << 22;
 
@@ -71,7 +73,7 @@ constexpr int kIxSampleTiles = 8;                      // most chunks of a CTA's
 constexpr int kIxSampleMax = kIxSampleTiles * kIxTile;
 
 struct IxLayout {                                      // offsets from a 1024-byte aligned base
-    static constexpr int kSlots = 0;                                  // [5][32 KB]
+    static constexpr int kSlots = 0;                                  // [kIxSlots][32 KB]
     static constexpr int kQ = kSlots + kIxSlots * kIxSlotBytes;       // 32 heads x 128 dims fp16
     static constexpr int kHist = kQ + kIdxHeads * kIdxDim * 2;        // 2048 uint32
     static constexpr int kLocal = kHist + kHistBins * 4;              // kIxLocalCap fp32 scores
@@ -96,10 +98,10 @@ constexpr int kFlThr = 0;       // the sample threshold: a candidate's key is at
 constexpr int kFlWait = 1;      // a wait on the query's other CTAs gave up
 
 // mbarrier indices
-constexpr int kBarStFull = 0;     // [5] slot filled (producer, tx bytes)
-constexpr int kBarStRead = 5;     // [5] slot read into registers (8 converter warps)
-constexpr int kBarStConv = 10;    // [5] slot converted in place (8 converter warps)
-constexpr int kBarStEmpty = 15;   // [5] slot read by the MMAs (commit)
+constexpr int kBarStFull = 0;     // [kIxSlots <= 5] slot filled (producer, tx bytes)
+constexpr int kBarStRead = 5;     // [kIxSlots] slot read into registers (8 converter warps)
+constexpr int kBarStConv = 10;    // [kIxSlots] slot converted in place (8 converter warps)
+constexpr int kBarStEmpty = 15;   // [kIxSlots] slot read by the MMAs (commit)
 constexpr int kBarAccFull = 20;   // [2] accumulator ready (commit)
 constexpr int kBarAccEmpty = 22;  // [2] accumulator read (4 epilogue warps)
 constexpr int kBarSample = 24;    // the sample keys are in shared memory (2 epilogue warps)

@@ -168,3 +168,29 @@ def test_fp4_step_equals_separate_calls_and_stores_the_oracles_rows(cuda):
         valid = rows[n][rows[n] >= 0]
         cr = oracle.dequant_rows_fp4(want, valid)
         assert_attention_close(o32[n], oracle.attention_f64(qf[n], cr, cr, inp.sm_scale, shared=True), n)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "fp4"])
+def test_long_decode_full_size_on_fp8_and_fp4_rows(cuda, fmt):
+    # the benchmark's long-decode workload (262,144 tokens, 65,536 pools) through the one-call step
+    # with FP8 or 4-bit cache rows: every stored row equals the oracle's, the selection and
+    # expansion the oracle's (the index path does not depend on the row format), the attention
+    # the oracle's fp64 attention over the dequantised rows it selected
+    from kpool_indexer_int8_b200 import pipeline as P
+    from synth import device as sdev
+    inp = synth.generate(synth.LONG_DECODE)
+    b = sdev.allocate_for(inp, cuda, keep_scores=True, keep_f32=True, fp8=fmt == "fp8", fp4=fmt == "fp4")
+    sdev.load(inp, b, build_prefix=True)
+    b.out_f32.fill_(3.0)
+    P.run_step(b)
+    torch.cuda.synchronize()
+    want = np.zeros(tuple(b.cache.shape), np.uint8)
+    (oracle.store_fp8 if fmt == "fp8" else oracle.store_fp4)(inp.latent, inp.slots, want)
+    assert np.array_equal(np_(b.cache), want)
+    ref = oracle.decode_query(inp, 0, oracle.build_cache(inp), oracle.build_pools(inp))
+    assert np.array_equal(np_(b.topk)[0], ref["topk"])
+    assert np.array_equal(np_(b.tok)[0], ref["tok"]) and np.array_equal(np_(b.rows)[0], ref["rows"])
+    valid = ref["rows"][ref["rows"] >= 0]
+    c = (oracle.dequant_rows_fp8 if fmt == "fp8" else oracle.dequant_rows_fp4)(want, valid)
+    qf = synth.bf16_bits_to_f32(inp.q[0]).astype(np.float64)
+    assert_attention_close(np_(b.out_f32)[0], oracle.attention_f64(qf, c, c, inp.sm_scale, shared=True), fmt)
