@@ -191,9 +191,17 @@ int glm_kpool_build_q8(const glm_dsa_dims *dims, const void *k_dev, const void *
  *               Its last 256 bytes start with a status word set nonzero if a wait gave up (on the
  *               tensor cores, or of the CTAs of one query for one another); the outputs are then
  *               invalid. The library never clears it.
- * 1 <= select_k <= 2048. The q . pooled products run on the tensor cores: each fp32 pooled key is
- * split exactly into three bf16 terms, so with the bf16 queries exact the dot products carry fp32
- * accumulation error only (relative error far below 1e-4); relu and the head weights in fp32.
+ * 1 <= select_k <= 2048. The q . pooled products run on the tensor cores: each (query, head) is
+ * scaled by a power of two and taken exactly as fp16; each fp32 pooled key is scaled by a power
+ * of two and split into two fp16 terms (together the key to 2^-22 of its largest element), so the
+ * dot products carry that and fp32 accumulation error only (relative error far below 1e-4); relu
+ * and the head weights in fp32.
+ * Fewer than 128 queries: one fused launch (scores, selection, expansion), one or more CTAs per
+ * query streaming its visible pools. 128 queries or more (fp32 keys): the many-query path -- a
+ * query preparation kernel, a scoring kernel whose CTAs each convert 256 pooled keys once for
+ * every query of their sequence (pools on the MMA M dimension, 4 queries x 32 heads on N), then
+ * the selection of glm_topk_pools on those scores (and the expansion): five launches, the same
+ * outputs under the same rules; the workspace then also holds the queries as fp16 (8 KB each).
  */
 int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx_dev, const float *w_dev,
                           const float *pooled_dev, int64_t ld_pools, const int32_t *q_seq_dev,
@@ -203,7 +211,8 @@ int glm_index_scores_topk(const glm_dsa_dims *dims, const void *q_idx_dev, const
                           size_t ws_bytes, void *stream);
 
 /*
- * glm_index_scores_topk followed by glm_expand_selection, in one launch: the same scores, top-k
+ * glm_index_scores_topk followed by glm_expand_selection, in one launch (fewer than 128 queries;
+ * else the many-query path of glm_index_scores_topk, then the expansion): the same scores, top-k
  * row and n_sel, plus the expansion of the selection into token positions and cache rows
  * ("Module glm5next_dsa_ref", expand_selection; the rules and arguments of glm_expand_selection:
  * slot_map_dev int64 [batch, ld_slot] or NULL, tok_dev / rows_dev int32 [n_q, out_width], at

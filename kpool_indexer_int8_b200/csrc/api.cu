@@ -78,6 +78,18 @@ size_t sel_words_bytes(int n_q) { return align_up(static_cast<size_t>(n_q) * glm
 size_t sel_bytes(int n_q, int64_t ld) {
     return align_up(sel_zero_bytes(n_q), 256) + sel_fine_bytes(n_q) + sel_words_bytes(n_q) + 2 * sel_list_bytes(n_q, ld);
 }
+// The score rows of the selection ([n_q][ld] fp32) and, for many queries, the scratch of the
+// GEMM scoring path (queries as scaled fp16, w', visible counts), laid out after sel_bytes.
+size_t score_rows_bytes(int n_q, int64_t ld) {
+    return align_up(static_cast<size_t>(n_q) * static_cast<size_t>(ld > 0 ? ld : 0) * sizeof(float), 256);
+}
+size_t gemm_scratch_bytes(int n_q) {
+    return n_q >= glm::kIndexGemmMinQueries ? align_up(glm::index_gemm_scratch_bytes(n_q), 256) : 0;
+}
+// fp32 keys, many queries: scores by the GEMM kernel, then the selection on them.
+bool index_by_gemm(int n_q, int64_t ld_pools, int batch, const float *key_scales) {
+    return key_scales == nullptr && n_q >= glm::kIndexGemmMinQueries && ld_pools > 0 && batch <= 65535;
+}
 SelWs sel_layout(void *base, int n_q, int64_t ld) {
     char *p = static_cast<char *>(base);
     SelWs w;
@@ -146,8 +158,7 @@ struct StepLayout {
 };
 StepLayout step_layout(const glm_dsa_dims *dims, int n_q, int64_t ld, int width) {
     StepLayout L;
-    const size_t idx = sel_bytes(n_q, ld) +
-                       align_up(static_cast<size_t>(n_q) * static_cast<size_t>(ld > 0 ? ld : 0) * sizeof(float), 256) + 256;
+    const size_t idx = sel_bytes(n_q, ld) + score_rows_bytes(n_q, ld) + gemm_scratch_bytes(n_q) + 256;
     L.idx = 0;
     L.mla = idx;
     L.total = idx + mla_workspace(n_q, dims->n_heads, width) + 256;
@@ -244,8 +255,7 @@ size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
     switch (op) {
         case GLM_OP_INDEX_SCORES_TOPK:
             if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
-            return sel_bytes(n_q, max_pools) +
-                   align_up(static_cast<size_t>(n_q) * static_cast<size_t>(max_pools) * sizeof(float), 256) + 256;
+            return sel_bytes(n_q, max_pools) + score_rows_bytes(n_q, max_pools) + gemm_scratch_bytes(n_q) + 256;
         case GLM_OP_TOPK_POOLS:
             if (max_pools < 0 || select_k < 1 || select_k > glm::kMaxSelect) return static_cast<size_t>(-1);
             return sel_bytes(n_q, max_pools);
@@ -324,6 +334,24 @@ int enqueue_index_select(const void *q_idx, const float *w, const void *keys, co
     const SelWs sw = sel_layout(workspace, n_q, ld_pools);
     char *ws = static_cast<char *>(workspace);
     float *sbuf = scores ? scores : reinterpret_cast<float *>(ws + sel_bytes(n_q, ld_pools));
+    if (index_by_gemm(n_q, ld_pools, batch, key_scales)) {
+        // zero the selection's words, score every (query, pool), select, expand
+        int rc = GLM_OK;
+        if (zero) rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
+        if (rc != GLM_OK) return rc;
+        void *scratch = ws + sel_bytes(n_q, ld_pools) + score_rows_bytes(n_q, ld_pools);
+        rc = cuda_status(glm::launch_index_gemm(q_idx, w, static_cast<const float *>(keys), ld_pools, q_seq, q_pos, pad,
+                                                len, batch, n_q, sbuf, scratch, status, sms, st));
+        if (rc != GLM_OK) return rc;
+        const glm::NvisSource src{nullptr, q_seq, q_pos, pad, len, batch, ld_pools};
+        rc = cuda_status(glm::launch_topk_hist(sbuf, src, n_q, sw.hist, st));
+        if (rc != GLM_OK) return rc;
+        rc = cuda_status(glm::launch_topk_collect(sbuf, src, sw.hist, sw.hist2, sw.counters, sw.words, sw.alist,
+                                                  sw.blist, n_q, select_k, topk, n_sel, st));
+        if (rc != GLM_OK || (!tok && !rows)) return rc;
+        return cuda_status(glm::launch_expand(topk, n_sel, q_seq, q_pos, pad, len, batch, n_q, select_k, slot_map,
+                                              ld_slot, out_width, tok, rows, st));
+    }
     if (zero && glm::index_select_ctas(n_q, ld_pools, sms) > 1) {
         const int rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
         if (rc != GLM_OK) return rc;
@@ -620,7 +648,8 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     int *status = reinterpret_cast<int *>(ws + L.total - 256);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int sms = num_sms();
-    const bool idx_multi = a->n_q > 0 && glm::index_select_ctas(a->n_q, a->ld_pools, sms) > 1;
+    const bool idx_multi = a->n_q > 0 && (index_by_gemm(a->n_q, a->ld_pools, a->batch, q8 ? a->pooled_scales_dev : nullptr) ||
+                                          glm::index_select_ctas(a->n_q, a->ld_pools, sms) > 1);
     const SelWs sw = sel_layout(ws + L.idx, a->n_q, a->ld_pools);
     glm::StepPrepArgs p{};
     p.latent = static_cast<const uint16_t *>(a->latent_dev);

@@ -60,6 +60,16 @@ struct IxSelectArgs {
     int new_pools;
 };
 int index_select_ctas(int n_q, int64_t ld_pools, int num_sms);
+
+// Scores of many queries at once (index_gemm.cu): queries of one sequence share the converted
+// pooled keys; scratch of index_gemm_scratch_bytes(n_q) bytes, 256-byte aligned. Every score of
+// rows [0, n_q) x [0, ld_pools) is written (-inf past the query's visible pools).
+constexpr int kIndexGemmMinQueries = 128;   // fp32 keys and at least this many queries: the GEMM path
+size_t index_gemm_scratch_bytes(int n_q);
+cudaError_t launch_index_gemm(const void *q_idx, const float *w, const float *pooled, int64_t ld_pools,
+                              const int32_t *q_seq, const int32_t *q_pos, const int32_t *pad, const int32_t *len,
+                              int batch, int n_q, float *scores, void *scratch, int *status, int num_sms,
+                              cudaStream_t stream);
 cudaError_t set_cross_cta_wait_limit(uint32_t polls);   // the index kernel's meetings (current device)
 cudaError_t launch_index_select_tc(const void *q_idx, const float *w, const void *keys,
                                    const float *key_scales, int64_t ld_pools, const int32_t *q_seq,

@@ -163,23 +163,10 @@ __global__ void __launch_bounds__(kVuThreads, 1) mla_vup_kernel(const __grid_con
     }
 }
 
-namespace {
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        void *p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
-    return fn;
-}
-}  // namespace
 
 cudaError_t launch_mla_vup(const void *o_lat, const void *w_kv_b, int n_heads, int dk, int dv, int n_q, void *out_v,
                            float *out_f32, cudaStream_t stream) {
-    auto encode = encode_fn();
+    auto encode = tc::tensor_map_encoder();
     if (!encode) return cudaErrorNotSupported;
     CUtensorMap map_a, map_w;
     // o_lat bf16 [n_q][n_heads][512]: dims (512, n_heads, n_q), boxes of 64 dims x 1 head x 128 queries
