@@ -108,11 +108,18 @@ SelWs sel_layout(void *base, int n_q, int64_t ld) {
     return w;
 }
 
-// Workspace of the sparse MLA: partial accumulators and (m, l) pairs per (query, chunk, head),
+// Workspace of the sparse MLA: partial accumulators and (m, l) pairs per (query, part, head),
 // then a 256-byte tail whose first word is the kernels' status (nonzero after a timed-out wait).
+// Sized for the plan of n_q queries and for every smaller count: up to the few-query maximum
+// the plan keeps one partial per chunk; above it at most that many partials, or one per query.
 size_t mla_parts(int n_q, int n_heads, int width) {
-    const int chunk = glm::mla_tc_chunk();
-    return static_cast<size_t>(n_q) * static_cast<size_t>((width + chunk - 1) / chunk) * n_heads;
+    const int sms = num_sms();
+    const long long chunks = (width + glm::mla_tc_chunk() - 1) / glm::mla_tc_chunk();
+    const long long few_max = glm::mla_few_query_max(n_heads, sms);
+    if (n_q <= few_max) return static_cast<size_t>(n_q) * static_cast<size_t>(chunks) * n_heads;
+    const glm::MlaPlan p = glm::mla_plan(n_q, n_heads, width, sms);
+    const long long per = static_cast<long long>(n_q) * p.n_parts;
+    return static_cast<size_t>(per > few_max * chunks ? per : few_max * chunks) * n_heads;
 }
 size_t mla_acc_bytes(size_t parts) { return align_up(parts * glm::kLatent * sizeof(float), 256); }
 size_t mla_ml_bytes(size_t parts) { return align_up(parts * 2 * sizeof(float), 256); }
@@ -526,9 +533,9 @@ int sparse_mla_entry(const glm_dsa_dims *dims, const void *q, const int8_t *cach
     int *status = reinterpret_cast<int *>(ws + mla_acc_bytes(parts) + mla_ml_bytes(parts));
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     rc = cuda_status(glm::launch_mla_split_tc(plan, q, H, cache, n_rows, rows, n_q, width, sm_scale, part_acc, part_ml,
-                                              status, st, false, format));
-    if (rc != GLM_OK) return rc;
-    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32, lse, st));
+                                              status, st, false, format, out, out_f32, lse));
+    if (rc != GLM_OK || !plan.combine) return rc;
+    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_parts, out, out_f32, lse, st));
 }
 }  // namespace
 
@@ -691,9 +698,10 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     float *part_acc = reinterpret_cast<float *>(ws + L.mla);
     float *part_ml = reinterpret_cast<float *>(ws + L.mla + mla_acc_bytes(parts));
     rc = cuda_status(glm::launch_mla_split_tc(plan, a->q_dev, H, a->cache_dev, a->n_rows, a->rows_dev, a->n_q, a->out_width,
-                                              a->sm_scale, part_acc, part_ml, status, st, true, a->cache_format));
-    if (rc != GLM_OK || a->stop_after == 3) return rc;
-    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, plan.n_chunks, a->out_dev, a->out_f32_dev,
+                                              a->sm_scale, part_acc, part_ml, status, st, true, a->cache_format,
+                                              a->out_dev, a->out_f32_dev, a->lse_dev));
+    if (rc != GLM_OK || a->stop_after == 3 || !plan.combine) return rc;
+    return cuda_status(glm::launch_mla_combine(part_acc, part_ml, a->n_q, H, plan.n_parts, a->out_dev, a->out_f32_dev,
                                                a->lse_dev, st));
 }
 

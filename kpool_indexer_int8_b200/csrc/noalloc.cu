@@ -57,8 +57,8 @@ extern "C" int glm_sparse_mla_decode_noalloc(const glm_dsa_dims *dims, const voi
     if (rc != GLM_OK) return rc;
     const glm::MlaPlan plan = glm::mla_plan(n_q, H, width, glm::abi::num_sms());
     rc = glm::abi::cuda_status(glm::launch_mla_split_tc(plan, q, H, cache, n_rows, rows, n_q, width, sm_scale,
-                                                        part_acc, part_ml, status, st));
-    if (rc != GLM_OK) return rc;
-    return glm::abi::cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_chunks, out, out_f32,
+                                                        part_acc, part_ml, status, st, false, 0, out, out_f32, lse));
+    if (rc != GLM_OK || !plan.combine) return rc;   // (without a combine the kernel writes NaN itself on a give-up)
+    return glm::abi::cuda_status(glm::launch_mla_combine(part_acc, part_ml, n_q, H, plan.n_parts, out, out_f32,
                                                          lse, st, status));
 }

@@ -57,6 +57,22 @@ FAKE = C.c_void_p(0x10000)        # 16-byte aligned, never dereferenced: every c
 MIS = C.c_void_p(0x10004)         # misaligned for 16-byte operands
 
 
+def test_workspace_sizes_cover_every_smaller_query_count():
+    # a workspace sized for n_q queries serves any smaller count: the attention's plan changes
+    # with the count (one partial per chunk for few queries, runs of chunks for many), the size
+    # must not shrink as the count grows; the many-query index scratch likewise
+    for heads in (16, 64, 128):
+        d = kp.make_dims(heads)
+        for op, kw in ((kp.GLM_OP_SPARSE_MLA, dict(width=2176)),
+                       (kp.GLM_OP_INDEX_SCORES_TOPK, dict(max_pools=33792, select_k=512)),
+                       (kp.GLM_OP_DECODE_STEP, dict(max_pools=33792, select_k=512, width=2176))):
+            prev = 0
+            for nq in sorted(set(range(1, 400, 7)) | {127, 128, 129, 295, 296, 297, 591, 592, 593, 1000, 4096, 65535}):
+                size = kp.glm_dsa_workspace_size(d, op, nq, **kw)
+                assert size >= prev, (heads, op, nq)
+                prev = size
+
+
 def test_store_rejects_before_launch():
     L = kp.lib
     d = C.byref(kp.make_dims(64))
