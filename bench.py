@@ -37,8 +37,19 @@ import synth  # noqa: E402
 
 # Kernels of one glm_dsa_decode_step: store + pool build + zeroing of the selection words, scores +
 # top-k + expansion, MLA split, MLA combine.
-KERNELS_PER_STEP = 4
-STEP_KERNELS = ("step_prep", "index_select_tc", "mla_split_tc", "mla_combine")
+
+
+def step_kernels(kp, wl, ld_pools: int, int8_keys: bool):
+    """Kernels the one-call step enqueues for this workload (the library's own plan) and the names
+    of its four stages (the step prefixes stop_after = 1, 2, 3 and the whole step)."""
+    k, paths = kp.glm_dsa_step_plan(kp.make_dims(wl.n_heads), wl.n_queries, ld_pools, wl.batch, wl.out_width,
+                                    int8_keys)
+    names = ("step_prep",
+             "index_qprep + index_gemm + topk_hist + topk_collect + expand" if paths & kp.GLM_PLAN_INDEX_MANY
+             else "index_select_tc",
+             "mla_multi_tc" if paths & kp.GLM_PLAN_MLA_MANY else "mla_split_tc",
+             "mla_combine" if paths & kp.GLM_PLAN_MLA_COMBINE else "(no combine: mla_multi_tc writes the output)")
+    return k, paths, names
 
 
 def algorithmic_bytes(inp, key_bytes: int = 512, row_bytes: int = 528) -> dict:
@@ -73,6 +84,15 @@ def measured_peaks():
         d = json.load(open(p))
         return float(d["hbm_gbs"]), "measured"
     return 6650.0, "fallback"
+
+
+def measured_tensor_peak():
+    """Dense fp16/bf16 tensor TFLOP/s (the same rate for both 16-bit kinds): the measured burst
+    figure (the kernel is timed over well under a second), else the fallback."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        return float(json.load(open(p))["bf16_tflops"]), "measured bf16_tflops (burst)"
+    return 1590.0, "fallback bf16_tflops (burst)"
 
 
 def kernel_source_sha(name: str) -> str:
@@ -185,15 +205,18 @@ class ClockSampler:
 # the CPU oracle leg (cpu_baseline and --impl reference)
 # ------------------------------------------------------------------------------------------------
 
-def oracle_decode_throughput(wl, budget_s: float = 12.0, max_queries: int = 64):
+def oracle_decode_throughput(wl, budget_s: float = 12.0, max_queries: int = 64, warmup: int = 0):
     """Time the fp64 oracle on decode queries of state 0 of the workload: per query the store of
     its new row, the pool that row completes, scores over all visible pools, top-k, expand and the
-    sparse MLA. The oracle's state (cache, pools) is built beforehand, untimed."""
+    sparse MLA. The oracle's state (cache, pools) is built beforehand, untimed, and `warmup`
+    queries run untimed before the timed ones."""
     import oracle
     inp = synth.generate(wl, state=0)
     cache = oracle.build_cache(inp)
     pools = oracle.build_pools(inp)
     new = np.nonzero(inp.new_token_mask())[0]
+    for w in range(warmup):
+        oracle.decode_query(inp, w % len(inp.q_pos), cache, pools)
     done, t0 = 0, time.perf_counter()
     elapsed = 0.0
     while done < max_queries and (elapsed < budget_s or done == 0):
@@ -218,10 +241,10 @@ def run_reference(args, wl):
     if rank != 0:
         return 0
     # one reference step = one whole decode query of the oracle; K steps, cut at ~4 minutes
-    qps, done, el = oracle_decode_throughput(wl, budget_s=240.0, max_queries=max(1, args.steps))
+    qps, done, el = oracle_decode_throughput(wl, budget_s=240.0, max_queries=max(1, args.steps), warmup=args.warmup)
     line = {
         "impl": "reference", "metric": METRIC, "value": qps, "unit": "queries/s",
-        "n_gpus": args.gpus, "steps": done, "warmup": 0,
+        "n_gpus": args.gpus, "steps": done, "warmup": args.warmup,
         "ms_per_step": 1e3 / qps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(wl, args),
@@ -308,6 +331,7 @@ def run_kernels(args, wl):
         del inp
     ab = algorithmic_bytes(inps[0], key_bytes=132 if args.pooled == "int8" else 512,
                            row_bytes=304 if args.cache == "fp4" else 528)
+    n_kernels, paths, stage_names = step_kernels(kp, wl, bufs[0].pooled.shape[1], args.pooled == "int8")
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
 
@@ -483,11 +507,26 @@ def run_kernels(args, wl):
     del e2e_graphs
 
     peak, peak_kind = measured_peaks()
-    # dominant kernel: the fused scores + selection + expansion launch (each timed launch also
-    # carries the tiny zeroing launch of the multi-CTA selection words)
-    idx_ms = idx_launch_ms
-    achieved = ab["index"] / (idx_ms / 1e3) / 1e9
-    traffic = recorded_traffic("index_select_tc.cu", wl.name + ("_q8" if args.pooled == "int8" else ""))
+    if paths & kp.GLM_PLAN_MLA_MANY and kernel_ms[2] >= max(kernel_ms):
+        # dominant kernel: the walking attention (many queries), a tensor-core contraction:
+        # q . k and p . v over every gathered row, 2 x 2 x 512 FLOP per (row, head)
+        flop = ab["gathered"] * wl.n_heads * 512 * 2 * 2
+        t_peak, t_kind = measured_tensor_peak()
+        mla_s = kernel_ms[2] / 1e3
+        roofline = {"kernel": "mla_multi_tc (walking attention; its share of the step, step prefixes)",
+                    "bound": "tensor", "achieved": flop / mla_s / 1e12, "peak": t_peak, "peak_kind": t_kind,
+                    "unit": "TFLOP/s", "frac": flop / mla_s / 1e12 / t_peak, "traffic": None,
+                    "algorithmic_flop_per_launch": flop, "launch_us": kernel_ms[2] * 1e3}
+    else:
+        # dominant kernel: the fused scores + selection + expansion launch (each timed launch also
+        # carries the tiny zeroing launch of the multi-CTA selection words)
+        idx_ms = idx_launch_ms
+        achieved = ab["index"] / (idx_ms / 1e3) / 1e9
+        traffic = recorded_traffic("index_select_tc.cu", wl.name + ("_q8" if args.pooled == "int8" else ""))
+        roofline = {"kernel": "index_select_tc (scores + top-k + expansion)", "bound": "hbm", "achieved": achieved,
+                    "peak": peak, "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
+                    "traffic": traffic, "algorithmic_bytes_per_launch": ab["index"],
+                    "launch_us": idx_ms * 1e3}
     line = {
         "metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
@@ -497,21 +536,18 @@ def run_kernels(args, wl):
         "achieved_hbm_gbs_per_gpu": ab["total"] / (ms_per_step / 1e3) / 1e9,
         "algorithmic_bytes_per_step": ab["total"],
         "tokens_gathered_per_s": ab["gathered"] * args.steps * world / (ms / 1e3),
-        "kernel_us_in_step": {nm: v * 1e3 for nm, v in zip(STEP_KERNELS, kernel_ms)},
+        "kernel_us_in_step": {nm: v * 1e3 for nm, v in zip(stage_names, kernel_ms)},
         "kernel_us_method": "step prefixes (stop_after = 1, 2, 3, whole) as graphs of the rotating states; "
                             "each kernel = difference of consecutive prefixes; their sum is the whole step "
                             f"timed the same way ({prefix_ms[3] * 1e3:.2f} us)",
-        "roofline": {"kernel": "index_select_tc (scores + top-k + expansion)", "bound": "hbm", "achieved": achieved, "peak": peak,
-                     "peak_kind": f"{peak_kind} hbm_gbs", "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": traffic, "algorithmic_bytes_per_launch": ab["index"],
-                     "launch_us": idx_ms * 1e3},
+        "roofline": roofline,
         "e2e": {"value": e2e_qps, "unit": "queries/s", "h2d_bytes_per_step": int(h2d),
                 "d2h_bytes_per_step": int(d2h), "steps": n_e2e,
                 "api": "glm_dsa_decode_step through the binding with its host copies (pinned, one packed "
                        "H2D of the step inputs + the new k/gate rows, one D2H of out) captured per state "
                        "as a CUDA graph, replayed per step; the host waits for each step's output by "
                        "polling an event recorded after it"},
-        "gpu_launches": KERNELS_PER_STEP * args.steps,
+        "gpu_launches": n_kernels * args.steps,
         "clocks": sampler.summary(),
     }
     line["achieved_hbm_frac_per_gpu"] = line["achieved_hbm_gbs_per_gpu"] / peak

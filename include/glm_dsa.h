@@ -538,6 +538,25 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *step, void
 size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
                               int64_t max_pools, int32_t select_k, int32_t width);
 
+/*
+ * How glm_dsa_decode_step runs a step of this shape on the current device: *launches receives
+ * the number of kernels it enqueues (stop_after = 0), *paths (or NULL) a mask of
+ *   GLM_PLAN_INDEX_MANY  -- 128 or more queries on fp32 keys: the many-query scoring kernel (pooled
+ *                           keys shared by the queries of a sequence), then the selection and the
+ *                           expansion as separate kernels; otherwise one fused index kernel;
+ *   GLM_PLAN_MLA_MANY    -- enough queries to fill the SMs twice: each attention CTA walks a run
+ *                           of a query's chunks; otherwise one CTA per 64-entry chunk;
+ *   GLM_PLAN_MLA_COMBINE -- a combine kernel merges partials (absent when each query's entries
+ *                           are covered by one CTA, which then writes the output itself).
+ * int8_keys: nonzero for the INT8 indexer state. A host-side query: nothing is enqueued.
+ * Returns GLM_OK, or the argument errors of glm_dsa_decode_step's shape checks.
+ */
+#define GLM_PLAN_INDEX_MANY 1
+#define GLM_PLAN_MLA_MANY 2
+#define GLM_PLAN_MLA_COMBINE 4
+int glm_dsa_step_plan(const glm_dsa_dims *dims, int32_t n_q, int64_t ld_pools, int32_t batch, int32_t width,
+                      int32_t int8_keys, int32_t *launches, int32_t *paths);
+
 #ifdef __cplusplus
 }
 #endif

@@ -34,6 +34,7 @@ GLM_OP_INDEX_SCORES_TOPK = 1
 GLM_OP_TOPK_POOLS = 2
 GLM_OP_SPARSE_MLA = 3
 GLM_OP_DECODE_STEP = 4
+GLM_PLAN_INDEX_MANY, GLM_PLAN_MLA_MANY, GLM_PLAN_MLA_COMBINE = 1, 2, 4
 
 EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv_store_int8",
            "glm_kpool_build", "glm_kpool_build_q8", "glm_index_scores", "glm_index_scores_topk",
@@ -42,7 +43,7 @@ EXPORTS = ("glm_check_dims", "glm_status_string", "glm_last_cuda_error", "glm_kv
            "glm_topk_pools", "glm_expand_selection",
            "glm_sparse_mla_decode", "glm_dsa_workspace_size", "glm_kv_store_fp8", "glm_sparse_mla_decode_fp8",
            "glm_debug_set_cross_cta_wait_limit", "glm_mla_v_up", "glm_cp_candidates", "glm_merge_topk",
-           "glm_lse_merge", "glm_kv_store_fp4", "glm_sparse_mla_decode_fp4")
+           "glm_lse_merge", "glm_kv_store_fp4", "glm_sparse_mla_decode_fp4", "glm_dsa_step_plan")
 
 
 class glm_dsa_dims(C.Structure):
@@ -101,6 +102,8 @@ lib.glm_index_topk_expand.argtypes = [_D, _P, _P, _P, _I64, _P, _P, _P, _P, _I32
 lib.glm_index_topk_expand.restype = C.c_int
 lib.glm_dsa_decode_step.argtypes = [_D, C.POINTER(glm_dsa_step), _P, _SZ, _P]
 lib.glm_dsa_decode_step.restype = C.c_int
+lib.glm_dsa_step_plan.argtypes = [_D, _I32, _I64, _I32, _I32, _I32, C.POINTER(C.c_int32), C.POINTER(C.c_int32)]
+lib.glm_dsa_step_plan.restype = C.c_int
 lib.glm_kpool_build_q8.argtypes = [_D, _P, _P, _I64, _P, _P, _F32, _P, _P, _P, _I32, _I32, _P, _P, _I64, _P, _P]
 lib.glm_kpool_build_q8.restype = C.c_int
 lib.glm_index_topk_expand_q8.argtypes = [_D, _P, _P, _P, _P, _I64, _P, _P, _P, _P, _I32, _I32, _I32, _P, _I64,
@@ -165,6 +168,14 @@ def _dev(t, dtype, name, ndim=None):
 
 def check_dims(dims: glm_dsa_dims) -> int:
     return lib.glm_check_dims(C.byref(dims))
+
+
+def glm_dsa_step_plan(dims, n_q, ld_pools, batch, width, int8_keys=False):
+    """(kernels glm_dsa_decode_step enqueues, mask of GLM_PLAN_*) for a step of this shape."""
+    k, f = C.c_int32(0), C.c_int32(0)
+    _check(lib.glm_dsa_step_plan(C.byref(dims), n_q, ld_pools, batch, width, 1 if int8_keys else 0, C.byref(k),
+                                 C.byref(f)), "glm_dsa_step_plan")
+    return int(k.value), int(f.value)
 
 
 def glm_dsa_workspace_size(dims, op, n_q, max_pools=0, select_k=1, width=1) -> int:

@@ -256,6 +256,29 @@ int glm_kpool_build_q8(const glm_dsa_dims *dims, const void *k, const void *gate
                                                pooled_scales));
 }
 
+int glm_dsa_step_plan(const glm_dsa_dims *dims, int32_t n_q, int64_t ld_pools, int32_t batch, int32_t width,
+                      int32_t int8_keys, int32_t *launches, int32_t *paths) {
+    const int rc = glm_check_dims(dims);
+    if (rc != GLM_OK) return rc;
+    if (n_q < 0 || ld_pools < 0 || batch < 0 || width < 1 || width > 65536 || !launches) return GLM_ERR_INVALID_ARG;
+    int k = 1, f = 0;   // step_prep
+    if (n_q > 0) {
+        if (index_by_gemm(n_q, ld_pools, batch, int8_keys ? reinterpret_cast<const float *>(&k) : nullptr)) {
+            f |= GLM_PLAN_INDEX_MANY;
+            k += 5;   // query preparation, scores, histogram, selection, expansion
+        } else {
+            k += 1;   // the fused scores + selection + expansion
+        }
+        const glm::MlaPlan plan = glm::mla_plan(n_q, dims->n_heads, width, num_sms());
+        if (plan.multi) f |= GLM_PLAN_MLA_MANY;
+        if (plan.combine) f |= GLM_PLAN_MLA_COMBINE;
+        k += plan.combine ? 2 : 1;
+    }
+    *launches = k;
+    if (paths) *paths = f;
+    return GLM_OK;
+}
+
 size_t glm_dsa_workspace_size(const glm_dsa_dims *dims, int32_t op, int32_t n_q,
                               int64_t max_pools, int32_t select_k, int32_t width) {
     if (glm_check_dims(dims) != GLM_OK || n_q < 0) return static_cast<size_t>(-1);

@@ -73,6 +73,22 @@ def test_workspace_sizes_cover_every_smaller_query_count():
                 prev = size
 
 
+def test_step_plan_counts_the_kernels_of_each_path():
+    d = kp.make_dims(64)
+    # one decode query: step_prep, the fused index kernel, the split attention and its combine
+    assert kp.glm_dsa_step_plan(d, 1, 65536, 1, 2176) == (4, kp.GLM_PLAN_MLA_COMBINE)
+    # 4,096 prefill queries: step_prep, query preparation, scores, histogram, selection, expansion,
+    # the walking attention writing its output (one run per query)
+    k, f = kp.glm_dsa_step_plan(d, 4096, 33792, 1, 2176)
+    assert (k, f) == (7, kp.GLM_PLAN_INDEX_MANY | kp.GLM_PLAN_MLA_MANY)
+    # the INT8 indexer state keeps the fused index kernel
+    assert kp.glm_dsa_step_plan(d, 4096, 33792, 1, 2176, int8_keys=True)[1] == kp.GLM_PLAN_MLA_MANY
+    # no query: step_prep only
+    assert kp.glm_dsa_step_plan(d, 0, 16, 1, 2176) == (1, 0)
+    with pytest.raises(kp.GlmError):
+        kp.glm_dsa_step_plan(d, -1, 16, 1, 2176)
+
+
 def test_store_rejects_before_launch():
     L = kp.lib
     d = C.byref(kp.make_dims(64))
