@@ -497,11 +497,8 @@ done:
 //     the reference m_ref moves to m_c only when m_c > m_ref + 8, so exp2(s - m_ref) <= 2^8;
 //   * the row-scale reference sigma (a power of two) moves to the next power of two >= the
 //     chunk's largest row scale only when that exceeds 16 sigma;
-//   * P' = exp2(s - m_ref) scale_row / sigma (<= 2^12) as an fp16 hi + lo pair; each row slot of
-//     the chunk tile keeps its own sums of exp2(s - m_ref) per head in registers (times alpha_h
-//     when the reference moves), added up into l once at the end;
-//   * in the steady state no reference moves: a block vote on "some score passes its reference
-//     by 2^8" skips the chunk maxima altogether;
+//   * P' = exp2(s - m_ref) scale_row / sigma (<= 2^12) as an fp16 hi + lo pair, l = l alpha + sum
+//     of exp2(s - m_ref) over the chunk's rows;
 //   * when a reference moves, the accumulator is first multiplied in tensor memory by
 //     alpha_h beta (alpha_h = exp2(m_ref,old - m_ref,new), beta = sigma_old / sigma_new);
 //   * O^T += C^T . P'_hi^T + C^T . P'_lo^T into one accumulator of 4 tiles of 128 latent dims x 64
@@ -527,9 +524,7 @@ struct MlaMultiLayout {
     static constexpr int kMref = kQmax + NH * 4;                      // NH reference maxima (log2 units)
     static constexpr int kLsum = kMref + NH * 4;                      // NH running sums
     static constexpr int kFac = kLsum + NH * 4;                       // NH factors of the accumulator
-    static constexpr int kThr = kFac + NH * 4;                        // NH reference + 8
-    static constexpr int kAl = kThr + NH * 4;                         // NH factors of the sums
-    static constexpr int kWords = kAl + NH * 4;                       // [0..1] chunk scale maxima (bits), [2] tmem base
+    static constexpr int kWords = kFac + NH * 4;                      // [0..1] chunk scale maxima (bits), [2] tmem base
     static constexpr int kBar = kWords + 16;                          // 2 mbarriers
     static constexpr int kBytes = kBar + 2 * 8;
     static_assert(kQ % 16 == 0 && kP % 16 == 0 && kBar % 8 == 0, "alignment");
@@ -578,8 +573,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_multi_tc_kernel(
     float *mref = reinterpret_cast<float *>(smem + L::kMref);
     float *lsum = reinterpret_cast<float *>(smem + L::kLsum);
     float *fac = reinterpret_cast<float *>(smem + L::kFac);
-    float *mthr = reinterpret_cast<float *>(smem + L::kThr);
-    float *alph = reinterpret_cast<float *>(smem + L::kAl);
     unsigned *words = reinterpret_cast<unsigned *>(smem + L::kWords);
     const uint32_t bar0 = tc::smem_addr(smem + L::kBar);
     const uint32_t bar_s = bar0, bar_o = bar0 + 8;
@@ -598,7 +591,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_multi_tc_kernel(
     if (tid < NH) {
         qmax[tid] = 0u;
         mref[tid] = -INFINITY;
-        mthr[tid] = -INFINITY;
         lsum[tid] = 0.0f;
     }
     if (tid < 2) words[tid] = 0u;
@@ -647,21 +639,10 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_multi_tc_kernel(
     uint32_t s_phase = 0, o_phase = 0;   // commits issued on each barrier
     bool have_o = false;                 // the accumulator holds a chunk
     float sigma = 0.0f;                  // row-scale reference (0: none yet); the same in every thread
+    float alpha = 1.0f;                  // tid < NH: this chunk's factor of l
     int fail = 0;
     const int quad = warp & 3, hh = warp >> 2;
     const int j = lane < 16 ? quad * 16 + lane : -1;   // the S row of this lane (M = 64: lanes 0-15 of a quadrant)
-    float lacc[V];   // this lane's row slot: sum over its chunks of exp2(s - m_ref) for heads [V hh, +V)
-#pragma unroll
-    for (int e = 0; e < V; e++) lacc[e] = 0.0f;
-    // descriptors of the fixed operands; a start address advances by adding its 16-byte units
-    const uint64_t dq = tc::desc(tc::smem_addr(Qs), 128, 8192);
-    const uint64_t dp = tc::desc(tc::smem_addr(Ps), kLboP, 128);
-    const uint32_t idesc_s = tc::idesc_f16(ROWS, NH, false, false);
-    const uint32_t idesc_o = tc::idesc_f16(128, NH, true, true);
-    const float4 *qk4 = reinterpret_cast<const float4 *>(qk + hh * V);
-    const float4 *thr4 = reinterpret_cast<const float4 *>(mthr + hh * V);
-    const float4 *mref4 = reinterpret_cast<const float4 *>(mref + hh * V);
-    const float4 *al4 = reinterpret_cast<const float4 *>(alph + hh * V);
 
     for (int c = c0, i = 0; c < c1; c++, i++) {
         const int buf = i & 1;
@@ -677,15 +658,16 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_multi_tc_kernel(
             r_next = row_of(c + 2);
         }
         if (nv > 0) {
-            const uint64_t dc = tc::desc(tc::smem_addr(Cs + buf * L::kCBytes), 128, 8192);
             // b. S^T = C . Q^T (M = 64 rows, N = NH heads, K = 512); its completion also means that
             //    every earlier accumulation has completed
             if (tid == 0) {
                 tc::fence_after_sync();
-#pragma unroll
+                const uint32_t idesc = tc::idesc_f16(ROWS, NH, false, false);
+                const uint32_t ca = tc::smem_addr(Cs + buf * L::kCBytes), qa = tc::smem_addr(Qs);
+#pragma unroll 4
                 for (int ks = 0; ks < kLatent / 16; ks++)
-                    tc::mma_bf16(tmem + kSCol, dc + static_cast<uint64_t>(ks * 16), dq + static_cast<uint64_t>(ks * 16),
-                                 idesc_s, ks > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + kSCol, tc::desc(ca + ks * 256, 128, 8192), tc::desc(qa + ks * 256, 128, 8192),
+                                 idesc, ks > 0 ? 1u : 0u);
                 tc::mma_commit(bar_s);
             }
             const bool ok = tc::mbar_wait(bar_s, s_phase & 1u, kMlaWaitLimit);
@@ -700,87 +682,61 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_multi_tc_kernel(
             const float beta = sigma == 0.0f ? 1.0f : sigma / sig_new;   // powers of two: exact
             const float inv_sig = 1.0f / sig_new;
 
-            // c. the scores of this lane's row for heads [V hh, +V) (s = S scale_row qk_h), and whether
-            //    one passes its head's reference by 2^8
+            // c. softmax: warp w reads TMEM lane quadrant w % 4 (row 16 (w % 4) + lane, lanes < 16)
+            //    and heads [V (w / 4), +V)
             uint32_t r[V];
             tmem_ld_v<V>(tmem + (static_cast<uint32_t>(quad * 32) << 16) + kSCol + hh * V, r);
             tc::tmem_wait_ld();
             const bool rv = j >= 0 && ridx[buf * ROWS + j] >= 0;
             const float sc = rv ? scl[buf * ROWS + j] : 0.0f;
-            float sv[V];
-            bool up = false;
+            float sv[V], t[V];
 #pragma unroll
-            for (int e4 = 0; e4 < V / 4; e4++) {
-                const float4 k4 = qk4[e4], t4 = thr4[e4];
-                const float kk[4] = {k4.x, k4.y, k4.z, k4.w}, tt[4] = {t4.x, t4.y, t4.z, t4.w};
-#pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    const int e = 4 * e4 + k;
-                    sv[e] = rv ? __uint_as_float(r[e]) * sc * kk[k] : -INFINITY;
-                    up |= sv[e] > tt[k];
-                }
+            for (int e = 0; e < V; e++) {
+                sv[e] = rv ? __uint_as_float(r[e]) * sc * qk[hh * V + e] : -INFINITY;
+                t[e] = sv[e];
             }
-            const bool moved = __syncthreads_or(up) != 0;
-            if (moved) {
-                // the chunk maxima of every head; a head's reference moves to its maximum when that
-                // passes it by 2^8 (or none is set yet); alpha_h = exp2(old - new) rescales its sums
-                float t[V];
-#pragma unroll
-                for (int e = 0; e < V; e++) t[e] = sv[e];
-                const float bm = butterfly<V, true>(t);
-                if ((lane & kLow) == 0) red[quad * NH + hh * V + ((lane >> kShift) & (V - 1))] = bm;
-                __syncthreads();
-                if (tid < NH) {
-                    const float mc = fmaxf(fmaxf(red[tid], red[NH + tid]), fmaxf(red[2 * NH + tid], red[3 * NH + tid]));
-                    const float mo = mref[tid];
-                    const float mn = (mo == -INFINITY || mc > mo + kMaxGrow) ? mc : mo;
-                    const float al = mo == -INFINITY ? 0.0f : exp2f(mo - mn);
-                    mref[tid] = mn;
-                    mthr[tid] = mn + kMaxGrow;
-                    alph[tid] = al;
-                    fac[tid] = al * beta;
-                }
-                __syncthreads();
-#pragma unroll
-                for (int e4 = 0; e4 < V / 4; e4++) {
-                    const float4 a4 = al4[e4];
-                    lacc[4 * e4] *= a4.x;
-                    lacc[4 * e4 + 1] *= a4.y;
-                    lacc[4 * e4 + 2] *= a4.z;
-                    lacc[4 * e4 + 3] *= a4.w;
-                }
+            const float bm = butterfly<V, true>(t);
+            if ((lane & kLow) == 0) red[quad * NH + hh * V + ((lane >> kShift) & (V - 1))] = bm;
+            __syncthreads();
+            bool need = false;
+            if (tid < NH) {
+                const float mc = fmaxf(fmaxf(red[tid], red[NH + tid]), fmaxf(red[2 * NH + tid], red[3 * NH + tid]));
+                const float mo = mref[tid];
+                const float mn = (mo == -INFINITY || mc > mo + kMaxGrow) ? mc : mo;
+                alpha = mo == -INFINITY ? 0.0f : exp2f(mo - mn);
+                mref[tid] = mn;
+                const float f = alpha * beta;
+                fac[tid] = f;
+                need = have_o && f != 1.0f;
             }
-            const bool rescale = have_o && (moved || beta != 1.0f);
+            const bool rescale = __syncthreads_or(need) != 0;
             sigma = sig_new;
             const float ratio = sc * inv_sig;   // scale_row / sigma (exact: sigma a power of two)
 #pragma unroll
-            for (int e4 = 0; e4 < V / 4; e4++) {
-                const float4 m4 = mref4[e4];
-                const float mm[4] = {m4.x, m4.y, m4.z, m4.w};
-#pragma unroll
-                for (int k = 0; k < 4; k++) {
-                    const int e = 4 * e4 + k;
-                    const float pv = rv ? exp2f(sv[e] - mm[k]) : 0.0f;
-                    lacc[e] += pv;
-                    sv[e] = pv * ratio;
-                }
+            for (int e = 0; e < V; e++) {
+                const float m = mref[hh * V + e];
+                const float pv = rv ? exp2f(sv[e] - m) : 0.0f;
+                sv[e] = pv;
+                t[e] = pv;
             }
+            const float bl = butterfly<V, false>(t);
+            if ((lane & kLow) == 0) red2[quad * NH + hh * V + ((lane >> kShift) & (V - 1))] = bl;
             if (j >= 0) {   // P' of this row as fp16 hi + lo, 8 heads per 16-byte line
 #pragma unroll
                 for (int g = 0; g < V / 8; g++) {
                     uint32_t hi4[4], lo4[4];
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
-                        const float x0 = sv[8 * g + 2 * e], x1 = sv[8 * g + 2 * e + 1];
-                        hi4[e] = f16x2_rn(x0, x1);
-                        lo4[e] = f16x2_rn(x0 - f16_lo_f(hi4[e]), x1 - f16_hi_f(hi4[e]));
+                        const float a = sv[8 * g + 2 * e] * ratio, b = sv[8 * g + 2 * e + 1] * ratio;
+                        hi4[e] = f16x2_rn(a, b);
+                        lo4[e] = f16x2_rn(a - f16_lo_f(hi4[e]), b - f16_hi_f(hi4[e]));
                     }
                     unsigned char *line = Ps + (j >> 3) * kLboP + (hh * (V / 8) + g) * 128 + (j & 7) * 16;
                     *reinterpret_cast<uint4 *>(line) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
                     *reinterpret_cast<uint4 *>(line + L::kPTerm) = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
                 }
             }
-            if (rescale) {   // the accumulator times alpha_h beta: lane quadrant w % 4 of tiles w / 4 and w / 4 + 2
+            if (rescale) {   // the accumulator times fac[h]: lane quadrant w % 4 of tiles w / 4 and w / 4 + 2
 #pragma unroll 1
                 for (int mt = hh; mt < 4; mt += 2) {
 #pragma unroll 1
@@ -790,8 +746,7 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_multi_tc_kernel(
                         tc::tmem_ld32(ta, a);
                         tc::tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 32; e++)
-                            a[e] = __float_as_uint(__uint_as_float(a[e]) * (moved ? fac[cb + e] : beta));
+                        for (int e = 0; e < 32; e++) a[e] = __float_as_uint(__uint_as_float(a[e]) * fac[cb + e]);
                         tc::tmem_st32(ta, a);
                     }
                 }
@@ -800,22 +755,23 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_multi_tc_kernel(
             tc::fence_before_sync();
             tc::fence_proxy_async();
             __syncthreads();
+            if (tid < NH)
+                lsum[tid] = fmaf(lsum[tid], alpha, (red2[tid] + red2[NH + tid]) + (red2[2 * NH + tid] + red2[3 * NH + tid]));
 
             // d. O^T += C^T . P'_hi^T + C^T . P'_lo^T (M = 128 latent dims per tile, N = NH heads,
             //    K = 64 rows per term)
             if (tid == 0) {
                 tc::fence_after_sync();
-                const uint64_t dct = tc::desc(tc::smem_addr(Cs + buf * L::kCBytes), 8192, 128);   // C^T, MN-major
+                const uint32_t idesc = tc::idesc_f16(128, NH, true, true);
+                const uint32_t pa = tc::smem_addr(Ps), ca = tc::smem_addr(Cs + buf * L::kCBytes);
 #pragma unroll
                 for (int ks = 0; ks < ROWS / 16; ks++) {
 #pragma unroll
                     for (int mt = 0; mt < kLatent / 128; mt++) {
-                        // row groups 2 ks, 2 ks + 1 (8192 B apart), dim groups 16 mt .. (128 B apart)
-                        const uint64_t da = dct + static_cast<uint64_t>((ks * 2 * 8192 + mt * 16 * 128) / 16);
-                        tc::mma_bf16(tmem + mt * NH, da, dp + static_cast<uint64_t>(ks * 2 * kLboP / 16), idesc_o,
+                        const uint64_t da = tc::desc(ca + ks * 2 * 8192 + mt * 16 * 128, 8192, 128);
+                        tc::mma_bf16(tmem + mt * NH, da, tc::desc(pa + ks * 2 * kLboP, kLboP, 128), idesc,
                                      (have_o || ks > 0) ? 1u : 0u);
-                        tc::mma_bf16(tmem + mt * NH, da, dp + static_cast<uint64_t>((L::kPTerm + ks * 2 * kLboP) / 16),
-                                     idesc_o, 1u);
+                        tc::mma_bf16(tmem + mt * NH, da, tc::desc(pa + L::kPTerm + ks * 2 * kLboP, kLboP, 128), idesc, 1u);
                     }
                 }
                 tc::mma_commit(bar_o);
@@ -845,14 +801,6 @@ __global__ void __launch_bounds__(kMlaThreads, 1) mla_multi_tc_kernel(
         nv = nv_next;
     }
     if (!fail && have_o) {
-        // l of every head: the row slots' sums (a transposing butterfly, then the four quadrants)
-        float t[V];
-#pragma unroll
-        for (int e = 0; e < V; e++) t[e] = lacc[e];
-        const float bl = butterfly<V, false>(t);
-        if ((lane & kLow) == 0) red2[quad * NH + hh * V + ((lane >> kShift) & (V - 1))] = bl;
-        __syncthreads();
-        if (tid < NH) lsum[tid] = (red2[tid] + red2[NH + tid]) + (red2[2 * NH + tid] + red2[3 * NH + tid]);
         const bool ok = tc::mbar_wait(bar_o, (o_phase - 1) & 1u, kMlaWaitLimit);
         if (!__syncthreads_and(ok)) fail = 2;
     }
