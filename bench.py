@@ -53,11 +53,14 @@ def step_kernels(kp, wl, ld_pools: int, int8_keys: bool):
 
 
 def algorithmic_bytes(inp, key_bytes: int = 512, row_bytes: int = 528) -> dict:
-    """Bytes the method must move per step (no partials, no score spills): per query the visible
-    pooled keys (512 B each, 132 for the INT8 indexer state), q_idx + w, the gathered cache rows
-    (528 B each, 304 for 4-bit rows), q + out, indices; per step the store of the new rows and the
-    pools they complete."""
+    """Bytes the method must move per step (no partials, no score spills): each sequence's visible
+    pooled keys once, its queries sharing them (512 B each, 132 for the INT8 indexer state), and
+    per query q_idx + w and the top-k entries; each sequence's gathered cache rows once, at most
+    its tokens (528 B each, 304 for 4-bit rows), and per query q + out and the indices; per step the
+    store of the new rows and the pools they complete. With one query per sequence (decode) every
+    term is that query's. `gathered` counts (query, row) pairs, the attention's work."""
     wl = inp.wl
+    keys, rows = {}, {}   # per sequence: most visible pools of its queries, rows its queries gather
     per_q_idx = 0
     per_q_mla = 0
     gathered = 0
@@ -67,15 +70,19 @@ def algorithmic_bytes(inp, key_bytes: int = 512, row_bytes: int = 528) -> dict:
         n_vis = min(int(inp.len[s]), upto) // 4
         n_sel = min(n_vis, wl.select_k)
         tail = min(upto, int(inp.len[s])) - 4 * n_vis
-        per_q_idx += n_vis * key_bytes + 32 * 128 * 2 + 32 * 4 + wl.select_k * 4
-        per_q_mla += (4 * n_sel + tail) * row_bytes + 2 * wl.n_heads * 512 * 2 + wl.out_width * 4
+        keys[s] = max(keys.get(s, 0), n_vis)
+        rows[s] = rows.get(s, 0) + 4 * n_sel + tail
+        per_q_idx += 32 * 128 * 2 + 32 * 4 + wl.select_k * 4
+        per_q_mla += 2 * wl.n_heads * 512 * 2 + wl.out_width * 4
         gathered += 4 * n_sel + tail
+    index = per_q_idx + sum(keys.values()) * key_bytes
+    mla = per_q_mla + sum(min(r, int(inp.len[s])) for s, r in rows.items()) * row_bytes
     n_new = int(inp.new_token_mask().sum())
     store = n_new * (1024 + row_bytes + 8)
     new_pools = sum(1 for qs, qp in zip(inp.q_seq, inp.q_pos) if (qp - inp.pad[qs] + 1) % 4 == 0)
     kpool = new_pools * (4 * (256 + 256) + 512)
-    return dict(index=per_q_idx, mla=per_q_mla, store=store, kpool=kpool, gathered=gathered,
-                total=per_q_idx + per_q_mla + store + kpool)
+    return dict(index=index, mla=mla, store=store, kpool=kpool, gathered=gathered,
+                total=index + mla + store + kpool)
 
 
 def measured_peaks():

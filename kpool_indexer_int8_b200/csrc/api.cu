@@ -87,8 +87,8 @@ size_t gemm_scratch_bytes(int n_q) {
     return n_q >= glm::kIndexGemmMinQueries ? align_up(glm::index_gemm_scratch_bytes(n_q), 256) : 0;
 }
 // fp32 keys, many queries: scores by the GEMM kernel, then the selection on them.
-bool index_by_gemm(int n_q, int64_t ld_pools, int batch, const float *key_scales) {
-    return key_scales == nullptr && n_q >= glm::kIndexGemmMinQueries && ld_pools > 0 && batch <= 65535;
+bool index_by_gemm(int n_q, int64_t ld_pools, int batch, bool int8_keys) {
+    return !int8_keys && n_q >= glm::kIndexGemmMinQueries && ld_pools > 0 && batch <= 65535;
 }
 SelWs sel_layout(void *base, int n_q, int64_t ld) {
     char *p = static_cast<char *>(base);
@@ -263,7 +263,7 @@ int glm_dsa_step_plan(const glm_dsa_dims *dims, int32_t n_q, int64_t ld_pools, i
     if (n_q < 0 || ld_pools < 0 || batch < 0 || width < 1 || width > 65536 || !launches) return GLM_ERR_INVALID_ARG;
     int k = 1, f = 0;   // step_prep
     if (n_q > 0) {
-        if (index_by_gemm(n_q, ld_pools, batch, int8_keys ? reinterpret_cast<const float *>(&k) : nullptr)) {
+        if (index_by_gemm(n_q, ld_pools, batch, int8_keys != 0)) {
             f |= GLM_PLAN_INDEX_MANY;
             k += 5;   // query preparation, scores, histogram, selection, expansion
         } else {
@@ -364,7 +364,7 @@ int enqueue_index_select(const void *q_idx, const float *w, const void *keys, co
     const SelWs sw = sel_layout(workspace, n_q, ld_pools);
     char *ws = static_cast<char *>(workspace);
     float *sbuf = scores ? scores : reinterpret_cast<float *>(ws + sel_bytes(n_q, ld_pools));
-    if (index_by_gemm(n_q, ld_pools, batch, key_scales)) {
+    if (index_by_gemm(n_q, ld_pools, batch, key_scales != nullptr)) {
         // zero the selection's words, score every (query, pool), select, expand
         int rc = GLM_OK;
         if (zero) rc = cuda_status(glm::launch_zero(sw.hist, align_up(sw.zero_bytes, 16), st));
@@ -678,7 +678,7 @@ int glm_dsa_decode_step(const glm_dsa_dims *dims, const glm_dsa_step *a, void *w
     int *status = reinterpret_cast<int *>(ws + L.total - 256);
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const int sms = num_sms();
-    const bool idx_multi = a->n_q > 0 && (index_by_gemm(a->n_q, a->ld_pools, a->batch, q8 ? a->pooled_scales_dev : nullptr) ||
+    const bool idx_multi = a->n_q > 0 && (index_by_gemm(a->n_q, a->ld_pools, a->batch, q8) ||
                                           glm::index_select_ctas(a->n_q, a->ld_pools, sms) > 1);
     const SelWs sw = sel_layout(ws + L.idx, a->n_q, a->ld_pools);
     glm::StepPrepArgs p{};
