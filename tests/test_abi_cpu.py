@@ -262,3 +262,30 @@ def test_algorithmic_bytes_of_the_tiny_decode():
     assert ab["mla"] == 64 * 528 + 2 * 16 * 1024 + 80 * 4
     assert ab["store"] == 1560 and ab["kpool"] == 2560 and ab["gathered"] == 64
     assert ab["total"] == ab["index"] + ab["mla"] + ab["store"] + ab["kpool"] == 144920
+
+
+def test_algorithmic_bytes_count_a_prefill_chunks_shared_data_once():
+    # 300 causal queries at the end of one 6,000-token sequence: its 1,500 pooled keys once (the
+    # last query sees them all) and its rows at most once each (the queries gather 300 x 512 and
+    # more of them); per query q_idx + w + 128 top-k ids, q + out (64 heads) + 515 indices
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    wl = synth.custom("prefill_bytes", (0,), (6000,), n_heads=64, select_k=128, out_width=515, chunk=300, seed=44)
+    ab = bench.algorithmic_bytes(synth.generate(wl))
+    assert ab["index"] == 1500 * 512 + 300 * (8192 + 128 + 128 * 4)
+    assert ab["mla"] == 6000 * 528 + 300 * (2 * 64 * 1024 + 515 * 4)
+    assert ab["gathered"] >= 300 * 512   # the attention's work stays per (query, row)
+
+
+def test_bench_stage_names_follow_the_step_plan():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    k, paths, names = bench.step_kernels(kp, synth.WORKLOADS["long_decode"], 65536, False)
+    assert k == 4 and names == ("step_prep", "index_select_tc", "mla_split_tc", "mla_combine")
+    k, paths, names = bench.step_kernels(kp, synth.CHUNKED_PREFILL, 33792, False)
+    assert k == 7 and paths == kp.GLM_PLAN_INDEX_MANY | kp.GLM_PLAN_MLA_MANY
+    assert "index_gemm" in names[1] and names[2] == "mla_multi_tc" and "no combine" in names[3]
